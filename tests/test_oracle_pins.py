@@ -1,0 +1,307 @@
+"""Pins for the CPU oracle: it is checked against facts fixed by the pages and
+by mathematics, never against itself.
+
+* the SSA window geometry (QbitAI LoZA article, 1024-token sparse window
+  paragraph): closed-form row counts and a hand-derived golden table;
+* q = 0 makes every allowed key equally likely, so LSE_i = ln|J(i)| exactly and
+  O_i is the plain mean of the allowed values (written from the interval form
+  of the window, not the block rule);
+* when the window covers the whole prefix, SSA is textbook causal attention
+  ("LoZA：ZigZag稀疏注意力机制" §2.1, first formula with j <= i);
+* constant values return that value; identical keys give uniform weights;
+* a materialised-mask brute force in numpy agrees on tiny inputs;
+* decode is invariant to where pages sit, equals prefill row t under the
+  shared-latent broadcast, and packed varlen equals per-sequence prefill.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import ssa_oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def closed_form_count(i, blk, n_sink, n_local):
+    r = i % blk
+    return min(i + 1, blk * (n_sink + n_local - 1) + r + 1)
+
+
+def interval_keys(i, blk, n_sink, n_local):
+    """J(i) written as two token intervals: the sink prefix and the local run."""
+    b = i // blk
+    sink_hi = min(i, n_sink * blk - 1)
+    keys = list(range(0, sink_hi + 1))
+    lo = max(n_sink * blk, (b - n_local + 1) * blk)
+    keys += list(range(lo, i + 1))
+    return keys
+
+
+def to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float64 -> bf16 (nearest-even) and return the bit patterns."""
+    f = x.astype(np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return rounded.astype(np.uint16)
+
+
+# ---------------------------------------------------------------- geometry
+
+def test_golden_row_counts_block128_sink1_local7():
+    rows = []
+    with open(os.path.join(GOLDEN, "ssa_window_row_counts.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                i, c = line.split()
+                rows.append((int(i), int(c)))
+    assert len(rows) >= 10
+    for i, c in rows:
+        assert orc.row_count(i, 128, 1, 7) == c, i
+
+
+def test_row_count_north_star_formula():
+    # min(i+1, 128*[b>=7] + 768 + (i mod 128) + 1) for 1 sink + 7 local blocks of 128
+    for i in list(range(0, 2200, 37)) + [895, 896, 1023, 1024, 5000]:
+        b = i // 128
+        want = min(i + 1, 128 * (b >= 7) + 768 + (i % 128) + 1)
+        assert orc.row_count(i, 128, 1, 7) == want, i
+
+
+@pytest.mark.parametrize("blk,n_sink,n_local", [(128, 1, 7), (4, 0, 1), (4, 2, 3), (8, 1, 1),
+                                                (16, 3, 5), (5, 1, 2), (128, 0, 8)])
+def test_row_count_closed_form(blk, n_sink, n_local):
+    for i in range(0, blk * (n_sink + n_local + 4), max(1, blk // 8)):
+        assert orc.row_count(i, blk, n_sink, n_local) == closed_form_count(i, blk, n_sink, n_local)
+
+
+@pytest.mark.parametrize("n_sink,n_local", [(1, 7), (0, 1), (2, 3), (3, 1), (1, 12)])
+def test_key_blocks_from_mask(n_sink, n_local):
+    blk = 8
+    for qb in range(0, 30):
+        got = orc.key_blocks(qb, seq_len=30 * blk, blk=blk, n_sink=n_sink, n_local=n_local)
+        want = sorted(set(range(min(n_sink, qb + 1))) |
+                      set(range(max(n_sink, qb - n_local + 1), qb + 1)))
+        assert got == want, qb
+        assert len(got) == min(qb + 1, n_sink + n_local)
+
+
+def test_key_blocks_partial_last_block():
+    # a ragged final block still touches its own (partial) block
+    assert orc.key_blocks(9, seq_len=9 * 128 + 3) == [0, 3, 4, 5, 6, 7, 8, 9]
+
+
+# ------------------------------------------------------------ attention math
+
+@pytest.mark.parametrize("blk,n_sink,n_local,L", [(128, 1, 7, 1300), (8, 1, 7, 200),
+                                                  (4, 0, 2, 50), (6, 2, 3, 97)])
+def test_q_zero_gives_log_count_and_mean(blk, n_sink, n_local, L):
+    rng = np.random.default_rng(3)
+    d = 16
+    q = np.zeros((1, 1, L, d))
+    k = rng.standard_normal((1, 1, L, d))
+    v = rng.standard_normal((1, 1, L, 8))
+    o, lse = orc.prefill(q, k, v, blk, n_sink, n_local, scale=0.25)
+    for i in range(L):
+        keys = interval_keys(i, blk, n_sink, n_local)
+        assert len(keys) == closed_form_count(i, blk, n_sink, n_local)
+        assert abs(lse[0, 0, i] - math.log(len(keys))) < 1e-12
+        np.testing.assert_allclose(o[0, 0, i], v[0, 0, keys].mean(axis=0), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("L,blk,n_sink,n_local", [(1024, 128, 1, 7), (700, 128, 1, 7),
+                                                  (64, 8, 1, 7), (90, 8, 0, 12), (33, 4, 2, 7)])
+def test_full_window_equals_causal(L, blk, n_sink, n_local):
+    assert L <= blk * (n_sink + n_local) or n_local >= -(-L // blk)
+    rng = np.random.default_rng(L)
+    q = rng.standard_normal((1, 2, L, 32))
+    k = rng.standard_normal((1, 2, L, 32))
+    v = rng.standard_normal((1, 2, L, 24))
+    o, lse = orc.prefill(q, k, v, blk, n_sink, n_local, scale=0.3)
+    o_ref, lse_ref = orc.causal_attention(q, k, v, scale=0.3)
+    np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=1e-11)
+
+
+def test_beyond_window_differs_from_causal():
+    # once the window no longer covers the prefix, SSA must NOT be causal attention
+    L = 1400
+    rng = np.random.default_rng(1)
+    q = rng.standard_normal((1, 1, L, 16))
+    k = rng.standard_normal((1, 1, L, 16))
+    v = rng.standard_normal((1, 1, L, 16))
+    o, _ = orc.prefill(q, k, v, scale=0.25)
+    o_ref, _ = orc.causal_attention(q, k, v, scale=0.25)
+    np.testing.assert_allclose(o[..., :1024, :], o_ref[..., :1024, :], atol=1e-11)
+    assert np.abs(o[..., 1024:, :] - o_ref[..., 1024:, :]).max() > 1e-3
+
+
+def test_constant_values_return_that_value():
+    rng = np.random.default_rng(5)
+    L = 300
+    q = rng.standard_normal((1, 1, L, 16)) * 3
+    k = rng.standard_normal((1, 1, L, 16)) * 3
+    row = rng.standard_normal(12)
+    v = np.broadcast_to(row, (1, 1, L, 12)).copy()
+    o, _ = orc.prefill(q, k, v, blk=16, n_sink=1, n_local=3, scale=0.5)
+    np.testing.assert_allclose(o[0, 0], np.broadcast_to(row, (L, 12)), atol=1e-12)
+
+
+def test_identical_keys_give_uniform_weights():
+    rng = np.random.default_rng(6)
+    L, blk, ns, nl = 200, 16, 2, 3
+    q = rng.standard_normal((1, 1, L, 8))
+    k = np.broadcast_to(rng.standard_normal(8), (1, 1, L, 8)).copy()
+    v = rng.standard_normal((1, 1, L, 5))
+    o, lse = orc.prefill(q, k, v, blk=blk, n_sink=ns, n_local=nl, scale=0.7)
+    s = 0.7 * q[0, 0] @ k[0, 0, 0]
+    for i in range(L):
+        keys = interval_keys(i, blk, ns, nl)
+        np.testing.assert_allclose(o[0, 0, i], v[0, 0, keys].mean(axis=0), atol=1e-12)
+        assert abs(lse[0, 0, i] - (s[i] + math.log(len(keys)))) < 1e-11
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_brute_force_mask_agrees(seed):
+    rng = np.random.default_rng(100 + seed)
+    blk = int(rng.integers(2, 9))
+    n_sink = int(rng.integers(0, 3))
+    n_local = int(rng.integers(1, 5))
+    L = int(rng.integers(1, 12 * blk))
+    q = rng.standard_normal((2, 2, L, 12))
+    k = rng.standard_normal((2, 2, L, 12))
+    v = rng.standard_normal((2, 2, L, 7))
+    o, lse = orc.prefill(q, k, v, blk, n_sink, n_local, scale=0.4)
+    o_bf, lse_bf = orc.brute_force_prefill(q, k, v, blk, n_sink, n_local, scale=0.4)
+    np.testing.assert_allclose(o, o_bf, atol=1e-11)
+    np.testing.assert_allclose(lse, lse_bf, atol=1e-11)
+
+
+def test_brute_force_block128_two_windows():
+    rng = np.random.default_rng(11)
+    L = 1300
+    q = to_bf16_bits(rng.standard_normal((1, 1, L, 64)))
+    k = to_bf16_bits(rng.standard_normal((1, 1, L, 64)))
+    v = to_bf16_bits(rng.standard_normal((1, 1, L, 64)))
+    o, lse = orc.prefill(q, k, v, scale=0.125)
+    o_bf, lse_bf = orc.brute_force_prefill(q, k, v, scale=0.125)
+    np.testing.assert_allclose(o, o_bf, atol=1e-11)
+    np.testing.assert_allclose(lse, lse_bf, atol=1e-11)
+
+
+def test_bf16_inputs_are_widened_exactly():
+    rng = np.random.default_rng(7)
+    bits = [to_bf16_bits(rng.standard_normal((1, 2, 150, 16))) for _ in range(3)]
+    wide = [orc.bf16_bits_to_f64(b) for b in bits]
+    o1, l1 = orc.prefill(*bits, blk=16, n_sink=1, n_local=2, scale=0.25)
+    o2, l2 = orc.prefill(*wide, blk=16, n_sink=1, n_local=2, scale=0.25)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+    # and the widening itself: bf16 1.5 = 0x3FC0, -2 = 0xC000
+    assert orc.bf16_bits_to_f64(np.array([0x3FC0, 0xC000], np.uint16)).tolist() == [1.5, -2.0]
+
+
+def test_row_subset_matches_full():
+    rng = np.random.default_rng(8)
+    q, k, v = (rng.standard_normal((2, 3, 90, 8)) for _ in range(3))
+    o, lse = orc.prefill(q, k, v, blk=8, n_sink=1, n_local=2)
+    rows = np.array([0, 5, 89, 90, 270, 539])
+    os_, ls_ = orc.prefill(q, k, v, blk=8, n_sink=1, n_local=2, rows=rows)
+    np.testing.assert_array_equal(os_, o.reshape(-1, 8)[rows])
+    np.testing.assert_array_equal(ls_, lse.reshape(-1)[rows])
+
+
+# ------------------------------------------------------------------- varlen
+
+def test_varlen_equals_per_sequence_prefill():
+    rng = np.random.default_rng(9)
+    lens = [37, 1, 64, 100, 16]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    H, total = 2, int(cu[-1])
+    q, k = (rng.standard_normal((H, total, 12)) for _ in range(2))
+    v = rng.standard_normal((H, total, 6))
+    o, lse = orc.prefill_varlen(q, k, v, cu, blk=8, n_sink=1, n_local=3, scale=0.3)
+    for s, n in enumerate(lens):
+        a, b = cu[s], cu[s + 1]
+        o_s, l_s = orc.prefill(q[None, :, a:b], k[None, :, a:b], v[None, :, a:b], blk=8,
+                               n_sink=1, n_local=3, scale=0.3)
+        np.testing.assert_array_equal(o[:, a:b], o_s[0])
+        np.testing.assert_array_equal(lse[:, a:b], l_s[0])
+
+
+def test_varlen_short_sequences_equal_causal():
+    rng = np.random.default_rng(10)
+    lens = [1024, 300, 1]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    q, k, v = (to_bf16_bits(rng.standard_normal((1, int(cu[-1]), 32))) for _ in range(3))
+    o, lse = orc.prefill_varlen(q, k, v, cu, scale=0.2)
+    for s in range(len(lens)):
+        a, b = cu[s], cu[s + 1]
+        o_c, l_c = orc.causal_attention(q[:, a:b], k[:, a:b], v[:, a:b], scale=0.2)
+        np.testing.assert_allclose(o[:, a:b], o_c, atol=1e-11)
+        np.testing.assert_allclose(lse[:, a:b], l_c, atol=1e-11)
+
+
+# ------------------------------------------------------------------- decode
+
+def _decode_case(seed, seq_lens, Hq=4, dqk=24, dv=16, ps=8, permute=True):
+    rng = np.random.default_rng(seed)
+    pages = [-(-n // ps) for n in seq_lens]
+    n_pages = sum(pages) + 3          # a few pages nobody references
+    perm = rng.permutation(n_pages) if permute else np.arange(n_pages)
+    table = np.full((len(seq_lens), max(pages) + 2), -1, np.int32)
+    off = 0
+    for b, n in enumerate(pages):
+        table[b, :n] = perm[off:off + n]
+        off += n
+    kv = rng.standard_normal((n_pages, ps, dqk))
+    q = rng.standard_normal((len(seq_lens), Hq, dqk))
+    return q, kv, table, np.array(seq_lens, np.int32)
+
+
+def test_decode_matches_brute_force():
+    q, kv, pt, sl = _decode_case(1, [1, 8, 9, 61, 100])
+    o, lse = orc.decode(q, kv, pt, sl, dv=16, page_size=8, n_sink=1, n_local=3, scale=0.3)
+    o_bf, lse_bf = orc.brute_force_decode(q, kv, pt, sl, dv=16, page_size=8, n_sink=1,
+                                          n_local=3, scale=0.3)
+    np.testing.assert_allclose(o, o_bf, atol=1e-11)
+    np.testing.assert_allclose(lse, lse_bf, atol=1e-11)
+
+
+def test_decode_page_permutation_invariant():
+    lens = [5, 40, 77]
+    q, kv_a, pt_a, sl = _decode_case(2, lens, permute=False)
+    # move every page to a new physical slot and rewrite the table to match
+    rng = np.random.default_rng(99)
+    perm = rng.permutation(kv_a.shape[0])
+    kv_b = np.empty_like(kv_a)
+    kv_b[perm] = kv_a
+    pt_b = np.where(pt_a >= 0, perm[np.maximum(pt_a, 0)], -1).astype(np.int32)
+    a = orc.decode(q, kv_a, pt_a, sl, dv=16, page_size=8, n_sink=1, n_local=2)
+    b = orc.decode(q, kv_b, pt_b, sl, dv=16, page_size=8, n_sink=1, n_local=2)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
+def test_decode_equals_prefill_last_row():
+    lens = [70, 33]
+    q, kv, pt, sl = _decode_case(3, lens, Hq=3)
+    o, lse = orc.decode(q, kv, pt, sl, dv=16, page_size=8, n_sink=2, n_local=3, scale=0.2)
+    for b, n in enumerate(lens):
+        logical = np.arange(n)
+        rows = kv.reshape(-1, kv.shape[-1])[pt[b][logical // 8] * 8 + logical % 8]
+        for h in range(3):
+            qq = np.zeros((1, 1, n, rows.shape[1]))
+            qq[0, 0, n - 1] = q[b, h]
+            o_p, l_p = orc.prefill(qq, rows[None, None], rows[None, None, :, :16], blk=8,
+                                   n_sink=2, n_local=3, scale=0.2, rows=np.array([n - 1]))
+            np.testing.assert_allclose(o[b, h], o_p[0], atol=1e-12)
+            assert abs(lse[b, h] - l_p[0]) < 1e-12
+
+
+def test_decode_rejects_bad_page_id():
+    q, kv, pt, sl = _decode_case(4, [20])
+    pt[0, 1] = kv.shape[0]          # out of range
+    with pytest.raises(ValueError):
+        orc.decode(q, kv, pt, sl, dv=16, page_size=8, n_sink=1, n_local=3)
