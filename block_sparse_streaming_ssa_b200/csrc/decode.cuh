@@ -1,0 +1,335 @@
+// decode.cuh -- paged SSA decode on sm_100a (absorbed-MLA layout).
+//
+// One new query token per sequence; H_q query heads (a group of up to 128 is
+// the M dimension of the MMA) share one latent key/value row of 576 bf16 per
+// token (512 latent + 64 rope); the value is the first 512 entries of the
+// same row.  The window of the query at t = seq_len - 1 is the sink page(s)
+// plus the n_local pages ending at t's page (QbitAI article on LongCat LoZA,
+// paragraph on the 1024-token sparse window), read through the page table.
+//
+// Split kernel: one CTA per (window page, head group, sequence).
+//   TMA     the 128-token page (9 swizzled boxes of 64 columns = 144 KB) into
+//           smem, Q of the head group streamed in 64-column boxes (2-deep ring)
+//   MMA     S[128 heads x 128 keys] = Q K^T   (K = 576: 9 boxes x 4 k-steps)
+//   softmax mask keys past t, row max, exp2, row sum; P (bf16) -> smem
+//   MMA     O[128 x 512] = P V, two N=256 halves, V = the page's first 8 boxes
+//           read as an MN-major operand (no transpose copy)
+//   out     normalised partial O (fp32) and its LSE to the workspace
+// TMEM: S uses columns [0,128); O uses [0,512) once S has been read.
+//
+// Merge kernel: LSE = logsumexp_s LSE_s, O = sum_s exp(LSE_s - LSE) O_s.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+#include "schedule.cuh"
+
+namespace loza {
+
+constexpr int kDecodeDqk = 576;
+constexpr int kDecodeDv = 512;
+
+struct DecodeParams {
+  const int* page_table;  // [B, max_pages]
+  const int* seq_lens;    // [B]
+  float* o_part;          // [B, HG, n_split, 128, 512]
+  float* lse_part;        // [B, HG, n_split, 128]
+  __nv_bfloat16* o;       // [B, H_q, 512]
+  float* lse;             // [B, H_q]
+  int B, H_q, HG, max_pages, n_pages, n_sink, n_local, n_split;
+  float scale_log2;
+};
+
+// The decode window of sequence b, as the kernels select it.  Returns the
+// number of window pages (0 for an invalid seq_len, flagged in the status).
+struct DecodeWindow {
+  int t;       // query position
+  int qb;      // logical page of the query
+  TileRange tr;
+};
+
+__device__ __forceinline__ bool decode_window(const DecodeParams& p, int b, DecodeWindow& w) {
+  const int len = __ldg(p.seq_lens + b);
+  if (len < 1 || (long long)len > (long long)p.max_pages * 128) return false;
+  w.t = len - 1;
+  w.qb = w.t >> 7;
+  w.tr = tile_range(w.qb, p.n_sink, p.n_local);
+  return true;
+}
+
+// Physical page of window tile `i`, or -1 if the table entry is outside the pool.
+__device__ __forceinline__ int decode_page(const DecodeParams& p, int b, const DecodeWindow& w,
+                                           int i) {
+  const int logical = tile_block(w.tr, i);
+  const int phys = __ldg(p.page_table + (size_t)b * p.max_pages + logical);
+  return (phys >= 0 && phys < p.n_pages) ? phys : -1;
+}
+
+struct DecodeLayout {
+  static constexpr int CHUNK = 128 * 128;  // [128 rows x 64 bf16], 128B swizzle
+  static constexpr int KV_CH = kDecodeDqk / 64;  // 9
+  static constexpr int OFF_KV = 0;
+  static constexpr int OFF_Q = OFF_KV + KV_CH * CHUNK;  // 2-deep ring
+  static constexpr int OFF_P = OFF_Q + 2 * CHUNK;       // P [128 x 128] bf16 as 2 boxes
+  static constexpr int OFF_BAR = OFF_P + 2 * CHUNK;
+  static constexpr int B_KV_FULL = 0;                   // 9
+  static constexpr int B_Q_FULL = B_KV_FULL + KV_CH;    // 2
+  static constexpr int B_Q_EMPTY = B_Q_FULL + 2;        // 2
+  static constexpr int B_S_FULL = B_Q_EMPTY + 2;
+  static constexpr int B_P_FULL = B_S_FULL + 1;
+  static constexpr int B_O_FULL = B_P_FULL + 1;
+  static constexpr int B_DRAIN = B_O_FULL + 1;
+  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+};
+
+__global__ void __launch_bounds__(192, 1)
+    ssa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_q,
+                            const __grid_constant__ CUtensorMap tm_kv, const DecodeParams p) {
+  using Lay = DecodeLayout;
+  const int sp = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t part = ((size_t)(b * p.HG + hg) * p.n_split + sp) * 128;
+
+  // ---- which page this CTA reads (uniform across the CTA; exits before any barrier)
+  DecodeWindow win;
+  int phys = -1, valid_keys = 0;
+  if (!decode_window(p, b, win)) {
+    if (threadIdx.x == 0 && sp == 0 && hg == 0) atomicOr(&g_loza_status, 4);
+  } else if (sp < win.tr.count) {
+    phys = decode_page(p, b, win, sp);
+    if (phys < 0) {
+      if (threadIdx.x == 0) atomicOr(&g_loza_status, 2);
+    } else {
+      const int logical = tile_block(win.tr, sp);
+      valid_keys = min(128, win.t - logical * 128 + 1);
+    }
+  }
+  if (phys < 0) {
+    if (threadIdx.x < 128) p.lse_part[part + threadIdx.x] = -INFINITY;  // empty split
+    return;
+  }
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sb = smem_u32(smem);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  auto bar = [&](int i) -> uint32_t { return sb + Lay::OFF_BAR + 8 * i; };
+  int* status = &g_loza_status;
+
+  if (threadIdx.x == 0) {
+    for (int c = 0; c < Lay::KV_CH; ++c) mbar_init(bar(Lay::B_KV_FULL + c), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(Lay::B_Q_FULL + s), 1);
+      mbar_init(bar(Lay::B_Q_EMPTY + s), 1);
+    }
+    mbar_init(bar(Lay::B_S_FULL), 1);
+    mbar_init(bar(Lay::B_P_FULL), 128);
+    mbar_init(bar(Lay::B_O_FULL), 1);
+    mbar_init(bar(Lay::B_DRAIN), 1);
+    misc[1] = 0;
+    fence_barrier_init();
+  }
+  if (warp == 4 && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_kv);
+  }
+  if (warp == 5) {
+    tmem_alloc(sb + Lay::OFF_MISC, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int q_issued = 0;
+      bool ok = true;
+      auto load_q = [&](int c) -> bool {
+        const int st = c & 1;
+        if (c >= 2 && !mbar_wait(bar(Lay::B_Q_EMPTY + st), ((c >> 1) - 1) & 1, abort_flag, status, 1))
+          return false;
+        mbar_arrive_expect_tx(bar(Lay::B_Q_FULL + st), Lay::CHUNK);
+        tma_load_3d(sb + Lay::OFF_Q + st * Lay::CHUNK, &tm_q, bar(Lay::B_Q_FULL + st), c * 64,
+                    hg * 128, b);
+        ++q_issued;
+        return true;
+      };
+      load_q(0);
+      for (int c = 0; c < Lay::KV_CH; ++c) {
+        mbar_arrive_expect_tx(bar(Lay::B_KV_FULL + c), Lay::CHUNK);
+        tma_load_2d(sb + Lay::OFF_KV + c * Lay::CHUNK, &tm_kv, bar(Lay::B_KV_FULL + c), c * 64,
+                    phys * 128);
+        if (c == 0) load_q(1);
+      }
+      for (int c = 2; ok && c < Lay::KV_CH; ++c) ok = load_q(c);
+      // every copy issued lands before the CTA exits (normally already consumed)
+      for (int c = 0; c < Lay::KV_CH; ++c) mbar_wait_drain(bar(Lay::B_KV_FULL + c), 0);
+      for (int st = 0; st < 2; ++st) {
+        const int n = (q_issued - st + 1) / 2;  // loads issued into ring slot st
+        if (n > 0) mbar_wait_drain(bar(Lay::B_Q_FULL + st), (n - 1) & 1);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t id_s = idesc_bf16_f32(128, 128, false);
+      const uint32_t id_o = idesc_bf16_f32(128, 256, true);
+      bool ok = true;
+      for (int c = 0; ok && c < Lay::KV_CH; ++c) {
+        const int st = c & 1;
+        ok = mbar_wait(bar(Lay::B_KV_FULL + c), 0, abort_flag, status, 1) &&
+             mbar_wait(bar(Lay::B_Q_FULL + st), (c >> 1) & 1, abort_flag, status, 1);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t adesc = sdesc_sw128(sb + Lay::OFF_Q + st * Lay::CHUNK + kk * 32, 16, 1024);
+          const uint64_t bdesc = sdesc_sw128(sb + Lay::OFF_KV + c * Lay::CHUNK + kk * 32, 16, 1024);
+          mma_ss(tmem, adesc, bdesc, id_s, (c > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(bar(Lay::B_Q_EMPTY + st));
+      }
+      if (ok) {
+        mma_commit(bar(Lay::B_S_FULL));
+        ok = mbar_wait(bar(Lay::B_P_FULL), 0, abort_flag, status, 1);
+      }
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t adesc =
+                sdesc_sw128(sb + Lay::OFF_P + (kk >> 2) * Lay::CHUNK + (kk & 3) * 32, 16, 1024);
+            const uint64_t bdesc = sdesc_sw128(
+                sb + Lay::OFF_KV + half * 4 * Lay::CHUNK + kk * 2048, Lay::CHUNK, 1024);
+            mma_ss(tmem + half * 256, adesc, bdesc, id_o, kk > 0 ? 1u : 0u);
+          }
+        }
+        mma_commit(bar(Lay::B_O_FULL));
+      }
+      mma_commit(bar(Lay::B_DRAIN));
+      mbar_wait_drain(bar(Lay::B_DRAIN), 0);
+    }
+  } else {
+    // ----------------------------------------------------- softmax + output
+    const int h = threadIdx.x;  // head row within the group
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const float sl2 = p.scale_log2;
+    do {
+      if (!mbar_wait(bar(Lay::B_S_FULL), 0, abort_flag, status, 1)) break;
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) tmem_ld32(tmem + lane_base + ch * 32, sr[ch]);
+      tmem_wait_ld();
+      float mx = -INFINITY;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          if (ch * 32 + c >= valid_keys) sr[ch][c] = __float_as_uint(-INFINITY);
+          mx = fmaxf(mx, __uint_as_float(sr[ch][c]));
+        }
+      const float m = mx * sl2;
+      float l = 0.f;
+      // P row h -> smem, K-major 128B-swizzled: box (key/64), row h, 16-byte unit u
+      // holding keys 8u..8u+7 lands at unit u ^ (h & 7).
+      uint8_t* prow = smem + Lay::OFF_P + h * 128;
+#pragma unroll
+      for (int box = 0; box < 2; ++box) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int col = box * 64 + u * 8 + 2 * e;
+            const float p0 = ex2_approx(fmaf(__uint_as_float(sr[col >> 5][col & 31]), sl2, -m));
+            const float p1 =
+                ex2_approx(fmaf(__uint_as_float(sr[(col + 1) >> 5][(col + 1) & 31]), sl2, -m));
+            l += p0 + p1;
+            w4[e] = pack_bf16x2(p0, p1);
+          }
+          *reinterpret_cast<uint4*>(prow + box * Lay::CHUNK + ((u ^ (h & 7)) << 4)) =
+              make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
+      }
+      fence_async_shared();
+      tc_fence_before();
+      mbar_arrive(bar(Lay::B_P_FULL));
+
+      if (!mbar_wait(bar(Lay::B_O_FULL), 0, abort_flag, status, 1)) break;
+      tc_fence_after();
+      const bool valid = hg * 128 + h < p.H_q;
+      float* dst = p.o_part + (part + h) * kDecodeDv;
+      const float inv_l = 1.f / l;
+#pragma unroll 1
+      for (int ch = 0; ch < kDecodeDv / 32; ++ch) {
+        uint32_t orr[32];
+        tmem_ld32(tmem + lane_base + ch * 32, orr);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            reinterpret_cast<float4*>(dst + ch * 32)[v] = make_float4(
+                __uint_as_float(orr[4 * v]) * inv_l, __uint_as_float(orr[4 * v + 1]) * inv_l,
+                __uint_as_float(orr[4 * v + 2]) * inv_l, __uint_as_float(orr[4 * v + 3]) * inv_l);
+        }
+      }
+      if (valid) p.lse_part[part + h] = (m + __log2f(l)) * kLn2;
+    } while (false);
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// One CTA of 128 threads per (sequence, head): each thread merges 4 of the
+// 512 output columns over the splits.
+__global__ void __launch_bounds__(128)
+    ssa_decode_merge_kernel(const DecodeParams p) {
+  const int b = blockIdx.x / p.H_q, h = blockIdx.x % p.H_q;
+  const int hg = h >> 7, hr = h & 127;
+  const size_t base = (size_t)(b * p.HG + hg) * p.n_split;
+  float lmax = -INFINITY;
+  for (int s = 0; s < p.n_split; ++s) lmax = fmaxf(lmax, p.lse_part[(base + s) * 128 + hr]);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  float denom = 0.f;
+  if (lmax > -INFINITY) {
+    for (int s = 0; s < p.n_split; ++s) {
+      const float ls = p.lse_part[(base + s) * 128 + hr];
+      if (ls == -INFINITY) continue;
+      const float wgt = __expf(ls - lmax);
+      denom += wgt;
+      const float4 v = reinterpret_cast<const float4*>(
+          p.o_part + ((base + s) * 128 + hr) * kDecodeDv)[threadIdx.x];
+      acc[0] += wgt * v.x;
+      acc[1] += wgt * v.y;
+      acc[2] += wgt * v.z;
+      acc[3] += wgt * v.w;
+    }
+  }
+  const float inv = denom > 0.f ? 1.f / denom : 0.f;
+  __nv_bfloat16* dst = p.o + ((size_t)b * p.H_q + h) * kDecodeDv + threadIdx.x * 4;
+  uint2 pk;
+  pk.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  pk.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+  *reinterpret_cast<uint2*>(dst) = pk;
+  if (threadIdx.x == 0)
+    p.lse[(size_t)b * p.H_q + h] = denom > 0.f ? lmax + __logf(denom) : -INFINITY;
+}
+
+}  // namespace loza

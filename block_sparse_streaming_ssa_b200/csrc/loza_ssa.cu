@@ -1,0 +1,379 @@
+// loza_ssa.cu -- the C ABI declared in include/loza_ssa.h: argument checks,
+// TMA tensor maps, and stream-ordered launches of the sm_100a kernels.
+// The library allocates no device memory and never synchronises the device
+// (except inside loza_ssa_get_last_device_status, whose job that is).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/loza_ssa.h"
+#include "decode.cuh"
+#include "prefill.cuh"
+#include "schedule.cuh"
+
+namespace {
+
+constexpr int kVersion = 10000;  // 1.0.0
+constexpr int kMaxVarlenSeqs = 4096;
+constexpr int kMaxDecodeWindow = 4096;
+constexpr int kMaxDevices = 64;
+
+thread_local char g_last_error[256] = "";
+
+int cuda_fail(cudaError_t e, const char* what) {
+  std::snprintf(g_last_error, sizeof g_last_error, "%s: %s", what, cudaGetErrorString(e));
+  return LOZA_SSA_ERR_CUDA;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::mutex g_mu;
+EncodeTiledFn g_encode = nullptr;
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+  int cc_major = 0, cc_minor = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+// Current device, its SM count, and a one-time check that it is sm_100.
+int device_info(DeviceInfo& out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) {
+    std::snprintf(g_last_error, sizeof g_last_error, "device ordinal %d unsupported", dev);
+    return LOZA_SSA_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    if ((e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute(SM count)");
+    cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+      if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+        return cuda_fail(e == cudaSuccess ? cudaErrorSymbolNotFound : e,
+                         "cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)");
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    d.ready = true;
+  }
+  if (d.cc_major != 10 || d.cc_minor != 0) {
+    std::snprintf(g_last_error, sizeof g_last_error,
+                  "libloza_ssa is built for sm_100a; device %d is sm_%d%d", dev, d.cc_major,
+                  d.cc_minor);
+    return LOZA_SSA_ERR_CUDA;
+  }
+  out = d;
+  return LOZA_SSA_OK;
+}
+
+// bf16 tensor map: dims {d0 (innermost), d1, d2}, box {64, 128, 1}, 128B swizzle.
+int make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, int rank) {
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank,
+                        const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return LOZA_SSA_ERR_CUDA;
+  }
+  return LOZA_SSA_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+template <int DQK, int DV>
+int launch_prefill(const void* q, const void* k, const void* v, loza::PrefillParams prm,
+                   uint64_t plane_rows, uint64_t planes, int items_upper, int n_prefix,
+                   cudaStream_t stream, const DeviceInfo& dev) {
+  using Lay = loza::PrefillLayout<DQK, DV>;
+  CUtensorMap mq, mk, mv;
+  int rc;
+  if ((rc = make_map(&mq, q, DQK, plane_rows, planes, 3)) != LOZA_SSA_OK) return rc;
+  if ((rc = make_map(&mk, k, DQK, plane_rows, planes, 3)) != LOZA_SSA_OK) return rc;
+  if ((rc = make_map(&mv, v, DV, plane_rows, planes, 3)) != LOZA_SSA_OK) return rc;
+  const size_t smem = Lay::smem_bytes(n_prefix);
+  auto kern = loza::ssa_prefill_kernel<DQK, DV>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)Lay::smem_bytes(kMaxVarlenSeqs + 1));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill)");
+  const int grid = items_upper < dev.num_sms ? items_upper : dev.num_sms;
+  kern<<<grid, 192, smem, stream>>>(mq, mk, mv, prm);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "prefill launch");
+  return LOZA_SSA_OK;
+}
+
+int dispatch_prefill(int d_qk, int d_v, const void* q, const void* k, const void* v,
+                     const loza::PrefillParams& prm, uint64_t plane_rows, uint64_t planes,
+                     int items_upper, int n_prefix, cudaStream_t s, const DeviceInfo& dev) {
+  if (d_qk == 64 && d_v == 64)
+    return launch_prefill<64, 64>(q, k, v, prm, plane_rows, planes, items_upper, n_prefix, s, dev);
+  if (d_qk == 128 && d_v == 128)
+    return launch_prefill<128, 128>(q, k, v, prm, plane_rows, planes, items_upper, n_prefix, s, dev);
+  if (d_qk == 192 && d_v == 128)
+    return launch_prefill<192, 128>(q, k, v, prm, plane_rows, planes, items_upper, n_prefix, s, dev);
+  return LOZA_SSA_ERR_HEAD_DIM;
+}
+
+bool prefill_dims_ok(int d_qk, int d_v) {
+  return (d_qk == 64 && d_v == 64) || (d_qk == 128 && d_v == 128) || (d_qk == 192 && d_v == 128);
+}
+
+__global__ void debug_tiles_kernel(int n_qb, int n_sink, int n_local, int* tiles, int* counts,
+                                   int max_tiles) {
+  const int qb = blockIdx.x * blockDim.x + threadIdx.x;
+  if (qb >= n_qb) return;
+  const loza::TileRange r = loza::tile_range(qb, n_sink, n_local);
+  counts[qb] = r.count;
+  for (int t = 0; t < r.count && t < max_tiles; ++t)
+    tiles[(size_t)qb * max_tiles + t] = loza::tile_block(r, t);
+}
+
+__global__ void debug_decode_pages_kernel(loza::DecodeParams p, int* pages, int* counts,
+                                          int max_tiles) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= p.B) return;
+  loza::DecodeWindow w;
+  if (!loza::decode_window(p, b, w)) {
+    counts[b] = 0;
+    atomicOr(&loza::g_loza_status, LOZA_SSA_DEV_BAD_SEQLEN);
+    return;
+  }
+  counts[b] = w.tr.count;
+  for (int i = 0; i < w.tr.count && i < max_tiles; ++i) {
+    const int phys = loza::decode_page(p, b, w, i);
+    if (phys < 0) atomicOr(&loza::g_loza_status, LOZA_SSA_DEV_BAD_PAGE);
+    pages[(size_t)b * max_tiles + i] = phys;
+  }
+}
+
+size_t decode_partial_floats(int B, int H_q, int n_split) {
+  const size_t hg = (size_t)(H_q + 127) / 128;
+  return (size_t)B * hg * (size_t)n_split * 128;
+}
+
+}  // namespace
+
+extern "C" {
+
+int loza_ssa_version(void) { return kVersion; }
+
+const char* loza_ssa_last_error_string(void) { return g_last_error; }
+
+const char* loza_ssa_status_string(int status) {
+  switch (status) {
+    case LOZA_SSA_OK: return "ok";
+    case LOZA_SSA_ERR_NULL: return "a required pointer is NULL";
+    case LOZA_SSA_ERR_SHAPE: return "a size is out of range, or scale is not finite";
+    case LOZA_SSA_ERR_HEAD_DIM: return "unsupported (d_qk, d_v)";
+    case LOZA_SSA_ERR_BLOCK: return "block / page_size must be 128";
+    case LOZA_SSA_ERR_WINDOW: return "n_sink / n_local out of range";
+    case LOZA_SSA_ERR_ALIGN: return "pointer not aligned (bf16 tensors: 16 B, lse: 4 B, workspace: 256 B)";
+    case LOZA_SSA_ERR_WORKSPACE: return "decode workspace missing or too small";
+    case LOZA_SSA_ERR_CUDA: return "CUDA error (see loza_ssa_last_error_string)";
+    default: return "unknown status";
+  }
+}
+
+int loza_ssa_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int H, int L, int d_qk, int d_v, int block, int n_sink, int n_local,
+                     float scale, loza_ssa_stream_t stream) {
+  if (!q || !k || !v || !o || !lse) return LOZA_SSA_ERR_NULL;
+  if (B < 1 || H < 1 || L < 1 || !std::isfinite(scale)) return LOZA_SSA_ERR_SHAPE;
+  if (!prefill_dims_ok(d_qk, d_v)) return LOZA_SSA_ERR_HEAD_DIM;
+  if (block != 128) return LOZA_SSA_ERR_BLOCK;
+  if (n_sink < 0 || n_local < 1) return LOZA_SSA_ERR_WINDOW;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return LOZA_SSA_ERR_ALIGN;
+  const long long nb = (L + 127) / 128;
+  const long long items = (long long)B * H * nb;
+  if (items >= (1ll << 31) || (long long)B * H >= (1ll << 31)) return LOZA_SSA_ERR_SHAPE;
+  DeviceInfo dev;
+  int rc = device_info(dev);
+  if (rc != LOZA_SSA_OK) return rc;
+  loza::PrefillParams prm{};
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  prm.cu_seqlens = nullptr;
+  prm.n_seqs = B;
+  prm.H = H;
+  prm.L = L;
+  prm.plane_rows = L;
+  prm.n_sink = n_sink;
+  prm.n_local = n_local;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.total_items = (int)items;
+  return dispatch_prefill(d_qk, d_v, q, k, v, prm, (uint64_t)L, (uint64_t)B * H, (int)items, 0,
+                          reinterpret_cast<cudaStream_t>(stream), dev);
+}
+
+int loza_ssa_prefill_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                            const int* cu_seqlens, int n_seqs, int total_tokens, int max_seqlen,
+                            int H, int d_qk, int d_v, int block, int n_sink, int n_local,
+                            float scale, loza_ssa_stream_t stream) {
+  if (!q || !k || !v || !o || !lse || !cu_seqlens) return LOZA_SSA_ERR_NULL;
+  if (n_seqs < 1 || n_seqs > kMaxVarlenSeqs || total_tokens < 1 || max_seqlen < 1 || H < 1 ||
+      !std::isfinite(scale))
+    return LOZA_SSA_ERR_SHAPE;
+  if (!prefill_dims_ok(d_qk, d_v)) return LOZA_SSA_ERR_HEAD_DIM;
+  if (block != 128) return LOZA_SSA_ERR_BLOCK;
+  if (n_sink < 0 || n_local < 1) return LOZA_SSA_ERR_WINDOW;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(lse, 4) || !aligned(cu_seqlens, 4))
+    return LOZA_SSA_ERR_ALIGN;
+  // sum_s ceil(len_s/128) <= total/128 + n_seqs bounds the work-item count
+  const long long upper = (long long)H * ((long long)total_tokens / 128 + n_seqs);
+  if (upper >= (1ll << 31)) return LOZA_SSA_ERR_SHAPE;
+  DeviceInfo dev;
+  int rc = device_info(dev);
+  if (rc != LOZA_SSA_OK) return rc;
+  loza::PrefillParams prm{};
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  prm.cu_seqlens = cu_seqlens;
+  prm.n_seqs = n_seqs;
+  prm.H = H;
+  prm.L = max_seqlen;
+  prm.plane_rows = total_tokens;
+  prm.n_sink = n_sink;
+  prm.n_local = n_local;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.total_items = 0;
+  return dispatch_prefill(d_qk, d_v, q, k, v, prm, (uint64_t)total_tokens, (uint64_t)H,
+                          (int)upper, n_seqs + 1, reinterpret_cast<cudaStream_t>(stream), dev);
+}
+
+size_t loza_ssa_decode_workspace_size(int B, int H_q, int d_v, int n_sink, int n_local) {
+  if (B < 1 || H_q < 1 || d_v != loza::kDecodeDv || n_sink < 0 || n_local < 1 ||
+      n_sink + n_local > kMaxDecodeWindow)
+    return 0;
+  const size_t rows = decode_partial_floats(B, H_q, n_sink + n_local);
+  const size_t o_bytes = rows * loza::kDecodeDv * sizeof(float);
+  const size_t lse_bytes = rows * sizeof(float);
+  return ((o_bytes + 255) / 256) * 256 + ((lse_bytes + 255) / 256) * 256;
+}
+
+int loza_ssa_decode(const void* q, const void* paged_kv, const int* page_table,
+                    const int* seq_lens, void* o, float* lse, int B, int H_q, int d_qk, int d_v,
+                    int page_size, int max_pages, int n_pages, int n_sink, int n_local,
+                    float scale, void* workspace, size_t workspace_bytes,
+                    loza_ssa_stream_t stream) {
+  if (!q || !paged_kv || !page_table || !seq_lens || !o || !lse) return LOZA_SSA_ERR_NULL;
+  if (B < 1 || H_q < 1 || max_pages < 1 || n_pages < 1 || !std::isfinite(scale))
+    return LOZA_SSA_ERR_SHAPE;
+  if (B > 65535 || (H_q + 127) / 128 > 65535 || (long long)n_pages * 128 >= (1ll << 31))
+    return LOZA_SSA_ERR_SHAPE;
+  if (d_qk != loza::kDecodeDqk || d_v != loza::kDecodeDv) return LOZA_SSA_ERR_HEAD_DIM;
+  if (page_size != 128) return LOZA_SSA_ERR_BLOCK;
+  if (n_sink < 0 || n_local < 1 || n_sink + n_local > kMaxDecodeWindow) return LOZA_SSA_ERR_WINDOW;
+  if (!aligned(q, 16) || !aligned(paged_kv, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+      !aligned(page_table, 4) || !aligned(seq_lens, 4))
+    return LOZA_SSA_ERR_ALIGN;
+  const size_t need = loza_ssa_decode_workspace_size(B, H_q, d_v, n_sink, n_local);
+  if (!workspace || workspace_bytes < need) return LOZA_SSA_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return LOZA_SSA_ERR_ALIGN;
+  DeviceInfo dev;
+  int rc = device_info(dev);
+  if (rc != LOZA_SSA_OK) return rc;
+
+  const int n_split = n_sink + n_local;
+  const int HG = (H_q + 127) / 128;
+  const size_t rows = decode_partial_floats(B, H_q, n_split);
+  loza::DecodeParams prm{};
+  prm.page_table = page_table;
+  prm.seq_lens = seq_lens;
+  prm.o_part = static_cast<float*>(workspace);
+  prm.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                          ((rows * loza::kDecodeDv * sizeof(float) + 255) / 256) * 256);
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  prm.B = B;
+  prm.H_q = H_q;
+  prm.HG = HG;
+  prm.max_pages = max_pages;
+  prm.n_pages = n_pages;
+  prm.n_sink = n_sink;
+  prm.n_local = n_local;
+  prm.n_split = n_split;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+
+  CUtensorMap mq, mkv;
+  if ((rc = make_map(&mq, q, loza::kDecodeDqk, (uint64_t)H_q, (uint64_t)B, 3)) != LOZA_SSA_OK)
+    return rc;
+  if ((rc = make_map(&mkv, paged_kv, loza::kDecodeDqk, (uint64_t)n_pages * 128, 1, 2)) != LOZA_SSA_OK)
+    return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaFuncSetAttribute(loza::ssa_decode_split_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       loza::DecodeLayout::SMEM_BYTES);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
+  dim3 grid(n_split, HG, B);
+  loza::ssa_decode_split_kernel<<<grid, 192, loza::DecodeLayout::SMEM_BYTES, s>>>(mq, mkv, prm);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "decode split launch");
+  loza::ssa_decode_merge_kernel<<<B * H_q, 128, 0, s>>>(prm);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "decode merge launch");
+  return LOZA_SSA_OK;
+}
+
+int loza_ssa_get_last_device_status(loza_ssa_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int v = 0;
+  if ((e = cudaMemcpyFromSymbol(&v, loza::g_loza_status, sizeof v)) != cudaSuccess)
+    return cuda_fail(e, "read device status");
+  const int zero = 0;
+  if ((e = cudaMemcpyToSymbol(loza::g_loza_status, &zero, sizeof zero)) != cudaSuccess)
+    return cuda_fail(e, "clear device status");
+  return v;
+}
+
+int loza_ssa_debug_enumerate_tiles(int n_qblocks, int n_sink, int n_local, int* tiles,
+                                   int* counts, int max_tiles, loza_ssa_stream_t stream) {
+  if (!tiles || !counts) return LOZA_SSA_ERR_NULL;
+  if (n_qblocks < 1 || max_tiles < 1) return LOZA_SSA_ERR_SHAPE;
+  if (n_sink < 0 || n_local < 1) return LOZA_SSA_ERR_WINDOW;
+  debug_tiles_kernel<<<(n_qblocks + 127) / 128, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      n_qblocks, n_sink, n_local, tiles, counts, max_tiles);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? LOZA_SSA_OK : cuda_fail(e, "debug tiles launch");
+}
+
+int loza_ssa_debug_decode_pages(const int* page_table, const int* seq_lens, int B, int max_pages,
+                                int n_pages, int page_size, int n_sink, int n_local, int* pages,
+                                int* counts, int max_tiles, loza_ssa_stream_t stream) {
+  if (!page_table || !seq_lens || !pages || !counts) return LOZA_SSA_ERR_NULL;
+  if (B < 1 || max_pages < 1 || n_pages < 1 || max_tiles < 1) return LOZA_SSA_ERR_SHAPE;
+  if (page_size != 128) return LOZA_SSA_ERR_BLOCK;
+  if (n_sink < 0 || n_local < 1) return LOZA_SSA_ERR_WINDOW;
+  loza::DecodeParams prm{};
+  prm.page_table = page_table;
+  prm.seq_lens = seq_lens;
+  prm.B = B;
+  prm.max_pages = max_pages;
+  prm.n_pages = n_pages;
+  prm.n_sink = n_sink;
+  prm.n_local = n_local;
+  debug_decode_pages_kernel<<<(B + 127) / 128, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      prm, pages, counts, max_tiles);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? LOZA_SSA_OK : cuda_fail(e, "debug decode pages launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,479 @@
+// prefill.cuh -- SSA prefill on sm_100a: TMA + tcgen05 (TMEM accumulators),
+// warp-specialised, persistent.
+//
+// One CTA per SM walks a static stride of work items (sequence, head, 128-row
+// query block).  For each item the tile scheduler lists the key blocks of the
+// SSA window (sink block(s) first, then the local run, the causal diagonal
+// block last).  Per key tile j:
+//
+//     S_j   = Q K_j^T                       tcgen05.mma, smem x smem -> TMEM (fp32)
+//     P_j   = exp2(S_j*scale*log2e - m)     softmax warps: tcgen05.ld, row max,
+//                                           exp2, row sum; P (bf16) written back
+//                                           into the S columns with tcgen05.st
+//     O    += P_j V_j                       tcgen05.mma, TMEM x smem -> TMEM (fp32)
+//
+// which is the max-subtracted ("CSA/HCA tutorial" §7.1) masked softmax of
+// "LoZA：ZigZag稀疏注意力机制" §2.1, computed online over the window's tiles:
+// the running max m only moves when a row's new maximum exceeds it by more
+// than kRescaleThreshold (log2 units); then the warp rescales its rows of O
+// in TMEM by exp2(m_old - m_new) before the next P.V.  The final O = acc / l
+// and LSE = (m + log2 l) ln 2 are exact for any choice of m.
+//
+// Warp roles (192 threads):
+//   warps 0-3  softmax + correction + epilogue; thread r owns query row r
+//              (TMEM lane r; a warp may only touch its own 32-lane quarter)
+//   warp 4     TMA producer (one elected lane)
+//   warp 5     TMEM allocator + MMA issuer (one elected lane)
+//
+// TMEM (512 columns x 128 lanes, fp32): S0 = cols [0,128), S1 = [128,256),
+// O = [256, 256+DV).  P_j (bf16 pairs) overwrites the first 64 columns of its
+// S buffer.  S is double-buffered so the tensor core computes S_{j+1} while
+// the softmax warps work on S_j.
+//
+// Shared memory (1024-byte aligned, 128B-swizzled TMA boxes of 64 bf16
+// columns x 128 rows = 16 KB "chunks"):  Q [DQK/64 chunks], K ring
+// [2 stages], V ring [2 stages], mbarriers, and for packed varlen input the
+// per-sequence work-item prefix.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+#include "schedule.cuh"
+
+namespace loza {
+
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: P values stay <= 2^8
+
+struct PrefillParams {
+  __nv_bfloat16* o;
+  float* lse;
+  const int* cu_seqlens;  // nullptr: dense [B,H,L,d]; else packed [H,total,d]
+  int n_seqs;             // dense: B
+  int H;
+  int L;                  // dense sequence length
+  int plane_rows;         // rows of one TMA plane: dense L, packed total_tokens
+  int n_sink;
+  int n_local;
+  float scale_log2;       // scale * log2(e)
+  int total_items;        // dense: B*H*ceil(L/128); packed: computed on the device
+};
+
+template <int DQK, int DV>
+struct PrefillLayout {
+  static constexpr int KCH = DQK / 64;
+  static constexpr int VCH = DV / 64;
+  static constexpr int CHUNK = 128 * 128;  // one swizzled [128 rows x 64 bf16] box
+  static constexpr int Q_BYTES = KCH * CHUNK;
+  static constexpr int K_BYTES = KCH * CHUNK;
+  static constexpr int V_BYTES = VCH * CHUNK;
+  static constexpr int KST = 2;  // K/V ring depth
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + KST * K_BYTES;
+  static constexpr int OFF_BAR = OFF_V + KST * V_BYTES;
+  // barrier indices
+  static constexpr int B_Q_FULL = 0, B_Q_EMPTY = 1;
+  static constexpr int B_K_FULL = 2, B_K_EMPTY = B_K_FULL + KST;
+  static constexpr int B_V_FULL = B_K_EMPTY + KST, B_V_EMPTY = B_V_FULL + KST;
+  static constexpr int B_S_FULL = B_V_EMPTY + KST;  // 2
+  static constexpr int B_P_FULL = B_S_FULL + 2;     // 2
+  static constexpr int B_O_DONE = B_P_FULL + 2;
+  static constexpr int B_O_EMPTY = B_O_DONE + 1;
+  static constexpr int B_DRAIN = B_O_EMPTY + 1;
+  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // [0] tmem base, [1] abort, [2] items
+  static constexpr int OFF_PREFIX = OFF_MISC + 16;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int TM_O = 256;
+  static constexpr int MIN_SMEM = 120 * 1024;  // keeps one CTA (and one TMEM owner) per SM
+  static constexpr size_t smem_bytes(int n_prefix) {
+    size_t need = (size_t)OFF_PREFIX + 4 * (size_t)n_prefix + 1024;  // + alignment slack
+    return need < (size_t)MIN_SMEM ? (size_t)MIN_SMEM : need;
+  }
+};
+
+struct WorkItem {
+  int z;          // TMA plane: dense b*H + h, packed h
+  int seq_start;  // first row of the sequence inside the plane
+  int len;        // sequence length
+  int qb;         // query block
+};
+
+__device__ __forceinline__ WorkItem decode_item(int item, const PrefillParams& p,
+                                                const int* prefix) {
+  WorkItem w;
+  if (p.cu_seqlens == nullptr) {
+    const int nb = (p.L + 127) >> 7;
+    w.qb = item % nb;
+    w.z = item / nb;
+    w.seq_start = 0;
+    w.len = p.L;
+  } else {
+    int lo = 0, hi = p.n_seqs - 1;  // largest s with prefix[s] <= item
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (prefix[mid] <= item) lo = mid; else hi = mid - 1;
+    }
+    const int start = __ldg(p.cu_seqlens + lo);
+    const int len = __ldg(p.cu_seqlens + lo + 1) - start;
+    const int nb = (len + 127) >> 7;
+    const int r = item - prefix[lo];
+    w.z = r / nb;
+    w.qb = r - w.z * nb;
+    w.seq_start = start;
+    w.len = len;
+  }
+  return w;
+}
+
+// Warp 0: work-item count (and, for packed input, the per-sequence prefix of
+// H * ceil(len/128) items).  Invalid cu_seqlens -> 0 items + status bit.
+__device__ __forceinline__ void prefill_count_items(const PrefillParams& p, int* prefix,
+                                                    uint32_t* misc, int lane) {
+  if (p.cu_seqlens == nullptr) {
+    if (lane == 0) misc[2] = (uint32_t)p.total_items;
+    return;
+  }
+  const int n = p.n_seqs;
+  const int per = (n + 31) / 32;
+  const int s0 = min(lane * per, n), s1 = min(s0 + per, n);
+  int local = 0, bad = 0;
+  for (int s = s0; s < s1; ++s) {
+    const int a = __ldg(p.cu_seqlens + s), b = __ldg(p.cu_seqlens + s + 1);
+    if (b < a) bad = 1;
+    local += p.H * ((b - a + 127) >> 7);
+  }
+  int incl = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  int run = incl - local;
+  for (int s = s0; s < s1; ++s) {
+    prefix[s] = run;
+    run += p.H * ((__ldg(p.cu_seqlens + s + 1) - __ldg(p.cu_seqlens + s) + 127) >> 7);
+  }
+  if (lane == 0 && (__ldg(p.cu_seqlens) != 0 || __ldg(p.cu_seqlens + n) != p.plane_rows)) bad = 1;
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  bad = __any_sync(0xffffffffu, bad);
+  if (lane == 0) {
+    prefix[n] = total;
+    misc[2] = bad ? 0u : (uint32_t)total;
+    if (bad) atomicOr(&g_loza_status, 8);
+  }
+}
+
+template <int DQK, int DV>
+__global__ void __launch_bounds__(192, 1)
+    ssa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
+  using Lay = PrefillLayout<DQK, DV>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  int* prefix = reinterpret_cast<int*>(smem + Lay::OFF_PREFIX);
+  auto bar = [&](int i) -> uint32_t { return sb + Lay::OFF_BAR + 8 * i; };
+  int* status = &g_loza_status;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(Lay::B_Q_FULL), 1);
+    mbar_init(bar(Lay::B_Q_EMPTY), 1);
+    for (int s = 0; s < Lay::KST; ++s) {
+      mbar_init(bar(Lay::B_K_FULL + s), 1);
+      mbar_init(bar(Lay::B_K_EMPTY + s), 1);
+      mbar_init(bar(Lay::B_V_FULL + s), 1);
+      mbar_init(bar(Lay::B_V_EMPTY + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(Lay::B_S_FULL + s), 1);
+      mbar_init(bar(Lay::B_P_FULL + s), 128);
+    }
+    mbar_init(bar(Lay::B_O_DONE), 1);
+    mbar_init(bar(Lay::B_O_EMPTY), 128);
+    mbar_init(bar(Lay::B_DRAIN), 1);
+    misc[1] = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) prefill_count_items(p, prefix, misc, lane);
+  if (warp == 4 && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+  }
+  if (warp == 5) {
+    tmem_alloc(sb + Lay::OFF_MISC, Lay::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+  const int total_items = (int)misc[2];
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int g = 0, it = 0;
+      int k_issued[Lay::KST] = {}, v_issued[Lay::KST] = {};
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++it) {
+        const WorkItem w = decode_item(item, p, prefix);
+        const TileRange tr = tile_range(w.qb, p.n_sink, p.n_local);
+        if (it > 0 && !mbar_wait(bar(Lay::B_Q_EMPTY), (it - 1) & 1, abort_flag, status, 1)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(bar(Lay::B_Q_FULL), Lay::Q_BYTES);
+#pragma unroll
+        for (int c = 0; c < Lay::KCH; ++c)
+          tma_load_3d(sb + Lay::OFF_Q + c * Lay::CHUNK, &tm_q, bar(Lay::B_Q_FULL), c * 64,
+                      w.seq_start + w.qb * 128, w.z);
+        for (int t = 0; t < tr.count; ++t, ++g) {
+          const int row = w.seq_start + tile_block(tr, t) * 128;
+          const int st = g % Lay::KST, use = g / Lay::KST;
+          if (use > 0 &&
+              !mbar_wait(bar(Lay::B_K_EMPTY + st), (use - 1) & 1, abort_flag, status, 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(Lay::B_K_FULL + st), Lay::K_BYTES);
+          ++k_issued[st];
+#pragma unroll
+          for (int c = 0; c < Lay::KCH; ++c)
+            tma_load_3d(sb + Lay::OFF_K + st * Lay::K_BYTES + c * Lay::CHUNK, &tm_k,
+                        bar(Lay::B_K_FULL + st), c * 64, row, w.z);
+          if (use > 0 &&
+              !mbar_wait(bar(Lay::B_V_EMPTY + st), (use - 1) & 1, abort_flag, status, 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(Lay::B_V_FULL + st), Lay::V_BYTES);
+          ++v_issued[st];
+#pragma unroll
+          for (int c = 0; c < Lay::VCH; ++c)
+            tma_load_3d(sb + Lay::OFF_V + st * Lay::V_BYTES + c * Lay::CHUNK, &tm_v,
+                        bar(Lay::B_V_FULL + st), c * 64, row, w.z);
+        }
+      }
+      if (!ok) {
+        // Let copies already in flight land before the CTA's smem goes away:
+        // a stage holds at most one unconsumed load, its newest phase.
+        for (int st = 0; st < Lay::KST; ++st) {
+          if (k_issued[st] > 0) mbar_wait_drain(bar(Lay::B_K_FULL + st), (k_issued[st] - 1) & 1);
+          if (v_issued[st] > 0) mbar_wait_drain(bar(Lay::B_V_FULL + st), (v_issued[st] - 1) & 1);
+        }
+        if (it > 0) mbar_wait_drain(bar(Lay::B_Q_FULL), (it - 1) & 1);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t id_s = idesc_bf16_f32(128, 128, false);
+      const uint32_t id_o = idesc_bf16_f32(128, DV, true);
+      int g0 = 0, it = 0;
+      bool ok = true;
+      // O += P_g V_g for tile t (global index g) of the current item
+      auto issue_pv = [&](int g, int t) -> bool {
+        const int st = g % Lay::KST;
+        if (!mbar_wait(bar(Lay::B_P_FULL + (g & 1)), (g >> 1) & 1, abort_flag, status, 1))
+          return false;
+        if (!mbar_wait(bar(Lay::B_V_FULL + st), (g / Lay::KST) & 1, abort_flag, status, 1))
+          return false;
+        if (t == 0 && it > 0 &&
+            !mbar_wait(bar(Lay::B_O_EMPTY), (it - 1) & 1, abort_flag, status, 1))
+          return false;
+        tc_fence_after();
+        const uint32_t p_tmem = tmem + (uint32_t)((g & 1) * 128);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t bdesc = sdesc_sw128(
+              sb + Lay::OFF_V + st * Lay::V_BYTES + kk * 2048, Lay::CHUNK, 1024);
+          mma_ts(tmem + Lay::TM_O, p_tmem + kk * 8, bdesc, id_o, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(bar(Lay::B_O_DONE));
+        mma_commit(bar(Lay::B_V_EMPTY + st));
+        return true;
+      };
+      for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++it) {
+        const WorkItem w = decode_item(item, p, prefix);
+        const TileRange tr = tile_range(w.qb, p.n_sink, p.n_local);
+        if (!mbar_wait(bar(Lay::B_Q_FULL), it & 1, abort_flag, status, 1)) {
+          ok = false;
+          break;
+        }
+        for (int t = 0; t < tr.count; ++t) {
+          const int g = g0 + t, st = g % Lay::KST;
+          if (!mbar_wait(bar(Lay::B_K_FULL + st), (g / Lay::KST) & 1, abort_flag, status, 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t s_tmem = tmem + (uint32_t)((g & 1) * 128);
+#pragma unroll
+          for (int kk = 0; kk < DQK / 16; ++kk) {
+            const uint32_t koff = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
+            const uint64_t adesc = sdesc_sw128(sb + Lay::OFF_Q + koff, 16, 1024);
+            const uint64_t bdesc = sdesc_sw128(sb + Lay::OFF_K + st * Lay::K_BYTES + koff, 16, 1024);
+            mma_ss(s_tmem, adesc, bdesc, id_s, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(Lay::B_S_FULL + (g & 1)));
+          mma_commit(bar(Lay::B_K_EMPTY + st));
+          if (t == tr.count - 1) mma_commit(bar(Lay::B_Q_EMPTY));
+          if (t > 0 && !issue_pv(g - 1, t - 1)) {
+            ok = false;
+            break;
+          }
+        }
+        if (!ok || !issue_pv(g0 + tr.count - 1, tr.count - 1)) {
+          ok = false;
+          break;
+        }
+        g0 += tr.count;
+      }
+      // every tcgen05.mma issued above has finished before TMEM is released
+      mma_commit(bar(Lay::B_DRAIN));
+      mbar_wait_drain(bar(Lay::B_DRAIN), 0);
+    }
+  } else {
+    // -------------------------------------------- softmax / correction / epilogue
+    const int row = threadIdx.x;                              // 0..127
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;   // this warp's TMEM lanes
+    const float sl2 = p.scale_log2;
+    int g0 = 0;
+    for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
+      const WorkItem w = decode_item(item, p, prefix);
+      const TileRange tr = tile_range(w.qb, p.n_sink, p.n_local);
+      float m = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int t = 0; t < tr.count; ++t) {
+        const int g = g0 + t;
+        const uint32_t s_tmem = tmem + lane_base + (uint32_t)((g & 1) * 128);
+        if (!mbar_wait(bar(Lay::B_S_FULL + (g & 1)), (g >> 1) & 1, abort_flag, status, 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) tmem_ld32(s_tmem + ch * 32, sr[ch]);
+        tmem_wait_ld();
+        if (t == tr.count - 1) {
+          // diagonal block: key c of the tile is visible to row r iff c <= r
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (ch * 32 + c > row) sr[ch][c] = __float_as_uint(-INFINITY);
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+          for (int c = 0; c < 32; ++c) mx = fmaxf(mx, __uint_as_float(sr[ch][c]));
+        const float m_tile = mx * sl2;
+        const bool first = (t == 0);
+        const float m_new = fmaxf(m, m_tile);
+        const bool need = !first && (m_new > m + kRescaleThreshold);
+        const bool rescale = __any_sync(0xffffffffu, need);
+        const float m_use = (first || rescale) ? m_new : m;
+        float rsum = 0.f;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int col = half * 64 + 2 * c;
+            const float x0 = __uint_as_float(sr[col >> 5][col & 31]);
+            const float x1 = __uint_as_float(sr[(col + 1) >> 5][(col + 1) & 31]);
+            const float p0 = ex2_approx(fmaf(x0, sl2, -m_use));
+            const float p1 = ex2_approx(fmaf(x1, sl2, -m_use));
+            rsum += p0 + p1;
+            pk[c] = pack_bf16x2(p0, p1);
+          }
+          tmem_st32(s_tmem + half * 32, pk);
+        }
+        if (!first) {
+          // O must hold P_{g-1} V_{g-1} before it is rescaled or read again
+          if (!mbar_wait(bar(Lay::B_O_DONE), (g - 1) & 1, abort_flag, status, 1)) {
+            ok = false;
+            break;
+          }
+          if (rescale) {
+            tc_fence_after();
+            const float alpha = ex2_approx(m - m_use);
+            l *= alpha;
+            const uint32_t o_tmem = tmem + lane_base + Lay::TM_O;
+#pragma unroll 1
+            for (int ch = 0; ch < DV / 32; ++ch) {
+              uint32_t orr[32];
+              tmem_ld32(o_tmem + ch * 32, orr);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; ++c)
+                orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
+              tmem_st32(o_tmem + ch * 32, orr);
+            }
+          }
+        }
+        l += rsum;
+        m = m_use;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(Lay::B_P_FULL + (g & 1)));
+      }
+      if (!ok) break;
+      // epilogue: O = acc / l (bf16), LSE = (m + log2 l) ln 2
+      const int gl = g0 + tr.count - 1;
+      if (!mbar_wait(bar(Lay::B_O_DONE), gl & 1, abort_flag, status, 1)) break;
+      tc_fence_after();
+      const int r_in_seq = w.qb * 128 + row;
+      const bool valid = r_in_seq < w.len;
+      const size_t orow = (size_t)w.z * (size_t)p.plane_rows + (size_t)(w.seq_start + r_in_seq);
+      const float inv_l = 1.f / l;
+      const uint32_t o_tmem = tmem + lane_base + Lay::TM_O;
+#pragma unroll 1
+      for (int ch = 0; ch < DV / 32; ++ch) {
+        uint32_t orr[32];
+        tmem_ld32(o_tmem + ch * 32, orr);
+        tmem_wait_ld();
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(p.o + orow * DV + ch * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 pkt;
+            pkt.x = pack_bf16x2(__uint_as_float(orr[8 * v + 0]) * inv_l,
+                                __uint_as_float(orr[8 * v + 1]) * inv_l);
+            pkt.y = pack_bf16x2(__uint_as_float(orr[8 * v + 2]) * inv_l,
+                                __uint_as_float(orr[8 * v + 3]) * inv_l);
+            pkt.z = pack_bf16x2(__uint_as_float(orr[8 * v + 4]) * inv_l,
+                                __uint_as_float(orr[8 * v + 5]) * inv_l);
+            pkt.w = pack_bf16x2(__uint_as_float(orr[8 * v + 6]) * inv_l,
+                                __uint_as_float(orr[8 * v + 7]) * inv_l);
+            dst[v] = pkt;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(Lay::B_O_EMPTY));
+      if (valid) p.lse[orow] = (m + __log2f(l)) * kLn2;
+      g0 += tr.count;
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Lay::TMEM_COLS);
+  }
+}
+
+}  // namespace loza

@@ -1,0 +1,222 @@
+"""Thin Python binding of libloza_ssa.so (argument marshalling only).
+
+Every function here has the name of the C entry point it calls (see
+include/loza_ssa.h) and does nothing but check that tensors are CUDA,
+contiguous and of the right dtype, allocate outputs the caller did not pass,
+and hand raw pointers, sizes and the current CUDA stream to the library.
+All attention work runs in the library's sm_100a kernels; if the library is
+missing this module raises instead of falling back to anything else.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libloza_ssa.so")
+_lib = None
+
+LOZA_SSA_DEV_WAIT_TIMEOUT = 1
+LOZA_SSA_DEV_BAD_PAGE = 2
+LOZA_SSA_DEV_BAD_SEQLEN = 4
+LOZA_SSA_DEV_BAD_CU_SEQLENS = 8
+
+
+class LozaSsaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(message)
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m block_sparse_streaming_ssa_b200.build`"
+                " (there is no fallback implementation)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.loza_ssa_prefill.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
+                                       f32, vp]
+        L.loza_ssa_prefill.restype = i32
+        L.loza_ssa_prefill_varlen.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                              i32, i32, i32, f32, vp]
+        L.loza_ssa_prefill_varlen.restype = i32
+        L.loza_ssa_decode.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                      i32, i32, f32, vp, sz, vp]
+        L.loza_ssa_decode.restype = i32
+        L.loza_ssa_decode_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+        L.loza_ssa_decode_workspace_size.restype = sz
+        L.loza_ssa_status_string.argtypes = [i32]
+        L.loza_ssa_status_string.restype = ctypes.c_char_p
+        L.loza_ssa_last_error_string.argtypes = []
+        L.loza_ssa_last_error_string.restype = ctypes.c_char_p
+        L.loza_ssa_get_last_device_status.argtypes = [vp]
+        L.loza_ssa_get_last_device_status.restype = i32
+        L.loza_ssa_debug_enumerate_tiles.argtypes = [i32, i32, i32, vp, vp, i32, vp]
+        L.loza_ssa_debug_enumerate_tiles.restype = i32
+        L.loza_ssa_debug_decode_pages.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp, vp,
+                                                  i32, vp]
+        L.loza_ssa_debug_decode_pages.restype = i32
+        L.loza_ssa_version.argtypes = []
+        L.loza_ssa_version.restype = i32
+        _lib = L
+    return _lib
+
+
+def loza_ssa_status_string(status: int) -> str:
+    return lib().loza_ssa_status_string(status).decode()
+
+
+def loza_ssa_last_error_string() -> str:
+    return lib().loza_ssa_last_error_string().decode()
+
+
+def loza_ssa_version() -> int:
+    return lib().loza_ssa_version()
+
+
+def _check(rc: int) -> None:
+    if rc != 0:
+        detail = loza_ssa_last_error_string() if rc == -8 else ""
+        raise LozaSsaError(rc, f"libloza_ssa: {loza_ssa_status_string(rc)} ({rc}) {detail}".strip())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: torch.Tensor) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t: torch.Tensor, dtype, name: str) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def loza_ssa_prefill(q, k, v, o=None, lse=None, block=128, n_sink=1, n_local=7, scale=None,
+                     stream=None):
+    """Dense SSA prefill.  q, k: bf16 [B,H,L,d_qk]; v: bf16 [B,H,L,d_v].
+    Returns (o bf16 [B,H,L,d_v], lse fp32 [B,H,L])."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, n)
+    B, H, L, d_qk = q.shape
+    d_v = v.shape[-1]
+    if tuple(k.shape) != (B, H, L, d_qk) or tuple(v.shape[:3]) != (B, H, L):
+        raise ValueError("q, k, v shapes disagree")
+    if o is None:
+        o = torch.empty((B, H, L, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    _need(o, torch.bfloat16, "o")
+    _need(lse, torch.float32, "lse")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d_qk)
+    _check(lib().loza_ssa_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, L, d_qk,
+                                  d_v, block, n_sink, n_local, float(scale), _stream(stream)))
+    return o, lse
+
+
+def loza_ssa_prefill_varlen(q, k, v, cu_seqlens, max_seqlen, o=None, lse=None, block=128,
+                            n_sink=1, n_local=7, scale=None, stream=None):
+    """Packed varlen SSA prefill.  q, k: bf16 [H,total,d_qk]; v: bf16 [H,total,d_v];
+    cu_seqlens: int32 CUDA [n_seqs+1].  Returns (o [H,total,d_v], lse [H,total])."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, n)
+    _need(cu_seqlens, torch.int32, "cu_seqlens")
+    H, total, d_qk = q.shape
+    d_v = v.shape[-1]
+    if o is None:
+        o = torch.empty((H, total, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((H, total), dtype=torch.float32, device=q.device)
+    _need(o, torch.bfloat16, "o")
+    _need(lse, torch.float32, "lse")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d_qk)
+    n_seqs = cu_seqlens.numel() - 1
+    _check(lib().loza_ssa_prefill_varlen(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens), n_seqs, total,
+        int(max_seqlen), H, d_qk, d_v, block, n_sink, n_local, float(scale), _stream(stream)))
+    return o, lse
+
+
+def loza_ssa_decode_workspace_size(B, H_q, d_v=512, n_sink=1, n_local=7) -> int:
+    return int(lib().loza_ssa_decode_workspace_size(B, H_q, d_v, n_sink, n_local))
+
+
+def loza_ssa_decode(q, paged_kv, page_table, seq_lens, d_v=512, o=None, lse=None, page_size=128,
+                    n_sink=1, n_local=7, scale=None, workspace=None, stream=None):
+    """Paged SSA decode.  q: bf16 [B,H_q,d_qk]; paged_kv: bf16 [n_pages,page_size,d_qk];
+    page_table: int32 [B,max_pages]; seq_lens: int32 [B] (including the new token).
+    Returns (o bf16 [B,H_q,d_v], lse fp32 [B,H_q])."""
+    _need(q, torch.bfloat16, "q")
+    _need(paged_kv, torch.bfloat16, "paged_kv")
+    _need(page_table, torch.int32, "page_table")
+    _need(seq_lens, torch.int32, "seq_lens")
+    B, H_q, d_qk = q.shape
+    n_pages = paged_kv.shape[0]
+    max_pages = page_table.shape[1]
+    if o is None:
+        o = torch.empty((B, H_q, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H_q), dtype=torch.float32, device=q.device)
+    _need(o, torch.bfloat16, "o")
+    _need(lse, torch.float32, "lse")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d_qk)
+    need = loza_ssa_decode_workspace_size(B, H_q, d_v, n_sink, n_local)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _need(workspace, torch.uint8, "workspace")
+    _check(lib().loza_ssa_decode(
+        _ptr(q), _ptr(paged_kv), _ptr(page_table), _ptr(seq_lens), _ptr(o), _ptr(lse), B, H_q,
+        d_qk, d_v, page_size, max_pages, n_pages, n_sink, n_local, float(scale), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
+    return o, lse
+
+
+def loza_ssa_get_last_device_status(stream=None) -> int:
+    rc = lib().loza_ssa_get_last_device_status(_stream(stream))
+    if rc < 0:
+        _check(rc)
+    return rc
+
+
+def loza_ssa_debug_enumerate_tiles(n_qblocks, n_sink=1, n_local=7, max_tiles=None, device="cuda",
+                                   stream=None):
+    """The kernels' tile scheduler run on the device: (tiles [n_qblocks,max_tiles], counts)."""
+    if max_tiles is None:
+        max_tiles = n_sink + n_local
+    tiles = torch.full((n_qblocks, max_tiles), -1, dtype=torch.int32, device=device)
+    counts = torch.zeros(n_qblocks, dtype=torch.int32, device=device)
+    _check(lib().loza_ssa_debug_enumerate_tiles(n_qblocks, n_sink, n_local, _ptr(tiles),
+                                                _ptr(counts), max_tiles, _stream(stream)))
+    return tiles, counts
+
+
+def loza_ssa_debug_decode_pages(page_table, seq_lens, n_pages, page_size=128, n_sink=1, n_local=7,
+                                max_tiles=None, stream=None):
+    """The decode kernel's page selection run on the device: (pages [B,max_tiles], counts)."""
+    _need(page_table, torch.int32, "page_table")
+    _need(seq_lens, torch.int32, "seq_lens")
+    B, max_pages = page_table.shape
+    if max_tiles is None:
+        max_tiles = n_sink + n_local
+    pages = torch.full((B, max_tiles), -2, dtype=torch.int32, device=page_table.device)
+    counts = torch.zeros(B, dtype=torch.int32, device=page_table.device)
+    _check(lib().loza_ssa_debug_decode_pages(
+        _ptr(page_table), _ptr(seq_lens), B, max_pages, n_pages, page_size, n_sink, n_local,
+        _ptr(pages), _ptr(counts), max_tiles, _stream(stream)))
+    return pages, counts

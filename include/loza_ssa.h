@@ -1,0 +1,165 @@
+/*
+ * loza_ssa.h -- C ABI of libloza_ssa.so: streaming sparse attention (SSA) for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (all entry points): masked softmax attention
+ *
+ *     O_i = sum_{j : M_ij = 1} exp(scale * q_i.k_j) v_j / sum_{j : M_ij = 1} exp(scale * q_i.k_j)
+ *
+ * ("LoZA：ZigZag稀疏注意力机制", §2.1 问题形式化, second formula) with the SSA
+ * mask of LongCat's LoZA (QbitAI article on LoZA, paragraph on the 1024-token
+ * sparse window: one global block plus seven local blocks, 128 tokens each):
+ *
+ *     M_ij = 1  iff  j <= i  and  floor(j/block) in W(floor(i/block))
+ *     W(b) = {0 .. n_sink-1}  U  {max(n_sink, b-n_local+1) .. b}
+ *
+ * The defaults n_sink = 1, n_local = 7, block = 128 give the paper's window:
+ * the global block 0 plus the query's own block and the six before it.  The
+ * global block sits at the start of the sequence (LongCat LSA article,
+ * 机制 1 流感知索引: sink tokens are the first tokens of the sequence).
+ * Alongside O every call writes LSE_i = ln sum_{j : M_ij = 1} exp(scale * q_i.k_j)
+ * (natural log, scale included) in fp32.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers, caller-owned, row-major and
+ *     contiguous.  bf16 tensors hold IEEE bfloat16; lse is fp32.
+ *   - bf16 tensor pointers must be 16-byte aligned, lse 4-byte aligned.
+ *   - Work is enqueued on `stream` and is asynchronous; no call synchronises
+ *     the device, and no call allocates device memory.  Inputs are never
+ *     modified.  Calls on different streams may run concurrently.
+ *   - On any non-zero status nothing has been launched.
+ *   - Errors found by the kernels themselves (a page id outside the pool, a
+ *     sequence length outside the page table, bad cu_seqlens, a pipeline wait
+ *     that timed out) are recorded in a per-device status word instead of
+ *     faulting; read it with loza_ssa_get_last_device_status().
+ *
+ * Status codes (return values) are the LOZA_SSA_* values below.
+ */
+#ifndef LOZA_SSA_H
+#define LOZA_SSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; 0 is the legacy default stream. */
+typedef struct CUstream_st* loza_ssa_stream_t;
+
+enum {
+  LOZA_SSA_OK = 0,
+  LOZA_SSA_ERR_NULL = -1,           /* a required pointer is NULL                              */
+  LOZA_SSA_ERR_SHAPE = -2,          /* a size is out of range (<= 0, too large), scale not finite */
+  LOZA_SSA_ERR_HEAD_DIM = -3,       /* (d_qk, d_v) not supported by the kernels                 */
+  LOZA_SSA_ERR_BLOCK = -4,          /* block / page_size other than 128                         */
+  LOZA_SSA_ERR_WINDOW = -5,         /* n_sink < 0, n_local < 1, or too many window blocks      */
+  LOZA_SSA_ERR_ALIGN = -6,          /* a pointer is not aligned as required                     */
+  LOZA_SSA_ERR_WORKSPACE = -7,      /* workspace missing or smaller than the size query says    */
+  LOZA_SSA_ERR_CUDA = -8,           /* a CUDA runtime call failed (see loza_ssa_last_error_string) */
+};
+
+/* Bits of the device status word (loza_ssa_get_last_device_status). */
+enum {
+  LOZA_SSA_DEV_WAIT_TIMEOUT = 1,    /* a pipeline wait gave up; that CTA skipped its work      */
+  LOZA_SSA_DEV_BAD_PAGE = 2,        /* page_table entry outside [0, n_pages); split skipped    */
+  LOZA_SSA_DEV_BAD_SEQLEN = 4,      /* decode seq_len < 1 or > max_pages * page_size           */
+  LOZA_SSA_DEV_BAD_CU_SEQLENS = 8,  /* cu_seqlens not starting at 0, decreasing, or != total   */
+};
+
+/*
+ * Dense SSA prefill (causal self-attention of every token of every sequence).
+ *   q, k : bf16 [B, H, L, d_qk]        v, o : bf16 [B, H, L, d_v]      lse : fp32 [B, H, L]
+ *   (d_qk, d_v) in {(64,64), (128,128), (192,128)}; block must be 128;
+ *   n_sink >= 0, n_local >= 1; scale finite (e.g. 1/sqrt(d_qk), the sqrt(d)
+ *   of "LoZA：ZigZag稀疏注意力机制" §2.1).  L need not be a multiple of 128.
+ * Returns LOZA_SSA_OK or a negative status; o and lse are written on success.
+ */
+int loza_ssa_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int H, int L, int d_qk, int d_v, int block, int n_sink, int n_local,
+                     float scale, loza_ssa_stream_t stream);
+
+/*
+ * Packed variable-length SSA prefill.  Sequence s occupies tokens
+ * [cu_seqlens[s], cu_seqlens[s+1]) of the packed axis; block indices count from
+ * each sequence's own first token, and no key crosses a sequence boundary.
+ *   q, k : bf16 [H, total_tokens, d_qk]   v, o : bf16 [H, total_tokens, d_v]
+ *   lse  : fp32 [H, total_tokens]         cu_seqlens : DEVICE int32 [n_seqs + 1]
+ *   1 <= n_seqs <= 4096.  max_seqlen is the caller's bound on any sequence
+ *   length (used to size the launch; a longer sequence is still computed).
+ * Other arguments as for loza_ssa_prefill.
+ */
+int loza_ssa_prefill_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                            const int* cu_seqlens, int n_seqs, int total_tokens, int max_seqlen,
+                            int H, int d_qk, int d_v, int block, int n_sink, int n_local,
+                            float scale, loza_ssa_stream_t stream);
+
+/*
+ * Paged SSA decode, absorbed-MLA layout: one new query token per sequence,
+ * H_q query heads all attending one shared latent key/value row per token.
+ *   q          : bf16 [B, H_q, d_qk]
+ *   paged_kv   : bf16 [n_pages, page_size, d_qk]; the value of a token is the
+ *                first d_v entries of its row
+ *   page_table : DEVICE int32 [B, max_pages]; logical page p of sequence b is
+ *                physical page page_table[b*max_pages + p]
+ *   seq_lens   : DEVICE int32 [B]; the length INCLUDING the new token, whose
+ *                position t = seq_len - 1 is the query position
+ *   o          : bf16 [B, H_q, d_v]          lse : fp32 [B, H_q]
+ *   (d_qk, d_v) must be (576, 512); page_size must be 128; the window reads
+ *   logical pages {0..n_sink-1} and the n_local pages ending at t's page.
+ *   workspace  : DEVICE scratch of at least
+ *                loza_ssa_decode_workspace_size(B, H_q, d_v, n_sink, n_local)
+ *                bytes, 256-byte aligned, owned by the caller, contents
+ *                irrelevant on entry and overwritten.
+ */
+int loza_ssa_decode(const void* q, const void* paged_kv, const int* page_table,
+                    const int* seq_lens, void* o, float* lse, int B, int H_q, int d_qk, int d_v,
+                    int page_size, int max_pages, int n_pages, int n_sink, int n_local,
+                    float scale, void* workspace, size_t workspace_bytes,
+                    loza_ssa_stream_t stream);
+
+/* Bytes of workspace loza_ssa_decode needs (0 on invalid arguments). */
+size_t loza_ssa_decode_workspace_size(int B, int H_q, int d_v, int n_sink, int n_local);
+
+/* Static description of a status code (never NULL). */
+const char* loza_ssa_status_string(int status);
+
+/* Text of the last CUDA error seen by this thread's calls ("" if none). */
+const char* loza_ssa_last_error_string(void);
+
+/*
+ * Waits for `stream`, then returns and clears the current device's status
+ * word: 0 if no kernel reported a problem since the last read, else an OR of
+ * LOZA_SSA_DEV_* bits.  Returns LOZA_SSA_ERR_CUDA if the wait or read failed.
+ */
+int loza_ssa_get_last_device_status(loza_ssa_stream_t stream);
+
+/*
+ * Debug: run the kernels' own tile scheduler on the device.  For every query
+ * block qb in [0, n_qblocks) writes the key blocks it visits, ascending, to
+ * tiles[qb*max_tiles ...] and their number to counts[qb] (DEVICE int32 buffers
+ * of n_qblocks*max_tiles and n_qblocks entries).  A count above max_tiles is
+ * reported but only max_tiles ids are written.
+ */
+int loza_ssa_debug_enumerate_tiles(int n_qblocks, int n_sink, int n_local, int* tiles,
+                                   int* counts, int max_tiles, loza_ssa_stream_t stream);
+
+/*
+ * Debug: run the decode kernel's page selection on the device.  For every
+ * sequence b writes the PHYSICAL pages the decode window reads (logical order)
+ * to pages[b*max_tiles ...] and their number to counts[b]; entries it would
+ * reject are written as -1 and flagged in the device status word.
+ */
+int loza_ssa_debug_decode_pages(const int* page_table, const int* seq_lens, int B, int max_pages,
+                                int n_pages, int page_size, int n_sink, int n_local, int* pages,
+                                int* counts, int max_tiles, loza_ssa_stream_t stream);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int loza_ssa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LOZA_SSA_H */

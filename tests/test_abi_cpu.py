@@ -1,0 +1,142 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every
+entry point include/loza_ssa.h declares, and rejects bad arguments with the
+documented status codes before touching CUDA (no compute calls here)."""
+import ctypes
+import os
+import re
+import shutil
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "loza_ssa.h")
+
+pytestmark = pytest.mark.skipif(shutil.which("nvcc") is None and not os.path.exists(
+    os.path.join(ROOT, "block_sparse_streaming_ssa_b200", "libloza_ssa.so")),
+    reason="neither nvcc nor a built library is available")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from block_sparse_streaming_ssa_b200 import build, loza_ssa
+    build.build()
+    return loza_ssa.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(loza_ssa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("loza_ssa_prefill", "loza_ssa_prefill_varlen", "loza_ssa_decode",
+                     "loza_ssa_decode_workspace_size", "loza_ssa_status_string",
+                     "loza_ssa_get_last_device_status", "loza_ssa_debug_enumerate_tiles",
+                     "loza_ssa_debug_decode_pages"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+        assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
+
+
+def test_status_strings(L):
+    from block_sparse_streaming_ssa_b200 import loza_ssa as api
+    for code in range(0, -9, -1):
+        s = api.loza_ssa_status_string(code)
+        assert s and s != "unknown status", code
+    assert api.loza_ssa_status_string(-99) == "unknown status"
+    assert api.loza_ssa_version() >= 10000
+
+
+def test_decode_workspace_size(L):
+    from block_sparse_streaming_ssa_b200 import loza_ssa as api
+    # B * ceil(H_q/128) * (n_sink+n_local) * 128 rows of 512 fp32 (+1 fp32 LSE), 256-B rounded
+    rows = 32 * 1 * 8 * 128
+    want = -(-rows * 512 * 4 // 256) * 256 + -(-rows * 4 // 256) * 256
+    assert api.loza_ssa_decode_workspace_size(32, 128, 512, 1, 7) == want
+    assert api.loza_ssa_decode_workspace_size(2, 200, 512, 1, 7) == \
+        -(-2 * 2 * 8 * 128 * 2048 // 256) * 256 + -(-2 * 2 * 8 * 128 * 4 // 256) * 256
+    assert api.loza_ssa_decode_workspace_size(32, 128, 256, 1, 7) == 0      # d_v unsupported
+    assert api.loza_ssa_decode_workspace_size(32, 128, 512, 1, 0) == 0      # n_local < 1
+
+
+def _prefill(L, q=0x1000, k=0x1000, v=0x1000, o=0x1000, lse=0x1000, B=1, H=2, Ln=256, dqk=64,
+             dv=64, block=128, ns=1, nl=7, scale=0.125):
+    vp = ctypes.c_void_p
+    return L.loza_ssa_prefill(vp(q), vp(k), vp(v), vp(o), vp(lse), B, H, Ln, dqk, dv, block, ns,
+                              nl, ctypes.c_float(scale), None)
+
+
+def test_prefill_argument_errors(L):
+    assert _prefill(L, q=0) == -1
+    assert _prefill(L, lse=0) == -1
+    assert _prefill(L, Ln=0) == -2
+    assert _prefill(L, B=0) == -2
+    assert _prefill(L, scale=float("nan")) == -2
+    assert _prefill(L, scale=float("inf")) == -2
+    assert _prefill(L, dqk=96, dv=96) == -3
+    assert _prefill(L, dqk=128, dv=64) == -3
+    assert _prefill(L, block=64) == -4
+    assert _prefill(L, ns=-1) == -5
+    assert _prefill(L, nl=0) == -5
+    assert _prefill(L, q=0x1008) == -6
+    assert _prefill(L, lse=0x1002) == -6
+
+
+def _decode(L, B=2, Hq=128, dqk=576, dv=512, ps=128, max_pages=16, n_pages=32, ns=1, nl=7,
+            ws=0x10000, ws_bytes=1 << 30, q=0x1000, pt=0x1000):
+    vp = ctypes.c_void_p
+    return L.loza_ssa_decode(vp(q), vp(0x1000), vp(pt), vp(0x1000), vp(0x1000), vp(0x1000), B,
+                             Hq, dqk, dv, ps, max_pages, n_pages, ns, nl, ctypes.c_float(0.04),
+                             vp(ws), ws_bytes, None)
+
+
+def test_decode_argument_errors(L):
+    assert _decode(L, q=0) == -1
+    assert _decode(L, B=0) == -2
+    assert _decode(L, n_pages=0) == -2
+    assert _decode(L, dqk=512) == -3
+    assert _decode(L, dv=256) == -3
+    assert _decode(L, ps=64) == -4
+    assert _decode(L, nl=0) == -5
+    assert _decode(L, ns=-1) == -5
+    assert _decode(L, q=0x1004) == -6
+    assert _decode(L, pt=0x1002) == -6
+    assert _decode(L, ws=0) == -7
+    assert _decode(L, ws_bytes=1024) == -7
+    assert _decode(L, ws=0x10010) == -6
+
+
+def test_varlen_argument_errors(L):
+    vp = ctypes.c_void_p
+    f = ctypes.c_float(0.1)
+    args = dict(n_seqs=2, total=300, maxlen=200, H=2, dqk=128, dv=128, block=128, ns=1, nl=7)
+
+    def call(cu=0x1000, **kw):
+        a = {**args, **kw}
+        return L.loza_ssa_prefill_varlen(vp(0x1000), vp(0x1000), vp(0x1000), vp(0x1000),
+                                          vp(0x1000), vp(cu), a["n_seqs"], a["total"],
+                                          a["maxlen"], a["H"], a["dqk"], a["dv"], a["block"],
+                                          a["ns"], a["nl"], f, None)
+    assert call(cu=0) == -1
+    assert call(n_seqs=0) == -2
+    assert call(n_seqs=5000) == -2
+    assert call(total=0) == -2
+    assert call(dqk=192, dv=192) == -3
+    assert call(block=256) == -4
+    assert call(nl=0) == -5
+    assert call(cu=0x1002) == -6
+
+
+def test_debug_argument_errors(L):
+    vp = ctypes.c_void_p
+    assert L.loza_ssa_debug_enumerate_tiles(4, 1, 7, vp(0), vp(0x1000), 8, None) == -1
+    assert L.loza_ssa_debug_enumerate_tiles(0, 1, 7, vp(0x1000), vp(0x1000), 8, None) == -2
+    assert L.loza_ssa_debug_enumerate_tiles(4, 1, 0, vp(0x1000), vp(0x1000), 8, None) == -5
+    assert L.loza_ssa_debug_decode_pages(vp(0x1000), vp(0x1000), 2, 8, 8, 64, 1, 7, vp(0x1000),
+                                         vp(0x1000), 8, None) == -4
