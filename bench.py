@@ -243,13 +243,13 @@ def e2e_prefill(w, steps):
 
 # ----------------------------------------------------------------- decode
 
-def decode_bench(iters, warmup, peaks, seed=0):
+def decode_bench(iters, warmup, peaks, seed=0, len_hi=None):
     import torch
     from block_sparse_streaming_ssa_b200 import synth
     from block_sparse_streaming_ssa_b200.loza_ssa import (loza_ssa_decode,
                                                           loza_ssa_decode_workspace_size)
     s = synth.DECODE
-    lens = synth.decode_seq_lens(seed, s.B, s.len_lo, s.len_hi)
+    lens = synth.decode_seq_lens(seed, s.B, s.len_lo, len_hi or s.len_hi)
     q, kv, pt, sl = synth.decode_inputs(lens, s.H_q, s.d_qk, seed=seed, device="cuda")
     ws = torch.empty(loza_ssa_decode_workspace_size(s.B, s.H_q, s.d_v), dtype=torch.uint8,
                      device="cuda")
@@ -274,7 +274,7 @@ def decode_bench(iters, warmup, peaks, seed=0):
     gbs = algo_bytes / (mean_ms * 1e-3) / 1e9
     return {
         "workload": f"ssa_decode B={s.B} H_q={s.H_q} d_qk={s.d_qk} d_v={s.d_v} paged 128, "
-                    f"seq_len U[{s.len_lo},{s.len_hi}] seed {seed}, random page permutation "
+                    f"seq_len U[{s.len_lo},{len_hi or s.len_hi}] seed {seed}, random page permutation "
                     f"over {kv.shape[0]} pages",
         "value": round(gbs, 1), "unit": "GB/s", "us_per_step": round(mean_ms * 1e3, 2),
         "median_us": round(statistics.median(ms) * 1e3, 2),
@@ -334,6 +334,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--decode-iters", type=int, default=30)
+    ap.add_argument("--decode-len-hi", type=int, default=None,
+                    help="shorter decode contexts (smaller page pool), for profiler captures")
     ap.add_argument("--cpu-budget-s", type=float, default=10.0)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -397,7 +399,8 @@ def main():
     if not args.no_decode:
         del w
         torch.cuda.empty_cache()
-        decode = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank)
+        decode = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
+                              len_hi=args.decode_len_hi)
 
     if rank != 0:
         if dist:

@@ -9,18 +9,21 @@
 //
 // Split kernel: one CTA per (window page, head group, sequence).
 //   TMA     the 128-token page (9 swizzled boxes of 64 columns = 144 KB) into
-//           smem, Q of the head group streamed in 64-column boxes (2-deep ring)
+//           smem, Q of the head group streamed in 64-column boxes (4-deep ring)
 //   MMA     S[128 heads x 128 keys] = Q K^T   (K = 576: 9 boxes x 4 k-steps)
-//   softmax mask keys past t, row max, exp2, row sum; P (bf16) -> smem
+//   softmax mask keys past t, row max, exp2, row sum; P (bf16) -> smem over
+//           the first two (by then consumed) Q ring slots
 //   MMA     O[128 x 512] = P V, two N=256 halves, V = the page's first 8 boxes
 //           read as an MN-major operand (no transpose copy)
-//   out     normalised partial O (fp32) and its LSE to the workspace
+//   out     normalised partial O (fp16) and its LSE (fp32) to the workspace
 // TMEM: S uses columns [0,128); O uses [0,512) once S has been read.
 //
-// Merge kernel: LSE = logsumexp_s LSE_s, O = sum_s exp(LSE_s - LSE) O_s.
+// Merge kernel (programmatic dependent launch after the split kernel):
+// LSE = logsumexp_s LSE_s, O = sum_s exp(LSE_s - LSE) O_s.
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "ptx.cuh"
 #include "schedule.cuh"
@@ -33,7 +36,7 @@ constexpr int kDecodeDv = 512;
 struct DecodeParams {
   const int* page_table;  // [B, max_pages]
   const int* seq_lens;    // [B]
-  float* o_part;          // [B, HG, n_split, 128, 512]
+  __half* o_part;         // [B, HG, n_split, 128, 512]
   float* lse_part;        // [B, HG, n_split, 128]
   __nv_bfloat16* o;       // [B, H_q, 512]
   float* lse;             // [B, H_q]
@@ -41,14 +44,14 @@ struct DecodeParams {
   float scale_log2;
 };
 
-// The decode window of sequence b, as the kernels select it.  Returns the
-// number of window pages (0 for an invalid seq_len, flagged in the status).
+// The decode window of sequence b, as the kernels select it.
 struct DecodeWindow {
   int t;       // query position
   int qb;      // logical page of the query
   TileRange tr;
 };
 
+// False for a seq_len outside [1, max_pages * 128].
 __device__ __forceinline__ bool decode_window(const DecodeParams& p, int b, DecodeWindow& w) {
   const int len = __ldg(p.seq_lens + b);
   if (len < 1 || (long long)len > (long long)p.max_pages * 128) return false;
@@ -69,14 +72,15 @@ __device__ __forceinline__ int decode_page(const DecodeParams& p, int b, const D
 struct DecodeLayout {
   static constexpr int CHUNK = 128 * 128;  // [128 rows x 64 bf16], 128B swizzle
   static constexpr int KV_CH = kDecodeDqk / 64;  // 9
+  static constexpr int QST = 4;                  // Q ring depth
   static constexpr int OFF_KV = 0;
-  static constexpr int OFF_Q = OFF_KV + KV_CH * CHUNK;  // 2-deep ring
-  static constexpr int OFF_P = OFF_Q + 2 * CHUNK;       // P [128 x 128] bf16 as 2 boxes
-  static constexpr int OFF_BAR = OFF_P + 2 * CHUNK;
-  static constexpr int B_KV_FULL = 0;                   // 9
-  static constexpr int B_Q_FULL = B_KV_FULL + KV_CH;    // 2
-  static constexpr int B_Q_EMPTY = B_Q_FULL + 2;        // 2
-  static constexpr int B_S_FULL = B_Q_EMPTY + 2;
+  static constexpr int OFF_Q = OFF_KV + KV_CH * CHUNK;
+  static constexpr int OFF_P = OFF_Q;  // P [128 x 128] bf16 (2 boxes) reuses Q slots 0-1
+  static constexpr int OFF_BAR = OFF_Q + QST * CHUNK;
+  static constexpr int B_KV_FULL = 0;                    // 9
+  static constexpr int B_Q_FULL = B_KV_FULL + KV_CH;     // QST
+  static constexpr int B_Q_EMPTY = B_Q_FULL + QST;       // QST
+  static constexpr int B_S_FULL = B_Q_EMPTY + QST;
   static constexpr int B_P_FULL = B_S_FULL + 1;
   static constexpr int B_O_FULL = B_P_FULL + 1;
   static constexpr int B_DRAIN = B_O_FULL + 1;
@@ -109,6 +113,7 @@ __global__ void __launch_bounds__(192, 1)
   }
   if (phys < 0) {
     if (threadIdx.x < 128) p.lse_part[part + threadIdx.x] = -INFINITY;  // empty split
+    asm volatile("griddepcontrol.launch_dependents;");
     return;
   }
 
@@ -123,7 +128,7 @@ __global__ void __launch_bounds__(192, 1)
 
   if (threadIdx.x == 0) {
     for (int c = 0; c < Lay::KV_CH; ++c) mbar_init(bar(Lay::B_KV_FULL + c), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < Lay::QST; ++s) {
       mbar_init(bar(Lay::B_Q_FULL + s), 1);
       mbar_init(bar(Lay::B_Q_EMPTY + s), 1);
     }
@@ -153,8 +158,9 @@ __global__ void __launch_bounds__(192, 1)
       int q_issued = 0;
       bool ok = true;
       auto load_q = [&](int c) -> bool {
-        const int st = c & 1;
-        if (c >= 2 && !mbar_wait(bar(Lay::B_Q_EMPTY + st), ((c >> 1) - 1) & 1, abort_flag, status, 1))
+        const int st = c % Lay::QST;
+        if (c >= Lay::QST &&
+            !mbar_wait(bar(Lay::B_Q_EMPTY + st), (c / Lay::QST - 1) & 1, abort_flag, status, 1))
           return false;
         mbar_arrive_expect_tx(bar(Lay::B_Q_FULL + st), Lay::CHUNK);
         tma_load_3d(sb + Lay::OFF_Q + st * Lay::CHUNK, &tm_q, bar(Lay::B_Q_FULL + st), c * 64,
@@ -162,18 +168,19 @@ __global__ void __launch_bounds__(192, 1)
         ++q_issued;
         return true;
       };
-      load_q(0);
+      // interleave the first Q boxes with the page so the first MMAs can start
+      // early; then the rest of the page; then Q boxes as ring slots free up
       for (int c = 0; c < Lay::KV_CH; ++c) {
+        if (c < Lay::QST) load_q(c);
         mbar_arrive_expect_tx(bar(Lay::B_KV_FULL + c), Lay::CHUNK);
         tma_load_2d(sb + Lay::OFF_KV + c * Lay::CHUNK, &tm_kv, bar(Lay::B_KV_FULL + c), c * 64,
                     phys * 128);
-        if (c == 0) load_q(1);
       }
-      for (int c = 2; ok && c < Lay::KV_CH; ++c) ok = load_q(c);
+      for (int c = Lay::QST; ok && c < Lay::KV_CH; ++c) ok = load_q(c);
       // every copy issued lands before the CTA exits (normally already consumed)
       for (int c = 0; c < Lay::KV_CH; ++c) mbar_wait_drain(bar(Lay::B_KV_FULL + c), 0);
-      for (int st = 0; st < 2; ++st) {
-        const int n = (q_issued - st + 1) / 2;  // loads issued into ring slot st
+      for (int st = 0; st < Lay::QST; ++st) {
+        const int n = (q_issued - st + Lay::QST - 1) / Lay::QST;  // loads issued into slot st
         if (n > 0) mbar_wait_drain(bar(Lay::B_Q_FULL + st), (n - 1) & 1);
       }
     }
@@ -184,9 +191,9 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t id_o = idesc_bf16_f32(128, 256, true);
       bool ok = true;
       for (int c = 0; ok && c < Lay::KV_CH; ++c) {
-        const int st = c & 1;
+        const int st = c % Lay::QST;
         ok = mbar_wait(bar(Lay::B_KV_FULL + c), 0, abort_flag, status, 1) &&
-             mbar_wait(bar(Lay::B_Q_FULL + st), (c >> 1) & 1, abort_flag, status, 1);
+             mbar_wait(bar(Lay::B_Q_FULL + st), (c / Lay::QST) & 1, abort_flag, status, 1);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -231,16 +238,24 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) tmem_ld32(tmem + lane_base + ch * 32, sr[ch]);
       tmem_wait_ld();
-      float mx = -INFINITY;
+      if (valid_keys < 128) {
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch)
+        for (int ch = 0; ch < 4; ++ch)
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          if (ch * 32 + c >= valid_keys) sr[ch][c] = __float_as_uint(-INFINITY);
-          mx = fmaxf(mx, __uint_as_float(sr[ch][c]));
-        }
-      const float m = mx * sl2;
-      float l = 0.f;
+          for (int c = 0; c < 32; ++c)
+            if (ch * 32 + c >= valid_keys) sr[ch][c] = __float_as_uint(-INFINITY);
+      }
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int c = 0; c < 128; c += 8)
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+          mx4[a] = fmax3(mx4[a], __uint_as_float(sr[(c + 2 * a) >> 5][(c + 2 * a) & 31]),
+                         __uint_as_float(sr[(c + 2 * a + 1) >> 5][(c + 2 * a + 1) & 31]));
+      const float m = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * sl2;
+      const uint64_t sl2x2 = f2_pack(sl2, sl2);
+      const uint64_t negm2 = f2_pack(-m, -m);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
       // P row h -> smem, K-major 128B-swizzled: box (key/64), row h, 16-byte unit u
       // holding keys 8u..8u+7 lands at unit u ^ (h & 7).
       uint8_t* prow = smem + Lay::OFF_P + h * 128;
@@ -252,15 +267,24 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int col = box * 64 + u * 8 + 2 * e;
-            const float p0 = ex2_approx(fmaf(__uint_as_float(sr[col >> 5][col & 31]), sl2, -m));
-            const float p1 =
-                ex2_approx(fmaf(__uint_as_float(sr[(col + 1) >> 5][(col + 1) & 31]), sl2, -m));
-            l += p0 + p1;
+            const uint64_t xx = f2_pack(__uint_as_float(sr[col >> 5][col & 31]),
+                                        __uint_as_float(sr[(col + 1) >> 5][(col + 1) & 31]));
+            float y0, y1;
+            f2_unpack(f2_fma(xx, sl2x2, negm2), y0, y1);
+            const float p0 = ex2_approx(y0);
+            const float p1 = ex2_approx(y1);
+            acc[e] = f2_add(acc[e], f2_pack(p0, p1));
             w4[e] = pack_bf16x2(p0, p1);
           }
           *reinterpret_cast<uint4*>(prow + box * Lay::CHUNK + ((u ^ (h & 7)) << 4)) =
               make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
+      }
+      float l;
+      {
+        float a0, a1;
+        f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
+        l = a0 + a1;
       }
       fence_async_shared();
       tc_fence_before();
@@ -268,8 +292,9 @@ __global__ void __launch_bounds__(192, 1)
 
       if (!mbar_wait(bar(Lay::B_O_FULL), 0, abort_flag, status, 1)) break;
       tc_fence_after();
+      asm volatile("griddepcontrol.launch_dependents;");
       const bool valid = hg * 128 + h < p.H_q;
-      float* dst = p.o_part + (part + h) * kDecodeDv;
+      __half* dst = p.o_part + (part + h) * kDecodeDv;
       const float inv_l = 1.f / l;
 #pragma unroll 1
       for (int ch = 0; ch < kDecodeDv / 32; ++ch) {
@@ -278,10 +303,22 @@ __global__ void __launch_bounds__(192, 1)
         tmem_wait_ld();
         if (valid) {
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            reinterpret_cast<float4*>(dst + ch * 32)[v] = make_float4(
-                __uint_as_float(orr[4 * v]) * inv_l, __uint_as_float(orr[4 * v + 1]) * inv_l,
-                __uint_as_float(orr[4 * v + 2]) * inv_l, __uint_as_float(orr[4 * v + 3]) * inv_l);
+          for (int v = 0; v < 4; ++v) {
+            uint4 pk;
+            __half2 h0 = __floats2half2_rn(__uint_as_float(orr[8 * v + 0]) * inv_l,
+                                           __uint_as_float(orr[8 * v + 1]) * inv_l);
+            __half2 h1 = __floats2half2_rn(__uint_as_float(orr[8 * v + 2]) * inv_l,
+                                           __uint_as_float(orr[8 * v + 3]) * inv_l);
+            __half2 h2 = __floats2half2_rn(__uint_as_float(orr[8 * v + 4]) * inv_l,
+                                           __uint_as_float(orr[8 * v + 5]) * inv_l);
+            __half2 h3 = __floats2half2_rn(__uint_as_float(orr[8 * v + 6]) * inv_l,
+                                           __uint_as_float(orr[8 * v + 7]) * inv_l);
+            pk.x = *reinterpret_cast<uint32_t*>(&h0);
+            pk.y = *reinterpret_cast<uint32_t*>(&h1);
+            pk.z = *reinterpret_cast<uint32_t*>(&h2);
+            pk.w = *reinterpret_cast<uint32_t*>(&h3);
+            reinterpret_cast<uint4*>(dst + ch * 32)[v] = pk;
+          }
         }
       }
       if (valid) p.lse_part[part + h] = (m + __log2f(l)) * kLn2;
@@ -298,9 +335,11 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 // One CTA of 128 threads per (sequence, head): each thread merges 4 of the
-// 512 output columns over the splits.
+// 512 output columns over the splits.  Launched as a programmatic dependent of
+// the split kernel; it waits for the split kernel's results before reading.
 __global__ void __launch_bounds__(128)
     ssa_decode_merge_kernel(const DecodeParams p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int b = blockIdx.x / p.H_q, h = blockIdx.x % p.H_q;
   const int hg = h >> 7, hr = h & 127;
   const size_t base = (size_t)(b * p.HG + hg) * p.n_split;
@@ -314,12 +353,14 @@ __global__ void __launch_bounds__(128)
       if (ls == -INFINITY) continue;
       const float wgt = __expf(ls - lmax);
       denom += wgt;
-      const float4 v = reinterpret_cast<const float4*>(
+      const uint2 raw = reinterpret_cast<const uint2*>(
           p.o_part + ((base + s) * 128 + hr) * kDecodeDv)[threadIdx.x];
-      acc[0] += wgt * v.x;
-      acc[1] += wgt * v.y;
-      acc[2] += wgt * v.z;
-      acc[3] += wgt * v.w;
+      const float2 v01 = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+      const float2 v23 = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+      acc[0] += wgt * v01.x;
+      acc[1] += wgt * v01.y;
+      acc[2] += wgt * v23.x;
+      acc[3] += wgt * v23.y;
     }
   }
   const float inv = denom > 0.f ? 1.f / denom : 0.f;

@@ -18,7 +18,7 @@
 namespace {
 
 constexpr int kVersion = 10000;  // 1.0.0
-constexpr int kMaxVarlenSeqs = 4096;
+constexpr int kMaxVarlenSeqs = 4000;  // keeps the d_qk=192 layout within 227 KB
 constexpr int kMaxDecodeWindow = 4096;
 constexpr int kMaxDevices = 64;
 
@@ -115,7 +115,7 @@ int launch_prefill(const void* q, const void* k, const void* v, loza::PrefillPar
                                        (int)Lay::smem_bytes(kMaxVarlenSeqs + 1));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill)");
   const int grid = items_upper < dev.num_sms ? items_upper : dev.num_sms;
-  kern<<<grid, 192, smem, stream>>>(mq, mk, mv, prm);
+  kern<<<grid, loza::kPrefillThreads, smem, stream>>>(mq, mk, mv, prm);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "prefill launch");
   return LOZA_SSA_OK;
 }
@@ -265,7 +265,7 @@ size_t loza_ssa_decode_workspace_size(int B, int H_q, int d_v, int n_sink, int n
       n_sink + n_local > kMaxDecodeWindow)
     return 0;
   const size_t rows = decode_partial_floats(B, H_q, n_sink + n_local);
-  const size_t o_bytes = rows * loza::kDecodeDv * sizeof(float);
+  const size_t o_bytes = rows * loza::kDecodeDv * sizeof(__half);  // partial O is fp16
   const size_t lse_bytes = rows * sizeof(float);
   return ((o_bytes + 255) / 256) * 256 + ((lse_bytes + 255) / 256) * 256;
 }
@@ -299,9 +299,9 @@ int loza_ssa_decode(const void* q, const void* paged_kv, const int* page_table,
   loza::DecodeParams prm{};
   prm.page_table = page_table;
   prm.seq_lens = seq_lens;
-  prm.o_part = static_cast<float*>(workspace);
+  prm.o_part = static_cast<__half*>(workspace);
   prm.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                          ((rows * loza::kDecodeDv * sizeof(float) + 255) / 256) * 256);
+                                          ((rows * loza::kDecodeDv * sizeof(__half) + 255) / 256) * 256);
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.lse = lse;
   prm.B = B;
@@ -327,8 +327,20 @@ int loza_ssa_decode(const void* q, const void* paged_kv, const int* page_table,
   dim3 grid(n_split, HG, B);
   loza::ssa_decode_split_kernel<<<grid, 192, loza::DecodeLayout::SMEM_BYTES, s>>>(mq, mkv, prm);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "decode split launch");
-  loza::ssa_decode_merge_kernel<<<B * H_q, 128, 0, s>>>(prm);
-  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "decode merge launch");
+  // the merge is a programmatic dependent of the split kernel: it is scheduled
+  // as split CTAs retire and waits (griddepcontrol.wait) for their results
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(B * H_q);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if ((e = cudaLaunchKernelEx(&cfg, loza::ssa_decode_merge_kernel, prm)) != cudaSuccess)
+    return cuda_fail(e, "decode merge launch");
   return LOZA_SSA_OK;
 }
 

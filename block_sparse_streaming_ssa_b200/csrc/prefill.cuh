@@ -19,11 +19,17 @@
 // in TMEM by exp2(m_old - m_new) before the next P.V.  The final O = acc / l
 // and LSE = (m + log2 l) ln 2 are exact for any choice of m.
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax + correction + epilogue; thread r owns query row r
-//              (TMEM lane r; a warp may only touch its own 32-lane quarter)
-//   warp 4     TMA producer (one elected lane)
-//   warp 5     TMEM allocator + MMA issuer (one elected lane)
+// Warp roles (320 threads):
+//   warps 0-7  softmax + correction + epilogue.  Warp w reads TMEM lanes
+//              32*(w%4)..+31 (a warp may only touch its own lane quarter), so
+//              query row r is shared by thread r of warpgroup 0 (key columns
+//              0-63 of every tile, O columns [0, DV/2)) and thread r of
+//              warpgroup 1 (key columns 64-127, O columns [DV/2, DV)); the two
+//              halves exchange their row maxima through shared memory once per
+//              tile and their row sums once per item.  Two warps per SM
+//              sub-partition keep the exp2 / FMA pipes busy.
+//   warp 8     TMA producer (one elected lane)
+//   warp 9     TMEM allocator + MMA issuer (one elected lane)
 //
 // TMEM (512 columns x 128 lanes, fp32): S0 = cols [0,128), S1 = [128,256),
 // O = [256, 256+DV).  P_j (bf16 pairs) overwrites the first 64 columns of its
@@ -81,9 +87,12 @@ struct PrefillLayout {
   static constexpr int B_O_DONE = B_P_FULL + 2;
   static constexpr int B_O_EMPTY = B_O_DONE + 1;
   static constexpr int B_DRAIN = B_O_EMPTY + 1;
-  static constexpr int NBAR = B_DRAIN + 1;
-  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // [0] tmem base, [1] abort, [2] items
-  static constexpr int OFF_PREFIX = OFF_MISC + 16;
+  static constexpr int B_XCHG = B_DRAIN + 1;  // the two softmax warpgroups' row exchange
+  static constexpr int NBAR = B_XCHG + 1;
+  static constexpr int OFF_MISC = OFF_BAR + 256;      // [0] tmem base, [1] abort, [2] items
+  static constexpr int OFF_RED = OFF_MISC + 16;       // float [2 buffers][2 halves][128 rows]
+  static constexpr int OFF_PREFIX = OFF_RED + 2 * 2 * 128 * 4;
+  static_assert(NBAR * 8 <= 256, "barrier area");
   static constexpr int TMEM_COLS = 512;
   static constexpr int TM_O = 256;
   static constexpr int MIN_SMEM = 120 * 1024;  // keeps one CTA (and one TMEM owner) per SM
@@ -165,8 +174,11 @@ __device__ __forceinline__ void prefill_count_items(const PrefillParams& p, int*
   }
 }
 
+constexpr int kPrefillThreads = 320;
+constexpr int kSoftmaxThreads = 256;
+
 template <int DQK, int DV>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kPrefillThreads, 1)
     ssa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
@@ -193,21 +205,22 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(Lay::B_S_FULL + s), 1);
-      mbar_init(bar(Lay::B_P_FULL + s), 128);
+      mbar_init(bar(Lay::B_P_FULL + s), kSoftmaxThreads);
     }
     mbar_init(bar(Lay::B_O_DONE), 1);
-    mbar_init(bar(Lay::B_O_EMPTY), 128);
+    mbar_init(bar(Lay::B_O_EMPTY), kSoftmaxThreads);
     mbar_init(bar(Lay::B_DRAIN), 1);
+    mbar_init(bar(Lay::B_XCHG), kSoftmaxThreads);
     misc[1] = 0;
     fence_barrier_init();
   }
   if (warp == 0) prefill_count_items(p, prefix, misc, lane);
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(sb + Lay::OFF_MISC, Lay::TMEM_COLS);
     tmem_relinquish();
   }
@@ -217,7 +230,7 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = misc[0];
   const int total_items = (int)misc[2];
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int g = 0, it = 0;
@@ -272,7 +285,7 @@ __global__ void __launch_bounds__(192, 1)
         if (it > 0) mbar_wait_drain(bar(Lay::B_Q_FULL), (it - 1) & 1);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------- MMA
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16_f32(128, 128, false);
@@ -343,14 +356,30 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // -------------------------------------------- softmax / correction / epilogue
-    const int row = threadIdx.x;                              // 0..127
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;   // this warp's TMEM lanes
+    const int wg = warp >> 2;                                     // column half
+    const int row = threadIdx.x & 127;                            // query row = TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16; // this warp's lane quarter
+    const int col0 = wg * 64;                                     // first key column of the half
+    constexpr int OH = DV / 2;                                    // O columns per half
+    const uint32_t o_tmem = tmem + lane_base + Lay::TM_O + wg * OH;
+    float* red = reinterpret_cast<float*>(smem + Lay::OFF_RED);
     const float sl2 = p.scale_log2;
     int g0 = 0;
+    uint32_t xc = 0;  // exchanges done (selects the red buffer and the barrier phase)
+    // Publish v for this row, wait for the other half's value for the same row.
+    auto exchange = [&](float v, float& other) -> bool {
+      float* buf = red + (xc & 1) * 256;
+      buf[wg * 128 + row] = v;
+      mbar_arrive(bar(Lay::B_XCHG));
+      const bool okx = mbar_wait(bar(Lay::B_XCHG), xc & 1, abort_flag, status, 1);
+      other = buf[(wg ^ 1) * 128 + row];
+      ++xc;
+      return okx;
+    };
     for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
       const WorkItem w = decode_item(item, p, prefix);
       const TileRange tr = tile_range(w.qb, p.n_sink, p.n_local);
-      float m = -INFINITY, l = 0.f;
+      float m = -INFINITY, l = 0.f;  // l: this half's share of the row sum
       bool ok = true;
       for (int t = 0; t < tr.count; ++t) {
         const int g = g0 + t;
@@ -360,44 +389,65 @@ __global__ void __launch_bounds__(192, 1)
           break;
         }
         tc_fence_after();
-        uint32_t sr[4][32];
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) tmem_ld32(s_tmem + ch * 32, sr[ch]);
+        uint32_t sr[2][32];
+        tmem_ld32(s_tmem + col0, sr[0]);
+        tmem_ld32(s_tmem + col0 + 32, sr[1]);
         tmem_wait_ld();
         if (t == tr.count - 1) {
           // diagonal block: key c of the tile is visible to row r iff c <= r
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch)
+          for (int ch = 0; ch < 2; ++ch)
 #pragma unroll
             for (int c = 0; c < 32; ++c)
-              if (ch * 32 + c > row) sr[ch][c] = __float_as_uint(-INFINITY);
+              if (col0 + ch * 32 + c > row) sr[ch][c] = __float_as_uint(-INFINITY);
         }
-        float mx = -INFINITY;
+        // this half's row max: four independent 3-input max chains
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch)
+        for (int c = 0; c < 64; c += 8)
 #pragma unroll
-          for (int c = 0; c < 32; ++c) mx = fmaxf(mx, __uint_as_float(sr[ch][c]));
+          for (int a = 0; a < 4; ++a)
+            mx4[a] = fmax3(mx4[a], __uint_as_float(sr[(c + 2 * a) >> 5][(c + 2 * a) & 31]),
+                           __uint_as_float(sr[(c + 2 * a + 1) >> 5][(c + 2 * a + 1) & 31]));
+        float mx = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+        float mx_other;
+        if (!exchange(mx, mx_other)) {
+          ok = false;
+          break;
+        }
+        mx = fmaxf(mx, mx_other);
         const float m_tile = mx * sl2;
         const bool first = (t == 0);
         const float m_new = fmaxf(m, m_tile);
+        // both halves see the same row maxima, so they take the same decision
         const bool need = !first && (m_new > m + kRescaleThreshold);
         const bool rescale = __any_sync(0xffffffffu, need);
         const float m_use = (first || rescale) ? m_new : m;
-        float rsum = 0.f;
+        // p = exp2(s*scale*log2e - m): packed FMA for the affine part, four
+        // independent packed row-sum accumulators
+        const uint64_t sl2x2 = f2_pack(sl2, sl2);
+        const uint64_t negm2 = f2_pack(-m_use, -m_use);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+        uint32_t pk[32];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int col = half * 64 + 2 * c;
-            const float x0 = __uint_as_float(sr[col >> 5][col & 31]);
-            const float x1 = __uint_as_float(sr[(col + 1) >> 5][(col + 1) & 31]);
-            const float p0 = ex2_approx(fmaf(x0, sl2, -m_use));
-            const float p1 = ex2_approx(fmaf(x1, sl2, -m_use));
-            rsum += p0 + p1;
-            pk[c] = pack_bf16x2(p0, p1);
-          }
-          tmem_st32(s_tmem + half * 32, pk);
+        for (int c = 0; c < 32; ++c) {
+          const uint64_t xx = f2_pack(__uint_as_float(sr[c >> 4][(2 * c) & 31]),
+                                      __uint_as_float(sr[c >> 4][(2 * c + 1) & 31]));
+          float y0, y1;
+          f2_unpack(f2_fma(xx, sl2x2, negm2), y0, y1);
+          const float p0 = ex2_approx(y0);
+          const float p1 = ex2_approx(y1);
+          acc[c & 3] = f2_add(acc[c & 3], f2_pack(p0, p1));
+          pk[c] = pack_bf16x2(p0, p1);
+        }
+        // P (bf16 pairs) over the first 64 columns of the S buffer: keys 2c, 2c+1
+        // of this half land in column col0/2 + c
+        tmem_st32(s_tmem + col0 / 2, pk);
+        float rsum;
+        {
+          float a0, a1;
+          f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
+          rsum = a0 + a1;
         }
         if (!first) {
           // O must hold P_{g-1} V_{g-1} before it is rescaled or read again
@@ -409,9 +459,8 @@ __global__ void __launch_bounds__(192, 1)
             tc_fence_after();
             const float alpha = ex2_approx(m - m_use);
             l *= alpha;
-            const uint32_t o_tmem = tmem + lane_base + Lay::TM_O;
 #pragma unroll 1
-            for (int ch = 0; ch < DV / 32; ++ch) {
+            for (int ch = 0; ch < OH / 32; ++ch) {
               uint32_t orr[32];
               tmem_ld32(o_tmem + ch * 32, orr);
               tmem_wait_ld();
@@ -430,21 +479,23 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (!ok) break;
       // epilogue: O = acc / l (bf16), LSE = (m + log2 l) ln 2
+      float l_other;
+      if (!exchange(l, l_other)) break;
+      const float l_row = l + l_other;
       const int gl = g0 + tr.count - 1;
       if (!mbar_wait(bar(Lay::B_O_DONE), gl & 1, abort_flag, status, 1)) break;
       tc_fence_after();
       const int r_in_seq = w.qb * 128 + row;
       const bool valid = r_in_seq < w.len;
       const size_t orow = (size_t)w.z * (size_t)p.plane_rows + (size_t)(w.seq_start + r_in_seq);
-      const float inv_l = 1.f / l;
-      const uint32_t o_tmem = tmem + lane_base + Lay::TM_O;
+      const float inv_l = 1.f / l_row;
 #pragma unroll 1
-      for (int ch = 0; ch < DV / 32; ++ch) {
+      for (int ch = 0; ch < OH / 32; ++ch) {
         uint32_t orr[32];
         tmem_ld32(o_tmem + ch * 32, orr);
         tmem_wait_ld();
         if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(p.o + orow * DV + ch * 32);
+          uint4* dst = reinterpret_cast<uint4*>(p.o + orow * DV + wg * OH + ch * 32);
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             uint4 pkt;
@@ -462,7 +513,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       tc_fence_before();
       mbar_arrive(bar(Lay::B_O_EMPTY));
-      if (valid) p.lse[orow] = (m + __log2f(l)) * kLn2;
+      if (valid && wg == 0) p.lse[orow] = (m + __log2f(l_row)) * kLn2;
       g0 += tr.count;
     }
   }
@@ -470,7 +521,7 @@ __global__ void __launch_bounds__(192, 1)
   __syncwarp();
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, Lay::TMEM_COLS);
   }

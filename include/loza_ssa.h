@@ -86,7 +86,7 @@ int loza_ssa_prefill(const void* q, const void* k, const void* v, void* o, float
  * each sequence's own first token, and no key crosses a sequence boundary.
  *   q, k : bf16 [H, total_tokens, d_qk]   v, o : bf16 [H, total_tokens, d_v]
  *   lse  : fp32 [H, total_tokens]         cu_seqlens : DEVICE int32 [n_seqs + 1]
- *   1 <= n_seqs <= 4096.  max_seqlen is the caller's bound on any sequence
+ *   1 <= n_seqs <= 4000.  max_seqlen is the caller's bound on any sequence
  *   length (used to size the launch; a longer sequence is still computed).
  * Other arguments as for loza_ssa_prefill.
  */
