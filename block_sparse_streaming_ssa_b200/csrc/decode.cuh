@@ -334,41 +334,52 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-// One CTA of 128 threads per (sequence, head): each thread merges 4 of the
-// 512 output columns over the splits.  Launched as a programmatic dependent of
-// the split kernel; it waits for the split kernel's results before reading.
-__global__ void __launch_bounds__(128)
+// One CTA of 64 threads per (sequence, head): each thread merges 8 of the 512
+// output columns (one 16-byte fp16 load per split).  Launched as a programmatic
+// dependent of the split kernel; it waits for the split kernel's results
+// before reading.  Splits whose LSE is -inf are empty and contribute nothing
+// (their partial O is never read into the sum).
+constexpr int kMergeThreads = kDecodeDv / 8;
+
+__global__ void __launch_bounds__(kMergeThreads)
     ssa_decode_merge_kernel(const DecodeParams p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int b = blockIdx.x / p.H_q, h = blockIdx.x % p.H_q;
   const int hg = h >> 7, hr = h & 127;
   const size_t base = (size_t)(b * p.HG + hg) * p.n_split;
+  const float* lsep = p.lse_part + base * 128 + hr;              // split stride 128
+  const uint4* op = reinterpret_cast<const uint4*>(p.o_part + (base * 128 + hr) * kDecodeDv) +
+                    threadIdx.x;                                // split stride 128*512/8
+  constexpr size_t kSplitStride = 128 * kDecodeDv / 8;
   float lmax = -INFINITY;
-  for (int s = 0; s < p.n_split; ++s) lmax = fmaxf(lmax, p.lse_part[(base + s) * 128 + hr]);
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+  for (int s = 0; s < p.n_split; ++s) lmax = fmaxf(lmax, __ldg(lsep + s * 128));
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   float denom = 0.f;
   if (lmax > -INFINITY) {
+#pragma unroll 8
     for (int s = 0; s < p.n_split; ++s) {
-      const float ls = p.lse_part[(base + s) * 128 + hr];
+      const float ls = __ldg(lsep + s * 128);
+      const uint4 raw = __ldg(op + s * kSplitStride);
       if (ls == -INFINITY) continue;
       const float wgt = __expf(ls - lmax);
       denom += wgt;
-      const uint2 raw = reinterpret_cast<const uint2*>(
-          p.o_part + ((base + s) * 128 + hr) * kDecodeDv)[threadIdx.x];
-      const float2 v01 = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-      const float2 v23 = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-      acc[0] += wgt * v01.x;
-      acc[1] += wgt * v01.y;
-      acc[2] += wgt * v23.x;
-      acc[3] += wgt * v23.y;
+      const __half2* hv = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(hv[e]);
+        acc[2 * e] += wgt * f.x;
+        acc[2 * e + 1] += wgt * f.y;
+      }
     }
   }
   const float inv = denom > 0.f ? 1.f / denom : 0.f;
-  __nv_bfloat16* dst = p.o + ((size_t)b * p.H_q + h) * kDecodeDv + threadIdx.x * 4;
-  uint2 pk;
+  uint4 pk;
   pk.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
   pk.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-  *reinterpret_cast<uint2*>(dst) = pk;
+  pk.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+  pk.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+  *(reinterpret_cast<uint4*>(p.o + ((size_t)b * p.H_q + h) * kDecodeDv) + threadIdx.x) = pk;
   if (threadIdx.x == 0)
     p.lse[(size_t)b * p.H_q + h] = denom > 0.f ? lmax + __logf(denom) : -INFINITY;
 }

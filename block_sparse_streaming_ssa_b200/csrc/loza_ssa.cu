@@ -13,6 +13,7 @@
 #include "../../include/loza_ssa.h"
 #include "decode.cuh"
 #include "prefill.cuh"
+#include "prefill_pair.cuh"
 #include "schedule.cuh"
 
 namespace {
@@ -99,36 +100,61 @@ int make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint6
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-template <int DQK, int DV>
+// PAIR: the two-query-block kernel (prefill_pair.cuh, d_qk <= 128); else the
+// one-block kernel (prefill.cuh).  Dense inputs get their exact work-item count
+// here; packed inputs count theirs on the device (items_upper bounds the grid).
+template <int DQK, int DV, bool PAIR>
 int launch_prefill(const void* q, const void* k, const void* v, loza::PrefillParams prm,
-                   uint64_t plane_rows, uint64_t planes, int items_upper, int n_prefix,
+                   uint64_t plane_rows, uint64_t planes, long long items_upper, int n_prefix,
                    cudaStream_t stream, const DeviceInfo& dev) {
-  using Lay = loza::PrefillLayout<DQK, DV>;
+  using Single = loza::PrefillLayout<DQK, DV>;
+  using Pair = loza::PairLayout<DQK, DV>;
   CUtensorMap mq, mk, mv;
   int rc;
   if ((rc = make_map(&mq, q, DQK, plane_rows, planes, 3)) != LOZA_SSA_OK) return rc;
   if ((rc = make_map(&mk, k, DQK, plane_rows, planes, 3)) != LOZA_SSA_OK) return rc;
   if ((rc = make_map(&mv, v, DV, plane_rows, planes, 3)) != LOZA_SSA_OK) return rc;
-  const size_t smem = Lay::smem_bytes(n_prefix);
-  auto kern = loza::ssa_prefill_kernel<DQK, DV>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)Lay::smem_bytes(kMaxVarlenSeqs + 1));
+  if (prm.cu_seqlens == nullptr) {
+    const long long nb = (prm.L + 127) / 128;
+    items_upper = (long long)planes * (PAIR ? (nb + 1) / 2 : nb);
+    prm.total_items = (int)items_upper;
+  }
+  size_t smem, smem_max;
+  int threads;
+  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, loza::PrefillParams);
+  if constexpr (PAIR) {
+    smem = Pair::smem_bytes(n_prefix);
+    smem_max = Pair::smem_bytes(kMaxVarlenSeqs + 1);
+    kern = loza::ssa_prefill_pair_kernel<DQK, DV>;
+    threads = loza::kPairThreads;
+  } else {
+    smem = Single::smem_bytes(n_prefix);
+    smem_max = Single::smem_bytes(kMaxVarlenSeqs + 1);
+    kern = loza::ssa_prefill_kernel<DQK, DV>;
+    threads = loza::kPrefillThreads;
+  }
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill)");
-  const int grid = items_upper < dev.num_sms ? items_upper : dev.num_sms;
-  kern<<<grid, loza::kPrefillThreads, smem, stream>>>(mq, mk, mv, prm);
+  const int grid = items_upper < dev.num_sms ? (int)items_upper : dev.num_sms;
+  if (grid < 1) return LOZA_SSA_OK;
+  kern<<<grid, threads, smem, stream>>>(mq, mk, mv, prm);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "prefill launch");
   return LOZA_SSA_OK;
 }
 
 int dispatch_prefill(int d_qk, int d_v, const void* q, const void* k, const void* v,
                      const loza::PrefillParams& prm, uint64_t plane_rows, uint64_t planes,
-                     int items_upper, int n_prefix, cudaStream_t s, const DeviceInfo& dev) {
+                     long long items_upper, int n_prefix, cudaStream_t s, const DeviceInfo& dev) {
   if (d_qk == 64 && d_v == 64)
-    return launch_prefill<64, 64>(q, k, v, prm, plane_rows, planes, items_upper, n_prefix, s, dev);
+    return launch_prefill<64, 64, true>(q, k, v, prm, plane_rows, planes, items_upper, n_prefix,
+                                        s, dev);
   if (d_qk == 128 && d_v == 128)
-    return launch_prefill<128, 128>(q, k, v, prm, plane_rows, planes, items_upper, n_prefix, s, dev);
+    return launch_prefill<128, 128, true>(q, k, v, prm, plane_rows, planes, items_upper,
+                                          n_prefix, s, dev);
   if (d_qk == 192 && d_v == 128)
-    return launch_prefill<192, 128>(q, k, v, prm, plane_rows, planes, items_upper, n_prefix, s, dev);
+    return launch_prefill<192, 128, false>(q, k, v, prm, plane_rows, planes, items_upper,
+                                           n_prefix, s, dev);
   return LOZA_SSA_ERR_HEAD_DIM;
 }
 
@@ -220,7 +246,7 @@ int loza_ssa_prefill(const void* q, const void* k, const void* v, void* o, float
   prm.n_local = n_local;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.total_items = (int)items;
-  return dispatch_prefill(d_qk, d_v, q, k, v, prm, (uint64_t)L, (uint64_t)B * H, (int)items, 0,
+  return dispatch_prefill(d_qk, d_v, q, k, v, prm, (uint64_t)L, (uint64_t)B * H, items, 0,
                           reinterpret_cast<cudaStream_t>(stream), dev);
 }
 
@@ -257,7 +283,7 @@ int loza_ssa_prefill_varlen(const void* q, const void* k, const void* v, void* o
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.total_items = 0;
   return dispatch_prefill(d_qk, d_v, q, k, v, prm, (uint64_t)total_tokens, (uint64_t)H,
-                          (int)upper, n_seqs + 1, reinterpret_cast<cudaStream_t>(stream), dev);
+                          upper, n_seqs + 1, reinterpret_cast<cudaStream_t>(stream), dev);
 }
 
 size_t loza_ssa_decode_workspace_size(int B, int H_q, int d_v, int n_sink, int n_local) {
@@ -331,7 +357,7 @@ int loza_ssa_decode(const void* q, const void* paged_kv, const int* page_table,
   // as split CTAs retire and waits (griddepcontrol.wait) for their results
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(B * H_q);
-  cfg.blockDim = dim3(128);
+  cfg.blockDim = dim3(loza::kMergeThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];

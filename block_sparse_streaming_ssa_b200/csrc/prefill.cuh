@@ -19,27 +19,30 @@
 // in TMEM by exp2(m_old - m_new) before the next P.V.  The final O = acc / l
 // and LSE = (m + log2 l) ln 2 are exact for any choice of m.
 //
-// Warp roles (320 threads):
+// Warp roles (352 threads):
 //   warps 0-7  softmax + correction + epilogue.  Warp w reads TMEM lanes
 //              32*(w%4)..+31 (a warp may only touch its own lane quarter), so
 //              query row r is shared by thread r of warpgroup 0 (key columns
 //              0-63 of every tile, O columns [0, DV/2)) and thread r of
 //              warpgroup 1 (key columns 64-127, O columns [DV/2, DV)); the two
 //              halves exchange their row maxima through shared memory once per
-//              tile and their row sums once per item.  Two warps per SM
-//              sub-partition keep the exp2 / FMA pipes busy.
-//   warp 8     TMA producer (one elected lane)
+//              tile and their row sums once per item.
+//   warp 8     TMA producer of Q and K (one elected lane)
 //   warp 9     TMEM allocator + MMA issuer (one elected lane)
+//   warp 10    TMA producer of V (one elected lane)
+// K and V have their own producers so a K load never queues behind a V load
+// that is waiting for its ring slot: the MMA consumes K_{j+1} before V_j.
 //
 // TMEM (512 columns x 128 lanes, fp32): S0 = cols [0,128), S1 = [128,256),
-// O = [256, 256+DV).  P_j (bf16 pairs) overwrites the first 64 columns of its
-// S buffer.  S is double-buffered so the tensor core computes S_{j+1} while
-// the softmax warps work on S_j.
+// O buffers from 256 (two of them when 2*DV <= 256, so the next item's first
+// P.V never waits for this item's epilogue).  P_j (bf16 pairs) overwrites the
+// first 64 columns of its S buffer.  S is double-buffered so the tensor core
+// computes S_{j+1} while the softmax warps work on S_j.
 //
 // Shared memory (1024-byte aligned, 128B-swizzled TMA boxes of 64 bf16
-// columns x 128 rows = 16 KB "chunks"):  Q [DQK/64 chunks], K ring
-// [2 stages], V ring [2 stages], mbarriers, and for packed varlen input the
-// per-sequence work-item prefix.
+// columns x 128 rows = 16 KB "chunks"):  Q ring, K ring, V ring, mbarriers,
+// the softmax exchange buffer and, for packed varlen input, the per-sequence
+// work-item prefix.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -50,6 +53,15 @@
 namespace loza {
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P values stay <= 2^8
+
+// Of every 8 exp2 pairs a softmax thread evaluates, this many run as a
+// polynomial on the FMA pipe (exp2_poly_x2) and the rest on the MUFU unit.
+// Measured on B200 the MUFU unit is not the limit of this kernel, so the
+// default keeps every exp2 on MUFU.
+#ifndef LOZA_POLY_PAIRS
+#define LOZA_POLY_PAIRS 0
+#endif
+constexpr int kPolyPairsPer8 = LOZA_POLY_PAIRS;
 
 struct PrefillParams {
   __nv_bfloat16* o;
@@ -73,20 +85,23 @@ struct PrefillLayout {
   static constexpr int Q_BYTES = KCH * CHUNK;
   static constexpr int K_BYTES = KCH * CHUNK;
   static constexpr int V_BYTES = VCH * CHUNK;
-  static constexpr int KST = 2;  // K/V ring depth
+  static constexpr int QST = DQK <= 128 ? 2 : 1;  // Q ring depth (d_qk=192: no room for 2)
+  static constexpr int KST = 2;                   // K ring depth
+  static constexpr int VST = 2;                   // V ring depth
+  static constexpr int NOB = 256 + 2 * DV <= 512 ? 2 : 1;  // O buffers in TMEM
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_K = OFF_Q + QST * Q_BYTES;
   static constexpr int OFF_V = OFF_K + KST * K_BYTES;
-  static constexpr int OFF_BAR = OFF_V + KST * V_BYTES;
+  static constexpr int OFF_BAR = OFF_V + VST * V_BYTES;
   // barrier indices
-  static constexpr int B_Q_FULL = 0, B_Q_EMPTY = 1;
-  static constexpr int B_K_FULL = 2, B_K_EMPTY = B_K_FULL + KST;
-  static constexpr int B_V_FULL = B_K_EMPTY + KST, B_V_EMPTY = B_V_FULL + KST;
-  static constexpr int B_S_FULL = B_V_EMPTY + KST;  // 2
+  static constexpr int B_Q_FULL = 0, B_Q_EMPTY = B_Q_FULL + QST;
+  static constexpr int B_K_FULL = B_Q_EMPTY + QST, B_K_EMPTY = B_K_FULL + KST;
+  static constexpr int B_V_FULL = B_K_EMPTY + KST, B_V_EMPTY = B_V_FULL + VST;
+  static constexpr int B_S_FULL = B_V_EMPTY + VST;  // 2
   static constexpr int B_P_FULL = B_S_FULL + 2;     // 2
   static constexpr int B_O_DONE = B_P_FULL + 2;
-  static constexpr int B_O_EMPTY = B_O_DONE + 1;
-  static constexpr int B_DRAIN = B_O_EMPTY + 1;
+  static constexpr int B_O_EMPTY = B_O_DONE + 1;    // NOB
+  static constexpr int B_DRAIN = B_O_EMPTY + NOB;
   static constexpr int B_XCHG = B_DRAIN + 1;  // the two softmax warpgroups' row exchange
   static constexpr int NBAR = B_XCHG + 1;
   static constexpr int OFF_MISC = OFF_BAR + 256;      // [0] tmem base, [1] abort, [2] items
@@ -174,7 +189,7 @@ __device__ __forceinline__ void prefill_count_items(const PrefillParams& p, int*
   }
 }
 
-constexpr int kPrefillThreads = 320;
+constexpr int kPrefillThreads = 352;
 constexpr int kSoftmaxThreads = 256;
 
 template <int DQK, int DV>
@@ -195,11 +210,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   int* status = &g_loza_status;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(Lay::B_Q_FULL), 1);
-    mbar_init(bar(Lay::B_Q_EMPTY), 1);
+    for (int s = 0; s < Lay::QST; ++s) {
+      mbar_init(bar(Lay::B_Q_FULL + s), 1);
+      mbar_init(bar(Lay::B_Q_EMPTY + s), 1);
+    }
     for (int s = 0; s < Lay::KST; ++s) {
       mbar_init(bar(Lay::B_K_FULL + s), 1);
       mbar_init(bar(Lay::B_K_EMPTY + s), 1);
+    }
+    for (int s = 0; s < Lay::VST; ++s) {
       mbar_init(bar(Lay::B_V_FULL + s), 1);
       mbar_init(bar(Lay::B_V_EMPTY + s), 1);
     }
@@ -208,7 +227,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       mbar_init(bar(Lay::B_P_FULL + s), kSoftmaxThreads);
     }
     mbar_init(bar(Lay::B_O_DONE), 1);
-    mbar_init(bar(Lay::B_O_EMPTY), kSoftmaxThreads);
+    for (int s = 0; s < Lay::NOB; ++s) mbar_init(bar(Lay::B_O_EMPTY + s), kSoftmaxThreads);
     mbar_init(bar(Lay::B_DRAIN), 1);
     mbar_init(bar(Lay::B_XCHG), kSoftmaxThreads);
     misc[1] = 0;
@@ -218,8 +237,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   if (warp == 8 && lane == 0) {
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_k);
-    prefetch_tensormap(&tm_v);
   }
+  if (warp == 10 && lane == 0) prefetch_tensormap(&tm_v);
   if (warp == 9) {
     tmem_alloc(sb + Lay::OFF_MISC, Lay::TMEM_COLS);
     tmem_relinquish();
@@ -231,23 +250,35 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int total_items = (int)misc[2];
 
   if (warp == 8) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------- Q / K producer
     if (lane == 0) {
       int g = 0, it = 0;
-      int k_issued[Lay::KST] = {}, v_issued[Lay::KST] = {};
+      int q_issued[Lay::QST] = {}, k_issued[Lay::KST] = {};
       bool ok = true;
       for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++it) {
         const WorkItem w = decode_item(item, p, prefix);
         const TileRange tr = tile_range(w.qb, p.n_sink, p.n_local);
-        if (it > 0 && !mbar_wait(bar(Lay::B_Q_EMPTY), (it - 1) & 1, abort_flag, status, 1)) {
+        const int qs = it % Lay::QST;
+        if (it >= Lay::QST && !mbar_wait(bar(Lay::B_Q_EMPTY + qs), (it / Lay::QST - 1) & 1,
+                                         abort_flag, status, 1)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(bar(Lay::B_Q_FULL), Lay::Q_BYTES);
+        mbar_arrive_expect_tx(bar(Lay::B_Q_FULL + qs), Lay::Q_BYTES);
+        ++q_issued[qs];
 #pragma unroll
         for (int c = 0; c < Lay::KCH; ++c)
-          tma_load_3d(sb + Lay::OFF_Q + c * Lay::CHUNK, &tm_q, bar(Lay::B_Q_FULL), c * 64,
-                      w.seq_start + w.qb * 128, w.z);
+          tma_load_3d(sb + Lay::OFF_Q + qs * Lay::Q_BYTES + c * Lay::CHUNK, &tm_q,
+                      bar(Lay::B_Q_FULL + qs), c * 64, w.seq_start + w.qb * 128, w.z);
+        // the item after the ring's reach is first-touch HBM data: start
+        // pulling its Q into L2 now
+        const int ahead = item + Lay::QST * (int)gridDim.x;
+        if (ahead < total_items) {
+          const WorkItem wn = decode_item(ahead, p, prefix);
+#pragma unroll
+          for (int c = 0; c < Lay::KCH; ++c)
+            tma_prefetch_3d(&tm_q, c * 64, wn.seq_start + wn.qb * 128, wn.z);
+        }
         for (int t = 0; t < tr.count; ++t, ++g) {
           const int row = w.seq_start + tile_block(tr, t) * 128;
           const int st = g % Lay::KST, use = g / Lay::KST;
@@ -262,6 +293,29 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           for (int c = 0; c < Lay::KCH; ++c)
             tma_load_3d(sb + Lay::OFF_K + st * Lay::K_BYTES + c * Lay::CHUNK, &tm_k,
                         bar(Lay::B_K_FULL + st), c * 64, row, w.z);
+        }
+      }
+      if (!ok) {
+        // Let copies already in flight land before the CTA's smem goes away:
+        // a slot holds at most one unconsumed load, its newest phase.
+        for (int s = 0; s < Lay::KST; ++s)
+          if (k_issued[s] > 0) mbar_wait_drain(bar(Lay::B_K_FULL + s), (k_issued[s] - 1) & 1);
+        for (int s = 0; s < Lay::QST; ++s)
+          if (q_issued[s] > 0) mbar_wait_drain(bar(Lay::B_Q_FULL + s), (q_issued[s] - 1) & 1);
+      }
+    }
+  } else if (warp == 10) {
+    // ----------------------------------------------------------- V producer
+    if (lane == 0) {
+      int g = 0;
+      int v_issued[Lay::VST] = {};
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
+        const WorkItem w = decode_item(item, p, prefix);
+        const TileRange tr = tile_range(w.qb, p.n_sink, p.n_local);
+        for (int t = 0; t < tr.count; ++t, ++g) {
+          const int row = w.seq_start + tile_block(tr, t) * 128;
+          const int st = g % Lay::VST, use = g / Lay::VST;
           if (use > 0 &&
               !mbar_wait(bar(Lay::B_V_EMPTY + st), (use - 1) & 1, abort_flag, status, 1)) {
             ok = false;
@@ -275,15 +329,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         bar(Lay::B_V_FULL + st), c * 64, row, w.z);
         }
       }
-      if (!ok) {
-        // Let copies already in flight land before the CTA's smem goes away:
-        // a stage holds at most one unconsumed load, its newest phase.
-        for (int st = 0; st < Lay::KST; ++st) {
-          if (k_issued[st] > 0) mbar_wait_drain(bar(Lay::B_K_FULL + st), (k_issued[st] - 1) & 1);
-          if (v_issued[st] > 0) mbar_wait_drain(bar(Lay::B_V_FULL + st), (v_issued[st] - 1) & 1);
-        }
-        if (it > 0) mbar_wait_drain(bar(Lay::B_Q_FULL), (it - 1) & 1);
-      }
+      if (!ok)
+        for (int s = 0; s < Lay::VST; ++s)
+          if (v_issued[s] > 0) mbar_wait_drain(bar(Lay::B_V_FULL + s), (v_issued[s] - 1) & 1);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------- MMA
@@ -292,23 +340,24 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const uint32_t id_o = idesc_bf16_f32(128, DV, true);
       int g0 = 0, it = 0;
       bool ok = true;
-      // O += P_g V_g for tile t (global index g) of the current item
-      auto issue_pv = [&](int g, int t) -> bool {
-        const int st = g % Lay::KST;
+      // O_ob += P_g V_g for tile t (global index g) of the current item
+      auto issue_pv = [&](int g, int t, int ob) -> bool {
+        const int st = g % Lay::VST;
         if (!mbar_wait(bar(Lay::B_P_FULL + (g & 1)), (g >> 1) & 1, abort_flag, status, 1))
           return false;
-        if (!mbar_wait(bar(Lay::B_V_FULL + st), (g / Lay::KST) & 1, abort_flag, status, 1))
+        if (!mbar_wait(bar(Lay::B_V_FULL + st), (g / Lay::VST) & 1, abort_flag, status, 1))
           return false;
-        if (t == 0 && it > 0 &&
-            !mbar_wait(bar(Lay::B_O_EMPTY), (it - 1) & 1, abort_flag, status, 1))
+        if (t == 0 && it >= Lay::NOB &&
+            !mbar_wait(bar(Lay::B_O_EMPTY + ob), (it / Lay::NOB - 1) & 1, abort_flag, status, 1))
           return false;
         tc_fence_after();
         const uint32_t p_tmem = tmem + (uint32_t)((g & 1) * 128);
+        const uint32_t o_tmem = tmem + Lay::TM_O + ob * DV;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t bdesc = sdesc_sw128(
               sb + Lay::OFF_V + st * Lay::V_BYTES + kk * 2048, Lay::CHUNK, 1024);
-          mma_ts(tmem + Lay::TM_O, p_tmem + kk * 8, bdesc, id_o, (t > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(o_tmem, p_tmem + kk * 8, bdesc, id_o, (t > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(bar(Lay::B_O_DONE));
         mma_commit(bar(Lay::B_V_EMPTY + st));
@@ -317,7 +366,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++it) {
         const WorkItem w = decode_item(item, p, prefix);
         const TileRange tr = tile_range(w.qb, p.n_sink, p.n_local);
-        if (!mbar_wait(bar(Lay::B_Q_FULL), it & 1, abort_flag, status, 1)) {
+        const int qs = it % Lay::QST, ob = it % Lay::NOB;
+        const uint32_t q_base = sb + Lay::OFF_Q + qs * Lay::Q_BYTES;
+        if (!mbar_wait(bar(Lay::B_Q_FULL + qs), (it / Lay::QST) & 1, abort_flag, status, 1)) {
           ok = false;
           break;
         }
@@ -332,19 +383,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < DQK / 16; ++kk) {
             const uint32_t koff = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
-            const uint64_t adesc = sdesc_sw128(sb + Lay::OFF_Q + koff, 16, 1024);
+            const uint64_t adesc = sdesc_sw128(q_base + koff, 16, 1024);
             const uint64_t bdesc = sdesc_sw128(sb + Lay::OFF_K + st * Lay::K_BYTES + koff, 16, 1024);
             mma_ss(s_tmem, adesc, bdesc, id_s, kk > 0 ? 1u : 0u);
           }
           mma_commit(bar(Lay::B_S_FULL + (g & 1)));
           mma_commit(bar(Lay::B_K_EMPTY + st));
-          if (t == tr.count - 1) mma_commit(bar(Lay::B_Q_EMPTY));
-          if (t > 0 && !issue_pv(g - 1, t - 1)) {
+          if (t == tr.count - 1) mma_commit(bar(Lay::B_Q_EMPTY + qs));
+          if (t > 0 && !issue_pv(g - 1, t - 1, ob)) {
             ok = false;
             break;
           }
         }
-        if (!ok || !issue_pv(g0 + tr.count - 1, tr.count - 1)) {
+        if (!ok || !issue_pv(g0 + tr.count - 1, tr.count - 1, ob)) {
           ok = false;
           break;
         }
@@ -361,10 +412,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16; // this warp's lane quarter
     const int col0 = wg * 64;                                     // first key column of the half
     constexpr int OH = DV / 2;                                    // O columns per half
-    const uint32_t o_tmem = tmem + lane_base + Lay::TM_O + wg * OH;
     float* red = reinterpret_cast<float*>(smem + Lay::OFF_RED);
     const float sl2 = p.scale_log2;
-    int g0 = 0;
+    int g0 = 0, it = 0;
     uint32_t xc = 0;  // exchanges done (selects the red buffer and the barrier phase)
     // Publish v for this row, wait for the other half's value for the same row.
     auto exchange = [&](float v, float& other) -> bool {
@@ -376,9 +426,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       ++xc;
       return okx;
     };
-    for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
+    for (int item = blockIdx.x; item < total_items; item += gridDim.x, ++it) {
       const WorkItem w = decode_item(item, p, prefix);
       const TileRange tr = tile_range(w.qb, p.n_sink, p.n_local);
+      const int ob = it % Lay::NOB;
+      const uint32_t o_tmem = tmem + lane_base + Lay::TM_O + ob * DV + wg * OH;
       float m = -INFINITY, l = 0.f;  // l: this half's share of the row sum
       bool ok = true;
       for (int t = 0; t < tr.count; ++t) {
@@ -433,10 +485,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         for (int c = 0; c < 32; ++c) {
           const uint64_t xx = f2_pack(__uint_as_float(sr[c >> 4][(2 * c) & 31]),
                                       __uint_as_float(sr[c >> 4][(2 * c + 1) & 31]));
-          float y0, y1;
+          float y0, y1, p0, p1;
           f2_unpack(f2_fma(xx, sl2x2, negm2), y0, y1);
-          const float p0 = ex2_approx(y0);
-          const float p1 = ex2_approx(y1);
+          if ((c & 7) < kPolyPairsPer8) {
+            exp2_poly_x2(y0, y1, p0, p1);
+          } else {
+            p0 = ex2_approx(y0);
+            p1 = ex2_approx(y1);
+          }
           acc[c & 3] = f2_add(acc[c & 3], f2_pack(p0, p1));
           pk[c] = pack_bf16x2(p0, p1);
         }
@@ -489,31 +545,29 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const bool valid = r_in_seq < w.len;
       const size_t orow = (size_t)w.z * (size_t)p.plane_rows + (size_t)(w.seq_start + r_in_seq);
       const float inv_l = 1.f / l_row;
-#pragma unroll 1
-      for (int ch = 0; ch < OH / 32; ++ch) {
-        uint32_t orr[32];
-        tmem_ld32(o_tmem + ch * 32, orr);
-        tmem_wait_ld();
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(p.o + orow * DV + wg * OH + ch * 32);
+      uint32_t orr[OH / 32][32];
+#pragma unroll
+      for (int ch = 0; ch < OH / 32; ++ch) tmem_ld32(o_tmem + ch * 32, orr[ch]);
+      tmem_wait_ld();
+      // O buffer free for the item NOB after this one
+      tc_fence_before();
+      mbar_arrive(bar(Lay::B_O_EMPTY + ob));
+      if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(p.o + orow * DV + wg * OH);
+#pragma unroll
+        for (int ch = 0; ch < OH / 32; ++ch)
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
+            const uint32_t* r8 = &orr[ch][8 * v];
             uint4 pkt;
-            pkt.x = pack_bf16x2(__uint_as_float(orr[8 * v + 0]) * inv_l,
-                                __uint_as_float(orr[8 * v + 1]) * inv_l);
-            pkt.y = pack_bf16x2(__uint_as_float(orr[8 * v + 2]) * inv_l,
-                                __uint_as_float(orr[8 * v + 3]) * inv_l);
-            pkt.z = pack_bf16x2(__uint_as_float(orr[8 * v + 4]) * inv_l,
-                                __uint_as_float(orr[8 * v + 5]) * inv_l);
-            pkt.w = pack_bf16x2(__uint_as_float(orr[8 * v + 6]) * inv_l,
-                                __uint_as_float(orr[8 * v + 7]) * inv_l);
-            dst[v] = pkt;
+            pkt.x = pack_bf16x2(__uint_as_float(r8[0]) * inv_l, __uint_as_float(r8[1]) * inv_l);
+            pkt.y = pack_bf16x2(__uint_as_float(r8[2]) * inv_l, __uint_as_float(r8[3]) * inv_l);
+            pkt.z = pack_bf16x2(__uint_as_float(r8[4]) * inv_l, __uint_as_float(r8[5]) * inv_l);
+            pkt.w = pack_bf16x2(__uint_as_float(r8[6]) * inv_l, __uint_as_float(r8[7]) * inv_l);
+            dst[ch * 4 + v] = pkt;
           }
-        }
+        if (wg == 0) p.lse[orow] = (m + __log2f(l_row)) * kLn2;
       }
-      tc_fence_before();
-      mbar_arrive(bar(Lay::B_O_EMPTY));
-      if (valid && wg == 0) p.lse[orow] = (m + __log2f(l_row)) * kLn2;
       g0 += tr.count;
     }
   }

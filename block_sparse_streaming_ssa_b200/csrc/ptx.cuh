@@ -95,6 +95,16 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   return true;
 }
 
+// Teardown of a TMA ring after `issued` loads into `stages` slots (load i went
+// to slot i % stages): wait for each slot's newest load to land.
+__device__ __forceinline__ void drain_ring(uint32_t full_bar0, int stages, int issued) {
+  for (int s = 0; s < stages; ++s) {
+    if (issued <= s) continue;
+    const int last = issued - 1 - ((issued - 1 - s) % stages);
+    mbar_wait_drain(full_bar0 + 8 * s, (last / stages) & 1);
+  }
+}
+
 // ---------------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
@@ -117,6 +127,14 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
+}
+
+// Warm L2 with a tile that a later tma_load_3d will read (no smem, no barrier).
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
 }
 
 // Generic-proxy shared-memory writes -> visible to the async proxy (tensor core).
@@ -223,6 +241,17 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
+// registers -> TMEM: 32 lanes x 32 bit, 16 consecutive columns per thread.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -262,6 +291,36 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("add.rn.ftz.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
+}
+
+// 2^y for two lanes on the FMA pipe instead of the MUFU unit.
+// Cody–Waite range reduction 2^y = 2^j * 2^f with j = rint(y), f = y - j in
+// [-1/2, 1/2]; 2^f by a degree-3 polynomial whose coefficients minimise the
+// maximum relative error on that interval (fitted by fit_exp2_poly.py: 7.5e-5,
+// far below the bf16 rounding of P); 2^j added straight into the exponent field.
+// y is clamped to >= -125 so the exponent stays normal: such terms are
+// < 2^-125 of the row maximum's weight (masked -inf keys become 2^-125 instead of 0).
+__device__ __forceinline__ void exp2_poly_x2(float y0, float y1, float& p0, float& p1) {
+  const uint64_t magic = f2_pack(12582912.f, 12582912.f);     // 1.5 * 2^23
+  const uint64_t neg_magic = f2_pack(-12582912.f, -12582912.f);
+  const uint64_t neg_one = f2_pack(-1.f, -1.f);
+  const uint64_t c0 = f2_pack(9.999280572e-01f, 9.999280572e-01f);
+  const uint64_t c1 = f2_pack(6.932608485e-01f, 6.932608485e-01f);
+  const uint64_t c2 = f2_pack(2.426111549e-01f, 2.426111549e-01f);
+  const uint64_t c3 = f2_pack(5.517221987e-02f, 5.517221987e-02f);
+  const uint64_t yy = f2_pack(fmaxf(y0, -125.f), fmaxf(y1, -125.f));
+  const uint64_t t = f2_add(yy, magic);               // rint(y) sits in the low mantissa bits
+  const uint64_t j = f2_add(t, neg_magic);            // rint(y) as a float (exact)
+  const uint64_t f = f2_fma(j, neg_one, yy);          // y - rint(y), exact
+  uint64_t p = f2_fma(f, c3, c2);
+  p = f2_fma(p, f, c1);
+  p = f2_fma(p, f, c0);
+  float pf0, pf1, t0, t1;
+  f2_unpack(p, pf0, pf1);
+  f2_unpack(t, t0, t1);
+  // bits(t) << 23 == rint(y) << 23 (mod 2^32): the magic's own bits shift out
+  p0 = __uint_as_float(__float_as_uint(pf0) + (__float_as_uint(t0) << 23));
+  p1 = __uint_as_float(__float_as_uint(pf1) + (__float_as_uint(t1) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
