@@ -190,6 +190,35 @@ __global__ void debug_decode_pages_kernel(loza::DecodeParams p, int* pages, int*
   }
 }
 
+// Scratch for loza_ssa_decode_static_scratch: the decode workspace of up to
+// LOZA_SSA_STATIC_SCRATCH_SLOTS split slots (fp16 partial O, 256-byte aligned,
+// then fp32 partial LSE), resident on every device that loads the library.
+// In host code the name only stands for the array; the kernels get its device
+// address, looked up once per device.
+static __device__ __align__(256) unsigned char g_decode_scratch[LOZA_SSA_STATIC_SCRATCH_BYTES];
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_decode_scratch on the current device (looked up on the
+// first call for that device, with the device current).
+int static_scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) {
+    std::snprintf(g_last_error, sizeof g_last_error, "device ordinal %d unsupported", dev);
+    return LOZA_SSA_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
+    if (e != cudaSuccess || !ptr) return cuda_fail(e, "cudaGetSymbolAddress(decode scratch)");
+    g_scratch_ptr[dev] = ptr;
+  }
+  *out = g_scratch_ptr[dev];
+  return LOZA_SSA_OK;
+}
+
 size_t decode_partial_floats(int B, int H_q, int n_split) {
   const size_t hg = (size_t)(H_q + 127) / 128;
   return (size_t)B * hg * (size_t)n_split * 128;
@@ -214,6 +243,7 @@ const char* loza_ssa_status_string(int status) {
     case LOZA_SSA_ERR_ALIGN: return "pointer not aligned (bf16 tensors: 16 B, lse: 4 B, workspace: 256 B)";
     case LOZA_SSA_ERR_WORKSPACE: return "decode workspace missing or too small";
     case LOZA_SSA_ERR_CUDA: return "CUDA error (see loza_ssa_last_error_string)";
+    case LOZA_SSA_ERR_SCRATCH_LIMIT: return "decode needs more split slots than the built-in scratch holds";
     default: return "unknown status";
   }
 }
@@ -368,6 +398,40 @@ int loza_ssa_decode(const void* q, const void* paged_kv, const int* page_table,
   if ((e = cudaLaunchKernelEx(&cfg, loza::ssa_decode_merge_kernel, prm)) != cudaSuccess)
     return cuda_fail(e, "decode merge launch");
   return LOZA_SSA_OK;
+}
+
+int loza_ssa_decode_static_scratch(const void* q, const void* paged_kv, const int* page_table,
+                                   const int* seq_lens, void* o, float* lse, int B, int H_q,
+                                   int d_qk, int d_v, int page_size, int max_pages, int n_pages,
+                                   int n_sink, int n_local, float scale,
+                                   loza_ssa_stream_t stream) {
+  // Same checks and kernels as loza_ssa_decode; only the workspace differs.
+  if (B >= 1 && H_q >= 1 && n_sink >= 0 && n_local >= 1 &&
+      n_sink + n_local <= kMaxDecodeWindow) {
+    const long long slots = (long long)B * ((H_q + 127) / 128) * (n_sink + n_local);
+    if (slots > LOZA_SSA_STATIC_SCRATCH_SLOTS) {
+      std::snprintf(g_last_error, sizeof g_last_error,
+                    "decode_static_scratch: B * ceil(H_q/128) * (n_sink + n_local) = %lld split "
+                    "slots, the built-in scratch holds %d",
+                    slots, LOZA_SSA_STATIC_SCRATCH_SLOTS);
+      return LOZA_SSA_ERR_SCRATCH_LIMIT;
+    }
+  }
+  const size_t need = loza_ssa_decode_workspace_size(B, H_q, d_v, n_sink, n_local);
+  void* scratch = nullptr;
+  if (need > 0) {  // invalid arguments are left for loza_ssa_decode to report
+    if (need > sizeof(g_decode_scratch)) {
+      std::snprintf(g_last_error, sizeof g_last_error,
+                    "decode_static_scratch: needs %zu scratch bytes, the built-in scratch holds %zu",
+                    need, sizeof(g_decode_scratch));
+      return LOZA_SSA_ERR_SCRATCH_LIMIT;
+    }
+    const int rc = static_scratch_address(&scratch);
+    if (rc != LOZA_SSA_OK) return rc;
+  }
+  return loza_ssa_decode(q, paged_kv, page_table, seq_lens, o, lse, B, H_q, d_qk, d_v, page_size,
+                         max_pages, n_pages, n_sink, n_local, scale, scratch,
+                         scratch ? sizeof(g_decode_scratch) : 0, stream);
 }
 
 int loza_ssa_get_last_device_status(loza_ssa_stream_t stream) {

@@ -23,6 +23,8 @@ LOZA_SSA_DEV_WAIT_TIMEOUT = 1
 LOZA_SSA_DEV_BAD_PAGE = 2
 LOZA_SSA_DEV_BAD_SEQLEN = 4
 LOZA_SSA_DEV_BAD_CU_SEQLENS = 8
+LOZA_SSA_ERR_SCRATCH_LIMIT = -9
+LOZA_SSA_STATIC_SCRATCH_SLOTS = 128
 
 
 class LozaSsaError(RuntimeError):
@@ -63,6 +65,9 @@ def lib() -> ctypes.CDLL:
         L.loza_ssa_debug_decode_pages.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp, vp,
                                                   i32, vp]
         L.loza_ssa_debug_decode_pages.restype = i32
+        L.loza_ssa_decode_static_scratch.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
+                                                     i32, i32, i32, i32, i32, f32, vp]
+        L.loza_ssa_decode_static_scratch.restype = i32
         L.loza_ssa_version.argtypes = []
         L.loza_ssa_version.restype = i32
         _lib = L
@@ -184,6 +189,34 @@ def loza_ssa_decode(q, paged_kv, page_table, seq_lens, d_v=512, o=None, lse=None
         _ptr(q), _ptr(paged_kv), _ptr(page_table), _ptr(seq_lens), _ptr(o), _ptr(lse), B, H_q,
         d_qk, d_v, page_size, max_pages, n_pages, n_sink, n_local, float(scale), _ptr(workspace),
         workspace.numel(), _stream(stream)))
+    return o, lse
+
+
+def loza_ssa_decode_static_scratch(q, paged_kv, page_table, seq_lens, d_v=512, o=None, lse=None,
+                                   page_size=128, n_sink=1, n_local=7, scale=None, stream=None):
+    """loza_ssa_decode without a workspace: the library uses its built-in
+    scratch array instead, so nothing is allocated for the split partials (for
+    callers that cannot provide device memory when they launch).  Limited to
+    B * ceil(H_q/128) * (n_sink + n_local) <= LOZA_SSA_STATIC_SCRATCH_SLOTS;
+    calls whose kernels overlap on the GPU share that scratch and must not run
+    concurrently.  Returns (o bf16 [B,H_q,d_v], lse fp32 [B,H_q])."""
+    _need(q, torch.bfloat16, "q")
+    _need(paged_kv, torch.bfloat16, "paged_kv")
+    _need(page_table, torch.int32, "page_table")
+    _need(seq_lens, torch.int32, "seq_lens")
+    B, H_q, d_qk = q.shape
+    if o is None:
+        o = torch.empty((B, H_q, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H_q), dtype=torch.float32, device=q.device)
+    _need(o, torch.bfloat16, "o")
+    _need(lse, torch.float32, "lse")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d_qk)
+    _check(lib().loza_ssa_decode_static_scratch(
+        _ptr(q), _ptr(paged_kv), _ptr(page_table), _ptr(seq_lens), _ptr(o), _ptr(lse), B, H_q,
+        d_qk, d_v, page_size, page_table.shape[1], paged_kv.shape[0], n_sink, n_local,
+        float(scale), _stream(stream)))
     return o, lse
 
 

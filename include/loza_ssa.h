@@ -58,6 +58,7 @@ enum {
   LOZA_SSA_ERR_ALIGN = -6,          /* a pointer is not aligned as required                     */
   LOZA_SSA_ERR_WORKSPACE = -7,      /* workspace missing or smaller than the size query says    */
   LOZA_SSA_ERR_CUDA = -8,           /* a CUDA runtime call failed (see loza_ssa_last_error_string) */
+  LOZA_SSA_ERR_SCRATCH_LIMIT = -9,  /* the call needs more than the built-in decode scratch holds */
 };
 
 /* Bits of the device status word (loza_ssa_get_last_device_status). */
@@ -154,6 +155,41 @@ int loza_ssa_debug_enumerate_tiles(int n_qblocks, int n_sink, int n_local, int* 
 int loza_ssa_debug_decode_pages(const int* page_table, const int* seq_lens, int B, int max_pages,
                                 int n_pages, int page_size, int n_sink, int n_local, int* pages,
                                 int* counts, int max_tiles, loza_ssa_stream_t stream);
+
+/*
+ * Paged SSA decode that allocates nothing and takes no workspace.
+ *
+ * The pages have no counterpart for this entry point; it exists for callers
+ * that cannot hand the library device memory at the point of the call: a
+ * plugin's enqueue step inside a framework that owns every allocation, or
+ * latency-critical code that must not call cudaMalloc (which can synchronise
+ * the device and take milliseconds) just to obtain scratch space.
+ *
+ * Arguments, layouts and results are those of loza_ssa_decode without the
+ * workspace: the split partials live instead in one scratch array compiled
+ * into the library, LOZA_SSA_STATIC_SCRATCH_BYTES long, which every GPU that
+ * loads the library holds until the process exits.  It holds
+ * LOZA_SSA_STATIC_SCRATCH_SLOTS split slots; a call needs
+ * B * ceil(H_q/128) * (n_sink + n_local) of them (e.g. 16 sequences with the
+ * default 8-page window and up to 128 heads) and is rejected with
+ * LOZA_SSA_ERR_SCRATCH_LIMIT, before anything is launched, if it needs more.
+ *
+ * The first call on a device looks up that device's address of the array
+ * (with the device current); make that first call before any stream
+ * capture on the device.  All calls on a device share the one array: calls
+ * whose kernels overlap on the GPU (for example on two streams at once) race
+ * and corrupt each other's results, so order them on one stream.  The array
+ * keeps the last call's contents; nothing in it needs to start at zero,
+ * because every slot a call reads is first written by the same call.
+ * The library calls no allocation routine for this entry point.
+ */
+#define LOZA_SSA_STATIC_SCRATCH_SLOTS 128
+#define LOZA_SSA_STATIC_SCRATCH_BYTES (LOZA_SSA_STATIC_SCRATCH_SLOTS * 128 * (512 * 2 + 4))
+int loza_ssa_decode_static_scratch(const void* q, const void* paged_kv, const int* page_table,
+                                   const int* seq_lens, void* o, float* lse, int B, int H_q,
+                                   int d_qk, int d_v, int page_size, int max_pages, int n_pages,
+                                   int n_sink, int n_local, float scale,
+                                   loza_ssa_stream_t stream);
 
 /* Library version, major*10000 + minor*100 + patch. */
 int loza_ssa_version(void);
