@@ -15,7 +15,9 @@
 //           the first two (by then consumed) Q ring slots
 //   MMA     O[128 x 512] = P V, two N=256 halves, V = the page's first 8 boxes
 //           read as an MN-major operand (no transpose copy)
-//   out     normalised partial O (fp16) and its LSE (fp32) to the workspace
+//   out     normalised partial O (fp16), staged in the page buffer (free once
+//           P V is done) in the TMA layout and written with 8 bulk-tensor
+//           stores; its LSE (fp32) with plain stores
 // TMEM: S uses columns [0,128); O uses [0,512) once S has been read.
 //
 // Merge kernel (programmatic dependent launch after the split kernel):
@@ -32,6 +34,10 @@ namespace loza {
 
 constexpr int kDecodeDqk = 576;
 constexpr int kDecodeDv = 512;
+// Of every 8 exp2 pairs in the decode softmax, this many run as a polynomial on
+// the FMA pipe: with one softmax warp per SM sub-partition the 16 exp2/clock of
+// the MUFU unit bound this step (128 x 128 exponentials per page).
+constexpr int kDecodePolyPairsPer8 = 3;
 
 struct DecodeParams {
   const int* page_table;  // [B, max_pages]
@@ -41,6 +47,7 @@ struct DecodeParams {
   __nv_bfloat16* o;       // [B, H_q, 512]
   float* lse;             // [B, H_q]
   int B, H_q, HG, max_pages, n_pages, n_sink, n_local, n_split;
+  int wave;  // CTAs resident at once (one per SM): the CTA `wave` later runs on a freed SM
   float scale_log2;
 };
 
@@ -84,14 +91,16 @@ struct DecodeLayout {
   static constexpr int B_P_FULL = B_S_FULL + 1;
   static constexpr int B_O_FULL = B_P_FULL + 1;
   static constexpr int B_DRAIN = B_O_FULL + 1;
-  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int B_EPI = B_DRAIN + 1;  // staged partial O complete (128 arrivals)
+  static constexpr int NBAR = B_EPI + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
 };
 
 __global__ void __launch_bounds__(192, 1)
     ssa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_q,
-                            const __grid_constant__ CUtensorMap tm_kv, const DecodeParams p) {
+                            const __grid_constant__ CUtensorMap tm_kv,
+                            const __grid_constant__ CUtensorMap tm_part, const DecodeParams p) {
   using Lay = DecodeLayout;
   const int sp = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -136,12 +145,14 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(bar(Lay::B_P_FULL), 128);
     mbar_init(bar(Lay::B_O_FULL), 1);
     mbar_init(bar(Lay::B_DRAIN), 1);
+    mbar_init(bar(Lay::B_EPI), 128);
     misc[1] = 0;
     fence_barrier_init();
   }
   if (warp == 4 && lane == 0) {
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_kv);
+    prefetch_tensormap(&tm_part);
   }
   if (warp == 5) {
     tmem_alloc(sb + Lay::OFF_MISC, 512);
@@ -177,6 +188,24 @@ __global__ void __launch_bounds__(192, 1)
                     phys * 128);
       }
       for (int c = Lay::QST; ok && c < Lay::KV_CH; ++c) ok = load_q(c);
+      // The CTA one wave later starts only when an SM frees up: pull its page
+      // and query boxes into L2 now so that its loads hit L2 instead of paying
+      // a cold HBM (and page-table) latency after this wave.
+      const int lin = (b * p.HG + hg) * p.n_split + sp;
+      const int nxt = lin + p.wave;
+      if (ok && nxt < p.B * p.HG * p.n_split) {
+        const int sp2 = nxt % p.n_split, hg2 = (nxt / p.n_split) % p.HG, b2 = nxt / (p.n_split * p.HG);
+        DecodeWindow w2;
+        if (decode_window(p, b2, w2) && sp2 < w2.tr.count) {
+          const int phys2 = decode_page(p, b2, w2, sp2);
+          if (phys2 >= 0) {
+            for (int c = 0; c < Lay::KV_CH; ++c) {
+              tma_prefetch_2d(&tm_kv, c * 64, phys2 * 128);
+              tma_prefetch_3d(&tm_q, c * 64, hg2 * 128, b2);
+            }
+          }
+        }
+      }
       // every copy issued lands before the CTA exits (normally already consumed)
       for (int c = 0; c < Lay::KV_CH; ++c) mbar_wait_drain(bar(Lay::B_KV_FULL + c), 0);
       for (int st = 0; st < Lay::QST; ++st) {
@@ -269,10 +298,14 @@ __global__ void __launch_bounds__(192, 1)
             const int col = box * 64 + u * 8 + 2 * e;
             const uint64_t xx = f2_pack(__uint_as_float(sr[col >> 5][col & 31]),
                                         __uint_as_float(sr[(col + 1) >> 5][(col + 1) & 31]));
-            float y0, y1;
+            float y0, y1, p0, p1;
             f2_unpack(f2_fma(xx, sl2x2, negm2), y0, y1);
-            const float p0 = ex2_approx(y0);
-            const float p1 = ex2_approx(y1);
+            if (((u * 4 + e) & 7) < kDecodePolyPairsPer8) {
+              exp2_poly_x2(y0, y1, p0, p1);
+            } else {
+              p0 = ex2_approx(y0);
+              p1 = ex2_approx(y1);
+            }
             acc[e] = f2_add(acc[e], f2_pack(p0, p1));
             w4[e] = pack_bf16x2(p0, p1);
           }
@@ -294,32 +327,39 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       asm volatile("griddepcontrol.launch_dependents;");
       const bool valid = hg * 128 + h < p.H_q;
-      __half* dst = p.o_part + (part + h) * kDecodeDv;
       const float inv_l = 1.f / l;
+      // Stage row h of the partial O (fp16) in the page buffer, laid out as the
+      // 128B-swizzled [128 rows x 64 columns] boxes a TMA store reads:
+      // 16-byte unit u of box c, row h, sits at unit u ^ (h & 7).
+      uint8_t* srow = smem + Lay::OFF_KV + h * 128;
 #pragma unroll 1
-      for (int ch = 0; ch < kDecodeDv / 32; ++ch) {
-        uint32_t orr[32];
-        tmem_ld32(tmem + lane_base + ch * 32, orr);
+      for (int j = 0; j < kDecodeDv / 64; ++j) {
+        uint32_t orr[2][32];
+        tmem_ld32(tmem + lane_base + j * 64, orr[0]);
+        tmem_ld32(tmem + lane_base + j * 64 + 32, orr[1]);
         tmem_wait_ld();
-        if (valid) {
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 pk;
-            __half2 h0 = __floats2half2_rn(__uint_as_float(orr[8 * v + 0]) * inv_l,
-                                           __uint_as_float(orr[8 * v + 1]) * inv_l);
-            __half2 h1 = __floats2half2_rn(__uint_as_float(orr[8 * v + 2]) * inv_l,
-                                           __uint_as_float(orr[8 * v + 3]) * inv_l);
-            __half2 h2 = __floats2half2_rn(__uint_as_float(orr[8 * v + 4]) * inv_l,
-                                           __uint_as_float(orr[8 * v + 5]) * inv_l);
-            __half2 h3 = __floats2half2_rn(__uint_as_float(orr[8 * v + 6]) * inv_l,
-                                           __uint_as_float(orr[8 * v + 7]) * inv_l);
-            pk.x = *reinterpret_cast<uint32_t*>(&h0);
-            pk.y = *reinterpret_cast<uint32_t*>(&h1);
-            pk.z = *reinterpret_cast<uint32_t*>(&h2);
-            pk.w = *reinterpret_cast<uint32_t*>(&h3);
-            reinterpret_cast<uint4*>(dst + ch * 32)[v] = pk;
+        for (int u = 0; u < 8; ++u) {
+          const uint32_t* r8 = &orr[u >> 2][(u & 3) * 8];
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            __half2 hv = __floats2half2_rn(__uint_as_float(r8[2 * e]) * inv_l,
+                                           __uint_as_float(r8[2 * e + 1]) * inv_l);
+            w[e] = *reinterpret_cast<uint32_t*>(&hv);
           }
+          *reinterpret_cast<uint4*>(srow + j * Lay::CHUNK + ((u ^ (h & 7)) << 4)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
         }
+      }
+      fence_async_shared();
+      mbar_arrive(bar(Lay::B_EPI));
+      if (h == 0 && mbar_wait(bar(Lay::B_EPI), 0, abort_flag, status, 1)) {
+        // rows part..part+127 of the [rows x 512] fp16 workspace, 8 boxes
+#pragma unroll
+        for (int j = 0; j < kDecodeDv / 64; ++j)
+          tma_store_2d(&tm_part, sb + Lay::OFF_KV + j * Lay::CHUNK, j * 64, (int)part);
+        tma_store_commit_and_wait_read();  // smem is read before the CTA exits
       }
       if (valid) p.lse_part[part + h] = (m + __log2f(l)) * kLn2;
     } while (false);

@@ -81,13 +81,14 @@ int device_info(DeviceInfo& out) {
   return LOZA_SSA_OK;
 }
 
-// bf16 tensor map: dims {d0 (innermost), d1, d2}, box {64, 128, 1}, 128B swizzle.
-int make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, int rank) {
+// 16-bit tensor map: dims {d0 (innermost), d1, d2}, box {64, 128, 1}, 128B swizzle.
+int make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, int rank,
+             CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   cuuint64_t dims[3] = {d0, d1, d2};
   cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
   cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank,
+  CUresult r = g_encode(map, dtype, (cuuint32_t)rank,
                         const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -352,6 +353,7 @@ int loza_ssa_decode(const void* q, const void* paged_kv, const int* page_table,
   const int n_split = n_sink + n_local;
   const int HG = (H_q + 127) / 128;
   const size_t rows = decode_partial_floats(B, H_q, n_split);
+  if (rows >= (1ull << 31)) return LOZA_SSA_ERR_SHAPE;  // TMA row coordinates are 32-bit
   loza::DecodeParams prm{};
   prm.page_table = page_table;
   prm.seq_lens = seq_lens;
@@ -369,11 +371,15 @@ int loza_ssa_decode(const void* q, const void* paged_kv, const int* page_table,
   prm.n_local = n_local;
   prm.n_split = n_split;
   prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.wave = dev.num_sms;
 
-  CUtensorMap mq, mkv;
+  CUtensorMap mq, mkv, mpart;
   if ((rc = make_map(&mq, q, loza::kDecodeDqk, (uint64_t)H_q, (uint64_t)B, 3)) != LOZA_SSA_OK)
     return rc;
   if ((rc = make_map(&mkv, paged_kv, loza::kDecodeDqk, (uint64_t)n_pages * 128, 1, 2)) != LOZA_SSA_OK)
+    return rc;
+  if ((rc = make_map(&mpart, prm.o_part, loza::kDecodeDv, (uint64_t)rows, 1, 2,
+                     CU_TENSOR_MAP_DATA_TYPE_FLOAT16)) != LOZA_SSA_OK)
     return rc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaFuncSetAttribute(loza::ssa_decode_split_kernel,
@@ -381,7 +387,8 @@ int loza_ssa_decode(const void* q, const void* paged_kv, const int* page_table,
                                        loza::DecodeLayout::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
   dim3 grid(n_split, HG, B);
-  loza::ssa_decode_split_kernel<<<grid, 192, loza::DecodeLayout::SMEM_BYTES, s>>>(mq, mkv, prm);
+  loza::ssa_decode_split_kernel<<<grid, 192, loza::DecodeLayout::SMEM_BYTES, s>>>(mq, mkv, mpart,
+                                                                                  prm);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "decode split launch");
   // the merge is a programmatic dependent of the split kernel: it is scheduled
   // as split CTAs retire and waits (griddepcontrol.wait) for their results
