@@ -7,18 +7,27 @@
 // plus the n_local pages ending at t's page (QbitAI article on LongCat LoZA,
 // paragraph on the 1024-token sparse window), read through the page table.
 //
-// Split kernel: one CTA per (window page, head group, sequence).
-//   TMA     the 128-token page (9 swizzled boxes of 64 columns = 144 KB) into
-//           smem, Q of the head group streamed in 64-column boxes (4-deep ring)
-//   MMA     S[128 heads x 128 keys] = Q K^T   (K = 576: 9 boxes x 4 k-steps)
-//   softmax mask keys past t, row max, exp2, row sum; P (bf16) -> smem over
-//           the first two (by then consumed) Q ring slots
-//   MMA     O[128 x 512] = P V, two N=256 halves, V = the page's first 8 boxes
-//           read as an MN-major operand (no transpose copy)
-//   out     normalised partial O (fp16), staged in the page buffer (free once
-//           P V is done) in the TMA layout and written with 8 bulk-tensor
-//           stores; its LSE (fp32) with plain stores
-// TMEM: S uses columns [0,128); O uses [0,512) once S has been read.
+// Split kernel: one CTA (one per SM) per (pair of window pages, head group,
+// sequence).  The two pages A and B share the query, so S over both is one
+// 128 x 256 product and their softmax is joint (no rescaling).
+//   TMA     a 4-stage ring of 48 KB stages (Q box | K_A box | K_B box):
+//             9 S stages, K boxes in the order 8, 0, 1, .., 7 (576 columns)
+//           The last four S stages hold K boxes 4..7, which are also V columns
+//           256..511: they stay in the ring for O half 1.  V columns 0..255
+//           are read again (L2 hits): page A's boxes into the Q slots (free
+//           once S is done), page B's into the K_B slots (free once O half 1
+//           is done).
+//   MMA     S[128 heads x 256 keys] = Q [K_A; K_B]^T into TMEM columns
+//           [0,256) -- K_A and K_B boxes sit side by side, one N=256 operand
+//   softmax warpgroup 0 takes page A's 128 keys of every head row, warpgroup 1
+//           page B's; the row max and row sum are exchanged through shared
+//           memory; P (bf16 pairs) goes over the first half of each page's
+//           S columns (P_A in [0,64), P_B in [128,192)) with tcgen05.st
+//   MMA     O half = P [V_A; V_B][:, 256 columns] (A = P in TMEM, N = 256) into
+//           TMEM columns [256,512): half 1 first, then half 0
+//   out     each half, normalised, as fp16 to the workspace in the layout
+//           [CTA][64 groups of 8 columns][128 heads][8] (a warp's stores of
+//           a group are 512 contiguous bytes); the LSE as fp32
 //
 // Merge kernel (programmatic dependent launch after the split kernel):
 // LSE = logsumexp_s LSE_s, O = sum_s exp(LSE_s - LSE) O_s.
@@ -34,20 +43,21 @@ namespace loza {
 
 constexpr int kDecodeDqk = 576;
 constexpr int kDecodeDv = 512;
-// Of every 8 exp2 pairs in the decode softmax, this many run as a polynomial on
-// the FMA pipe: with one softmax warp per SM sub-partition the 16 exp2/clock of
-// the MUFU unit bound this step (128 x 128 exponentials per page).
+constexpr int kDecodePagesPerSplit = 2;
+// Of every 8 exp2 pairs in the decode softmax, this many run as a polynomial
+// on the FMA pipe instead of the MUFU unit.
 constexpr int kDecodePolyPairsPer8 = 3;
 
 struct DecodeParams {
   const int* page_table;  // [B, max_pages]
   const int* seq_lens;    // [B]
-  __half* o_part;         // [B, HG, n_split, 128, 512]
-  float* lse_part;        // [B, HG, n_split, 128]
+  __half* o_part;         // [B*HG*n_split CTAs][64 column groups][128 heads][8]
+  float* lse_part;        // [B*HG*n_split CTAs][128 heads]
   __nv_bfloat16* o;       // [B, H_q, 512]
   float* lse;             // [B, H_q]
-  int B, H_q, HG, max_pages, n_pages, n_sink, n_local, n_split;
-  int wave;  // CTAs resident at once (one per SM): the CTA `wave` later runs on a freed SM
+  int B, H_q, HG, max_pages, n_pages, n_sink, n_local;
+  int n_split;  // split CTAs per (sequence, head group): ceil(window pages / 2)
+  int wave;     // CTAs resident at once: the CTA `wave` later runs on a freed SM
   float scale_log2;
 };
 
@@ -76,86 +86,128 @@ __device__ __forceinline__ int decode_page(const DecodeParams& p, int b, const D
   return (phys >= 0 && phys < p.n_pages) ? phys : -1;
 }
 
+// Keys of window tile `i` at or before the query (1..128).
+__device__ __forceinline__ int decode_valid_keys(const DecodeWindow& w, int i) {
+  return min(128, w.t - tile_block(w.tr, i) * 128 + 1);
+}
+
 struct DecodeLayout {
-  static constexpr int CHUNK = 128 * 128;  // [128 rows x 64 bf16], 128B swizzle
-  static constexpr int KV_CH = kDecodeDqk / 64;  // 9
-  static constexpr int QST = 4;                  // Q ring depth
-  static constexpr int OFF_KV = 0;
-  static constexpr int OFF_Q = OFF_KV + KV_CH * CHUNK;
-  static constexpr int OFF_P = OFF_Q;  // P [128 x 128] bf16 (2 boxes) reuses Q slots 0-1
-  static constexpr int OFF_BAR = OFF_Q + QST * CHUNK;
-  static constexpr int B_KV_FULL = 0;                    // 9
-  static constexpr int B_Q_FULL = B_KV_FULL + KV_CH;     // QST
-  static constexpr int B_Q_EMPTY = B_Q_FULL + QST;       // QST
-  static constexpr int B_S_FULL = B_Q_EMPTY + QST;
-  static constexpr int B_P_FULL = B_S_FULL + 1;
-  static constexpr int B_O_FULL = B_P_FULL + 1;
-  static constexpr int B_DRAIN = B_O_FULL + 1;
-  static constexpr int B_EPI = B_DRAIN + 1;  // staged partial O complete (128 arrivals)
-  static constexpr int NBAR = B_EPI + 1;
+  static constexpr int CHUNK = 128 * 128;        // [128 rows x 64 bf16], 128B swizzle
+  static constexpr int KV_CH = kDecodeDqk / 64;  // 9 boxes per 576-wide row block
+  static constexpr int NST = 4;                  // ring stages
+  static constexpr int STAGE = 3 * CHUNK;        // slots: Q box | K_A box | K_B box
+  static constexpr int N_KEEP = 4;               // last S stages kept for P V (boxes 4..7)
+  static constexpr int OFF_RING = 0;
+  static constexpr int OFF_XCHG = NST * STAGE;  // float [2 warpgroups][128 rows] x (max, sum)
+  static constexpr int OFF_BAR = OFF_XCHG + 2 * 2 * 128 * 4;
+  static constexpr int B_FULL = 0;              // NST
+  static constexpr int B_EMPTY = B_FULL + NST;  // NST
+  static constexpr int B_VA_FULL = B_EMPTY + NST;  // V_A boxes 0..3 in the Q slots
+  static constexpr int B_VB_FULL = B_VA_FULL + 1;  // V_B boxes 0..3 in the K_B slots
+  static constexpr int B_S_FULL = B_VB_FULL + 1;
+  static constexpr int B_P_FULL = B_S_FULL + 1;   // 256 arrivals
+  static constexpr int B_XCHG = B_P_FULL + 1;     // 256 arrivals; phase 0 max, 1 sum
+  static constexpr int B_O_FULL = B_XCHG + 1;     // phase 0: O half 1, phase 1: O half 0
+  static constexpr int B_O_EMPTY = B_O_FULL + 1;  // 256 arrivals, one phase per half
+  static constexpr int B_DRAIN = B_O_EMPTY + 1;
+  static constexpr int NBAR = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int TMEM_COLS = 512;  // S [0,256) (P inside it), O half [256,512)
+  static constexpr int TM_O = 256;
 };
 
-__global__ void __launch_bounds__(192, 1)
+// S stage i (0..8) loads K box decode_s_box(i) -- the rope box first, then the
+// latent boxes in order -- into ring stage decode_s_stage(i), numbered so that
+// the last N_KEEP stages (boxes 4..7 = V columns 256..511) land in stages
+// 0..3 in order, one STAGE apart: an MN-major operand with a constant stride.
+__host__ __device__ constexpr int decode_s_box(int i) { return i == 0 ? 8 : i - 1; }
+__host__ __device__ constexpr int decode_s_stage(int i) { return (i + 3) & 3; }
+// How many earlier S stages used the same ring stage (the mbarrier phase).
+__host__ __device__ constexpr int decode_s_round(int i) {
+  return (i + 3) / 4 - (decode_s_stage(i) != 3 ? 1 : 0);
+}
+
+// Bit k set: key 32*ch + k of the page is at or before the query.
+__device__ __forceinline__ uint32_t decode_chunk_mask(int valid_keys, int ch) {
+  const int n = valid_keys - 32 * ch;
+  return n >= 32 ? 0xffffffffu : (n <= 0 ? 0u : (1u << n) - 1u);
+}
+
+__global__ void __launch_bounds__(320, 1)
     ssa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_q,
-                            const __grid_constant__ CUtensorMap tm_kv,
-                            const __grid_constant__ CUtensorMap tm_part, const DecodeParams p) {
+                            const __grid_constant__ CUtensorMap tm_kv, const DecodeParams p) {
   using Lay = DecodeLayout;
   const int sp = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const size_t part = ((size_t)(b * p.HG + hg) * p.n_split + sp) * 128;
+  const size_t cta = ((size_t)b * p.HG + hg) * p.n_split + sp;  // partial-result slot
 
-  // ---- which page this CTA reads (uniform across the CTA; exits before any barrier)
+  // The query boxes do not depend on the page table: start pulling them into
+  // L2 while the table is read.
+  if (threadIdx.x == 256)
+    for (int c = 0; c < kDecodeDqk / 64; ++c) tma_prefetch_3d(&tm_q, c * 64, hg * 128, b);
+
+  // ---- which pages this CTA reads (uniform across the CTA; exits before any barrier).
+  // A page whose table entry is bad is skipped (and flagged); if only one page
+  // is left it is page A.
   DecodeWindow win;
-  int phys = -1, valid_keys = 0;
+  int phys_a = -1, phys_b = -1, valid_a = 0, valid_b = 0;
   if (!decode_window(p, b, win)) {
     if (threadIdx.x == 0 && sp == 0 && hg == 0) atomicOr(&g_loza_status, 4);
-  } else if (sp < win.tr.count) {
-    phys = decode_page(p, b, win, sp);
-    if (phys < 0) {
-      if (threadIdx.x == 0) atomicOr(&g_loza_status, 2);
-    } else {
-      const int logical = tile_block(win.tr, sp);
-      valid_keys = min(128, win.t - logical * 128 + 1);
+  } else {
+    for (int i = kDecodePagesPerSplit * sp;
+         i < min(kDecodePagesPerSplit * (sp + 1), win.tr.count); ++i) {
+      const int ph = decode_page(p, b, win, i);
+      if (ph < 0) {
+        if (threadIdx.x == 0) atomicOr(&g_loza_status, 2);
+      } else if (phys_a < 0) {
+        phys_a = ph;
+        valid_a = decode_valid_keys(win, i);
+      } else {
+        phys_b = ph;
+        valid_b = decode_valid_keys(win, i);
+      }
     }
   }
-  if (phys < 0) {
-    if (threadIdx.x < 128) p.lse_part[part + threadIdx.x] = -INFINITY;  // empty split
+  if (phys_a < 0) {
+    if (threadIdx.x < 128) p.lse_part[cta * 128 + threadIdx.x] = -INFINITY;  // empty split
     asm volatile("griddepcontrol.launch_dependents;");
     return;
   }
+  const bool two = phys_b >= 0;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sb = smem_u32(smem);
+  const uint32_t ring = sb + Lay::OFF_RING;
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   auto bar = [&](int i) -> uint32_t { return sb + Lay::OFF_BAR + 8 * i; };
   int* status = &g_loza_status;
 
   if (threadIdx.x == 0) {
-    for (int c = 0; c < Lay::KV_CH; ++c) mbar_init(bar(Lay::B_KV_FULL + c), 1);
-    for (int s = 0; s < Lay::QST; ++s) {
-      mbar_init(bar(Lay::B_Q_FULL + s), 1);
-      mbar_init(bar(Lay::B_Q_EMPTY + s), 1);
+    for (int s = 0; s < Lay::NST; ++s) {
+      mbar_init(bar(Lay::B_FULL + s), 1);
+      mbar_init(bar(Lay::B_EMPTY + s), 1);
     }
+    mbar_init(bar(Lay::B_VA_FULL), 1);
+    mbar_init(bar(Lay::B_VB_FULL), 1);
     mbar_init(bar(Lay::B_S_FULL), 1);
-    mbar_init(bar(Lay::B_P_FULL), 128);
+    mbar_init(bar(Lay::B_P_FULL), 256);
+    mbar_init(bar(Lay::B_XCHG), 256);
     mbar_init(bar(Lay::B_O_FULL), 1);
+    mbar_init(bar(Lay::B_O_EMPTY), 256);
     mbar_init(bar(Lay::B_DRAIN), 1);
-    mbar_init(bar(Lay::B_EPI), 128);
     misc[1] = 0;
     fence_barrier_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_kv);
-    prefetch_tensormap(&tm_part);
   }
-  if (warp == 5) {
-    tmem_alloc(sb + Lay::OFF_MISC, 512);
+  if (warp == 9) {
+    tmem_alloc(sb + Lay::OFF_MISC, Lay::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -163,253 +215,324 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = misc[0];
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int q_issued = 0;
-      bool ok = true;
-      auto load_q = [&](int c) -> bool {
-        const int st = c % Lay::QST;
-        if (c >= Lay::QST &&
-            !mbar_wait(bar(Lay::B_Q_EMPTY + st), (c / Lay::QST - 1) & 1, abort_flag, status, 1))
-          return false;
-        mbar_arrive_expect_tx(bar(Lay::B_Q_FULL + st), Lay::CHUNK);
-        tma_load_3d(sb + Lay::OFF_Q + st * Lay::CHUNK, &tm_q, bar(Lay::B_Q_FULL + st), c * 64,
-                    hg * 128, b);
-        ++q_issued;
-        return true;
-      };
-      // interleave the first Q boxes with the page so the first MMAs can start
-      // early; then the rest of the page; then Q boxes as ring slots free up
-      for (int c = 0; c < Lay::KV_CH; ++c) {
-        if (c < Lay::QST) load_q(c);
-        mbar_arrive_expect_tx(bar(Lay::B_KV_FULL + c), Lay::CHUNK);
-        tma_load_2d(sb + Lay::OFF_KV + c * Lay::CHUNK, &tm_kv, bar(Lay::B_KV_FULL + c), c * 64,
-                    phys * 128);
-      }
-      for (int c = Lay::QST; ok && c < Lay::KV_CH; ++c) ok = load_q(c);
-      // The CTA one wave later starts only when an SM frees up: pull its page
-      // and query boxes into L2 now so that its loads hit L2 instead of paying
-      // a cold HBM (and page-table) latency after this wave.
-      const int lin = (b * p.HG + hg) * p.n_split + sp;
-      const int nxt = lin + p.wave;
-      if (ok && nxt < p.B * p.HG * p.n_split) {
-        const int sp2 = nxt % p.n_split, hg2 = (nxt / p.n_split) % p.HG, b2 = nxt / (p.n_split * p.HG);
-        DecodeWindow w2;
-        if (decode_window(p, b2, w2) && sp2 < w2.tr.count) {
-          const int phys2 = decode_page(p, b2, w2, sp2);
-          if (phys2 >= 0) {
-            for (int c = 0; c < Lay::KV_CH; ++c) {
-              tma_prefetch_2d(&tm_kv, c * 64, phys2 * 128);
-              tma_prefetch_3d(&tm_q, c * 64, hg2 * 128, b2);
+      const uint32_t s_bytes = (two ? 3 : 2) * Lay::CHUNK;
+      int issued = 0;        // S stages issued
+      bool va = false, vb = false;
+      do {
+        for (int i = 0; i < Lay::KV_CH; ++i) {
+          const int st = decode_s_stage(i), r = decode_s_round(i);
+          if (r > 0 && !mbar_wait(bar(Lay::B_EMPTY + st), (r - 1) & 1, abort_flag, status, 1))
+            break;
+          const int c = decode_s_box(i);
+          const uint32_t dst = ring + st * Lay::STAGE, full = bar(Lay::B_FULL + st);
+          mbar_arrive_expect_tx(full, s_bytes);
+          tma_load_3d(dst, &tm_q, full, c * 64, hg * 128, b);
+          tma_load_2d(dst + Lay::CHUNK, &tm_kv, full, c * 64, phys_a * 128);
+          if (two) tma_load_2d(dst + 2 * Lay::CHUNK, &tm_kv, full, c * 64, phys_b * 128);
+          ++issued;
+          if (i == 0) {
+            // A CTA one wave later starts only when an SM frees up: pull its
+            // pages into L2 now so that its loads hit L2.
+            const long long nxt = (long long)cta + p.wave;
+            if (nxt < (long long)p.B * p.HG * p.n_split) {
+              const int n2 = (int)nxt;
+              const int sp2 = n2 % p.n_split, hg2 = (n2 / p.n_split) % p.HG;
+              const int b2 = n2 / (p.n_split * p.HG);
+              DecodeWindow w2;
+              if (decode_window(p, b2, w2)) {
+                for (int i2 = kDecodePagesPerSplit * sp2;
+                     i2 < min(kDecodePagesPerSplit * (sp2 + 1), w2.tr.count); ++i2) {
+                  const int ph2 = decode_page(p, b2, w2, i2);
+                  if (ph2 < 0) continue;
+                  for (int c2 = 0; c2 < Lay::KV_CH; ++c2)
+                    tma_prefetch_2d(&tm_kv, c2 * 64, ph2 * 128);
+                }
+                for (int c2 = 0; c2 < Lay::KV_CH; ++c2)
+                  tma_prefetch_3d(&tm_q, c2 * 64, hg2 * 128, b2);
+              }
             }
           }
         }
+        if (issued < Lay::KV_CH) break;
+        // V columns 0..255 (boxes 0..3) again: page A's into the Q slots, free
+        // once S is done; page B's into the K_B slots, free once O half 1
+        // (which reads boxes 4..7 there) is done.  Box e goes to stage e.
+        if (!mbar_wait(bar(Lay::B_S_FULL), 0, abort_flag, status, 1)) break;
+        mbar_arrive_expect_tx(bar(Lay::B_VA_FULL), 4 * Lay::CHUNK);
+        for (int e = 0; e < 4; ++e)
+          tma_load_2d(ring + e * Lay::STAGE, &tm_kv, bar(Lay::B_VA_FULL), e * 64, phys_a * 128);
+        va = true;
+        if (!two) break;
+        if (!mbar_wait(bar(Lay::B_O_FULL), 0, abort_flag, status, 1)) break;
+        mbar_arrive_expect_tx(bar(Lay::B_VB_FULL), 4 * Lay::CHUNK);
+        for (int e = 0; e < 4; ++e)
+          tma_load_2d(ring + e * Lay::STAGE + 2 * Lay::CHUNK, &tm_kv, bar(Lay::B_VB_FULL), e * 64,
+                      phys_b * 128);
+        vb = true;
+      } while (false);
+      // every copy issued lands before the CTA exits
+      for (int s = 0; s < Lay::NST; ++s) {
+        int last = -1;  // newest S stage issued into ring stage s
+        for (int i = 0; i < issued; ++i)
+          if (decode_s_stage(i) == s) last = i;
+        if (last >= 0) mbar_wait_drain(bar(Lay::B_FULL + s), decode_s_round(last) & 1);
       }
-      // every copy issued lands before the CTA exits (normally already consumed)
-      for (int c = 0; c < Lay::KV_CH; ++c) mbar_wait_drain(bar(Lay::B_KV_FULL + c), 0);
-      for (int st = 0; st < Lay::QST; ++st) {
-        const int n = (q_issued - st + Lay::QST - 1) / Lay::QST;  // loads issued into slot st
-        if (n > 0) mbar_wait_drain(bar(Lay::B_Q_FULL + st), (n - 1) & 1);
-      }
+      if (va) mbar_wait_drain(bar(Lay::B_VA_FULL), 0);
+      if (vb) mbar_wait_drain(bar(Lay::B_VB_FULL), 0);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------- MMA
     if (lane == 0) {
-      const uint32_t id_s = idesc_bf16_f32(128, 128, false);
+      const uint32_t id_s = idesc_bf16_f32(128, two ? 256 : 128, false);
       const uint32_t id_o = idesc_bf16_f32(128, 256, true);
+      const uint32_t o_tm = tmem + Lay::TM_O;
       bool ok = true;
-      for (int c = 0; ok && c < Lay::KV_CH; ++c) {
-        const int st = c % Lay::QST;
-        ok = mbar_wait(bar(Lay::B_KV_FULL + c), 0, abort_flag, status, 1) &&
-             mbar_wait(bar(Lay::B_Q_FULL + st), (c / Lay::QST) & 1, abort_flag, status, 1);
-        if (!ok) break;
+      for (int i = 0; i < Lay::KV_CH; ++i) {
+        const int st = decode_s_stage(i);
+        if (!(ok = mbar_wait(bar(Lay::B_FULL + st), decode_s_round(i) & 1, abort_flag, status, 1)))
+          break;
         tc_fence_after();
+        const uint32_t base = ring + st * Lay::STAGE;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t adesc = sdesc_sw128(sb + Lay::OFF_Q + st * Lay::CHUNK + kk * 32, 16, 1024);
-          const uint64_t bdesc = sdesc_sw128(sb + Lay::OFF_KV + c * Lay::CHUNK + kk * 32, 16, 1024);
-          mma_ss(tmem, adesc, bdesc, id_s, (c > 0 || kk > 0) ? 1u : 0u);
+          // A: the Q box; B: the K_A box and the K_B box right after it, one
+          // K-major operand of 256 rows.
+          const uint64_t adesc = sdesc_sw128(base + kk * 32, 16, 1024);
+          const uint64_t bdesc = sdesc_sw128(base + Lay::CHUNK + kk * 32, 16, 1024);
+          mma_ss(tmem, adesc, bdesc, id_s, (i > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(bar(Lay::B_Q_EMPTY + st));
+        if (i < Lay::KV_CH - Lay::N_KEEP) mma_commit(bar(Lay::B_EMPTY + st));  // else kept
       }
       if (ok) {
         mma_commit(bar(Lay::B_S_FULL));
         ok = mbar_wait(bar(Lay::B_P_FULL), 0, abort_flag, status, 1);
       }
-      if (ok) {
+      // O half = P V[:, 256 columns]: V rows (keys) 16kk .. 16kk+15 of page A
+      // (then B) across four 64-column boxes one STAGE apart, MN-major; the
+      // P_A / P_B words of those keys are TMEM columns 8kk .. (128 + 8kk ..).
+      auto pv_page = [&](uint32_t v_base, uint32_t p_col, bool first) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(o_tm, tmem + p_col + kk * 8, sdesc_sw128(v_base + kk * 2048, Lay::STAGE, 1024),
+                 id_o, (!first || kk > 0) ? 1u : 0u);
+      };
+      if (ok) {  // half 1 (columns 256..511): the kept S stages
         tc_fence_after();
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t adesc =
-                sdesc_sw128(sb + Lay::OFF_P + (kk >> 2) * Lay::CHUNK + (kk & 3) * 32, 16, 1024);
-            const uint64_t bdesc = sdesc_sw128(
-                sb + Lay::OFF_KV + half * 4 * Lay::CHUNK + kk * 2048, Lay::CHUNK, 1024);
-            mma_ss(tmem + half * 256, adesc, bdesc, id_o, kk > 0 ? 1u : 0u);
-          }
-        }
+        pv_page(ring + Lay::CHUNK, 0, true);
+        if (two) pv_page(ring + 2 * Lay::CHUNK, 128, false);
         mma_commit(bar(Lay::B_O_FULL));
+        ok = mbar_wait(bar(Lay::B_VA_FULL), 0, abort_flag, status, 1) &&
+             mbar_wait(bar(Lay::B_O_EMPTY), 0, abort_flag, status, 1);
+      }
+      if (ok) {  // half 0 (columns 0..255): the reloaded boxes
+        tc_fence_after();
+        pv_page(ring, 0, true);
+        if (two && (ok = mbar_wait(bar(Lay::B_VB_FULL), 0, abort_flag, status, 1))) {
+          tc_fence_after();
+          pv_page(ring + 2 * Lay::CHUNK, 128, false);
+        }
+        if (ok) mma_commit(bar(Lay::B_O_FULL));
       }
       mma_commit(bar(Lay::B_DRAIN));
       mbar_wait_drain(bar(Lay::B_DRAIN), 0);
     }
   } else {
     // ----------------------------------------------------- softmax + output
-    const int h = threadIdx.x;  // head row within the group
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int wg = warp >> 2;             // 0: page A, 1: page B
+    const int h = threadIdx.x & 127;      // head row within the group
+    const uint32_t t_row = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t s_col = wg * 128;
+    const int valid_keys = wg == 0 ? valid_a : (two ? valid_b : 0);  // warp-uniform
+    const bool partial = valid_keys < 128;
+    float* xmax = reinterpret_cast<float*>(smem + Lay::OFF_XCHG);
+    float* xsum = xmax + 256;
     const float sl2 = p.scale_log2;
     do {
       if (!mbar_wait(bar(Lay::B_S_FULL), 0, abort_flag, status, 1)) break;
       tc_fence_after();
-      uint32_t sr[4][32];
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) tmem_ld32(tmem + lane_base + ch * 32, sr[ch]);
-      tmem_wait_ld();
-      if (valid_keys < 128) {
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch)
-#pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (ch * 32 + c >= valid_keys) sr[ch][c] = __float_as_uint(-INFINITY);
-      }
+      // Pass 1: this page's row max, 64 keys at a time.
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (valid_keys > 0) {
 #pragma unroll
-      for (int c = 0; c < 128; c += 8)
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t v[2][32];
+          tmem_ld32(t_row + s_col + hf * 64, v[0]);
+          tmem_ld32(t_row + s_col + hf * 64 + 32, v[1]);
+          tmem_wait_ld();
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
-          mx4[a] = fmax3(mx4[a], __uint_as_float(sr[(c + 2 * a) >> 5][(c + 2 * a) & 31]),
-                         __uint_as_float(sr[(c + 2 * a + 1) >> 5][(c + 2 * a + 1) & 31]));
-      const float m = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * sl2;
+          for (int jj = 0; jj < 2; ++jj) {
+            const uint32_t vm = partial ? decode_chunk_mask(valid_keys, 2 * hf + jj) : 0xffffffffu;
+#pragma unroll
+            for (int c = 0; c < 32; c += 8)
+#pragma unroll
+              for (int a = 0; a < 4; ++a) {
+                const int k0 = c + 2 * a;
+                const float x0 = ((vm >> k0) & 1u) ? __uint_as_float(v[jj][k0]) : -INFINITY;
+                const float x1 =
+                    ((vm >> (k0 + 1)) & 1u) ? __uint_as_float(v[jj][k0 + 1]) : -INFINITY;
+                mx4[a] = fmax3(mx4[a], x0, x1);
+              }
+          }
+        }
+      }
+      const float mloc = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+      xmax[wg * 128 + h] = mloc;
+      mbar_arrive(bar(Lay::B_XCHG));
+      if (!mbar_wait(bar(Lay::B_XCHG), 0, abort_flag, status, 1)) break;
+      const float m = fmaxf(mloc, xmax[(wg ^ 1) * 128 + h]) * sl2;  // finite: page A has a key
       const uint64_t sl2x2 = f2_pack(sl2, sl2);
       const uint64_t negm2 = f2_pack(-m, -m);
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-      // P row h -> smem, K-major 128B-swizzled: box (key/64), row h, 16-byte unit u
-      // holding keys 8u..8u+7 lands at unit u ^ (h & 7).
-      uint8_t* prow = smem + Lay::OFF_P + h * 128;
+      // Pass 2: p = exp2(s * scale * log2(e) - m) 32 keys at a time (masked
+      // keys: exp2(-inf) = 0), packed to bf16 pairs.  The P words of keys
+      // 32ch .. 32ch+31 go to columns 16ch .. 16ch+15 of this page's S
+      // columns, which this thread has already read.
+      if (valid_keys > 0) {
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t v[32], pk16[16];
+          tmem_ld32(t_row + s_col + ch * 32, v);
+          tmem_wait_ld();
+          const uint32_t vm = partial ? decode_chunk_mask(valid_keys, ch) : 0xffffffffu;
 #pragma unroll
-      for (int box = 0; box < 2; ++box) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          uint32_t w4[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int col = box * 64 + u * 8 + 2 * e;
-            const uint64_t xx = f2_pack(__uint_as_float(sr[col >> 5][col & 31]),
-                                        __uint_as_float(sr[(col + 1) >> 5][(col + 1) & 31]));
+          for (int c = 0; c < 16; ++c) {
+            const float v0 = ((vm >> (2 * c)) & 1u) ? __uint_as_float(v[2 * c]) : -INFINITY;
+            const float v1 =
+                ((vm >> (2 * c + 1)) & 1u) ? __uint_as_float(v[2 * c + 1]) : -INFINITY;
             float y0, y1, p0, p1;
-            f2_unpack(f2_fma(xx, sl2x2, negm2), y0, y1);
-            if (((u * 4 + e) & 7) < kDecodePolyPairsPer8) {
+            f2_unpack(f2_fma(f2_pack(v0, v1), sl2x2, negm2), y0, y1);
+            if ((c & 7) < kDecodePolyPairsPer8) {
               exp2_poly_x2(y0, y1, p0, p1);
             } else {
               p0 = ex2_approx(y0);
               p1 = ex2_approx(y1);
             }
-            acc[e] = f2_add(acc[e], f2_pack(p0, p1));
-            w4[e] = pack_bf16x2(p0, p1);
+            acc[c & 3] = f2_add(acc[c & 3], f2_pack(p0, p1));
+            pk16[c] = pack_bf16x2(p0, p1);
           }
-          *reinterpret_cast<uint4*>(prow + box * Lay::CHUNK + ((u ^ (h & 7)) << 4)) =
-              make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          tmem_st16(t_row + s_col + ch * 16, pk16);
         }
+        tmem_wait_st();
       }
-      float l;
+      tc_fence_before();
+      mbar_arrive(bar(Lay::B_P_FULL));
+      float lloc;
       {
         float a0, a1;
         f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
-        l = a0 + a1;
+        lloc = a0 + a1;
       }
-      fence_async_shared();
-      tc_fence_before();
-      mbar_arrive(bar(Lay::B_P_FULL));
+      xsum[wg * 128 + h] = lloc;
+      mbar_arrive(bar(Lay::B_XCHG));
+      if (!mbar_wait(bar(Lay::B_XCHG), 1, abort_flag, status, 1)) break;
+      const float l = lloc + xsum[(wg ^ 1) * 128 + h];
 
-      if (!mbar_wait(bar(Lay::B_O_FULL), 0, abort_flag, status, 1)) break;
-      tc_fence_after();
-      asm volatile("griddepcontrol.launch_dependents;");
       const bool valid = hg * 128 + h < p.H_q;
       const float inv_l = 1.f / l;
-      // Stage row h of the partial O (fp16) in the page buffer, laid out as the
-      // 128B-swizzled [128 rows x 64 columns] boxes a TMA store reads:
-      // 16-byte unit u of box c, row h, sits at unit u ^ (h & 7).
-      uint8_t* srow = smem + Lay::OFF_KV + h * 128;
+      // O half hf (1 first): warpgroup wg takes its 128 columns 128wg .. of the
+      // half, i.e. 8-column groups 32hf + 16wg + g of the row.
+      uint4* dst = reinterpret_cast<uint4*>(p.o_part) + cta * (64 * 128) + h;
+      bool ok = true;
 #pragma unroll 1
-      for (int j = 0; j < kDecodeDv / 64; ++j) {
-        uint32_t orr[2][32];
-        tmem_ld32(tmem + lane_base + j * 64, orr[0]);
-        tmem_ld32(tmem + lane_base + j * 64 + 32, orr[1]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint32_t* r8 = &orr[u >> 2][(u & 3) * 8];
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            __half2 hv = __floats2half2_rn(__uint_as_float(r8[2 * e]) * inv_l,
-                                           __uint_as_float(r8[2 * e + 1]) * inv_l);
-            w[e] = *reinterpret_cast<uint32_t*>(&hv);
+      for (int n = 0; n < 2; ++n) {
+        const int hf = 1 - n;
+        if (!(ok = mbar_wait(bar(Lay::B_O_FULL), n, abort_flag, status, 1))) break;
+        tc_fence_after();
+        if (n == 1) asm volatile("griddepcontrol.launch_dependents;");
+#pragma unroll 1
+        for (int part = 0; part < 2; ++part) {  // 64 columns at a time
+          uint32_t orr[2][32];
+          tmem_ld32(t_row + Lay::TM_O + 128 * wg + 64 * part, orr[0]);
+          tmem_ld32(t_row + Lay::TM_O + 128 * wg + 64 * part + 32, orr[1]);
+          tmem_wait_ld();
+          if (part == 1) {
+            tc_fence_before();
+            mbar_arrive(bar(Lay::B_O_EMPTY));  // the MMA may reuse the buffer now
           }
-          *reinterpret_cast<uint4*>(srow + j * Lay::CHUNK + ((u ^ (h & 7)) << 4)) =
-              make_uint4(w[0], w[1], w[2], w[3]);
+          if (valid) {
+#pragma unroll
+            for (int g = 0; g < 8; ++g) {
+              const uint32_t* r8 = &orr[g >> 2][(g & 3) * 8];
+              uint32_t w[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                __half2 hv = __floats2half2_rn(__uint_as_float(r8[2 * q]) * inv_l,
+                                               __uint_as_float(r8[2 * q + 1]) * inv_l);
+                w[q] = *reinterpret_cast<uint32_t*>(&hv);
+              }
+              dst[(32 * hf + 16 * wg + 8 * part + g) * 128] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          }
         }
       }
-      fence_async_shared();
-      mbar_arrive(bar(Lay::B_EPI));
-      if (h == 0 && mbar_wait(bar(Lay::B_EPI), 0, abort_flag, status, 1)) {
-        // rows part..part+127 of the [rows x 512] fp16 workspace, 8 boxes
-#pragma unroll
-        for (int j = 0; j < kDecodeDv / 64; ++j)
-          tma_store_2d(&tm_part, sb + Lay::OFF_KV + j * Lay::CHUNK, j * 64, (int)part);
-        tma_store_commit_and_wait_read();  // smem is read before the CTA exits
-      }
-      if (valid) p.lse_part[part + h] = (m + __log2f(l)) * kLn2;
+      if (ok && valid && wg == 0) p.lse_part[cta * 128 + h] = (m + __log2f(l)) * kLn2;
     } while (false);
   }
 
   __syncwarp();
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, Lay::TMEM_COLS);
   }
 }
 
-// One CTA of 64 threads per (sequence, head): each thread merges 8 of the 512
-// output columns (one 16-byte fp16 load per split).  Launched as a programmatic
-// dependent of the split kernel; it waits for the split kernel's results
-// before reading.  Splits whose LSE is -inf are empty and contribute nothing
-// (their partial O is never read into the sum).
-constexpr int kMergeThreads = kDecodeDv / 8;
+// Merge: one CTA per (sequence, 8 heads); thread (column group g, head hh)
+// reads 16 bytes per split, so that a warp's reads of one split are four runs
+// of 128 contiguous bytes, four splits' loads in flight at once.  Launched as
+// a programmatic dependent of the split kernel; it waits for the split
+// kernel's results before reading.  Splits whose LSE is -inf are empty and
+// contribute nothing (their partial O is never read into the sum).
+constexpr int kMergeHeads = 8;
+constexpr int kMergeThreads = (kDecodeDv / 8) * kMergeHeads;  // 512
+constexpr int kMergeBatch = 4;
 
 __global__ void __launch_bounds__(kMergeThreads)
     ssa_decode_merge_kernel(const DecodeParams p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int b = blockIdx.x / p.H_q, h = blockIdx.x % p.H_q;
+  const int groups = (p.H_q + kMergeHeads - 1) / kMergeHeads;
+  const int b = blockIdx.x / groups;
+  const int hh = threadIdx.x % kMergeHeads, g = threadIdx.x / kMergeHeads;
+  const int h = (blockIdx.x % groups) * kMergeHeads + hh;
+  if (h >= p.H_q) return;
   const int hg = h >> 7, hr = h & 127;
-  const size_t base = (size_t)(b * p.HG + hg) * p.n_split;
-  const float* lsep = p.lse_part + base * 128 + hr;              // split stride 128
-  const uint4* op = reinterpret_cast<const uint4*>(p.o_part + (base * 128 + hr) * kDecodeDv) +
-                    threadIdx.x;                                // split stride 128*512/8
-  constexpr size_t kSplitStride = 128 * kDecodeDv / 8;
+  const size_t cta0 = ((size_t)b * p.HG + hg) * p.n_split;
+  const float* lsep = p.lse_part + cta0 * 128 + hr;  // split stride 128
+  const uint4* op = reinterpret_cast<const uint4*>(p.o_part) + (cta0 * 64 + g) * 128 + hr;
+  constexpr size_t kSplitStride = 64 * 128;  // uint4 per split
+  const int n = p.n_split;
   float lmax = -INFINITY;
-#pragma unroll 8
-  for (int s = 0; s < p.n_split; ++s) lmax = fmaxf(lmax, __ldg(lsep + s * 128));
+  for (int s = 0; s < n; ++s) lmax = fmaxf(lmax, __ldg(lsep + (size_t)s * 128));
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   float denom = 0.f;
   if (lmax > -INFINITY) {
-#pragma unroll 8
-    for (int s = 0; s < p.n_split; ++s) {
-      const float ls = __ldg(lsep + s * 128);
-      const uint4 raw = __ldg(op + s * kSplitStride);
-      if (ls == -INFINITY) continue;
-      const float wgt = __expf(ls - lmax);
-      denom += wgt;
-      const __half2* hv = reinterpret_cast<const __half2*>(&raw);
+    for (int s0 = 0; s0 < n; s0 += kMergeBatch) {
+      float ls[kMergeBatch];
+      uint4 raw[kMergeBatch];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __half22float2(hv[e]);
-        acc[2 * e] += wgt * f.x;
-        acc[2 * e + 1] += wgt * f.y;
+      for (int j = 0; j < kMergeBatch; ++j) {
+        ls[j] = -INFINITY;
+        if (s0 + j < n) {
+          ls[j] = __ldg(lsep + (size_t)(s0 + j) * 128);
+          raw[j] = __ldg(op + (size_t)(s0 + j) * kSplitStride);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kMergeBatch; ++j) {
+        if (ls[j] == -INFINITY) continue;
+        const float wgt = __expf(ls[j] - lmax);
+        denom += wgt;
+        const __half2* hv = reinterpret_cast<const __half2*>(&raw[j]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(hv[e]);
+          acc[2 * e] += wgt * f.x;
+          acc[2 * e + 1] += wgt * f.y;
+        }
       }
     }
   }
@@ -419,9 +542,8 @@ __global__ void __launch_bounds__(kMergeThreads)
   pk.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
   pk.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
   pk.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
-  *(reinterpret_cast<uint4*>(p.o + ((size_t)b * p.H_q + h) * kDecodeDv) + threadIdx.x) = pk;
-  if (threadIdx.x == 0)
-    p.lse[(size_t)b * p.H_q + h] = denom > 0.f ? lmax + __logf(denom) : -INFINITY;
+  *(reinterpret_cast<uint4*>(p.o + ((size_t)b * p.H_q + h) * kDecodeDv) + g) = pk;
+  if (g == 0) p.lse[(size_t)b * p.H_q + h] = denom > 0.f ? lmax + __logf(denom) : -INFINITY;
 }
 
 }  // namespace loza

@@ -220,6 +220,11 @@ int static_scratch_address(void** out) {
   return LOZA_SSA_OK;
 }
 
+// Split CTAs per (sequence, head group): window pages taken two at a time.
+int decode_splits(int n_sink, int n_local) {
+  return (n_sink + n_local + loza::kDecodePagesPerSplit - 1) / loza::kDecodePagesPerSplit;
+}
+
 size_t decode_partial_floats(int B, int H_q, int n_split) {
   const size_t hg = (size_t)(H_q + 127) / 128;
   return (size_t)B * hg * (size_t)n_split * 128;
@@ -321,7 +326,7 @@ size_t loza_ssa_decode_workspace_size(int B, int H_q, int d_v, int n_sink, int n
   if (B < 1 || H_q < 1 || d_v != loza::kDecodeDv || n_sink < 0 || n_local < 1 ||
       n_sink + n_local > kMaxDecodeWindow)
     return 0;
-  const size_t rows = decode_partial_floats(B, H_q, n_sink + n_local);
+  const size_t rows = decode_partial_floats(B, H_q, decode_splits(n_sink, n_local));
   const size_t o_bytes = rows * loza::kDecodeDv * sizeof(__half);  // partial O is fp16
   const size_t lse_bytes = rows * sizeof(float);
   return ((o_bytes + 255) / 256) * 256 + ((lse_bytes + 255) / 256) * 256;
@@ -350,10 +355,10 @@ int loza_ssa_decode(const void* q, const void* paged_kv, const int* page_table,
   int rc = device_info(dev);
   if (rc != LOZA_SSA_OK) return rc;
 
-  const int n_split = n_sink + n_local;
+  const int n_split = decode_splits(n_sink, n_local);
   const int HG = (H_q + 127) / 128;
   const size_t rows = decode_partial_floats(B, H_q, n_split);
-  if (rows >= (1ull << 31)) return LOZA_SSA_ERR_SHAPE;  // TMA row coordinates are 32-bit
+  if (rows >= (1ull << 31)) return LOZA_SSA_ERR_SHAPE;  // keeps the CTA index math in int
   loza::DecodeParams prm{};
   prm.page_table = page_table;
   prm.seq_lens = seq_lens;
@@ -371,15 +376,12 @@ int loza_ssa_decode(const void* q, const void* paged_kv, const int* page_table,
   prm.n_local = n_local;
   prm.n_split = n_split;
   prm.scale_log2 = scale * 1.4426950408889634f;
-  prm.wave = dev.num_sms;
+  prm.wave = dev.num_sms;  // one split CTA per SM
 
-  CUtensorMap mq, mkv, mpart;
+  CUtensorMap mq, mkv;
   if ((rc = make_map(&mq, q, loza::kDecodeDqk, (uint64_t)H_q, (uint64_t)B, 3)) != LOZA_SSA_OK)
     return rc;
   if ((rc = make_map(&mkv, paged_kv, loza::kDecodeDqk, (uint64_t)n_pages * 128, 1, 2)) != LOZA_SSA_OK)
-    return rc;
-  if ((rc = make_map(&mpart, prm.o_part, loza::kDecodeDv, (uint64_t)rows, 1, 2,
-                     CU_TENSOR_MAP_DATA_TYPE_FLOAT16)) != LOZA_SSA_OK)
     return rc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaFuncSetAttribute(loza::ssa_decode_split_kernel,
@@ -387,13 +389,12 @@ int loza_ssa_decode(const void* q, const void* paged_kv, const int* page_table,
                                        loza::DecodeLayout::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
   dim3 grid(n_split, HG, B);
-  loza::ssa_decode_split_kernel<<<grid, 192, loza::DecodeLayout::SMEM_BYTES, s>>>(mq, mkv, mpart,
-                                                                                  prm);
+  loza::ssa_decode_split_kernel<<<grid, 320, loza::DecodeLayout::SMEM_BYTES, s>>>(mq, mkv, prm);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "decode split launch");
   // the merge is a programmatic dependent of the split kernel: it is scheduled
   // as split CTAs retire and waits (griddepcontrol.wait) for their results
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(B * H_q);
+  cfg.gridDim = dim3(B * ((H_q + loza::kMergeHeads - 1) / loza::kMergeHeads));
   cfg.blockDim = dim3(loza::kMergeThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
@@ -415,10 +416,11 @@ int loza_ssa_decode_static_scratch(const void* q, const void* paged_kv, const in
   // Same checks and kernels as loza_ssa_decode; only the workspace differs.
   if (B >= 1 && H_q >= 1 && n_sink >= 0 && n_local >= 1 &&
       n_sink + n_local <= kMaxDecodeWindow) {
-    const long long slots = (long long)B * ((H_q + 127) / 128) * (n_sink + n_local);
+    const long long slots =
+        (long long)B * ((H_q + 127) / 128) * decode_splits(n_sink, n_local);
     if (slots > LOZA_SSA_STATIC_SCRATCH_SLOTS) {
       std::snprintf(g_last_error, sizeof g_last_error,
-                    "decode_static_scratch: B * ceil(H_q/128) * (n_sink + n_local) = %lld split "
+                    "decode_static_scratch: B * ceil(H_q/128) * ceil((n_sink + n_local)/2) = %lld split "
                     "slots, the built-in scratch holds %d",
                     slots, LOZA_SSA_STATIC_SCRATCH_SLOTS);
       return LOZA_SSA_ERR_SCRATCH_LIMIT;

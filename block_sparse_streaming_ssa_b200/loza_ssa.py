@@ -197,7 +197,7 @@ def loza_ssa_decode_static_scratch(q, paged_kv, page_table, seq_lens, d_v=512, o
     """loza_ssa_decode without a workspace: the library uses its built-in
     scratch array instead, so nothing is allocated for the split partials (for
     callers that cannot provide device memory when they launch).  Limited to
-    B * ceil(H_q/128) * (n_sink + n_local) <= LOZA_SSA_STATIC_SCRATCH_SLOTS;
+    B * ceil(H_q/128) * ceil((n_sink + n_local)/2) <= LOZA_SSA_STATIC_SCRATCH_SLOTS;
     calls whose kernels overlap on the GPU share that scratch and must not run
     concurrently.  Returns (o bf16 [B,H_q,d_v], lse fp32 [B,H_q])."""
     _need(q, torch.bfloat16, "q")

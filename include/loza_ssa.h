@@ -169,9 +169,10 @@ int loza_ssa_debug_decode_pages(const int* page_table, const int* seq_lens, int 
  * workspace: the split partials live instead in one scratch array compiled
  * into the library, LOZA_SSA_STATIC_SCRATCH_BYTES long, which every GPU that
  * loads the library holds until the process exits.  It holds
- * LOZA_SSA_STATIC_SCRATCH_SLOTS split slots; a call needs
- * B * ceil(H_q/128) * (n_sink + n_local) of them (e.g. 16 sequences with the
- * default 8-page window and up to 128 heads) and is rejected with
+ * LOZA_SSA_STATIC_SCRATCH_SLOTS split slots (one per split of the decode:
+ * two window pages of one sequence and head group of up to 128 heads); a call
+ * needs B * ceil(H_q/128) * ceil((n_sink + n_local)/2) of them (e.g. 32
+ * sequences with the default 8-page window and up to 128 heads) and is rejected with
  * LOZA_SSA_ERR_SCRATCH_LIMIT, before anything is launched, if it needs more.
  *
  * The first call on a device looks up that device's address of the array

@@ -55,12 +55,15 @@ def test_status_strings(L):
 
 def test_decode_workspace_size(L):
     from block_sparse_streaming_ssa_b200 import loza_ssa as api
-    # B * ceil(H_q/128) * (n_sink+n_local) * 128 rows of 512 fp16 (+1 fp32 LSE), 256-B rounded
-    rows = 32 * 1 * 8 * 128
+    # one split per two window pages: B * ceil(H_q/128) * ceil((n_sink+n_local)/2) * 128
+    # rows of 512 fp16 (+1 fp32 LSE), each part rounded up to 256 bytes
+    rows = 32 * 1 * 4 * 128
     want = -(-rows * 512 * 2 // 256) * 256 + -(-rows * 4 // 256) * 256
     assert api.loza_ssa_decode_workspace_size(32, 128, 512, 1, 7) == want
     assert api.loza_ssa_decode_workspace_size(2, 200, 512, 1, 7) == \
-        -(-2 * 2 * 8 * 128 * 1024 // 256) * 256 + -(-2 * 2 * 8 * 128 * 4 // 256) * 256
+        -(-2 * 2 * 4 * 128 * 1024 // 256) * 256 + -(-2 * 2 * 4 * 128 * 4 // 256) * 256
+    assert api.loza_ssa_decode_workspace_size(2, 128, 512, 1, 6) == \
+        api.loza_ssa_decode_workspace_size(2, 128, 512, 1, 7)        # 7 pages: 4 splits
     assert api.loza_ssa_decode_workspace_size(32, 128, 256, 1, 7) == 0      # d_v unsupported
     assert api.loza_ssa_decode_workspace_size(32, 128, 512, 1, 0) == 0      # n_local < 1
 

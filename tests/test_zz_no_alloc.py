@@ -30,8 +30,8 @@ D_QK, D_V = 576, 512
 
 def test_matches_workspace_decode_on_two_calls_in_a_row():
     scale = 1 / 24.0
-    # first call: 16 sequences x 8 window pages = all 128 built-in slots
-    lens_a = [4096 + 3000 * i for i in range(15)] + [100]
+    # first call: 32 sequences x 4 splits (8 window pages) = all 128 built-in slots
+    lens_a = [4096 + 3000 * i for i in range(31)] + [100]
     # second call: fewer, shorter sequences (most slots keep the first call's data)
     lens_b = [129, 2000, 1, 777]
     for lens, seed in ((lens_a, 1), (lens_b, 2)):
@@ -45,14 +45,15 @@ def test_matches_workspace_decode_on_two_calls_in_a_row():
 
 
 def test_rejects_more_than_the_scratch_holds():
-    q, kv, pt, sl = synth.decode_inputs([300] * 17, 128, D_QK, seed=3, device="cuda")
-    o = torch.empty((17, 128, D_V), dtype=torch.bfloat16, device="cuda")
-    lse = torch.empty((17, 128), dtype=torch.float32, device="cuda")
-    assert 17 * 8 > LOZA_SSA_STATIC_SCRATCH_SLOTS
+    n = 33
+    q, kv, pt, sl = synth.decode_inputs([300] * n, 128, D_QK, seed=3, device="cuda")
+    o = torch.empty((n, 128, D_V), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((n, 128), dtype=torch.float32, device="cuda")
+    assert n * 4 > LOZA_SSA_STATIC_SCRATCH_SLOTS
     vp = ctypes.c_void_p
     rc = lib().loza_ssa_decode_static_scratch(
         vp(q.data_ptr()), vp(kv.data_ptr()), vp(pt.data_ptr()), vp(sl.data_ptr()),
-        vp(o.data_ptr()), vp(lse.data_ptr()), 17, 128, D_QK, D_V, 128, pt.shape[1], kv.shape[0],
+        vp(o.data_ptr()), vp(lse.data_ptr()), n, 128, D_QK, D_V, 128, pt.shape[1], kv.shape[0],
         1, 7, ctypes.c_float(1 / 24.0), vp(torch.cuda.current_stream().cuda_stream))
     assert rc == LOZA_SSA_ERR_SCRATCH_LIMIT
     assert b"split slots" in lib().loza_ssa_last_error_string()
