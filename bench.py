@@ -2,7 +2,8 @@
 """Benchmark of the SSA hot path on B200 through the C ABI.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--config mha|tiny|mla|varlen] [--no-decode] [--no-cpu-baseline]
+                    [--config mha|tiny|mla|varlen] [--no-decode] [--no-prefill]
+                    [--no-cpu-baseline]
 
 One JSON line on rank 0.  A step is one SSA prefill call over the chosen
 workload (default: B=1, H=32, L=32768, d=128, 1 sink + 7 local blocks of 128);
@@ -68,10 +69,20 @@ def row_pairs(i: np.ndarray, blk=128, n_sink=1, n_local=7) -> np.ndarray:
     return np.minimum(i + 1, blk * (n_sink + n_local - 1) + (i % blk) + 1)
 
 
-def source_hash() -> str:
+# Kernel sources each profiled kernel is built from: a committed traffic figure
+# stays valid only while these files are unchanged.
+KERNEL_SOURCES = {
+    "ssa_prefill_pair_kernel": ("prefill_pair.cuh", "prefill.cuh", "ptx.cuh", "schedule.cuh"),
+    "ssa_prefill_kernel": ("prefill.cuh", "ptx.cuh", "schedule.cuh"),
+    "ssa_decode_split_kernel": ("decode.cuh", "ptx.cuh", "schedule.cuh"),
+    "ssa_decode_merge_kernel": ("decode.cuh", "ptx.cuh", "schedule.cuh"),
+}
+
+
+def source_hash(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_sparse_streaming_ssa_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:12]
@@ -85,7 +96,7 @@ def traffic_lookup(kernel: str, workload: str):
         lines = open(path).read().splitlines()
     except OSError:
         return None
-    cur = source_hash()
+    cur = source_hash(kernel)
     for ln in lines:
         parts = ln.split()
         if len(parts) == 4 and not ln.startswith("#") and parts[0] == kernel and \
@@ -141,6 +152,26 @@ class ClockSampler:
         names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
                 "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------ multi-rank
+
+def max_over_ranks(ms: float) -> float:
+    """Slowest rank's device time (every rank times its own replica; the job
+    is done when the slowest one is).  Single process: the value itself."""
+    import torch
+    import torch.distributed as td
+    if not (td.is_available() and td.is_initialized()):
+        return ms
+    dev = "cuda" if td.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    td.all_reduce(t, op=td.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, units_per_rank_step: float, steps: int, max_ms: float) -> float:
+    """Whole-job rate: the units all ranks processed / the slowest rank's time."""
+    return world * units_per_rank_step * steps / (max_ms * 1e-3)
 
 
 # ---------------------------------------------------------------- prefill
@@ -243,7 +274,15 @@ def e2e_prefill(w, steps):
 
 # ----------------------------------------------------------------- decode
 
-def decode_bench(iters, warmup, peaks, seed=0, len_hi=None):
+def decode_bench(iters, warmup, peaks, seed=0, len_hi=None, n_sets=8, world=1):
+    """Paged decode through the public call.  ``value``: algorithmic bytes per
+    call / device time per call, with the calls captured in a CUDA graph (the
+    way a serving loop issues decode steps) and rotating over ``n_sets``
+    batches that share the page pool but read different pages (own page
+    table and queries each), so that consecutive calls find nothing of their
+    inputs in L2.  ``eager_flush_us``: one eager call per step after a 2x L2
+    write, for comparison (it also pays the write-back of the flushed lines
+    and, when the GPU runs dry, the host-side cost of the call)."""
     import torch
     from block_sparse_streaming_ssa_b200 import synth
     from block_sparse_streaming_ssa_b200.loza_ssa import (loza_ssa_decode,
@@ -257,36 +296,75 @@ def decode_bench(iters, warmup, peaks, seed=0, len_hi=None):
     keys = int(sum(row_pairs(np.array([n - 1]))[0] for n in lens))
     algo_bytes = keys * s.d_qk * 2 + q.numel() * 2 + o.numel() * 2 + lse.numel() * 4
     flops = 2 * (s.d_qk + s.d_v) * keys * s.H_q
-    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
-    for _ in range(warmup):
-        loza_ssa_decode(q, kv, pt, sl, s.d_v, o=o, lse=lse, scale=s.scale, workspace=ws)
-    times = []
-    for _ in range(iters):
-        flush.fill_(1)   # cold L2 for every timed step
+
+    gen = torch.Generator(device="cpu").manual_seed(1000 + seed)
+    sets = [(q, pt)]
+    for _ in range(n_sets - 1):
+        perm = torch.randperm(kv.shape[0], generator=gen).to(torch.int32).cuda()
+        sets.append((torch.randn(q.shape, generator=gen).to(torch.bfloat16).cuda(),
+                     torch.where(pt >= 0, perm[pt.clamp(min=0).long()], pt)))
+    distinct_kv = n_sets * keys * s.d_qk * 2
+
+    def call(i):
+        qq, pp = sets[i % n_sets]
+        loza_ssa_decode(qq, kv, pp, sl, s.d_v, o=o, lse=lse, scale=s.scale, workspace=ws)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for i in range(max(warmup, n_sets)):
+            call(i)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        for i in range(iters):
+            call(i)
+    torch.cuda.synchronize()
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    reps = []
+    for _ in range(5):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        loza_ssa_decode(q, kv, pt, sl, s.d_v, o=o, lse=lse, scale=s.scale, workspace=ws)
+        graph.replay()
         b.record()
-        times.append((a, b))
+        torch.cuda.synchronize()
+        reps.append(a.elapsed_time(b) / iters)
+    ms = max_over_ranks(statistics.median(reps))
+
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+    eager = []
+    for i in range(iters):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        call(i)
+        b.record()
+        eager.append((a, b))
     torch.cuda.synchronize()
-    ms = [a.elapsed_time(b) for a, b in times]
-    mean_ms = sum(ms) / len(ms)
-    gbs = algo_bytes / (mean_ms * 1e-3) / 1e9
+    eager_ms = statistics.median([a.elapsed_time(b) for a, b in eager])
+    del graph
+
+    gbs = job_throughput(world, algo_bytes, 1, ms) / 1e9
     return {
         "workload": f"ssa_decode B={s.B} H_q={s.H_q} d_qk={s.d_qk} d_v={s.d_v} paged 128, "
                     f"seq_len U[{s.len_lo},{len_hi or s.len_hi}] seed {seed}, random page permutation "
                     f"over {kv.shape[0]} pages",
-        "value": round(gbs, 1), "unit": "GB/s", "us_per_step": round(mean_ms * 1e3, 2),
-        "median_us": round(statistics.median(ms) * 1e3, 2),
+        "value": round(gbs, 1), "unit": "GB/s", "us_per_step": round(ms * 1e3, 2),
         "algorithmic_bytes_per_step": algo_bytes, "useful_gflop_per_step": round(flops / 1e9, 3),
-        "tflops": round(flops / (mean_ms * 1e-3) / 1e12, 1),
-        "l2": "flushed (2x L2 write) before every timed step",
-        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+        "tflops": round(flops / (ms * 1e-3) / 1e12, 1),
+        "l2": f"inputs larger than L2: {n_sets} rotating batches with their own page tables "
+              f"and queries ({distinct_kv / 2**20:.0f} MiB of distinct KV pages), "
+              f"{iters} calls per CUDA graph replay",
+        "eager_flush_us": round(eager_ms * 1e3, 2),
+        "roofline": {"bound": "hbm", "achieved": round(gbs / world, 1), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(gbs / world / peaks["hbm_gbs"], 4),
                      "traffic": traffic_lookup("ssa_decode_split_kernel", "decode"),
                      "peak_source": peaks["source"],
                      "note": "time of the whole call: split kernel + LSE merge kernel"},
-        "gpu_launches": 2 * iters,
+        "gpu_launches": 2 * iters * 5 + 2 * iters,
     }
 
 
@@ -316,9 +394,13 @@ def oracle_sample(config, budget_s, seed=0):
     fl, dt, n = run(64)
     n2 = int(min(H * sp.L, max(64, 64 * budget_s / max(dt, 1e-3))))
     fl, dt, n = run(n2)
-    return fl, dt, n, orc.num_threads(), (
-        f"{n} random query rows of {H} heads of the {sp.name} workload (B=1, L={sp.L}, "
-        f"d_qk={sp.d_qk}, d_v={sp.d_v}), each against its full SSA window, float64")
+    passes = 1
+    while dt < budget_s:  # every row of the sample already taken: run fresh samples
+        f2, d2, _ = run(n2)
+        fl, dt, passes = fl + f2, dt + d2, passes + 1
+    return fl, dt, n * passes, orc.num_threads(), (
+        f"{passes} x {n} random query rows of {H} heads of the {sp.name} workload (B=1, "
+        f"L={sp.L}, d_qk={sp.d_qk}, d_v={sp.d_v}), each against its full SSA window, float64")
 
 
 # ------------------------------------------------------------------- main
@@ -331,12 +413,16 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", choices=["mha", "tiny", "mla", "varlen"], default="mha")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="time only the decode workload (for profiler captures of it)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--decode-iters", type=int, default=30)
     ap.add_argument("--decode-len-hi", type=int, default=None,
                     help="shorter decode contexts (smaller page pool), for profiler captures")
     ap.add_argument("--cpu-budget-s", type=float, default=10.0)
+    ap.add_argument("--ref-budget-s", type=float, default=60.0,
+                    help="--impl reference: CPU seconds over all warm-up and timed steps")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -348,7 +434,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        per_step_budget = max(0.5, 60.0 / (args.steps + args.warmup))
+        per_step_budget = max(0.1, args.ref_budget_s / (args.steps + args.warmup))
         fl_tot, t_tot, rows_tot = 0, 0.0, 0
         threads, desc = 1, ""
         for i in range(args.warmup + args.steps):
@@ -380,15 +466,21 @@ def main():
     else:
         torch.cuda.set_device(0)
 
+    if args.no_prefill:
+        decode = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
+                              len_hi=args.decode_len_hi, world=world)
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "decode": decode}), flush=True)
+        if dist:
+            torch.distributed.destroy_process_group()
+        return
+
     w = make_prefill(args.config, "cuda", seed=rank)
     total_ms, per, clocks = time_prefill(w, args.steps, args.warmup, dist)
-    t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-    if dist:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = max_over_ranks(total_ms)
     ms_step = max_ms / args.steps
     flops = 2 * (w["spec"].d_qk + w["spec"].d_v) * w["pairs"]
-    value = world * flops * args.steps / (max_ms * 1e-3) / 1e12
+    value = job_throughput(world, flops, args.steps, max_ms) / 1e12
     avg_launch_ms = sum(per) / len(per)
     achieved = flops / (avg_launch_ms * 1e-3) / 1e12
     e2e_ms, h2d, d2h = e2e_prefill(w, args.e2e_steps)
@@ -400,7 +492,7 @@ def main():
         del w
         torch.cuda.empty_cache()
         decode = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
-                              len_hi=args.decode_len_hi)
+                              len_hi=args.decode_len_hi, world=world)
 
     if rank != 0:
         if dist:
@@ -412,7 +504,8 @@ def main():
         fl, dt, n, threads, desc = oracle_sample(args.config, args.cpu_budget_s)
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": desc + f", {dt:.1f} s"}
-    kname = "ssa_prefill_kernel"
+    # d_qk <= 128 runs the two-query-block kernel, d_qk = 192 the one-block kernel
+    kname = "ssa_prefill_pair_kernel" if w_desc.get("d_qk", 128) <= 128 else "ssa_prefill_kernel"
     wl = {"mha": "mha", "tiny": "tiny", "mla": "mla", "varlen": "varlen"}[args.config]
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
@@ -422,7 +515,7 @@ def main():
         "config": {**w_desc, "n_sink": 1, "n_local": 7, "block": 128,
                    "parallelism": f"{world} independent replicas (weak scaling, no data-path collective)",
                    "l2": "inputs larger than L2 (q, k, v re-read from HBM every step)"},
-        "tokens_per_s": round(world * w_tokens * args.steps / (max_ms * 1e-3), 1),
+        "tokens_per_s": round(job_throughput(world, w_tokens, args.steps, max_ms), 1),
         "useful_tflop_per_step": round(flops / 1e12, 4),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
