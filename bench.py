@@ -72,7 +72,6 @@ def row_pairs(i: np.ndarray, blk=128, n_sink=1, n_local=7) -> np.ndarray:
 # Kernel sources each profiled kernel is built from: a committed traffic figure
 # stays valid only while these files are unchanged.
 KERNEL_SOURCES = {
-    "ssa_prefill_pair_kernel": ("prefill_pair.cuh", "prefill.cuh", "ptx.cuh", "schedule.cuh"),
     "ssa_prefill_kernel": ("prefill.cuh", "ptx.cuh", "schedule.cuh"),
     "ssa_decode_split_kernel": ("decode.cuh", "ptx.cuh", "schedule.cuh"),
     "ssa_decode_merge_kernel": ("decode.cuh", "ptx.cuh", "schedule.cuh"),
@@ -504,8 +503,14 @@ def main():
         fl, dt, n, threads, desc = oracle_sample(args.config, args.cpu_budget_s)
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": desc + f", {dt:.1f} s"}
-    # d_qk <= 128 runs the two-query-block kernel, d_qk = 192 the one-block kernel
-    kname = "ssa_prefill_pair_kernel" if w_desc.get("d_qk", 128) <= 128 else "ssa_prefill_kernel"
+    kname = "ssa_prefill_kernel"
+    # A kernel timed back to back for more than ~0.1 s runs under the power
+    # cap: compare it with the sustained GEMM figure, a short burst with the
+    # burst figure.
+    sustained = max_ms > 100.0
+    peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    peak_note = (" (sustained bf16 GEMM: the timed region is %.0f ms of back-to-back launches)"
+                 if sustained else " (burst bf16 GEMM: the timed region is %.0f ms)") % max_ms
     wl = {"mha": "mha", "tiny": "tiny", "mla": "mla", "varlen": "varlen"}[args.config]
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
@@ -518,10 +523,10 @@ def main():
         "tokens_per_s": round(job_throughput(world, w_tokens, args.steps, max_ms), 1),
         "useful_tflop_per_step": round(flops / 1e12, 4),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
-                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": round(achieved / peaks["bf16_tflops"], 4),
+                     "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4),
                      "traffic": traffic_lookup(kname, wl), "peak_source": peaks["source"] +
-                     " (burst bf16 GEMM: the kernel is timed alone)",
+                     peak_note,
                      "kernel": kname, "avg_launch_ms": round(avg_launch_ms, 4)},
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_val, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,

@@ -13,7 +13,6 @@
 #include "../../include/loza_ssa.h"
 #include "decode.cuh"
 #include "prefill.cuh"
-#include "prefill_pair.cuh"
 #include "schedule.cuh"
 
 namespace {
@@ -101,15 +100,13 @@ int make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint6
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// PAIR: the two-query-block kernel (prefill_pair.cuh, d_qk <= 128); else the
-// one-block kernel (prefill.cuh).  Dense inputs get their exact work-item count
-// here; packed inputs count theirs on the device (items_upper bounds the grid).
-template <int DQK, int DV, bool PAIR>
+// Dense inputs get their exact work-item count here; packed inputs count
+// theirs on the device (items_upper bounds the grid).
+template <int DQK, int DV>
 int launch_prefill(const void* q, const void* k, const void* v, loza::PrefillParams prm,
                    uint64_t plane_rows, uint64_t planes, long long items_upper, int n_prefix,
                    cudaStream_t stream, const DeviceInfo& dev) {
-  using Single = loza::PrefillLayout<DQK, DV>;
-  using Pair = loza::PairLayout<DQK, DV>;
+  using Lay = loza::PrefillLayout<DQK, DV>;
   CUtensorMap mq, mk, mv;
   int rc;
   if ((rc = make_map(&mq, q, DQK, plane_rows, planes, 3)) != LOZA_SSA_OK) return rc;
@@ -117,29 +114,19 @@ int launch_prefill(const void* q, const void* k, const void* v, loza::PrefillPar
   if ((rc = make_map(&mv, v, DV, plane_rows, planes, 3)) != LOZA_SSA_OK) return rc;
   if (prm.cu_seqlens == nullptr) {
     const long long nb = (prm.L + 127) / 128;
-    items_upper = (long long)planes * (PAIR ? (nb + 1) / 2 : nb);
+    items_upper = (long long)planes * nb;
     prm.total_items = (int)items_upper;
   }
-  size_t smem, smem_max;
-  int threads;
-  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, loza::PrefillParams);
-  if constexpr (PAIR) {
-    smem = Pair::smem_bytes(n_prefix);
-    smem_max = Pair::smem_bytes(kMaxVarlenSeqs + 1);
-    kern = loza::ssa_prefill_pair_kernel<DQK, DV>;
-    threads = loza::kPairThreads;
-  } else {
-    smem = Single::smem_bytes(n_prefix);
-    smem_max = Single::smem_bytes(kMaxVarlenSeqs + 1);
-    kern = loza::ssa_prefill_kernel<DQK, DV>;
-    threads = loza::kPrefillThreads;
-  }
+  const size_t smem = Lay::smem_bytes(n_prefix);
+  const size_t smem_max = Lay::smem_bytes(kMaxVarlenSeqs + 1);
+  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, loza::PrefillParams) =
+      loza::ssa_prefill_kernel<DQK, DV>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill)");
   const int grid = items_upper < dev.num_sms ? (int)items_upper : dev.num_sms;
   if (grid < 1) return LOZA_SSA_OK;
-  kern<<<grid, threads, smem, stream>>>(mq, mk, mv, prm);
+  kern<<<grid, loza::kPrefillThreads, smem, stream>>>(mq, mk, mv, prm);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "prefill launch");
   return LOZA_SSA_OK;
 }
@@ -148,14 +135,14 @@ int dispatch_prefill(int d_qk, int d_v, const void* q, const void* k, const void
                      const loza::PrefillParams& prm, uint64_t plane_rows, uint64_t planes,
                      long long items_upper, int n_prefix, cudaStream_t s, const DeviceInfo& dev) {
   if (d_qk == 64 && d_v == 64)
-    return launch_prefill<64, 64, true>(q, k, v, prm, plane_rows, planes, items_upper, n_prefix,
-                                        s, dev);
+    return launch_prefill<64, 64>(q, k, v, prm, plane_rows, planes, items_upper, n_prefix, s,
+                                  dev);
   if (d_qk == 128 && d_v == 128)
-    return launch_prefill<128, 128, true>(q, k, v, prm, plane_rows, planes, items_upper,
-                                          n_prefix, s, dev);
+    return launch_prefill<128, 128>(q, k, v, prm, plane_rows, planes, items_upper, n_prefix, s,
+                                    dev);
   if (d_qk == 192 && d_v == 128)
-    return launch_prefill<192, 128, false>(q, k, v, prm, plane_rows, planes, items_upper,
-                                           n_prefix, s, dev);
+    return launch_prefill<192, 128>(q, k, v, prm, plane_rows, planes, items_upper, n_prefix, s,
+                                    dev);
   return LOZA_SSA_ERR_HEAD_DIM;
 }
 

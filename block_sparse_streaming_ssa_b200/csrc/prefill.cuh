@@ -19,7 +19,7 @@
 // in TMEM by exp2(m_old - m_new) before the next P.V.  The final O = acc / l
 // and LSE = (m + log2 l) ln 2 are exact for any choice of m.
 //
-// Warp roles (352 threads):
+// Warp roles (384 threads):
 //   warps 0-7  softmax + correction + epilogue.  Warp w reads TMEM lanes
 //              32*(w%4)..+31 (a warp may only touch its own lane quarter), so
 //              query row r is shared by thread r of warpgroup 0 (key columns
@@ -28,16 +28,22 @@
 //              halves exchange their row maxima through shared memory once per
 //              tile and their row sums once per item.
 //   warp 8     TMA producer of Q and K (one elected lane)
-//   warp 9     TMEM allocator + MMA issuer (one elected lane)
+//   warp 9     TMEM allocator + issuer of the S = Q K^T MMAs (one elected lane)
 //   warp 10    TMA producer of V (one elected lane)
+//   warp 11    issuer of the O += P V MMAs (one elected lane)
 // K and V have their own producers so a K load never queues behind a V load
-// that is waiting for its ring slot: the MMA consumes K_{j+1} before V_j.
+// that is waiting for its ring slot: S consumes K_{j+1} before P.V reads V_j.
+// S and P.V have their own issuers because one thread issues a tcgen05.mma
+// only every ~100-200 SM cycles (measured on B200): with a single issuer the
+// chain P_j ready -> P_j V_j issued -> S_{j+2} issued sits on the softmax's
+// critical path.
 //
-// TMEM (512 columns x 128 lanes, fp32): S0 = cols [0,128), S1 = [128,256),
-// O buffers from 256 (two of them when 2*DV <= 256, so the next item's first
-// P.V never waits for this item's epilogue).  P_j (bf16 pairs) overwrites the
-// first 64 columns of its S buffer.  S is double-buffered so the tensor core
-// computes S_{j+1} while the softmax warps work on S_j.
+// TMEM (512 columns x 128 lanes, fp32): S buffers [0,128), [128,256),
+// [256,384), O buffers from 384 (two of them when 2*DV <= 128, so the next
+// item's first P.V never waits for this item's epilogue).  P_j (bf16 pairs)
+// overwrites the first 64 columns of its S buffer.  With three S buffers the
+// tensor core computes S_{j+1} and S_{j+2} while the softmax warps work on
+// S_j; S_{j+3} waits until P_j V_j has read buffer j's P.
 //
 // Shared memory (1024-byte aligned, 128B-swizzled TMA boxes of 64 bf16
 // columns x 128 rows = 16 KB "chunks"):  Q ring, K ring, V ring, mbarriers,
@@ -55,11 +61,11 @@ namespace loza {
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P values stay <= 2^8
 
 // Of every 8 exp2 pairs a softmax thread evaluates, this many run as a
-// polynomial on the FMA pipe (exp2_poly_x2) and the rest on the MUFU unit.
-// Measured on B200 the MUFU unit is not the limit of this kernel, so the
-// default keeps every exp2 on MUFU.
+// polynomial on the FMA pipe (exp2_poly_x2) and the rest on the MUFU unit
+// (16 exp2 per clock per SM).  3 of 8 measured fastest on B200 (2 and 4 were
+// slower), once the softmax is what the tile loop waits on.
 #ifndef LOZA_POLY_PAIRS
-#define LOZA_POLY_PAIRS 0
+#define LOZA_POLY_PAIRS 3
 #endif
 constexpr int kPolyPairsPer8 = LOZA_POLY_PAIRS;
 
@@ -88,7 +94,10 @@ struct PrefillLayout {
   static constexpr int QST = DQK <= 128 ? 2 : 1;  // Q ring depth (d_qk=192: no room for 2)
   static constexpr int KST = 2;                   // K ring depth
   static constexpr int VST = 2;                   // V ring depth
-  static constexpr int NOB = 256 + 2 * DV <= 512 ? 2 : 1;  // O buffers in TMEM
+  static constexpr int NSB = 3;                   // S buffers in TMEM (128 columns each)
+  static constexpr int TM_O = NSB * 128;          // O buffers after the S buffers
+  static constexpr int NOB = TM_O + 2 * DV <= 512 ? 2 : 1;  // O buffers in TMEM
+  static_assert(TM_O + DV <= 512, "S buffers and one O buffer must fit in TMEM");
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + QST * Q_BYTES;
   static constexpr int OFF_V = OFF_K + KST * K_BYTES;
@@ -97,19 +106,19 @@ struct PrefillLayout {
   static constexpr int B_Q_FULL = 0, B_Q_EMPTY = B_Q_FULL + QST;
   static constexpr int B_K_FULL = B_Q_EMPTY + QST, B_K_EMPTY = B_K_FULL + KST;
   static constexpr int B_V_FULL = B_K_EMPTY + KST, B_V_EMPTY = B_V_FULL + VST;
-  static constexpr int B_S_FULL = B_V_EMPTY + VST;  // 2
-  static constexpr int B_P_FULL = B_S_FULL + 2;     // 2
-  static constexpr int B_O_DONE = B_P_FULL + 2;
+  static constexpr int B_S_FULL = B_V_EMPTY + VST;  // NSB
+  static constexpr int B_P_FULL = B_S_FULL + NSB;   // NSB
+  static constexpr int B_S_FREE = B_P_FULL + NSB;   // NSB: the buffer's P has been read
+  static constexpr int B_O_DONE = B_S_FREE + NSB;
   static constexpr int B_O_EMPTY = B_O_DONE + 1;    // NOB
-  static constexpr int B_DRAIN = B_O_EMPTY + NOB;
-  static constexpr int B_XCHG = B_DRAIN + 1;  // the two softmax warpgroups' row exchange
+  static constexpr int B_DRAIN = B_O_EMPTY + NOB;   // 2: one per MMA issuer
+  static constexpr int B_XCHG = B_DRAIN + 2;  // the two softmax warpgroups' row exchange
   static constexpr int NBAR = B_XCHG + 1;
   static constexpr int OFF_MISC = OFF_BAR + 256;      // [0] tmem base, [1] abort, [2] items
   static constexpr int OFF_RED = OFF_MISC + 16;       // float [2 buffers][2 halves][128 rows]
   static constexpr int OFF_PREFIX = OFF_RED + 2 * 2 * 128 * 4;
   static_assert(NBAR * 8 <= 256, "barrier area");
   static constexpr int TMEM_COLS = 512;
-  static constexpr int TM_O = 256;
   static constexpr int MIN_SMEM = 120 * 1024;  // keeps one CTA (and one TMEM owner) per SM
   static constexpr size_t smem_bytes(int n_prefix) {
     size_t need = (size_t)OFF_PREFIX + 4 * (size_t)n_prefix + 1024;  // + alignment slack
@@ -189,7 +198,7 @@ __device__ __forceinline__ void prefill_count_items(const PrefillParams& p, int*
   }
 }
 
-constexpr int kPrefillThreads = 352;
+constexpr int kPrefillThreads = 384;
 constexpr int kSoftmaxThreads = 256;
 
 template <int DQK, int DV>
@@ -222,13 +231,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       mbar_init(bar(Lay::B_V_FULL + s), 1);
       mbar_init(bar(Lay::B_V_EMPTY + s), 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < Lay::NSB; ++s) {
       mbar_init(bar(Lay::B_S_FULL + s), 1);
       mbar_init(bar(Lay::B_P_FULL + s), kSoftmaxThreads);
+      mbar_init(bar(Lay::B_S_FREE + s), 1);
     }
     mbar_init(bar(Lay::B_O_DONE), 1);
     for (int s = 0; s < Lay::NOB; ++s) mbar_init(bar(Lay::B_O_EMPTY + s), kSoftmaxThreads);
     mbar_init(bar(Lay::B_DRAIN), 1);
+    mbar_init(bar(Lay::B_DRAIN + 1), 1);
     mbar_init(bar(Lay::B_XCHG), kSoftmaxThreads);
     misc[1] = 0;
     fence_barrier_init();
@@ -334,52 +345,34 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           if (v_issued[s] > 0) mbar_wait_drain(bar(Lay::B_V_FULL + s), (v_issued[s] - 1) & 1);
     }
   } else if (warp == 9) {
-    // ------------------------------------------------------------- MMA
+    // ------------------------------------------------------ MMA issuer: S
+    // One thread issues a tcgen05.mma only every ~100-200 SM cycles, so S and
+    // P.V have an issuer each; with three S buffers the S issuer runs up to
+    // two tiles ahead of the softmax.
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16_f32(128, 128, false);
-      const uint32_t id_o = idesc_bf16_f32(128, DV, true);
-      int g0 = 0, it = 0;
+      int g = 0, it = 0;
       bool ok = true;
-      // O_ob += P_g V_g for tile t (global index g) of the current item
-      auto issue_pv = [&](int g, int t, int ob) -> bool {
-        const int st = g % Lay::VST;
-        if (!mbar_wait(bar(Lay::B_P_FULL + (g & 1)), (g >> 1) & 1, abort_flag, status, 1))
-          return false;
-        if (!mbar_wait(bar(Lay::B_V_FULL + st), (g / Lay::VST) & 1, abort_flag, status, 1))
-          return false;
-        if (t == 0 && it >= Lay::NOB &&
-            !mbar_wait(bar(Lay::B_O_EMPTY + ob), (it / Lay::NOB - 1) & 1, abort_flag, status, 1))
-          return false;
-        tc_fence_after();
-        const uint32_t p_tmem = tmem + (uint32_t)((g & 1) * 128);
-        const uint32_t o_tmem = tmem + Lay::TM_O + ob * DV;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bdesc = sdesc_sw128(
-              sb + Lay::OFF_V + st * Lay::V_BYTES + kk * 2048, Lay::CHUNK, 1024);
-          mma_ts(o_tmem, p_tmem + kk * 8, bdesc, id_o, (t > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(bar(Lay::B_O_DONE));
-        mma_commit(bar(Lay::B_V_EMPTY + st));
-        return true;
-      };
       for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++it) {
         const WorkItem w = decode_item(item, p, prefix);
         const TileRange tr = tile_range(w.qb, p.n_sink, p.n_local);
-        const int qs = it % Lay::QST, ob = it % Lay::NOB;
+        const int qs = it % Lay::QST;
         const uint32_t q_base = sb + Lay::OFF_Q + qs * Lay::Q_BYTES;
         if (!mbar_wait(bar(Lay::B_Q_FULL + qs), (it / Lay::QST) & 1, abort_flag, status, 1)) {
           ok = false;
           break;
         }
-        for (int t = 0; t < tr.count; ++t) {
-          const int g = g0 + t, st = g % Lay::KST;
-          if (!mbar_wait(bar(Lay::B_K_FULL + st), (g / Lay::KST) & 1, abort_flag, status, 1)) {
+        for (int t = 0; t < tr.count; ++t, ++g) {
+          const int st = g % Lay::KST, sbuf = g % Lay::NSB;
+          // S buffer sbuf last held P_{g-NSB}: wait until its P.V has read it
+          if (!mbar_wait(bar(Lay::B_K_FULL + st), (g / Lay::KST) & 1, abort_flag, status, 1) ||
+              (g >= Lay::NSB && !mbar_wait(bar(Lay::B_S_FREE + sbuf), (g / Lay::NSB - 1) & 1,
+                                           abort_flag, status, 1))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t s_tmem = tmem + (uint32_t)((g & 1) * 128);
+          const uint32_t s_tmem = tmem + (uint32_t)(sbuf * 128);
 #pragma unroll
           for (int kk = 0; kk < DQK / 16; ++kk) {
             const uint32_t koff = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
@@ -387,23 +380,52 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             const uint64_t bdesc = sdesc_sw128(sb + Lay::OFF_K + st * Lay::K_BYTES + koff, 16, 1024);
             mma_ss(s_tmem, adesc, bdesc, id_s, kk > 0 ? 1u : 0u);
           }
-          mma_commit(bar(Lay::B_S_FULL + (g & 1)));
+          mma_commit(bar(Lay::B_S_FULL + sbuf));
           mma_commit(bar(Lay::B_K_EMPTY + st));
           if (t == tr.count - 1) mma_commit(bar(Lay::B_Q_EMPTY + qs));
-          if (t > 0 && !issue_pv(g - 1, t - 1, ob)) {
-            ok = false;
-            break;
-          }
         }
-        if (!ok || !issue_pv(g0 + tr.count - 1, tr.count - 1, ob)) {
-          ok = false;
-          break;
-        }
-        g0 += tr.count;
       }
       // every tcgen05.mma issued above has finished before TMEM is released
       mma_commit(bar(Lay::B_DRAIN));
       mbar_wait_drain(bar(Lay::B_DRAIN), 0);
+    }
+  } else if (warp == 11) {
+    // ---------------------------------------------------- MMA issuer: P.V
+    if (lane == 0) {
+      const uint32_t id_o = idesc_bf16_f32(128, DV, true);
+      int g = 0, it = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++it) {
+        const WorkItem w = decode_item(item, p, prefix);
+        const TileRange tr = tile_range(w.qb, p.n_sink, p.n_local);
+        const int ob = it % Lay::NOB;
+        const uint32_t o_tmem = tmem + Lay::TM_O + ob * DV;
+        for (int t = 0; t < tr.count; ++t, ++g) {
+          // O_ob += P_g V_g
+          const int st = g % Lay::VST, sbuf = g % Lay::NSB;
+          if (!mbar_wait(bar(Lay::B_P_FULL + sbuf), (g / Lay::NSB) & 1, abort_flag, status, 1) ||
+              !mbar_wait(bar(Lay::B_V_FULL + st), (g / Lay::VST) & 1, abort_flag, status, 1) ||
+              (t == 0 && it >= Lay::NOB &&
+               !mbar_wait(bar(Lay::B_O_EMPTY + ob), (it / Lay::NOB - 1) & 1, abort_flag, status,
+                          1))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t p_tmem = tmem + (uint32_t)(sbuf * 128);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t bdesc = sdesc_sw128(
+                sb + Lay::OFF_V + st * Lay::V_BYTES + kk * 2048, Lay::CHUNK, 1024);
+            mma_ts(o_tmem, p_tmem + kk * 8, bdesc, id_o, (t > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(Lay::B_O_DONE));
+          mma_commit(bar(Lay::B_V_EMPTY + st));
+          mma_commit(bar(Lay::B_S_FREE + sbuf));
+        }
+      }
+      mma_commit(bar(Lay::B_DRAIN + 1));
+      mbar_wait_drain(bar(Lay::B_DRAIN + 1), 0);
     }
   } else {
     // -------------------------------------------- softmax / correction / epilogue
@@ -426,6 +448,54 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       ++xc;
       return okx;
     };
+    // The epilogue of an item runs after the next item's first tile has been
+    // handed to the P.V issuer: by then the item's last P.V has finished, so
+    // the wait for it is off the softmax's path.
+    struct Done {
+      WorkItem w;
+      float m, l;  // running max (log2 units) and this half's row sum
+      int ob, gl;  // O buffer, global index of the item's last tile
+    };
+    Done prev{};
+    bool have_prev = false;
+    auto epilogue = [&](const Done& d) -> bool {
+      // O = acc / l (bf16), LSE = (m + log2 l) ln 2
+      float l_other;
+      if (!exchange(d.l, l_other)) return false;
+      const float l_row = d.l + l_other;
+      if (!mbar_wait(bar(Lay::B_O_DONE), d.gl & 1, abort_flag, status, 1)) return false;
+      tc_fence_after();
+      const uint32_t o_tmem = tmem + lane_base + Lay::TM_O + d.ob * DV + wg * OH;
+      const int r_in_seq = d.w.qb * 128 + row;
+      const bool valid = r_in_seq < d.w.len;
+      const size_t orow =
+          (size_t)d.w.z * (size_t)p.plane_rows + (size_t)(d.w.seq_start + r_in_seq);
+      const float inv_l = 1.f / l_row;
+      uint32_t orr[OH / 32][32];
+#pragma unroll
+      for (int ch = 0; ch < OH / 32; ++ch) tmem_ld32(o_tmem + ch * 32, orr[ch]);
+      tmem_wait_ld();
+      // O buffer free for the item NOB after this one
+      tc_fence_before();
+      mbar_arrive(bar(Lay::B_O_EMPTY + d.ob));
+      if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(p.o + orow * DV + wg * OH);
+#pragma unroll
+        for (int ch = 0; ch < OH / 32; ++ch)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint32_t* r8 = &orr[ch][8 * v];
+            uint4 pkt;
+            pkt.x = pack_bf16x2(__uint_as_float(r8[0]) * inv_l, __uint_as_float(r8[1]) * inv_l);
+            pkt.y = pack_bf16x2(__uint_as_float(r8[2]) * inv_l, __uint_as_float(r8[3]) * inv_l);
+            pkt.z = pack_bf16x2(__uint_as_float(r8[4]) * inv_l, __uint_as_float(r8[5]) * inv_l);
+            pkt.w = pack_bf16x2(__uint_as_float(r8[6]) * inv_l, __uint_as_float(r8[7]) * inv_l);
+            dst[ch * 4 + v] = pkt;
+          }
+        if (wg == 0) p.lse[orow] = (d.m + __log2f(l_row)) * kLn2;
+      }
+      return true;
+    };
     for (int item = blockIdx.x; item < total_items; item += gridDim.x, ++it) {
       const WorkItem w = decode_item(item, p, prefix);
       const TileRange tr = tile_range(w.qb, p.n_sink, p.n_local);
@@ -435,8 +505,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       bool ok = true;
       for (int t = 0; t < tr.count; ++t) {
         const int g = g0 + t;
-        const uint32_t s_tmem = tmem + lane_base + (uint32_t)((g & 1) * 128);
-        if (!mbar_wait(bar(Lay::B_S_FULL + (g & 1)), (g >> 1) & 1, abort_flag, status, 1)) {
+        const int sbuf = g % Lay::NSB;
+        const uint32_t s_tmem = tmem + lane_base + (uint32_t)(sbuf * 128);
+        if (!mbar_wait(bar(Lay::B_S_FULL + sbuf), (g / Lay::NSB) & 1, abort_flag, status, 1)) {
           ok = false;
           break;
         }
@@ -531,45 +602,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         m = m_use;
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(Lay::B_P_FULL + (g & 1)));
+        mbar_arrive(bar(Lay::B_P_FULL + sbuf));
+        if (t == 0 && have_prev) {
+          have_prev = false;
+          if (!epilogue(prev)) {
+            ok = false;
+            break;
+          }
+        }
       }
       if (!ok) break;
-      // epilogue: O = acc / l (bf16), LSE = (m + log2 l) ln 2
-      float l_other;
-      if (!exchange(l, l_other)) break;
-      const float l_row = l + l_other;
-      const int gl = g0 + tr.count - 1;
-      if (!mbar_wait(bar(Lay::B_O_DONE), gl & 1, abort_flag, status, 1)) break;
-      tc_fence_after();
-      const int r_in_seq = w.qb * 128 + row;
-      const bool valid = r_in_seq < w.len;
-      const size_t orow = (size_t)w.z * (size_t)p.plane_rows + (size_t)(w.seq_start + r_in_seq);
-      const float inv_l = 1.f / l_row;
-      uint32_t orr[OH / 32][32];
-#pragma unroll
-      for (int ch = 0; ch < OH / 32; ++ch) tmem_ld32(o_tmem + ch * 32, orr[ch]);
-      tmem_wait_ld();
-      // O buffer free for the item NOB after this one
-      tc_fence_before();
-      mbar_arrive(bar(Lay::B_O_EMPTY + ob));
-      if (valid) {
-        uint4* dst = reinterpret_cast<uint4*>(p.o + orow * DV + wg * OH);
-#pragma unroll
-        for (int ch = 0; ch < OH / 32; ++ch)
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const uint32_t* r8 = &orr[ch][8 * v];
-            uint4 pkt;
-            pkt.x = pack_bf16x2(__uint_as_float(r8[0]) * inv_l, __uint_as_float(r8[1]) * inv_l);
-            pkt.y = pack_bf16x2(__uint_as_float(r8[2]) * inv_l, __uint_as_float(r8[3]) * inv_l);
-            pkt.z = pack_bf16x2(__uint_as_float(r8[4]) * inv_l, __uint_as_float(r8[5]) * inv_l);
-            pkt.w = pack_bf16x2(__uint_as_float(r8[6]) * inv_l, __uint_as_float(r8[7]) * inv_l);
-            dst[ch * 4 + v] = pkt;
-          }
-        if (wg == 0) p.lse[orow] = (m + __log2f(l_row)) * kLn2;
-      }
+      prev = Done{w, m, l, ob, g0 + tr.count - 1};
+      have_prev = true;
       g0 += tr.count;
     }
+    if (have_prev) epilogue(prev);
   }
 
   __syncwarp();
