@@ -480,17 +480,18 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       mbar_arrive(bar(Lay::B_O_EMPTY + d.ob));
       if (valid) {
         uint4* dst = reinterpret_cast<uint4*>(p.o + orow * DV + wg * OH);
+        // 32-byte stores: each writes a whole L2 sector (16-byte stores left
+        // half sectors per instruction and measured ~4-7 % slower overall)
 #pragma unroll
         for (int ch = 0; ch < OH / 32; ++ch)
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const uint32_t* r8 = &orr[ch][8 * v];
-            uint4 pkt;
-            pkt.x = pack_bf16x2(__uint_as_float(r8[0]) * inv_l, __uint_as_float(r8[1]) * inv_l);
-            pkt.y = pack_bf16x2(__uint_as_float(r8[2]) * inv_l, __uint_as_float(r8[3]) * inv_l);
-            pkt.z = pack_bf16x2(__uint_as_float(r8[4]) * inv_l, __uint_as_float(r8[5]) * inv_l);
-            pkt.w = pack_bf16x2(__uint_as_float(r8[6]) * inv_l, __uint_as_float(r8[7]) * inv_l);
-            dst[ch * 4 + v] = pkt;
+          for (int v = 0; v < 4; v += 2) {
+            uint32_t w8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              w8[e] = pack_bf16x2(__uint_as_float(orr[ch][8 * v + 2 * e]) * inv_l,
+                                  __uint_as_float(orr[ch][8 * v + 2 * e + 1]) * inv_l);
+            st_global_v8(dst + ch * 4 + v, w8);
           }
         if (wg == 0) p.lse[orow] = (d.m + __log2f(l_row)) * kLn2;
       }

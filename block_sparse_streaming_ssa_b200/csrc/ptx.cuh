@@ -343,6 +343,14 @@ __device__ __forceinline__ void exp2_poly_x2(float y0, float y1, float& p0, floa
   p1 = __uint_as_float(__float_as_uint(pf1) + (__float_as_uint(t1) << 23));
 }
 
+// 32-byte global store (one full L2 sector per thread); `addr` 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* addr, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(addr),
+               "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]),
+               "r"(w[7])
+               : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   // cvt packs its first source into the upper half.
