@@ -107,11 +107,12 @@ int launch_prefill(const void* q, const void* k, const void* v, loza::PrefillPar
                    uint64_t plane_rows, uint64_t planes, long long items_upper, int n_prefix,
                    cudaStream_t stream, const DeviceInfo& dev) {
   using Lay = loza::PrefillLayout<DQK, DV>;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   int rc;
   if ((rc = make_map(&mq, q, DQK, plane_rows, planes, 3)) != LOZA_SSA_OK) return rc;
   if ((rc = make_map(&mk, k, DQK, plane_rows, planes, 3)) != LOZA_SSA_OK) return rc;
   if ((rc = make_map(&mv, v, DV, plane_rows, planes, 3)) != LOZA_SSA_OK) return rc;
+  if ((rc = make_map(&mo, prm.o, DV, plane_rows, planes, 3)) != LOZA_SSA_OK) return rc;
   if (prm.cu_seqlens == nullptr) {
     const long long nb = (prm.L + 127) / 128;
     items_upper = (long long)planes * nb;
@@ -119,14 +120,14 @@ int launch_prefill(const void* q, const void* k, const void* v, loza::PrefillPar
   }
   const size_t smem = Lay::smem_bytes(n_prefix);
   const size_t smem_max = Lay::smem_bytes(kMaxVarlenSeqs + 1);
-  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, loza::PrefillParams) =
+  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, loza::PrefillParams) =
       loza::ssa_prefill_kernel<DQK, DV>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill)");
   const int grid = items_upper < dev.num_sms ? (int)items_upper : dev.num_sms;
   if (grid < 1) return LOZA_SSA_OK;
-  kern<<<grid, loza::kPrefillThreads, smem, stream>>>(mq, mk, mv, prm);
+  kern<<<grid, loza::kPrefillThreads, smem, stream>>>(mq, mk, mv, mo, prm);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "prefill launch");
   return LOZA_SSA_OK;
 }

@@ -91,7 +91,9 @@ struct PrefillLayout {
   static constexpr int Q_BYTES = KCH * CHUNK;
   static constexpr int K_BYTES = KCH * CHUNK;
   static constexpr int V_BYTES = VCH * CHUNK;
-  static constexpr int QST = DQK <= 128 ? 2 : 1;  // Q ring depth (d_qk=192: no room for 2)
+  // Q ring depth: one stage measured as fast as two (the S issuer runs ahead of
+  // the softmax by two tiles, which covers the next item's Q load)
+  static constexpr int QST = 1;
   static constexpr int KST = 2;                   // K ring depth
   static constexpr int VST = 2;                   // V ring depth
   static constexpr int NSB = 3;                   // S buffers in TMEM (128 columns each)
@@ -101,7 +103,12 @@ struct PrefillLayout {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + QST * Q_BYTES;
   static constexpr int OFF_V = OFF_K + KST * K_BYTES;
-  static constexpr int OFF_BAR = OFF_V + VST * V_BYTES;
+  // d_qk = d_v = 128: O goes out through TMA stores from a staging buffer
+  // (one swizzled [128 rows x 64 columns] box per softmax warpgroup); the
+  // other head dims write O from registers.
+  static constexpr bool TMA_OUT = DQK == 128 && DV == 128;
+  static constexpr int OFF_OST = OFF_V + VST * V_BYTES;
+  static constexpr int OFF_BAR = OFF_OST + (TMA_OUT ? VCH * CHUNK : 0);
   // barrier indices
   static constexpr int B_Q_FULL = 0, B_Q_EMPTY = B_Q_FULL + QST;
   static constexpr int B_K_FULL = B_Q_EMPTY + QST, B_K_EMPTY = B_K_FULL + KST;
@@ -113,7 +120,9 @@ struct PrefillLayout {
   static constexpr int B_O_EMPTY = B_O_DONE + 1;    // NOB
   static constexpr int B_DRAIN = B_O_EMPTY + NOB;   // 2: one per MMA issuer
   static constexpr int B_XCHG = B_DRAIN + 2;  // the two softmax warpgroups' row exchange
-  static constexpr int NBAR = B_XCHG + 1;
+  static constexpr int B_OST_FULL = B_XCHG + 1;     // 2, per warpgroup: box written (128)
+  static constexpr int B_OST_FREE = B_OST_FULL + 2; // 2, per warpgroup: box read by its store
+  static constexpr int NBAR = B_OST_FREE + 2;
   static constexpr int OFF_MISC = OFF_BAR + 256;      // [0] tmem base, [1] abort, [2] items
   static constexpr int OFF_RED = OFF_MISC + 16;       // float [2 buffers][2 halves][128 rows]
   static constexpr int OFF_PREFIX = OFF_RED + 2 * 2 * 128 * 4;
@@ -205,7 +214,8 @@ template <int DQK, int DV>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     ssa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
+                       const __grid_constant__ CUtensorMap tm_v,
+                       const __grid_constant__ CUtensorMap tm_o, const PrefillParams p) {
   using Lay = PrefillLayout<DQK, DV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -241,6 +251,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     mbar_init(bar(Lay::B_DRAIN), 1);
     mbar_init(bar(Lay::B_DRAIN + 1), 1);
     mbar_init(bar(Lay::B_XCHG), kSoftmaxThreads);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(bar(Lay::B_OST_FULL + w), kSoftmaxThreads / 2);
+      mbar_init(bar(Lay::B_OST_FREE + w), 1);
+    }
     misc[1] = 0;
     fence_barrier_init();
   }
@@ -249,7 +263,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_k);
   }
-  if (warp == 10 && lane == 0) prefetch_tensormap(&tm_v);
+  if (warp == 10 && lane == 0) {
+    prefetch_tensormap(&tm_v);
+    if (Lay::TMA_OUT) prefetch_tensormap(&tm_o);
+  }
   if (warp == 9) {
     tmem_alloc(sb + Lay::OFF_MISC, Lay::TMEM_COLS);
     tmem_relinquish();
@@ -458,6 +475,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     };
     Done prev{};
     bool have_prev = false;
+    int n_out = 0;  // TMA-store epilogues this warpgroup has done
     auto epilogue = [&](const Done& d) -> bool {
       // O = acc / l (bf16), LSE = (m + log2 l) ln 2
       float l_other;
@@ -478,7 +496,44 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       // O buffer free for the item NOB after this one
       tc_fence_before();
       mbar_arrive(bar(Lay::B_O_EMPTY + d.ob));
-      if (valid) {
+      // Dense rows past L fall outside the tensor map and are not written; a
+      // packed sequence's last block would spill into the next sequence, so
+      // it keeps the register path.
+      const bool tma_out =
+          Lay::TMA_OUT && (p.cu_seqlens == nullptr || (d.w.qb + 1) * 128 <= d.w.len);
+      if (tma_out) {
+        const uint32_t box = sb + Lay::OFF_OST + wg * Lay::CHUNK;
+        if (n_out > 0) {
+          // the box's previous store has read it (its issuer checks, then tells the rest)
+          if (row == 0) {
+            tma_store_wait_read();
+            mbar_arrive(bar(Lay::B_OST_FREE + wg));
+          }
+          if (!mbar_wait(bar(Lay::B_OST_FREE + wg), (n_out - 1) & 1, abort_flag, status, 1))
+            return false;
+        }
+        // row `row` of the box in the 128B-swizzled layout the tensor map reads:
+        // 16-byte unit j at j ^ (row & 7)
+        uint8_t* rowp = smem + Lay::OFF_OST + wg * Lay::CHUNK + row * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t* r8 = &orr[j >> 2][(j & 3) * 8];
+          *reinterpret_cast<uint4*>(rowp + ((j ^ (row & 7)) << 4)) =
+              make_uint4(pack_bf16x2(__uint_as_float(r8[0]) * inv_l, __uint_as_float(r8[1]) * inv_l),
+                         pack_bf16x2(__uint_as_float(r8[2]) * inv_l, __uint_as_float(r8[3]) * inv_l),
+                         pack_bf16x2(__uint_as_float(r8[4]) * inv_l, __uint_as_float(r8[5]) * inv_l),
+                         pack_bf16x2(__uint_as_float(r8[6]) * inv_l, __uint_as_float(r8[7]) * inv_l));
+        }
+        fence_async_shared();
+        mbar_arrive(bar(Lay::B_OST_FULL + wg));
+        if (row == 0) {
+          if (!mbar_wait(bar(Lay::B_OST_FULL + wg), n_out & 1, abort_flag, status, 1)) return false;
+          tma_store_3d(&tm_o, box, wg * 64, d.w.seq_start + d.w.qb * 128, d.w.z);
+          tma_store_commit();
+        }
+        ++n_out;
+        if (valid && wg == 0) p.lse[orow] = (d.m + __log2f(l_row)) * kLn2;
+      } else if (valid) {
         uint4* dst = reinterpret_cast<uint4*>(p.o + orow * DV + wg * OH);
         // 32-byte stores: each writes a whole L2 sector (16-byte stores left
         // half sectors per instruction and measured ~4-7 % slower overall)
@@ -618,6 +673,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       g0 += tr.count;
     }
     if (have_prev) epilogue(prev);
+    if (Lay::TMA_OUT && row == 0) tma_store_wait_all();  // stores done before the CTA exits
   }
 
   __syncwarp();
