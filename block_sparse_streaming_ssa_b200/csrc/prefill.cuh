@@ -119,8 +119,10 @@ struct PrefillLayout {
   static constexpr int B_O_DONE = B_S_FREE + NSB;
   static constexpr int B_O_EMPTY = B_O_DONE + 1;    // NOB
   static constexpr int B_DRAIN = B_O_EMPTY + NOB;   // 2: one per MMA issuer
-  static constexpr int B_XCHG = B_DRAIN + 2;  // the two softmax warpgroups' row exchange
-  static constexpr int B_OST_FULL = B_XCHG + 1;     // 2, per warpgroup: box written (128)
+  // the two softmax warpgroups' row exchange: one barrier per TMEM lane
+  // quarter, i.e. per pair of warps (w, w + 4) that share rows
+  static constexpr int B_XCHG = B_DRAIN + 2;        // 4
+  static constexpr int B_OST_FULL = B_XCHG + 4;     // 2, per warpgroup: box written (128)
   static constexpr int B_OST_FREE = B_OST_FULL + 2; // 2, per warpgroup: box read by its store
   static constexpr int NBAR = B_OST_FREE + 2;
   static constexpr int OFF_MISC = OFF_BAR + 256;      // [0] tmem base, [1] abort, [2] items
@@ -250,7 +252,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     for (int s = 0; s < Lay::NOB; ++s) mbar_init(bar(Lay::B_O_EMPTY + s), kSoftmaxThreads);
     mbar_init(bar(Lay::B_DRAIN), 1);
     mbar_init(bar(Lay::B_DRAIN + 1), 1);
-    mbar_init(bar(Lay::B_XCHG), kSoftmaxThreads);
+    for (int qd = 0; qd < 4; ++qd) mbar_init(bar(Lay::B_XCHG + qd), 64);
     for (int w = 0; w < 2; ++w) {
       mbar_init(bar(Lay::B_OST_FULL + w), kSoftmaxThreads / 2);
       mbar_init(bar(Lay::B_OST_FREE + w), 1);
@@ -459,8 +461,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     auto exchange = [&](float v, float& other) -> bool {
       float* buf = red + (xc & 1) * 256;
       buf[wg * 128 + row] = v;
-      mbar_arrive(bar(Lay::B_XCHG));
-      const bool okx = mbar_wait(bar(Lay::B_XCHG), xc & 1, abort_flag, status, 1);
+      mbar_arrive(bar(Lay::B_XCHG + (warp & 3)));
+      const bool okx = mbar_wait(bar(Lay::B_XCHG + (warp & 3)), xc & 1, abort_flag, status, 1);
       other = buf[(wg ^ 1) * 128 + row];
       ++xc;
       return okx;
