@@ -115,9 +115,12 @@ struct PrefillLayout {
   static constexpr int B_V_FULL = B_K_EMPTY + KST, B_V_EMPTY = B_V_FULL + VST;
   static constexpr int B_S_FULL = B_V_EMPTY + VST;  // NSB
   static constexpr int B_P_FULL = B_S_FULL + NSB;   // NSB
-  static constexpr int B_S_FREE = B_P_FULL + NSB;   // NSB: the buffer's P has been read
-  static constexpr int B_O_DONE = B_S_FREE + NSB;
-  static constexpr int B_O_EMPTY = B_O_DONE + 1;    // NOB
+  // NSB: committed after P_j V_j, so it also says "O holds P_j V_j": the
+  // softmax waits on it only to rescale O and before the epilogue reads O.
+  // A waiter for tile j is never more than one phase behind (S_{j} was issued
+  // after P_{j-NSB} V_{j-NSB} finished) nor ahead (P_{j+NSB} is not yet written).
+  static constexpr int B_S_FREE = B_P_FULL + NSB;
+  static constexpr int B_O_EMPTY = B_S_FREE + NSB;  // NOB
   static constexpr int B_DRAIN = B_O_EMPTY + NOB;   // 2: one per MMA issuer
   // the two softmax warpgroups' row exchange: one barrier per TMEM lane
   // quarter, i.e. per pair of warps (w, w + 4) that share rows
@@ -248,7 +251,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       mbar_init(bar(Lay::B_P_FULL + s), kSoftmaxThreads);
       mbar_init(bar(Lay::B_S_FREE + s), 1);
     }
-    mbar_init(bar(Lay::B_O_DONE), 1);
     for (int s = 0; s < Lay::NOB; ++s) mbar_init(bar(Lay::B_O_EMPTY + s), kSoftmaxThreads);
     mbar_init(bar(Lay::B_DRAIN), 1);
     mbar_init(bar(Lay::B_DRAIN + 1), 1);
@@ -438,7 +440,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 sb + Lay::OFF_V + st * Lay::V_BYTES + kk * 2048, Lay::CHUNK, 1024);
             mma_ts(o_tmem, p_tmem + kk * 8, bdesc, id_o, (t > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(bar(Lay::B_O_DONE));
           mma_commit(bar(Lay::B_V_EMPTY + st));
           mma_commit(bar(Lay::B_S_FREE + sbuf));
         }
@@ -483,7 +484,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       float l_other;
       if (!exchange(d.l, l_other)) return false;
       const float l_row = d.l + l_other;
-      if (!mbar_wait(bar(Lay::B_O_DONE), d.gl & 1, abort_flag, status, 1)) return false;
+      if (!mbar_wait(bar(Lay::B_S_FREE + d.gl % Lay::NSB), (d.gl / Lay::NSB) & 1, abort_flag,
+                     status, 1))
+        return false;
       tc_fence_after();
       const uint32_t o_tmem = tmem + lane_base + Lay::TM_O + d.ob * DV + wg * OH;
       const int r_in_seq = d.w.qb * 128 + row;
@@ -635,12 +638,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           rsum = a0 + a1;
         }
         if (!first) {
-          // O must hold P_{g-1} V_{g-1} before it is rescaled or read again
-          if (!mbar_wait(bar(Lay::B_O_DONE), (g - 1) & 1, abort_flag, status, 1)) {
-            ok = false;
-            break;
-          }
           if (rescale) {
+            // O must hold P_{g-1} V_{g-1} before it is rescaled
+            const int gp = g - 1;
+            if (!mbar_wait(bar(Lay::B_S_FREE + gp % Lay::NSB), (gp / Lay::NSB) & 1, abort_flag,
+                           status, 1)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
             const float alpha = ex2_approx(m - m_use);
             l *= alpha;
