@@ -62,10 +62,10 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: P values stay <= 2^8
 
 // Of every 8 exp2 pairs a softmax thread evaluates, this many run as a
 // polynomial on the FMA pipe (exp2_poly_x2) and the rest on the MUFU unit
-// (16 exp2 per clock per SM).  3 of 8 measured fastest on B200 (2 and 4 were
-// slower), once the softmax is what the tile loop waits on.
+// (16 exp2 per clock per SM).  Measured on B200 with the mha workload:
+// 0 -> 0.566 ms, 1 -> 0.558, 2 -> 0.555, 3 -> 0.565, 4 -> 0.608.
 #ifndef LOZA_POLY_PAIRS
-#define LOZA_POLY_PAIRS 3
+#define LOZA_POLY_PAIRS 2
 #endif
 constexpr int kPolyPairsPer8 = LOZA_POLY_PAIRS;
 
