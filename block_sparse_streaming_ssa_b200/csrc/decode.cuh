@@ -481,44 +481,57 @@ __global__ void __launch_bounds__(320, 1)
   }
 }
 
-// Merge: one CTA per (sequence, 8 heads); thread (column group g, head hh)
-// reads 16 bytes per split, so that a warp's reads of one split are four runs
-// of 128 contiguous bytes, four splits' loads in flight at once.  Launched as
-// a programmatic dependent of the split kernel; it waits for the split
+// Merge: one CTA per (sequence, 8 heads); thread (head hh, column group pair
+// gp) merges the 8-column groups gp and gp + 32 of its head, reading 16 bytes
+// of each per split, so that a warp's reads of one group of one split are
+// four runs of 128 contiguous bytes, and all of a thread's loads are in
+// flight at once.  Two groups per thread keep every CTA of the 32-sequence
+// workload resident in one wave (512 threads per CTA at one group each did
+// not fit in the register file and ran a second wave).  Launched as a
+// programmatic dependent of the split kernel; it waits for the split
 // kernel's results before reading.  Splits whose LSE is -inf are empty and
 // contribute nothing (their partial O is never read into the sum).
 constexpr int kMergeHeads = 8;
-constexpr int kMergeThreads = (kDecodeDv / 8) * kMergeHeads;  // 512
+constexpr int kMergeGroups = 2;  // 8-column groups per thread
+constexpr int kMergeThreads = (kDecodeDv / 8 / kMergeGroups) * kMergeHeads;  // 256
 constexpr int kMergeBatch = 4;
 
-__global__ void __launch_bounds__(kMergeThreads)
+// four CTAs per SM: 148 x 4 slots hold the 512 CTAs of the 32-sequence workload
+__global__ void __launch_bounds__(kMergeThreads, 4)
     ssa_decode_merge_kernel(const DecodeParams p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int groups = (p.H_q + kMergeHeads - 1) / kMergeHeads;
-  const int b = blockIdx.x / groups;
-  const int hh = threadIdx.x % kMergeHeads, g = threadIdx.x / kMergeHeads;
-  const int h = (blockIdx.x % groups) * kMergeHeads + hh;
+  const int heads = (p.H_q + kMergeHeads - 1) / kMergeHeads;
+  const int b = blockIdx.x / heads;
+  const int hh = threadIdx.x % kMergeHeads, gp = threadIdx.x / kMergeHeads;
+  const int h = (blockIdx.x % heads) * kMergeHeads + hh;
   if (h >= p.H_q) return;
   const int hg = h >> 7, hr = h & 127;
+  constexpr int kGroupStride = kDecodeDv / 8 / kMergeGroups;  // 32: groups gp, gp + 32
   const size_t cta0 = ((size_t)b * p.HG + hg) * p.n_split;
   const float* lsep = p.lse_part + cta0 * 128 + hr;  // split stride 128
-  const uint4* op = reinterpret_cast<const uint4*>(p.o_part) + (cta0 * 64 + g) * 128 + hr;
+  const uint4* op = reinterpret_cast<const uint4*>(p.o_part) + (cta0 * 64 + gp) * 128 + hr;
   constexpr size_t kSplitStride = 64 * 128;  // uint4 per split
   const int n = p.n_split;
   float lmax = -INFINITY;
   for (int s = 0; s < n; ++s) lmax = fmaxf(lmax, __ldg(lsep + (size_t)s * 128));
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float acc[kMergeGroups][8];
+#pragma unroll
+  for (int q = 0; q < kMergeGroups; ++q)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[q][e] = 0.f;
   float denom = 0.f;
   if (lmax > -INFINITY) {
     for (int s0 = 0; s0 < n; s0 += kMergeBatch) {
       float ls[kMergeBatch];
-      uint4 raw[kMergeBatch];
+      uint4 raw[kMergeBatch][kMergeGroups];
 #pragma unroll
       for (int j = 0; j < kMergeBatch; ++j) {
         ls[j] = -INFINITY;
         if (s0 + j < n) {
           ls[j] = __ldg(lsep + (size_t)(s0 + j) * 128);
-          raw[j] = __ldg(op + (size_t)(s0 + j) * kSplitStride);
+#pragma unroll
+          for (int q = 0; q < kMergeGroups; ++q)
+            raw[j][q] = __ldg(op + (size_t)(s0 + j) * kSplitStride + q * kGroupStride * 128);
         }
       }
 #pragma unroll
@@ -526,24 +539,31 @@ __global__ void __launch_bounds__(kMergeThreads)
         if (ls[j] == -INFINITY) continue;
         const float wgt = __expf(ls[j] - lmax);
         denom += wgt;
-        const __half2* hv = reinterpret_cast<const __half2*>(&raw[j]);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __half22float2(hv[e]);
-          acc[2 * e] += wgt * f.x;
-          acc[2 * e + 1] += wgt * f.y;
+        for (int q = 0; q < kMergeGroups; ++q) {
+          const __half2* hv = reinterpret_cast<const __half2*>(&raw[j][q]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(hv[e]);
+            acc[q][2 * e] += wgt * f.x;
+            acc[q][2 * e + 1] += wgt * f.y;
+          }
         }
       }
     }
   }
   const float inv = denom > 0.f ? 1.f / denom : 0.f;
-  uint4 pk;
-  pk.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-  pk.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-  pk.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
-  pk.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
-  *(reinterpret_cast<uint4*>(p.o + ((size_t)b * p.H_q + h) * kDecodeDv) + g) = pk;
-  if (g == 0) p.lse[(size_t)b * p.H_q + h] = denom > 0.f ? lmax + __logf(denom) : -INFINITY;
+  uint4* orow = reinterpret_cast<uint4*>(p.o + ((size_t)b * p.H_q + h) * kDecodeDv);
+#pragma unroll
+  for (int q = 0; q < kMergeGroups; ++q) {
+    uint4 pk;
+    pk.x = pack_bf16x2(acc[q][0] * inv, acc[q][1] * inv);
+    pk.y = pack_bf16x2(acc[q][2] * inv, acc[q][3] * inv);
+    pk.z = pack_bf16x2(acc[q][4] * inv, acc[q][5] * inv);
+    pk.w = pack_bf16x2(acc[q][6] * inv, acc[q][7] * inv);
+    orow[gp + q * kGroupStride] = pk;
+  }
+  if (gp == 0) p.lse[(size_t)b * p.H_q + h] = denom > 0.f ? lmax + __logf(denom) : -INFINITY;
 }
 
 }  // namespace loza
