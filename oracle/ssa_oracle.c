@@ -117,8 +117,9 @@ int64_t oracle_ssa_key_blocks(int64_t qb, int64_t blk, int64_t seq_len, int64_t 
 static int attend_row(const void* q, int64_t q_off, int q_elt, const void* k, const void* v,
                       int kv_elt, int64_t kv_off_k, int64_t kv_off_v, int64_t k_ld, int64_t v_ld,
                       const int32_t* page_table, int64_t n_pages, int64_t i, int64_t blk,
-                      int64_t n_sink, int64_t n_local, int dqk, int dv, double scale, double* s_buf,
-                      int64_t* j_buf, double* qd, double* o_out, double* lse_out) {
+                      int64_t n_sink, int64_t n_local, const int32_t* extra, int64_t n_extra,
+                      int dqk, int dv, double scale, double* s_buf, int64_t* j_buf, double* qd,
+                      double* o_out, double* lse_out) {
   for (int c = 0; c < dqk; ++c) qd[c] = widen(q, q_off + c, q_elt);
 
   /* pass 1: every score over J(i), and the row max */
@@ -126,7 +127,10 @@ static int attend_row(const void* q, int64_t q_off, int q_elt, const void* k, co
   double m = -INFINITY;
   int64_t qb = i / blk;
   for (int64_t kb = 0; kb <= qb; ++kb) {
-    if (!oracle_ssa_block_in_window(qb, kb, n_sink, n_local)) continue;
+    /* block kb is attended if it is in the SSA window or in the extra list */
+    int in = oracle_ssa_block_in_window(qb, kb, n_sink, n_local);
+    for (int64_t e = 0; e < n_extra && !in; ++e) in = (extra[e] == kb);
+    if (!in) continue;
     int64_t j_end = (kb + 1) * blk - 1;
     if (j_end > i) j_end = i;
     for (int64_t j = kb * blk; j <= j_end; ++j) {
@@ -191,7 +195,7 @@ int oracle_ssa_prefill_rows(const void* q, const void* k, const void* v, int elt
       }
       int64_t bh = flat / L, i = flat % L;
       int rc = attend_row(q, flat * dqk, elt, k, v, elt, bh * L * dqk, bh * L * dv, dqk, dv, NULL,
-                          0, i, blk, n_sink, n_local, dqk, dv, scale, s_buf, j_buf, qd,
+                          0, i, blk, n_sink, n_local, NULL, 0, dqk, dv, scale, s_buf, j_buf, qd,
                           o + r * dv, lse + r);
       if (rc) {
 #pragma omp atomic write
@@ -243,8 +247,8 @@ int oracle_ssa_prefill_varlen_rows(const void* q, const void* k, const void* v, 
       int64_t start = cu_seqlens[s];
       int64_t i = tok - start;
       int rc = attend_row(q, flat * dqk, elt, k, v, elt, (h * total + start) * dqk,
-                          (h * total + start) * dv, dqk, dv, NULL, 0, i, blk, n_sink, n_local, dqk,
-                          dv, scale, s_buf, j_buf, qd, o + r * dv, lse + r);
+                          (h * total + start) * dv, dqk, dv, NULL, 0, i, blk, n_sink, n_local,
+                          NULL, 0, dqk, dv, scale, s_buf, j_buf, qd, o + r * dv, lse + r);
       if (rc) {
 #pragma omp atomic write
         err = rc;
@@ -264,17 +268,18 @@ int oracle_ssa_prefill_varlen_rows(const void* q, const void* k, const void* v, 
  * rows are flat r = b*Hq + h; o: [n_rows, dv]; lse: [n_rows].
  * Returns -1 for a page id outside [0, n_pages), -4 for a bad seq_len.
  */
-int oracle_ssa_decode_rows(const void* q, const void* kv, int elt, const int32_t* page_table,
-                           const int32_t* seq_lens, int64_t B, int64_t Hq, int dqk, int dv,
-                           int64_t page_size, int64_t max_pages, int64_t n_pages, int64_t n_sink,
-                           int64_t n_local, double scale, const int64_t* rows, int64_t n_rows,
-                           double* o, double* lse) {
+static int decode_rows(const void* q, const void* kv, int elt, const int32_t* page_table,
+                       const int32_t* seq_lens, const int32_t* extra_pages, int64_t max_extra,
+                       int64_t B, int64_t Hq, int dqk, int dv, int64_t page_size,
+                       int64_t max_pages, int64_t n_pages, int64_t n_sink, int64_t n_local,
+                       double scale, const int64_t* rows, int64_t n_rows, double* o,
+                       double* lse) {
   int64_t longest = 1;
   for (int64_t b = 0; b < B; ++b) {
     if (seq_lens[b] < 1 || seq_lens[b] > max_pages * page_size) return -4;
     if (seq_lens[b] > longest) longest = seq_lens[b];
   }
-  int64_t cap = max_keys(longest, page_size, n_sink, n_local);
+  int64_t cap = max_keys(longest, page_size, n_sink + max_extra, n_local);
   int err = 0;
 #pragma omp parallel
   {
@@ -292,8 +297,9 @@ int oracle_ssa_decode_rows(const void* q, const void* kv, int elt, const int32_t
       int64_t b = flat / Hq;
       int64_t t = (int64_t)seq_lens[b] - 1;
       int rc = attend_row(q, flat * dqk, elt, kv, kv, elt, 0, 0, dqk, dqk,
-                          page_table + b * max_pages, n_pages, t, page_size, n_sink, n_local, dqk,
-                          dv, scale, s_buf, j_buf, qd, o + r * dv, lse + r);
+                          page_table + b * max_pages, n_pages, t, page_size, n_sink, n_local,
+                          extra_pages ? extra_pages + b * max_extra : NULL, max_extra, dqk, dv,
+                          scale, s_buf, j_buf, qd, o + r * dv, lse + r);
       if (rc) {
 #pragma omp atomic write
         err = rc;
@@ -304,6 +310,34 @@ int oracle_ssa_decode_rows(const void* q, const void* kv, int elt, const int32_t
     free(qd);
   }
   return err;
+}
+
+int oracle_ssa_decode_rows(const void* q, const void* kv, int elt, const int32_t* page_table,
+                           const int32_t* seq_lens, int64_t B, int64_t Hq, int dqk, int dv,
+                           int64_t page_size, int64_t max_pages, int64_t n_pages, int64_t n_sink,
+                           int64_t n_local, double scale, const int64_t* rows, int64_t n_rows,
+                           double* o, double* lse) {
+  return decode_rows(q, kv, elt, page_table, seq_lens, NULL, 0, B, Hq, dqk, dv, page_size,
+                     max_pages, n_pages, n_sink, n_local, scale, rows, n_rows, o, lse);
+}
+
+/*
+ * Decode over the SSA window plus selected pages: the fixed sink + sliding
+ * window budget plus pages chosen per sequence by a page-level indexer
+ * (LongCat sparse-attention article, 机制 1 流感知索引 and 机制 3 分层索引,
+ * pages of P = 128 tokens).  extra_pages: [B, max_extra] logical page ids
+ * of each sequence; any entry that is negative, past the query's page, or
+ * already in the window adds nothing, and a page listed twice counts once:
+ * the keys are J(t) = { j <= t : page(j) in W(page(t)) or page(j) listed }.
+ */
+int oracle_ssa_decode_sel_rows(const void* q, const void* kv, int elt, const int32_t* page_table,
+                               const int32_t* seq_lens, const int32_t* extra_pages,
+                               int64_t max_extra, int64_t B, int64_t Hq, int dqk, int dv,
+                               int64_t page_size, int64_t max_pages, int64_t n_pages,
+                               int64_t n_sink, int64_t n_local, double scale, const int64_t* rows,
+                               int64_t n_rows, double* o, double* lse) {
+  return decode_rows(q, kv, elt, page_table, seq_lens, extra_pages, max_extra, B, Hq, dqk, dv,
+                     page_size, max_pages, n_pages, n_sink, n_local, scale, rows, n_rows, o, lse);
 }
 
 /* Threads the oracle's parallel regions use (for reporting the CPU baseline). */

@@ -76,6 +76,10 @@ def _load():
         lib.oracle_ssa_decode_rows.argtypes = [
             vp, vp, i32, vp, vp, i64, i64, i32, i32, i64, i64, i64, i64, i64, dbl, vp, i64, vp, vp]
         lib.oracle_ssa_decode_rows.restype = i32
+        lib.oracle_ssa_decode_sel_rows.argtypes = [
+            vp, vp, i32, vp, vp, vp, i64, i64, i64, i32, i32, i64, i64, i64, i64, i64, ctypes.c_double,
+            vp, i64, vp, vp]
+        lib.oracle_ssa_decode_sel_rows.restype = i32
         lib.oracle_ssa_num_threads.argtypes = []
         lib.oracle_ssa_num_threads.restype = i32
         _lib = lib
@@ -204,6 +208,43 @@ def decode(q, kv, page_table, seq_lens, dv, page_size=128, n_sink=1, n_local=7, 
     return o, lse
 
 
+def decode_selected(q, kv, page_table, seq_lens, extra_pages, dv, page_size=128, n_sink=1,
+                    n_local=7, scale=None, rows=None):
+    """Paged decode over the SSA window plus selected pages (LongCat
+    sparse-attention article, 机制 1 and 机制 3: a fixed sink + sliding-window
+    budget plus pages of P = 128 tokens chosen by a page-level indexer).
+    extra_pages: [B, max_extra] int32 logical page ids per sequence; an entry
+    that is negative, past the query's page or already in the window adds
+    nothing, and a page listed twice counts once.  Other arguments as decode().
+    """
+    q = np.ascontiguousarray(q)
+    kv = np.ascontiguousarray(kv)
+    pt = np.ascontiguousarray(page_table, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    ex = np.ascontiguousarray(extra_pages, dtype=np.int32)
+    B, Hq, dqk = q.shape
+    assert ex.ndim == 2 and ex.shape[0] == B
+    n_pages = kv.shape[0]
+    assert kv.shape[1] == page_size and kv.shape[2] == dqk
+    elt = _elt(q)
+    assert _elt(kv) == elt
+    if scale is None:
+        scale = 1.0 / np.sqrt(dqk)
+    full = rows is None
+    rows = np.arange(B * Hq, dtype=np.int64) if full else np.ascontiguousarray(rows, dtype=np.int64)
+    o = np.empty((rows.size, dv), dtype=np.float64)
+    lse = np.empty(rows.size, dtype=np.float64)
+    rc = _load().oracle_ssa_decode_sel_rows(
+        _ptr(q), _ptr(kv), elt, _ptr(pt), _ptr(sl), _ptr(ex), ex.shape[1], B, Hq, dqk, dv,
+        page_size, pt.shape[1], n_pages, n_sink, n_local, float(scale), _ptr(rows), rows.size,
+        _ptr(o), _ptr(lse))
+    if rc:
+        raise ValueError(f"oracle decode (selected pages) failed ({rc})")
+    if full:
+        return o.reshape(B, Hq, dv), lse.reshape(B, Hq)
+    return o, lse
+
+
 # ---------------------------------------------------------------------------
 # Independent numpy implementations (tiny inputs only)
 # ---------------------------------------------------------------------------
@@ -268,6 +309,36 @@ def brute_force_decode(q, kv, page_table, seq_lens, dv, page_size=128, n_sink=1,
         s = np.where(allowed[None, :], s, -np.inf)
         smax = s.max(axis=-1, keepdims=True)
         p = np.where(allowed[None, :], np.exp(s - smax), 0.0)
+        den = p.sum(axis=-1, keepdims=True)
+        o[b] = p @ keys[:, :dv] / den
+        lse[b] = smax[:, 0] + np.log(den[:, 0])
+    return o, lse
+
+
+def brute_force_decode_selected(q, kv, page_table, seq_lens, extra_pages, dv, page_size=128,
+                                n_sink=1, n_local=7, scale=None):
+    """Decode over an explicitly built key set: the window's keys (read off the
+    materialised mask) plus every key of each listed page that lies at or
+    before the query, gathered through the page table.  q: [B,Hq,dqk]."""
+    q, kv = _as_f64(q), _as_f64(kv)
+    B, Hq, dqk = q.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(dqk)
+    o = np.zeros((B, Hq, dv))
+    lse = np.zeros((B, Hq))
+    for b in range(B):
+        n = int(seq_lens[b])
+        allowed = mask_matrix(n, page_size, n_sink, n_local)[n - 1].copy()
+        for e in np.asarray(extra_pages[b]):
+            if e >= 0:
+                allowed[e * page_size:(e + 1) * page_size] = True   # keys past n are cut below
+        allowed = allowed[:n]
+        logical = np.nonzero(allowed)[0]
+        phys = np.asarray(page_table[b])[logical // page_size] * page_size + logical % page_size
+        keys = kv.reshape(-1, dqk)[phys]
+        s = scale * q[b] @ keys.T
+        smax = s.max(axis=-1, keepdims=True)
+        p = np.exp(s - smax)
         den = p.sum(axis=-1, keepdims=True)
         o[b] = p @ keys[:, :dv] / den
         lse[b] = smax[:, 0] + np.log(den[:, 0])

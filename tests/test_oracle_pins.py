@@ -305,3 +305,73 @@ def test_decode_rejects_bad_page_id():
     pt[0, 1] = kv.shape[0]          # out of range
     with pytest.raises(ValueError):
         orc.decode(q, kv, pt, sl, dv=16, page_size=8, n_sink=1, n_local=3)
+
+
+# --- decode over the window plus selected pages (LongCat sparse-attention
+# article, 机制 1 / 机制 3: fixed sink + sliding window plus indexer-chosen pages)
+
+def test_decode_selected_matches_brute_force():
+    lens = [1, 9, 61, 100, 100]
+    q, kv, pt, sl = _decode_case(11, lens)
+    # per sequence: chosen pages with negatives, duplicates, pages already in
+    # the window, pages past the query's page
+    extra = np.array([[-1, -1, -1, -1, -1],
+                      [0, 0, 1, -1, 5],
+                      [2, 2, 3, 7, -4],
+                      [1, 4, 4, 11, 12],
+                      [3, -1, 6, 2, 9]], np.int32)
+    o, lse = orc.decode_selected(q, kv, pt, sl, extra, dv=16, page_size=8, n_sink=1, n_local=3,
+                                 scale=0.3)
+    o_bf, lse_bf = orc.brute_force_decode_selected(q, kv, pt, sl, extra, dv=16, page_size=8,
+                                                   n_sink=1, n_local=3, scale=0.3)
+    np.testing.assert_allclose(o, o_bf, atol=1e-11)
+    np.testing.assert_allclose(lse, lse_bf, atol=1e-11)
+
+
+def test_decode_selected_with_every_page_is_causal_attention():
+    """Listing every page between the sinks and the window turns the key set
+    into all keys j <= t: textbook causal attention of the last row."""
+    lens = [77, 40]
+    q, kv, pt, sl = _decode_case(12, lens, Hq=3)
+    extra = np.full((2, 10), -1, np.int32)
+    for b, n in enumerate(lens):
+        pages = list(range(-(-n // 8)))
+        extra[b, :len(pages)] = pages
+    o, lse = orc.decode_selected(q, kv, pt, sl, extra, dv=16, page_size=8, n_sink=1, n_local=2,
+                                 scale=0.25)
+    for b, n in enumerate(lens):
+        logical = np.arange(n)
+        rows = kv.reshape(-1, kv.shape[-1])[pt[b][logical // 8] * 8 + logical % 8]
+        for h in range(3):
+            qq = np.zeros((n, rows.shape[1]))
+            qq[n - 1] = q[b, h]
+            ref_o, ref_lse = orc.causal_attention(qq, rows, rows[:, :16], scale=0.25)
+            np.testing.assert_allclose(o[b, h], ref_o[-1], atol=1e-12)
+            np.testing.assert_allclose(lse[b, h], ref_lse[-1], atol=1e-12)
+
+
+def test_decode_selected_key_count():
+    """q = 0: LSE = ln |J(t)|, with |J(t)| counted from the definition: the
+    window's keys plus 8 keys for every distinct listed page strictly between
+    the sinks and the window."""
+    lens = [100, 61]
+    q, kv, pt, sl = _decode_case(13, lens)
+    q[:] = 0.0
+    extra = np.array([[2, 2, 5, 11, -1, 12], [1, 3, 3, 0, 6, 7]], np.int32)
+    o, lse = orc.decode_selected(q, kv, pt, sl, extra, dv=16, page_size=8, n_sink=1, n_local=3)
+    for b, n in enumerate(lens):
+        t = n - 1
+        qb = t // 8
+        lo = max(1, qb - 3 + 1)                       # first local page (n_sink = 1, n_local = 3)
+        window = min(t + 1, 8) + sum(min(8, t - 8 * p + 1) for p in range(lo, qb + 1) if p >= 1)
+        chosen = {int(e) for e in extra[b] if 1 <= e < lo}
+        np.testing.assert_allclose(lse[b], np.log(window + 8 * len(chosen)), atol=1e-12)
+
+
+def test_decode_selected_without_pages_is_decode():
+    q, kv, pt, sl = _decode_case(14, [33, 90])
+    extra = np.full((2, 4), -1, np.int32)
+    a = orc.decode_selected(q, kv, pt, sl, extra, dv=16, page_size=8, n_sink=1, n_local=3)
+    b = orc.decode(q, kv, pt, sl, dv=16, page_size=8, n_sink=1, n_local=3)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
