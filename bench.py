@@ -3,14 +3,16 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--config mha|tiny|mla|varlen] [--no-decode] [--no-prefill]
-                    [--no-cpu-baseline]
+                    [--no-cpu-baseline] [--decode-extra N]
 
 One JSON line on rank 0.  A step is one SSA prefill call over the chosen
 workload (default: B=1, H=32, L=32768, d=128, 1 sink + 7 local blocks of 128);
 ``value`` is useful TFLOP/s = 2 (d_qk + d_v) * (number of unmasked (i, j)
 pairs) per step / device time, summed over ranks.  The same run also times the
 paged decode workload (32 sequences, 128 heads, 576/512, random page table over
-a ~20 GB pool) and reports it under ``decode`` in GB/s of algorithmic bytes.
+a ~20 GB pool) and reports it under ``decode`` in GB/s of algorithmic bytes,
+and the same decode with 8 distinct selected pages per sequence on top of the
+window under ``decode_selected`` (``--decode-extra``).
 
 Under torchrun every rank runs its own replica of the workload (weak scaling,
 no collective on the data path; NCCL only reduces the timing).
@@ -273,26 +275,53 @@ def e2e_prefill(w, steps):
 
 # ----------------------------------------------------------------- decode
 
-def decode_bench(iters, warmup, peaks, seed=0, len_hi=None, n_sets=8, world=1):
+def decode_extra_pages(lens, n_extra, seed, n_sink=1, n_local=7, blk=128):
+    """Per sequence, ``n_extra`` distinct logical pages drawn uniformly from the
+    pages between the sink and the local run (fewer when there are not that
+    many); -1 pads.  Returns the [B, n_extra] int32 list and the keys it adds."""
+    rng = np.random.default_rng(2000 + seed)
+    ex = np.full((len(lens), n_extra), -1, np.int32)
+    added = 0
+    for b, n in enumerate(lens):
+        qb = (n - 1) // blk
+        lo = max(n_sink, qb - n_local + 1)
+        pool = np.arange(n_sink, lo)
+        pick = rng.choice(pool, size=min(n_extra, pool.size), replace=False)
+        ex[b, :pick.size] = pick
+        added += pick.size * blk
+    return ex, added
+
+
+def decode_bench(iters, warmup, peaks, seed=0, len_hi=None, n_sets=8, world=1, n_extra=0):
     """Paged decode through the public call.  ``value``: algorithmic bytes per
     call / device time per call, with the calls captured in a CUDA graph (the
     way a serving loop issues decode steps) and rotating over ``n_sets``
     batches that share the page pool but read different pages (own page
     table and queries each), so that consecutive calls find nothing of their
-    inputs in L2.  ``eager_flush_us``: one eager call per step after a 2x L2
+    inputs in L2.  ``n_extra`` > 0: the selected-pages decode, each sequence
+    also attending ``n_extra`` distinct pages chosen between its sink and its
+    local run.  ``eager_flush_us``: one eager call per step after a 2x L2
     write, for comparison (it also pays the write-back of the flushed lines
     and, when the GPU runs dry, the host-side cost of the call)."""
     import torch
     from block_sparse_streaming_ssa_b200 import synth
-    from block_sparse_streaming_ssa_b200.loza_ssa import (loza_ssa_decode,
-                                                          loza_ssa_decode_workspace_size)
+    from block_sparse_streaming_ssa_b200.loza_ssa import (loza_ssa_decode, loza_ssa_decode_selected,
+                                                          loza_ssa_decode_selected_workspace_size)
     s = synth.DECODE
     lens = synth.decode_seq_lens(seed, s.B, s.len_lo, len_hi or s.len_hi)
     q, kv, pt, sl = synth.decode_inputs(lens, s.H_q, s.d_qk, seed=seed, device="cuda")
-    ws = torch.empty(loza_ssa_decode_workspace_size(s.B, s.H_q, s.d_v), dtype=torch.uint8,
-                     device="cuda")
-    o, lse = loza_ssa_decode(q, kv, pt, sl, s.d_v, scale=s.scale, workspace=ws)
-    keys = int(sum(row_pairs(np.array([n - 1]))[0] for n in lens))
+    ex_h, extra_keys = decode_extra_pages(lens, n_extra, seed)
+    extra = torch.as_tensor(ex_h, device="cuda")
+    ws = torch.empty(loza_ssa_decode_selected_workspace_size(s.B, s.H_q, s.d_v, 1, 7, n_extra),
+                     dtype=torch.uint8, device="cuda")
+    def decode(qq, pp, **kw):
+        if n_extra:
+            return loza_ssa_decode_selected(qq, kv, pp, sl, extra, s.d_v, scale=s.scale,
+                                            workspace=ws, **kw)
+        return loza_ssa_decode(qq, kv, pp, sl, s.d_v, scale=s.scale, workspace=ws, **kw)
+
+    o, lse = decode(q, pt)
+    keys = int(sum(row_pairs(np.array([n - 1]))[0] for n in lens)) + extra_keys
     algo_bytes = keys * s.d_qk * 2 + q.numel() * 2 + o.numel() * 2 + lse.numel() * 4
     flops = 2 * (s.d_qk + s.d_v) * keys * s.H_q
 
@@ -306,7 +335,7 @@ def decode_bench(iters, warmup, peaks, seed=0, len_hi=None, n_sets=8, world=1):
 
     def call(i):
         qq, pp = sets[i % n_sets]
-        loza_ssa_decode(qq, kv, pp, sl, s.d_v, o=o, lse=lse, scale=s.scale, workspace=ws)
+        decode(qq, pp, o=o, lse=lse)
 
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
@@ -350,7 +379,8 @@ def decode_bench(iters, warmup, peaks, seed=0, len_hi=None, n_sets=8, world=1):
     return {
         "workload": f"ssa_decode B={s.B} H_q={s.H_q} d_qk={s.d_qk} d_v={s.d_v} paged 128, "
                     f"seq_len U[{s.len_lo},{len_hi or s.len_hi}] seed {seed}, random page permutation "
-                    f"over {kv.shape[0]} pages",
+                    f"over {kv.shape[0]} pages"
+                    + (f", plus {n_extra} distinct selected pages per sequence" if n_extra else ""),
         "value": round(gbs, 1), "unit": "GB/s", "us_per_step": round(ms * 1e3, 2),
         "algorithmic_bytes_per_step": algo_bytes, "useful_gflop_per_step": round(flops / 1e9, 3),
         "tflops": round(flops / (ms * 1e-3) / 1e12, 1),
@@ -419,6 +449,9 @@ def main():
     ap.add_argument("--decode-iters", type=int, default=30)
     ap.add_argument("--decode-len-hi", type=int, default=None,
                     help="shorter decode contexts (smaller page pool), for profiler captures")
+    ap.add_argument("--decode-extra", type=int, default=8,
+                    help="also time the selected-pages decode with this many chosen pages per "
+                         "sequence (0: skip it)")
     ap.add_argument("--cpu-budget-s", type=float, default=10.0)
     ap.add_argument("--ref-budget-s", type=float, default=60.0,
                     help="--impl reference: CPU seconds over all warm-up and timed steps")
@@ -468,8 +501,14 @@ def main():
     if args.no_prefill:
         decode = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
                               len_hi=args.decode_len_hi, world=world)
+        selected = None
+        if args.decode_extra:
+            selected = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
+                                    len_hi=args.decode_len_hi, world=world,
+                                    n_extra=args.decode_extra)
         if rank == 0:
-            print(json.dumps({"metric": METRIC, "decode": decode}), flush=True)
+            print(json.dumps({"metric": METRIC, "decode": decode, "decode_selected": selected}),
+                  flush=True)
         if dist:
             torch.distributed.destroy_process_group()
         return
@@ -486,12 +525,16 @@ def main():
     e2e_val = world * flops / (e2e_ms * 1e-3) / 1e12  # every rank runs the same e2e loop
 
     w_desc, w_tokens = w["desc"], w["tokens"]
-    decode = None
+    decode = selected = None
     if not args.no_decode:
         del w
         torch.cuda.empty_cache()
         decode = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
                               len_hi=args.decode_len_hi, world=world)
+        if args.decode_extra:
+            selected = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
+                                    len_hi=args.decode_len_hi, world=world,
+                                    n_extra=args.decode_extra)
 
     if rank != 0:
         if dist:
@@ -534,6 +577,7 @@ def main():
         "clocks": clocks,
         "gpu_launches": args.steps,
         "decode": decode,
+        "decode_selected": selected,
     }
     print(json.dumps(line), flush=True)
     if dist:

@@ -56,7 +56,11 @@ struct DecodeParams {
   __nv_bfloat16* o;       // [B, H_q, 512]
   float* lse;             // [B, H_q]
   int B, H_q, HG, max_pages, n_pages, n_sink, n_local;
-  int n_split;  // split CTAs per (sequence, head group): ceil(window pages / 2)
+  int n_split;  // split CTAs per (sequence, head group): ceil(listed pages / 2)
+  // Optional pages chosen per sequence on top of the window (nullptr: none):
+  // [B, max_extra] logical page ids.
+  const int* extra_pages;
+  int max_extra;
   int wave;     // CTAs resident at once: the CTA `wave` later runs on a freed SM
   float scale_log2;
 };
@@ -78,17 +82,44 @@ __device__ __forceinline__ bool decode_window(const DecodeParams& p, int b, Deco
   return true;
 }
 
-// Physical page of window tile `i`, or -1 if the table entry is outside the pool.
-__device__ __forceinline__ int decode_page(const DecodeParams& p, int b, const DecodeWindow& w,
-                                           int i) {
-  const int logical = tile_block(w.tr, i);
+// Logical pages of split `sp` of sequence b: entries 2sp and 2sp+1 of the
+// sequence's page list, which holds the window's tiles in order, then the
+// sequence's extra pages that lie strictly between the sink pages and the local
+// run (others are in the window or after the query) and were not listed
+// before.  Returns how many of the two entries exist (0..2).  The extra pages
+// are the page-level selection of the LongCat sparse-attention article (机制 1:
+// fixed sink + sliding window plus indexer-chosen tokens; 机制 3: chosen in
+// pages of P = 128).  One pass over the list; the duplicate check makes it
+// O(max_extra^2) loads at worst, all from one small L1-resident row.
+__device__ __forceinline__ int decode_split_pages(const DecodeParams& p, int b,
+                                                  const DecodeWindow& w, int sp, int (&lg)[2]) {
+  int n = 0, i = kDecodePagesPerSplit * sp;
+  for (; i < w.tr.count && n < 2; ++i) lg[n++] = tile_block(w.tr, i);
+  if (n == 2 || p.max_extra == 0) return n;
+  int k = i - w.tr.count;  // index among the extra pages of the next entry wanted
+  const int* ex = p.extra_pages + (size_t)b * p.max_extra;
+  for (int j = 0; j < p.max_extra && n < 2; ++j) {
+    const int e = __ldg(ex + j);
+    if (e < p.n_sink || e >= w.tr.local_lo) continue;
+    bool dup = false;
+    for (int j2 = 0; j2 < j && !dup; ++j2) dup = __ldg(ex + j2) == e;
+    if (dup) continue;
+    if (k == 0) lg[n++] = e;
+    else --k;
+  }
+  return n;
+}
+
+// Physical page of a logical page of sequence b, or -1 if the table entry is
+// outside the pool.
+__device__ __forceinline__ int decode_page(const DecodeParams& p, int b, int logical) {
   const int phys = __ldg(p.page_table + (size_t)b * p.max_pages + logical);
   return (phys >= 0 && phys < p.n_pages) ? phys : -1;
 }
 
-// Keys of window tile `i` at or before the query (1..128).
-__device__ __forceinline__ int decode_valid_keys(const DecodeWindow& w, int i) {
-  return min(128, w.t - tile_block(w.tr, i) * 128 + 1);
+// Keys of a logical page at or before the query (1..128).
+__device__ __forceinline__ int decode_valid_keys(const DecodeWindow& w, int logical) {
+  return min(128, w.t - logical * 128 + 1);
 }
 
 struct DecodeLayout {
@@ -155,17 +186,19 @@ __global__ void __launch_bounds__(320, 1)
   if (!decode_window(p, b, win)) {
     if (threadIdx.x == 0 && sp == 0 && hg == 0) atomicOr(&g_loza_status, 4);
   } else {
-    for (int i = kDecodePagesPerSplit * sp;
-         i < min(kDecodePagesPerSplit * (sp + 1), win.tr.count); ++i) {
-      const int ph = decode_page(p, b, win, i);
+    int lg[2];
+    const int n_lg = decode_split_pages(p, b, win, sp, lg);
+    for (int i = 0; i < n_lg; ++i) {
+      const int logical = lg[i];
+      const int ph = decode_page(p, b, logical);
       if (ph < 0) {
         if (threadIdx.x == 0) atomicOr(&g_loza_status, 2);
       } else if (phys_a < 0) {
         phys_a = ph;
-        valid_a = decode_valid_keys(win, i);
+        valid_a = decode_valid_keys(win, logical);
       } else {
         phys_b = ph;
-        valid_b = decode_valid_keys(win, i);
+        valid_b = decode_valid_keys(win, logical);
       }
     }
   }
@@ -243,9 +276,10 @@ __global__ void __launch_bounds__(320, 1)
               const int b2 = n2 / (p.n_split * p.HG);
               DecodeWindow w2;
               if (decode_window(p, b2, w2)) {
-                for (int i2 = kDecodePagesPerSplit * sp2;
-                     i2 < min(kDecodePagesPerSplit * (sp2 + 1), w2.tr.count); ++i2) {
-                  const int ph2 = decode_page(p, b2, w2, i2);
+                int lg2[2];
+                const int n_lg2 = decode_split_pages(p, b2, w2, sp2, lg2);
+                for (int i2 = 0; i2 < n_lg2; ++i2) {
+                  const int ph2 = decode_page(p, b2, lg2[i2]);
                   if (ph2 < 0) continue;
                   for (int c2 = 0; c2 < Lay::KV_CH; ++c2)
                     tma_prefetch_2d(&tm_kv, c2 * 64, ph2 * 128);

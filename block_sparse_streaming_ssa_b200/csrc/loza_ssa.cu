@@ -173,7 +173,7 @@ __global__ void debug_decode_pages_kernel(loza::DecodeParams p, int* pages, int*
   }
   counts[b] = w.tr.count;
   for (int i = 0; i < w.tr.count && i < max_tiles; ++i) {
-    const int phys = loza::decode_page(p, b, w, i);
+    const int phys = loza::decode_page(p, b, loza::tile_block(w.tr, i));
     if (phys < 0) atomicOr(&loza::g_loza_status, LOZA_SSA_DEV_BAD_PAGE);
     pages[(size_t)b * max_tiles + i] = phys;
   }
@@ -208,9 +208,10 @@ int static_scratch_address(void** out) {
   return LOZA_SSA_OK;
 }
 
-// Split CTAs per (sequence, head group): window pages taken two at a time.
-int decode_splits(int n_sink, int n_local) {
-  return (n_sink + n_local + loza::kDecodePagesPerSplit - 1) / loza::kDecodePagesPerSplit;
+// Split CTAs per (sequence, head group): listed pages taken two at a time.
+int decode_splits(int n_sink, int n_local, int max_extra = 0) {
+  return (n_sink + n_local + max_extra + loza::kDecodePagesPerSplit - 1) /
+         loza::kDecodePagesPerSplit;
 }
 
 size_t decode_partial_floats(int B, int H_q, int n_split) {
@@ -310,40 +311,56 @@ int loza_ssa_prefill_varlen(const void* q, const void* k, const void* v, void* o
                           upper, n_seqs + 1, reinterpret_cast<cudaStream_t>(stream), dev);
 }
 
-size_t loza_ssa_decode_workspace_size(int B, int H_q, int d_v, int n_sink, int n_local) {
+size_t loza_ssa_decode_selected_workspace_size(int B, int H_q, int d_v, int n_sink, int n_local,
+                                               int max_extra) {
   if (B < 1 || H_q < 1 || d_v != loza::kDecodeDv || n_sink < 0 || n_local < 1 ||
-      n_sink + n_local > kMaxDecodeWindow)
+      max_extra < 0 || (long long)n_sink + n_local + max_extra > kMaxDecodeWindow)
     return 0;
-  const size_t rows = decode_partial_floats(B, H_q, decode_splits(n_sink, n_local));
+  const size_t rows = decode_partial_floats(B, H_q, decode_splits(n_sink, n_local, max_extra));
   const size_t o_bytes = rows * loza::kDecodeDv * sizeof(__half);  // partial O is fp16
   const size_t lse_bytes = rows * sizeof(float);
   return ((o_bytes + 255) / 256) * 256 + ((lse_bytes + 255) / 256) * 256;
 }
 
-int loza_ssa_decode(const void* q, const void* paged_kv, const int* page_table,
-                    const int* seq_lens, void* o, float* lse, int B, int H_q, int d_qk, int d_v,
-                    int page_size, int max_pages, int n_pages, int n_sink, int n_local,
-                    float scale, void* workspace, size_t workspace_bytes,
-                    loza_ssa_stream_t stream) {
+size_t loza_ssa_decode_workspace_size(int B, int H_q, int d_v, int n_sink, int n_local) {
+  return loza_ssa_decode_selected_workspace_size(B, H_q, d_v, n_sink, n_local, 0);
+}
+
+}  // extern "C"
+
+namespace {
+
+// loza_ssa_decode with an optional per-sequence list of extra pages
+// (extra_pages == nullptr and max_extra == 0: the plain window).
+int decode_impl(const void* q, const void* paged_kv, const int* page_table, const int* seq_lens,
+                const int* extra_pages, int max_extra, void* o, float* lse, int B, int H_q,
+                int d_qk, int d_v, int page_size, int max_pages, int n_pages, int n_sink,
+                int n_local, float scale, void* workspace, size_t workspace_bytes,
+                loza_ssa_stream_t stream) {
   if (!q || !paged_kv || !page_table || !seq_lens || !o || !lse) return LOZA_SSA_ERR_NULL;
+  if (max_extra < 0) return LOZA_SSA_ERR_SHAPE;
+  if (max_extra > 0 && !extra_pages) return LOZA_SSA_ERR_NULL;
+  if (max_extra > 0 && !aligned(extra_pages, 4)) return LOZA_SSA_ERR_ALIGN;
   if (B < 1 || H_q < 1 || max_pages < 1 || n_pages < 1 || !std::isfinite(scale))
     return LOZA_SSA_ERR_SHAPE;
   if (B > 65535 || (H_q + 127) / 128 > 65535 || (long long)n_pages * 128 >= (1ll << 31))
     return LOZA_SSA_ERR_SHAPE;
   if (d_qk != loza::kDecodeDqk || d_v != loza::kDecodeDv) return LOZA_SSA_ERR_HEAD_DIM;
   if (page_size != 128) return LOZA_SSA_ERR_BLOCK;
-  if (n_sink < 0 || n_local < 1 || n_sink + n_local > kMaxDecodeWindow) return LOZA_SSA_ERR_WINDOW;
+  if (n_sink < 0 || n_local < 1 || (long long)n_sink + n_local + max_extra > kMaxDecodeWindow)
+    return LOZA_SSA_ERR_WINDOW;
   if (!aligned(q, 16) || !aligned(paged_kv, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
       !aligned(page_table, 4) || !aligned(seq_lens, 4))
     return LOZA_SSA_ERR_ALIGN;
-  const size_t need = loza_ssa_decode_workspace_size(B, H_q, d_v, n_sink, n_local);
+  const size_t need =
+      loza_ssa_decode_selected_workspace_size(B, H_q, d_v, n_sink, n_local, max_extra);
   if (!workspace || workspace_bytes < need) return LOZA_SSA_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return LOZA_SSA_ERR_ALIGN;
   DeviceInfo dev;
   int rc = device_info(dev);
   if (rc != LOZA_SSA_OK) return rc;
 
-  const int n_split = decode_splits(n_sink, n_local);
+  const int n_split = decode_splits(n_sink, n_local, max_extra);
   const int HG = (H_q + 127) / 128;
   const size_t rows = decode_partial_floats(B, H_q, n_split);
   if (rows >= (1ull << 31)) return LOZA_SSA_ERR_SHAPE;  // keeps the CTA index math in int
@@ -363,6 +380,8 @@ int loza_ssa_decode(const void* q, const void* paged_kv, const int* page_table,
   prm.n_sink = n_sink;
   prm.n_local = n_local;
   prm.n_split = n_split;
+  prm.extra_pages = max_extra > 0 ? extra_pages : nullptr;
+  prm.max_extra = max_extra > 0 ? max_extra : 0;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.wave = dev.num_sms;  // one split CTA per SM
 
@@ -394,6 +413,31 @@ int loza_ssa_decode(const void* q, const void* paged_kv, const int* page_table,
   if ((e = cudaLaunchKernelEx(&cfg, loza::ssa_decode_merge_kernel, prm)) != cudaSuccess)
     return cuda_fail(e, "decode merge launch");
   return LOZA_SSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int loza_ssa_decode(const void* q, const void* paged_kv, const int* page_table,
+                    const int* seq_lens, void* o, float* lse, int B, int H_q, int d_qk, int d_v,
+                    int page_size, int max_pages, int n_pages, int n_sink, int n_local,
+                    float scale, void* workspace, size_t workspace_bytes,
+                    loza_ssa_stream_t stream) {
+  return decode_impl(q, paged_kv, page_table, seq_lens, nullptr, 0, o, lse, B, H_q, d_qk, d_v,
+                     page_size, max_pages, n_pages, n_sink, n_local, scale, workspace,
+                     workspace_bytes, stream);
+}
+
+int loza_ssa_decode_selected(const void* q, const void* paged_kv, const int* page_table,
+                             const int* seq_lens, const int* extra_pages, int max_extra, void* o,
+                             float* lse, int B, int H_q, int d_qk, int d_v, int page_size,
+                             int max_pages, int n_pages, int n_sink, int n_local, float scale,
+                             void* workspace, size_t workspace_bytes,
+                             loza_ssa_stream_t stream) {
+  return decode_impl(q, paged_kv, page_table, seq_lens, extra_pages, max_extra, o, lse, B, H_q,
+                     d_qk, d_v, page_size, max_pages, n_pages, n_sink, n_local, scale, workspace,
+                     workspace_bytes, stream);
 }
 
 int loza_ssa_decode_static_scratch(const void* q, const void* paged_kv, const int* page_table,

@@ -54,6 +54,11 @@ def lib() -> ctypes.CDLL:
         L.loza_ssa_decode.restype = i32
         L.loza_ssa_decode_workspace_size.argtypes = [i32, i32, i32, i32, i32]
         L.loza_ssa_decode_workspace_size.restype = sz
+        L.loza_ssa_decode_selected.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32,
+                                               i32, i32, i32, i32, i32, i32, f32, vp, sz, vp]
+        L.loza_ssa_decode_selected.restype = i32
+        L.loza_ssa_decode_selected_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
+        L.loza_ssa_decode_selected_workspace_size.restype = sz
         L.loza_ssa_status_string.argtypes = [i32]
         L.loza_ssa_status_string.restype = ctypes.c_char_p
         L.loza_ssa_last_error_string.argtypes = []
@@ -189,6 +194,49 @@ def loza_ssa_decode(q, paged_kv, page_table, seq_lens, d_v=512, o=None, lse=None
         _ptr(q), _ptr(paged_kv), _ptr(page_table), _ptr(seq_lens), _ptr(o), _ptr(lse), B, H_q,
         d_qk, d_v, page_size, max_pages, n_pages, n_sink, n_local, float(scale), _ptr(workspace),
         workspace.numel(), _stream(stream)))
+    return o, lse
+
+
+def loza_ssa_decode_selected_workspace_size(B, H_q, d_v=512, n_sink=1, n_local=7,
+                                            max_extra=0) -> int:
+    return int(lib().loza_ssa_decode_selected_workspace_size(B, H_q, d_v, n_sink, n_local,
+                                                             max_extra))
+
+
+def loza_ssa_decode_selected(q, paged_kv, page_table, seq_lens, extra_pages, d_v=512, o=None,
+                             lse=None, page_size=128, n_sink=1, n_local=7, scale=None,
+                             workspace=None, stream=None):
+    """Paged decode over the SSA window plus per-sequence chosen pages.
+    extra_pages: int32 CUDA [B, max_extra] logical page ids (entries that are
+    negative, in the window or after it add nothing; duplicates count once).
+    Other arguments and the result as loza_ssa_decode."""
+    _need(q, torch.bfloat16, "q")
+    _need(paged_kv, torch.bfloat16, "paged_kv")
+    _need(page_table, torch.int32, "page_table")
+    _need(seq_lens, torch.int32, "seq_lens")
+    _need(extra_pages, torch.int32, "extra_pages")
+    B, H_q, d_qk = q.shape
+    if extra_pages.dim() != 2 or extra_pages.shape[0] != B:
+        raise ValueError("extra_pages must be [B, max_extra]")
+    max_extra = extra_pages.shape[1]
+    n_pages = paged_kv.shape[0]
+    max_pages = page_table.shape[1]
+    if o is None:
+        o = torch.empty((B, H_q, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H_q), dtype=torch.float32, device=q.device)
+    _need(o, torch.bfloat16, "o")
+    _need(lse, torch.float32, "lse")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d_qk)
+    need = loza_ssa_decode_selected_workspace_size(B, H_q, d_v, n_sink, n_local, max_extra)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _need(workspace, torch.uint8, "workspace")
+    _check(lib().loza_ssa_decode_selected(
+        _ptr(q), _ptr(paged_kv), _ptr(page_table), _ptr(seq_lens), _ptr(extra_pages), max_extra,
+        _ptr(o), _ptr(lse), B, H_q, d_qk, d_v, page_size, max_pages, n_pages, n_sink, n_local,
+        float(scale), _ptr(workspace), workspace.numel(), _stream(stream)))
     return o, lse
 
 

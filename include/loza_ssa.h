@@ -123,6 +123,34 @@ int loza_ssa_decode(const void* q, const void* paged_kv, const int* page_table,
 /* Bytes of workspace loza_ssa_decode needs (0 on invalid arguments). */
 size_t loza_ssa_decode_workspace_size(int B, int H_q, int d_v, int n_sink, int n_local);
 
+/*
+ * Paged decode over the SSA window plus pages chosen per sequence: the fixed
+ * sink + sliding-window budget plus pages selected by a page-level indexer
+ * (LongCat sparse-attention article, 机制 1 流感知索引 and 机制 3 分层索引, pages
+ * of P = 128 tokens; the indexer itself is the caller's).
+ *   extra_pages : DEVICE int32 [B, max_extra]; row b lists logical pages of
+ *                 sequence b.  An entry that is negative, at or after the first
+ *                 local page of the window, or below n_sink (i.e. not strictly
+ *                 between the sink pages and the local run) adds nothing, and
+ *                 a page listed twice counts once.  Every listed page lies
+ *                 before the query's page, so all 128 of its keys are visible.
+ *   max_extra   : >= 0; n_sink + n_local + max_extra <= 4096.
+ * The keys of sequence b are { j <= t : page(j) in W(page(t)) or page(j) listed }.
+ * workspace: at least loza_ssa_decode_selected_workspace_size(B, H_q, d_v,
+ * n_sink, n_local, max_extra) bytes.  Other arguments, layouts, ownership and
+ * statuses as for loza_ssa_decode (max_extra = 0 gives the same result).
+ */
+int loza_ssa_decode_selected(const void* q, const void* paged_kv, const int* page_table,
+                             const int* seq_lens, const int* extra_pages, int max_extra, void* o,
+                             float* lse, int B, int H_q, int d_qk, int d_v, int page_size,
+                             int max_pages, int n_pages, int n_sink, int n_local, float scale,
+                             void* workspace, size_t workspace_bytes,
+                             loza_ssa_stream_t stream);
+
+/* Bytes of workspace loza_ssa_decode_selected needs (0 on invalid arguments). */
+size_t loza_ssa_decode_selected_workspace_size(int B, int H_q, int d_v, int n_sink, int n_local,
+                                               int max_extra);
+
 /* Static description of a status code (never NULL). */
 const char* loza_ssa_status_string(int status);
 

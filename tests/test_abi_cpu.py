@@ -68,6 +68,26 @@ def test_decode_workspace_size(L):
     assert api.loza_ssa_decode_workspace_size(32, 128, 512, 1, 0) == 0      # n_local < 1
 
 
+def test_decode_selected_workspace_size(L):
+    from block_sparse_streaming_ssa_b200 import loza_ssa as api
+    # one split per two listed pages: window 8 + 8 chosen pages -> 8 splits
+    rows = 32 * 1 * 8 * 128
+    want = -(-rows * 512 * 2 // 256) * 256 + -(-rows * 4 // 256) * 256
+    assert api.loza_ssa_decode_selected_workspace_size(32, 128, 512, 1, 7, 8) == want
+    assert api.loza_ssa_decode_selected_workspace_size(32, 128, 512, 1, 7, 0) == \
+        api.loza_ssa_decode_workspace_size(32, 128, 512, 1, 7)
+    assert api.loza_ssa_decode_selected_workspace_size(32, 128, 512, 1, 7, -1) == 0
+    assert api.loza_ssa_decode_selected_workspace_size(32, 128, 512, 1, 7, 4089) == 0
+
+
+def test_decode_selected_rejects_missing_list(L):
+    vp = ctypes.c_void_p
+    rc = L.loza_ssa_decode_selected(vp(0x1000), vp(0x1000), vp(0x1000), vp(0x1000), None, 4,
+                                    vp(0x1000), vp(0x1000), 2, 128, 576, 512, 128, 8, 16, 1, 7,
+                                    ctypes.c_float(0.04), vp(0x1000), 1 << 20, None)
+    assert rc == -1   # LOZA_SSA_ERR_NULL: max_extra > 0 without a list
+
+
 def _prefill(L, q=0x1000, k=0x1000, v=0x1000, o=0x1000, lse=0x1000, B=1, H=2, Ln=256, dqk=64,
              dv=64, block=128, ns=1, nl=7, scale=0.125):
     vp = ctypes.c_void_p
