@@ -390,7 +390,8 @@ def decode_bench(iters, warmup, peaks, seed=0, len_hi=None, n_sets=8, world=1, n
         "eager_flush_us": round(eager_ms * 1e3, 2),
         "roofline": {"bound": "hbm", "achieved": round(gbs / world, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(gbs / world / peaks["hbm_gbs"], 4),
-                     "traffic": traffic_lookup("ssa_decode_split_kernel", "decode"),
+                     "traffic": traffic_lookup("ssa_decode_split_kernel",
+                                               "decode_selected" if n_extra else "decode"),
                      "peak_source": peaks["source"],
                      "note": "time of the whole call: split kernel + LSE merge kernel"},
         "gpu_launches": 2 * iters * 5 + 2 * iters,
