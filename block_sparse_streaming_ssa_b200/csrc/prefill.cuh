@@ -33,10 +33,12 @@
 //   warp 11    issuer of the O += P V MMAs (one elected lane)
 // K and V have their own producers so a K load never queues behind a V load
 // that is waiting for its ring slot: S consumes K_{j+1} before P.V reads V_j.
-// S and P.V have their own issuers because one thread issues a tcgen05.mma
-// only every ~100-200 SM cycles (measured on B200): with a single issuer the
-// chain P_j ready -> P_j V_j issued -> S_{j+2} issued sits on the softmax's
-// critical path.
+// S and P.V have their own issuers because an issuer blocks on its barrier
+// waits: with a single issuer the wait for P_j also held back the S MMAs of
+// later tiles, so the chain P_j ready -> P_j V_j issued -> S_{j+2} issued sat
+// on the softmax's critical path.  (Issue rate itself is not the limit: a
+// lone lane starts a 128x128x16 MMA every ~86 SM cycles in a tight loop,
+// measured on B200.)
 //
 // TMEM (512 columns x 128 lanes, fp32): S buffers [0,128), [128,256),
 // [256,384), O buffers from 384 (two of them when 2*DV <= 128, so the next
@@ -367,9 +369,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------ MMA issuer: S
-    // One thread issues a tcgen05.mma only every ~100-200 SM cycles, so S and
-    // P.V have an issuer each; with three S buffers the S issuer runs up to
-    // two tiles ahead of the softmax.
+    // S and P.V have an issuer each, so a wait for P never holds back S; with
+    // three S buffers the S issuer runs up to two tiles ahead of the softmax.
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16_f32(128, 128, false);
       int g = 0, it = 0;
