@@ -270,13 +270,14 @@ int oracle_ssa_prefill_varlen_rows(const void* q, const void* k, const void* v, 
  */
 static int decode_rows(const void* q, const void* kv, int elt, const int32_t* page_table,
                        const int32_t* seq_lens, const int32_t* extra_pages, int64_t max_extra,
-                       int64_t B, int64_t Hq, int dqk, int dv, int64_t page_size,
+                       int64_t q_len, int64_t B, int64_t Hq, int dqk, int dv, int64_t page_size,
                        int64_t max_pages, int64_t n_pages, int64_t n_sink, int64_t n_local,
                        double scale, const int64_t* rows, int64_t n_rows, double* o,
                        double* lse) {
   int64_t longest = 1;
+  if (q_len < 1) return -4;
   for (int64_t b = 0; b < B; ++b) {
-    if (seq_lens[b] < 1 || seq_lens[b] > max_pages * page_size) return -4;
+    if (seq_lens[b] < q_len || seq_lens[b] > max_pages * page_size) return -4;
     if (seq_lens[b] > longest) longest = seq_lens[b];
   }
   int64_t cap = max_keys(longest, page_size, n_sink + max_extra, n_local);
@@ -289,13 +290,16 @@ static int decode_rows(const void* q, const void* kv, int elt, const int32_t* pa
 #pragma omp for schedule(dynamic, 4)
     for (int64_t r = 0; r < n_rows; ++r) {
       int64_t flat = rows[r];
-      if (flat < 0 || flat >= B * Hq) {
+      if (flat < 0 || flat >= B * q_len * Hq) {
 #pragma omp atomic write
         err = -2;
         continue;
       }
-      int64_t b = flat / Hq;
-      int64_t t = (int64_t)seq_lens[b] - 1;
+      /* row flat = (b * q_len + token) * Hq + h; token k of sequence b sits at
+         position seq_len - q_len + k */
+      int64_t b = flat / (q_len * Hq);
+      int64_t token = (flat / Hq) % q_len;
+      int64_t t = (int64_t)seq_lens[b] - q_len + token;
       int rc = attend_row(q, flat * dqk, elt, kv, kv, elt, 0, 0, dqk, dqk,
                           page_table + b * max_pages, n_pages, t, page_size, n_sink, n_local,
                           extra_pages ? extra_pages + b * max_extra : NULL, max_extra, dqk, dv,
@@ -317,7 +321,25 @@ int oracle_ssa_decode_rows(const void* q, const void* kv, int elt, const int32_t
                            int64_t page_size, int64_t max_pages, int64_t n_pages, int64_t n_sink,
                            int64_t n_local, double scale, const int64_t* rows, int64_t n_rows,
                            double* o, double* lse) {
-  return decode_rows(q, kv, elt, page_table, seq_lens, NULL, 0, B, Hq, dqk, dv, page_size,
+  return decode_rows(q, kv, elt, page_table, seq_lens, NULL, 0, 1, B, Hq, dqk, dv, page_size,
+                     max_pages, n_pages, n_sink, n_local, scale, rows, n_rows, o, lse);
+}
+
+/*
+ * Paged decode with q_len query tokens per sequence (a speculative or
+ * multi-token step): token k of sequence b is the query at position
+ * t = seq_len - q_len + k, attending J(t) as defined at the top of this file
+ * -- the same mask applied to each query position, so the new tokens see
+ * each other causally.  q: [B, q_len, Hq, dqk]; rows are flat
+ * r = (b*q_len + k)*Hq + h; seq_lens[b] >= q_len.  Other arguments as
+ * oracle_ssa_decode_rows.
+ */
+int oracle_ssa_decode_mtp_rows(const void* q, const void* kv, int elt, const int32_t* page_table,
+                               const int32_t* seq_lens, int64_t q_len, int64_t B, int64_t Hq,
+                               int dqk, int dv, int64_t page_size, int64_t max_pages,
+                               int64_t n_pages, int64_t n_sink, int64_t n_local, double scale,
+                               const int64_t* rows, int64_t n_rows, double* o, double* lse) {
+  return decode_rows(q, kv, elt, page_table, seq_lens, NULL, 0, q_len, B, Hq, dqk, dv, page_size,
                      max_pages, n_pages, n_sink, n_local, scale, rows, n_rows, o, lse);
 }
 
@@ -336,7 +358,7 @@ int oracle_ssa_decode_sel_rows(const void* q, const void* kv, int elt, const int
                                int64_t page_size, int64_t max_pages, int64_t n_pages,
                                int64_t n_sink, int64_t n_local, double scale, const int64_t* rows,
                                int64_t n_rows, double* o, double* lse) {
-  return decode_rows(q, kv, elt, page_table, seq_lens, extra_pages, max_extra, B, Hq, dqk, dv,
+  return decode_rows(q, kv, elt, page_table, seq_lens, extra_pages, max_extra, 1, B, Hq, dqk, dv,
                      page_size, max_pages, n_pages, n_sink, n_local, scale, rows, n_rows, o, lse);
 }
 

@@ -80,6 +80,10 @@ def _load():
             vp, vp, i32, vp, vp, vp, i64, i64, i64, i32, i32, i64, i64, i64, i64, i64, ctypes.c_double,
             vp, i64, vp, vp]
         lib.oracle_ssa_decode_sel_rows.restype = i32
+        lib.oracle_ssa_decode_mtp_rows.argtypes = [
+            vp, vp, i32, vp, vp, i64, i64, i64, i32, i32, i64, i64, i64, i64, i64, dbl, vp, i64,
+            vp, vp]
+        lib.oracle_ssa_decode_mtp_rows.restype = i32
         lib.oracle_ssa_num_threads.argtypes = []
         lib.oracle_ssa_num_threads.restype = i32
         _lib = lib
@@ -242,6 +246,39 @@ def decode_selected(q, kv, page_table, seq_lens, extra_pages, dv, page_size=128,
         raise ValueError(f"oracle decode (selected pages) failed ({rc})")
     if full:
         return o.reshape(B, Hq, dv), lse.reshape(B, Hq)
+    return o, lse
+
+
+def decode_mtp(q, kv, page_table, seq_lens, dv, page_size=128, n_sink=1, n_local=7, scale=None,
+               rows=None):
+    """Paged decode with q_len query tokens per sequence: q [B, q_len, Hq, dqk];
+    token k of sequence b is the query at position seq_lens[b] - q_len + k and
+    attends J(t) of the SSA mask (QbitAI LoZA article, 1024-token window
+    paragraph) at its own position.  ``rows``: optional flat indices
+    (b*q_len + k)*Hq + h.  Returns o [B, q_len, Hq, dv], lse [B, q_len, Hq]."""
+    q = np.ascontiguousarray(q)
+    kv = np.ascontiguousarray(kv)
+    pt = np.ascontiguousarray(page_table, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    B, q_len, Hq, dqk = q.shape
+    n_pages = kv.shape[0]
+    assert kv.shape[1] == page_size and kv.shape[2] == dqk
+    elt = _elt(q)
+    assert _elt(kv) == elt
+    if scale is None:
+        scale = 1.0 / np.sqrt(dqk)
+    full = rows is None
+    n_all = B * q_len * Hq
+    rows = np.arange(n_all, dtype=np.int64) if full else np.ascontiguousarray(rows, dtype=np.int64)
+    o = np.empty((rows.size, dv), dtype=np.float64)
+    lse = np.empty(rows.size, dtype=np.float64)
+    rc = _load().oracle_ssa_decode_mtp_rows(
+        _ptr(q), _ptr(kv), elt, _ptr(pt), _ptr(sl), q_len, B, Hq, dqk, dv, page_size, pt.shape[1],
+        n_pages, n_sink, n_local, float(scale), _ptr(rows), rows.size, _ptr(o), _ptr(lse))
+    if rc:
+        raise ValueError(f"oracle decode (q_len tokens) failed ({rc})")
+    if full:
+        return o.reshape(B, q_len, Hq, dv), lse.reshape(B, q_len, Hq)
     return o, lse
 
 

@@ -375,3 +375,70 @@ def test_decode_selected_without_pages_is_decode():
     b = orc.decode(q, kv, pt, sl, dv=16, page_size=8, n_sink=1, n_local=3)
     np.testing.assert_array_equal(a[0], b[0])
     np.testing.assert_array_equal(a[1], b[1])
+
+
+# --- decode with several query tokens per sequence (speculative / multi-token
+# steps): token k of sequence b is the query at position seq_len - q_len + k
+
+def _mtp_case(seed, seq_lens, q_len, Hq=2, dqk=24):
+    q1, kv, pt, sl = _decode_case(seed, seq_lens, Hq=Hq, dqk=dqk)
+    rng = np.random.default_rng(seed + 1000)
+    q = rng.standard_normal((len(seq_lens), q_len, Hq, dqk))
+    return q, kv, pt, sl
+
+
+def test_decode_mtp_matches_brute_force_per_token():
+    q_len = 3
+    q, kv, pt, sl = _mtp_case(21, [3, 9, 17, 61, 100], q_len)
+    o, lse = orc.decode_mtp(q, kv, pt, sl, dv=16, page_size=8, n_sink=1, n_local=3, scale=0.3)
+    for k in range(q_len):
+        # token k alone: a plain decode whose sequence ends at its position
+        o_bf, lse_bf = orc.brute_force_decode(q[:, k], kv, pt, sl - q_len + k + 1, dv=16,
+                                              page_size=8, n_sink=1, n_local=3, scale=0.3)
+        np.testing.assert_allclose(o[:, k], o_bf, atol=1e-11)
+        np.testing.assert_allclose(lse[:, k], lse_bf, atol=1e-11)
+
+
+def test_decode_mtp_equals_masked_prefill_rows():
+    """The q_len new tokens are the last q_len rows of a prefill over the
+    gathered sequence: checked against the materialised-mask brute force."""
+    q_len, n = 4, 45
+    q, kv, pt, sl = _mtp_case(22, [n], q_len, Hq=2, dqk=16)
+    o, lse = orc.decode_mtp(q, kv, pt, sl, dv=8, page_size=8, n_sink=2, n_local=2, scale=0.25)
+    logical = np.arange(n)
+    rows = kv.reshape(-1, kv.shape[-1])[pt[0][logical // 8] * 8 + logical % 8]
+    for h in range(2):
+        qq = np.zeros((n, 16))
+        qq[n - q_len:] = q[0, :, h]
+        o_p, l_p = orc.brute_force_prefill(qq, rows, rows[:, :8], blk=8, n_sink=2, n_local=2,
+                                           scale=0.25)
+        np.testing.assert_allclose(o[0, :, h], o_p[n - q_len:], atol=1e-12)
+        np.testing.assert_allclose(lse[0, :, h], l_p[n - q_len:], atol=1e-12)
+
+
+def test_decode_mtp_key_count():
+    """q = 0: LSE = ln|J(t)| with |J(t)| = min(t+1, blk*(n_sink+n_local-1) + t%blk + 1)."""
+    q_len = 5
+    lens = [5, 16, 33, 64, 129]
+    q, kv, pt, sl = _mtp_case(23, lens, q_len)
+    q[:] = 0.0
+    _, lse = orc.decode_mtp(q, kv, pt, sl, dv=16, page_size=8, n_sink=1, n_local=3)
+    for b, n in enumerate(lens):
+        for k in range(q_len):
+            t = n - q_len + k
+            count = min(t + 1, 8 * (1 + 3 - 1) + t % 8 + 1)
+            np.testing.assert_allclose(lse[b, k], np.log(count), atol=1e-12)
+
+
+def test_decode_mtp_last_token_is_decode():
+    q, kv, pt, sl = _mtp_case(24, [7, 50, 90], 2)
+    o, lse = orc.decode_mtp(q, kv, pt, sl, dv=16, page_size=8, n_sink=1, n_local=3)
+    o1, lse1 = orc.decode(q[:, -1], kv, pt, sl, dv=16, page_size=8, n_sink=1, n_local=3)
+    np.testing.assert_array_equal(o[:, -1], o1)
+    np.testing.assert_array_equal(lse[:, -1], lse1)
+
+
+def test_decode_mtp_rejects_short_sequence():
+    q, kv, pt, sl = _mtp_case(25, [2, 40], 3)
+    with pytest.raises(ValueError):
+        orc.decode_mtp(q, kv, pt, sl, dv=16, page_size=8, n_sink=1, n_local=3)
