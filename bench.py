@@ -3,7 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--config mha|tiny|mla|varlen] [--no-decode] [--no-prefill]
-                    [--no-cpu-baseline] [--decode-extra N]
+                    [--no-cpu-baseline] [--decode-extra N] [--decode-mtp Q]
 
 One JSON line on rank 0.  A step is one SSA prefill call over the chosen
 workload (default: B=1, H=32, L=32768, d=128, 1 sink + 7 local blocks of 128);
@@ -12,7 +12,8 @@ pairs) per step / device time, summed over ranks.  The same run also times the
 paged decode workload (32 sequences, 128 heads, 576/512, random page table over
 a ~20 GB pool) and reports it under ``decode`` in GB/s of algorithmic bytes,
 and the same decode with 8 distinct selected pages per sequence on top of the
-window under ``decode_selected`` (``--decode-extra``).
+window under ``decode_selected`` (``--decode-extra``), and the decode with 2
+query tokens per sequence under ``decode_mtp`` (``--decode-mtp``).
 
 Under torchrun every rank runs its own replica of the workload (weak scaling,
 no collective on the data path; NCCL only reduces the timing).
@@ -292,7 +293,20 @@ def decode_extra_pages(lens, n_extra, seed, n_sink=1, n_local=7, blk=128):
     return ex, added
 
 
-def decode_bench(iters, warmup, peaks, seed=0, len_hi=None, n_sets=8, world=1, n_extra=0):
+def union_window_keys(n: int, q_len: int, blk=128, n_sink=1, n_local=7) -> int:
+    """Distinct keys the last q_len positions of a length-n sequence attend
+    (the union of their SSA key sets), counted block by block."""
+    keys = set()
+    for t in range(n - q_len, n):
+        qb = t // blk
+        for kb in range(qb + 1):
+            if kb < n_sink or qb - kb < n_local:
+                keys.update(range(kb * blk, min((kb + 1) * blk, t + 1)))
+    return len(keys)
+
+
+def decode_bench(iters, warmup, peaks, seed=0, len_hi=None, n_sets=8, world=1, n_extra=0,
+                 q_len=1):
     """Paged decode through the public call.  ``value``: algorithmic bytes per
     call / device time per call, with the calls captured in a CUDA graph (the
     way a serving loop issues decode steps) and rotating over ``n_sets``
@@ -300,29 +314,40 @@ def decode_bench(iters, warmup, peaks, seed=0, len_hi=None, n_sets=8, world=1, n
     table and queries each), so that consecutive calls find nothing of their
     inputs in L2.  ``n_extra`` > 0: the selected-pages decode, each sequence
     also attending ``n_extra`` distinct pages chosen between its sink and its
-    local run.  ``eager_flush_us``: one eager call per step after a 2x L2
+    local run.  ``q_len`` > 1: several query tokens per sequence (the
+    multi-token decode); the bytes count the union of the tokens' key sets
+    once, the FLOPs every token's own set.  ``eager_flush_us``: one eager call per step after a 2x L2
     write, for comparison (it also pays the write-back of the flushed lines
     and, when the GPU runs dry, the host-side cost of the call)."""
     import torch
     from block_sparse_streaming_ssa_b200 import synth
-    from block_sparse_streaming_ssa_b200.loza_ssa import (loza_ssa_decode, loza_ssa_decode_selected,
+    from block_sparse_streaming_ssa_b200.loza_ssa import (loza_ssa_decode, loza_ssa_decode_mtp,
+                                                          loza_ssa_decode_mtp_workspace_size,
+                                                          loza_ssa_decode_selected,
                                                           loza_ssa_decode_selected_workspace_size)
     s = synth.DECODE
     lens = synth.decode_seq_lens(seed, s.B, s.len_lo, len_hi or s.len_hi)
-    q, kv, pt, sl = synth.decode_inputs(lens, s.H_q, s.d_qk, seed=seed, device="cuda")
+    q, kv, pt, sl = synth.decode_inputs(lens, s.H_q, s.d_qk, seed=seed, device="cuda",
+                                        q_len=q_len if q_len > 1 else None)
     ex_h, extra_keys = decode_extra_pages(lens, n_extra, seed)
     extra = torch.as_tensor(ex_h, device="cuda")
-    ws = torch.empty(loza_ssa_decode_selected_workspace_size(s.B, s.H_q, s.d_v, 1, 7, n_extra),
-                     dtype=torch.uint8, device="cuda")
+    ws_bytes = (loza_ssa_decode_mtp_workspace_size(s.B, q_len, s.H_q, s.d_v, 1, 7) if q_len > 1
+                else loza_ssa_decode_selected_workspace_size(s.B, s.H_q, s.d_v, 1, 7, n_extra))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+
     def decode(qq, pp, **kw):
+        if q_len > 1:
+            return loza_ssa_decode_mtp(qq, kv, pp, sl, s.d_v, scale=s.scale, workspace=ws, **kw)
         if n_extra:
             return loza_ssa_decode_selected(qq, kv, pp, sl, extra, s.d_v, scale=s.scale,
                                             workspace=ws, **kw)
         return loza_ssa_decode(qq, kv, pp, sl, s.d_v, scale=s.scale, workspace=ws, **kw)
 
     o, lse = decode(q, pt)
-    keys = int(sum(row_pairs(np.array([n - 1]))[0] for n in lens)) + extra_keys
-    algo_bytes = keys * s.d_qk * 2 + q.numel() * 2 + o.numel() * 2 + lse.numel() * 4
+    keys = int(sum(row_pairs(np.arange(n - q_len, n)).sum() for n in lens)) + extra_keys
+    read_keys = (int(sum(union_window_keys(n, q_len) for n in lens)) + extra_keys if q_len > 1
+                 else keys)
+    algo_bytes = read_keys * s.d_qk * 2 + q.numel() * 2 + o.numel() * 2 + lse.numel() * 4
     flops = 2 * (s.d_qk + s.d_v) * keys * s.H_q
 
     gen = torch.Generator(device="cpu").manual_seed(1000 + seed)
@@ -380,7 +405,8 @@ def decode_bench(iters, warmup, peaks, seed=0, len_hi=None, n_sets=8, world=1, n
         "workload": f"ssa_decode B={s.B} H_q={s.H_q} d_qk={s.d_qk} d_v={s.d_v} paged 128, "
                     f"seq_len U[{s.len_lo},{len_hi or s.len_hi}] seed {seed}, random page permutation "
                     f"over {kv.shape[0]} pages"
-                    + (f", plus {n_extra} distinct selected pages per sequence" if n_extra else ""),
+                    + (f", plus {n_extra} distinct selected pages per sequence" if n_extra else "")
+                    + (f", {q_len} query tokens per sequence" if q_len > 1 else ""),
         "value": round(gbs, 1), "unit": "GB/s", "us_per_step": round(ms * 1e3, 2),
         "algorithmic_bytes_per_step": algo_bytes, "useful_gflop_per_step": round(flops / 1e9, 3),
         "tflops": round(flops / (ms * 1e-3) / 1e12, 1),
@@ -391,7 +417,8 @@ def decode_bench(iters, warmup, peaks, seed=0, len_hi=None, n_sets=8, world=1, n
         "roofline": {"bound": "hbm", "achieved": round(gbs / world, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(gbs / world / peaks["hbm_gbs"], 4),
                      "traffic": traffic_lookup("ssa_decode_split_kernel",
-                                               "decode_selected" if n_extra else "decode"),
+                                               "decode_selected" if n_extra else
+                                               f"decode_mtp{q_len}" if q_len > 1 else "decode"),
                      "peak_source": peaks["source"],
                      "note": "time of the whole call: split kernel + LSE merge kernel"},
         "gpu_launches": 2 * iters * 5 + 2 * iters,
@@ -453,6 +480,9 @@ def main():
     ap.add_argument("--decode-extra", type=int, default=8,
                     help="also time the selected-pages decode with this many chosen pages per "
                          "sequence (0: skip it)")
+    ap.add_argument("--decode-mtp", type=int, default=2,
+                    help="also time the decode with this many query tokens per sequence "
+                         "(<= 1: skip it)")
     ap.add_argument("--cpu-budget-s", type=float, default=10.0)
     ap.add_argument("--ref-budget-s", type=float, default=60.0,
                     help="--impl reference: CPU seconds over all warm-up and timed steps")
@@ -507,9 +537,13 @@ def main():
             selected = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
                                     len_hi=args.decode_len_hi, world=world,
                                     n_extra=args.decode_extra)
+        mtp = None
+        if args.decode_mtp > 1:
+            mtp = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
+                               len_hi=args.decode_len_hi, world=world, q_len=args.decode_mtp)
         if rank == 0:
-            print(json.dumps({"metric": METRIC, "decode": decode, "decode_selected": selected}),
-                  flush=True)
+            print(json.dumps({"metric": METRIC, "decode": decode, "decode_selected": selected,
+                              "decode_mtp": mtp}), flush=True)
         if dist:
             torch.distributed.destroy_process_group()
         return
@@ -526,7 +560,7 @@ def main():
     e2e_val = world * flops / (e2e_ms * 1e-3) / 1e12  # every rank runs the same e2e loop
 
     w_desc, w_tokens = w["desc"], w["tokens"]
-    decode = selected = None
+    decode = selected = mtp = None
     if not args.no_decode:
         del w
         torch.cuda.empty_cache()
@@ -536,6 +570,9 @@ def main():
             selected = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
                                     len_hi=args.decode_len_hi, world=world,
                                     n_extra=args.decode_extra)
+        if args.decode_mtp > 1:
+            mtp = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
+                               len_hi=args.decode_len_hi, world=world, q_len=args.decode_mtp)
 
     if rank != 0:
         if dist:
@@ -579,6 +616,7 @@ def main():
         "gpu_launches": args.steps,
         "decode": decode,
         "decode_selected": selected,
+        "decode_mtp": mtp,
     }
     print(json.dumps(line), flush=True)
     if dist:

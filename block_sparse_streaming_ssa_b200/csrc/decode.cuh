@@ -48,14 +48,19 @@ constexpr int kDecodePagesPerSplit = 2;
 // on the FMA pipe instead of the MUFU unit.
 constexpr int kDecodePolyPairsPer8 = 3;
 
+// Rows of the decode: one per (sequence, query token).  With q_len query
+// tokens per sequence, row v is token v % q_len of sequence v / q_len, at
+// position seq_len - q_len + v % q_len; q, o and lse are indexed by row.
 struct DecodeParams {
-  const int* page_table;  // [B, max_pages]
-  const int* seq_lens;    // [B]
+  const int* page_table;  // [sequences, max_pages]
+  const int* seq_lens;    // [sequences]
   __half* o_part;         // [B*HG*n_split CTAs][64 column groups][128 heads][8]
   float* lse_part;        // [B*HG*n_split CTAs][128 heads]
-  __nv_bfloat16* o;       // [B, H_q, 512]
-  float* lse;             // [B, H_q]
-  int B, H_q, HG, max_pages, n_pages, n_sink, n_local;
+  __nv_bfloat16* o;       // [B rows, H_q, 512]
+  float* lse;             // [B rows, H_q]
+  int B;                  // rows: sequences * q_len
+  int q_len;              // query tokens per sequence (1: plain decode)
+  int H_q, HG, max_pages, n_pages, n_sink, n_local;
   int n_split;  // split CTAs per (sequence, head group): ceil(listed pages / 2)
   // Optional pages chosen per sequence on top of the window (nullptr: none):
   // [B, max_extra] logical page ids.
@@ -65,24 +70,29 @@ struct DecodeParams {
   float scale_log2;
 };
 
-// The decode window of sequence b, as the kernels select it.
+__device__ __forceinline__ int decode_seq(const DecodeParams& p, int row) {
+  return p.q_len == 1 ? row : row / p.q_len;
+}
+
+// The decode window of row b, as the kernels select it.
 struct DecodeWindow {
   int t;       // query position
   int qb;      // logical page of the query
   TileRange tr;
 };
 
-// False for a seq_len outside [1, max_pages * 128].
+// False for a seq_len outside [q_len, max_pages * 128].
 __device__ __forceinline__ bool decode_window(const DecodeParams& p, int b, DecodeWindow& w) {
-  const int len = __ldg(p.seq_lens + b);
-  if (len < 1 || (long long)len > (long long)p.max_pages * 128) return false;
-  w.t = len - 1;
+  const int s = decode_seq(p, b);
+  const int len = __ldg(p.seq_lens + s);
+  if (len < p.q_len || (long long)len > (long long)p.max_pages * 128) return false;
+  w.t = len - p.q_len + (b - s * p.q_len);
   w.qb = w.t >> 7;
   w.tr = tile_range(w.qb, p.n_sink, p.n_local);
   return true;
 }
 
-// Logical pages of split `sp` of sequence b: entries 2sp and 2sp+1 of the
+// Logical pages of split `sp` of row b: entries 2sp and 2sp+1 of the
 // sequence's page list, which holds the window's tiles in order, then the
 // sequence's extra pages that lie strictly between the sink pages and the local
 // run (others are in the window or after the query) and were not listed
@@ -97,7 +107,7 @@ __device__ __forceinline__ int decode_split_pages(const DecodeParams& p, int b,
   for (; i < w.tr.count && n < 2; ++i) lg[n++] = tile_block(w.tr, i);
   if (n == 2 || p.max_extra == 0) return n;
   int k = i - w.tr.count;  // index among the extra pages of the next entry wanted
-  const int* ex = p.extra_pages + (size_t)b * p.max_extra;
+  const int* ex = p.extra_pages + (size_t)decode_seq(p, b) * p.max_extra;
   for (int j = 0; j < p.max_extra && n < 2; ++j) {
     const int e = __ldg(ex + j);
     if (e < p.n_sink || e >= w.tr.local_lo) continue;
@@ -110,10 +120,10 @@ __device__ __forceinline__ int decode_split_pages(const DecodeParams& p, int b,
   return n;
 }
 
-// Physical page of a logical page of sequence b, or -1 if the table entry is
+// Physical page of a logical page of row b's sequence, or -1 if the table entry is
 // outside the pool.
 __device__ __forceinline__ int decode_page(const DecodeParams& p, int b, int logical) {
-  const int phys = __ldg(p.page_table + (size_t)b * p.max_pages + logical);
+  const int phys = __ldg(p.page_table + (size_t)decode_seq(p, b) * p.max_pages + logical);
   return (phys >= 0 && phys < p.n_pages) ? phys : -1;
 }
 

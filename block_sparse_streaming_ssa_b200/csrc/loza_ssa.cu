@@ -326,19 +326,29 @@ size_t loza_ssa_decode_workspace_size(int B, int H_q, int d_v, int n_sink, int n
   return loza_ssa_decode_selected_workspace_size(B, H_q, d_v, n_sink, n_local, 0);
 }
 
+size_t loza_ssa_decode_mtp_workspace_size(int B, int q_len, int H_q, int d_v, int n_sink,
+                                          int n_local) {
+  if (B < 1 || q_len < 1 || (long long)B * q_len > 65535) return 0;
+  return loza_ssa_decode_selected_workspace_size(B * q_len, H_q, d_v, n_sink, n_local, 0);
+}
+
 }  // extern "C"
 
 namespace {
 
 // loza_ssa_decode with an optional per-sequence list of extra pages
-// (extra_pages == nullptr and max_extra == 0: the plain window).
+// (extra_pages == nullptr and max_extra == 0: the plain window) and q_len
+// query tokens per sequence (q_len == 1: one).  B counts sequences.
 int decode_impl(const void* q, const void* paged_kv, const int* page_table, const int* seq_lens,
-                const int* extra_pages, int max_extra, void* o, float* lse, int B, int H_q,
-                int d_qk, int d_v, int page_size, int max_pages, int n_pages, int n_sink,
+                const int* extra_pages, int max_extra, int q_len, void* o, float* lse, int B,
+                int H_q, int d_qk, int d_v, int page_size, int max_pages, int n_pages, int n_sink,
                 int n_local, float scale, void* workspace, size_t workspace_bytes,
                 loza_ssa_stream_t stream) {
   if (!q || !paged_kv || !page_table || !seq_lens || !o || !lse) return LOZA_SSA_ERR_NULL;
-  if (max_extra < 0) return LOZA_SSA_ERR_SHAPE;
+  if (max_extra < 0 || q_len < 1) return LOZA_SSA_ERR_SHAPE;
+  if (q_len > 1 && max_extra > 0) return LOZA_SSA_ERR_SHAPE;  // no public call combines them
+  if (B >= 1 && (long long)B * q_len > 65535) return LOZA_SSA_ERR_SHAPE;
+  B *= q_len;  // from here on B counts rows: (sequence, query token) pairs
   if (max_extra > 0 && !extra_pages) return LOZA_SSA_ERR_NULL;
   if (max_extra > 0 && !aligned(extra_pages, 4)) return LOZA_SSA_ERR_ALIGN;
   if (B < 1 || H_q < 1 || max_pages < 1 || n_pages < 1 || !std::isfinite(scale))
@@ -373,6 +383,7 @@ int decode_impl(const void* q, const void* paged_kv, const int* page_table, cons
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.lse = lse;
   prm.B = B;
+  prm.q_len = q_len;
   prm.H_q = H_q;
   prm.HG = HG;
   prm.max_pages = max_pages;
@@ -424,8 +435,18 @@ int loza_ssa_decode(const void* q, const void* paged_kv, const int* page_table,
                     int page_size, int max_pages, int n_pages, int n_sink, int n_local,
                     float scale, void* workspace, size_t workspace_bytes,
                     loza_ssa_stream_t stream) {
-  return decode_impl(q, paged_kv, page_table, seq_lens, nullptr, 0, o, lse, B, H_q, d_qk, d_v,
-                     page_size, max_pages, n_pages, n_sink, n_local, scale, workspace,
+  return decode_impl(q, paged_kv, page_table, seq_lens, nullptr, 0, 1, o, lse, B, H_q, d_qk,
+                     d_v, page_size, max_pages, n_pages, n_sink, n_local, scale, workspace,
+                     workspace_bytes, stream);
+}
+
+int loza_ssa_decode_mtp(const void* q, const void* paged_kv, const int* page_table,
+                        const int* seq_lens, int q_len, void* o, float* lse, int B, int H_q,
+                        int d_qk, int d_v, int page_size, int max_pages, int n_pages, int n_sink,
+                        int n_local, float scale, void* workspace, size_t workspace_bytes,
+                        loza_ssa_stream_t stream) {
+  return decode_impl(q, paged_kv, page_table, seq_lens, nullptr, 0, q_len, o, lse, B, H_q, d_qk,
+                     d_v, page_size, max_pages, n_pages, n_sink, n_local, scale, workspace,
                      workspace_bytes, stream);
 }
 
@@ -435,9 +456,9 @@ int loza_ssa_decode_selected(const void* q, const void* paged_kv, const int* pag
                              int max_pages, int n_pages, int n_sink, int n_local, float scale,
                              void* workspace, size_t workspace_bytes,
                              loza_ssa_stream_t stream) {
-  return decode_impl(q, paged_kv, page_table, seq_lens, extra_pages, max_extra, o, lse, B, H_q,
-                     d_qk, d_v, page_size, max_pages, n_pages, n_sink, n_local, scale, workspace,
-                     workspace_bytes, stream);
+  return decode_impl(q, paged_kv, page_table, seq_lens, extra_pages, max_extra, 1, o, lse, B,
+                     H_q, d_qk, d_v, page_size, max_pages, n_pages, n_sink, n_local, scale,
+                     workspace, workspace_bytes, stream);
 }
 
 int loza_ssa_decode_static_scratch(const void* q, const void* paged_kv, const int* page_table,
@@ -509,6 +530,7 @@ int loza_ssa_debug_decode_pages(const int* page_table, const int* seq_lens, int 
   prm.page_table = page_table;
   prm.seq_lens = seq_lens;
   prm.B = B;
+  prm.q_len = 1;
   prm.max_pages = max_pages;
   prm.n_pages = n_pages;
   prm.n_sink = n_sink;

@@ -59,6 +59,11 @@ def lib() -> ctypes.CDLL:
         L.loza_ssa_decode_selected.restype = i32
         L.loza_ssa_decode_selected_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
         L.loza_ssa_decode_selected_workspace_size.restype = sz
+        L.loza_ssa_decode_mtp.argtypes = [vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32,
+                                          i32, i32, i32, i32, f32, vp, sz, vp]
+        L.loza_ssa_decode_mtp.restype = i32
+        L.loza_ssa_decode_mtp_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
+        L.loza_ssa_decode_mtp_workspace_size.restype = sz
         L.loza_ssa_status_string.argtypes = [i32]
         L.loza_ssa_status_string.restype = ctypes.c_char_p
         L.loza_ssa_last_error_string.argtypes = []
@@ -237,6 +242,42 @@ def loza_ssa_decode_selected(q, paged_kv, page_table, seq_lens, extra_pages, d_v
         _ptr(q), _ptr(paged_kv), _ptr(page_table), _ptr(seq_lens), _ptr(extra_pages), max_extra,
         _ptr(o), _ptr(lse), B, H_q, d_qk, d_v, page_size, max_pages, n_pages, n_sink, n_local,
         float(scale), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return o, lse
+
+
+def loza_ssa_decode_mtp_workspace_size(B, q_len, H_q, d_v=512, n_sink=1, n_local=7) -> int:
+    return int(lib().loza_ssa_decode_mtp_workspace_size(B, q_len, H_q, d_v, n_sink, n_local))
+
+
+def loza_ssa_decode_mtp(q, paged_kv, page_table, seq_lens, d_v=512, o=None, lse=None,
+                        page_size=128, n_sink=1, n_local=7, scale=None, workspace=None,
+                        stream=None):
+    """Paged SSA decode with q_len query tokens per sequence (positions
+    seq_len-q_len .. seq_len-1).  q: bf16 [B,q_len,H_q,d_qk]; other inputs as
+    loza_ssa_decode.  Returns (o bf16 [B,q_len,H_q,d_v], lse fp32 [B,q_len,H_q])."""
+    _need(q, torch.bfloat16, "q")
+    _need(paged_kv, torch.bfloat16, "paged_kv")
+    _need(page_table, torch.int32, "page_table")
+    _need(seq_lens, torch.int32, "seq_lens")
+    B, q_len, H_q, d_qk = q.shape
+    n_pages = paged_kv.shape[0]
+    max_pages = page_table.shape[1]
+    if o is None:
+        o = torch.empty((B, q_len, H_q, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, q_len, H_q), dtype=torch.float32, device=q.device)
+    _need(o, torch.bfloat16, "o")
+    _need(lse, torch.float32, "lse")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d_qk)
+    need = loza_ssa_decode_mtp_workspace_size(B, q_len, H_q, d_v, n_sink, n_local)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _need(workspace, torch.uint8, "workspace")
+    _check(lib().loza_ssa_decode_mtp(
+        _ptr(q), _ptr(paged_kv), _ptr(page_table), _ptr(seq_lens), q_len, _ptr(o), _ptr(lse), B,
+        H_q, d_qk, d_v, page_size, max_pages, n_pages, n_sink, n_local, float(scale),
+        _ptr(workspace), workspace.numel(), _stream(stream)))
     return o, lse
 
 

@@ -175,13 +175,15 @@ def decode_page_table(seq_lens, page_size=BLOCK, seed=0, max_pages=None, permute
 
 
 def decode_inputs(seq_lens, H_q, d_qk, seed=0, device="cpu", page_size=BLOCK, permute=True,
-                  max_pages=None):
-    """q [B,H_q,d_qk] bf16; paged kv [n_pages,page_size,d_qk] bf16; page_table
-    [B,max_pages] int32 (device tensor); seq_lens [B] int32 (device tensor)."""
+                  max_pages=None, q_len=None):
+    """q [B,H_q,d_qk] bf16 ([B,q_len,H_q,d_qk] when q_len is given: several
+    query tokens per sequence); paged kv [n_pages,page_size,d_qk] bf16;
+    page_table [B,max_pages] int32 (device tensor); seq_lens [B] int32 (device
+    tensor)."""
     table, n_pages = decode_page_table(seq_lens, page_size, seed, max_pages, permute)
     g = _gen(seed, device)
     B = len(seq_lens)
-    q = _randn_bf16((B, H_q, d_qk), g, device)
+    q = _randn_bf16((B, H_q, d_qk) if q_len is None else (B, q_len, H_q, d_qk), g, device)
     kv = _randn_bf16((n_pages, page_size, d_qk), g, device)
     pt = torch.from_numpy(table).to(device)
     sl = torch.tensor(seq_lens, dtype=torch.int32, device=device)

@@ -65,7 +65,7 @@ enum {
 enum {
   LOZA_SSA_DEV_WAIT_TIMEOUT = 1,    /* a pipeline wait gave up; that CTA skipped its work      */
   LOZA_SSA_DEV_BAD_PAGE = 2,        /* page_table entry outside [0, n_pages); split skipped    */
-  LOZA_SSA_DEV_BAD_SEQLEN = 4,      /* decode seq_len < 1 or > max_pages * page_size           */
+  LOZA_SSA_DEV_BAD_SEQLEN = 4,      /* decode seq_len < q_len (1) or > max_pages * page_size   */
   LOZA_SSA_DEV_BAD_CU_SEQLENS = 8,  /* cu_seqlens not starting at 0, decreasing, or != total   */
 };
 
@@ -150,6 +150,33 @@ int loza_ssa_decode_selected(const void* q, const void* paged_kv, const int* pag
 /* Bytes of workspace loza_ssa_decode_selected needs (0 on invalid arguments). */
 size_t loza_ssa_decode_selected_workspace_size(int B, int H_q, int d_v, int n_sink, int n_local,
                                                int max_extra);
+
+/*
+ * Paged SSA decode with q_len query tokens per sequence (speculative or
+ * multi-token-prediction steps): the tokens of sequence b sit at positions
+ * t = seq_len[b] - q_len .. seq_len[b] - 1, and token t attends the keys
+ * J(t) = { j <= t : page(j) in W(page(t)) } -- the SSA mask of the QbitAI
+ * LoZA article's 1024-token window paragraph (one global block plus seven
+ * local blocks of 128 tokens) applied to each query position, so the tokens
+ * see each other causally and each has its own window.
+ *   q     : bf16 [B, q_len, H_q, d_qk]     o : bf16 [B, q_len, H_q, d_v]
+ *   lse   : fp32 [B, q_len, H_q]
+ *   q_len : >= 1, B * q_len <= 65535; every seq_len must be >= q_len (a
+ *           shorter one sets LOZA_SSA_DEV_BAD_SEQLEN in the device status
+ *           word and its rows come out as O = 0, LSE = -inf).
+ * workspace: at least loza_ssa_decode_mtp_workspace_size(B, q_len, H_q, d_v,
+ * n_sink, n_local) bytes.  Other arguments, layouts, ownership and statuses as
+ * for loza_ssa_decode (q_len = 1 gives the same result).
+ */
+int loza_ssa_decode_mtp(const void* q, const void* paged_kv, const int* page_table,
+                        const int* seq_lens, int q_len, void* o, float* lse, int B, int H_q,
+                        int d_qk, int d_v, int page_size, int max_pages, int n_pages, int n_sink,
+                        int n_local, float scale, void* workspace, size_t workspace_bytes,
+                        loza_ssa_stream_t stream);
+
+/* Bytes of workspace loza_ssa_decode_mtp needs (0 on invalid arguments). */
+size_t loza_ssa_decode_mtp_workspace_size(int B, int q_len, int H_q, int d_v, int n_sink,
+                                          int n_local);
 
 /* Static description of a status code (never NULL). */
 const char* loza_ssa_status_string(int status);

@@ -80,6 +80,26 @@ def test_decode_selected_workspace_size(L):
     assert api.loza_ssa_decode_selected_workspace_size(32, 128, 512, 1, 7, 4089) == 0
 
 
+def test_decode_mtp_workspace_size(L):
+    from block_sparse_streaming_ssa_b200 import loza_ssa as api
+    # q_len tokens per sequence: the workspace of B * q_len one-token rows
+    assert api.loza_ssa_decode_mtp_workspace_size(32, 2, 128, 512, 1, 7) == \
+        api.loza_ssa_decode_workspace_size(64, 128, 512, 1, 7)
+    assert api.loza_ssa_decode_mtp_workspace_size(32, 1, 128, 512, 1, 7) == \
+        api.loza_ssa_decode_workspace_size(32, 128, 512, 1, 7)
+    assert api.loza_ssa_decode_mtp_workspace_size(32, 0, 128, 512, 1, 7) == 0
+    assert api.loza_ssa_decode_mtp_workspace_size(40000, 2, 128, 512, 1, 7) == 0
+
+
+def test_decode_mtp_rejects_bad_q_len(L):
+    vp = ctypes.c_void_p
+    for q_len, B in ((0, 2), (2, 40000)):
+        rc = L.loza_ssa_decode_mtp(vp(0x1000), vp(0x1000), vp(0x1000), vp(0x1000), q_len,
+                                   vp(0x1000), vp(0x1000), B, 128, 576, 512, 128, 8, 16, 1, 7,
+                                   ctypes.c_float(0.04), vp(0x1000), 1 << 30, None)
+        assert rc == -2   # LOZA_SSA_ERR_SHAPE
+
+
 def test_decode_selected_rejects_missing_list(L):
     vp = ctypes.c_void_p
     rc = L.loza_ssa_decode_selected(vp(0x1000), vp(0x1000), vp(0x1000), vp(0x1000), None, 4,
