@@ -362,6 +362,99 @@ int oracle_ssa_decode_sel_rows(const void* q, const void* kv, int elt, const int
                      page_size, max_pages, n_pages, n_sink, n_local, scale, rows, n_rows, o, lse);
 }
 
+/*
+ * Backward pass of the dense SSA prefill: the gradients of a loss whose
+ * gradient with respect to O is dO.  Written from the definition of the
+ * forward pass above (softmax over J(i) of the scaled scores, "LoZA：ZigZag
+ * 稀疏注意力机制" §2.1), differentiated by the chain rule:
+ *
+ *   P_ij  = exp(s_ij - m_i) / l_i                      (j in J(i))
+ *   dP_ij = sum_c dO_ic v_jc                           (dL/dP_ij)
+ *   D_i   = sum_j P_ij dP_ij                           (= dO_i . O_i)
+ *   dS_ij = P_ij (dP_ij - D_i)                         (dL/ds_ij, softmax Jacobian)
+ *   dQ_i  = scale sum_j dS_ij k_j
+ *   dK_j  = scale sum_i dS_ij q_i                      (over the i with j in J(i))
+ *   dV_j  = sum_i P_ij dO_i
+ *
+ * q, k, dout: [B,H,L,dqk] / [B,H,L,dv] as for the forward; outputs float64
+ * dq [B,H,L,dqk], dk [B,H,L,dqk], dv [B,H,L,dv].  Planes (b, h) run in
+ * parallel; inside a plane rows are visited in order and dK, dV accumulate
+ * in that order.
+ */
+int oracle_ssa_prefill_bwd(const void* q, const void* k, const void* v, const void* dout, int elt,
+                           int64_t B, int64_t H, int64_t L, int dqk, int dv, int64_t blk,
+                           int64_t n_sink, int64_t n_local, double scale, double* dq, double* dk,
+                           double* dvv) {
+  int64_t cap = max_keys(L, blk, n_sink, n_local);
+  int err = 0;
+  memset(dk, 0, sizeof(double) * B * H * L * dqk);
+  memset(dvv, 0, sizeof(double) * B * H * L * dv);
+#pragma omp parallel
+  {
+    double* s_buf = (double*)malloc(sizeof(double) * cap);
+    double* dp_buf = (double*)malloc(sizeof(double) * cap);
+    int64_t* j_buf = (int64_t*)malloc(sizeof(int64_t) * cap);
+    double* qd = (double*)malloc(sizeof(double) * dqk);
+    double* gd = (double*)malloc(sizeof(double) * dv);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+      for (int64_t i = 0; i < L; ++i) {
+        const int64_t qrow = bh * L + i;
+        for (int c = 0; c < dqk; ++c) qd[c] = widen(q, qrow * dqk + c, elt);
+        for (int c = 0; c < dv; ++c) gd[c] = widen(dout, qrow * dv + c, elt);
+        /* scores over J(i) and the row max */
+        int64_t n = 0;
+        double m = -INFINITY;
+        const int64_t qb = i / blk;
+        for (int64_t j = 0; j <= i; ++j) {
+          if (!oracle_ssa_block_in_window(qb, j / blk, n_sink, n_local)) continue;
+          const int64_t krow = bh * L + j;
+          double dot = 0.0;
+          for (int c = 0; c < dqk; ++c) dot += qd[c] * widen(k, krow * dqk + c, elt);
+          s_buf[n] = scale * dot;
+          j_buf[n] = krow;
+          if (s_buf[n] > m) m = s_buf[n];
+          ++n;
+        }
+        if (n > cap) {
+#pragma omp atomic write
+          err = -3;
+          break;
+        }
+        /* P_ij, dP_ij and D_i */
+        double l = 0.0;
+        for (int64_t t = 0; t < n; ++t) l += exp(s_buf[t] - m);
+        double D = 0.0;
+        for (int64_t t = 0; t < n; ++t) {
+          s_buf[t] = exp(s_buf[t] - m) / l; /* now P_ij */
+          double dot = 0.0;
+          for (int c = 0; c < dv; ++c) dot += gd[c] * widen(v, j_buf[t] * dv + c, elt);
+          dp_buf[t] = dot;
+          D += s_buf[t] * dot;
+        }
+        /* dS_ij, then the three gradients */
+        for (int c = 0; c < dqk; ++c) dq[qrow * dqk + c] = 0.0;
+        for (int64_t t = 0; t < n; ++t) {
+          const double p = s_buf[t];
+          const double ds = p * (dp_buf[t] - D);
+          const int64_t krow = j_buf[t];
+          for (int c = 0; c < dqk; ++c) {
+            dq[qrow * dqk + c] += scale * ds * widen(k, krow * dqk + c, elt);
+            dk[krow * dqk + c] += scale * ds * qd[c];
+          }
+          for (int c = 0; c < dv; ++c) dvv[krow * dv + c] += p * gd[c];
+        }
+      }
+    }
+    free(s_buf);
+    free(dp_buf);
+    free(j_buf);
+    free(qd);
+    free(gd);
+  }
+  return err;
+}
+
 /* Threads the oracle's parallel regions use (for reporting the CPU baseline). */
 int oracle_ssa_num_threads(void) {
   int n = 1;

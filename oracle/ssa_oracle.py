@@ -84,6 +84,9 @@ def _load():
             vp, vp, i32, vp, vp, i64, i64, i64, i32, i32, i64, i64, i64, i64, i64, dbl, vp, i64,
             vp, vp]
         lib.oracle_ssa_decode_mtp_rows.restype = i32
+        lib.oracle_ssa_prefill_bwd.argtypes = [
+            vp, vp, vp, vp, i32, i64, i64, i64, i32, i32, i64, i64, i64, dbl, vp, vp, vp]
+        lib.oracle_ssa_prefill_bwd.restype = i32
         lib.oracle_ssa_num_threads.argtypes = []
         lib.oracle_ssa_num_threads.restype = i32
         _lib = lib
@@ -249,6 +252,29 @@ def decode_selected(q, kv, page_table, seq_lens, extra_pages, dv, page_size=128,
     return o, lse
 
 
+def prefill_bwd(q, k, v, dout, blk=128, n_sink=1, n_local=7, scale=None):
+    """Gradients (dq, dk, dv) of the dense SSA prefill for upstream gradient
+    dout = dL/dO, float64.  q, k: [B,H,L,dqk]; v, dout: [B,H,L,dv] (float64 or
+    bf16 bit patterns, all the same kind)."""
+    q, k, v, dout = (np.ascontiguousarray(a) for a in (q, k, v, dout))
+    B, H, L, dqk = q.shape
+    dv = v.shape[-1]
+    assert k.shape == q.shape and v.shape == (B, H, L, dv) and dout.shape == v.shape
+    elt = _elt(q)
+    assert _elt(k) == elt and _elt(v) == elt and _elt(dout) == elt
+    if scale is None:
+        scale = 1.0 / np.sqrt(dqk)
+    dq = np.empty((B, H, L, dqk))
+    dk = np.empty((B, H, L, dqk))
+    dvv = np.empty((B, H, L, dv))
+    rc = _load().oracle_ssa_prefill_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), elt, B, H, L, dqk,
+                                        dv, blk, n_sink, n_local, float(scale), _ptr(dq), _ptr(dk),
+                                        _ptr(dvv))
+    if rc:
+        raise ValueError(f"oracle prefill backward failed ({rc})")
+    return dq, dk, dvv
+
+
 def decode_mtp(q, kv, page_table, seq_lens, dv, page_size=128, n_sink=1, n_local=7, scale=None,
                rows=None):
     """Paged decode with q_len query tokens per sequence: q [B, q_len, Hq, dqk];
@@ -324,6 +350,28 @@ def brute_force_prefill(q, k, v, blk=128, n_sink=1, n_local=7, scale=None):
     o = np.einsum("...ij,...jc->...ic", p, v) / den
     lse = smax[..., 0] + np.log(den[..., 0])
     return o, lse
+
+
+def brute_force_prefill_bwd(q, k, v, dout, blk=128, n_sink=1, n_local=7, scale=None):
+    """Backward of brute_force_prefill with the materialised mask, numpy
+    float64, written as matrix products: P = softmax(masked S), dP = dO V^T,
+    dS = P * (dP - rowsum(P * dP)), dQ = scale dS K, dK = scale dS^T Q,
+    dV = P^T dO."""
+    q, k, v, dout = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(dout)
+    L, dqk = q.shape[-2:]
+    if scale is None:
+        scale = 1.0 / np.sqrt(dqk)
+    m = mask_matrix(L, blk, n_sink, n_local)
+    s = np.where(m, scale * np.einsum("...ic,...jc->...ij", q, k), -np.inf)
+    p = np.exp(s - s.max(axis=-1, keepdims=True))
+    p = np.where(m, p, 0.0)
+    p /= p.sum(axis=-1, keepdims=True)
+    dp = np.einsum("...ic,...jc->...ij", dout, v)
+    ds = p * (dp - (p * dp).sum(axis=-1, keepdims=True))
+    dq = scale * np.einsum("...ij,...jc->...ic", ds, k)
+    dk = scale * np.einsum("...ij,...ic->...jc", ds, q)
+    dvv = np.einsum("...ij,...ic->...jc", p, dout)
+    return dq, dk, dvv
 
 
 def brute_force_decode(q, kv, page_table, seq_lens, dv, page_size=128, n_sink=1, n_local=7,

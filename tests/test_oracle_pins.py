@@ -442,3 +442,74 @@ def test_decode_mtp_rejects_short_sequence():
     q, kv, pt, sl = _mtp_case(25, [2, 40], 3)
     with pytest.raises(ValueError):
         orc.decode_mtp(q, kv, pt, sl, dv=16, page_size=8, n_sink=1, n_local=3)
+
+
+# --- backward of the dense prefill (gradients of a loss with dL/dO = dout)
+
+def _bwd_case(seed, B=1, H=2, L=13, dqk=5, dv=3):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((B, H, L, dqk)), rng.standard_normal((B, H, L, dqk)),
+            rng.standard_normal((B, H, L, dv)), rng.standard_normal((B, H, L, dv)))
+
+
+def test_prefill_bwd_matches_finite_differences():
+    """Central differences of the forward oracle's loss sum(O * dout), every
+    element of q, k and v (independent of the backward's formulas)."""
+    q, k, v, g = _bwd_case(31)
+    kw = dict(blk=4, n_sink=1, n_local=2, scale=0.7)
+    dq, dk, dvv = orc.prefill_bwd(q, k, v, g, **kw)
+
+    def loss(qq, kk, vv):
+        o, _ = orc.prefill(qq, kk, vv, **kw)
+        return float((o * g).sum())
+
+    eps = 1e-5
+    for name, x, grad in (("q", q, dq), ("k", k, dk), ("v", v, dvv)):
+        num = np.empty_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = [xp if n == name else a for n, a in (("q", q), ("k", k), ("v", v))]
+            args_m = [xm if n == name else a for n, a in (("q", q), ("k", k), ("v", v))]
+            num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+        np.testing.assert_allclose(grad, num, atol=1e-7, err_msg=f"d{name}")
+
+
+def test_prefill_bwd_matches_masked_brute_force():
+    for seed, (n_sink, n_local) in enumerate([(1, 3), (2, 2), (0, 1), (1, 7)]):
+        q, k, v, g = _bwd_case(40 + seed, B=2, H=2, L=50, dqk=8, dv=6)
+        got = orc.prefill_bwd(q, k, v, g, blk=8, n_sink=n_sink, n_local=n_local, scale=0.4)
+        ref = orc.brute_force_prefill_bwd(q, k, v, g, blk=8, n_sink=n_sink, n_local=n_local,
+                                          scale=0.4)
+        for a, b in zip(got, ref):
+            np.testing.assert_allclose(a, b, atol=1e-12)
+
+
+def test_prefill_bwd_short_sequence_is_causal_autograd():
+    """L <= window: SSA is causal attention, whose gradients torch autograd
+    computes in float64."""
+    import torch
+    q, k, v, g = _bwd_case(50, B=1, H=3, L=30, dqk=7, dv=5)
+    dq, dk, dvv = orc.prefill_bwd(q, k, v, g, blk=8, n_sink=1, n_local=3, scale=0.5)
+    tq, tk, tv = (torch.tensor(a, requires_grad=True) for a in (q, k, v))
+    s = 0.5 * tq @ tk.transpose(-1, -2)
+    causal = torch.ones(30, 30, dtype=torch.bool).tril()
+    o = torch.softmax(s.masked_fill(~causal, float("-inf")), dim=-1) @ tv
+    (o * torch.tensor(g)).sum().backward()
+    np.testing.assert_allclose(dq, tq.grad.numpy(), atol=1e-12)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), atol=1e-12)
+    np.testing.assert_allclose(dvv, tv.grad.numpy(), atol=1e-12)
+
+
+def test_prefill_bwd_invariants():
+    q, k, v, g = _bwd_case(60, B=1, H=2, L=40, dqk=6, dv=4)
+    kw = dict(blk=8, n_sink=1, n_local=2, scale=0.6)
+    _, dk, _ = orc.prefill_bwd(q, k, v, g, **kw)
+    # each row's dS sums to zero, so dK summed over the keys of a plane is 0
+    np.testing.assert_allclose(dk.sum(axis=2), 0.0, atol=1e-12)
+    # a value row shared by every key makes O independent of the scores
+    v_const = np.broadcast_to(v[:, :, :1], v.shape).copy()
+    dq, dk, _ = orc.prefill_bwd(q, k, v_const, g, **kw)
+    np.testing.assert_allclose(dq, 0.0, atol=1e-12)
+    np.testing.assert_allclose(dk, 0.0, atol=1e-12)
