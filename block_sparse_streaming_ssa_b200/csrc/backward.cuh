@@ -1,0 +1,802 @@
+// backward.cuh -- gradients of the SSA prefill on sm_100a (dense layout,
+// d_qk = d_v = DIM in {64, 128}).
+//
+// For a loss with upstream gradient dO = dL/dO, differentiating the masked
+// softmax attention of "LoZA：ZigZag稀疏注意力机制" §2.1 over the SSA key sets
+// J(i) (QbitAI LoZA article, 1024-token window paragraph) gives, with
+// P_ij = exp(s_ij - LSE_i) for j in J(i) and s_ij = scale * q_i . k_j:
+//
+//     D_i   = sum_c dO_ic O_ic                 (= sum_j P_ij dP_ij)
+//     dP_ij = dO_i . v_j
+//     dS_ij = P_ij (dP_ij - D_i)
+//     dQ_i  = scale sum_j dS_ij k_j
+//     dK_j  = scale sum_i dS_ij q_i            (over the i with j in J(i))
+//     dV_j  = sum_i P_ij dO_i
+//
+// Three kernels:
+//   ssa_bwd_preprocess_kernel  D_i for every row (CUDA cores; reads O and dO once).
+//   ssa_bwd_dq_kernel          per query block: for each key tile of its window
+//                              S = Q K^T and dP = dO V^T on tcgen05 into TMEM,
+//                              dS in registers, dQ += dS K as a TMEM x smem MMA.
+//   ssa_bwd_dkdv_kernel        per key block: for each query block whose window
+//                              holds it, S^T = K Q^T and dP^T = V dO^T (TMEM lanes =
+//                              keys), P^T and dS^T in registers, then
+//                              dV += P^T dO and dK += dS^T Q as TMEM x smem MMAs.
+//                              The sink blocks are seen by every later query
+//                              block, so their query lists are cut into chunks
+//                              of kSinkChunk blocks whose fp32 partial dK / dV
+//                              ssa_bwd_sink_reduce_kernel adds up.
+// LSE_i = ln sum_j exp(s_ij) comes from the forward pass, so no row max is
+// recomputed: P is exact up to rounding and dS goes to the MMAs as bf16.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+#include "schedule.cuh"
+
+namespace loza {
+
+constexpr int kBwdThreads = 320;     // warps 0-7 compute, 8 TMA producer, 9 MMA issuer
+constexpr int kBwdComputeThreads = 256;
+constexpr int kSinkChunk = 8;        // query blocks per sink work item
+
+struct BwdParams {
+  const float* lse;        // [planes * L], natural log, from the forward pass
+  const float* dsum;       // [planes * L], D_i
+  __nv_bfloat16* dq;       // [planes, L, DIM]
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  float* part;             // sink partials: [planes * sink_items][2][128][DIM] (dK then dV)
+  int L, planes, n_sink, n_local;
+  int nb;                  // query / key blocks per plane
+  int sink_items;          // sink work items per plane
+  float scale, scale_log2;
+};
+
+// Sink work items of one plane: key block j < min(n_sink, nb) is seen by
+// query blocks j .. nb-1, cut into chunks of kSinkChunk.
+__host__ __device__ __forceinline__ int bwd_sink_chunks(int j, int nb) {
+  return (nb - j + kSinkChunk - 1) / kSinkChunk;
+}
+__host__ __device__ __forceinline__ int bwd_sink_items(int n_sink, int nb) {
+  int n = 0;
+  for (int j = 0; j < n_sink && j < nb; ++j) n += bwd_sink_chunks(j, nb);
+  return n;
+}
+
+struct BwdKItem {
+  int plane, kb;     // key block
+  int q_lo, q_hi;    // query blocks q_lo .. q_hi (inclusive)
+  int slot;          // sink partial slot, -1 for a regular key block (written directly)
+};
+
+__device__ __forceinline__ BwdKItem bwd_kv_item(const BwdParams& p, int item) {
+  const int per_plane = p.sink_items + (p.nb > p.n_sink ? p.nb - p.n_sink : 0);
+  BwdKItem w;
+  w.plane = item / per_plane;
+  int r = item - w.plane * per_plane;
+  if (r < p.sink_items) {
+    w.slot = w.plane * p.sink_items + r;
+    int j = 0;
+    while (r >= bwd_sink_chunks(j, p.nb)) {
+      r -= bwd_sink_chunks(j, p.nb);
+      ++j;
+    }
+    w.kb = j;
+    w.q_lo = j + r * kSinkChunk;
+    w.q_hi = min(p.nb - 1, w.q_lo + kSinkChunk - 1);
+  } else {
+    w.slot = -1;
+    w.kb = p.n_sink + (r - p.sink_items);
+    w.q_lo = w.kb;
+    w.q_hi = min(p.nb - 1, w.kb + p.n_local - 1);
+  }
+  return w;
+}
+
+// ---------------------------------------------------------------- D_i
+
+// D_i = dO_i . O_i for every row; DIM / 8 lanes share a row (16 bytes each).
+template <int DIM>
+__global__ void __launch_bounds__(256) ssa_bwd_preprocess_kernel(const __nv_bfloat16* o,
+                                                                  const __nv_bfloat16* dout,
+                                                                  float* dsum, long long rows) {
+  constexpr int LPR = DIM / 8;  // lanes per row
+  constexpr int RPW = 32 / LPR;  // rows per warp step
+  const int lane = threadIdx.x & 31;
+  const long long warp = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
+  const long long n_warps = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long r0 = warp * RPW; r0 < rows; r0 += n_warps * RPW) {
+    const long long r = r0 + lane / LPR;
+    float acc = 0.f;
+    if (r < rows) {
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + r * DIM) + (lane % LPR));
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(dout + r * DIM) + (lane % LPR));
+      const __nv_bfloat162* ah = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* bh = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 x = __bfloat1622float2(ah[e]), y = __bfloat1622float2(bh[e]);
+        acc = fmaf(x.x, y.x, acc);
+        acc = fmaf(x.y, y.y, acc);
+      }
+    }
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (r < rows && lane % LPR == 0) dsum[r] = acc;
+  }
+}
+
+// ------------------------------------------------------------------ dQ
+
+template <int DIM>
+struct BwdDqLayout {
+  static constexpr int CH = DIM / 64;
+  static constexpr int CHUNK = 128 * 128;  // one swizzled [128 rows x 64 bf16] box
+  static constexpr int TILE = CH * CHUNK;  // [128 rows x DIM]
+  static constexpr int KST = 2, VST = 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_DO = TILE;
+  static constexpr int OFF_K = 2 * TILE;
+  static constexpr int OFF_V = OFF_K + KST * TILE;
+  static constexpr int OFF_BAR = OFF_V + VST * TILE;
+  // TMEM columns
+  static constexpr int TM_S = 0, TM_DP = 128, TM_DS = 256, TM_DQ = 384;
+  // barriers
+  static constexpr int B_QD_FULL = 0, B_QD_EMPTY = 1;
+  static constexpr int B_K_FULL = 2, B_K_EMPTY = B_K_FULL + KST;
+  static constexpr int B_V_FULL = B_K_EMPTY + KST, B_V_EMPTY = B_V_FULL + VST;
+  static constexpr int B_S_FULL = B_V_EMPTY + VST;    // S and dP of a tile issued (commit)
+  static constexpr int B_SDP_FREE = B_S_FULL + 1;     // compute warps have loaded S and dP
+  static constexpr int B_DS_FULL = B_SDP_FREE + 1;    // dS written to TMEM
+  static constexpr int B_DS_FREE = B_DS_FULL + 1;     // dQ MMA of the tile done
+  static constexpr int B_DQ_FULL = B_DS_FREE + 1;     // the item's last dQ MMA done
+  static constexpr int B_DQ_EMPTY = B_DQ_FULL + 1;    // epilogue has read dQ
+  static constexpr int B_DRAIN = B_DQ_EMPTY + 1;
+  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;  // [0] tmem base, [1] abort
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+template <int DIM>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    ssa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
+  using Lay = BwdDqLayout<DIM>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  auto bar = [&](int i) -> uint32_t { return sb + Lay::OFF_BAR + 8 * i; };
+  int* status = &g_loza_status;
+  const int total_items = p.planes * p.nb;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(Lay::B_QD_FULL), 1);
+    mbar_init(bar(Lay::B_QD_EMPTY), 1);
+    for (int s = 0; s < Lay::KST; ++s) {
+      mbar_init(bar(Lay::B_K_FULL + s), 1);
+      mbar_init(bar(Lay::B_K_EMPTY + s), 1);
+    }
+    for (int s = 0; s < Lay::VST; ++s) {
+      mbar_init(bar(Lay::B_V_FULL + s), 1);
+      mbar_init(bar(Lay::B_V_EMPTY + s), 1);
+    }
+    mbar_init(bar(Lay::B_S_FULL), 1);
+    mbar_init(bar(Lay::B_SDP_FREE), kBwdComputeThreads);
+    mbar_init(bar(Lay::B_DS_FULL), kBwdComputeThreads);
+    mbar_init(bar(Lay::B_DS_FREE), 1);
+    mbar_init(bar(Lay::B_DQ_FULL), 1);
+    mbar_init(bar(Lay::B_DQ_EMPTY), kBwdComputeThreads);
+    mbar_init(bar(Lay::B_DRAIN), 1);
+    misc[1] = 0;
+    fence_barrier_init();
+  }
+  if (warp == 8 && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+    prefetch_tensormap(&tm_do);
+  }
+  if (warp == 9) {
+    tmem_alloc(sb + Lay::OFF_MISC, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int g = 0, it = 0, qd_issued = 0;
+      int k_issued[Lay::KST] = {}, v_issued[Lay::VST] = {};
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++it) {
+        const int plane = item / p.nb, qb = item - plane * p.nb;
+        const TileRange tr = tile_range(qb, p.n_sink, p.n_local);
+        if (it > 0 && !mbar_wait(bar(Lay::B_QD_EMPTY), (it - 1) & 1, abort_flag, status, 1)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(bar(Lay::B_QD_FULL), 2 * Lay::TILE);
+        ++qd_issued;
+#pragma unroll
+        for (int c = 0; c < Lay::CH; ++c) {
+          tma_load_3d(sb + Lay::OFF_Q + c * Lay::CHUNK, &tm_q, bar(Lay::B_QD_FULL), c * 64,
+                      qb * 128, plane);
+          tma_load_3d(sb + Lay::OFF_DO + c * Lay::CHUNK, &tm_do, bar(Lay::B_QD_FULL), c * 64,
+                      qb * 128, plane);
+        }
+        for (int t = 0; t < tr.count; ++t, ++g) {
+          const int row = tile_block(tr, t) * 128;
+          const int st = g % Lay::KST, use = g / Lay::KST;
+          if (use > 0 &&
+              !mbar_wait(bar(Lay::B_K_EMPTY + st), (use - 1) & 1, abort_flag, status, 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(Lay::B_K_FULL + st), Lay::TILE);
+          ++k_issued[st];
+#pragma unroll
+          for (int c = 0; c < Lay::CH; ++c)
+            tma_load_3d(sb + Lay::OFF_K + st * Lay::TILE + c * Lay::CHUNK, &tm_k,
+                        bar(Lay::B_K_FULL + st), c * 64, row, plane);
+          const int vs = g % Lay::VST, vuse = g / Lay::VST;
+          if (vuse > 0 &&
+              !mbar_wait(bar(Lay::B_V_EMPTY + vs), (vuse - 1) & 1, abort_flag, status, 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(Lay::B_V_FULL + vs), Lay::TILE);
+          ++v_issued[vs];
+#pragma unroll
+          for (int c = 0; c < Lay::CH; ++c)
+            tma_load_3d(sb + Lay::OFF_V + vs * Lay::TILE + c * Lay::CHUNK, &tm_v,
+                        bar(Lay::B_V_FULL + vs), c * 64, row, plane);
+        }
+      }
+      if (!ok) {
+        // let the copies in flight land before the CTA's shared memory goes away
+        for (int s = 0; s < Lay::KST; ++s)
+          if (k_issued[s] > 0) mbar_wait_drain(bar(Lay::B_K_FULL + s), (k_issued[s] - 1) & 1);
+        for (int s = 0; s < Lay::VST; ++s)
+          if (v_issued[s] > 0) mbar_wait_drain(bar(Lay::B_V_FULL + s), (v_issued[s] - 1) & 1);
+        if (qd_issued > 0) mbar_wait_drain(bar(Lay::B_QD_FULL), (qd_issued - 1) & 1);
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    // Order: S/dP of tile 0, then for every tile g: S/dP of tile g+1 (as soon
+    // as the compute warps have loaded tile g's S and dP), then dQ += dS_g K_g.
+    if (lane == 0) {
+      const uint32_t id_s = idesc_bf16_f32(128, 128, false);
+      const uint32_t id_q = idesc_bf16_f32(128, DIM, true);
+      bool ok = true;
+      // cursor over (item, tile) for the S/dP MMAs
+      int a_item = blockIdx.x, a_it = 0, a_t = 0, a_g = 0;
+      auto issue_sdp = [&]() -> bool {
+        const int plane = a_item / p.nb, qb = a_item - plane * p.nb;
+        (void)plane;
+        const TileRange tr = tile_range(qb, p.n_sink, p.n_local);
+        if (a_t == 0 && !mbar_wait(bar(Lay::B_QD_FULL), a_it & 1, abort_flag, status, 1))
+          return false;
+        const int st = a_g % Lay::KST, vs = a_g % Lay::VST;
+        if (a_g > 0 && !mbar_wait(bar(Lay::B_SDP_FREE), (a_g - 1) & 1, abort_flag, status, 1))
+          return false;
+        if (!mbar_wait(bar(Lay::B_K_FULL + st), (a_g / Lay::KST) & 1, abort_flag, status, 1) ||
+            !mbar_wait(bar(Lay::B_V_FULL + vs), (a_g / Lay::VST) & 1, abort_flag, status, 1))
+          return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < DIM / 16; ++kk) {
+          const uint32_t koff = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
+          mma_ss(tmem + Lay::TM_S, sdesc_sw128(sb + Lay::OFF_Q + koff, 16, 1024),
+                 sdesc_sw128(sb + Lay::OFF_K + st * Lay::TILE + koff, 16, 1024), id_s,
+                 kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < DIM / 16; ++kk) {
+          const uint32_t koff = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
+          mma_ss(tmem + Lay::TM_DP, sdesc_sw128(sb + Lay::OFF_DO + koff, 16, 1024),
+                 sdesc_sw128(sb + Lay::OFF_V + vs * Lay::TILE + koff, 16, 1024), id_s,
+                 kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(Lay::B_S_FULL));
+        mma_commit(bar(Lay::B_V_EMPTY + vs));
+        if (a_t == tr.count - 1) {
+          mma_commit(bar(Lay::B_QD_EMPTY));
+          a_t = 0;
+          ++a_it;
+          a_item += gridDim.x;
+        } else {
+          ++a_t;
+        }
+        ++a_g;
+        return true;
+      };
+      if (a_item < total_items) ok = issue_sdp();
+      int b_it = 0, b_g = 0;
+      for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++b_it) {
+        const int qb = item % p.nb;
+        const TileRange tr = tile_range(qb, p.n_sink, p.n_local);
+        for (int t = 0; ok && t < tr.count; ++t, ++b_g) {
+          if (a_item < total_items && !(ok = issue_sdp())) break;
+          const int st = b_g % Lay::KST;
+          if (!(ok = mbar_wait(bar(Lay::B_DS_FULL), b_g & 1, abort_flag, status, 1))) break;
+          if (t == 0 && b_it > 0 &&
+              !(ok = mbar_wait(bar(Lay::B_DQ_EMPTY), (b_it - 1) & 1, abort_flag, status, 1)))
+            break;
+          tc_fence_after();
+          // dQ += dS K: dS (bf16 pairs) in TMEM columns TM_DS.., K MN-major
+          // (keys 16kk .. 16kk+15 of each 64-column box are 2048 bytes in)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + Lay::TM_DQ, tmem + Lay::TM_DS + kk * 8,
+                   sdesc_sw128(sb + Lay::OFF_K + st * Lay::TILE + kk * 2048, Lay::CHUNK, 1024),
+                   id_q, (t > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(Lay::B_DS_FREE));
+          mma_commit(bar(Lay::B_K_EMPTY + st));
+          if (t == tr.count - 1) mma_commit(bar(Lay::B_DQ_FULL));
+        }
+      }
+      mma_commit(bar(Lay::B_DRAIN));
+      mbar_wait_drain(bar(Lay::B_DRAIN), 0);
+    }
+  } else {
+    // ------------------------------------------------------- compute warps
+    const int wg = warp >> 2;                                      // key-column half
+    const int row = threadIdx.x & 127;                             // query row = TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const int col0 = wg * 64;
+    const float sl2 = p.scale_log2;
+    int g = 0, it = 0;
+    for (int item = blockIdx.x; item < total_items; item += gridDim.x, ++it) {
+      const int plane = item / p.nb, qb = item - plane * p.nb;
+      const TileRange tr = tile_range(qb, p.n_sink, p.n_local);
+      const int r_in_seq = qb * 128 + row;
+      const bool valid = r_in_seq < p.L;
+      const size_t grow = (size_t)plane * p.L + r_in_seq;
+      // rows past L: zero Q and dO rows (TMA fill), and P = 0 here
+      const float lse2 = valid ? __ldg(p.lse + grow) * 1.4426950408889634f : INFINITY;
+      const float dsum = valid ? __ldg(p.dsum + grow) : 0.f;
+      bool ok = true;
+      for (int t = 0; t < tr.count; ++t, ++g) {
+        if (!mbar_wait(bar(Lay::B_S_FULL), g & 1, abort_flag, status, 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const bool diag = (t == tr.count - 1);
+        uint32_t pk[32];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t sr[32], dr[32];
+          tmem_ld32(tmem + lane_base + Lay::TM_S + col0 + h * 32, sr);
+          tmem_ld32(tmem + lane_base + Lay::TM_DP + col0 + h * 32, dr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const int key0 = col0 + h * 32 + c;
+            float p0 = ex2_approx(__uint_as_float(sr[c]) * sl2 - lse2);
+            float p1 = ex2_approx(__uint_as_float(sr[c + 1]) * sl2 - lse2);
+            if (diag && key0 > row) p0 = 0.f;
+            if (diag && key0 + 1 > row) p1 = 0.f;
+            const float ds0 = p0 * (__uint_as_float(dr[c]) - dsum);
+            const float ds1 = p1 * (__uint_as_float(dr[c + 1]) - dsum);
+            pk[h * 16 + c / 2] = pack_bf16x2(ds0, ds1);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar(Lay::B_SDP_FREE));
+        // the previous tile's dQ MMA has read the dS columns
+        if (g > 0 && !mbar_wait(bar(Lay::B_DS_FREE), (g - 1) & 1, abort_flag, status, 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        tmem_st32(tmem + lane_base + Lay::TM_DS + col0 / 2, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(Lay::B_DS_FULL));
+      }
+      if (!ok) break;
+      // epilogue: dQ = scale * acc, bf16
+      if (!mbar_wait(bar(Lay::B_DQ_FULL), it & 1, abort_flag, status, 1)) break;
+      tc_fence_after();
+      constexpr int OH = DIM / 2;
+      uint32_t orr[OH / 32][32];
+#pragma unroll
+      for (int ch = 0; ch < OH / 32; ++ch)
+        tmem_ld32(tmem + lane_base + Lay::TM_DQ + wg * OH + ch * 32, orr[ch]);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(Lay::B_DQ_EMPTY));
+      if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(p.dq + grow * DIM + wg * OH);
+#pragma unroll
+        for (int ch = 0; ch < OH / 32; ++ch)
+#pragma unroll
+          for (int v = 0; v < 4; v += 2) {
+            uint32_t w8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              w8[e] = pack_bf16x2(__uint_as_float(orr[ch][8 * v + 2 * e]) * p.scale,
+                                  __uint_as_float(orr[ch][8 * v + 2 * e + 1]) * p.scale);
+            st_global_v8(dst + ch * 4 + v, w8);
+          }
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- dK, dV
+
+template <int DIM>
+struct BwdKvLayout {
+  static constexpr int CH = DIM / 64;
+  static constexpr int CHUNK = 128 * 128;
+  static constexpr int TILE = CH * CHUNK;
+  static constexpr int QST = 2;                    // (Q, dO) ring depth
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = TILE;
+  static constexpr int OFF_Q = 2 * TILE;           // QST x [Q | dO]
+  static constexpr int OFF_ROW = OFF_Q + QST * 2 * TILE;  // float [2 steps][2: lse2, D][128]
+  static constexpr int OFF_BAR = OFF_ROW + 2 * 2 * 128 * 4;
+  // TMEM: S^T, dP^T (P^T / dS^T as bf16 pairs over their first 64 columns), dV, dK
+  static constexpr int TM_ST = 0, TM_DPT = 128, TM_DV = 256, TM_DK = 256 + DIM;
+  static_assert(TM_DK + DIM <= 512, "TMEM");
+  // barriers
+  static constexpr int B_KV_FULL = 0, B_KV_EMPTY = 1;
+  static constexpr int B_Q_FULL = 2, B_Q_EMPTY = B_Q_FULL + QST;
+  static constexpr int B_ST_FULL = B_Q_EMPTY + QST;  // S^T and dP^T issued (commit)
+  static constexpr int B_SYNC_A = B_ST_FULL + 1;     // compute warps: the step's rows staged
+  static constexpr int B_SYNC_B = B_SYNC_A + 1;      // compute warps: S^T, dP^T all read
+  static constexpr int B_PDS_FULL = B_SYNC_B + 1;    // P^T and dS^T written
+  static constexpr int B_PDS_FREE = B_PDS_FULL + 1;  // dV, dK MMAs of the step done
+  static constexpr int B_ACC_FULL = B_PDS_FREE + 1;  // the item's last dV, dK MMAs done
+  static constexpr int B_ACC_EMPTY = B_ACC_FULL + 1; // epilogue has read dV, dK
+  static constexpr int B_DRAIN = B_ACC_EMPTY + 1;
+  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+template <int DIM>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    ssa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
+  using Lay = BwdKvLayout<DIM>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  auto bar = [&](int i) -> uint32_t { return sb + Lay::OFF_BAR + 8 * i; };
+  int* status = &g_loza_status;
+  const int per_plane = p.sink_items + (p.nb > p.n_sink ? p.nb - p.n_sink : 0);
+  const int total_items = p.planes * per_plane;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(Lay::B_KV_FULL), 1);
+    mbar_init(bar(Lay::B_KV_EMPTY), 1);
+    for (int s = 0; s < Lay::QST; ++s) {
+      mbar_init(bar(Lay::B_Q_FULL + s), 1);
+      mbar_init(bar(Lay::B_Q_EMPTY + s), 1);
+    }
+    mbar_init(bar(Lay::B_ST_FULL), 1);
+    mbar_init(bar(Lay::B_SYNC_A), kBwdComputeThreads);
+    mbar_init(bar(Lay::B_SYNC_B), kBwdComputeThreads);
+    mbar_init(bar(Lay::B_PDS_FULL), kBwdComputeThreads);
+    mbar_init(bar(Lay::B_PDS_FREE), 1);
+    mbar_init(bar(Lay::B_ACC_FULL), 1);
+    mbar_init(bar(Lay::B_ACC_EMPTY), kBwdComputeThreads);
+    mbar_init(bar(Lay::B_DRAIN), 1);
+    misc[1] = 0;
+    fence_barrier_init();
+  }
+  if (warp == 8 && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+    prefetch_tensormap(&tm_do);
+  }
+  if (warp == 9) {
+    tmem_alloc(sb + Lay::OFF_MISC, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int s = 0, it = 0, kv_issued = 0;
+      int q_issued[Lay::QST] = {};
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++it) {
+        const BwdKItem w = bwd_kv_item(p, item);
+        if (it > 0 && !mbar_wait(bar(Lay::B_KV_EMPTY), (it - 1) & 1, abort_flag, status, 1)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(bar(Lay::B_KV_FULL), 2 * Lay::TILE);
+        ++kv_issued;
+#pragma unroll
+        for (int c = 0; c < Lay::CH; ++c) {
+          tma_load_3d(sb + Lay::OFF_K + c * Lay::CHUNK, &tm_k, bar(Lay::B_KV_FULL), c * 64,
+                      w.kb * 128, w.plane);
+          tma_load_3d(sb + Lay::OFF_V + c * Lay::CHUNK, &tm_v, bar(Lay::B_KV_FULL), c * 64,
+                      w.kb * 128, w.plane);
+        }
+        for (int qi = w.q_lo; qi <= w.q_hi; ++qi, ++s) {
+          const int st = s % Lay::QST, use = s / Lay::QST;
+          if (use > 0 &&
+              !mbar_wait(bar(Lay::B_Q_EMPTY + st), (use - 1) & 1, abort_flag, status, 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(Lay::B_Q_FULL + st), 2 * Lay::TILE);
+          ++q_issued[st];
+          const uint32_t base = sb + Lay::OFF_Q + st * 2 * Lay::TILE;
+#pragma unroll
+          for (int c = 0; c < Lay::CH; ++c) {
+            tma_load_3d(base + c * Lay::CHUNK, &tm_q, bar(Lay::B_Q_FULL + st), c * 64, qi * 128,
+                        w.plane);
+            tma_load_3d(base + Lay::TILE + c * Lay::CHUNK, &tm_do, bar(Lay::B_Q_FULL + st),
+                        c * 64, qi * 128, w.plane);
+          }
+        }
+      }
+      if (!ok) {
+        for (int st = 0; st < Lay::QST; ++st)
+          if (q_issued[st] > 0) mbar_wait_drain(bar(Lay::B_Q_FULL + st), (q_issued[st] - 1) & 1);
+        if (kv_issued > 0) mbar_wait_drain(bar(Lay::B_KV_FULL), (kv_issued - 1) & 1);
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t id_s = idesc_bf16_f32(128, 128, false);   // M = keys, N = queries
+      const uint32_t id_a = idesc_bf16_f32(128, DIM, true);    // dV, dK: B = dO / Q, MN-major
+      int s = 0, it = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++it) {
+        const BwdKItem w = bwd_kv_item(p, item);
+        if (!(ok = mbar_wait(bar(Lay::B_KV_FULL), it & 1, abort_flag, status, 1))) break;
+        for (int qi = w.q_lo; qi <= w.q_hi; ++qi, ++s) {
+          const int st = s % Lay::QST;
+          const uint32_t qbase = sb + Lay::OFF_Q + st * 2 * Lay::TILE;
+          // S^T / dP^T overwrite the P^T / dS^T columns the previous step's MMAs read
+          if ((s > 0 &&
+               !(ok = mbar_wait(bar(Lay::B_PDS_FREE), (s - 1) & 1, abort_flag, status, 1))) ||
+              !(ok = mbar_wait(bar(Lay::B_Q_FULL + st), (s / Lay::QST) & 1, abort_flag, status,
+                               1)))
+            break;
+          tc_fence_after();
+          // S^T = K Q^T, dP^T = V dO^T (all operands K-major: rows x DIM boxes)
+#pragma unroll
+          for (int kk = 0; kk < DIM / 16; ++kk) {
+            const uint32_t koff = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
+            mma_ss(tmem + Lay::TM_ST, sdesc_sw128(sb + Lay::OFF_K + koff, 16, 1024),
+                   sdesc_sw128(qbase + koff, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < DIM / 16; ++kk) {
+            const uint32_t koff = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
+            mma_ss(tmem + Lay::TM_DPT, sdesc_sw128(sb + Lay::OFF_V + koff, 16, 1024),
+                   sdesc_sw128(qbase + Lay::TILE + koff, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(Lay::B_ST_FULL));
+          if (!(ok = mbar_wait(bar(Lay::B_PDS_FULL), s & 1, abort_flag, status, 1))) break;
+          const bool first = (qi == w.q_lo);
+          if (first && it > 0 &&
+              !(ok = mbar_wait(bar(Lay::B_ACC_EMPTY), (it - 1) & 1, abort_flag, status, 1)))
+            break;
+          tc_fence_after();
+          // dV += P^T dO, dK += dS^T Q: A = P^T / dS^T in TMEM (keys x queries,
+          // bf16 pairs), B = dO / Q MN-major (queries 16kk .. 16kk+15 of each
+          // 64-column box are 2048 bytes in)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + Lay::TM_DV, tmem + Lay::TM_ST + kk * 8,
+                   sdesc_sw128(qbase + Lay::TILE + kk * 2048, Lay::CHUNK, 1024), id_a,
+                   (!first || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + Lay::TM_DK, tmem + Lay::TM_DPT + kk * 8,
+                   sdesc_sw128(qbase + kk * 2048, Lay::CHUNK, 1024), id_a,
+                   (!first || kk > 0) ? 1u : 0u);
+          mma_commit(bar(Lay::B_PDS_FREE));
+          mma_commit(bar(Lay::B_Q_EMPTY + st));
+          if (qi == w.q_hi) {
+            mma_commit(bar(Lay::B_ACC_FULL));
+            mma_commit(bar(Lay::B_KV_EMPTY));
+          }
+        }
+      }
+      mma_commit(bar(Lay::B_DRAIN));
+      mbar_wait_drain(bar(Lay::B_DRAIN), 0);
+    }
+  } else {
+    // ------------------------------------------------------- compute warps
+    const int wg = warp >> 2;                                      // query-column half
+    const int r = threadIdx.x & 127;                               // key row = TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const int col0 = wg * 64;
+    const float sl2 = p.scale_log2;
+    float* rows_smem = reinterpret_cast<float*>(smem + Lay::OFF_ROW);
+    int s = 0, it = 0;
+    for (int item = blockIdx.x; item < total_items; item += gridDim.x, ++it) {
+      const BwdKItem w = bwd_kv_item(p, item);
+      const int key = w.kb * 128 + r;
+      bool ok = true;
+      for (int qi = w.q_lo; qi <= w.q_hi; ++qi, ++s) {
+        // stage lse2 and D of the step's 128 queries (rows past L: 0, harmless:
+        // their Q and dO rows are zero, so their dS^T and dV terms vanish)
+        float* lse_s = rows_smem + (s & 1) * 256;
+        float* d_s = lse_s + 128;
+        if (wg == 0) {
+          const int qrow = qi * 128 + r;
+          const size_t gq = (size_t)w.plane * p.L + qrow;
+          lse_s[r] = qrow < p.L ? __ldg(p.lse + gq) * 1.4426950408889634f : 0.f;
+          d_s[r] = qrow < p.L ? __ldg(p.dsum + gq) : 0.f;
+        }
+        mbar_arrive(bar(Lay::B_SYNC_A));
+        if (!mbar_wait(bar(Lay::B_SYNC_A), s & 1, abort_flag, status, 1) ||
+            !mbar_wait(bar(Lay::B_ST_FULL), s & 1, abort_flag, status, 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const bool diag = (qi == w.kb);
+        uint32_t pk[32], dk_[32];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t st_r[32], dp_r[32];
+          tmem_ld32(tmem + lane_base + Lay::TM_ST + col0 + h * 32, st_r);
+          tmem_ld32(tmem + lane_base + Lay::TM_DPT + col0 + h * 32, dp_r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const int qc = col0 + h * 32 + c;  // query column within the block
+            float p0 = ex2_approx(__uint_as_float(st_r[c]) * sl2 - lse_s[qc]);
+            float p1 = ex2_approx(__uint_as_float(st_r[c + 1]) * sl2 - lse_s[qc + 1]);
+            if (diag && qc < r) p0 = 0.f;       // the key comes after the query
+            if (diag && qc + 1 < r) p1 = 0.f;
+            const float ds0 = p0 * (__uint_as_float(dp_r[c]) - d_s[qc]);
+            const float ds1 = p1 * (__uint_as_float(dp_r[c + 1]) - d_s[qc + 1]);
+            pk[h * 16 + c / 2] = pack_bf16x2(p0, p1);
+            dk_[h * 16 + c / 2] = pack_bf16x2(ds0, ds1);
+          }
+        }
+        // P^T / dS^T go over the first 64 columns of S^T / dP^T: wait until
+        // every compute thread has read its columns
+        tc_fence_before();
+        mbar_arrive(bar(Lay::B_SYNC_B));
+        if (!mbar_wait(bar(Lay::B_SYNC_B), s & 1, abort_flag, status, 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        tmem_st32(tmem + lane_base + Lay::TM_ST + col0 / 2, pk);
+        tmem_st32(tmem + lane_base + Lay::TM_DPT + col0 / 2, dk_);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(Lay::B_PDS_FULL));
+      }
+      if (!ok) break;
+      // epilogue: dK = scale * acc, then dV = acc, one accumulator at a time;
+      // sink chunks go out as fp32 partials that the reduce kernel adds up
+      if (!mbar_wait(bar(Lay::B_ACC_FULL), it & 1, abort_flag, status, 1)) break;
+      tc_fence_after();
+      constexpr int OH = DIM / 2;
+      const size_t grow = (size_t)w.plane * p.L + key;
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {  // 0: dK, 1: dV
+        const float mul = which == 0 ? p.scale : 1.f;
+        uint32_t ar[OH / 32][32];
+#pragma unroll
+        for (int ch = 0; ch < OH / 32; ++ch)
+          tmem_ld32(tmem + lane_base + (which == 0 ? Lay::TM_DK : Lay::TM_DV) + wg * OH + ch * 32,
+                    ar[ch]);
+        tmem_wait_ld();
+        if (w.slot >= 0) {
+          float* dst = p.part + (((size_t)w.slot * 2 + which) * 128 + r) * DIM + wg * OH;
+#pragma unroll
+          for (int ch = 0; ch < OH / 32; ++ch)
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4*>(dst + ch * 32 + e) =
+                  make_float4(__uint_as_float(ar[ch][e]) * mul,
+                              __uint_as_float(ar[ch][e + 1]) * mul,
+                              __uint_as_float(ar[ch][e + 2]) * mul,
+                              __uint_as_float(ar[ch][e + 3]) * mul);
+        } else if (key < p.L) {
+          uint4* dst = reinterpret_cast<uint4*>((which == 0 ? p.dk : p.dv) + grow * DIM + wg * OH);
+#pragma unroll
+          for (int ch = 0; ch < OH / 32; ++ch)
+#pragma unroll
+            for (int v = 0; v < 4; v += 2) {
+              uint32_t a8[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                a8[e] = pack_bf16x2(__uint_as_float(ar[ch][8 * v + 2 * e]) * mul,
+                                    __uint_as_float(ar[ch][8 * v + 2 * e + 1]) * mul);
+              st_global_v8(dst + ch * 4 + v, a8);
+            }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(Lay::B_ACC_EMPTY));
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// The sink blocks' dK, dV: the sum of their chunks' fp32 partials, as bf16.
+// One thread per (plane, sink block, key row, 4 columns).
+template <int DIM>
+__global__ void __launch_bounds__(256) ssa_bwd_sink_reduce_kernel(const BwdParams p) {
+  const int n_sink = min(p.n_sink, p.nb);
+  const long long quads = (long long)p.planes * n_sink * 128 * (DIM / 4);
+  for (long long x = blockIdx.x * (long long)blockDim.x + threadIdx.x; x < quads;
+       x += (long long)gridDim.x * blockDim.x) {
+    const int c4 = (int)(x % (DIM / 4));
+    const int r = (int)((x / (DIM / 4)) % 128);
+    const int j = (int)((x / (DIM / 4) / 128) % n_sink);
+    const int plane = (int)(x / (DIM / 4) / 128 / n_sink);
+    const int key = j * 128 + r;
+    if (key >= p.L) continue;
+    int slot = plane * p.sink_items;
+    for (int j2 = 0; j2 < j; ++j2) slot += bwd_sink_chunks(j2, p.nb);
+    float4 ak = make_float4(0.f, 0.f, 0.f, 0.f), av = ak;
+    for (int c = 0; c < bwd_sink_chunks(j, p.nb); ++c) {
+      const float* base = p.part + ((size_t)(slot + c) * 2 * 128 + r) * DIM + 4 * c4;
+      const float4 k4 = *reinterpret_cast<const float4*>(base);
+      const float4 v4 = *reinterpret_cast<const float4*>(base + (size_t)128 * DIM);
+      ak.x += k4.x; ak.y += k4.y; ak.z += k4.z; ak.w += k4.w;
+      av.x += v4.x; av.y += v4.y; av.z += v4.z; av.w += v4.w;
+    }
+    const size_t grow = (size_t)plane * p.L + key;
+    uint2 ko, vo;
+    ko.x = pack_bf16x2(ak.x, ak.y);
+    ko.y = pack_bf16x2(ak.z, ak.w);
+    vo.x = pack_bf16x2(av.x, av.y);
+    vo.y = pack_bf16x2(av.z, av.w);
+    *reinterpret_cast<uint2*>(p.dk + grow * DIM + 4 * c4) = ko;
+    *reinterpret_cast<uint2*>(p.dv + grow * DIM + 4 * c4) = vo;
+  }
+}
+
+}  // namespace loza

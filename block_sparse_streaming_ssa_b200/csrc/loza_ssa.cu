@@ -5,12 +5,14 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
 
 #include "../../include/loza_ssa.h"
+#include "backward.cuh"
 #include "decode.cuh"
 #include "prefill.cuh"
 #include "schedule.cuh"
@@ -147,6 +149,68 @@ int dispatch_prefill(int d_qk, int d_v, const void* q, const void* k, const void
   return LOZA_SSA_ERR_HEAD_DIM;
 }
 
+// Backward workspace: D_i (fp32 per row, 256-byte aligned), then the sink
+// blocks' fp32 partial dK / dV.
+struct BwdWorkspace {
+  size_t d_bytes, part_bytes;
+};
+BwdWorkspace bwd_workspace(long long planes, int L, int dim, int n_sink) {
+  const int nb = (L + 127) / 128;
+  const long long rows = planes * L;
+  BwdWorkspace w;
+  w.d_bytes = (size_t)(((rows * 4) + 255) / 256) * 256;
+  w.part_bytes = (size_t)planes * loza::bwd_sink_items(n_sink, nb) * 2 * 128 * dim * 4;
+  return w;
+}
+
+template <int DIM>
+int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+               loza::BwdParams prm, cudaStream_t s, const DeviceInfo& dev) {
+  CUtensorMap mq, mk, mv, mdo;
+  int rc;
+  const uint64_t L = (uint64_t)prm.L, planes = (uint64_t)prm.planes;
+  if ((rc = make_map(&mq, q, DIM, L, planes, 3)) != LOZA_SSA_OK) return rc;
+  if ((rc = make_map(&mk, k, DIM, L, planes, 3)) != LOZA_SSA_OK) return rc;
+  if ((rc = make_map(&mv, v, DIM, L, planes, 3)) != LOZA_SSA_OK) return rc;
+  if ((rc = make_map(&mdo, dout, DIM, L, planes, 3)) != LOZA_SSA_OK) return rc;
+  const long long rows = (long long)prm.planes * prm.L;
+  const int pre_grid = (int)std::min<long long>((rows + 63) / 64, (long long)dev.num_sms * 16);
+  loza::ssa_bwd_preprocess_kernel<DIM><<<pre_grid, 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout),
+      const_cast<float*>(prm.dsum), rows);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "backward preprocess launch");
+
+  using LQ = loza::BwdDqLayout<DIM>;
+  if ((e = cudaFuncSetAttribute(loza::ssa_bwd_dq_kernel<DIM>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, LQ::SMEM_BYTES)) !=
+      cudaSuccess)
+    return cuda_fail(e, "cudaFuncSetAttribute(backward dq)");
+  const long long dq_items = (long long)prm.planes * prm.nb;
+  loza::ssa_bwd_dq_kernel<DIM><<<(int)std::min<long long>(dq_items, dev.num_sms), loza::kBwdThreads,
+                                 LQ::SMEM_BYTES, s>>>(mq, mk, mv, mdo, prm);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward dq launch");
+
+  using LK = loza::BwdKvLayout<DIM>;
+  if ((e = cudaFuncSetAttribute(loza::ssa_bwd_dkdv_kernel<DIM>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, LK::SMEM_BYTES)) !=
+      cudaSuccess)
+    return cuda_fail(e, "cudaFuncSetAttribute(backward dkdv)");
+  const long long kv_items =
+      (long long)prm.planes * (prm.sink_items + (prm.nb > prm.n_sink ? prm.nb - prm.n_sink : 0));
+  loza::ssa_bwd_dkdv_kernel<DIM><<<(int)std::min<long long>(kv_items, dev.num_sms),
+                                   loza::kBwdThreads, LK::SMEM_BYTES, s>>>(mq, mk, mv, mdo, prm);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward dkdv launch");
+
+  if (prm.sink_items > 0) {
+    const long long quads = (long long)prm.planes * std::min(prm.n_sink, prm.nb) * 128 * (DIM / 4);
+    const int red_grid = (int)std::min<long long>((quads + 255) / 256, (long long)dev.num_sms * 8);
+    loza::ssa_bwd_sink_reduce_kernel<DIM><<<red_grid, 256, 0, s>>>(prm);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward reduce launch");
+  }
+  return LOZA_SSA_OK;
+}
+
 bool prefill_dims_ok(int d_qk, int d_v) {
   return (d_qk == 64 && d_v == 64) || (d_qk == 128 && d_v == 128) || (d_qk == 192 && d_v == 128);
 }
@@ -273,6 +337,62 @@ int loza_ssa_prefill(const void* q, const void* k, const void* v, void* o, float
   prm.total_items = (int)items;
   return dispatch_prefill(d_qk, d_v, q, k, v, prm, (uint64_t)L, (uint64_t)B * H, items, 0,
                           reinterpret_cast<cudaStream_t>(stream), dev);
+}
+
+size_t loza_ssa_prefill_bwd_workspace_size(int B, int H, int L, int d_qk, int d_v, int n_sink,
+                                           int n_local) {
+  if (B < 1 || H < 1 || L < 1 || d_qk != d_v || (d_qk != 64 && d_qk != 128) || n_sink < 0 ||
+      n_local < 1)
+    return 0;
+  const BwdWorkspace w = bwd_workspace((long long)B * H, L, d_qk, n_sink);
+  return w.d_bytes + w.part_bytes;
+}
+
+int loza_ssa_prefill_bwd(const void* q, const void* k, const void* v, const void* o,
+                         const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                         int H, int L, int d_qk, int d_v, int block, int n_sink, int n_local,
+                         float scale, void* workspace, size_t workspace_bytes,
+                         loza_ssa_stream_t stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return LOZA_SSA_ERR_NULL;
+  if (B < 1 || H < 1 || L < 1 || !std::isfinite(scale)) return LOZA_SSA_ERR_SHAPE;
+  if (d_qk != d_v || (d_qk != 64 && d_qk != 128)) return LOZA_SSA_ERR_HEAD_DIM;
+  if (block != 128) return LOZA_SSA_ERR_BLOCK;
+  if (n_sink < 0 || n_local < 1) return LOZA_SSA_ERR_WINDOW;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+      !aligned(lse, 4))
+    return LOZA_SSA_ERR_ALIGN;
+  const long long nb = (L + 127) / 128;
+  const long long planes = (long long)B * H;
+  const long long sink_items = loza::bwd_sink_items(n_sink, (int)std::min<long long>(nb, 1 << 30));
+  if (planes * nb >= (1ll << 31) || planes * (sink_items + nb) >= (1ll << 31) ||
+      planes * L >= (1ll << 40))
+    return LOZA_SSA_ERR_SHAPE;
+  const size_t need = loza_ssa_prefill_bwd_workspace_size(B, H, L, d_qk, d_v, n_sink, n_local);
+  if (!workspace || workspace_bytes < need) return LOZA_SSA_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return LOZA_SSA_ERR_ALIGN;
+  DeviceInfo dev;
+  int rc = device_info(dev);
+  if (rc != LOZA_SSA_OK) return rc;
+  const BwdWorkspace w = bwd_workspace(planes, L, d_qk, n_sink);
+  loza::BwdParams prm{};
+  prm.lse = lse;
+  prm.dsum = reinterpret_cast<const float*>(workspace);
+  prm.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + w.d_bytes);
+  prm.dq = static_cast<__nv_bfloat16*>(dq);
+  prm.dk = static_cast<__nv_bfloat16*>(dk);
+  prm.dv = static_cast<__nv_bfloat16*>(dv);
+  prm.L = L;
+  prm.planes = (int)planes;
+  prm.n_sink = n_sink;
+  prm.n_local = n_local;
+  prm.nb = (int)nb;
+  prm.sink_items = (int)sink_items;
+  prm.scale = scale;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d_qk == 64) return launch_bwd<64>(q, k, v, o, dout, prm, s, dev);
+  return launch_bwd<128>(q, k, v, o, dout, prm, s, dev);
 }
 
 int loza_ssa_prefill_varlen(const void* q, const void* k, const void* v, void* o, float* lse,

@@ -97,6 +97,35 @@ int loza_ssa_prefill_varlen(const void* q, const void* k, const void* v, void* o
                             float scale, loza_ssa_stream_t stream);
 
 /*
+ * Backward pass of the dense SSA prefill (loza_ssa_prefill's gradients):
+ * given the upstream gradient dout = dL/dO, computes
+ *   D_i = dO_i . O_i,  dP_ij = dO_i . v_j,  dS_ij = P_ij (dP_ij - D_i),
+ *   dq_i = scale sum_j dS_ij k_j,  dk_j = scale sum_i dS_ij q_i,
+ *   dv_j = sum_i P_ij dO_i,
+ * over the same SSA key sets J(i) as the forward pass, with
+ * P_ij = exp(scale q_i.k_j - lse_i) -- the chain rule applied to the masked
+ * softmax attention of "LoZA：ZigZag稀疏注意力机制" §2.1.
+ *   q, k, dq, dk : bf16 [B, H, L, d]     v, o, dout, dv : bf16 [B, H, L, d]
+ *   lse          : fp32 [B, H, L] as written by loza_ssa_prefill
+ *   d_qk == d_v in {64, 128}; block must be 128.
+ *   workspace    : DEVICE scratch of at least
+ *                  loza_ssa_prefill_bwd_workspace_size(...) bytes, 256-byte
+ *                  aligned, owned by the caller, contents irrelevant on entry.
+ * dq, dk, dv are overwritten (not accumulated into).  Statuses as for
+ * loza_ssa_prefill; LOZA_SSA_ERR_HEAD_DIM for other head dims.
+ */
+int loza_ssa_prefill_bwd(const void* q, const void* k, const void* v, const void* o,
+                         const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                         int H, int L, int d_qk, int d_v, int block, int n_sink, int n_local,
+                         float scale, void* workspace, size_t workspace_bytes,
+                         loza_ssa_stream_t stream);
+
+/* Bytes of workspace loza_ssa_prefill_bwd needs (0 on invalid arguments):
+ * fp32 D per row plus fp32 partial dK / dV of the sink blocks' chunks. */
+size_t loza_ssa_prefill_bwd_workspace_size(int B, int H, int L, int d_qk, int d_v, int n_sink,
+                                           int n_local);
+
+/*
  * Paged SSA decode, absorbed-MLA layout: one new query token per sequence,
  * H_q query heads all attending one shared latent key/value row per token.
  *   q          : bf16 [B, H_q, d_qk]
