@@ -13,7 +13,8 @@ paged decode workload (32 sequences, 128 heads, 576/512, random page table over
 a ~20 GB pool) and reports it under ``decode`` in GB/s of algorithmic bytes,
 and the same decode with 8 distinct selected pages per sequence on top of the
 window under ``decode_selected`` (``--decode-extra``), and the decode with 2
-query tokens per sequence under ``decode_mtp`` (``--decode-mtp``).
+query tokens per sequence under ``decode_mtp`` (``--decode-mtp``).  The
+prefill's backward pass on the same workload is timed under ``backward``.
 
 Under torchrun every rank runs its own replica of the workload (weak scaling,
 no collective on the data path; NCCL only reduces the timing).
@@ -246,6 +247,45 @@ def time_prefill(w, steps, warmup, dist):
     return total_ms, per, clk.summary()
 
 
+def backward_bench(w, steps, warmup, peaks, world=1):
+    """The prefill's backward (loza_ssa_prefill_bwd) on the same workload,
+    with o and lse from the forward pass and a seeded random dO.  Useful FLOPs
+    follow the usual attention-backward count, 2.5x the forward: the five
+    products dP = dO V^T, dV += P^T dO, dQ += dS K, dK += dS^T Q and one
+    recomputation of S = Q K^T, each 2 d per unmasked (i, j) pair (the dK/dV
+    kernel recomputes S and dP a second time; that work is not counted)."""
+    import torch
+    from block_sparse_streaming_ssa_b200.loza_ssa import loza_ssa_prefill_bwd
+    sp = w["spec"]
+    if w["varlen"] or sp.d_qk != sp.d_v or sp.d_qk not in (64, 128):
+        return None
+    o, lse = prefill_call(w)
+    g = torch.Generator(device="cuda").manual_seed(4242)
+    dout = torch.randn(w["v"].shape, generator=g, device="cuda").to(torch.bfloat16)
+    grads = loza_ssa_prefill_bwd(w["q"], w["k"], w["v"], o, lse, dout, scale=sp.scale)
+    for _ in range(warmup):
+        loza_ssa_prefill_bwd(w["q"], w["k"], w["v"], o, lse, dout, *grads, scale=sp.scale)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        loza_ssa_prefill_bwd(w["q"], w["k"], w["v"], o, lse, dout, *grads, scale=sp.scale)
+    t1.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps)
+    flops = 2.5 * 2 * (sp.d_qk + sp.d_v) * w["pairs"]
+    tf = flops / (ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    return {"workload": w["desc"]["workload"] + ", backward (dQ, dK, dV)",
+            "value": round(job_throughput(world, flops, 1, ms) / 1e12, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 4), "useful_tflop_per_step": round(flops / 1e12, 4),
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peak,
+                         "unit": "TFLOP/s", "frac": round(tf / peak, 4), "traffic": None,
+                         "peak_source": peaks["source"] + " (burst bf16 GEMM)",
+                         "note": "whole call: D preprocess, dQ kernel, dK/dV kernel, sink reduce"},
+            "gpu_launches": 4 * steps}
+
+
 def e2e_prefill(w, steps):
     """Same metric through the public call with host buffers: pinned host ->
     device copy of q, k, v, the call, device -> host copy of o and lse, every step."""
@@ -473,6 +513,8 @@ def main():
     ap.add_argument("--no-prefill", action="store_true",
                     help="time only the decode workload (for profiler captures of it)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip timing the prefill's backward pass")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--decode-iters", type=int, default=30)
     ap.add_argument("--decode-len-hi", type=int, default=None,
@@ -559,6 +601,8 @@ def main():
     e2e_ms, h2d, d2h = e2e_prefill(w, args.e2e_steps)
     e2e_val = world * flops / (e2e_ms * 1e-3) / 1e12  # every rank runs the same e2e loop
 
+    backward = None if args.no_backward else backward_bench(w, max(3, args.steps // 5),
+                                                              args.warmup, peaks, world)
     w_desc, w_tokens = w["desc"], w["tokens"]
     decode = selected = mtp = None
     if not args.no_decode:
@@ -614,6 +658,7 @@ def main():
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)},
         "clocks": clocks,
         "gpu_launches": args.steps,
+        "backward": backward,
         "decode": decode,
         "decode_selected": selected,
         "decode_mtp": mtp,
