@@ -37,7 +37,8 @@
 
 namespace loza {
 
-constexpr int kBwdThreads = 320;     // warps 0-7 compute, 8 TMA producer, 9 MMA issuer
+// warps 0-7 compute, 8 TMA producer, 9 and 10 MMA issuers
+constexpr int kBwdThreads = 352;
 constexpr int kBwdComputeThreads = 256;
 constexpr int kSinkChunk = 8;        // query blocks per sink work item
 
@@ -153,8 +154,8 @@ struct BwdDqLayout {
   static constexpr int B_DS_FREE = B_DS_FULL + 1;     // dQ MMA of the tile done
   static constexpr int B_DQ_FULL = B_DS_FREE + 1;     // the item's last dQ MMA done
   static constexpr int B_DQ_EMPTY = B_DQ_FULL + 1;    // epilogue has read dQ
-  static constexpr int B_DRAIN = B_DQ_EMPTY + 1;
-  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int B_DRAIN = B_DQ_EMPTY + 1;     // 2: one per MMA issuer
+  static constexpr int NBAR = B_DRAIN + 2;
   static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;  // [0] tmem base, [1] abort
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -196,6 +197,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(bar(Lay::B_DQ_FULL), 1);
     mbar_init(bar(Lay::B_DQ_EMPTY), kBwdComputeThreads);
     mbar_init(bar(Lay::B_DRAIN), 1);
+    mbar_init(bar(Lay::B_DRAIN + 1), 1);
     misc[1] = 0;
     fence_barrier_init();
   }
@@ -274,82 +276,87 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
   } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    // Order: S/dP of tile 0, then for every tile g: S/dP of tile g+1 (as soon
-    // as the compute warps have loaded tile g's S and dP), then dQ += dS_g K_g.
+    // ------------------------------------------------- MMA issuer: S and dP
+    // S/dP of tile g+1 go out as soon as the compute warps have loaded tile
+    // g's S and dP; the dQ products have their own issuer (warp 10), so a
+    // wait for dS never holds them back.
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16_f32(128, 128, false);
-      const uint32_t id_q = idesc_bf16_f32(128, DIM, true);
+      const uint64_t q_desc = sdesc_sw128(sb + Lay::OFF_Q, 16, 1024);
+      const uint64_t do_desc = sdesc_sw128(sb + Lay::OFF_DO, 16, 1024);
+      const uint64_t k_desc0 = sdesc_sw128(sb + Lay::OFF_K, 16, 1024);
+      const uint64_t v_desc0 = sdesc_sw128(sb + Lay::OFF_V, 16, 1024);
+      int g = 0, it = 0;
       bool ok = true;
-      // cursor over (item, tile) for the S/dP MMAs
-      int a_item = blockIdx.x, a_it = 0, a_t = 0, a_g = 0;
-      auto issue_sdp = [&]() -> bool {
-        const int plane = a_item / p.nb, qb = a_item - plane * p.nb;
-        (void)plane;
-        const TileRange tr = tile_range(qb, p.n_sink, p.n_local);
-        if (a_t == 0 && !mbar_wait(bar(Lay::B_QD_FULL), a_it & 1, abort_flag, status, 1))
-          return false;
-        const int st = a_g % Lay::KST, vs = a_g % Lay::VST;
-        if (a_g > 0 && !mbar_wait(bar(Lay::B_SDP_FREE), (a_g - 1) & 1, abort_flag, status, 1))
-          return false;
-        if (!mbar_wait(bar(Lay::B_K_FULL + st), (a_g / Lay::KST) & 1, abort_flag, status, 1) ||
-            !mbar_wait(bar(Lay::B_V_FULL + vs), (a_g / Lay::VST) & 1, abort_flag, status, 1))
-          return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < DIM / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
-          mma_ss(tmem + Lay::TM_S, sdesc_sw128(sb + Lay::OFF_Q + koff, 16, 1024),
-                 sdesc_sw128(sb + Lay::OFF_K + st * Lay::TILE + koff, 16, 1024), id_s,
-                 kk > 0 ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < DIM / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
-          mma_ss(tmem + Lay::TM_DP, sdesc_sw128(sb + Lay::OFF_DO + koff, 16, 1024),
-                 sdesc_sw128(sb + Lay::OFF_V + vs * Lay::TILE + koff, 16, 1024), id_s,
-                 kk > 0 ? 1u : 0u);
-        }
-        mma_commit(bar(Lay::B_S_FULL));
-        mma_commit(bar(Lay::B_V_EMPTY + vs));
-        if (a_t == tr.count - 1) {
-          mma_commit(bar(Lay::B_QD_EMPTY));
-          a_t = 0;
-          ++a_it;
-          a_item += gridDim.x;
-        } else {
-          ++a_t;
-        }
-        ++a_g;
-        return true;
-      };
-      if (a_item < total_items) ok = issue_sdp();
-      int b_it = 0, b_g = 0;
-      for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++b_it) {
+      for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++it) {
         const int qb = item % p.nb;
         const TileRange tr = tile_range(qb, p.n_sink, p.n_local);
-        for (int t = 0; ok && t < tr.count; ++t, ++b_g) {
-          if (a_item < total_items && !(ok = issue_sdp())) break;
-          const int st = b_g % Lay::KST;
-          if (!(ok = mbar_wait(bar(Lay::B_DS_FULL), b_g & 1, abort_flag, status, 1))) break;
-          if (t == 0 && b_it > 0 &&
-              !(ok = mbar_wait(bar(Lay::B_DQ_EMPTY), (b_it - 1) & 1, abort_flag, status, 1)))
+        if (!(ok = mbar_wait(bar(Lay::B_QD_FULL), it & 1, abort_flag, status, 1))) break;
+        for (int t = 0; t < tr.count; ++t, ++g) {
+          const int st = g % Lay::KST, vs = g % Lay::VST;
+          if ((g > 0 &&
+               !(ok = mbar_wait(bar(Lay::B_SDP_FREE), (g - 1) & 1, abort_flag, status, 1))) ||
+              !(ok = mbar_wait(bar(Lay::B_K_FULL + st), (g / Lay::KST) & 1, abort_flag, status,
+                               1)) ||
+              !(ok = mbar_wait(bar(Lay::B_V_FULL + vs), (g / Lay::VST) & 1, abort_flag, status,
+                               1)))
             break;
           tc_fence_after();
-          // dQ += dS K: dS (bf16 pairs) in TMEM columns TM_DS.., K MN-major
-          // (keys 16kk .. 16kk+15 of each 64-column box are 2048 bytes in)
+          const uint64_t k_desc = k_desc0 + (uint64_t)(st * (Lay::TILE >> 4));
+          const uint64_t v_desc = v_desc0 + (uint64_t)(vs * (Lay::TILE >> 4));
+#pragma unroll
+          for (int kk = 0; kk < DIM / 16; ++kk) {
+            const uint64_t koff = (uint64_t)(((kk >> 2) * Lay::CHUNK + (kk & 3) * 32) >> 4);
+            mma_ss(tmem + Lay::TM_S, q_desc + koff, k_desc + koff, id_s, kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < DIM / 16; ++kk) {
+            const uint64_t koff = (uint64_t)(((kk >> 2) * Lay::CHUNK + (kk & 3) * 32) >> 4);
+            mma_ss(tmem + Lay::TM_DP, do_desc + koff, v_desc + koff, id_s, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(Lay::B_S_FULL));
+          mma_commit(bar(Lay::B_V_EMPTY + vs));
+          if (t == tr.count - 1) mma_commit(bar(Lay::B_QD_EMPTY));
+        }
+      }
+      mma_commit(bar(Lay::B_DRAIN));
+      mbar_wait_drain(bar(Lay::B_DRAIN), 0);
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------------- MMA issuer: dQ += dS K
+    if (lane == 0) {
+      const uint32_t id_q = idesc_bf16_f32(128, DIM, true);
+      // K read MN-major: keys 16kk .. 16kk+15 of each 64-column box are 2048 bytes in
+      const uint64_t k_desc0 = sdesc_sw128(sb + Lay::OFF_K, Lay::CHUNK, 1024);
+      int g = 0, it = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++it) {
+        const int qb = item % p.nb;
+        const TileRange tr = tile_range(qb, p.n_sink, p.n_local);
+        for (int t = 0; t < tr.count; ++t, ++g) {
+          const int st = g % Lay::KST;
+          // K(g) is in place (its slot is released only by this issuer) and
+          // dS(g) is in TMEM; the item's first product overwrites dQ, which
+          // the previous item's epilogue must have read
+          if (!(ok = mbar_wait(bar(Lay::B_K_FULL + st), (g / Lay::KST) & 1, abort_flag, status,
+                               1)) ||
+              !(ok = mbar_wait(bar(Lay::B_DS_FULL), g & 1, abort_flag, status, 1)) ||
+              (t == 0 && it > 0 &&
+               !(ok = mbar_wait(bar(Lay::B_DQ_EMPTY), (it - 1) & 1, abort_flag, status, 1))))
+            break;
+          tc_fence_after();
+          const uint64_t k_desc = k_desc0 + (uint64_t)(st * (Lay::TILE >> 4));
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(tmem + Lay::TM_DQ, tmem + Lay::TM_DS + kk * 8,
-                   sdesc_sw128(sb + Lay::OFF_K + st * Lay::TILE + kk * 2048, Lay::CHUNK, 1024),
-                   id_q, (t > 0 || kk > 0) ? 1u : 0u);
+                   k_desc + (uint64_t)(kk * (2048 >> 4)), id_q, (t > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bar(Lay::B_DS_FREE));
           mma_commit(bar(Lay::B_K_EMPTY + st));
           if (t == tr.count - 1) mma_commit(bar(Lay::B_DQ_FULL));
         }
       }
-      mma_commit(bar(Lay::B_DRAIN));
-      mbar_wait_drain(bar(Lay::B_DRAIN), 0);
+      mma_commit(bar(Lay::B_DRAIN + 1));
+      mbar_wait_drain(bar(Lay::B_DRAIN + 1), 0);
     }
   } else {
     // ------------------------------------------------------- compute warps
@@ -447,6 +454,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 // ---------------------------------------------------------------- dK, dV
+//
+// Each query block is taken as two halves of 64 queries.  Compute warpgroup h
+// owns half h of every step: TMEM holds S^T_h and dP^T_h (keys on the lanes,
+// 64 query columns each) for both halves at once, so while one warpgroup
+// turns its half into P^T / dS^T the tensor core works on the other half.
 
 template <int DIM>
 struct BwdKvLayout {
@@ -457,23 +469,23 @@ struct BwdKvLayout {
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = TILE;
   static constexpr int OFF_Q = 2 * TILE;           // QST x [Q | dO]
-  static constexpr int OFF_ROW = OFF_Q + QST * 2 * TILE;  // float [2 steps][2: lse2, D][128]
-  static constexpr int OFF_BAR = OFF_ROW + 2 * 2 * 128 * 4;
-  // TMEM: S^T, dP^T (P^T / dS^T as bf16 pairs over their first 64 columns), dV, dK
-  static constexpr int TM_ST = 0, TM_DPT = 128, TM_DV = 256, TM_DK = 256 + DIM;
+  static constexpr int OFF_ROW = OFF_Q + QST * 2 * TILE;  // float [2 steps][2 halves][lse2, D][64]
+  static constexpr int OFF_BAR = OFF_ROW + 2 * 2 * 2 * 64 * 4;
+  // TMEM: per half h, S^T_h at 128h and dP^T_h at 128h + 64 (P^T_h / dS^T_h as
+  // bf16 pairs over their first 32 columns), then dV and dK
+  static constexpr int TM_DV = 256, TM_DK = 256 + DIM;
   static_assert(TM_DK + DIM <= 512, "TMEM");
   // barriers
   static constexpr int B_KV_FULL = 0, B_KV_EMPTY = 1;
   static constexpr int B_Q_FULL = 2, B_Q_EMPTY = B_Q_FULL + QST;
-  static constexpr int B_ST_FULL = B_Q_EMPTY + QST;  // S^T and dP^T issued (commit)
-  static constexpr int B_SYNC_A = B_ST_FULL + 1;     // compute warps: the step's rows staged
-  static constexpr int B_SYNC_B = B_SYNC_A + 1;      // compute warps: S^T, dP^T all read
-  static constexpr int B_PDS_FULL = B_SYNC_B + 1;    // P^T and dS^T written
-  static constexpr int B_PDS_FREE = B_PDS_FULL + 1;  // dV, dK MMAs of the step done
-  static constexpr int B_ACC_FULL = B_PDS_FREE + 1;  // the item's last dV, dK MMAs done
+  static constexpr int B_ST_FULL = B_Q_EMPTY + QST;  // [2] S^T_h, dP^T_h issued (commit)
+  static constexpr int B_SYNC = B_ST_FULL + 2;       // [2] warpgroup h: its rows staged
+  static constexpr int B_PDS_FULL = B_SYNC + 2;      // [2] P^T_h, dS^T_h written
+  static constexpr int B_PDS_FREE = B_PDS_FULL + 2;  // [2] dV, dK products of half h done
+  static constexpr int B_ACC_FULL = B_PDS_FREE + 2;  // the item's last dV, dK products done
   static constexpr int B_ACC_EMPTY = B_ACC_FULL + 1; // epilogue has read dV, dK
-  static constexpr int B_DRAIN = B_ACC_EMPTY + 1;
-  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int B_DRAIN = B_ACC_EMPTY + 1;    // [2] one per issuer
+  static constexpr int NBAR = B_DRAIN + 2;
   static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -505,14 +517,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bar(Lay::B_Q_FULL + s), 1);
       mbar_init(bar(Lay::B_Q_EMPTY + s), 1);
     }
-    mbar_init(bar(Lay::B_ST_FULL), 1);
-    mbar_init(bar(Lay::B_SYNC_A), kBwdComputeThreads);
-    mbar_init(bar(Lay::B_SYNC_B), kBwdComputeThreads);
-    mbar_init(bar(Lay::B_PDS_FULL), kBwdComputeThreads);
-    mbar_init(bar(Lay::B_PDS_FREE), 1);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(bar(Lay::B_ST_FULL + h), 1);
+      mbar_init(bar(Lay::B_SYNC + h), kBwdComputeThreads / 2);
+      mbar_init(bar(Lay::B_PDS_FULL + h), kBwdComputeThreads / 2);
+      mbar_init(bar(Lay::B_PDS_FREE + h), 1);
+      mbar_init(bar(Lay::B_DRAIN + h), 1);
+    }
     mbar_init(bar(Lay::B_ACC_FULL), 1);
     mbar_init(bar(Lay::B_ACC_EMPTY), kBwdComputeThreads);
-    mbar_init(bar(Lay::B_DRAIN), 1);
     misc[1] = 0;
     fence_barrier_init();
   }
@@ -578,75 +591,105 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
   } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------ MMA issuer: S^T_h and dP^T_h
     if (lane == 0) {
-      const uint32_t id_s = idesc_bf16_f32(128, 128, false);   // M = keys, N = queries
-      const uint32_t id_a = idesc_bf16_f32(128, DIM, true);    // dV, dK: B = dO / Q, MN-major
+      const uint32_t id_s = idesc_bf16_f32(128, 64, false);   // M = keys, N = 64 queries
+      const uint64_t k_desc = sdesc_sw128(sb + Lay::OFF_K, 16, 1024);
+      const uint64_t v_desc = sdesc_sw128(sb + Lay::OFF_V, 16, 1024);
+      const uint64_t q_desc0 = sdesc_sw128(sb + Lay::OFF_Q, 16, 1024);
       int s = 0, it = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++it) {
         const BwdKItem w = bwd_kv_item(p, item);
         if (!(ok = mbar_wait(bar(Lay::B_KV_FULL), it & 1, abort_flag, status, 1))) break;
-        for (int qi = w.q_lo; qi <= w.q_hi; ++qi, ++s) {
+        for (int qi = w.q_lo; ok && qi <= w.q_hi; ++qi, ++s) {
           const int st = s % Lay::QST;
-          const uint32_t qbase = sb + Lay::OFF_Q + st * 2 * Lay::TILE;
-          // S^T / dP^T overwrite the P^T / dS^T columns the previous step's MMAs read
-          if ((s > 0 &&
-               !(ok = mbar_wait(bar(Lay::B_PDS_FREE), (s - 1) & 1, abort_flag, status, 1))) ||
-              !(ok = mbar_wait(bar(Lay::B_Q_FULL + st), (s / Lay::QST) & 1, abort_flag, status,
+          if (!(ok = mbar_wait(bar(Lay::B_Q_FULL + st), (s / Lay::QST) & 1, abort_flag, status,
                                1)))
             break;
-          tc_fence_after();
-          // S^T = K Q^T, dP^T = V dO^T (all operands K-major: rows x DIM boxes)
+          const uint64_t q_desc = q_desc0 + (uint64_t)(st * ((2 * Lay::TILE) >> 4));
+          const uint64_t do_desc = q_desc + (uint64_t)(Lay::TILE >> 4);
+#pragma unroll 1
+          for (int h = 0; h < 2; ++h) {
+            // S^T_h / dP^T_h overwrite P^T_h / dS^T_h of the previous step
+            if (s > 0 &&
+                !(ok = mbar_wait(bar(Lay::B_PDS_FREE + h), (s - 1) & 1, abort_flag, status, 1)))
+              break;
+            tc_fence_after();
+            const uint32_t st_t = tmem + 128 * h, dpt_t = st_t + 64;
+            // queries 64h .. 64h+63: rows 64h.. of every box (8192 bytes in)
+            const uint64_t hoff = (uint64_t)((8192 * h) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < DIM / 16; ++kk) {
-            const uint32_t koff = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
-            mma_ss(tmem + Lay::TM_ST, sdesc_sw128(sb + Lay::OFF_K + koff, 16, 1024),
-                   sdesc_sw128(qbase + koff, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < DIM / 16; ++kk) {
+              const uint64_t koff = (uint64_t)(((kk >> 2) * Lay::CHUNK + (kk & 3) * 32) >> 4);
+              mma_ss(st_t, k_desc + koff, q_desc + hoff + koff, id_s, kk > 0 ? 1u : 0u);
+            }
+#pragma unroll
+            for (int kk = 0; kk < DIM / 16; ++kk) {
+              const uint64_t koff = (uint64_t)(((kk >> 2) * Lay::CHUNK + (kk & 3) * 32) >> 4);
+              mma_ss(dpt_t, v_desc + koff, do_desc + hoff + koff, id_s, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(bar(Lay::B_ST_FULL + h));
           }
-#pragma unroll
-          for (int kk = 0; kk < DIM / 16; ++kk) {
-            const uint32_t koff = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
-            mma_ss(tmem + Lay::TM_DPT, sdesc_sw128(sb + Lay::OFF_V + koff, 16, 1024),
-                   sdesc_sw128(qbase + Lay::TILE + koff, 16, 1024), id_s, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(bar(Lay::B_ST_FULL));
-          if (!(ok = mbar_wait(bar(Lay::B_PDS_FULL), s & 1, abort_flag, status, 1))) break;
-          const bool first = (qi == w.q_lo);
-          if (first && it > 0 &&
-              !(ok = mbar_wait(bar(Lay::B_ACC_EMPTY), (it - 1) & 1, abort_flag, status, 1)))
-            break;
-          tc_fence_after();
-          // dV += P^T dO, dK += dS^T Q: A = P^T / dS^T in TMEM (keys x queries,
-          // bf16 pairs), B = dO / Q MN-major (queries 16kk .. 16kk+15 of each
-          // 64-column box are 2048 bytes in)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + Lay::TM_DV, tmem + Lay::TM_ST + kk * 8,
-                   sdesc_sw128(qbase + Lay::TILE + kk * 2048, Lay::CHUNK, 1024), id_a,
-                   (!first || kk > 0) ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + Lay::TM_DK, tmem + Lay::TM_DPT + kk * 8,
-                   sdesc_sw128(qbase + kk * 2048, Lay::CHUNK, 1024), id_a,
-                   (!first || kk > 0) ? 1u : 0u);
-          mma_commit(bar(Lay::B_PDS_FREE));
-          mma_commit(bar(Lay::B_Q_EMPTY + st));
-          if (qi == w.q_hi) {
-            mma_commit(bar(Lay::B_ACC_FULL));
-            mma_commit(bar(Lay::B_KV_EMPTY));
-          }
+          if (ok && qi == w.q_hi) mma_commit(bar(Lay::B_KV_EMPTY));  // K, V read for the last time
         }
       }
       mma_commit(bar(Lay::B_DRAIN));
       mbar_wait_drain(bar(Lay::B_DRAIN), 0);
     }
+  } else if (warp == 10) {
+    // ------------------------------------ MMA issuer: dV += P^T dO, dK += dS^T Q
+    if (lane == 0) {
+      const uint32_t id_a = idesc_bf16_f32(128, DIM, true);  // B = dO / Q, MN-major
+      // queries 16kk .. of half h: rows 64h + 16kk of every box (2048 bytes per 16 rows)
+      const uint64_t q_desc0 = sdesc_sw128(sb + Lay::OFF_Q, Lay::CHUNK, 1024);
+      int s = 0, it = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++it) {
+        const BwdKItem w = bwd_kv_item(p, item);
+        for (int qi = w.q_lo; ok && qi <= w.q_hi; ++qi, ++s) {
+          const int st = s % Lay::QST;
+          const uint64_t q_desc = q_desc0 + (uint64_t)(st * ((2 * Lay::TILE) >> 4));
+          const uint64_t do_desc = q_desc + (uint64_t)(Lay::TILE >> 4);
+          if (!(ok = mbar_wait(bar(Lay::B_Q_FULL + st), (s / Lay::QST) & 1, abort_flag, status,
+                               1)))
+            break;
+#pragma unroll 1
+          for (int h = 0; h < 2; ++h) {
+            const bool first = (qi == w.q_lo && h == 0);
+            if (!(ok = mbar_wait(bar(Lay::B_PDS_FULL + h), s & 1, abort_flag, status, 1)) ||
+                (first && it > 0 &&
+                 !(ok = mbar_wait(bar(Lay::B_ACC_EMPTY), (it - 1) & 1, abort_flag, status, 1))))
+              break;
+            tc_fence_after();
+            const uint32_t pt_t = tmem + 128 * h, dst_t = pt_t + 64;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t off = (uint64_t)((8192 * h + 2048 * kk) >> 4);
+              mma_ts(tmem + Lay::TM_DV, pt_t + kk * 8, do_desc + off, id_a,
+                     (!first || kk > 0) ? 1u : 0u);
+            }
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t off = (uint64_t)((8192 * h + 2048 * kk) >> 4);
+              mma_ts(tmem + Lay::TM_DK, dst_t + kk * 8, q_desc + off, id_a,
+                     (!first || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(bar(Lay::B_PDS_FREE + h));
+          }
+          if (!ok) break;
+          mma_commit(bar(Lay::B_Q_EMPTY + st));
+          if (qi == w.q_hi) mma_commit(bar(Lay::B_ACC_FULL));
+        }
+      }
+      mma_commit(bar(Lay::B_DRAIN + 1));
+      mbar_wait_drain(bar(Lay::B_DRAIN + 1), 0);
+    }
   } else {
     // ------------------------------------------------------- compute warps
-    const int wg = warp >> 2;                                      // query-column half
+    const int h = warp >> 2;                                       // query half of every step
     const int r = threadIdx.x & 127;                               // key row = TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const int col0 = wg * 64;
     const float sl2 = p.scale_log2;
     float* rows_smem = reinterpret_cast<float*>(smem + Lay::OFF_ROW);
     int s = 0, it = 0;
@@ -655,58 +698,52 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int key = w.kb * 128 + r;
       bool ok = true;
       for (int qi = w.q_lo; qi <= w.q_hi; ++qi, ++s) {
-        // stage lse2 and D of the step's 128 queries (rows past L: 0, harmless:
+        // stage lse2 and D of this half's 64 queries (rows past L: 0, harmless:
         // their Q and dO rows are zero, so their dS^T and dV terms vanish)
-        float* lse_s = rows_smem + (s & 1) * 256;
-        float* d_s = lse_s + 128;
-        if (wg == 0) {
-          const int qrow = qi * 128 + r;
+        float* lse_s = rows_smem + ((s & 1) * 2 + h) * 128;
+        float* d_s = lse_s + 64;
+        {
+          const int t = r & 63;
+          const int qrow = qi * 128 + h * 64 + t;
           const size_t gq = (size_t)w.plane * p.L + qrow;
-          lse_s[r] = qrow < p.L ? __ldg(p.lse + gq) * 1.4426950408889634f : 0.f;
-          d_s[r] = qrow < p.L ? __ldg(p.dsum + gq) : 0.f;
+          if (r < 64) lse_s[t] = qrow < p.L ? __ldg(p.lse + gq) * 1.4426950408889634f : 0.f;
+          else d_s[t] = qrow < p.L ? __ldg(p.dsum + gq) : 0.f;
         }
-        mbar_arrive(bar(Lay::B_SYNC_A));
-        if (!mbar_wait(bar(Lay::B_SYNC_A), s & 1, abort_flag, status, 1) ||
-            !mbar_wait(bar(Lay::B_ST_FULL), s & 1, abort_flag, status, 1)) {
+        mbar_arrive(bar(Lay::B_SYNC + h));
+        if (!mbar_wait(bar(Lay::B_SYNC + h), s & 1, abort_flag, status, 1) ||
+            !mbar_wait(bar(Lay::B_ST_FULL + h), s & 1, abort_flag, status, 1)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const bool diag = (qi == w.kb);
+        const uint32_t st_t = tmem + lane_base + 128 * h, dpt_t = st_t + 64;
         uint32_t pk[32], dk_[32];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int c2 = 0; c2 < 2; ++c2) {
           uint32_t st_r[32], dp_r[32];
-          tmem_ld32(tmem + lane_base + Lay::TM_ST + col0 + h * 32, st_r);
-          tmem_ld32(tmem + lane_base + Lay::TM_DPT + col0 + h * 32, dp_r);
+          tmem_ld32(st_t + c2 * 32, st_r);
+          tmem_ld32(dpt_t + c2 * 32, dp_r);
           tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
-            const int qc = col0 + h * 32 + c;  // query column within the block
+            const int qc = c2 * 32 + c;                 // query within the half
             float p0 = ex2_approx(__uint_as_float(st_r[c]) * sl2 - lse_s[qc]);
             float p1 = ex2_approx(__uint_as_float(st_r[c + 1]) * sl2 - lse_s[qc + 1]);
-            if (diag && qc < r) p0 = 0.f;       // the key comes after the query
-            if (diag && qc + 1 < r) p1 = 0.f;
+            if (diag && h * 64 + qc < r) p0 = 0.f;      // the key comes after the query
+            if (diag && h * 64 + qc + 1 < r) p1 = 0.f;
             const float ds0 = p0 * (__uint_as_float(dp_r[c]) - d_s[qc]);
             const float ds1 = p1 * (__uint_as_float(dp_r[c + 1]) - d_s[qc + 1]);
-            pk[h * 16 + c / 2] = pack_bf16x2(p0, p1);
-            dk_[h * 16 + c / 2] = pack_bf16x2(ds0, ds1);
+            pk[c2 * 16 + c / 2] = pack_bf16x2(p0, p1);
+            dk_[c2 * 16 + c / 2] = pack_bf16x2(ds0, ds1);
           }
         }
-        // P^T / dS^T go over the first 64 columns of S^T / dP^T: wait until
-        // every compute thread has read its columns
-        tc_fence_before();
-        mbar_arrive(bar(Lay::B_SYNC_B));
-        if (!mbar_wait(bar(Lay::B_SYNC_B), s & 1, abort_flag, status, 1)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        tmem_st32(tmem + lane_base + Lay::TM_ST + col0 / 2, pk);
-        tmem_st32(tmem + lane_base + Lay::TM_DPT + col0 / 2, dk_);
+        // this thread's row is read: P^T / dS^T over its first 32 columns
+        tmem_st32(st_t, pk);
+        tmem_st32(dpt_t, dk_);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(Lay::B_PDS_FULL));
+        mbar_arrive(bar(Lay::B_PDS_FULL + h));
       }
       if (!ok) break;
       // epilogue: dK = scale * acc, then dV = acc, one accumulator at a time;
@@ -721,11 +758,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         uint32_t ar[OH / 32][32];
 #pragma unroll
         for (int ch = 0; ch < OH / 32; ++ch)
-          tmem_ld32(tmem + lane_base + (which == 0 ? Lay::TM_DK : Lay::TM_DV) + wg * OH + ch * 32,
+          tmem_ld32(tmem + lane_base + (which == 0 ? Lay::TM_DK : Lay::TM_DV) + h * OH + ch * 32,
                     ar[ch]);
         tmem_wait_ld();
         if (w.slot >= 0) {
-          float* dst = p.part + (((size_t)w.slot * 2 + which) * 128 + r) * DIM + wg * OH;
+          float* dst = p.part + (((size_t)w.slot * 2 + which) * 128 + r) * DIM + h * OH;
 #pragma unroll
           for (int ch = 0; ch < OH / 32; ++ch)
 #pragma unroll
@@ -736,7 +773,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                               __uint_as_float(ar[ch][e + 2]) * mul,
                               __uint_as_float(ar[ch][e + 3]) * mul);
         } else if (key < p.L) {
-          uint4* dst = reinterpret_cast<uint4*>((which == 0 ? p.dk : p.dv) + grow * DIM + wg * OH);
+          uint4* dst = reinterpret_cast<uint4*>((which == 0 ? p.dk : p.dv) + grow * DIM + h * OH);
 #pragma unroll
           for (int ch = 0; ch < OH / 32; ++ch)
 #pragma unroll
