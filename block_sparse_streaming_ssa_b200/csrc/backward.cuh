@@ -726,16 +726,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tmem_ld32(dpt_t + c2 * 32, dp_r);
           tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; c += 2) {
+          for (int c = 0; c < 32; c += 4) {
             const int qc = c2 * 32 + c;                 // query within the half
-            float p0 = ex2_approx(__uint_as_float(st_r[c]) * sl2 - lse_s[qc]);
-            float p1 = ex2_approx(__uint_as_float(st_r[c + 1]) * sl2 - lse_s[qc + 1]);
-            if (diag && h * 64 + qc < r) p0 = 0.f;      // the key comes after the query
-            if (diag && h * 64 + qc + 1 < r) p1 = 0.f;
-            const float ds0 = p0 * (__uint_as_float(dp_r[c]) - d_s[qc]);
-            const float ds1 = p1 * (__uint_as_float(dp_r[c + 1]) - d_s[qc + 1]);
-            pk[c2 * 16 + c / 2] = pack_bf16x2(p0, p1);
-            dk_[c2 * 16 + c / 2] = pack_bf16x2(ds0, ds1);
+            // the staged rows are read four at a time (every thread reads the
+            // same address: one broadcast per warp)
+            const float4 l4 = *reinterpret_cast<const float4*>(lse_s + qc);
+            const float4 d4 = *reinterpret_cast<const float4*>(d_s + qc);
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+            float pp[4], dd[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              pp[e] = ex2_approx(__uint_as_float(st_r[c + e]) * sl2 - lv[e]);
+              if (diag && h * 64 + qc + e < r) pp[e] = 0.f;  // the key comes after the query
+              dd[e] = pp[e] * (__uint_as_float(dp_r[c + e]) - dv4[e]);
+            }
+            pk[c2 * 16 + c / 2] = pack_bf16x2(pp[0], pp[1]);
+            pk[c2 * 16 + c / 2 + 1] = pack_bf16x2(pp[2], pp[3]);
+            dk_[c2 * 16 + c / 2] = pack_bf16x2(dd[0], dd[1]);
+            dk_[c2 * 16 + c / 2 + 1] = pack_bf16x2(dd[2], dd[3]);
           }
         }
         // this thread's row is read: P^T / dS^T over its first 32 columns
