@@ -100,6 +100,42 @@ def test_decode_mtp_rejects_bad_q_len(L):
         assert rc == -2   # LOZA_SSA_ERR_SHAPE
 
 
+def test_prefill_bwd_workspace_size(L):
+    from block_sparse_streaming_ssa_b200 import loza_ssa as api
+    # fp32 D per row (256-byte aligned) + fp32 partial dK and dV of every sink
+    # chunk: key block 0 of a 32-block sequence is seen by 32 query blocks,
+    # cut into chunks of 8
+    B, H, L, d = 1, 2, 4096, 128
+    rows = B * H * L
+    d_bytes = -(-rows * 4 // 256) * 256
+    part = B * H * 4 * 2 * 128 * d * 4
+    assert api.loza_ssa_prefill_bwd_workspace_size(B, H, L, d, d, 1, 7) == d_bytes + part
+    # no sink blocks: no partials
+    assert api.loza_ssa_prefill_bwd_workspace_size(B, H, L, d, d, 0, 7) == d_bytes
+    # two sink blocks: 32 - 0 and 32 - 1 query blocks -> 4 + 4 chunks
+    assert api.loza_ssa_prefill_bwd_workspace_size(B, H, L, d, d, 2, 7) == d_bytes + 2 * part
+    # unsupported head dims / windows
+    assert api.loza_ssa_prefill_bwd_workspace_size(B, H, L, 192, 128, 1, 7) == 0
+    assert api.loza_ssa_prefill_bwd_workspace_size(B, H, L, 128, 128, 1, 0) == 0
+
+
+def test_prefill_bwd_rejects_bad_arguments(L):
+    vp = ctypes.c_void_p
+    a = vp(0x1000)
+
+    def call(B=1, H=2, Lq=1024, dqk=128, dv=128, block=128, n_sink=1, n_local=7, ptr=a,
+             ws_bytes=1 << 30):
+        return L.loza_ssa_prefill_bwd(ptr, a, a, a, a, a, a, a, a, B, H, Lq, dqk, dv, block, n_sink,
+                                      n_local, ctypes.c_float(0.08), a, ws_bytes, None)
+    assert call(ptr=None) == -1           # LOZA_SSA_ERR_NULL
+    assert call(B=0) == -2                # LOZA_SSA_ERR_SHAPE
+    assert call(dqk=192) == -3            # LOZA_SSA_ERR_HEAD_DIM
+    assert call(block=64) == -4           # LOZA_SSA_ERR_BLOCK
+    assert call(n_local=0) == -5          # LOZA_SSA_ERR_WINDOW
+    assert call(ptr=vp(0x1002)) == -6     # LOZA_SSA_ERR_ALIGN
+    assert call(ws_bytes=16) == -7        # LOZA_SSA_ERR_WORKSPACE
+
+
 def test_decode_selected_rejects_missing_list(L):
     vp = ctypes.c_void_p
     rc = L.loza_ssa_decode_selected(vp(0x1000), vp(0x1000), vp(0x1000), vp(0x1000), None, 4,
