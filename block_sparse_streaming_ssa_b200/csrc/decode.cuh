@@ -556,42 +556,55 @@ __global__ void __launch_bounds__(kMergeThreads, 4)
   const uint4* op = reinterpret_cast<const uint4*>(p.o_part) + (cta0 * 64 + gp) * 128 + hr;
   constexpr size_t kSplitStride = 64 * 128;  // uint4 per split
   const int n = p.n_split;
+  // One pass, kMergeBatch splits at a time: a batch's LSEs and partial O are
+  // loaded together (one round trip to L2 for the usual four splits), and
+  // the running max only rescales what earlier batches summed.
   float lmax = -INFINITY;
-  for (int s = 0; s < n; ++s) lmax = fmaxf(lmax, __ldg(lsep + (size_t)s * 128));
   float acc[kMergeGroups][8];
 #pragma unroll
   for (int q = 0; q < kMergeGroups; ++q)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[q][e] = 0.f;
   float denom = 0.f;
-  if (lmax > -INFINITY) {
-    for (int s0 = 0; s0 < n; s0 += kMergeBatch) {
-      float ls[kMergeBatch];
-      uint4 raw[kMergeBatch][kMergeGroups];
+  for (int s0 = 0; s0 < n; s0 += kMergeBatch) {
+    float ls[kMergeBatch];
+    uint4 raw[kMergeBatch][kMergeGroups];
 #pragma unroll
-      for (int j = 0; j < kMergeBatch; ++j) {
-        ls[j] = -INFINITY;
-        if (s0 + j < n) {
-          ls[j] = __ldg(lsep + (size_t)(s0 + j) * 128);
+    for (int j = 0; j < kMergeBatch; ++j) {
+      ls[j] = -INFINITY;
+      if (s0 + j < n) {
+        ls[j] = __ldg(lsep + (size_t)(s0 + j) * 128);
 #pragma unroll
-          for (int q = 0; q < kMergeGroups; ++q)
-            raw[j][q] = __ldg(op + (size_t)(s0 + j) * kSplitStride + q * kGroupStride * 128);
-        }
+        for (int q = 0; q < kMergeGroups; ++q)
+          raw[j][q] = __ldg(op + (size_t)(s0 + j) * kSplitStride + q * kGroupStride * 128);
       }
+    }
+    float bmax = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < kMergeBatch; ++j) {
-        if (ls[j] == -INFINITY) continue;
-        const float wgt = __expf(ls[j] - lmax);
-        denom += wgt;
+    for (int j = 0; j < kMergeBatch; ++j) bmax = fmaxf(bmax, ls[j]);
+    if (bmax == -INFINITY) continue;  // only empty splits in this batch
+    if (bmax > lmax) {
+      const float r = __expf(lmax - bmax);  // 0 while nothing is summed yet
+      denom *= r;
 #pragma unroll
-        for (int q = 0; q < kMergeGroups; ++q) {
-          const __half2* hv = reinterpret_cast<const __half2*>(&raw[j][q]);
+      for (int q = 0; q < kMergeGroups; ++q)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __half22float2(hv[e]);
-            acc[q][2 * e] += wgt * f.x;
-            acc[q][2 * e + 1] += wgt * f.y;
-          }
+        for (int e = 0; e < 8; ++e) acc[q][e] *= r;
+      lmax = bmax;
+    }
+#pragma unroll
+    for (int j = 0; j < kMergeBatch; ++j) {
+      if (ls[j] == -INFINITY) continue;  // empty split: its partial O was never written
+      const float wgt = __expf(ls[j] - lmax);
+      denom += wgt;
+#pragma unroll
+      for (int q = 0; q < kMergeGroups; ++q) {
+        const __half2* hv = reinterpret_cast<const __half2*>(&raw[j][q]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(hv[e]);
+          acc[q][2 * e] += wgt * f.x;
+          acc[q][2 * e + 1] += wgt * f.y;
         }
       }
     }
