@@ -275,6 +275,26 @@ def prefill_bwd(q, k, v, dout, blk=128, n_sink=1, n_local=7, scale=None):
     return dq, dk, dvv
 
 
+def prefill_varlen_bwd(q, k, v, dout, cu_seqlens, blk=128, n_sink=1, n_local=7, scale=None):
+    """Gradients of the packed varlen prefill: q, k: [H,total,dqk]; v, dout:
+    [H,total,dv].  Every sequence is its own attention problem (its block
+    indices count from its first token and no key crosses its boundary), so
+    its gradients are those of the dense prefill over its slice; keys and
+    queries of different sequences never meet."""
+    q, k, v, dout = (np.ascontiguousarray(a) for a in (q, k, v, dout))
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    dq = np.empty(q.shape)
+    dk = np.empty(k.shape)
+    dvv = np.empty(v.shape)
+    for a, b in zip(cu[:-1], cu[1:]):
+        if b <= a:
+            continue
+        g = prefill_bwd(q[None, :, a:b], k[None, :, a:b], v[None, :, a:b], dout[None, :, a:b],
+                        blk, n_sink, n_local, scale)
+        dq[:, a:b], dk[:, a:b], dvv[:, a:b] = (x[0] for x in g)
+    return dq, dk, dvv
+
+
 def decode_mtp(q, kv, page_table, seq_lens, dv, page_size=128, n_sink=1, n_local=7, scale=None,
                rows=None):
     """Paged decode with q_len query tokens per sequence: q [B, q_len, Hq, dqk];
