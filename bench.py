@@ -255,21 +255,30 @@ def backward_bench(w, steps, warmup, peaks, world=1):
     recomputation of S = Q K^T, each 2 d per unmasked (i, j) pair (the dK/dV
     kernel recomputes S and dP a second time; that work is not counted)."""
     import torch
-    from block_sparse_streaming_ssa_b200.loza_ssa import loza_ssa_prefill_bwd
+    from block_sparse_streaming_ssa_b200.loza_ssa import (loza_ssa_prefill_bwd,
+                                                          loza_ssa_prefill_varlen_bwd)
     sp = w["spec"]
-    if w["varlen"] or sp.d_qk != sp.d_v or sp.d_qk not in (64, 128):
+    if sp.d_qk != sp.d_v or sp.d_qk not in (64, 128):
         return None
     o, lse = prefill_call(w)
     g = torch.Generator(device="cuda").manual_seed(4242)
     dout = torch.randn(w["v"].shape, generator=g, device="cuda").to(torch.bfloat16)
-    grads = loza_ssa_prefill_bwd(w["q"], w["k"], w["v"], o, lse, dout, scale=sp.scale)
+
+    def bwd(grads=()):
+        if w["varlen"]:
+            return loza_ssa_prefill_varlen_bwd(w["q"], w["k"], w["v"], o, lse, dout, w["cu"],
+                                               w["max_len"], *grads, scale=sp.scale)
+        return loza_ssa_prefill_bwd(w["q"], w["k"], w["v"], o, lse, dout, *grads,
+                                    scale=sp.scale)
+
+    grads = bwd()
     for _ in range(warmup):
-        loza_ssa_prefill_bwd(w["q"], w["k"], w["v"], o, lse, dout, *grads, scale=sp.scale)
+        bwd(grads)
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record()
     for _ in range(steps):
-        loza_ssa_prefill_bwd(w["q"], w["k"], w["v"], o, lse, dout, *grads, scale=sp.scale)
+        bwd(grads)
     t1.record()
     torch.cuda.synchronize()
     ms = max_over_ranks(t0.elapsed_time(t1) / steps)
@@ -282,8 +291,9 @@ def backward_bench(w, steps, warmup, peaks, world=1):
             "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peak,
                          "unit": "TFLOP/s", "frac": round(tf / peak, 4), "traffic": None,
                          "peak_source": peaks["source"] + " (burst bf16 GEMM)",
-                         "note": "whole call: D preprocess, dQ kernel, dK/dV kernel, sink reduce"},
-            "gpu_launches": 4 * steps}
+                         "note": "whole call: D preprocess, dQ kernel, dK/dV kernel, sink reduce"
+                                 + (" (and the packed-sequence prefix setup)" if w["varlen"] else "")},
+            "gpu_launches": (5 if w["varlen"] else 4) * steps}
 
 
 def e2e_prefill(w, steps):

@@ -43,17 +43,63 @@ constexpr int kBwdComputeThreads = 256;
 constexpr int kSinkChunk = 8;        // query blocks per sink work item
 
 struct BwdParams {
-  const float* lse;        // [planes * L], natural log, from the forward pass
-  const float* dsum;       // [planes * L], D_i
-  __nv_bfloat16* dq;       // [planes, L, DIM]
+  const float* lse;        // [planes * plane_rows], natural log, from the forward pass
+  const float* dsum;       // [planes * plane_rows], D_i
+  __nv_bfloat16* dq;       // [planes, plane_rows, DIM]
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
-  float* part;             // sink partials: [planes * sink_items][2][128][DIM] (dK then dV)
+  float* part;             // sink partials: [sink slots][2][128][DIM] (dK then dV)
   int L, planes, n_sink, n_local;
-  int nb;                  // query / key blocks per plane
-  int sink_items;          // sink work items per plane
+  int nb;                  // dense: query / key blocks per plane
+  int sink_items;          // dense: sink work items per plane
   float scale, scale_log2;
+  // Packed variable-length input (cu_seqlens != nullptr): planes = heads,
+  // plane_rows = total tokens, and pfx holds three exclusive prefixes over the
+  // sequences, [3][n_seqs + 1]: dQ work items, dK/dV work items and sink
+  // partial slots (each counted over all heads).
+  const int* cu_seqlens;
+  const int* pfx;
+  int n_seqs;
+  int plane_rows;          // dense: L
 };
+
+// Largest s with a[s] <= x, for a non-decreasing a[0..n] with a[0] = 0 <= x.
+__device__ __forceinline__ int bwd_find(const int* a, int n, int x) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(a + mid) <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// A dQ work item: one query block of one (sequence, head).
+struct BwdQItem {
+  int plane, seq_start, len, qb;
+};
+
+__device__ __forceinline__ int bwd_q_items(const BwdParams& p) {
+  return p.cu_seqlens == nullptr ? p.planes * p.nb : __ldg(p.pfx + p.n_seqs);
+}
+
+__device__ __forceinline__ BwdQItem bwd_q_item(const BwdParams& p, int item) {
+  BwdQItem w;
+  if (p.cu_seqlens == nullptr) {
+    w.plane = item / p.nb;
+    w.qb = item - w.plane * p.nb;
+    w.seq_start = 0;
+    w.len = p.L;
+  } else {
+    const int s = bwd_find(p.pfx, p.n_seqs, item);
+    w.seq_start = __ldg(p.cu_seqlens + s);
+    w.len = __ldg(p.cu_seqlens + s + 1) - w.seq_start;
+    const int nb = (w.len + 127) >> 7;
+    const int r = item - __ldg(p.pfx + s);
+    w.plane = r / nb;
+    w.qb = r - w.plane * nb;
+  }
+  return w;
+}
 
 // Sink work items of one plane: key block j < min(n_sink, nb) is seen by
 // query blocks j .. nb-1, cut into chunks of kSinkChunk.
@@ -66,34 +112,129 @@ __host__ __device__ __forceinline__ int bwd_sink_items(int n_sink, int nb) {
   return n;
 }
 
+// A dK/dV work item: one key block of one (sequence, head) with its query
+// blocks q_lo .. q_hi (a sink block's list is cut into chunks).
 struct BwdKItem {
-  int plane, kb;     // key block
+  int plane, seq_start, len, kb;
   int q_lo, q_hi;    // query blocks q_lo .. q_hi (inclusive)
   int slot;          // sink partial slot, -1 for a regular key block (written directly)
 };
 
+__device__ __forceinline__ int bwd_kv_items(const BwdParams& p) {
+  return p.cu_seqlens == nullptr
+             ? p.planes * (p.sink_items + (p.nb > p.n_sink ? p.nb - p.n_sink : 0))
+             : __ldg(p.pfx + (p.n_seqs + 1) + p.n_seqs);
+}
+
 __device__ __forceinline__ BwdKItem bwd_kv_item(const BwdParams& p, int item) {
-  const int per_plane = p.sink_items + (p.nb > p.n_sink ? p.nb - p.n_sink : 0);
   BwdKItem w;
-  w.plane = item / per_plane;
-  int r = item - w.plane * per_plane;
-  if (r < p.sink_items) {
-    w.slot = w.plane * p.sink_items + r;
+  int nb, sink_items, r, slot0;
+  if (p.cu_seqlens == nullptr) {
+    nb = p.nb;
+    sink_items = p.sink_items;
+    const int per_plane = sink_items + (nb > p.n_sink ? nb - p.n_sink : 0);
+    w.plane = item / per_plane;
+    r = item - w.plane * per_plane;
+    w.seq_start = 0;
+    w.len = p.L;
+    slot0 = w.plane * sink_items;
+  } else {
+    const int* pfx_kv = p.pfx + (p.n_seqs + 1);
+    const int* pfx_sink = pfx_kv + (p.n_seqs + 1);
+    const int s = bwd_find(pfx_kv, p.n_seqs, item);
+    w.seq_start = __ldg(p.cu_seqlens + s);
+    w.len = __ldg(p.cu_seqlens + s + 1) - w.seq_start;
+    nb = (w.len + 127) >> 7;
+    sink_items = bwd_sink_items(p.n_sink, nb);
+    const int per_plane = sink_items + (nb > p.n_sink ? nb - p.n_sink : 0);
+    r = item - __ldg(pfx_kv + s);
+    w.plane = r / per_plane;
+    r -= w.plane * per_plane;
+    slot0 = __ldg(pfx_sink + s) + w.plane * sink_items;
+  }
+  if (r < sink_items) {
+    w.slot = slot0 + r;
     int j = 0;
-    while (r >= bwd_sink_chunks(j, p.nb)) {
-      r -= bwd_sink_chunks(j, p.nb);
+    while (r >= bwd_sink_chunks(j, nb)) {
+      r -= bwd_sink_chunks(j, nb);
       ++j;
     }
     w.kb = j;
     w.q_lo = j + r * kSinkChunk;
-    w.q_hi = min(p.nb - 1, w.q_lo + kSinkChunk - 1);
+    w.q_hi = min(nb - 1, w.q_lo + kSinkChunk - 1);
   } else {
     w.slot = -1;
-    w.kb = p.n_sink + (r - p.sink_items);
+    w.kb = p.n_sink + (r - sink_items);
     w.q_lo = w.kb;
-    w.q_hi = min(p.nb - 1, w.kb + p.n_local - 1);
+    w.q_hi = min(nb - 1, w.kb + p.n_local - 1);
   }
   return w;
+}
+
+// Packed input: the three prefixes of BwdParams::pfx from cu_seqlens, one CTA
+// of 1024 threads.  Invalid cu_seqlens (not starting at 0, not ending at
+// total, decreasing), or more sink slots than the workspace holds, give zero
+// work everywhere and set a device status bit.
+__global__ void __launch_bounds__(1024) ssa_bwd_varlen_setup_kernel(const int* cu, int n_seqs,
+                                                                    int total, int H, int n_sink,
+                                                                    long long slot_capacity,
+                                                                    int* pfx) {
+  __shared__ int warp_tot[3][32];
+  __shared__ int bad;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  if (t == 0) bad = (__ldg(cu) != 0 || __ldg(cu + n_seqs) != total) ? 1 : 0;
+  __syncthreads();
+  const int per = (n_seqs + 1023) / 1024;
+  const int s0 = min(t * per, n_seqs), s1 = min(s0 + per, n_seqs);
+  int loc[3] = {0, 0, 0};
+  for (int s = s0; s < s1; ++s) {
+    const int len = __ldg(cu + s + 1) - __ldg(cu + s);
+    if (len < 0) bad = 1;
+    const int nb = len > 0 ? (len + 127) >> 7 : 0;
+    const int si = bwd_sink_items(n_sink, nb);
+    loc[0] += H * nb;
+    loc[1] += H * (si + (nb > n_sink ? nb - n_sink : 0));
+    loc[2] += H * si;
+  }
+  int inc[3];
+#pragma unroll
+  for (int a = 0; a < 3; ++a) {
+    inc[a] = loc[a];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, inc[a], off);
+      if (lane >= off) inc[a] += v;
+    }
+    if (lane == 31) warp_tot[a][warp] = inc[a];
+  }
+  __syncthreads();
+  if (warp == 0) {
+#pragma unroll
+    for (int a = 0; a < 3; ++a) {
+      int v = warp_tot[a][lane];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += u;
+      }
+      warp_tot[a][lane] = v;  // inclusive over warps
+    }
+  }
+  __syncthreads();
+  const bool invalid = bad != 0 || (long long)warp_tot[2][31] > slot_capacity;
+#pragma unroll
+  for (int a = 0; a < 3; ++a) {
+    int run = inc[a] - loc[a] + (warp > 0 ? warp_tot[a][warp - 1] : 0);
+    for (int s = s0; s < s1; ++s) {
+      pfx[a * (n_seqs + 1) + s] = invalid ? 0 : run;
+      const int len = __ldg(cu + s + 1) - __ldg(cu + s);
+      const int nb = len > 0 ? (len + 127) >> 7 : 0;
+      const int si = bwd_sink_items(n_sink, nb);
+      run += a == 0 ? H * nb : a == 1 ? H * (si + (nb > n_sink ? nb - n_sink : 0)) : H * si;
+    }
+    if (t == 1023) pfx[a * (n_seqs + 1) + n_seqs] = invalid ? 0 : warp_tot[a][31];
+  }
+  if (t == 0 && invalid) atomicOr(&g_loza_status, 8);
 }
 
 // ---------------------------------------------------------------- D_i
@@ -177,7 +318,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   auto bar = [&](int i) -> uint32_t { return sb + Lay::OFF_BAR + 8 * i; };
   int* status = &g_loza_status;
-  const int total_items = p.planes * p.nb;
+  const int total_items = bwd_q_items(p);
 
   if (threadIdx.x == 0) {
     mbar_init(bar(Lay::B_QD_FULL), 1);
@@ -223,8 +364,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int k_issued[Lay::KST] = {}, v_issued[Lay::VST] = {};
       bool ok = true;
       for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++it) {
-        const int plane = item / p.nb, qb = item - plane * p.nb;
-        const TileRange tr = tile_range(qb, p.n_sink, p.n_local);
+        const BwdQItem w = bwd_q_item(p, item);
+        const TileRange tr = tile_range(w.qb, p.n_sink, p.n_local);
         if (it > 0 && !mbar_wait(bar(Lay::B_QD_EMPTY), (it - 1) & 1, abort_flag, status, 1)) {
           ok = false;
           break;
@@ -234,12 +375,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int c = 0; c < Lay::CH; ++c) {
           tma_load_3d(sb + Lay::OFF_Q + c * Lay::CHUNK, &tm_q, bar(Lay::B_QD_FULL), c * 64,
-                      qb * 128, plane);
+                      w.seq_start + w.qb * 128, w.plane);
           tma_load_3d(sb + Lay::OFF_DO + c * Lay::CHUNK, &tm_do, bar(Lay::B_QD_FULL), c * 64,
-                      qb * 128, plane);
+                      w.seq_start + w.qb * 128, w.plane);
         }
         for (int t = 0; t < tr.count; ++t, ++g) {
-          const int row = tile_block(tr, t) * 128;
+          const int row = w.seq_start + tile_block(tr, t) * 128;
           const int st = g % Lay::KST, use = g / Lay::KST;
           if (use > 0 &&
               !mbar_wait(bar(Lay::B_K_EMPTY + st), (use - 1) & 1, abort_flag, status, 1)) {
@@ -251,7 +392,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int c = 0; c < Lay::CH; ++c)
             tma_load_3d(sb + Lay::OFF_K + st * Lay::TILE + c * Lay::CHUNK, &tm_k,
-                        bar(Lay::B_K_FULL + st), c * 64, row, plane);
+                        bar(Lay::B_K_FULL + st), c * 64, row, w.plane);
           const int vs = g % Lay::VST, vuse = g / Lay::VST;
           if (vuse > 0 &&
               !mbar_wait(bar(Lay::B_V_EMPTY + vs), (vuse - 1) & 1, abort_flag, status, 1)) {
@@ -263,7 +404,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int c = 0; c < Lay::CH; ++c)
             tma_load_3d(sb + Lay::OFF_V + vs * Lay::TILE + c * Lay::CHUNK, &tm_v,
-                        bar(Lay::B_V_FULL + vs), c * 64, row, plane);
+                        bar(Lay::B_V_FULL + vs), c * 64, row, w.plane);
         }
       }
       if (!ok) {
@@ -289,8 +430,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int g = 0, it = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++it) {
-        const int qb = item % p.nb;
-        const TileRange tr = tile_range(qb, p.n_sink, p.n_local);
+        const TileRange tr = tile_range(bwd_q_item(p, item).qb, p.n_sink, p.n_local);
         if (!(ok = mbar_wait(bar(Lay::B_QD_FULL), it & 1, abort_flag, status, 1))) break;
         for (int t = 0; t < tr.count; ++t, ++g) {
           const int st = g % Lay::KST, vs = g % Lay::VST;
@@ -331,8 +471,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int g = 0, it = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++it) {
-        const int qb = item % p.nb;
-        const TileRange tr = tile_range(qb, p.n_sink, p.n_local);
+        const TileRange tr = tile_range(bwd_q_item(p, item).qb, p.n_sink, p.n_local);
         for (int t = 0; t < tr.count; ++t, ++g) {
           const int st = g % Lay::KST;
           // K(g) is in place (its slot is released only by this issuer) and
@@ -367,12 +506,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const float sl2 = p.scale_log2;
     int g = 0, it = 0;
     for (int item = blockIdx.x; item < total_items; item += gridDim.x, ++it) {
-      const int plane = item / p.nb, qb = item - plane * p.nb;
-      const TileRange tr = tile_range(qb, p.n_sink, p.n_local);
-      const int r_in_seq = qb * 128 + row;
-      const bool valid = r_in_seq < p.L;
-      const size_t grow = (size_t)plane * p.L + r_in_seq;
-      // rows past L: zero Q and dO rows (TMA fill), and P = 0 here
+      const BwdQItem w = bwd_q_item(p, item);
+      const TileRange tr = tile_range(w.qb, p.n_sink, p.n_local);
+      const int r_in_seq = w.qb * 128 + row;
+      const bool valid = r_in_seq < w.len;
+      const size_t grow = (size_t)w.plane * p.plane_rows + w.seq_start + r_in_seq;
+      // rows past the sequence: P = 0 here, and their dQ is not written
       const float lse2 = valid ? __ldg(p.lse + grow) * 1.4426950408889634f : INFINITY;
       const float dsum = valid ? __ldg(p.dsum + grow) : 0.f;
       bool ok = true;
@@ -507,8 +646,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   auto bar = [&](int i) -> uint32_t { return sb + Lay::OFF_BAR + 8 * i; };
   int* status = &g_loza_status;
-  const int per_plane = p.sink_items + (p.nb > p.n_sink ? p.nb - p.n_sink : 0);
-  const int total_items = p.planes * per_plane;
+  const int total_items = bwd_kv_items(p);
 
   if (threadIdx.x == 0) {
     mbar_init(bar(Lay::B_KV_FULL), 1);
@@ -561,9 +699,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int c = 0; c < Lay::CH; ++c) {
           tma_load_3d(sb + Lay::OFF_K + c * Lay::CHUNK, &tm_k, bar(Lay::B_KV_FULL), c * 64,
-                      w.kb * 128, w.plane);
+                      w.seq_start + w.kb * 128, w.plane);
           tma_load_3d(sb + Lay::OFF_V + c * Lay::CHUNK, &tm_v, bar(Lay::B_KV_FULL), c * 64,
-                      w.kb * 128, w.plane);
+                      w.seq_start + w.kb * 128, w.plane);
         }
         for (int qi = w.q_lo; qi <= w.q_hi; ++qi, ++s) {
           const int st = s % Lay::QST, use = s / Lay::QST;
@@ -577,10 +715,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const uint32_t base = sb + Lay::OFF_Q + st * 2 * Lay::TILE;
 #pragma unroll
           for (int c = 0; c < Lay::CH; ++c) {
-            tma_load_3d(base + c * Lay::CHUNK, &tm_q, bar(Lay::B_Q_FULL + st), c * 64, qi * 128,
-                        w.plane);
+            tma_load_3d(base + c * Lay::CHUNK, &tm_q, bar(Lay::B_Q_FULL + st), c * 64,
+                        w.seq_start + qi * 128, w.plane);
             tma_load_3d(base + Lay::TILE + c * Lay::CHUNK, &tm_do, bar(Lay::B_Q_FULL + st),
-                        c * 64, qi * 128, w.plane);
+                        c * 64, w.seq_start + qi * 128, w.plane);
           }
         }
       }
@@ -698,16 +836,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int key = w.kb * 128 + r;
       bool ok = true;
       for (int qi = w.q_lo; qi <= w.q_hi; ++qi, ++s) {
-        // stage lse2 and D of this half's 64 queries (rows past L: 0, harmless:
-        // their Q and dO rows are zero, so their dS^T and dV terms vanish)
+        // stage lse2 and D of this half's 64 queries; rows past the sequence
+        // (zero fill, or the next packed sequence) get lse2 = +inf: P = 0
         float* lse_s = rows_smem + ((s & 1) * 2 + h) * 128;
         float* d_s = lse_s + 64;
         {
           const int t = r & 63;
           const int qrow = qi * 128 + h * 64 + t;
-          const size_t gq = (size_t)w.plane * p.L + qrow;
-          if (r < 64) lse_s[t] = qrow < p.L ? __ldg(p.lse + gq) * 1.4426950408889634f : 0.f;
-          else d_s[t] = qrow < p.L ? __ldg(p.dsum + gq) : 0.f;
+          const size_t gq = (size_t)w.plane * p.plane_rows + w.seq_start + qrow;
+          if (r < 64) lse_s[t] = qrow < w.len ? __ldg(p.lse + gq) * 1.4426950408889634f : INFINITY;
+          else d_s[t] = qrow < w.len ? __ldg(p.dsum + gq) : 0.f;
         }
         mbar_arrive(bar(Lay::B_SYNC + h));
         if (!mbar_wait(bar(Lay::B_SYNC + h), s & 1, abort_flag, status, 1) ||
@@ -759,7 +897,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!mbar_wait(bar(Lay::B_ACC_FULL), it & 1, abort_flag, status, 1)) break;
       tc_fence_after();
       constexpr int OH = DIM / 2;
-      const size_t grow = (size_t)w.plane * p.L + key;
+      const size_t grow = (size_t)w.plane * p.plane_rows + w.seq_start + key;
 #pragma unroll 1
       for (int which = 0; which < 2; ++which) {  // 0: dK, 1: dV
         const float mul = which == 0 ? p.scale : 1.f;
@@ -780,7 +918,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                               __uint_as_float(ar[ch][e + 1]) * mul,
                               __uint_as_float(ar[ch][e + 2]) * mul,
                               __uint_as_float(ar[ch][e + 3]) * mul);
-        } else if (key < p.L) {
+        } else if (key < w.len) {
           uint4* dst = reinterpret_cast<uint4*>((which == 0 ? p.dk : p.dv) + grow * DIM + h * OH);
 #pragma unroll
           for (int ch = 0; ch < OH / 32; ++ch)
@@ -810,11 +948,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 // The sink blocks' dK, dV: the sum of their chunks' fp32 partials, as bf16.
-// One thread per (plane, sink block, key row, 4 columns).
+// Dense: one thread per (plane, sink block, key row, 4 columns).  Packed:
+// blockIdx.y is the sequence and the threads of its column of CTAs walk its
+// (head, sink block, key row, 4 columns).
 template <int DIM>
 __global__ void __launch_bounds__(256) ssa_bwd_sink_reduce_kernel(const BwdParams p) {
-  const int n_sink = min(p.n_sink, p.nb);
-  const long long quads = (long long)p.planes * n_sink * 128 * (DIM / 4);
+  int n_sink, nb, len, seq_start, planes;
+  long long slot_base;  // slot of chunk 0 of sink block 0 of head 0
+  int per_head;         // sink slots per head
+  if (p.cu_seqlens == nullptr) {
+    nb = p.nb;
+    len = p.L;
+    seq_start = 0;
+    planes = p.planes;
+    slot_base = 0;
+    per_head = p.sink_items;
+  } else {
+    const int sq = blockIdx.y;
+    seq_start = __ldg(p.cu_seqlens + sq);
+    len = __ldg(p.cu_seqlens + sq + 1) - seq_start;
+    if (len <= 0) return;
+    nb = (len + 127) >> 7;
+    planes = p.planes;
+    const int* pfx_sink = p.pfx + 2 * (p.n_seqs + 1);
+    slot_base = __ldg(pfx_sink + sq);
+    per_head = bwd_sink_items(p.n_sink, nb);
+    if (__ldg(pfx_sink + p.n_seqs) == 0) return;  // invalid cu_seqlens: nothing was computed
+  }
+  n_sink = min(p.n_sink, nb);
+  const long long quads = (long long)planes * n_sink * 128 * (DIM / 4);
   for (long long x = blockIdx.x * (long long)blockDim.x + threadIdx.x; x < quads;
        x += (long long)gridDim.x * blockDim.x) {
     const int c4 = (int)(x % (DIM / 4));
@@ -822,18 +984,18 @@ __global__ void __launch_bounds__(256) ssa_bwd_sink_reduce_kernel(const BwdParam
     const int j = (int)((x / (DIM / 4) / 128) % n_sink);
     const int plane = (int)(x / (DIM / 4) / 128 / n_sink);
     const int key = j * 128 + r;
-    if (key >= p.L) continue;
-    int slot = plane * p.sink_items;
-    for (int j2 = 0; j2 < j; ++j2) slot += bwd_sink_chunks(j2, p.nb);
+    if (key >= len) continue;
+    long long slot = slot_base + (long long)plane * per_head;
+    for (int j2 = 0; j2 < j; ++j2) slot += bwd_sink_chunks(j2, nb);
     float4 ak = make_float4(0.f, 0.f, 0.f, 0.f), av = ak;
-    for (int c = 0; c < bwd_sink_chunks(j, p.nb); ++c) {
+    for (int c = 0; c < bwd_sink_chunks(j, nb); ++c) {
       const float* base = p.part + ((size_t)(slot + c) * 2 * 128 + r) * DIM + 4 * c4;
       const float4 k4 = *reinterpret_cast<const float4*>(base);
       const float4 v4 = *reinterpret_cast<const float4*>(base + (size_t)128 * DIM);
       ak.x += k4.x; ak.y += k4.y; ak.z += k4.z; ak.w += k4.w;
       av.x += v4.x; av.y += v4.y; av.z += v4.z; av.w += v4.w;
     }
-    const size_t grow = (size_t)plane * p.L + key;
+    const size_t grow = (size_t)plane * p.plane_rows + seq_start + key;
     uint2 ko, vo;
     ko.x = pack_bf16x2(ak.x, ak.y);
     ko.y = pack_bf16x2(ak.z, ak.w);

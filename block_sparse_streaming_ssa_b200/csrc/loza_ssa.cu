@@ -163,17 +163,20 @@ BwdWorkspace bwd_workspace(long long planes, int L, int dim, int n_sink) {
   return w;
 }
 
+// q_items / kv_items: the work-item counts (dense) or upper bounds on them
+// (packed: the kernels read the exact counts from the prefixes).
 template <int DIM>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
-               loza::BwdParams prm, cudaStream_t s, const DeviceInfo& dev) {
+               loza::BwdParams prm, long long q_items, long long kv_items, cudaStream_t s,
+               const DeviceInfo& dev) {
   CUtensorMap mq, mk, mv, mdo;
   int rc;
-  const uint64_t L = (uint64_t)prm.L, planes = (uint64_t)prm.planes;
+  const uint64_t L = (uint64_t)prm.plane_rows, planes = (uint64_t)prm.planes;
   if ((rc = make_map(&mq, q, DIM, L, planes, 3)) != LOZA_SSA_OK) return rc;
   if ((rc = make_map(&mk, k, DIM, L, planes, 3)) != LOZA_SSA_OK) return rc;
   if ((rc = make_map(&mv, v, DIM, L, planes, 3)) != LOZA_SSA_OK) return rc;
   if ((rc = make_map(&mdo, dout, DIM, L, planes, 3)) != LOZA_SSA_OK) return rc;
-  const long long rows = (long long)prm.planes * prm.L;
+  const long long rows = (long long)prm.planes * prm.plane_rows;
   const int pre_grid = (int)std::min<long long>((rows + 63) / 64, (long long)dev.num_sms * 16);
   loza::ssa_bwd_preprocess_kernel<DIM><<<pre_grid, 256, 0, s>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout),
@@ -186,9 +189,9 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, LQ::SMEM_BYTES)) !=
       cudaSuccess)
     return cuda_fail(e, "cudaFuncSetAttribute(backward dq)");
-  const long long dq_items = (long long)prm.planes * prm.nb;
-  loza::ssa_bwd_dq_kernel<DIM><<<(int)std::min<long long>(dq_items, dev.num_sms), loza::kBwdThreads,
-                                 LQ::SMEM_BYTES, s>>>(mq, mk, mv, mdo, prm);
+  if (q_items > 0)
+    loza::ssa_bwd_dq_kernel<DIM><<<(int)std::min<long long>(q_items, dev.num_sms),
+                                   loza::kBwdThreads, LQ::SMEM_BYTES, s>>>(mq, mk, mv, mdo, prm);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward dq launch");
 
   using LK = loza::BwdKvLayout<DIM>;
@@ -196,16 +199,19 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, LK::SMEM_BYTES)) !=
       cudaSuccess)
     return cuda_fail(e, "cudaFuncSetAttribute(backward dkdv)");
-  const long long kv_items =
-      (long long)prm.planes * (prm.sink_items + (prm.nb > prm.n_sink ? prm.nb - prm.n_sink : 0));
-  loza::ssa_bwd_dkdv_kernel<DIM><<<(int)std::min<long long>(kv_items, dev.num_sms),
-                                   loza::kBwdThreads, LK::SMEM_BYTES, s>>>(mq, mk, mv, mdo, prm);
+  if (kv_items > 0)
+    loza::ssa_bwd_dkdv_kernel<DIM><<<(int)std::min<long long>(kv_items, dev.num_sms),
+                                     loza::kBwdThreads, LK::SMEM_BYTES, s>>>(mq, mk, mv, mdo, prm);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward dkdv launch");
 
-  if (prm.sink_items > 0) {
+  if (prm.cu_seqlens == nullptr && prm.sink_items > 0) {
     const long long quads = (long long)prm.planes * std::min(prm.n_sink, prm.nb) * 128 * (DIM / 4);
     const int red_grid = (int)std::min<long long>((quads + 255) / 256, (long long)dev.num_sms * 8);
     loza::ssa_bwd_sink_reduce_kernel<DIM><<<red_grid, 256, 0, s>>>(prm);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward reduce launch");
+  } else if (prm.cu_seqlens != nullptr && prm.n_sink > 0) {
+    // one column of CTAs per sequence; each walks its (head, sink block, row, 4 columns)
+    loza::ssa_bwd_sink_reduce_kernel<DIM><<<dim3(8, prm.n_seqs), 256, 0, s>>>(prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward reduce launch");
   }
   return LOZA_SSA_OK;
@@ -390,9 +396,108 @@ int loza_ssa_prefill_bwd(const void* q, const void* k, const void* v, const void
   prm.sink_items = (int)sink_items;
   prm.scale = scale;
   prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.cu_seqlens = nullptr;
+  prm.pfx = nullptr;
+  prm.n_seqs = B;
+  prm.plane_rows = L;
+  const long long q_items = planes * nb;
+  const long long kv_items = planes * (sink_items + (nb > n_sink ? nb - n_sink : 0));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d_qk == 64) return launch_bwd<64>(q, k, v, o, dout, prm, s, dev);
-  return launch_bwd<128>(q, k, v, o, dout, prm, s, dev);
+  if (d_qk == 64) return launch_bwd<64>(q, k, v, o, dout, prm, q_items, kv_items, s, dev);
+  return launch_bwd<128>(q, k, v, o, dout, prm, q_items, kv_items, s, dev);
+}
+
+// Packed backward workspace: D per row, the three prefixes, then the sink
+// partials for an upper bound on the sink slots: sequence s has at most
+// n_sink sink blocks of at most ceil(nb_s / 8) chunks, and
+// sum_s nb_s <= total / 128 + n_seqs (the bound holds whatever the lengths;
+// the setup kernel also refuses a count above it).
+struct BwdVarlenWorkspace {
+  size_t d_bytes, pfx_bytes, part_bytes;
+  long long q_items_upper, kv_items_upper, sink_slots;
+};
+BwdVarlenWorkspace bwd_varlen_workspace(int n_seqs, int total, int max_seqlen, int H, int dim,
+                                        int n_sink, int n_local) {
+  (void)n_local;
+  BwdVarlenWorkspace w;
+  (void)max_seqlen;
+  const long long sum_nb = (long long)total / 128 + n_seqs;
+  const long long sink_slots =
+      (long long)H * n_sink * ((sum_nb + 7 * (long long)n_seqs) / 8 + n_seqs);
+  w.d_bytes = (size_t)((((long long)H * total * 4) + 255) / 256) * 256;
+  w.pfx_bytes = (size_t)((3 * ((long long)n_seqs + 1) * 4 + 255) / 256) * 256;
+  w.part_bytes = (size_t)sink_slots * 2 * 128 * dim * 4;
+  w.q_items_upper = (long long)H * sum_nb;
+  w.kv_items_upper = w.q_items_upper + sink_slots;
+  w.sink_slots = sink_slots;
+  return w;
+}
+
+size_t loza_ssa_prefill_varlen_bwd_workspace_size(int n_seqs, int total_tokens, int max_seqlen,
+                                                  int H, int d_qk, int d_v, int n_sink,
+                                                  int n_local) {
+  if (n_seqs < 1 || n_seqs > kMaxVarlenSeqs || total_tokens < 1 || max_seqlen < 1 || H < 1 ||
+      d_qk != d_v || (d_qk != 64 && d_qk != 128) || n_sink < 0 || n_local < 1)
+    return 0;
+  const BwdVarlenWorkspace w =
+      bwd_varlen_workspace(n_seqs, total_tokens, max_seqlen, H, d_qk, n_sink, n_local);
+  return w.d_bytes + w.pfx_bytes + w.part_bytes;
+}
+
+int loza_ssa_prefill_varlen_bwd(const void* q, const void* k, const void* v, const void* o,
+                                const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                                const int* cu_seqlens, int n_seqs, int total_tokens,
+                                int max_seqlen, int H, int d_qk, int d_v, int block, int n_sink,
+                                int n_local, float scale, void* workspace, size_t workspace_bytes,
+                                loza_ssa_stream_t stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !cu_seqlens)
+    return LOZA_SSA_ERR_NULL;
+  if (n_seqs < 1 || n_seqs > kMaxVarlenSeqs || total_tokens < 1 || max_seqlen < 1 || H < 1 ||
+      !std::isfinite(scale))
+    return LOZA_SSA_ERR_SHAPE;
+  if (d_qk != d_v || (d_qk != 64 && d_qk != 128)) return LOZA_SSA_ERR_HEAD_DIM;
+  if (block != 128) return LOZA_SSA_ERR_BLOCK;
+  if (n_sink < 0 || n_local < 1) return LOZA_SSA_ERR_WINDOW;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+      !aligned(lse, 4) || !aligned(cu_seqlens, 4))
+    return LOZA_SSA_ERR_ALIGN;
+  const BwdVarlenWorkspace w =
+      bwd_varlen_workspace(n_seqs, total_tokens, max_seqlen, H, d_qk, n_sink, n_local);
+  if (w.kv_items_upper >= (1ll << 31)) return LOZA_SSA_ERR_SHAPE;
+  const size_t need = w.d_bytes + w.pfx_bytes + w.part_bytes;
+  if (!workspace || workspace_bytes < need) return LOZA_SSA_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return LOZA_SSA_ERR_ALIGN;
+  DeviceInfo dev;
+  int rc = device_info(dev);
+  if (rc != LOZA_SSA_OK) return rc;
+  char* ws = static_cast<char*>(workspace);
+  int* pfx = reinterpret_cast<int*>(ws + w.d_bytes);
+  loza::BwdParams prm{};
+  prm.lse = lse;
+  prm.dsum = reinterpret_cast<const float*>(ws);
+  prm.part = reinterpret_cast<float*>(ws + w.d_bytes + w.pfx_bytes);
+  prm.dq = static_cast<__nv_bfloat16*>(dq);
+  prm.dk = static_cast<__nv_bfloat16*>(dk);
+  prm.dv = static_cast<__nv_bfloat16*>(dv);
+  prm.L = max_seqlen;
+  prm.planes = H;
+  prm.n_sink = n_sink;
+  prm.n_local = n_local;
+  prm.scale = scale;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.cu_seqlens = cu_seqlens;
+  prm.pfx = pfx;
+  prm.n_seqs = n_seqs;
+  prm.plane_rows = total_tokens;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  loza::ssa_bwd_varlen_setup_kernel<<<1, 1024, 0, s>>>(cu_seqlens, n_seqs, total_tokens, H,
+                                                        n_sink, w.sink_slots, pfx);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "backward varlen setup launch");
+  if (d_qk == 64)
+    return launch_bwd<64>(q, k, v, o, dout, prm, w.q_items_upper, w.kv_items_upper, s, dev);
+  return launch_bwd<128>(q, k, v, o, dout, prm, w.q_items_upper, w.kv_items_upper, s, dev);
 }
 
 int loza_ssa_prefill_varlen(const void* q, const void* k, const void* v, void* o, float* lse,

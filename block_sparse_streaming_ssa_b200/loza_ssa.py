@@ -69,6 +69,13 @@ def lib() -> ctypes.CDLL:
         L.loza_ssa_prefill_bwd.restype = i32
         L.loza_ssa_prefill_bwd_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32, i32]
         L.loza_ssa_prefill_bwd_workspace_size.restype = sz
+        L.loza_ssa_prefill_varlen_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32,
+                                                  i32, i32, i32, i32, i32, i32, i32, i32, f32,
+                                                  vp, sz, vp]
+        L.loza_ssa_prefill_varlen_bwd.restype = i32
+        L.loza_ssa_prefill_varlen_bwd_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32,
+                                                                 i32, i32]
+        L.loza_ssa_prefill_varlen_bwd_workspace_size.restype = sz
         L.loza_ssa_status_string.argtypes = [i32]
         L.loza_ssa_status_string.restype = ctypes.c_char_p
         L.loza_ssa_last_error_string.argtypes = []
@@ -201,6 +208,45 @@ def loza_ssa_prefill_bwd(q, k, v, o, lse, dout, dq=None, dk=None, dv=None, block
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
         B, H, L, d_qk, d_v, block, n_sink, n_local, float(scale), _ptr(workspace),
         workspace.numel(), _stream(stream)))
+    return dq, dk, dv
+
+
+def loza_ssa_prefill_varlen_bwd_workspace_size(n_seqs, total, max_seqlen, H, d_qk, d_v,
+                                               n_sink=1, n_local=7) -> int:
+    return int(lib().loza_ssa_prefill_varlen_bwd_workspace_size(n_seqs, total, max_seqlen, H,
+                                                                d_qk, d_v, n_sink, n_local))
+
+
+def loza_ssa_prefill_varlen_bwd(q, k, v, o, lse, dout, cu_seqlens, max_seqlen, dq=None, dk=None,
+                                dv=None, block=128, n_sink=1, n_local=7, scale=None,
+                                workspace=None, stream=None):
+    """Gradients of loza_ssa_prefill_varlen.  q, k: bf16 [H,total,d]; v, o,
+    dout: bf16 [H,total,d]; lse: fp32 [H,total]; cu_seqlens: int32 CUDA
+    [n_seqs+1].  Returns (dq, dk, dv)."""
+    for t, dt, name in ((q, torch.bfloat16, "q"), (k, torch.bfloat16, "k"),
+                        (v, torch.bfloat16, "v"), (o, torch.bfloat16, "o"),
+                        (lse, torch.float32, "lse"), (dout, torch.bfloat16, "dout"),
+                        (cu_seqlens, torch.int32, "cu_seqlens")):
+        _need(t, dt, name)
+    H, total, d_qk = q.shape
+    d_v = v.shape[-1]
+    n_seqs = cu_seqlens.numel() - 1
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for t, name in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _need(t, torch.bfloat16, name)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d_qk)
+    need = loza_ssa_prefill_varlen_bwd_workspace_size(n_seqs, total, int(max_seqlen), H, d_qk,
+                                                      d_v, n_sink, n_local)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _need(workspace, torch.uint8, "workspace")
+    _check(lib().loza_ssa_prefill_varlen_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+        _ptr(cu_seqlens), n_seqs, total, int(max_seqlen), H, d_qk, d_v, block, n_sink, n_local,
+        float(scale), _ptr(workspace), workspace.numel(), _stream(stream)))
     return dq, dk, dv
 
 

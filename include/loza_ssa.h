@@ -126,6 +126,35 @@ size_t loza_ssa_prefill_bwd_workspace_size(int B, int H, int L, int d_qk, int d_
                                            int n_local);
 
 /*
+ * Backward of the packed varlen prefill (loza_ssa_prefill_varlen's
+ * gradients).  Every sequence is its own attention problem: its gradients are
+ * those of the dense backward over its slice, and no key of one sequence
+ * reaches another's.
+ *   q, k, dq, dk : bf16 [H, total_tokens, d]   v, o, dout, dv : bf16 [H, total_tokens, d]
+ *   lse          : fp32 [H, total_tokens]      cu_seqlens     : DEVICE int32 [n_seqs + 1]
+ *   1 <= n_seqs <= 4000; d_qk == d_v in {64, 128}; max_seqlen only has to be >= 1.
+ *   workspace    : DEVICE scratch of at least
+ *                  loza_ssa_prefill_varlen_bwd_workspace_size(...) bytes,
+ *                  256-byte aligned, owned by the caller.
+ * Invalid cu_seqlens (not 0 .. total_tokens, or decreasing) compute nothing
+ * and set LOZA_SSA_DEV_BAD_CU_SEQLENS in the device status word.  Other
+ * statuses as for loza_ssa_prefill_bwd.
+ */
+int loza_ssa_prefill_varlen_bwd(const void* q, const void* k, const void* v, const void* o,
+                                const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                                const int* cu_seqlens, int n_seqs, int total_tokens,
+                                int max_seqlen, int H, int d_qk, int d_v, int block, int n_sink,
+                                int n_local, float scale, void* workspace, size_t workspace_bytes,
+                                loza_ssa_stream_t stream);
+
+/* Bytes of workspace loza_ssa_prefill_varlen_bwd needs (0 on invalid
+ * arguments): an upper bound that holds for any lengths summing to
+ * total_tokens. */
+size_t loza_ssa_prefill_varlen_bwd_workspace_size(int n_seqs, int total_tokens, int max_seqlen,
+                                                  int H, int d_qk, int d_v, int n_sink,
+                                                  int n_local);
+
+/*
  * Paged SSA decode, absorbed-MLA layout: one new query token per sequence,
  * H_q query heads all attending one shared latent key/value row per token.
  *   q          : bf16 [B, H_q, d_qk]

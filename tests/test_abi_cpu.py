@@ -136,6 +136,36 @@ def test_prefill_bwd_rejects_bad_arguments(L):
     assert call(ws_bytes=16) == -7        # LOZA_SSA_ERR_WORKSPACE
 
 
+def test_prefill_varlen_bwd_workspace_size(L):
+    from block_sparse_streaming_ssa_b200 import loza_ssa as api
+    # D per row + 3 prefixes of n_seqs + 1 ints + an upper bound on the sink
+    # slots: H * n_sink * ((total/128 + n_seqs + 7 n_seqs) / 8 + n_seqs)
+    n, total, H, d = 3, 5000, 2, 64
+    d_bytes = -(-H * total * 4 // 256) * 256
+    pfx = -(-3 * (n + 1) * 4 // 256) * 256
+    slots = H * 1 * ((total // 128 + n + 7 * n) // 8 + n)
+    want = d_bytes + pfx + slots * 2 * 128 * d * 4
+    assert api.loza_ssa_prefill_varlen_bwd_workspace_size(n, total, 4000, H, d, d, 1, 7) == want
+    assert api.loza_ssa_prefill_varlen_bwd_workspace_size(n, total, 4000, H, d, d, 0, 7) == \
+        d_bytes + pfx
+    assert api.loza_ssa_prefill_varlen_bwd_workspace_size(4001, total, 10, H, d, d, 1, 7) == 0
+    assert api.loza_ssa_prefill_varlen_bwd_workspace_size(n, total, 4000, H, 192, 128, 1, 7) == 0
+
+
+def test_prefill_varlen_bwd_rejects_bad_arguments(L):
+    vp = ctypes.c_void_p
+    a = vp(0x1000)
+
+    def call(n=2, total=300, H=2, d=64, cu=a, ws_bytes=1 << 30):
+        return L.loza_ssa_prefill_varlen_bwd(a, a, a, a, a, a, a, a, a, cu, n, total, 200, H, d, d,
+                                             128, 1, 7, ctypes.c_float(0.1), a, ws_bytes, None)
+    assert call(cu=None) == -1            # LOZA_SSA_ERR_NULL
+    assert call(n=0) == -2                # LOZA_SSA_ERR_SHAPE
+    assert call(d=192) == -3              # LOZA_SSA_ERR_HEAD_DIM
+    assert call(cu=vp(0x1002)) == -6      # LOZA_SSA_ERR_ALIGN
+    assert call(ws_bytes=8) == -7         # LOZA_SSA_ERR_WORKSPACE
+
+
 def test_decode_selected_rejects_missing_list(L):
     vp = ctypes.c_void_p
     rc = L.loza_ssa_decode_selected(vp(0x1000), vp(0x1000), vp(0x1000), vp(0x1000), None, 4,
