@@ -129,7 +129,7 @@ int launch_prefill(const void* q, const void* k, const void* v, loza::PrefillPar
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill)");
   const int grid = items_upper < dev.num_sms ? (int)items_upper : dev.num_sms;
   if (grid < 1) return LOZA_SSA_OK;
-  kern<<<grid, loza::kPrefillThreads, smem, stream>>>(mq, mk, mv, mo, prm);
+  kern<<<grid, Lay::THREADS, smem, stream>>>(mq, mk, mv, mo, prm);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "prefill launch");
   return LOZA_SSA_OK;
 }

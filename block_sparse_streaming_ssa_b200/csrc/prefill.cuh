@@ -19,7 +19,7 @@
 // in TMEM by exp2(m_old - m_new) before the next P.V.  The final O = acc / l
 // and LSE = (m + log2 l) ln 2 are exact for any choice of m.
 //
-// Warp roles (384 threads):
+// Warp roles (384 threads; 512 for d_qk = d_v = 128, see below):
 //   warps 0-7  softmax + correction + epilogue.  Warp w reads TMEM lanes
 //              32*(w%4)..+31 (a warp may only touch its own lane quarter), so
 //              query row r is shared by thread r of warpgroup 0 (key columns
@@ -31,6 +31,13 @@
 //   warp 9     TMEM allocator + issuer of the S = Q K^T MMAs (one elected lane)
 //   warp 10    TMA producer of V (one elected lane)
 //   warp 11    issuer of the O += P V MMAs (one elected lane)
+//   warps 12-15 (d_qk = d_v = 128 only) the epilogue: the softmax warps hand
+//              each item's row max and row sums over through shared memory and
+//              go straight on to the next item; these warps wait for the
+//              item's last P.V, read O from TMEM, normalise it and send it out
+//              through swizzled staging boxes and TMA stores.  The 512 threads
+//              launch with 128 registers each and rebalance with setmaxnreg:
+//              152 for the softmax warpgroups, 104 for the other two.
 // K and V have their own producers so a K load never queues behind a V load
 // that is waiting for its ring slot: S consumes K_{j+1} before P.V reads V_j.
 // S and P.V have their own issuers because an issuer blocks on its barrier
@@ -129,11 +136,21 @@ struct PrefillLayout {
   static constexpr int B_XCHG = B_DRAIN + 2;        // 4
   static constexpr int B_OST_FULL = B_XCHG + 4;     // 2, per warpgroup: box written (128)
   static constexpr int B_OST_FREE = B_OST_FULL + 2; // 2, per warpgroup: box read by its store
-  static constexpr int NBAR = B_OST_FREE + 2;
-  static constexpr int OFF_MISC = OFF_BAR + 256;      // [0] tmem base, [1] abort, [2] items
+  // With an epilogue warpgroup (d_qk = d_v = 128): the softmax warps hand each
+  // item's row max and row sums over in shared memory and go on to the next
+  // item; warps 12-15 normalise O and store it.
+  static constexpr bool EPI_WG = TMA_OUT;
+  static constexpr int THREADS = EPI_WG ? 512 : 384;
+  static constexpr int B_O_FULL = B_OST_FREE + 2;    // NOB: the item's last P.V done (commit)
+  static constexpr int B_ROWS_FULL = B_O_FULL + NOB; // 2: rows published (256)
+  static constexpr int B_ROWS_EMPTY = B_ROWS_FULL + 2;  // 2: rows read by the epilogue (128)
+  static constexpr int NBAR = EPI_WG ? B_ROWS_EMPTY + 2 : B_OST_FREE + 2;
+  static constexpr int BAR_BYTES = EPI_WG ? 512 : 256;
+  static constexpr int OFF_MISC = OFF_BAR + BAR_BYTES;  // [0] tmem base, [1] abort, [2] items
   static constexpr int OFF_RED = OFF_MISC + 16;       // float [2 buffers][2 halves][128 rows]
-  static constexpr int OFF_PREFIX = OFF_RED + 2 * 2 * 128 * 4;
-  static_assert(NBAR * 8 <= 256, "barrier area");
+  static constexpr int OFF_ROWS = OFF_RED + 2 * 2 * 128 * 4;  // float [2 items][m, l0, l1][128]
+  static constexpr int OFF_PREFIX = OFF_ROWS + (EPI_WG ? 2 * 3 * 128 * 4 : 0);
+  static_assert(NBAR * 8 <= BAR_BYTES, "barrier area");
   static constexpr int TMEM_COLS = 512;
   static constexpr int MIN_SMEM = 120 * 1024;  // keeps one CTA (and one TMEM owner) per SM
   static constexpr size_t smem_bytes(int n_prefix) {
@@ -214,11 +231,10 @@ __device__ __forceinline__ void prefill_count_items(const PrefillParams& p, int*
   }
 }
 
-constexpr int kPrefillThreads = 384;
 constexpr int kSoftmaxThreads = 256;
 
 template <int DQK, int DV>
-__global__ void __launch_bounds__(kPrefillThreads, 1)
+__global__ void __launch_bounds__(PrefillLayout<DQK, DV>::THREADS, 1)
     ssa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v,
@@ -253,13 +269,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       mbar_init(bar(Lay::B_P_FULL + s), kSoftmaxThreads);
       mbar_init(bar(Lay::B_S_FREE + s), 1);
     }
-    for (int s = 0; s < Lay::NOB; ++s) mbar_init(bar(Lay::B_O_EMPTY + s), kSoftmaxThreads);
+    for (int s = 0; s < Lay::NOB; ++s)
+      mbar_init(bar(Lay::B_O_EMPTY + s), Lay::EPI_WG ? 128 : kSoftmaxThreads);
     mbar_init(bar(Lay::B_DRAIN), 1);
     mbar_init(bar(Lay::B_DRAIN + 1), 1);
     for (int qd = 0; qd < 4; ++qd) mbar_init(bar(Lay::B_XCHG + qd), 64);
     for (int w = 0; w < 2; ++w) {
       mbar_init(bar(Lay::B_OST_FULL + w), kSoftmaxThreads / 2);
       mbar_init(bar(Lay::B_OST_FREE + w), 1);
+    }
+    if (Lay::EPI_WG) {
+      for (int s = 0; s < Lay::NOB; ++s) mbar_init(bar(Lay::B_O_FULL + s), 1);
+      for (int s = 0; s < 2; ++s) {
+        mbar_init(bar(Lay::B_ROWS_FULL + s), kSoftmaxThreads);
+        mbar_init(bar(Lay::B_ROWS_EMPTY + s), 128);
+      }
     }
     misc[1] = 0;
     fence_barrier_init();
@@ -282,6 +306,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   tc_fence_after();
   const uint32_t tmem = misc[0];
   const int total_items = (int)misc[2];
+  if constexpr (Lay::EPI_WG) {
+    // 512 threads launch with 128 registers each: the softmax warpgroups take
+    // 152, the producer / issuer and epilogue warpgroups keep 104
+    // (2 x 128 x 152 + 2 x 128 x 104 = 65536, the launch's total)
+    if (warp < 8) asm volatile("setmaxnreg.inc.sync.aligned.u32 152;");
+    else asm volatile("setmaxnreg.dec.sync.aligned.u32 104;");
+  }
 
   if (warp == 8) {
     // ------------------------------------------------------- Q / K producer
@@ -443,11 +474,99 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           }
           mma_commit(bar(Lay::B_V_EMPTY + st));
           mma_commit(bar(Lay::B_S_FREE + sbuf));
+          if (Lay::EPI_WG && t == tr.count - 1) mma_commit(bar(Lay::B_O_FULL + ob));
         }
       }
       mma_commit(bar(Lay::B_DRAIN + 1));
       mbar_wait_drain(bar(Lay::B_DRAIN + 1), 0);
     }
+  } else if (Lay::EPI_WG && warp >= 12) {
+    // ------------------------------------------------------ epilogue warpgroup
+    // Per item: the softmax warps' row max and row sums, then O from TMEM once
+    // the item's last P.V is done: O / l as bf16 through the staging boxes and
+    // TMA stores (rows past a packed sequence's end through plain stores),
+    // LSE = (m + log2 l) ln 2.
+    const int row = threadIdx.x - 12 * 32;                        // query row = TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const float* rows_all = reinterpret_cast<const float*>(smem + Lay::OFF_ROWS);
+    int it = 0, n_out = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++it) {
+      const WorkItem w = decode_item(item, p, prefix);
+      const int pr = it & 1, ob = it % Lay::NOB;
+      if (!mbar_wait(bar(Lay::B_ROWS_FULL + pr), (it >> 1) & 1, abort_flag, status, 1)) break;
+      const float* rows = rows_all + pr * 384;
+      const float m = rows[row];
+      const float l_row = rows[128 + row] + rows[256 + row];
+      mbar_arrive(bar(Lay::B_ROWS_EMPTY + pr));
+      if (!mbar_wait(bar(Lay::B_O_FULL + ob), (it / Lay::NOB) & 1, abort_flag, status, 1)) break;
+      tc_fence_after();
+      const int r_in_seq = w.qb * 128 + row;
+      const bool valid = r_in_seq < w.len;
+      const size_t orow = (size_t)w.z * (size_t)p.plane_rows + (size_t)(w.seq_start + r_in_seq);
+      const float inv_l = 1.f / l_row;
+      // dense rows past L fall outside the tensor map and are not written; a
+      // packed sequence's last block would spill into the next sequence
+      const bool tma_out = p.cu_seqlens == nullptr || (w.qb + 1) * 128 <= w.len;
+      if (tma_out && n_out > 0 &&
+          !mbar_wait(bar(Lay::B_OST_FREE), (n_out - 1) & 1, abort_flag, status, 1))
+        break;
+#pragma unroll 1
+      for (int q4 = 0; q4 < 2 * Lay::VCH; ++q4) {  // 32 columns at a time
+        uint32_t orr[32];
+        tmem_ld32(tmem + lane_base + Lay::TM_O + ob * DV + q4 * 32, orr);
+        tmem_wait_ld();
+        if (q4 == 2 * Lay::VCH - 1) {
+          // O buffer free for the item NOB after this one
+          tc_fence_before();
+          mbar_arrive(bar(Lay::B_O_EMPTY + ob));
+        }
+        if (tma_out) {
+          // row `row` of box q4/2 in the 128B-swizzled layout the tensor map
+          // reads: 16-byte unit j at j ^ (row & 7)
+          uint8_t* rowp = smem + Lay::OFF_OST + (q4 >> 1) * Lay::CHUNK + row * 128;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int j = (q4 & 1) * 4 + u;
+            const uint32_t* r8 = &orr[u * 8];
+            *reinterpret_cast<uint4*>(rowp + ((j ^ (row & 7)) << 4)) =
+                make_uint4(pack_bf16x2(__uint_as_float(r8[0]) * inv_l, __uint_as_float(r8[1]) * inv_l),
+                           pack_bf16x2(__uint_as_float(r8[2]) * inv_l, __uint_as_float(r8[3]) * inv_l),
+                           pack_bf16x2(__uint_as_float(r8[4]) * inv_l, __uint_as_float(r8[5]) * inv_l),
+                           pack_bf16x2(__uint_as_float(r8[6]) * inv_l, __uint_as_float(r8[7]) * inv_l));
+          }
+        } else if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(p.o + orow * DV + q4 * 32);
+#pragma unroll
+          for (int v = 0; v < 4; v += 2) {
+            uint32_t w8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              w8[e] = pack_bf16x2(__uint_as_float(orr[8 * v + 2 * e]) * inv_l,
+                                  __uint_as_float(orr[8 * v + 2 * e + 1]) * inv_l);
+            st_global_v8(dst + v, w8);
+          }
+        }
+      }
+      if (tma_out) {
+        fence_async_shared();
+        mbar_arrive(bar(Lay::B_OST_FULL));
+        if (row == 0) {
+          if (!(ok = mbar_wait(bar(Lay::B_OST_FULL), n_out & 1, abort_flag, status, 1))) break;
+#pragma unroll
+          for (int hh = 0; hh < Lay::VCH; ++hh)
+            tma_store_3d(&tm_o, sb + Lay::OFF_OST + hh * Lay::CHUNK, hh * 64,
+                         w.seq_start + w.qb * 128, w.z);
+          tma_store_commit();
+          // the boxes may be rewritten once these stores have read them
+          tma_store_wait_read();
+          mbar_arrive(bar(Lay::B_OST_FREE));
+        }
+        ++n_out;
+      }
+      if (valid) p.lse[orow] = (m + __log2f(l_row)) * kLn2;
+    }
+    if (row == 0) tma_store_wait_all();  // stores done before the CTA exits
   } else {
     // -------------------------------------------- softmax / correction / epilogue
     const int wg = warp >> 2;                                     // column half
@@ -676,12 +795,25 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
       }
       if (!ok) break;
-      prev = Done{w, m, l, ob, g0 + tr.count - 1};
-      have_prev = true;
+      if constexpr (Lay::EPI_WG) {
+        // hand the item's row max and this half's row sums to the epilogue
+        // warpgroup (rows buffer it & 1, read back two items ago)
+        const int pr = it & 1;
+        if (it >= 2 &&
+            !mbar_wait(bar(Lay::B_ROWS_EMPTY + pr), ((it >> 1) - 1) & 1, abort_flag, status, 1))
+          break;
+        float* rows = reinterpret_cast<float*>(smem + Lay::OFF_ROWS) + pr * 384;
+        if (wg == 0) rows[row] = m;
+        rows[128 + wg * 128 + row] = l;
+        mbar_arrive(bar(Lay::B_ROWS_FULL + pr));
+      } else {
+        prev = Done{w, m, l, ob, g0 + tr.count - 1};
+        have_prev = true;
+      }
       g0 += tr.count;
     }
     if (have_prev) epilogue(prev);
-    if (Lay::TMA_OUT && row == 0) tma_store_wait_all();  // stores done before the CTA exits
+    if (Lay::TMA_OUT && !Lay::EPI_WG && row == 0) tma_store_wait_all();  // stores done before exit
   }
 
   __syncwarp();
