@@ -14,7 +14,9 @@ a ~20 GB pool) and reports it under ``decode`` in GB/s of algorithmic bytes,
 and the same decode with 8 distinct selected pages per sequence on top of the
 window under ``decode_selected`` (``--decode-extra``), and the decode with 2
 query tokens per sequence under ``decode_mtp`` (``--decode-mtp``).  The
-prefill's backward pass on the same workload is timed under ``backward``.
+prefill's backward pass on the same workload is timed under ``backward``, and
+full-attention against SSA decode layers at 128K tokens of context under
+``decode_context`` (``--decode-context``).
 
 Under torchrun every rank runs its own replica of the workload (weak scaling,
 no collective on the data path; NCCL only reduces the timing).
@@ -475,6 +477,75 @@ def decode_bench(iters, warmup, peaks, seed=0, len_hi=None, n_sets=8, world=1, n
     }
 
 
+def context_bench(peaks, context=131072, iters=5, warmup=3, world=1, seed=0):
+    """Decode at one long context through the layer-stack call: a full-attention
+    (MLA) layer against an SSA layer, and a 4-layer ZigZag stack (full, SSA,
+    full, SSA -- the QbitAI LoZA article's layout, half the layers SSA) against
+    4 full layers.  32 sequences of ``context`` tokens each, 128 heads, 576/512,
+    every layer with its own query and page pool; a 2x L2 write before every
+    timed call.  Full-attention layers run as the SSA decode with a window of
+    every page."""
+    import torch
+    from block_sparse_streaming_ssa_b200 import synth
+    from block_sparse_streaming_ssa_b200.loza_ssa import (loza_ssa_decode_layers,
+                                                          loza_ssa_decode_layers_workspace_size)
+    s = synth.DECODE
+    lens = [context] * s.B
+    pools = []
+    for i in range(4):
+        q, kv, pt, sl = synth.decode_inputs(lens, s.H_q, s.d_qk, seed=seed + 17 * i,
+                                            device="cuda")
+        pools.append((q, kv))
+        if i == 0:
+            table, seq_lens = pt, sl
+    max_pages = table.shape[1]
+    ws = torch.empty(loza_ssa_decode_layers_workspace_size(s.B, s.H_q, s.d_v, max_pages, 1, 7,
+                                                           True), dtype=torch.uint8,
+                     device="cuda")
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+
+    def timed(pattern):
+        layers = [(pools[i][0], pools[i][1], full) for i, full in enumerate(pattern)]
+        for _ in range(warmup):
+            loza_ssa_decode_layers(layers, table, seq_lens, s.d_v, scale=s.scale, workspace=ws)
+        ev = []
+        for _ in range(iters):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            loza_ssa_decode_layers(layers, table, seq_lens, s.d_v, scale=s.scale, workspace=ws)
+            b.record()
+            ev.append((a, b))
+        torch.cuda.synchronize()
+        return max_over_ranks(statistics.median([a.elapsed_time(b) for a, b in ev]))
+
+    full_ms = timed((True,))
+    ssa_ms = timed((False,))
+    zigzag_ms = timed((True, False, True, False))
+    all_full_ms = timed((True, True, True, True))
+    full_bytes = s.B * (context * s.d_qk * 2 + s.H_q * (s.d_qk * 2 + s.d_v * 2 + 4))
+    full_flops = 2 * (s.d_qk + s.d_v) * s.B * s.H_q * context
+    gbs = full_bytes / (full_ms * 1e-3) / 1e9
+    del pools, ws, flush
+    torch.cuda.empty_cache()
+    return {
+        "workload": f"decode at {context} tokens of context: B={s.B} H_q={s.H_q} d_qk={s.d_qk} "
+                    f"d_v={s.d_v} paged 128, random page permutation, own pool per layer",
+        "full_layer_ms": round(full_ms, 4), "ssa_layer_ms": round(ssa_ms, 4),
+        "layer_speedup": round(full_ms / ssa_ms, 1),
+        "zigzag4_ms": round(zigzag_ms, 4), "full4_ms": round(all_full_ms, 4),
+        "stack_speedup": round(all_full_ms / zigzag_ms, 2),
+        "full_layer_gbs": round(gbs, 1),
+        "full_layer_tflops": round(full_flops / (full_ms * 1e-3) / 1e12, 1),
+        "full_layer_roofline": {"bound": "hbm", "achieved": round(gbs, 1),
+                                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                "frac": round(gbs / peaks["hbm_gbs"], 4),
+                                "peak_source": peaks["source"]},
+        "l2": "2x L2 write before every timed call",
+        "gpu_launches": 2 * (1 + 1 + 4 + 4) * (iters + warmup),
+    }
+
+
 # ----------------------------------------------------------- CPU oracle
 
 def oracle_sample(config, budget_s, seed=0):
@@ -535,6 +606,9 @@ def main():
     ap.add_argument("--decode-mtp", type=int, default=2,
                     help="also time the decode with this many query tokens per sequence "
                          "(<= 1: skip it)")
+    ap.add_argument("--decode-context", type=int, default=131072,
+                    help="also time full-attention vs SSA decode layers at this context "
+                         "(0: skip it)")
     ap.add_argument("--cpu-budget-s", type=float, default=10.0)
     ap.add_argument("--ref-budget-s", type=float, default=60.0,
                     help="--impl reference: CPU seconds over all warm-up and timed steps")
@@ -593,9 +667,11 @@ def main():
         if args.decode_mtp > 1:
             mtp = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
                                len_hi=args.decode_len_hi, world=world, q_len=args.decode_mtp)
+        ctx = (context_bench(peaks, args.decode_context, world=world, seed=rank)
+               if args.decode_context else None)
         if rank == 0:
             print(json.dumps({"metric": METRIC, "decode": decode, "decode_selected": selected,
-                              "decode_mtp": mtp}), flush=True)
+                              "decode_mtp": mtp, "decode_context": ctx}), flush=True)
         if dist:
             torch.distributed.destroy_process_group()
         return
@@ -614,7 +690,7 @@ def main():
     backward = None if args.no_backward else backward_bench(w, max(3, args.steps // 5),
                                                               args.warmup, peaks, world)
     w_desc, w_tokens = w["desc"], w["tokens"]
-    decode = selected = mtp = None
+    decode = selected = mtp = ctx = None
     if not args.no_decode:
         del w
         torch.cuda.empty_cache()
@@ -627,6 +703,8 @@ def main():
         if args.decode_mtp > 1:
             mtp = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
                                len_hi=args.decode_len_hi, world=world, q_len=args.decode_mtp)
+        if args.decode_context:
+            ctx = context_bench(peaks, args.decode_context, world=world, seed=rank)
 
     if rank != 0:
         if dist:
@@ -672,6 +750,7 @@ def main():
         "decode": decode,
         "decode_selected": selected,
         "decode_mtp": mtp,
+        "decode_context": ctx,
     }
     print(json.dumps(line), flush=True)
     if dist:

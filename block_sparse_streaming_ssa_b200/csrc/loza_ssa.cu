@@ -686,6 +686,35 @@ int loza_ssa_decode_selected(const void* q, const void* paged_kv, const int* pag
                      workspace, workspace_bytes, stream);
 }
 
+size_t loza_ssa_decode_layers_workspace_size(int B, int H_q, int d_v, int max_pages, int n_sink,
+                                             int n_local, int any_full) {
+  const size_t ssa = loza_ssa_decode_workspace_size(B, H_q, d_v, n_sink, n_local);
+  if (!any_full) return ssa;
+  const size_t full = loza_ssa_decode_workspace_size(B, H_q, d_v, 0, max_pages);
+  if (ssa == 0 || full == 0) return 0;
+  return full > ssa ? full : ssa;
+}
+
+int loza_ssa_decode_layers(const loza_ssa_decode_layer* layers, int n_layers,
+                           const int* page_table, const int* seq_lens, int B, int H_q, int d_qk,
+                           int d_v, int page_size, int max_pages, int n_pages, int n_sink,
+                           int n_local, float scale, void* workspace, size_t workspace_bytes,
+                           loza_ssa_stream_t stream) {
+  if (!layers) return LOZA_SSA_ERR_NULL;
+  if (n_layers < 1) return LOZA_SSA_ERR_SHAPE;
+  for (int i = 0; i < n_layers; ++i) {
+    const loza_ssa_decode_layer& l = layers[i];
+    // full attention: the window of all max_pages pages ending at the query's
+    const int ws = l.full_attention ? 0 : n_sink;
+    const int wl = l.full_attention ? max_pages : n_local;
+    const int rc = decode_impl(l.q, l.paged_kv, page_table, seq_lens, nullptr, 0, 1, l.o, l.lse,
+                               B, H_q, d_qk, d_v, page_size, max_pages, n_pages, ws, wl, scale,
+                               workspace, workspace_bytes, stream);
+    if (rc != LOZA_SSA_OK) return rc;
+  }
+  return LOZA_SSA_OK;
+}
+
 int loza_ssa_decode_static_scratch(const void* q, const void* paged_kv, const int* page_table,
                                    const int* seq_lens, void* o, float* lse, int B, int H_q,
                                    int d_qk, int d_v, int page_size, int max_pages, int n_pages,

@@ -27,6 +27,12 @@ LOZA_SSA_ERR_SCRATCH_LIMIT = -9
 LOZA_SSA_STATIC_SCRATCH_SLOTS = 128
 
 
+class LozaSsaDecodeLayer(ctypes.Structure):
+    """struct loza_ssa_decode_layer of the C header."""
+    _fields_ = [("q", ctypes.c_void_p), ("paged_kv", ctypes.c_void_p), ("o", ctypes.c_void_p),
+                ("lse", ctypes.c_void_p), ("full_attention", ctypes.c_int)]
+
+
 class LozaSsaError(RuntimeError):
     def __init__(self, status: int, message: str):
         super().__init__(message)
@@ -64,6 +70,12 @@ def lib() -> ctypes.CDLL:
         L.loza_ssa_decode_mtp.restype = i32
         L.loza_ssa_decode_mtp_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
         L.loza_ssa_decode_mtp_workspace_size.restype = sz
+        L.loza_ssa_decode_layers.argtypes = [ctypes.POINTER(LozaSsaDecodeLayer), i32, vp, vp,
+                                             i32, i32, i32, i32, i32, i32, i32, i32, i32, f32,
+                                             vp, sz, vp]
+        L.loza_ssa_decode_layers.restype = i32
+        L.loza_ssa_decode_layers_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32, i32]
+        L.loza_ssa_decode_layers_workspace_size.restype = sz
         L.loza_ssa_prefill_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
                                            i32, i32, i32, i32, f32, vp, sz, vp]
         L.loza_ssa_prefill_bwd.restype = i32
@@ -362,6 +374,52 @@ def loza_ssa_decode_mtp(q, paged_kv, page_table, seq_lens, d_v=512, o=None, lse=
         H_q, d_qk, d_v, page_size, max_pages, n_pages, n_sink, n_local, float(scale),
         _ptr(workspace), workspace.numel(), _stream(stream)))
     return o, lse
+
+
+def loza_ssa_decode_layers_workspace_size(B, H_q, d_v=512, max_pages=1, n_sink=1, n_local=7,
+                                          any_full=True) -> int:
+    return int(lib().loza_ssa_decode_layers_workspace_size(B, H_q, d_v, max_pages, n_sink,
+                                                           n_local, int(bool(any_full))))
+
+
+def loza_ssa_decode_layers(layers, page_table, seq_lens, d_v=512, page_size=128, n_sink=1,
+                           n_local=7, scale=None, workspace=None, stream=None):
+    """One decode step through a stack of layers sharing a page table.
+    layers: sequence of (q bf16 [B,H_q,d_qk], paged_kv bf16 [n_pages,page_size,d_qk],
+    full_attention bool).  Returns a list of (o bf16 [B,H_q,d_v], lse fp32 [B,H_q])."""
+    _need(page_table, torch.int32, "page_table")
+    _need(seq_lens, torch.int32, "seq_lens")
+    if len(layers) == 0:
+        raise ValueError("at least one layer")
+    q0, kv0, _ = layers[0]
+    B, H_q, d_qk = q0.shape
+    n_pages = kv0.shape[0]
+    max_pages = page_table.shape[1]
+    descs = (LozaSsaDecodeLayer * len(layers))()
+    outs = []
+    for i, (q, kv, is_full) in enumerate(layers):
+        _need(q, torch.bfloat16, "q")
+        _need(kv, torch.bfloat16, "paged_kv")
+        if tuple(q.shape) != (B, H_q, d_qk) or kv.shape[0] != n_pages:
+            raise ValueError("every layer needs the same q shape and page-pool size")
+        o = torch.empty((B, H_q, d_v), dtype=torch.bfloat16, device=q.device)
+        lse = torch.empty((B, H_q), dtype=torch.float32, device=q.device)
+        descs[i] = LozaSsaDecodeLayer(q.data_ptr(), kv.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                      int(bool(is_full)))
+        outs.append((o, lse))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d_qk)
+    any_full = any(bool(f) for _, _, f in layers)
+    need = loza_ssa_decode_layers_workspace_size(B, H_q, d_v, max_pages, n_sink, n_local,
+                                                 any_full)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q0.device)
+    _need(workspace, torch.uint8, "workspace")
+    _check(lib().loza_ssa_decode_layers(
+        descs, len(layers), _ptr(page_table), _ptr(seq_lens), B, H_q, d_qk, d_v, page_size,
+        max_pages, n_pages, n_sink, n_local, float(scale), _ptr(workspace), workspace.numel(),
+        _stream(stream)))
+    return outs
 
 
 def loza_ssa_decode_static_scratch(q, paged_kv, page_table, seq_lens, d_v=512, o=None, lse=None,

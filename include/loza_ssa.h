@@ -236,6 +236,44 @@ int loza_ssa_decode_mtp(const void* q, const void* paged_kv, const int* page_tab
 size_t loza_ssa_decode_mtp_workspace_size(int B, int q_len, int H_q, int d_v, int n_sink,
                                           int n_local);
 
+/*
+ * One attention layer of a LoZA decode step (the ZigZag layer stack of the
+ * QbitAI LoZA article: half of LongCat-Flash's MLA layers keep full attention,
+ * half become SSA).  All layers share one page table and one seq_lens array;
+ * each has its own query, cache pool and outputs.
+ */
+typedef struct loza_ssa_decode_layer {
+  const void* q;        /* bf16 [B, H_q, d_qk]                              */
+  const void* paged_kv; /* bf16 [n_pages, page_size, d_qk]: this layer's pool */
+  void* o;              /* bf16 [B, H_q, d_v]                               */
+  float* lse;           /* fp32 [B, H_q]                                    */
+  int full_attention;   /* nonzero: every key up to the query (an MLA layer);
+                           0: the SSA window n_sink + n_local                */
+} loza_ssa_decode_layer;
+
+/*
+ * Decode step over a stack of layers, in order, on one stream: each layer is
+ * loza_ssa_decode with its own window -- {n_sink, n_local} for SSA layers,
+ * all pages 0 .. page(t) for full-attention layers (computed as a window of
+ * max_pages local pages, so max_pages <= 4096, i.e. contexts up to 512K
+ * tokens, when any layer is full).
+ *   layers   : HOST array of n_layers descriptors (read during the call only).
+ *   workspace: at least loza_ssa_decode_layers_workspace_size(...) bytes; the
+ *              layers run one after another and reuse it.
+ * Other arguments as for loza_ssa_decode.  Returns the first failing layer's
+ * status; the layers before it have been launched.
+ */
+int loza_ssa_decode_layers(const loza_ssa_decode_layer* layers, int n_layers,
+                           const int* page_table, const int* seq_lens, int B, int H_q, int d_qk,
+                           int d_v, int page_size, int max_pages, int n_pages, int n_sink,
+                           int n_local, float scale, void* workspace, size_t workspace_bytes,
+                           loza_ssa_stream_t stream);
+
+/* Bytes of workspace loza_ssa_decode_layers needs for a stack that holds at
+ * least one full-attention layer (any_full != 0) or only SSA layers. */
+size_t loza_ssa_decode_layers_workspace_size(int B, int H_q, int d_v, int max_pages, int n_sink,
+                                             int n_local, int any_full);
+
 /* Static description of a status code (never NULL). */
 const char* loza_ssa_status_string(int status);
 

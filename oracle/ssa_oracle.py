@@ -450,6 +450,58 @@ def brute_force_decode_selected(q, kv, page_table, seq_lens, extra_pages, dv, pa
     return o, lse
 
 
+def decode_full(q, kv, page_table, seq_lens, dv, page_size=128, scale=None, rows=None):
+    """Full-attention decode (the MLA layers that LoZA keeps, "LoZA：ZigZag稀疏注意力机制"
+    §2.1, first formula, for the newest query token): softmax over every key
+    0 .. seq_len-1 of the sequence, gathered through the page table, float64.
+    q: [B,Hq,dqk]; kv: [n_pages,page_size,dqk]; the value is the first dv
+    entries of the key row.  ``rows``: optional flat indices b*Hq + h.
+    Returns (o, lse) shaped like decode()."""
+    q, kv = _as_f64(q), _as_f64(kv)
+    B, Hq, dqk = q.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(dqk)
+    full = rows is None
+    rows = np.arange(B * Hq, dtype=np.int64) if full else np.asarray(rows, dtype=np.int64)
+    o = np.empty((rows.size, dv))
+    lse = np.empty(rows.size)
+    flat_kv = kv.reshape(-1, dqk)
+    for b in np.unique(rows // Hq):
+        sel = np.nonzero(rows // Hq == b)[0]
+        heads = rows[sel] % Hq
+        n = int(seq_lens[b])
+        logical = np.arange(n)
+        phys = np.asarray(page_table[b])[logical // page_size].astype(np.int64) * page_size \
+            + logical % page_size
+        keys = flat_kv[phys]                                  # [n, dqk]
+        s = scale * q[b, heads] @ keys.T                      # [heads, n]
+        smax = s.max(axis=-1, keepdims=True)
+        p = np.exp(s - smax)
+        den = p.sum(axis=-1, keepdims=True)
+        o[sel] = p @ keys[:, :dv] / den
+        lse[sel] = smax[:, 0] + np.log(den[:, 0])
+    if full:
+        return o.reshape(B, Hq, dv), lse.reshape(B, Hq)
+    return o, lse
+
+
+def decode_layers(layers, page_table, seq_lens, dv, page_size=128, n_sink=1, n_local=7,
+                  scale=None, rows=None):
+    """One decode step through a stack of attention layers (the ZigZag layout
+    of the QbitAI LoZA article: some layers keep full MLA attention, the others
+    are SSA).  ``layers``: sequence of (q, kv, full_attention) sharing one page
+    table and seq_lens; each layer is decode_full() or decode() on its own
+    inputs.  Returns a list of (o, lse), one per layer."""
+    out = []
+    for q, kv, is_full in layers:
+        if is_full:
+            out.append(decode_full(q, kv, page_table, seq_lens, dv, page_size, scale, rows))
+        else:
+            out.append(decode(q, kv, page_table, seq_lens, dv, page_size, n_sink, n_local, scale,
+                              rows))
+    return out
+
+
 def causal_attention(q, k, v, scale=None):
     """Textbook causal softmax attention in float64 (keys j <= i)."""
     q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)

@@ -221,6 +221,36 @@ def test_decode_argument_errors(L):
     assert _decode(L, ws=0x10010) == -6
 
 
+def test_decode_layers_workspace_size(L):
+    from block_sparse_streaming_ssa_b200 import loza_ssa as api
+    # SSA layers only: the SSA decode's workspace; with a full-attention layer,
+    # the larger of that and a window of all max_pages pages
+    assert api.loza_ssa_decode_layers_workspace_size(32, 128, 512, 1024, 1, 7, False) == \
+        api.loza_ssa_decode_workspace_size(32, 128, 512, 1, 7)
+    assert api.loza_ssa_decode_layers_workspace_size(32, 128, 512, 1024, 1, 7, True) == \
+        api.loza_ssa_decode_workspace_size(32, 128, 512, 0, 1024)
+    assert api.loza_ssa_decode_layers_workspace_size(32, 128, 512, 3, 1, 7, True) == \
+        api.loza_ssa_decode_workspace_size(32, 128, 512, 1, 7)
+    assert api.loza_ssa_decode_layers_workspace_size(32, 128, 512, 4097, 1, 7, True) == 0
+
+
+def test_decode_layers_argument_errors(L):
+    from block_sparse_streaming_ssa_b200.loza_ssa import LozaSsaDecodeLayer
+    vp = ctypes.c_void_p
+
+    def call(layers, n, max_pages=16):
+        arr = (LozaSsaDecodeLayer * max(len(layers), 1))(*layers) if layers else None
+        return L.loza_ssa_decode_layers(arr, n, vp(0x1000), vp(0x1000), 2, 128, 576, 512, 128,
+                                        max_pages, 32, 1, 7, ctypes.c_float(0.04), vp(0x10000),
+                                        1 << 30, None)
+
+    ok = LozaSsaDecodeLayer(0x1000, 0x1000, 0x1000, 0x1000, 1)
+    assert call([], 1) == -1                                              # no layer array
+    assert call([ok], 0) == -2                                            # empty stack
+    assert call([LozaSsaDecodeLayer(0, 0x1000, 0x1000, 0x1000, 0)], 1) == -1   # layer 0: no q
+    assert call([ok], 1, max_pages=5000) == -5      # full attention over more than 4096 pages
+
+
 def test_varlen_argument_errors(L):
     vp = ctypes.c_void_p
     f = ctypes.c_float(0.1)

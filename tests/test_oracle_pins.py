@@ -377,6 +377,88 @@ def test_decode_selected_without_pages_is_decode():
     np.testing.assert_array_equal(a[1], b[1])
 
 
+# --- full-attention decode (the MLA layers LoZA keeps) and the layer stack
+
+
+def test_decode_full_is_causal_attention_last_row():
+    """Every key 0..t through the page table: the last row of textbook causal
+    attention over the sequence's logical key rows."""
+    lens = [1, 9, 77, 130]
+    q, kv, pt, sl = _decode_case(21, lens, Hq=3)
+    o, lse = orc.decode_full(q, kv, pt, sl, dv=16, page_size=8, scale=0.25)
+    for b, n in enumerate(lens):
+        logical = np.arange(n)
+        rows = kv.reshape(-1, kv.shape[-1])[pt[b][logical // 8] * 8 + logical % 8]
+        for h in range(3):
+            qq = np.zeros((n, rows.shape[1]))
+            qq[n - 1] = q[b, h]
+            ref_o, ref_lse = orc.causal_attention(qq, rows, rows[:, :16], scale=0.25)
+            np.testing.assert_allclose(o[b, h], ref_o[-1], atol=1e-12)
+            np.testing.assert_allclose(lse[b, h], ref_lse[-1], atol=1e-12)
+
+
+def test_decode_full_equals_ssa_decode_when_window_covers_prefix():
+    """A sequence no longer than the window (n_sink + n_local pages): the SSA
+    decode (C oracle) and the full decode (numpy) see the same keys."""
+    lens = [8, 31, 32, 5]
+    q, kv, pt, sl = _decode_case(22, lens)
+    a = orc.decode_full(q, kv, pt, sl, dv=16, page_size=8, scale=0.3)
+    b = orc.decode(q, kv, pt, sl, dv=16, page_size=8, n_sink=1, n_local=3, scale=0.3)
+    np.testing.assert_allclose(a[0], b[0], atol=1e-12)
+    np.testing.assert_allclose(a[1], b[1], atol=1e-12)
+
+
+def test_decode_full_differs_from_ssa_beyond_window():
+    q, kv, pt, sl = _decode_case(23, [100])
+    a = orc.decode_full(q, kv, pt, sl, dv=16, page_size=8)
+    b = orc.decode(q, kv, pt, sl, dv=16, page_size=8, n_sink=1, n_local=3)
+    assert np.abs(a[1] - b[1]).max() > 1e-3
+
+
+def test_decode_full_key_count_and_mean():
+    """q = 0: uniform weights over all seq_len keys, so LSE = ln(seq_len) and O
+    is the mean of the value rows."""
+    lens = [3, 57, 64]
+    q, kv, pt, sl = _decode_case(24, lens)
+    q[:] = 0.0
+    o, lse = orc.decode_full(q, kv, pt, sl, dv=16, page_size=8)
+    for b, n in enumerate(lens):
+        np.testing.assert_allclose(lse[b], np.log(n), atol=1e-13)
+        logical = np.arange(n)
+        rows = kv.reshape(-1, kv.shape[-1])[pt[b][logical // 8] * 8 + logical % 8]
+        for h in range(o.shape[1]):
+            np.testing.assert_allclose(o[b, h], rows[:, :16].mean(axis=0), atol=1e-12)
+
+
+def test_decode_full_row_subset_and_permutation():
+    lens = [40, 77]
+    q, kv_a, pt_a, sl = _decode_case(25, lens, permute=False)
+    rng = np.random.default_rng(5)
+    perm = rng.permutation(kv_a.shape[0])
+    kv_b = np.empty_like(kv_a)
+    kv_b[perm] = kv_a
+    pt_b = np.where(pt_a >= 0, perm[np.maximum(pt_a, 0)], -1).astype(np.int32)
+    o_a, l_a = orc.decode_full(q, kv_a, pt_a, sl, dv=16, page_size=8)
+    rows = np.array([7, 0, 5, 2])
+    o_b, l_b = orc.decode_full(q, kv_b, pt_b, sl, dv=16, page_size=8, rows=rows)
+    np.testing.assert_allclose(o_b, o_a.reshape(-1, 16)[rows], atol=1e-13)
+    np.testing.assert_allclose(l_b, l_a.reshape(-1)[rows], atol=1e-13)
+
+
+def test_decode_layers_dispatches_per_layer():
+    lens = [100, 20]
+    q0, kv0, pt, sl = _decode_case(26, lens)
+    q1, kv1, _, _ = _decode_case(27, lens)
+    out = orc.decode_layers([(q0, kv0, True), (q1, kv1, False), (q1, kv0, True)], pt, sl, 16,
+                            page_size=8, n_sink=1, n_local=3, scale=0.3)
+    ref = [orc.brute_force_decode(q0, kv0, pt, sl, 16, 8, n_sink=0, n_local=64, scale=0.3),
+           orc.brute_force_decode(q1, kv1, pt, sl, 16, 8, n_sink=1, n_local=3, scale=0.3),
+           orc.brute_force_decode(q1, kv0, pt, sl, 16, 8, n_sink=0, n_local=64, scale=0.3)]
+    for (o, lse), (o_r, l_r) in zip(out, ref):
+        np.testing.assert_allclose(o, o_r, atol=1e-11)
+        np.testing.assert_allclose(lse, l_r, atol=1e-11)
+
+
 # --- decode with several query tokens per sequence (speculative / multi-token
 # steps): token k of sequence b is the query at position seq_len - q_len + k
 
