@@ -16,7 +16,8 @@ window under ``decode_selected`` (``--decode-extra``), and the decode with 2
 query tokens per sequence under ``decode_mtp`` (``--decode-mtp``).  The
 prefill's backward pass on the same workload is timed under ``backward``, and
 full-attention against SSA decode layers at 128K tokens of context under
-``decode_context`` (``--decode-context``).
+``decode_context`` (``--decode-context``), and a full-attention against an SSA
+prefill layer at 128K tokens under ``prefill_context`` (``--prefill-context``).
 
 Under torchrun every rank runs its own replica of the workload (weak scaling,
 no collective on the data path; NCCL only reduces the timing).
@@ -477,6 +478,60 @@ def decode_bench(iters, warmup, peaks, seed=0, len_hi=None, n_sets=8, world=1, n
     }
 
 
+def prefill_context_bench(peaks, L=131072, world=1, seed=0):
+    """Prefill of one layer at a long context: full causal attention (a kept
+    MLA layer of the ZigZag stack: no sink, a window of every block) against
+    SSA, on the MLA-dims workload shape (B=1, H=64, d_qk=192, d_v=128) at L
+    tokens.  One warm-up and two timed calls of the full layer (each is a long
+    call, so it runs under the power cap); five of the SSA layer."""
+    import dataclasses
+    import torch
+    from block_sparse_streaming_ssa_b200 import synth
+    from block_sparse_streaming_ssa_b200.loza_ssa import loza_ssa_prefill
+    sp = dataclasses.replace(synth.MLA, L=L)
+    q, k, v = synth.prefill_spec_inputs(sp, seed=seed, device="cuda")
+    nb = (L + 127) // 128
+    o = torch.empty((sp.B, sp.H, L, sp.d_v), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((sp.B, sp.H, L), dtype=torch.float32, device="cuda")
+
+    def timed(n_sink, n_local, warmup, iters):
+        for _ in range(warmup):
+            loza_ssa_prefill(q, k, v, o=o, lse=lse, n_sink=n_sink, n_local=n_local,
+                             scale=sp.scale)
+        ev = []
+        for _ in range(iters):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            loza_ssa_prefill(q, k, v, o=o, lse=lse, n_sink=n_sink, n_local=n_local,
+                             scale=sp.scale)
+            b.record()
+            ev.append((a, b))
+        torch.cuda.synchronize()
+        return max_over_ranks(statistics.median([a.elapsed_time(b) for a, b in ev]))
+
+    ssa_ms = timed(1, 7, 3, 5)
+    full_ms = timed(0, nb, 1, 2)
+    full_flops = 2 * (sp.d_qk + sp.d_v) * sp.B * sp.H * (L * (L + 1) // 2)
+    ssa_flops = 2 * (sp.d_qk + sp.d_v) * sp.B * sp.H * window_pairs(L)
+    full_tf = full_flops / (full_ms * 1e-3) / 1e12
+    del q, k, v, o, lse
+    torch.cuda.empty_cache()
+    return {
+        "workload": f"prefill at {L} tokens: B={sp.B} H={sp.H} d_qk={sp.d_qk} d_v={sp.d_v} bf16; "
+                    f"full causal layer (window of all {nb} blocks) vs SSA layer (1 sink + 7 local)",
+        "full_layer_ms": round(full_ms, 3), "ssa_layer_ms": round(ssa_ms, 4),
+        "layer_speedup": round(full_ms / ssa_ms, 1),
+        "zigzag_pair_speedup": round(2 * full_ms / (full_ms + ssa_ms), 2),
+        "full_layer_tflops": round(full_tf, 1),
+        "ssa_layer_tflops": round(ssa_flops / (ssa_ms * 1e-3) / 1e12, 1),
+        "full_layer_roofline": {"bound": "tensor", "achieved": round(full_tf, 1),
+                                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                                "frac": round(full_tf / peaks["bf16_tflops_sustained"], 4),
+                                "peak_source": peaks["source"] + " (sustained bf16 GEMM)"},
+        "gpu_launches": 8 + 3,
+    }
+
+
 def context_bench(peaks, context=131072, iters=5, warmup=3, world=1, seed=0):
     """Decode at one long context through the layer-stack call: a full-attention
     (MLA) layer against an SSA layer, and a 4-layer ZigZag stack (full, SSA,
@@ -609,6 +664,9 @@ def main():
     ap.add_argument("--decode-context", type=int, default=131072,
                     help="also time full-attention vs SSA decode layers at this context "
                          "(0: skip it)")
+    ap.add_argument("--prefill-context", type=int, default=131072,
+                    help="also time a full-attention vs an SSA prefill layer at this length "
+                         "(0: skip it)")
     ap.add_argument("--cpu-budget-s", type=float, default=10.0)
     ap.add_argument("--ref-budget-s", type=float, default=60.0,
                     help="--impl reference: CPU seconds over all warm-up and timed steps")
@@ -690,10 +748,12 @@ def main():
     backward = None if args.no_backward else backward_bench(w, max(3, args.steps // 5),
                                                               args.warmup, peaks, world)
     w_desc, w_tokens = w["desc"], w["tokens"]
-    decode = selected = mtp = ctx = None
+    decode = selected = mtp = ctx = pctx = None
+    del w
+    torch.cuda.empty_cache()
+    if args.prefill_context:
+        pctx = prefill_context_bench(peaks, args.prefill_context, world=world, seed=rank)
     if not args.no_decode:
-        del w
-        torch.cuda.empty_cache()
         decode = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
                               len_hi=args.decode_len_hi, world=world)
         if args.decode_extra:
@@ -751,6 +811,7 @@ def main():
         "decode_selected": selected,
         "decode_mtp": mtp,
         "decode_context": ctx,
+        "prefill_context": pctx,
     }
     print(json.dumps(line), flush=True)
     if dist:

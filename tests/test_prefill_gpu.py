@@ -65,6 +65,32 @@ def test_short_sequences_equal_causal():
     assert_parity(o, lse, o_c, lse_c, "causal")
 
 
+@pytest.mark.parametrize("L,dqk,dv,n_local", [(3000, 128, 128, 24), (5000, 192, 128, 40),
+                                               (2049, 64, 64, 100000)])
+def test_full_attention_layer_is_causal(L, dqk, dv, n_local):
+    """A full-attention layer of the ZigZag stack: no sink and a window of at
+    least every block (n_local >= ceil(L/128), far more in the last case) is
+    textbook causal attention over the whole prefix."""
+    q, k, v = synth.prefill_inputs(1, 2, L, dqk, dv, seed=L, device="cuda")
+    o, lse = loza_ssa_prefill(q, k, v, n_sink=0, n_local=n_local, scale=1 / math.sqrt(dqk))
+    torch.cuda.synchronize()
+    assert loza_ssa_get_last_device_status() == 0
+    o_c, lse_c = orc.causal_attention(*(synth.bf16_bits(t) for t in (q, k, v)),
+                                      scale=1 / math.sqrt(dqk))
+    assert_parity(o, lse, o_c, lse_c, f"full attention L={L} d={dqk}/{dv}")
+
+
+def test_full_attention_layer_long_sampled():
+    """Full attention at L = 32768 (256 key tiles for the last query block),
+    sampled rows against the C oracle with the same all-covering window."""
+    rng = np.random.default_rng(4)
+    rows = np.sort(np.concatenate([rng.choice(2 * 32768, 600, replace=False),
+                                   [0, 32767, 32768, 65535]]))
+    o, lse, o_ref, lse_ref = run_case(1, 2, 32768, 128, 128, n_sink=0, n_local=256, seed=9,
+                                      std=0.5, rows=rows)
+    assert_parity(o, lse, o_ref, lse_ref, "full attention L=32768 sampled")
+
+
 def test_strong_sink_and_large_scores():
     """Keys with a +2 mean on one channel in the first two blocks, and a large
     scale, push the running max around (exercises the O rescale path)."""
