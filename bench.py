@@ -13,7 +13,8 @@ paged decode workload (32 sequences, 128 heads, 576/512, random page table over
 a ~20 GB pool) and reports it under ``decode`` in GB/s of algorithmic bytes,
 and the same decode with 8 distinct selected pages per sequence on top of the
 window under ``decode_selected`` (``--decode-extra``), and the decode with 2
-query tokens per sequence under ``decode_mtp`` (``--decode-mtp``).  The
+query tokens per sequence under ``decode_mtp`` (``--decode-mtp``), and the decode
+over an FP8 cache under ``decode_fp8`` (``--decode-fp8``).  The
 prefill's backward pass on the same workload is timed under ``backward``, and
 full-attention against SSA decode layers at 128K tokens of context under
 ``decode_context`` (``--decode-context``), and a full-attention against an SSA
@@ -359,7 +360,7 @@ def union_window_keys(n: int, q_len: int, blk=128, n_sink=1, n_local=7) -> int:
 
 
 def decode_bench(iters, warmup, peaks, seed=0, len_hi=None, n_sets=8, world=1, n_extra=0,
-                 q_len=1):
+                 q_len=1, fp8=False):
     """Paged decode through the public call.  ``value``: algorithmic bytes per
     call / device time per call, with the calls captured in a CUDA graph (the
     way a serving loop issues decode steps) and rotating over ``n_sets``
@@ -369,19 +370,27 @@ def decode_bench(iters, warmup, peaks, seed=0, len_hi=None, n_sets=8, world=1, n
     also attending ``n_extra`` distinct pages chosen between its sink and its
     local run.  ``q_len`` > 1: several query tokens per sequence (the
     multi-token decode); the bytes count the union of the tokens' key sets
-    once, the FLOPs every token's own set.  ``eager_flush_us``: one eager call per step after a 2x L2
+    once, the FLOPs every token's own set.  ``fp8``: the same workload over an
+    FP8 cache (e4m3 codes + one fp32 scale per token, 580 bytes per key).  ``eager_flush_us``: one eager call per step after a 2x L2
     write, for comparison (it also pays the write-back of the flushed lines
     and, when the GPU runs dry, the host-side cost of the call)."""
     import torch
     from block_sparse_streaming_ssa_b200 import synth
-    from block_sparse_streaming_ssa_b200.loza_ssa import (loza_ssa_decode, loza_ssa_decode_mtp,
+    from block_sparse_streaming_ssa_b200.loza_ssa import (loza_ssa_decode, loza_ssa_decode_fp8,
+                                                          loza_ssa_decode_mtp,
                                                           loza_ssa_decode_mtp_workspace_size,
                                                           loza_ssa_decode_selected,
                                                           loza_ssa_decode_selected_workspace_size)
     s = synth.DECODE
     lens = synth.decode_seq_lens(seed, s.B, s.len_lo, len_hi or s.len_hi)
-    q, kv, pt, sl = synth.decode_inputs(lens, s.H_q, s.d_qk, seed=seed, device="cuda",
-                                        q_len=q_len if q_len > 1 else None)
+    ksc = None
+    if fp8:
+        q, kv, ksc, pt, sl = synth.decode_inputs_fp8(lens, s.H_q, s.d_qk, seed=seed,
+                                                     device="cuda")
+    else:
+        q, kv, pt, sl = synth.decode_inputs(lens, s.H_q, s.d_qk, seed=seed, device="cuda",
+                                            q_len=q_len if q_len > 1 else None)
+    key_bytes = s.d_qk + 4 if fp8 else s.d_qk * 2
     ex_h, extra_keys = decode_extra_pages(lens, n_extra, seed)
     extra = torch.as_tensor(ex_h, device="cuda")
     ws_bytes = (loza_ssa_decode_mtp_workspace_size(s.B, q_len, s.H_q, s.d_v, 1, 7) if q_len > 1
@@ -389,6 +398,9 @@ def decode_bench(iters, warmup, peaks, seed=0, len_hi=None, n_sets=8, world=1, n
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
 
     def decode(qq, pp, **kw):
+        if fp8:
+            return loza_ssa_decode_fp8(qq, kv, ksc, pp, sl, s.d_v, scale=s.scale, workspace=ws,
+                                       **kw)
         if q_len > 1:
             return loza_ssa_decode_mtp(qq, kv, pp, sl, s.d_v, scale=s.scale, workspace=ws, **kw)
         if n_extra:
@@ -400,7 +412,7 @@ def decode_bench(iters, warmup, peaks, seed=0, len_hi=None, n_sets=8, world=1, n
     keys = int(sum(row_pairs(np.arange(n - q_len, n)).sum() for n in lens)) + extra_keys
     read_keys = (int(sum(union_window_keys(n, q_len) for n in lens)) + extra_keys if q_len > 1
                  else keys)
-    algo_bytes = read_keys * s.d_qk * 2 + q.numel() * 2 + o.numel() * 2 + lse.numel() * 4
+    algo_bytes = read_keys * key_bytes + q.numel() * 2 + o.numel() * 2 + lse.numel() * 4
     flops = 2 * (s.d_qk + s.d_v) * keys * s.H_q
 
     gen = torch.Generator(device="cpu").manual_seed(1000 + seed)
@@ -409,7 +421,7 @@ def decode_bench(iters, warmup, peaks, seed=0, len_hi=None, n_sets=8, world=1, n
         perm = torch.randperm(kv.shape[0], generator=gen).to(torch.int32).cuda()
         sets.append((torch.randn(q.shape, generator=gen).to(torch.bfloat16).cuda(),
                      torch.where(pt >= 0, perm[pt.clamp(min=0).long()], pt)))
-    distinct_kv = n_sets * keys * s.d_qk * 2
+    distinct_kv = n_sets * keys * key_bytes
 
     def call(i):
         qq, pp = sets[i % n_sets]
@@ -459,7 +471,8 @@ def decode_bench(iters, warmup, peaks, seed=0, len_hi=None, n_sets=8, world=1, n
                     f"seq_len U[{s.len_lo},{len_hi or s.len_hi}] seed {seed}, random page permutation "
                     f"over {kv.shape[0]} pages"
                     + (f", plus {n_extra} distinct selected pages per sequence" if n_extra else "")
-                    + (f", {q_len} query tokens per sequence" if q_len > 1 else ""),
+                    + (f", {q_len} query tokens per sequence" if q_len > 1 else "")
+                    + (", FP8 e4m3 cache with one fp32 scale per token" if fp8 else ""),
         "value": round(gbs, 1), "unit": "GB/s", "us_per_step": round(ms * 1e3, 2),
         "algorithmic_bytes_per_step": algo_bytes, "useful_gflop_per_step": round(flops / 1e9, 3),
         "tflops": round(flops / (ms * 1e-3) / 1e12, 1),
@@ -470,6 +483,7 @@ def decode_bench(iters, warmup, peaks, seed=0, len_hi=None, n_sets=8, world=1, n
         "roofline": {"bound": "hbm", "achieved": round(gbs / world, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(gbs / world / peaks["hbm_gbs"], 4),
                      "traffic": traffic_lookup("ssa_decode_split_kernel",
+                                               "decode_fp8" if fp8 else
                                                "decode_selected" if n_extra else
                                                f"decode_mtp{q_len}" if q_len > 1 else "decode"),
                      "peak_source": peaks["source"],
@@ -661,6 +675,8 @@ def main():
     ap.add_argument("--decode-mtp", type=int, default=2,
                     help="also time the decode with this many query tokens per sequence "
                          "(<= 1: skip it)")
+    ap.add_argument("--decode-fp8", type=int, default=1,
+                    help="also time the decode over an FP8 cache (0: skip it)")
     ap.add_argument("--decode-context", type=int, default=131072,
                     help="also time full-attention vs SSA decode layers at this context "
                          "(0: skip it)")
@@ -725,11 +741,15 @@ def main():
         if args.decode_mtp > 1:
             mtp = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
                                len_hi=args.decode_len_hi, world=world, q_len=args.decode_mtp)
+        dfp8 = (decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
+                             len_hi=args.decode_len_hi, world=world, fp8=True)
+                if args.decode_fp8 else None)
         ctx = (context_bench(peaks, args.decode_context, world=world, seed=rank)
                if args.decode_context else None)
         if rank == 0:
             print(json.dumps({"metric": METRIC, "decode": decode, "decode_selected": selected,
-                              "decode_mtp": mtp, "decode_context": ctx}), flush=True)
+                              "decode_mtp": mtp, "decode_fp8": dfp8, "decode_context": ctx}),
+                  flush=True)
         if dist:
             torch.distributed.destroy_process_group()
         return
@@ -748,7 +768,7 @@ def main():
     backward = None if args.no_backward else backward_bench(w, max(3, args.steps // 5),
                                                               args.warmup, peaks, world)
     w_desc, w_tokens = w["desc"], w["tokens"]
-    decode = selected = mtp = ctx = pctx = None
+    decode = selected = mtp = ctx = pctx = dfp8 = None
     del w
     torch.cuda.empty_cache()
     if args.prefill_context:
@@ -763,6 +783,9 @@ def main():
         if args.decode_mtp > 1:
             mtp = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
                                len_hi=args.decode_len_hi, world=world, q_len=args.decode_mtp)
+        if args.decode_fp8:
+            dfp8 = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
+                                len_hi=args.decode_len_hi, world=world, fp8=True)
         if args.decode_context:
             ctx = context_bench(peaks, args.decode_context, world=world, seed=rank)
 
@@ -810,6 +833,7 @@ def main():
         "decode": decode,
         "decode_selected": selected,
         "decode_mtp": mtp,
+        "decode_fp8": dfp8,
         "decode_context": ctx,
         "prefill_context": pctx,
     }

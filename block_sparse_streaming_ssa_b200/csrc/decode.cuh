@@ -29,6 +29,15 @@
 //           [CTA][64 groups of 8 columns][128 heads][8] (a warp's stores of
 //           a group are 512 contiguous bytes); the LSE as fp32
 //
+// FP8 cache (template argument FP8): each latent row is 576 e4m3 codes with
+// one fp32 scale per token, K_j = s_j k8_j.  The TMA puts a page's 64-channel
+// e4m3 box (8 KB) in the upper half of its 16 KB bf16 slot; the softmax
+// warpgroups, idle while S is built, expand it in place to the bf16 swizzled
+// box the MMA reads (e4m3 values are exact in bf16) and arrive on a second
+// barrier the MMA waits for.  The scale stays out of the products: S column j
+// is multiplied by s_j before the softmax, and P_ij s_j is what goes to TMEM
+// for the P V product, so O = sum_j p_ij s_j v8_j / l with l = sum_j p_ij.
+//
 // Merge kernel (programmatic dependent launch after the split kernel):
 // LSE = logsumexp_s LSE_s, O = sum_s exp(LSE_s - LSE) O_s.
 #pragma once
@@ -68,6 +77,8 @@ struct DecodeParams {
   int max_extra;
   int wave;     // CTAs resident at once: the CTA `wave` later runs on a freed SM
   float scale_log2;
+  // FP8 cache only: fp32 scale of every token, [n_pages, 128] by physical page.
+  const float* kv_scale;
 };
 
 __device__ __forceinline__ int decode_seq(const DecodeParams& p, int row) {
@@ -151,9 +162,18 @@ struct DecodeLayout {
   static constexpr int B_O_FULL = B_XCHG + 1;     // phase 0: O half 1, phase 1: O half 0
   static constexpr int B_O_EMPTY = B_O_FULL + 1;  // 256 arrivals, one phase per half
   static constexpr int B_DRAIN = B_O_EMPTY + 1;
-  static constexpr int NBAR = B_DRAIN + 1;
+  // FP8 cache: a stage's K boxes expanded to bf16, the V_A and the V_B boxes
+  // expanded
+  static constexpr int B_CONV = B_DRAIN + 1;  // NST
+  static constexpr int B_VA_CONV = B_CONV + NST;  // 256 arrivals: both warpgroups convert
+  static constexpr int B_VB_CONV = B_VA_CONV + 1;  // 256 arrivals
+  static constexpr int B_XP = B_VB_CONV + 1;  // 2, 128 arrivals: a warpgroup read its e4m3 box
+  static constexpr int NBAR = B_XP + 2;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  // FP8 cache: float [2 pages][128 tokens] of s_j * scale * log2(e), then of s_j
+  static constexpr int OFF_SCALE = OFF_MISC + 16;
+  static constexpr int SMEM_BYTES = OFF_SCALE + 2 * 2 * 128 * 4 + 1024;
+  static constexpr int CHUNK8 = CHUNK / 2;  // one e4m3 box: 128 rows x 64 bytes
   static constexpr int TMEM_COLS = 512;  // S [0,256) (P inside it), O half [256,512)
   static constexpr int TM_O = 256;
 };
@@ -175,6 +195,50 @@ __device__ __forceinline__ uint32_t decode_chunk_mask(int valid_keys, int ch) {
   return n >= 32 ? 0xffffffffu : (n <= 0 ? 0u : (1u << n) - 1u);
 }
 
+// Two e4m3 codes (bytes `sel` of w, picked by a byte permute) to a bf16x2
+// word, exactly: the code's magnitude bits placed at bf16 bits 4..10 read as
+// exponent e and mantissa m, i.e. 2^(e-127) (1 + m/8) (a bf16 subnormal m/8
+// 2^-126 when e = 0); one multiply by 2^120 (no rounding, subnormal inputs
+// supported) gives the e4m3 value 2^(e-7) (1 + m/8), or m/8 2^-6, and the
+// sign bit moves from bit 7 to bit 15.
+template <uint32_t SEL>
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t w) {
+  uint32_t y, r;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(y) : "r"(w), "n"(SEL));  // code bytes -> bytes 0, 2
+  const uint32_t bits = ((y << 4) & 0x07F007F0u) | ((y << 8) & 0x80008000u);
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(bits), "r"(0x7B807B80u));  // x 2^120
+  return r;
+}
+
+// FP8 cache: expand one e4m3 box (128 rows x 64 channels; row r at byte 64 r
+// of the slot's upper half, as the TMA wrote it) in place into the bf16
+// 128-byte-swizzled box the MMA reads (row r at byte 128 r, 16-byte chunk c
+// at chunk c ^ (r & 7)).  Thread `row` of a warpgroup takes one row.  The
+// bf16 rows 64.. overlap the e4m3 rows, so every row is read before any is
+// written: the warpgroup's threads arrive on `xp` (128 arrivals) once they
+// have read, and write only after the phase completes.  The wait is bounded,
+// so a thread that left early (its own wait failed) ends the others' wait
+// with the abort flag rather than holding them.  `uses` counts this
+// thread's uses of `xp` (its phase).
+__device__ __forceinline__ bool decode_expand_fp8_box(uint32_t slot, int row, uint32_t xp,
+                                                      uint32_t& uses, volatile int* abort_flag,
+                                                      int* status) {
+  uint32_t in[16];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) lds_v4(slot + DecodeLayout::CHUNK8 + 64 * row + 16 * j, in + 4 * j);
+  mbar_arrive(xp);
+  const bool ok = mbar_wait(xp, uses & 1, abort_flag, status, 1);
+  ++uses;
+  if (!ok) return false;
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    sts_v4(slot + 128 * row + 16 * (c ^ (row & 7)), e4m3x2_to_bf16x2<0x4140>(in[2 * c]),
+           e4m3x2_to_bf16x2<0x4342>(in[2 * c]), e4m3x2_to_bf16x2<0x4140>(in[2 * c + 1]),
+           e4m3x2_to_bf16x2<0x4342>(in[2 * c + 1]));
+  return true;
+}
+
+template <bool FP8>
 __global__ void __launch_bounds__(320, 1)
     ssa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                             const __grid_constant__ CUtensorMap tm_kv, const DecodeParams p) {
@@ -242,6 +306,13 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(bar(Lay::B_O_FULL), 1);
     mbar_init(bar(Lay::B_O_EMPTY), 256);
     mbar_init(bar(Lay::B_DRAIN), 1);
+    if (FP8) {
+      for (int s = 0; s < Lay::NST; ++s) mbar_init(bar(Lay::B_CONV + s), 256);
+      mbar_init(bar(Lay::B_VA_CONV), 256);
+      mbar_init(bar(Lay::B_VB_CONV), 256);
+      mbar_init(bar(Lay::B_XP), 128);
+      mbar_init(bar(Lay::B_XP + 1), 128);
+    }
     misc[1] = 0;
     fence_barrier_init();
   }
@@ -261,7 +332,10 @@ __global__ void __launch_bounds__(320, 1)
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const uint32_t s_bytes = (two ? 3 : 2) * Lay::CHUNK;
+      // K boxes: bf16 (a whole slot) or e4m3 (the slot's upper half)
+      const uint32_t kbox = FP8 ? Lay::CHUNK8 : Lay::CHUNK;
+      const uint32_t koff = FP8 ? Lay::CHUNK8 : 0;
+      const uint32_t s_bytes = Lay::CHUNK + (two ? 2 : 1) * kbox;
       int issued = 0;        // S stages issued
       bool va = false, vb = false;
       do {
@@ -273,8 +347,8 @@ __global__ void __launch_bounds__(320, 1)
           const uint32_t dst = ring + st * Lay::STAGE, full = bar(Lay::B_FULL + st);
           mbar_arrive_expect_tx(full, s_bytes);
           tma_load_3d(dst, &tm_q, full, c * 64, hg * 128, b);
-          tma_load_2d(dst + Lay::CHUNK, &tm_kv, full, c * 64, phys_a * 128);
-          if (two) tma_load_2d(dst + 2 * Lay::CHUNK, &tm_kv, full, c * 64, phys_b * 128);
+          tma_load_2d(dst + Lay::CHUNK + koff, &tm_kv, full, c * 64, phys_a * 128);
+          if (two) tma_load_2d(dst + 2 * Lay::CHUNK + koff, &tm_kv, full, c * 64, phys_b * 128);
           ++issued;
           if (i == 0) {
             // A CTA one wave later starts only when an SM frees up: pull its
@@ -305,16 +379,17 @@ __global__ void __launch_bounds__(320, 1)
         // once S is done; page B's into the K_B slots, free once O half 1
         // (which reads boxes 4..7 there) is done.  Box e goes to stage e.
         if (!mbar_wait(bar(Lay::B_S_FULL), 0, abort_flag, status, 1)) break;
-        mbar_arrive_expect_tx(bar(Lay::B_VA_FULL), 4 * Lay::CHUNK);
+        mbar_arrive_expect_tx(bar(Lay::B_VA_FULL), 4 * kbox);
         for (int e = 0; e < 4; ++e)
-          tma_load_2d(ring + e * Lay::STAGE, &tm_kv, bar(Lay::B_VA_FULL), e * 64, phys_a * 128);
+          tma_load_2d(ring + e * Lay::STAGE + koff, &tm_kv, bar(Lay::B_VA_FULL), e * 64,
+                      phys_a * 128);
         va = true;
         if (!two) break;
         if (!mbar_wait(bar(Lay::B_O_FULL), 0, abort_flag, status, 1)) break;
-        mbar_arrive_expect_tx(bar(Lay::B_VB_FULL), 4 * Lay::CHUNK);
+        mbar_arrive_expect_tx(bar(Lay::B_VB_FULL), 4 * kbox);
         for (int e = 0; e < 4; ++e)
-          tma_load_2d(ring + e * Lay::STAGE + 2 * Lay::CHUNK, &tm_kv, bar(Lay::B_VB_FULL), e * 64,
-                      phys_b * 128);
+          tma_load_2d(ring + e * Lay::STAGE + 2 * Lay::CHUNK + koff, &tm_kv, bar(Lay::B_VB_FULL),
+                      e * 64, phys_b * 128);
         vb = true;
       } while (false);
       // every copy issued lands before the CTA exits
@@ -337,6 +412,9 @@ __global__ void __launch_bounds__(320, 1)
       for (int i = 0; i < Lay::KV_CH; ++i) {
         const int st = decode_s_stage(i);
         if (!(ok = mbar_wait(bar(Lay::B_FULL + st), decode_s_round(i) & 1, abort_flag, status, 1)))
+          break;
+        if (FP8 && !(ok = mbar_wait(bar(Lay::B_CONV + st), decode_s_round(i) & 1, abort_flag,
+                                    status, 1)))
           break;
         tc_fence_after();
         const uint32_t base = ring + st * Lay::STAGE;
@@ -369,12 +447,14 @@ __global__ void __launch_bounds__(320, 1)
         if (two) pv_page(ring + 2 * Lay::CHUNK, 128, false);
         mma_commit(bar(Lay::B_O_FULL));
         ok = mbar_wait(bar(Lay::B_VA_FULL), 0, abort_flag, status, 1) &&
+             (!FP8 || mbar_wait(bar(Lay::B_VA_CONV), 0, abort_flag, status, 1)) &&
              mbar_wait(bar(Lay::B_O_EMPTY), 0, abort_flag, status, 1);
       }
       if (ok) {  // half 0 (columns 0..255): the reloaded boxes
         tc_fence_after();
         pv_page(ring, 0, true);
-        if (two && (ok = mbar_wait(bar(Lay::B_VB_FULL), 0, abort_flag, status, 1))) {
+        if (two && (ok = mbar_wait(bar(Lay::B_VB_FULL), 0, abort_flag, status, 1) &&
+                         (!FP8 || mbar_wait(bar(Lay::B_VB_CONV), 0, abort_flag, status, 1)))) {
           tc_fence_after();
           pv_page(ring + 2 * Lay::CHUNK, 128, false);
         }
@@ -394,7 +474,35 @@ __global__ void __launch_bounds__(320, 1)
     float* xmax = reinterpret_cast<float*>(smem + Lay::OFF_XCHG);
     float* xsum = xmax + 256;
     const float sl2 = p.scale_log2;
+    // FP8: this page's s_j * scale * log2(e) (ksl) and s_j (ksc)
+    const float* ksl = reinterpret_cast<const float*>(smem + Lay::OFF_SCALE) + wg * 128;
+    const float* ksc = ksl + 256;
+    const uint32_t xp = bar(Lay::B_XP + wg);
+    uint32_t xp_uses = 0;
     do {
+      if constexpr (FP8) {
+        // this page's token scales, then its K boxes as they land
+        const bool mine = wg == 0 || two;
+        if (mine) {
+          const float sj = __ldg(p.kv_scale + (size_t)(wg == 0 ? phys_a : phys_b) * 128 + h);
+          float* st_sc = reinterpret_cast<float*>(smem + Lay::OFF_SCALE) + wg * 128 + h;
+          st_sc[0] = sj * sl2;
+          st_sc[256] = sj;
+        }
+        bool okc = true;
+        for (int i = 0; i < Lay::KV_CH; ++i) {
+          const int st = decode_s_stage(i);
+          if (!(okc = mbar_wait(bar(Lay::B_FULL + st), decode_s_round(i) & 1, abort_flag, status,
+                                1)))
+            break;
+          if (mine && !(okc = decode_expand_fp8_box(ring + st * Lay::STAGE + Lay::CHUNK * (1 + wg),
+                                                    h, xp, xp_uses, abort_flag, status)))
+            break;
+          fence_async_shared();
+          mbar_arrive(bar(Lay::B_CONV + st));
+        }
+        if (!okc) break;
+      }
       if (!mbar_wait(bar(Lay::B_S_FULL), 0, abort_flag, status, 1)) break;
       tc_fence_after();
       // Pass 1: this page's row max, 64 keys at a time.
@@ -414,9 +522,13 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
               for (int a = 0; a < 4; ++a) {
                 const int k0 = c + 2 * a;
-                const float x0 = ((vm >> k0) & 1u) ? __uint_as_float(v[jj][k0]) : -INFINITY;
-                const float x1 =
-                    ((vm >> (k0 + 1)) & 1u) ? __uint_as_float(v[jj][k0 + 1]) : -INFINITY;
+                float s0 = __uint_as_float(v[jj][k0]), s1 = __uint_as_float(v[jj][k0 + 1]);
+                if constexpr (FP8) {  // already in log2 units
+                  s0 *= ksl[64 * hf + 32 * jj + k0];
+                  s1 *= ksl[64 * hf + 32 * jj + k0 + 1];
+                }
+                const float x0 = ((vm >> k0) & 1u) ? s0 : -INFINITY;
+                const float x1 = ((vm >> (k0 + 1)) & 1u) ? s1 : -INFINITY;
                 mx4[a] = fmax3(mx4[a], x0, x1);
               }
           }
@@ -426,7 +538,8 @@ __global__ void __launch_bounds__(320, 1)
       xmax[wg * 128 + h] = mloc;
       mbar_arrive(bar(Lay::B_XCHG));
       if (!mbar_wait(bar(Lay::B_XCHG), 0, abort_flag, status, 1)) break;
-      const float m = fmaxf(mloc, xmax[(wg ^ 1) * 128 + h]) * sl2;  // finite: page A has a key
+      // finite: page A has a key (FP8: the maxima are already in log2 units)
+      const float m = fmaxf(mloc, xmax[(wg ^ 1) * 128 + h]) * (FP8 ? 1.f : sl2);
       const uint64_t sl2x2 = f2_pack(sl2, sl2);
       const uint64_t negm2 = f2_pack(-m, -m);
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
@@ -443,11 +556,22 @@ __global__ void __launch_bounds__(320, 1)
           const uint32_t vm = partial ? decode_chunk_mask(valid_keys, ch) : 0xffffffffu;
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            const float v0 = ((vm >> (2 * c)) & 1u) ? __uint_as_float(v[2 * c]) : -INFINITY;
-            const float v1 =
-                ((vm >> (2 * c + 1)) & 1u) ? __uint_as_float(v[2 * c + 1]) : -INFINITY;
             float y0, y1, p0, p1;
-            f2_unpack(f2_fma(f2_pack(v0, v1), sl2x2, negm2), y0, y1);
+            if constexpr (FP8) {
+              // y = s * (s_j scale log2 e) - m; the mask after the product, so
+              // that a zero s_j never meets -inf
+              const uint64_t kl = *reinterpret_cast<const uint64_t*>(ksl + 32 * ch + 2 * c);
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])),
+                               kl, negm2),
+                        y0, y1);
+              y0 = ((vm >> (2 * c)) & 1u) ? y0 : -INFINITY;
+              y1 = ((vm >> (2 * c + 1)) & 1u) ? y1 : -INFINITY;
+            } else {
+              const float v0 = ((vm >> (2 * c)) & 1u) ? __uint_as_float(v[2 * c]) : -INFINITY;
+              const float v1 =
+                  ((vm >> (2 * c + 1)) & 1u) ? __uint_as_float(v[2 * c + 1]) : -INFINITY;
+              f2_unpack(f2_fma(f2_pack(v0, v1), sl2x2, negm2), y0, y1);
+            }
             if ((c & 7) < kDecodePolyPairsPer8) {
               exp2_poly_x2(y0, y1, p0, p1);
             } else {
@@ -455,7 +579,10 @@ __global__ void __launch_bounds__(320, 1)
               p1 = ex2_approx(y1);
             }
             acc[c & 3] = f2_add(acc[c & 3], f2_pack(p0, p1));
-            pk16[c] = pack_bf16x2(p0, p1);
+            if constexpr (FP8)
+              pk16[c] = pack_bf16x2(p0 * ksc[32 * ch + 2 * c], p1 * ksc[32 * ch + 2 * c + 1]);
+            else
+              pk16[c] = pack_bf16x2(p0, p1);
           }
           tmem_st16(t_row + s_col + ch * 16, pk16);
         }
@@ -473,6 +600,16 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive(bar(Lay::B_XCHG));
       if (!mbar_wait(bar(Lay::B_XCHG), 1, abort_flag, status, 1)) break;
       const float l = lloc + xsum[(wg ^ 1) * 128 + h];
+      if constexpr (FP8) {
+        // page A's V columns 0..255, reloaded into the Q slots, to bf16: boxes
+        // 2wg and 2wg+1 by warpgroup wg (this overlaps the MMAs of O half 1)
+        bool okv = mbar_wait(bar(Lay::B_VA_FULL), 0, abort_flag, status, 1);
+        for (int e = 2 * wg; e < 2 * wg + 2 && okv; ++e)
+          okv = decode_expand_fp8_box(ring + e * Lay::STAGE, h, xp, xp_uses, abort_flag, status);
+        if (!okv) break;
+        fence_async_shared();
+        mbar_arrive(bar(Lay::B_VA_CONV));
+      }
 
       const bool valid = hg * 128 + h < p.H_q;
       const float inv_l = 1.f / l;
@@ -509,6 +646,19 @@ __global__ void __launch_bounds__(320, 1)
               }
               dst[(32 * hf + 16 * wg + 8 * part + g) * 128] = make_uint4(w[0], w[1], w[2], w[3]);
             }
+          }
+        }
+        if constexpr (FP8) {
+          // page B's V columns 0..255, reloaded into the K_B slots once O half
+          // 1 is done, to bf16: boxes 2wg and 2wg+1 by warpgroup wg
+          if (n == 0 && two) {
+            bool okv = mbar_wait(bar(Lay::B_VB_FULL), 0, abort_flag, status, 1);
+            for (int e = 2 * wg; e < 2 * wg + 2 && okv; ++e)
+              okv = decode_expand_fp8_box(ring + e * Lay::STAGE + 2 * Lay::CHUNK, h, xp, xp_uses,
+                                          abort_flag, status);
+            if (!(ok = okv)) break;
+            fence_async_shared();
+            mbar_arrive(bar(Lay::B_VB_CONV));
           }
         }
       }

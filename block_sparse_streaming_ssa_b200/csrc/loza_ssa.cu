@@ -100,6 +100,24 @@ int make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint6
   return LOZA_SSA_OK;
 }
 
+// FP8 latent cache [rows, 576] e4m3: 64-byte boxes of 128 rows, unswizzled
+// (the kernel expands them to the bf16 swizzled layout itself).
+int make_map_kv8(CUtensorMap* map, const void* base, uint64_t rows) {
+  cuuint64_t dims[2] = {(cuuint64_t)loza::kDecodeDqk, rows};
+  cuuint64_t strides[1] = {(cuuint64_t)loza::kDecodeDqk};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return LOZA_SSA_ERR_CUDA;
+  }
+  return LOZA_SSA_OK;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // Dense inputs get their exact work-item count here; packed inputs count
@@ -562,13 +580,14 @@ size_t loza_ssa_decode_mtp_workspace_size(int B, int q_len, int H_q, int d_v, in
 namespace {
 
 // loza_ssa_decode with an optional per-sequence list of extra pages
-// (extra_pages == nullptr and max_extra == 0: the plain window) and q_len
-// query tokens per sequence (q_len == 1: one).  B counts sequences.
+// (extra_pages == nullptr and max_extra == 0: the plain window), q_len
+// query tokens per sequence (q_len == 1: one) and an FP8 cache (kv_scale !=
+// nullptr: paged_kv holds e4m3 codes).  B counts sequences.
 int decode_impl(const void* q, const void* paged_kv, const int* page_table, const int* seq_lens,
                 const int* extra_pages, int max_extra, int q_len, void* o, float* lse, int B,
                 int H_q, int d_qk, int d_v, int page_size, int max_pages, int n_pages, int n_sink,
                 int n_local, float scale, void* workspace, size_t workspace_bytes,
-                loza_ssa_stream_t stream) {
+                loza_ssa_stream_t stream, const float* kv_scale = nullptr) {
   if (!q || !paged_kv || !page_table || !seq_lens || !o || !lse) return LOZA_SSA_ERR_NULL;
   if (max_extra < 0 || q_len < 1) return LOZA_SSA_ERR_SHAPE;
   if (q_len > 1 && max_extra > 0) return LOZA_SSA_ERR_SHAPE;  // no public call combines them
@@ -585,7 +604,7 @@ int decode_impl(const void* q, const void* paged_kv, const int* page_table, cons
   if (n_sink < 0 || n_local < 1 || (long long)n_sink + n_local + max_extra > kMaxDecodeWindow)
     return LOZA_SSA_ERR_WINDOW;
   if (!aligned(q, 16) || !aligned(paged_kv, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
-      !aligned(page_table, 4) || !aligned(seq_lens, 4))
+      !aligned(page_table, 4) || !aligned(seq_lens, 4) || !aligned(kv_scale, 4))
     return LOZA_SSA_ERR_ALIGN;
   const size_t need =
       loza_ssa_decode_selected_workspace_size(B, H_q, d_v, n_sink, n_local, max_extra);
@@ -620,19 +639,22 @@ int decode_impl(const void* q, const void* paged_kv, const int* page_table, cons
   prm.max_extra = max_extra > 0 ? max_extra : 0;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.wave = dev.num_sms;  // one split CTA per SM
+  prm.kv_scale = kv_scale;
 
   CUtensorMap mq, mkv;
   if ((rc = make_map(&mq, q, loza::kDecodeDqk, (uint64_t)H_q, (uint64_t)B, 3)) != LOZA_SSA_OK)
     return rc;
-  if ((rc = make_map(&mkv, paged_kv, loza::kDecodeDqk, (uint64_t)n_pages * 128, 1, 2)) != LOZA_SSA_OK)
-    return rc;
+  rc = kv_scale ? make_map_kv8(&mkv, paged_kv, (uint64_t)n_pages * 128)
+                : make_map(&mkv, paged_kv, loza::kDecodeDqk, (uint64_t)n_pages * 128, 1, 2);
+  if (rc != LOZA_SSA_OK) return rc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaFuncSetAttribute(loza::ssa_decode_split_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+  void (*split)(CUtensorMap, CUtensorMap, loza::DecodeParams) =
+      kv_scale ? loza::ssa_decode_split_kernel<true> : loza::ssa_decode_split_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        loza::DecodeLayout::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
   dim3 grid(n_split, HG, B);
-  loza::ssa_decode_split_kernel<<<grid, 320, loza::DecodeLayout::SMEM_BYTES, s>>>(mq, mkv, prm);
+  split<<<grid, 320, loza::DecodeLayout::SMEM_BYTES, s>>>(mq, mkv, prm);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "decode split launch");
   // the merge is a programmatic dependent of the split kernel: it is scheduled
   // as split CTAs retire and waits (griddepcontrol.wait) for their results
@@ -684,6 +706,17 @@ int loza_ssa_decode_selected(const void* q, const void* paged_kv, const int* pag
   return decode_impl(q, paged_kv, page_table, seq_lens, extra_pages, max_extra, 1, o, lse, B,
                      H_q, d_qk, d_v, page_size, max_pages, n_pages, n_sink, n_local, scale,
                      workspace, workspace_bytes, stream);
+}
+
+int loza_ssa_decode_fp8(const void* q, const void* paged_kv_fp8, const float* kv_scale,
+                        const int* page_table, const int* seq_lens, void* o, float* lse, int B,
+                        int H_q, int d_qk, int d_v, int page_size, int max_pages, int n_pages,
+                        int n_sink, int n_local, float scale, void* workspace,
+                        size_t workspace_bytes, loza_ssa_stream_t stream) {
+  if (!kv_scale) return LOZA_SSA_ERR_NULL;
+  return decode_impl(q, paged_kv_fp8, page_table, seq_lens, nullptr, 0, 1, o, lse, B, H_q, d_qk,
+                     d_v, page_size, max_pages, n_pages, n_sink, n_local, scale, workspace,
+                     workspace_bytes, stream, kv_scale);
 }
 
 size_t loza_ssa_decode_layers_workspace_size(int B, int H_q, int d_v, int max_pages, int n_sink,

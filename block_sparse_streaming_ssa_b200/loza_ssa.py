@@ -70,6 +70,9 @@ def lib() -> ctypes.CDLL:
         L.loza_ssa_decode_mtp.restype = i32
         L.loza_ssa_decode_mtp_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
         L.loza_ssa_decode_mtp_workspace_size.restype = sz
+        L.loza_ssa_decode_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                          i32, i32, i32, i32, f32, vp, sz, vp]
+        L.loza_ssa_decode_fp8.restype = i32
         L.loza_ssa_decode_layers.argtypes = [ctypes.POINTER(LozaSsaDecodeLayer), i32, vp, vp,
                                              i32, i32, i32, i32, i32, i32, i32, i32, i32, f32,
                                              vp, sz, vp]
@@ -294,6 +297,41 @@ def loza_ssa_decode(q, paged_kv, page_table, seq_lens, d_v=512, o=None, lse=None
         _ptr(q), _ptr(paged_kv), _ptr(page_table), _ptr(seq_lens), _ptr(o), _ptr(lse), B, H_q,
         d_qk, d_v, page_size, max_pages, n_pages, n_sink, n_local, float(scale), _ptr(workspace),
         workspace.numel(), _stream(stream)))
+    return o, lse
+
+
+def loza_ssa_decode_fp8(q, paged_kv_fp8, kv_scale, page_table, seq_lens, d_v=512, o=None,
+                        lse=None, page_size=128, n_sink=1, n_local=7, scale=None, workspace=None,
+                        stream=None):
+    """Paged SSA decode over an FP8 cache.  paged_kv_fp8: uint8 [n_pages,page_size,576]
+    e4m3 codes; kv_scale: fp32 [n_pages,page_size] per-token scales (K = scale * code).
+    Other arguments and the result as loza_ssa_decode."""
+    _need(q, torch.bfloat16, "q")
+    _need(paged_kv_fp8, torch.uint8, "paged_kv_fp8")
+    _need(kv_scale, torch.float32, "kv_scale")
+    _need(page_table, torch.int32, "page_table")
+    _need(seq_lens, torch.int32, "seq_lens")
+    B, H_q, d_qk = q.shape
+    n_pages = paged_kv_fp8.shape[0]
+    if tuple(kv_scale.shape) != tuple(paged_kv_fp8.shape[:2]):
+        raise ValueError("kv_scale must be [n_pages, page_size]")
+    max_pages = page_table.shape[1]
+    if o is None:
+        o = torch.empty((B, H_q, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H_q), dtype=torch.float32, device=q.device)
+    _need(o, torch.bfloat16, "o")
+    _need(lse, torch.float32, "lse")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d_qk)
+    need = loza_ssa_decode_workspace_size(B, H_q, d_v, n_sink, n_local)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _need(workspace, torch.uint8, "workspace")
+    _check(lib().loza_ssa_decode_fp8(
+        _ptr(q), _ptr(paged_kv_fp8), _ptr(kv_scale), _ptr(page_table), _ptr(seq_lens), _ptr(o),
+        _ptr(lse), B, H_q, d_qk, d_v, page_size, max_pages, n_pages, n_sink, n_local,
+        float(scale), _ptr(workspace), workspace.numel(), _stream(stream)))
     return o, lse
 
 

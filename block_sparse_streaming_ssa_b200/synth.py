@@ -15,6 +15,8 @@ Workloads (all synthetic: the pages publish no dataset for this kernel):
              (512 latent + 64 rope), d_v=512, context lengths uniform integers
              in [4096, 1048576], 128-token pages placed by a random permutation
              of the whole pool, N(0,1) -> bf16, scale 1/sqrt(576).
+* ``decode`` over an FP8 cache: the same shapes; each token row N(0,1),
+             quantised to e4m3 codes with one fp32 scale max|x| / 440.
 * ``varlen`` 8 sequences, lengths uniform in [1024, 131072] rounded to the
              nearest multiple of 128, redrawn until the total is <= 524288,
              H=32, d=128, N(0,1) -> bf16, scale 1/sqrt(128).
@@ -188,6 +190,36 @@ def decode_inputs(seq_lens, H_q, d_qk, seed=0, device="cpu", page_size=BLOCK, pe
     pt = torch.from_numpy(table).to(device)
     sl = torch.tensor(seq_lens, dtype=torch.int32, device=device)
     return q, kv, pt, sl
+
+
+def decode_inputs_fp8(seq_lens, H_q, d_qk, seed=0, device="cpu", page_size=BLOCK, permute=True,
+                      max_pages=None, scale_spread=0.0, chunk_pages=2048):
+    """q [B,H_q,d_qk] bf16 and an FP8 page pool: kv8 [n_pages,page_size,d_qk]
+    uint8 e4m3 codes with kv_scale [n_pages,page_size] fp32 per token; page
+    table and seq_lens as decode_inputs.  Each token's row is drawn N(0,1)
+    (times exp(U(-spread, spread)) per token when scale_spread > 0), its scale
+    is max|x| / 440 and its codes are torch's round-to-nearest float8_e4m3fn
+    cast of x / scale (generated ``chunk_pages`` pages at a time)."""
+    table, n_pages = decode_page_table(seq_lens, page_size, seed, max_pages, permute)
+    g = _gen(seed, device)
+    B = len(seq_lens)
+    q = _randn_bf16((B, H_q, d_qk), g, device)
+    kv8 = torch.empty((n_pages, page_size, d_qk), dtype=torch.uint8, device=device)
+    kv_scale = torch.empty((n_pages, page_size), dtype=torch.float32, device=device)
+    for p0 in range(0, n_pages, chunk_pages):
+        p1 = min(n_pages, p0 + chunk_pages)
+        x = torch.randn((p1 - p0, page_size, d_qk), generator=g, device=device,
+                        dtype=torch.float32)
+        if scale_spread:
+            u = torch.rand((p1 - p0, page_size, 1), generator=g, device=device)
+            x.mul_(torch.exp((2 * u - 1) * scale_spread))
+        sc = x.abs().amax(dim=-1).clamp_min(1e-30) / 440.0
+        kv8[p0:p1] = (x / sc[..., None]).to(torch.float8_e4m3fn).view(torch.uint8)
+        kv_scale[p0:p1] = sc
+        del x
+    pt = torch.from_numpy(table).to(device)
+    sl = torch.tensor(seq_lens, dtype=torch.int32, device=device)
+    return q, kv8, kv_scale, pt, sl
 
 
 def bf16_bits(t: torch.Tensor) -> np.ndarray:

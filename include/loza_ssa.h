@@ -210,6 +210,28 @@ size_t loza_ssa_decode_selected_workspace_size(int B, int H_q, int d_v, int n_si
                                                int max_extra);
 
 /*
+ * Paged SSA decode over an FP8 latent cache.  Token j's cached row is 576
+ * e4m3 codes k8_j (OCP FP8 E4M3: 1 sign, 4 exponent bits with bias 7, 3
+ * mantissa bits, subnormals; 0x7f / 0xff are NaN and must not occur) and one
+ * fp32 scale s_j, standing for K_j = s_j * k8_j (V_j = its first 512 entries).
+ * The result is loza_ssa_decode's over those K_j: the SSA window of the QbitAI
+ * LoZA article, softmax in fp32.  (An FP8 cache is one of the variants of the
+ * decode workload; the LoZA pages' own FP8 remark is about compressed
+ * matrices and fixes no cache format, so the per-token scale is this
+ * library's choice: it keeps the scale out of the tensor-core products.)
+ *   paged_kv_fp8 : DEVICE uint8 [n_pages, page_size, 576] e4m3 codes, 16-byte aligned.
+ *   kv_scale     : DEVICE fp32 [n_pages, page_size], finite; 4-byte aligned.
+ * workspace: at least loza_ssa_decode_workspace_size(B, H_q, d_v, n_sink,
+ * n_local) bytes.  Other arguments, layouts, ownership and statuses as for
+ * loza_ssa_decode; kv_scale == NULL is LOZA_SSA_ERR_NULL.
+ */
+int loza_ssa_decode_fp8(const void* q, const void* paged_kv_fp8, const float* kv_scale,
+                        const int* page_table, const int* seq_lens, void* o, float* lse, int B,
+                        int H_q, int d_qk, int d_v, int page_size, int max_pages, int n_pages,
+                        int n_sink, int n_local, float scale, void* workspace,
+                        size_t workspace_bytes, loza_ssa_stream_t stream);
+
+/*
  * Paged SSA decode with q_len query tokens per sequence (speculative or
  * multi-token-prediction steps): the tokens of sequence b sit at positions
  * t = seq_len[b] - q_len .. seq_len[b] - 1, and token t attends the keys

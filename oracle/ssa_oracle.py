@@ -450,6 +450,40 @@ def brute_force_decode_selected(q, kv, page_table, seq_lens, extra_pages, dv, pa
     return o, lse
 
 
+def e4m3_to_f64(codes) -> np.ndarray:
+    """Values of OCP FP8 E4M3 codes (uint8), from the format's definition: bit
+    7 sign, bits 3..6 exponent e with bias 7, bits 0..2 mantissa m; e = 0 is
+    subnormal (m/8 * 2^-6), otherwise (1 + m/8) * 2^(e-7); e = 15 with m = 7
+    is NaN (there are no infinities)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((e == 15) & ((c & 0x7) == 7), np.nan, mag)
+    return sign * mag
+
+
+def dequant_fp8_cache(kv8, kv_scale) -> np.ndarray:
+    """K_j = s_j * k8_j, float64: kv8 [n_pages, page_size, d] e4m3 codes,
+    kv_scale [n_pages, page_size]."""
+    k = e4m3_to_f64(kv8)
+    if np.isnan(k).any():
+        raise ValueError("NaN code in the FP8 cache")
+    return k * np.asarray(kv_scale, dtype=np.float64)[..., None]
+
+
+def decode_fp8(q, kv8, kv_scale, page_table, seq_lens, dv, page_size=128, n_sink=1, n_local=7,
+               scale=None, rows=None):
+    """Paged SSA decode over an FP8 latent cache: every token's row is e4m3
+    codes times one fp32 scale.  The cache is dequantized exactly to float64
+    and decode() runs on it (the decode-workload variant with an FP8 KV cache;
+    the per-token scale layout is this library's reading, the pages fix none)."""
+    q64 = _as_f64(q)
+    kv = dequant_fp8_cache(kv8, kv_scale)
+    return decode(q64, kv, page_table, seq_lens, dv, page_size, n_sink, n_local, scale, rows)
+
+
 def decode_full(q, kv, page_table, seq_lens, dv, page_size=128, scale=None, rows=None):
     """Full-attention decode (the MLA layers that LoZA keeps, "LoZA：ZigZag稀疏注意力机制"
     §2.1, first formula, for the newest query token): softmax over every key

@@ -221,6 +221,21 @@ def test_decode_argument_errors(L):
     assert _decode(L, ws=0x10010) == -6
 
 
+def test_decode_fp8_argument_errors(L):
+    vp = ctypes.c_void_p
+
+    def call(ksc=0x1000, kv=0x1000, dqk=576):
+        return L.loza_ssa_decode_fp8(vp(0x1000), vp(kv), vp(ksc), vp(0x1000), vp(0x1000),
+                                     vp(0x1000), vp(0x1000), 2, 128, dqk, 512, 128, 16, 32, 1, 7,
+                                     ctypes.c_float(0.04), vp(0x10000), 1 << 30, None)
+
+    assert call(ksc=0) == -1            # no scales
+    assert call(kv=0) == -1
+    assert call(dqk=512) == -3
+    assert call(ksc=0x1002) == -6       # scales not 4-byte aligned
+    assert call(kv=0x1008) == -6        # codes not 16-byte aligned
+
+
 def test_decode_layers_workspace_size(L):
     from block_sparse_streaming_ssa_b200 import loza_ssa as api
     # SSA layers only: the SSA decode's workspace; with a full-attention layer,

@@ -377,6 +377,77 @@ def test_decode_selected_without_pages_is_decode():
     np.testing.assert_array_equal(a[1], b[1])
 
 
+# --- decode over an FP8 (e4m3 + per-token scale) latent cache
+
+
+def test_e4m3_known_values():
+    v = orc.e4m3_to_f64(np.array([0x00, 0x80, 0x38, 0x7E, 0x01, 0x07, 0x08, 0xC8, 0x3C, 0x77,
+                                  0x7F, 0xFF], np.uint8))
+    np.testing.assert_array_equal(v[:10], [0.0, -0.0, 1.0, 448.0, 2.0 ** -9, 7 * 2.0 ** -9,
+                                           2.0 ** -6, -4.0, 1.5, 240.0])
+    assert np.isnan(v[10]) and np.isnan(v[11])
+
+
+def test_e4m3_matches_torch_float8():
+    torch = pytest.importorskip("torch")
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(orc.e4m3_to_f64(codes), ref)
+
+
+def _fp8_case(seed, seq_lens, Hq=4, dqk=24, ps=8):
+    q, kv, pt, sl = _decode_case(seed, seq_lens, Hq=Hq, dqk=dqk, ps=ps)
+    rng = np.random.default_rng(seed + 50)
+    kv8 = rng.integers(0, 256, size=kv.shape, dtype=np.uint8)
+    kv8[(kv8 & 0x7F) == 0x7F] = 0x3C          # no NaN codes
+    kv_scale = np.exp(rng.uniform(-4, 4, size=kv.shape[:2]))
+    return q, kv8, kv_scale, pt, sl
+
+
+def test_decode_fp8_matches_brute_force_on_dequantized_cache():
+    q, kv8, ksc, pt, sl = _fp8_case(31, [1, 9, 61, 100])
+    o, lse = orc.decode_fp8(q, kv8, ksc, pt, sl, dv=16, page_size=8, n_sink=1, n_local=3,
+                            scale=0.02)
+    kv = orc.e4m3_to_f64(kv8) * ksc[..., None]
+    o_bf, lse_bf = orc.brute_force_decode(q, kv, pt, sl, dv=16, page_size=8, n_sink=1,
+                                          n_local=3, scale=0.02)
+    np.testing.assert_allclose(o, o_bf, rtol=1e-11, atol=1e-9)
+    np.testing.assert_allclose(lse, lse_bf, atol=1e-10)
+
+
+def test_decode_fp8_unit_scales_equal_bf16_decode():
+    """Scales of 1: the e4m3 values are exact in bf16, so the decode over the
+    bf16 bit patterns of the same values (C oracle, bf16 input path) agrees."""
+    torch = pytest.importorskip("torch")
+    q, kv8, _, pt, sl = _fp8_case(32, [40, 77])
+    ones = np.ones(kv8.shape[:2])
+    vals = torch.from_numpy(kv8).view(torch.float8_e4m3fn).to(torch.bfloat16)
+    kv_bits = vals.view(torch.int16).numpy().view(np.uint16)
+    q_bits = torch.from_numpy(q).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    a = orc.decode_fp8(q_bits, kv8, ones, pt, sl, dv=16, page_size=8, n_sink=1, n_local=3)
+    b = orc.decode(q_bits, kv_bits, pt, sl, dv=16, page_size=8, n_sink=1, n_local=3)
+    np.testing.assert_allclose(a[0], b[0], atol=1e-13)
+    np.testing.assert_allclose(a[1], b[1], atol=1e-13)
+
+
+def test_decode_fp8_scale_moves_between_cache_and_query():
+    """Doubling every token's scale doubles K_j and V_j; halving the attention
+    scale as well leaves every score, so the weights and the LSE are unchanged
+    and O, a weighted mean of the V_j, doubles."""
+    q, kv8, ksc, pt, sl = _fp8_case(33, [70, 33])
+    o1, l1 = orc.decode_fp8(q, kv8, ksc, pt, sl, dv=16, page_size=8, scale=0.02)
+    o2, l2 = orc.decode_fp8(q, kv8, 2 * ksc, pt, sl, dv=16, page_size=8, scale=0.01)
+    np.testing.assert_allclose(o2, 2 * o1, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(l2, l1, atol=1e-12)
+
+
+def test_decode_fp8_rejects_nan_codes():
+    q, kv8, ksc, pt, sl = _fp8_case(34, [20])
+    kv8[0, 0, 0] = 0x7F
+    with pytest.raises(ValueError):
+        orc.decode_fp8(q, kv8, ksc, pt, sl, dv=16, page_size=8)
+
+
 # --- full-attention decode (the MLA layers LoZA keeps) and the layer stack
 
 
