@@ -301,30 +301,46 @@ def backward_bench(w, steps, warmup, peaks, world=1):
 
 
 def e2e_prefill(w, steps):
-    """Same metric through the public call with host buffers: pinned host ->
-    device copy of q, k, v, the call, device -> host copy of o and lse, every step."""
+    """Same metric through the public call with host buffers: for the dense
+    workloads loza_ssa_prefill_host (pinned host q, k, v in, pinned host o,
+    lse out, copies inside the call, overlapped over chunks of planes); for the
+    packed workload pinned-host copies around loza_ssa_prefill_varlen."""
     import torch
+    from block_sparse_streaming_ssa_b200.loza_ssa import (loza_ssa_prefill_host,
+                                                          loza_ssa_prefill_host_workspace_size)
     hq, hk, hv = (t.cpu().pin_memory() for t in (w["q"], w["k"], w["v"]))
-    dq, dk, dv = (torch.empty_like(t) for t in (w["q"], w["k"], w["v"]))
     o, lse = prefill_call(w)
     ho, hl = o.cpu().pin_memory(), lse.cpu().pin_memory()
-    for _ in range(1):
-        dq.copy_(hq, non_blocking=True)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+    if not w["varlen"]:
+        sp = w["spec"]
+        ws = torch.empty(loza_ssa_prefill_host_workspace_size(sp.B, sp.H, sp.L, sp.d_qk, sp.d_v),
+                         dtype=torch.uint8, device="cuda")
+        del o, lse
+        torch.cuda.empty_cache()
+
+        def step():
+            loza_ssa_prefill_host(hq, hk, hv, o=ho, lse=hl, scale=sp.scale, workspace=ws)
+    else:
+        dq, dk, dv = (torch.empty_like(t) for t in (w["q"], w["k"], w["v"]))
+
+        def step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            prefill_call(w, dq, dk, dv, o=o, lse=lse)
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+    step()
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record()
     for _ in range(steps):
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        prefill_call(w, dq, dk, dv, o=o, lse=lse)
-        ho.copy_(o, non_blocking=True)
-        hl.copy_(lse, non_blocking=True)
+        step()
     t1.record()
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1) / steps
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
-    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
     return ms, h2d, d2h
 
 

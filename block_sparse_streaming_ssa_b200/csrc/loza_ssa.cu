@@ -10,6 +10,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "../../include/loza_ssa.h"
 #include "backward.cuh"
@@ -309,6 +310,62 @@ size_t decode_partial_floats(int B, int H_q, int n_split) {
 
 }  // namespace
 
+namespace {
+
+// Device staging of loza_ssa_prefill_host: q, k, v, o and lse, each 256-byte aligned.
+struct HostStaging {
+  size_t q, k, v, o, lse, total;
+};
+
+HostStaging host_staging(long long planes, int L, int d_qk, int d_v) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  HostStaging st;
+  st.q = up((size_t)planes * L * d_qk * 2);
+  st.k = st.q;
+  st.v = up((size_t)planes * L * d_v * 2);
+  st.o = st.v;
+  st.lse = up((size_t)planes * L * 4);
+  st.total = st.q + st.k + st.v + st.o + st.lse;
+  return st;
+}
+
+// Copy streams of the host-buffer call, one pair per device, created once.
+cudaStream_t g_h2d[kMaxDevices] = {};
+cudaStream_t g_d2h[kMaxDevices] = {};
+
+int copy_streams(cudaStream_t* h2d, cudaStream_t* d2h) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return LOZA_SSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_h2d[dev]) {
+    if ((e = cudaStreamCreateWithFlags(&g_h2d[dev], cudaStreamNonBlocking)) != cudaSuccess)
+      return cuda_fail(e, "cudaStreamCreateWithFlags(h2d)");
+    if ((e = cudaStreamCreateWithFlags(&g_d2h[dev], cudaStreamNonBlocking)) != cudaSuccess)
+      return cuda_fail(e, "cudaStreamCreateWithFlags(d2h)");
+  }
+  *h2d = g_h2d[dev];
+  *d2h = g_d2h[dev];
+  return LOZA_SSA_OK;
+}
+
+// Events of one host-buffer call: created per call, released by the driver
+// once the work that records them has completed.
+struct EventSet {
+  std::vector<cudaEvent_t> ev;
+  ~EventSet() {
+    for (cudaEvent_t e : ev) cudaEventDestroy(e);
+  }
+  cudaError_t make(cudaEvent_t* out) {
+    cudaError_t e = cudaEventCreateWithFlags(out, cudaEventDisableTiming);
+    if (e == cudaSuccess) ev.push_back(*out);
+    return e;
+  }
+};
+
+}  // namespace
+
 extern "C" {
 
 int loza_ssa_version(void) { return kVersion; }
@@ -361,6 +418,80 @@ int loza_ssa_prefill(const void* q, const void* k, const void* v, void* o, float
   prm.total_items = (int)items;
   return dispatch_prefill(d_qk, d_v, q, k, v, prm, (uint64_t)L, (uint64_t)B * H, items, 0,
                           reinterpret_cast<cudaStream_t>(stream), dev);
+}
+
+size_t loza_ssa_prefill_host_workspace_size(int B, int H, int L, int d_qk, int d_v) {
+  if (B < 1 || H < 1 || L < 1 || !prefill_dims_ok(d_qk, d_v)) return 0;
+  return host_staging((long long)B * H, L, d_qk, d_v).total;
+}
+
+int loza_ssa_prefill_host(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int H, int L, int d_qk, int d_v, int block, int n_sink,
+                          int n_local, float scale, int n_chunks, void* workspace,
+                          size_t workspace_bytes, loza_ssa_stream_t stream) {
+  if (!q || !k || !v || !o || !lse || !workspace) return LOZA_SSA_ERR_NULL;
+  if (B < 1 || H < 1 || L < 1 || n_chunks < 1 || !std::isfinite(scale)) return LOZA_SSA_ERR_SHAPE;
+  if (!prefill_dims_ok(d_qk, d_v)) return LOZA_SSA_ERR_HEAD_DIM;
+  if (block != 128) return LOZA_SSA_ERR_BLOCK;
+  if (n_sink < 0 || n_local < 1) return LOZA_SSA_ERR_WINDOW;
+  const long long planes = (long long)B * H;
+  const HostStaging st = host_staging(planes, L, d_qk, d_v);
+  if (workspace_bytes < st.total) return LOZA_SSA_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return LOZA_SSA_ERR_ALIGN;
+  cudaStream_t h2d, d2h;
+  int rc = copy_streams(&h2d, &d2h);
+  if (rc != LOZA_SSA_OK) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  char* dq = ws;
+  char* dk = dq + st.q;
+  char* dv = dk + st.k;
+  char* dout = dv + st.v;
+  char* dlse = dout + st.o;
+  const size_t q_plane = (size_t)L * d_qk * 2, v_plane = (size_t)L * d_v * 2,
+               l_plane = (size_t)L * 4;
+  const long long chunks = n_chunks < planes ? n_chunks : planes;
+  EventSet evs;
+  cudaEvent_t start, fin;
+  cudaError_t e;
+  // everything below follows the caller's earlier work on its stream (which
+  // may still read this staging from a previous call)
+  if ((e = evs.make(&start)) != cudaSuccess || (e = cudaEventRecord(start, s)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(h2d, start, 0)) != cudaSuccess)
+    return cuda_fail(e, "host prefill: start");
+  for (long long c = 0; c < chunks; ++c) {
+    const long long p0 = planes * c / chunks, p1 = planes * (c + 1) / chunks, np = p1 - p0;
+    const char* hq = static_cast<const char*>(q) + p0 * q_plane;
+    const char* hk = static_cast<const char*>(k) + p0 * q_plane;
+    const char* hv = static_cast<const char*>(v) + p0 * v_plane;
+    cudaEvent_t in, done;
+    if ((e = cudaMemcpyAsync(dq + p0 * q_plane, hq, np * q_plane, cudaMemcpyHostToDevice, h2d)) !=
+            cudaSuccess ||
+        (e = cudaMemcpyAsync(dk + p0 * q_plane, hk, np * q_plane, cudaMemcpyHostToDevice, h2d)) !=
+            cudaSuccess ||
+        (e = cudaMemcpyAsync(dv + p0 * v_plane, hv, np * v_plane, cudaMemcpyHostToDevice, h2d)) !=
+            cudaSuccess ||
+        (e = evs.make(&in)) != cudaSuccess || (e = cudaEventRecord(in, h2d)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(s, in, 0)) != cudaSuccess)
+      return cuda_fail(e, "host prefill: upload");
+    // the chunk's planes are whole (b, h) planes: one dense call over [1, np, L, d]
+    rc = loza_ssa_prefill(dq + p0 * q_plane, dk + p0 * q_plane, dv + p0 * v_plane,
+                          dout + p0 * v_plane, reinterpret_cast<float*>(dlse + p0 * l_plane), 1,
+                          (int)np, L, d_qk, d_v, block, n_sink, n_local, scale, stream);
+    if (rc != LOZA_SSA_OK) return rc;
+    if ((e = evs.make(&done)) != cudaSuccess || (e = cudaEventRecord(done, s)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(d2h, done, 0)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(static_cast<char*>(o) + p0 * v_plane, dout + p0 * v_plane,
+                             np * v_plane, cudaMemcpyDeviceToHost, d2h)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(reinterpret_cast<char*>(lse) + p0 * l_plane, dlse + p0 * l_plane,
+                             np * l_plane, cudaMemcpyDeviceToHost, d2h)) != cudaSuccess)
+      return cuda_fail(e, "host prefill: download");
+  }
+  // the caller's stream completes once the last download has
+  if ((e = evs.make(&fin)) != cudaSuccess || (e = cudaEventRecord(fin, d2h)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(s, fin, 0)) != cudaSuccess)
+    return cuda_fail(e, "host prefill: finish");
+  return LOZA_SSA_OK;
 }
 
 size_t loza_ssa_prefill_bwd_workspace_size(int B, int H, int L, int d_qk, int d_v, int n_sink,

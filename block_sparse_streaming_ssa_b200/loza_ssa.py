@@ -70,6 +70,11 @@ def lib() -> ctypes.CDLL:
         L.loza_ssa_decode_mtp.restype = i32
         L.loza_ssa_decode_mtp_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
         L.loza_ssa_decode_mtp_workspace_size.restype = sz
+        L.loza_ssa_prefill_host.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                            i32, i32, f32, i32, vp, sz, vp]
+        L.loza_ssa_prefill_host.restype = i32
+        L.loza_ssa_prefill_host_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+        L.loza_ssa_prefill_host_workspace_size.restype = sz
         L.loza_ssa_decode_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                           i32, i32, i32, i32, f32, vp, sz, vp]
         L.loza_ssa_decode_fp8.restype = i32
@@ -167,6 +172,51 @@ def loza_ssa_prefill(q, k, v, o=None, lse=None, block=128, n_sink=1, n_local=7, 
         scale = 1.0 / math.sqrt(d_qk)
     _check(lib().loza_ssa_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, L, d_qk,
                                   d_v, block, n_sink, n_local, float(scale), _stream(stream)))
+    return o, lse
+
+
+def _need_host(t: torch.Tensor, dtype, name: str) -> None:
+    if not isinstance(t, torch.Tensor) or t.is_cuda:
+        raise TypeError(f"{name} must be a host (CPU) tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def loza_ssa_prefill_host_workspace_size(B, H, L, d_qk, d_v) -> int:
+    return int(lib().loza_ssa_prefill_host_workspace_size(B, H, L, d_qk, d_v))
+
+
+def loza_ssa_prefill_host(q, k, v, o=None, lse=None, block=128, n_sink=1, n_local=7, scale=None,
+                          n_chunks=8, workspace=None, stream=None):
+    """Dense SSA prefill from host tensors (copies inside the call, overlapped
+    across chunks of (batch, head) planes).  q, k, v: CPU bf16 [B,H,L,d]
+    (pinned for overlap); o, lse: CPU outputs, allocated pinned if not given;
+    workspace: uint8 CUDA tensor of loza_ssa_prefill_host_workspace_size bytes.
+    The outputs are complete once `stream` (default: the current one) has
+    passed the call.  Returns (o, lse)."""
+    _need_host(q, torch.bfloat16, "q")
+    _need_host(k, torch.bfloat16, "k")
+    _need_host(v, torch.bfloat16, "v")
+    B, H, L, d_qk = q.shape
+    d_v = v.shape[-1]
+    if o is None:
+        o = torch.empty((B, H, L, d_v), dtype=torch.bfloat16).pin_memory()
+    if lse is None:
+        lse = torch.empty((B, H, L), dtype=torch.float32).pin_memory()
+    _need_host(o, torch.bfloat16, "o")
+    _need_host(lse, torch.float32, "lse")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d_qk)
+    need = loza_ssa_prefill_host_workspace_size(B, H, L, d_qk, d_v)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
+    _need(workspace, torch.uint8, "workspace")
+    _check(lib().loza_ssa_prefill_host(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, L, d_qk, d_v, block, n_sink,
+        n_local, float(scale), int(n_chunks), _ptr(workspace), workspace.numel(),
+        _stream(stream)))
     return o, lse
 
 

@@ -82,6 +82,33 @@ int loza_ssa_prefill(const void* q, const void* k, const void* v, void* o, float
                      float scale, loza_ssa_stream_t stream);
 
 /*
+ * Dense SSA prefill from HOST buffers: the same result as loza_ssa_prefill,
+ * with the copies inside the call.  The B*H (batch, head) planes are cut into
+ * n_chunks runs of whole planes; each run is uploaded on a copy stream of the
+ * library's, computed on `stream` once it has landed, and downloaded on a
+ * second copy stream, so uploads, kernels and downloads of different runs
+ * overlap (the two copy directions run at once).
+ *   q, k, v     : HOST bf16 [B, H, L, d] as loza_ssa_prefill; page-locked
+ *                 (cudaHostAlloc / cudaHostRegister) for the copies to overlap.
+ *   o, lse      : HOST outputs, page-locked likewise; complete once `stream`
+ *                 reaches the end of the call (synchronise it before reading).
+ *   n_chunks    : >= 1 (more than B*H acts as B*H); 8 suits large inputs.
+ *   workspace   : DEVICE, 256-byte aligned, at least
+ *                 loza_ssa_prefill_host_workspace_size(...) bytes: device
+ *                 copies of q, k, v, o, lse, owned by the caller and reusable
+ *                 once `stream` has passed the call.
+ * Statuses as loza_ssa_prefill, plus LOZA_SSA_ERR_WORKSPACE.  The host
+ * buffers must stay valid until `stream` has passed the call.
+ */
+int loza_ssa_prefill_host(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int H, int L, int d_qk, int d_v, int block, int n_sink,
+                          int n_local, float scale, int n_chunks, void* workspace,
+                          size_t workspace_bytes, loza_ssa_stream_t stream);
+
+/* Bytes of device workspace loza_ssa_prefill_host needs (0 on invalid sizes). */
+size_t loza_ssa_prefill_host_workspace_size(int B, int H, int L, int d_qk, int d_v);
+
+/*
  * Packed variable-length SSA prefill.  Sequence s occupies tokens
  * [cu_seqlens[s], cu_seqlens[s+1]) of the packed axis; block indices count from
  * each sequence's own first token, and no key crosses a sequence boundary.

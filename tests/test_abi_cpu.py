@@ -221,6 +221,27 @@ def test_decode_argument_errors(L):
     assert _decode(L, ws=0x10010) == -6
 
 
+def test_prefill_host_workspace_and_errors(L):
+    from block_sparse_streaming_ssa_b200 import loza_ssa as api
+    up = lambda x: -(-x // 256) * 256
+    B, H, Lq = 2, 3, 1000
+    want = 2 * up(B * H * Lq * 128 * 2) + 2 * up(B * H * Lq * 128 * 2) + up(B * H * Lq * 4)
+    assert api.loza_ssa_prefill_host_workspace_size(B, H, Lq, 128, 128) == want
+    assert api.loza_ssa_prefill_host_workspace_size(B, H, Lq, 96, 96) == 0
+    vp = ctypes.c_void_p
+
+    def call(q=0x1000, chunks=4, ws=0x10000, ws_bytes=1 << 30, dqk=128):
+        return L.loza_ssa_prefill_host(vp(q), vp(0x1000), vp(0x1000), vp(0x1000), vp(0x1000),
+                                       B, H, Lq, dqk, 128, 128, 1, 7, ctypes.c_float(0.09),
+                                       chunks, vp(ws), ws_bytes, None)
+    assert call(q=0) == -1
+    assert call(ws=0) == -1
+    assert call(chunks=0) == -2
+    assert call(dqk=96) == -3
+    assert call(ws_bytes=want - 1) == -7
+    assert call(ws=0x10010) == -6
+
+
 def test_decode_fp8_argument_errors(L):
     vp = ctypes.c_void_p
 
