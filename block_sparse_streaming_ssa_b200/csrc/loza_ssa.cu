@@ -380,7 +380,9 @@ const char* loza_ssa_status_string(int status) {
     case LOZA_SSA_ERR_HEAD_DIM: return "unsupported (d_qk, d_v)";
     case LOZA_SSA_ERR_BLOCK: return "block / page_size must be 128";
     case LOZA_SSA_ERR_WINDOW: return "n_sink / n_local out of range";
-    case LOZA_SSA_ERR_ALIGN: return "pointer not aligned (bf16 tensors: 16 B, lse: 4 B, workspace: 256 B)";
+    case LOZA_SSA_ERR_ALIGN:
+      return "pointer not aligned (bf16 tensors: 16 B; prefill o and backward dq, dk, dv: 32 B; "
+             "lse: 4 B; workspace: 256 B)";
     case LOZA_SSA_ERR_WORKSPACE: return "decode workspace missing or too small";
     case LOZA_SSA_ERR_CUDA: return "CUDA error (see loza_ssa_last_error_string)";
     case LOZA_SSA_ERR_SCRATCH_LIMIT: return "decode needs more split slots than the built-in scratch holds";
@@ -396,7 +398,7 @@ int loza_ssa_prefill(const void* q, const void* k, const void* v, void* o, float
   if (!prefill_dims_ok(d_qk, d_v)) return LOZA_SSA_ERR_HEAD_DIM;
   if (block != 128) return LOZA_SSA_ERR_BLOCK;
   if (n_sink < 0 || n_local < 1) return LOZA_SSA_ERR_WINDOW;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 32) || !aligned(lse, 4))
     return LOZA_SSA_ERR_ALIGN;
   const long long nb = (L + 127) / 128;
   const long long items = (long long)B * H * nb;
@@ -514,7 +516,7 @@ int loza_ssa_prefill_bwd(const void* q, const void* k, const void* v, const void
   if (block != 128) return LOZA_SSA_ERR_BLOCK;
   if (n_sink < 0 || n_local < 1) return LOZA_SSA_ERR_WINDOW;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
-      !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+      !aligned(dout, 16) || !aligned(dq, 32) || !aligned(dk, 32) || !aligned(dv, 32) ||
       !aligned(lse, 4))
     return LOZA_SSA_ERR_ALIGN;
   const long long nb = (L + 127) / 128;
@@ -608,7 +610,7 @@ int loza_ssa_prefill_varlen_bwd(const void* q, const void* k, const void* v, con
   if (block != 128) return LOZA_SSA_ERR_BLOCK;
   if (n_sink < 0 || n_local < 1) return LOZA_SSA_ERR_WINDOW;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
-      !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+      !aligned(dout, 16) || !aligned(dq, 32) || !aligned(dk, 32) || !aligned(dv, 32) ||
       !aligned(lse, 4) || !aligned(cu_seqlens, 4))
     return LOZA_SSA_ERR_ALIGN;
   const BwdVarlenWorkspace w =
@@ -660,7 +662,7 @@ int loza_ssa_prefill_varlen(const void* q, const void* k, const void* v, void* o
   if (!prefill_dims_ok(d_qk, d_v)) return LOZA_SSA_ERR_HEAD_DIM;
   if (block != 128) return LOZA_SSA_ERR_BLOCK;
   if (n_sink < 0 || n_local < 1) return LOZA_SSA_ERR_WINDOW;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 32) ||
       !aligned(lse, 4) || !aligned(cu_seqlens, 4))
     return LOZA_SSA_ERR_ALIGN;
   // sum_s ceil(len_s/128) <= total/128 + n_seqs bounds the work-item count

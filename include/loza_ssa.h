@@ -23,7 +23,10 @@
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers, caller-owned, row-major and
  *     contiguous.  bf16 tensors hold IEEE bfloat16; lse is fp32.
- *   - bf16 tensor pointers must be 16-byte aligned, lse 4-byte aligned.
+ *   - bf16 tensor pointers must be 16-byte aligned, lse 4-byte aligned; the
+ *     outputs the prefill and the backward write with 32-byte stores (o of
+ *     loza_ssa_prefill and loza_ssa_prefill_varlen, dq / dk / dv of the
+ *     backward calls) 32-byte aligned.
  *   - Work is enqueued on `stream` and is asynchronous; no call synchronises
  *     the device, and no call allocates device memory.  Inputs are never
  *     modified.  Calls on different streams may run concurrently.

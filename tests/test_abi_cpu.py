@@ -195,6 +195,17 @@ def test_prefill_argument_errors(L):
     assert _prefill(L, nl=0) == -5
     assert _prefill(L, q=0x1008) == -6
     assert _prefill(L, lse=0x1002) == -6
+    assert _prefill(L, o=0x1010) == -6      # o is written with 32-byte stores
+
+
+def test_backward_outputs_need_32_byte_alignment(L):
+    vp = ctypes.c_void_p
+    a = vp(0x1000)
+    for pos in (6, 7, 8):                   # dq, dk, dv
+        ptrs = [a] * 9
+        ptrs[pos] = vp(0x1010)
+        assert L.loza_ssa_prefill_bwd(*ptrs, 1, 2, 1024, 128, 128, 128, 1, 7,
+                                      ctypes.c_float(0.08), a, 1 << 30, None) == -6
 
 
 def _decode(L, B=2, Hq=128, dqk=576, dv=512, ps=128, max_pages=16, n_pages=32, ns=1, nl=7,

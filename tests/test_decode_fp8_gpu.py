@@ -5,7 +5,9 @@ import pytest
 import torch
 
 from block_sparse_streaming_ssa_b200 import synth
-from block_sparse_streaming_ssa_b200.loza_ssa import (loza_ssa_decode, loza_ssa_decode_fp8,
+from block_sparse_streaming_ssa_b200.loza_ssa import (LOZA_SSA_DEV_BAD_PAGE,
+                                                      LOZA_SSA_DEV_BAD_SEQLEN, loza_ssa_decode,
+                                                      loza_ssa_decode_fp8,
                                                       loza_ssa_get_last_device_status)
 from oracle import ssa_oracle as orc
 from tests.parity import LSE_MAX_ABS, O_REL_L2, assert_parity, errors
@@ -140,3 +142,23 @@ def test_fp8_full_workload_sampled():
     rows = np.sort(rng.choice(s.B * s.H_q, 256, replace=False))
     o, lse, o_ref, lse_ref = run(lens, seed=0, spread=0.0, rows=rows)
     assert_parity(o, lse, o_ref, lse_ref, "fp8 full workload")
+
+
+def test_fp8_bad_pages_and_lengths_are_flagged():
+    """A page id outside the pool and a length past the table set their status
+    bits; the other sequence's rows are unchanged."""
+    q, kv8, ksc, pt, sl = synth.decode_inputs_fp8([2000, 700], 128, D_QK, seed=4, device="cuda")
+    good, _ = loza_ssa_decode_fp8(q, kv8, ksc, pt, sl, D_V, scale=SCALE)
+    torch.cuda.synchronize()
+    assert loza_ssa_get_last_device_status() == 0
+    bad = pt.clone()
+    bad[1, 0] = kv8.shape[0] + 5                       # sink page outside the pool
+    o, _ = loza_ssa_decode_fp8(q, kv8, ksc, bad, sl, D_V, scale=SCALE)
+    torch.cuda.synchronize()
+    assert loza_ssa_get_last_device_status() & LOZA_SSA_DEV_BAD_PAGE
+    assert torch.equal(o[0], good[0])
+    long_len = torch.tensor([2000, pt.shape[1] * 128 + 1], dtype=torch.int32, device="cuda")
+    o, _ = loza_ssa_decode_fp8(q, kv8, ksc, pt, long_len, D_V, scale=SCALE)
+    torch.cuda.synchronize()
+    assert loza_ssa_get_last_device_status() & LOZA_SSA_DEV_BAD_SEQLEN
+    assert torch.equal(o[0], good[0])

@@ -7,7 +7,8 @@ import pytest
 import torch
 
 from block_sparse_streaming_ssa_b200 import synth
-from block_sparse_streaming_ssa_b200.loza_ssa import (loza_ssa_decode, loza_ssa_decode_layers,
+from block_sparse_streaming_ssa_b200.loza_ssa import (LOZA_SSA_DEV_BAD_PAGE, loza_ssa_decode,
+                                                      loza_ssa_decode_layers,
                                                       loza_ssa_get_last_device_status)
 from oracle import ssa_oracle as orc
 from tests.parity import assert_parity
@@ -85,3 +86,20 @@ def test_full_layer_with_fewer_heads():
     refs = oracle_stack(layers, pt, sl)
     for i, ((o, lse), (o_r, l_r)) in enumerate(zip(outs, refs)):
         assert_parity(o, lse, o_r, l_r, f"H_q=16 layer {i}")
+
+
+def test_bad_page_in_full_layer_is_flagged():
+    """A table entry outside the pool that only the full-attention layer reads
+    (a middle page, outside the SSA window) flags the full layer; the SSA
+    layer of the same stack and the other sequence are unaffected."""
+    layers, pt, sl = stack_inputs([5000, 3000], (True, False), seed=21)
+    good = loza_ssa_decode_layers(layers, pt, sl, D_V, scale=SCALE)
+    torch.cuda.synchronize()
+    assert loza_ssa_get_last_device_status() == 0
+    bad = pt.clone()
+    bad[0, 10] = layers[0][1].shape[0] + 3            # page 10 of 40: full layer only
+    outs = loza_ssa_decode_layers(layers, bad, sl, D_V, scale=SCALE)
+    torch.cuda.synchronize()
+    assert loza_ssa_get_last_device_status() & LOZA_SSA_DEV_BAD_PAGE
+    assert torch.equal(outs[0][0][1], good[0][0][1])   # full layer, other sequence
+    assert torch.equal(outs[1][0], good[1][0])         # SSA layer, both sequences
