@@ -28,7 +28,8 @@
  *     loza_ssa_prefill and loza_ssa_prefill_varlen, dq / dk / dv of the
  *     backward calls) 32-byte aligned.
  *   - Work is enqueued on `stream` and is asynchronous; no call synchronises
- *     the device, and no call allocates device memory.  Inputs are never
+ *     the device, and no call allocates device memory (loza_ssa_prefill_host
+ *     creates its two copy streams once per device, and CUDA events per call).  Inputs are never
  *     modified.  Calls on different streams may run concurrently.
  *   - On any non-zero status nothing has been launched.
  *   - Errors found by the kernels themselves (a page id outside the pool, a
