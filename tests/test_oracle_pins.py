@@ -62,7 +62,7 @@ def test_golden_row_counts_block128_sink1_local7():
         assert orc.row_count(i, 128, 1, 7) == c, i
 
 
-def test_row_count_north_star_formula():
+def test_row_count_sink_plus_local_formula():
     # min(i+1, 128*[b>=7] + 768 + (i mod 128) + 1) for 1 sink + 7 local blocks of 128
     for i in list(range(0, 2200, 37)) + [895, 896, 1023, 1024, 5000]:
         b = i // 128
