@@ -247,7 +247,8 @@ size_t loza_ssa_decode_selected_workspace_size(int B, int H_q, int d_v, int n_si
  * fp32 scale s_j, standing for K_j = s_j * k8_j (V_j = its first 512 entries).
  * The result is loza_ssa_decode's over those K_j: the SSA window of the QbitAI
  * LoZA article, softmax in fp32.  (An FP8 cache is one of the variants of the
- * decode workload; the LoZA pages' own FP8 remark is about compressed
+ * decode workload; the pages' only FP8 remark -- the CSA/HCA tutorial's
+ * section 5.1, item 3, on mixed-precision training -- is about compressed
  * matrices and fixes no cache format, so the per-token scale is this
  * library's choice: it keeps the scale out of the tensor-core products.)
  *   paged_kv_fp8 : DEVICE uint8 [n_pages, page_size, 576] e4m3 codes, 16-byte aligned.
