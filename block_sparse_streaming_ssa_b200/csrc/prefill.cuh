@@ -131,10 +131,9 @@ struct PrefillLayout {
   static constexpr int B_S_FREE = B_P_FULL + NSB;
   static constexpr int B_O_EMPTY = B_S_FREE + NSB;  // NOB
   static constexpr int B_DRAIN = B_O_EMPTY + NOB;   // 2: one per MMA issuer
-  // the two softmax warpgroups' row exchange: one barrier per TMEM lane
-  // quarter, i.e. per pair of warps (w, w + 4) that share rows
-  static constexpr int B_XCHG = B_DRAIN + 2;        // 4
-  static constexpr int B_OST_FULL = B_XCHG + 4;     // 2, per warpgroup: box written (128)
+  // (the two softmax warpgroups' row exchange uses named barriers 1-4, one
+  // per pair of warps (w, w + 4) that share TMEM lanes)
+  static constexpr int B_OST_FULL = B_DRAIN + 2;    // 2, per warpgroup: box written (128)
   static constexpr int B_OST_FREE = B_OST_FULL + 2; // 2, per warpgroup: box read by its store
   // With an epilogue warpgroup (d_qk = d_v = 128): the softmax warps hand each
   // item's row max and row sums over in shared memory and go on to the next
@@ -273,7 +272,6 @@ __global__ void __launch_bounds__(PrefillLayout<DQK, DV>::THREADS, 1)
       mbar_init(bar(Lay::B_O_EMPTY + s), Lay::EPI_WG ? 128 : kSoftmaxThreads);
     mbar_init(bar(Lay::B_DRAIN), 1);
     mbar_init(bar(Lay::B_DRAIN + 1), 1);
-    for (int qd = 0; qd < 4; ++qd) mbar_init(bar(Lay::B_XCHG + qd), 64);
     for (int w = 0; w < 2; ++w) {
       mbar_init(bar(Lay::B_OST_FULL + w), kSoftmaxThreads / 2);
       mbar_init(bar(Lay::B_OST_FREE + w), 1);
@@ -577,16 +575,20 @@ __global__ void __launch_bounds__(PrefillLayout<DQK, DV>::THREADS, 1)
     float* red = reinterpret_cast<float*>(smem + Lay::OFF_RED);
     const float sl2 = p.scale_log2;
     int g0 = 0, it = 0;
-    uint32_t xc = 0;  // exchanges done (selects the red buffer and the barrier phase)
-    // Publish v for this row, wait for the other half's value for the same row.
+    uint32_t xc = 0;  // exchanges done (selects the red buffer)
+    // Publish v for this row; the other half's value for the same row comes
+    // back in `other`.  Warps w and w + 4 (the same TMEM lanes) meet at named
+    // barrier 1 + (w & 3); the buffer alternates, so an exchange never
+    // overwrites a value the partner has still to read.  The barrier has no
+    // timeout: a thread that leaves the loops early (a failed wait) makes up
+    // the exchanges it skipped before it finishes (see the end of this branch).
     auto exchange = [&](float v, float& other) -> bool {
       float* buf = red + (xc & 1) * 256;
       buf[wg * 128 + row] = v;
-      mbar_arrive(bar(Lay::B_XCHG + (warp & 3)));
-      const bool okx = mbar_wait(bar(Lay::B_XCHG + (warp & 3)), xc & 1, abort_flag, status, 1);
+      named_bar_sync(1 + (warp & 3), 64);
       other = buf[(wg ^ 1) * 128 + row];
       ++xc;
-      return okx;
+      return true;
     };
     // The epilogue of an item runs after the next item's first tile has been
     // handed to the P.V issuer: by then the item's last P.V has finished, so
@@ -813,6 +815,19 @@ __global__ void __launch_bounds__(PrefillLayout<DQK, DV>::THREADS, 1)
       g0 += tr.count;
     }
     if (have_prev) epilogue(prev);
+    // Every softmax thread performs the same number of exchanges -- one per
+    // tile of each of this CTA's items, plus one per item for the row sums of
+    // the deferred epilogue -- so that no partner is left at a named barrier:
+    // a thread that left the loops early makes up the rest here.
+    if (*abort_flag) {
+      uint32_t total = 0;
+      for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
+        const WorkItem w = decode_item(item, p, prefix);
+        total += (uint32_t)tile_range(w.qb, p.n_sink, p.n_local).count + (Lay::EPI_WG ? 0u : 1u);
+      }
+      float unused;
+      while (xc < total) exchange(-INFINITY, unused);
+    }
     if (Lay::TMA_OUT && !Lay::EPI_WG && row == 0) tma_store_wait_all();  // stores done before exit
   }
 

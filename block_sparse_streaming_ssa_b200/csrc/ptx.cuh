@@ -177,6 +177,13 @@ __device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int c0, 
                : "memory");
 }
 
+// Named barrier `id` (1..15) over `n` threads (a multiple of 32).  It has no
+// timeout: every participant must arrive the same number of times.  The
+// non-.aligned form counts threads, so the lanes of a warp may arrive apart.
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 __device__ __forceinline__ void lds_v4(uint32_t addr, uint32_t* r) {
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
