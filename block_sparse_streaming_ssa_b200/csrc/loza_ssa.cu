@@ -341,10 +341,16 @@ int copy_streams(cudaStream_t* h2d, cudaStream_t* d2h) {
   if (dev < 0 || dev >= kMaxDevices) return LOZA_SSA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_mu);
   if (!g_h2d[dev]) {
-    if ((e = cudaStreamCreateWithFlags(&g_h2d[dev], cudaStreamNonBlocking)) != cudaSuccess)
+    // both streams or neither: a half-made pair is released, not kept
+    cudaStream_t up = nullptr, down = nullptr;
+    if ((e = cudaStreamCreateWithFlags(&up, cudaStreamNonBlocking)) != cudaSuccess)
       return cuda_fail(e, "cudaStreamCreateWithFlags(h2d)");
-    if ((e = cudaStreamCreateWithFlags(&g_d2h[dev], cudaStreamNonBlocking)) != cudaSuccess)
+    if ((e = cudaStreamCreateWithFlags(&down, cudaStreamNonBlocking)) != cudaSuccess) {
+      cudaStreamDestroy(up);
       return cuda_fail(e, "cudaStreamCreateWithFlags(d2h)");
+    }
+    g_d2h[dev] = down;
+    g_h2d[dev] = up;
   }
   *h2d = g_h2d[dev];
   *d2h = g_d2h[dev];

@@ -101,8 +101,10 @@ int loza_ssa_prefill(const void* q, const void* k, const void* v, void* o, float
  *                 loza_ssa_prefill_host_workspace_size(...) bytes: device
  *                 copies of q, k, v, o, lse, owned by the caller and reusable
  *                 once `stream` has passed the call.
- * Statuses as loza_ssa_prefill, plus LOZA_SSA_ERR_WORKSPACE.  The host
- * buffers must stay valid until `stream` has passed the call.
+ * Statuses as loza_ssa_prefill, plus LOZA_SSA_ERR_WORKSPACE.  Arguments are
+ * checked before anything is enqueued; a CUDA error part-way (LOZA_SSA_ERR_CUDA)
+ * can leave the earlier runs' copies and kernels enqueued.  The host buffers
+ * must stay valid until `stream` has passed the call.
  */
 int loza_ssa_prefill_host(const void* q, const void* k, const void* v, void* o, float* lse,
                           int B, int H, int L, int d_qk, int d_v, int block, int n_sink,
