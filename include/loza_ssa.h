@@ -31,7 +31,8 @@
  *     the device, and no call allocates device memory (loza_ssa_prefill_host
  *     creates its two copy streams once per device, and CUDA events per call).  Inputs are never
  *     modified.  Calls on different streams may run concurrently.
- *   - On any non-zero status nothing has been launched.
+ *   - On any non-zero status nothing has been launched, except where an entry
+ *     point says otherwise (loza_ssa_decode_layers, loza_ssa_prefill_host).
  *   - Errors found by the kernels themselves (a page id outside the pool, a
  *     sequence length outside the page table, bad cu_seqlens, a pipeline wait
  *     that timed out) are recorded in a per-device status word instead of
