@@ -2,7 +2,6 @@
 the debug exports: the tile scheduler's key-block lists and the decode
 kernel's (logical -> physical) page selection, against lists the oracle reads
 off the mask."""
-import numpy as np
 import pytest
 import torch
 
