@@ -666,20 +666,41 @@ def oracle_sample(config, budget_s, seed=0):
 
 # ------------------------------------------------------------------- main
 
+def prefill_leg(config, steps, warmup, peaks, dist, world, rank):
+    """Time one prefill workload: (compact entry, detail, raw timing)."""
+    import torch
+    w = make_prefill(config, "cuda", seed=rank)
+    total_ms, per, clocks = time_prefill(w, steps, warmup, dist)
+    max_ms = max_over_ranks(total_ms)
+    flops = 2 * (w["spec"].d_qk + w["spec"].d_v) * w["pairs"]
+    avg_launch_ms = sum(per) / len(per)
+    achieved = flops / (avg_launch_ms * 1e-3) / 1e12
+    value = job_throughput(world, flops, steps, max_ms) / 1e12
+    tok_s = job_throughput(world, w["tokens"], steps, max_ms)
+    entry = {"tflops": round(value, 1), "frac": round(achieved / peaks["bf16_tflops"], 4),
+             "ms": round(max_ms / steps, 4), "mtok_s": round(tok_s / 1e6, 2)}
+    return w, entry, dict(total_ms=total_ms, max_ms=max_ms, flops=flops, achieved=achieved,
+                          value=value, tok_s=tok_s, avg_launch_ms=avg_launch_ms, clocks=clocks)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", choices=["mha", "tiny", "mla", "varlen"], default="mha")
+    ap.add_argument("--config", choices=["mla", "mha", "tiny", "varlen"], default="mla",
+                    help="the headline prefill workload (default: the MLA-dims one, the largest "
+                         "that fits one GPU)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-prefill", action="store_true",
                     help="time only the decode workload (for profiler captures of it)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip timing the prefill's backward pass")
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-other-prefill", action="store_true",
+                    help="time only the headline prefill workload")
+    ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--decode-iters", type=int, default=30)
     ap.add_argument("--decode-len-hi", type=int, default=None,
                     help="shorter decode contexts (smaller page pool), for profiler captures")
@@ -743,65 +764,87 @@ def main():
     else:
         torch.cuda.set_device(0)
 
-    if args.no_prefill:
-        decode = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
-                              len_hi=args.decode_len_hi, world=world)
-        selected = None
+    def decode_legs():
+        legs = {"decode": decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
+                                       len_hi=args.decode_len_hi, world=world)}
         if args.decode_extra:
-            selected = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
-                                    len_hi=args.decode_len_hi, world=world,
-                                    n_extra=args.decode_extra)
-        mtp = None
+            legs[f"dec_sel{args.decode_extra}"] = decode_bench(
+                args.decode_iters, args.warmup, peaks, seed=rank, len_hi=args.decode_len_hi,
+                world=world, n_extra=args.decode_extra)
         if args.decode_mtp > 1:
-            mtp = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
-                               len_hi=args.decode_len_hi, world=world, q_len=args.decode_mtp)
-        dfp8 = (decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
-                             len_hi=args.decode_len_hi, world=world, fp8=True)
-                if args.decode_fp8 else None)
-        ctx = (context_bench(peaks, args.decode_context, world=world, seed=rank)
-               if args.decode_context else None)
+            legs[f"dec_mtp{args.decode_mtp}"] = decode_bench(
+                args.decode_iters, args.warmup, peaks, seed=rank, len_hi=args.decode_len_hi,
+                world=world, q_len=args.decode_mtp)
+        if args.decode_fp8:
+            legs["dec_fp8"] = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
+                                           len_hi=args.decode_len_hi, world=world, fp8=True)
+        if args.decode_context:
+            legs["ctx_dec"] = context_bench(peaks, args.decode_context, world=world, seed=rank)
+        return legs
+
+    def compact(name, d):
+        if d is None:
+            return None
+        if name == "ctx_dec":
+            return {"full_ms": d["full_layer_ms"], "ssa_us": round(d["ssa_layer_ms"] * 1e3, 1),
+                    "layer_x": d["layer_speedup"], "stack4_x": d["stack_speedup"],
+                    "full_frac": d["full_layer_roofline"]["frac"]}
+        if name == "ctx_pre":
+            return {"full_ms": d["full_layer_ms"], "ssa_ms": d["ssa_layer_ms"],
+                    "layer_x": d["layer_speedup"], "pair_x": d["zigzag_pair_speedup"]}
+        if name.startswith("bwd"):
+            return {"tflops": d["value"], "frac": d["roofline"]["frac"], "ms": d["ms_per_step"]}
+        return {"gbs": d["value"], "frac": d["roofline"]["frac"], "us": d["us_per_step"]}
+
+    if args.no_prefill:
+        legs = decode_legs()
         if rank == 0:
-            print(json.dumps({"metric": METRIC, "decode": decode, "decode_selected": selected,
-                              "decode_mtp": mtp, "decode_fp8": dfp8, "decode_context": ctx}),
+            print(json.dumps({"metric": METRIC, **legs}), file=sys.stderr, flush=True)
+            print(json.dumps({"metric": METRIC,
+                              "configs": {k: compact(k, v) for k, v in legs.items()}}),
                   flush=True)
         if dist:
             torch.distributed.destroy_process_group()
         return
 
-    w = make_prefill(args.config, "cuda", seed=rank)
-    total_ms, per, clocks = time_prefill(w, args.steps, args.warmup, dist)
-    max_ms = max_over_ranks(total_ms)
-    ms_step = max_ms / args.steps
-    flops = 2 * (w["spec"].d_qk + w["spec"].d_v) * w["pairs"]
-    value = job_throughput(world, flops, args.steps, max_ms) / 1e12
-    avg_launch_ms = sum(per) / len(per)
-    achieved = flops / (avg_launch_ms * 1e-3) / 1e12
+    # ---- headline prefill workload
+    w, head_entry, t = prefill_leg(args.config, args.steps, args.warmup, peaks, dist, world, rank)
     e2e_ms, h2d, d2h = e2e_prefill(w, args.e2e_steps)
-    e2e_val = world * flops / (e2e_ms * 1e-3) / 1e12  # every rank runs the same e2e loop
-
-    backward = None if args.no_backward else backward_bench(w, max(3, args.steps // 5),
-                                                              args.warmup, peaks, world)
-    w_desc, w_tokens = w["desc"], w["tokens"]
-    decode = selected = mtp = ctx = pctx = dfp8 = None
+    e2e_val = world * t["flops"] / (e2e_ms * 1e-3) / 1e12  # every rank runs the same e2e loop
+    w_desc, w_spec = w["desc"], w["spec"]
+    detail = {"headline": {"workload": w_desc, **head_entry,
+                           "e2e_ms": round(e2e_ms, 3), "clocks": t["clocks"]}}
+    configs = {}
+    backward = None
+    if not args.no_backward and w_spec.d_qk == w_spec.d_v:
+        backward = backward_bench(w, max(3, args.steps // 4), args.warmup, peaks, world)
     del w
     torch.cuda.empty_cache()
+
+    # ---- the other prefill workloads (each its own timed region, same timing rules)
+    if not args.no_other_prefill:
+        for other in ("mha", "varlen", "mla"):
+            if other == args.config:
+                continue
+            w2, entry, _ = prefill_leg(other, args.steps, args.warmup, peaks, dist, world, rank)
+            configs[other] = entry
+            detail[other] = {"workload": w2["desc"]["workload"], **entry}
+            if other == "mha" and not args.no_backward and backward is None:
+                backward = backward_bench(w2, max(3, args.steps // 4), args.warmup, peaks, world)
+            del w2
+            torch.cuda.empty_cache()
+    if backward is not None:
+        configs["bwd_mha" if "L=32768" in backward["workload"] else "bwd"] = \
+            compact("bwd", backward)
+        detail["backward"] = backward
     if args.prefill_context:
         pctx = prefill_context_bench(peaks, args.prefill_context, world=world, seed=rank)
+        configs["ctx_pre"] = compact("ctx_pre", pctx)
+        detail["ctx_pre"] = pctx
     if not args.no_decode:
-        decode = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
-                              len_hi=args.decode_len_hi, world=world)
-        if args.decode_extra:
-            selected = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
-                                    len_hi=args.decode_len_hi, world=world,
-                                    n_extra=args.decode_extra)
-        if args.decode_mtp > 1:
-            mtp = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
-                               len_hi=args.decode_len_hi, world=world, q_len=args.decode_mtp)
-        if args.decode_fp8:
-            dfp8 = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
-                                len_hi=args.decode_len_hi, world=world, fp8=True)
-        if args.decode_context:
-            ctx = context_bench(peaks, args.decode_context, world=world, seed=rank)
+        for k, v in decode_legs().items():
+            configs[k] = compact(k, v)
+            detail[k] = v
 
     if rank != 0:
         if dist:
@@ -812,45 +855,35 @@ def main():
     if not args.no_cpu_baseline and world == 1:
         fl, dt, n, threads, desc = oracle_sample(args.config, args.cpu_budget_s)
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-               "sample": desc + f", {dt:.1f} s"}
+               "sample": f"{n} random rows of the {args.config} workload, float64, {dt:.1f} s"}
+        detail["cpu_baseline"] = {**cpu, "sample": desc + f", {dt:.1f} s"}
     kname = "ssa_prefill_kernel"
-    # A kernel timed back to back for more than ~0.1 s runs under the power
-    # cap: compare it with the sustained GEMM figure, a short burst with the
-    # burst figure.
-    sustained = max_ms > 100.0
-    peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
-    peak_note = (" (sustained bf16 GEMM: the timed region is %.0f ms of back-to-back launches)"
-                 if sustained else " (burst bf16 GEMM: the timed region is %.0f ms)") % max_ms
-    wl = {"mha": "mha", "tiny": "tiny", "mla": "mla", "varlen": "varlen"}[args.config]
+    peak = peaks["bf16_tflops"]
+    clocks = t["clocks"]
     line = {
-        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "metric": METRIC, "value": round(t["value"], 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(t["max_ms"] / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1) bf16, per-rank seed)",
-        "config": {**w_desc, "n_sink": 1, "n_local": 7, "block": 128,
-                   "parallelism": f"{world} independent replicas (weak scaling, no data-path collective)",
-                   "l2": "inputs larger than L2 (q, k, v re-read from HBM every step)"},
-        "tokens_per_s": round(job_throughput(world, w_tokens, args.steps, max_ms), 1),
-        "useful_tflop_per_step": round(flops / 1e12, 4),
-        "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
-                     "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4),
-                     "traffic": traffic_lookup(kname, wl), "peak_source": peaks["source"] +
-                     peak_note,
-                     "kernel": kname, "avg_launch_ms": round(avg_launch_ms, 4)},
+        "data": "synthetic (seeded N(0,1) bf16)",
+        "config": {"workload": w_desc["workload"],
+                   "parallelism": f"{world} independent replica(s), no data-path collective",
+                   "l2": "inputs larger than L2"},
+        "tokens_per_s": round(t["tok_s"], 1),
+        "roofline": {"bound": "tensor", "achieved": round(t["achieved"], 1), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(t["achieved"] / peak, 4),
+                     "frac_sustained": round(t["achieved"] / peaks["bf16_tflops_sustained"], 4),
+                     "traffic": traffic_lookup(kname, args.config), "kernel": kname,
+                     "avg_launch_ms": round(t["avg_launch_ms"], 4),
+                     "peak_source": peaks["source"] + " bf16 burst"},
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_val, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)},
-        "clocks": clocks,
+        "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
         "gpu_launches": args.steps,
-        "backward": backward,
-        "decode": decode,
-        "decode_selected": selected,
-        "decode_mtp": mtp,
-        "decode_fp8": dfp8,
-        "decode_context": ctx,
-        "prefill_context": pctx,
+        "configs": configs,
     }
+    print(json.dumps(detail), file=sys.stderr, flush=True)
     print(json.dumps(line), flush=True)
     if dist:
         torch.distributed.destroy_process_group()

@@ -479,6 +479,7 @@ __global__ void __launch_bounds__(320, 1)
     const float* ksc = ksl + 256;
     const uint32_t xp = bar(Lay::B_XP + wg);
     uint32_t xp_uses = 0;
+    bool done = false;  // this split's LSE slot was written with its result
     do {
       if constexpr (FP8) {
         // this page's token scales, then its K boxes as they land
@@ -663,7 +664,12 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       if (ok && valid && wg == 0) p.lse_part[cta * 128 + h] = (m + __log2f(l)) * kLn2;
+      done = ok;
     } while (false);
+    // A wait that gave up leaves this split's partial O unfinished: mark the
+    // slot NaN, so that the merge writes NaN for these heads rather than mix
+    // in what an earlier call left in the workspace.
+    if (!done && wg == 0) p.lse_part[cta * 128 + h] = __int_as_float(0x7fc00000);
   }
 
   __syncwarp();
@@ -684,7 +690,8 @@ __global__ void __launch_bounds__(320, 1)
 // not fit in the register file and ran a second wave).  Launched as a
 // programmatic dependent of the split kernel; it waits for the split
 // kernel's results before reading.  Splits whose LSE is -inf are empty and
-// contribute nothing (their partial O is never read into the sum).
+// contribute nothing (their partial O is never read into the sum); a NaN LSE
+// marks a split that gave up on a wait, and makes the head's O and LSE NaN.
 constexpr int kMergeHeads = 8;
 constexpr int kMergeGroups = 2;  // 8-column groups per thread
 constexpr int kMergeThreads = (kDecodeDv / 8 / kMergeGroups) * kMergeHeads;  // 256
@@ -716,6 +723,7 @@ __global__ void __launch_bounds__(kMergeThreads, 4)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[q][e] = 0.f;
   float denom = 0.f;
+  bool poisoned = false;  // a split gave up (its LSE slot is NaN)
   for (int s0 = 0; s0 < n; s0 += kMergeBatch) {
     float ls[kMergeBatch];
     uint4 raw[kMergeBatch][kMergeGroups];
@@ -731,7 +739,10 @@ __global__ void __launch_bounds__(kMergeThreads, 4)
     }
     float bmax = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < kMergeBatch; ++j) bmax = fmaxf(bmax, ls[j]);
+    for (int j = 0; j < kMergeBatch; ++j) {
+      poisoned |= ls[j] != ls[j];
+      bmax = fmaxf(bmax, ls[j]);  // fmaxf skips a NaN operand
+    }
     if (bmax == -INFINITY) continue;  // only empty splits in this batch
     if (bmax > lmax) {
       const float r = __expf(lmax - bmax);  // 0 while nothing is summed yet
@@ -744,7 +755,8 @@ __global__ void __launch_bounds__(kMergeThreads, 4)
     }
 #pragma unroll
     for (int j = 0; j < kMergeBatch; ++j) {
-      if (ls[j] == -INFINITY) continue;  // empty split: its partial O was never written
+      // empty split (its partial O was never written) or one that gave up
+      if (ls[j] == -INFINITY || ls[j] != ls[j]) continue;
       const float wgt = __expf(ls[j] - lmax);
       denom += wgt;
 #pragma unroll
@@ -759,7 +771,7 @@ __global__ void __launch_bounds__(kMergeThreads, 4)
       }
     }
   }
-  const float inv = denom > 0.f ? 1.f / denom : 0.f;
+  const float inv = poisoned ? __int_as_float(0x7fc00000) : (denom > 0.f ? 1.f / denom : 0.f);
   uint4* orow = reinterpret_cast<uint4*>(p.o + ((size_t)b * p.H_q + h) * kDecodeDv);
 #pragma unroll
   for (int q = 0; q < kMergeGroups; ++q) {
@@ -770,7 +782,9 @@ __global__ void __launch_bounds__(kMergeThreads, 4)
     pk.w = pack_bf16x2(acc[q][6] * inv, acc[q][7] * inv);
     orow[gp + q * kGroupStride] = pk;
   }
-  if (gp == 0) p.lse[(size_t)b * p.H_q + h] = denom > 0.f ? lmax + __logf(denom) : -INFINITY;
+  if (gp == 0)
+    p.lse[(size_t)b * p.H_q + h] = poisoned ? __int_as_float(0x7fc00000)
+                                   : denom > 0.f ? lmax + __logf(denom) : -INFINITY;
 }
 
 }  // namespace loza

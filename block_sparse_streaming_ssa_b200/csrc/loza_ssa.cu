@@ -269,6 +269,37 @@ __global__ void debug_decode_pages_kernel(loza::DecodeParams p, int* pages, int*
   }
 }
 
+// One warp; thread 0 waits on an mbarrier that nothing arrives on, through
+// the pipelines' bounded wait with a limit of timeout_ns, then the other 31
+// threads wait on it too and must give up on the abort flag thread 0 set.
+// result[0] = 1 if thread 0's wait gave up, result[1] = how many of the
+// others' waits gave up.
+__global__ void debug_wait_timeout_kernel(unsigned long long timeout_ns, int* result) {
+  __shared__ __align__(8) unsigned long long bar_storage;
+  __shared__ int abort_storage;
+  const uint32_t bar = loza::smem_u32(&bar_storage);
+  volatile int* abort_flag = &abort_storage;
+  if (threadIdx.x == 0) {
+    loza::mbar_init(bar, 1);
+    *abort_flag = 0;
+    loza::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool ok = loza::mbar_wait_for(bar, 0, abort_flag, &loza::g_loza_status,
+                                        LOZA_SSA_DEV_WAIT_TIMEOUT, timeout_ns);
+    result[0] = ok ? 0 : 1;
+  }
+  __syncthreads();
+  if (threadIdx.x > 0) {
+    // ten times the limit, so that only the abort flag ends these waits in time
+    const bool ok = loza::mbar_wait_for(bar, 0, abort_flag, &loza::g_loza_status,
+                                        LOZA_SSA_DEV_WAIT_TIMEOUT, 10 * timeout_ns);
+    const unsigned gave_up = __ballot_sync(0xfffffffeu, !ok);
+    if (threadIdx.x == 1) result[1] = __popc(gave_up);
+  }
+}
+
 // Scratch for loza_ssa_decode_static_scratch: the decode workspace of up to
 // LOZA_SSA_STATIC_SCRATCH_SLOTS split slots (fp16 partial O, 256-byte aligned,
 // then fp32 partial LSE), resident on every device that loads the library.
@@ -719,15 +750,12 @@ size_t loza_ssa_decode_mtp_workspace_size(int B, int q_len, int H_q, int d_v, in
 
 namespace {
 
-// loza_ssa_decode with an optional per-sequence list of extra pages
-// (extra_pages == nullptr and max_extra == 0: the plain window), q_len
-// query tokens per sequence (q_len == 1: one) and an FP8 cache (kv_scale !=
-// nullptr: paged_kv holds e4m3 codes).  B counts sequences.
-int decode_impl(const void* q, const void* paged_kv, const int* page_table, const int* seq_lens,
-                const int* extra_pages, int max_extra, int q_len, void* o, float* lse, int B,
-                int H_q, int d_qk, int d_v, int page_size, int max_pages, int n_pages, int n_sink,
-                int n_local, float scale, void* workspace, size_t workspace_bytes,
-                loza_ssa_stream_t stream, const float* kv_scale = nullptr) {
+// The argument checks of decode_impl up to (not including) the workspace.
+int decode_check_args(const void* q, const void* paged_kv, const int* page_table,
+                      const int* seq_lens, const int* extra_pages, int max_extra, int q_len,
+                      const void* o, const float* lse, int B, int H_q, int d_qk, int d_v,
+                      int page_size, int max_pages, int n_pages, int n_sink, int n_local,
+                      float scale, const float* kv_scale) {
   if (!q || !paged_kv || !page_table || !seq_lens || !o || !lse) return LOZA_SSA_ERR_NULL;
   if (max_extra < 0 || q_len < 1) return LOZA_SSA_ERR_SHAPE;
   if (q_len > 1 && max_extra > 0) return LOZA_SSA_ERR_SHAPE;  // no public call combines them
@@ -746,12 +774,29 @@ int decode_impl(const void* q, const void* paged_kv, const int* page_table, cons
   if (!aligned(q, 16) || !aligned(paged_kv, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
       !aligned(page_table, 4) || !aligned(seq_lens, 4) || !aligned(kv_scale, 4))
     return LOZA_SSA_ERR_ALIGN;
+  return LOZA_SSA_OK;
+}
+
+// loza_ssa_decode with an optional per-sequence list of extra pages
+// (extra_pages == nullptr and max_extra == 0: the plain window), q_len
+// query tokens per sequence (q_len == 1: one) and an FP8 cache (kv_scale !=
+// nullptr: paged_kv holds e4m3 codes).  B counts sequences.
+int decode_impl(const void* q, const void* paged_kv, const int* page_table, const int* seq_lens,
+                const int* extra_pages, int max_extra, int q_len, void* o, float* lse, int B,
+                int H_q, int d_qk, int d_v, int page_size, int max_pages, int n_pages, int n_sink,
+                int n_local, float scale, void* workspace, size_t workspace_bytes,
+                loza_ssa_stream_t stream, const float* kv_scale = nullptr) {
+  int rc = decode_check_args(q, paged_kv, page_table, seq_lens, extra_pages, max_extra, q_len, o,
+                             lse, B, H_q, d_qk, d_v, page_size, max_pages, n_pages, n_sink,
+                             n_local, scale, kv_scale);
+  if (rc != LOZA_SSA_OK) return rc;
+  B *= q_len;  // from here on B counts rows: (sequence, query token) pairs
   const size_t need =
       loza_ssa_decode_selected_workspace_size(B, H_q, d_v, n_sink, n_local, max_extra);
   if (!workspace || workspace_bytes < need) return LOZA_SSA_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return LOZA_SSA_ERR_ALIGN;
   DeviceInfo dev;
-  int rc = device_info(dev);
+  rc = device_info(dev);
   if (rc != LOZA_SSA_OK) return rc;
 
   const int n_split = decode_splits(n_sink, n_local, max_extra);
@@ -901,33 +946,33 @@ int loza_ssa_decode_static_scratch(const void* q, const void* paged_kv, const in
                                    int n_sink, int n_local, float scale,
                                    loza_ssa_stream_t stream) {
   // Same checks and kernels as loza_ssa_decode; only the workspace differs.
-  if (B >= 1 && H_q >= 1 && n_sink >= 0 && n_local >= 1 &&
-      n_sink + n_local <= kMaxDecodeWindow) {
-    const long long slots =
-        (long long)B * ((H_q + 127) / 128) * decode_splits(n_sink, n_local);
-    if (slots > LOZA_SSA_STATIC_SCRATCH_SLOTS) {
-      std::snprintf(g_last_error, sizeof g_last_error,
-                    "decode_static_scratch: B * ceil(H_q/128) * ceil((n_sink + n_local)/2) = %lld split "
-                    "slots, the built-in scratch holds %d",
-                    slots, LOZA_SSA_STATIC_SCRATCH_SLOTS);
-      return LOZA_SSA_ERR_SCRATCH_LIMIT;
-    }
+  // The argument checks come first, so that a bad call gets the code
+  // loza_ssa_decode would give it; the scratch limit only applies to a
+  // valid one.
+  int rc = decode_check_args(q, paged_kv, page_table, seq_lens, nullptr, 0, 1, o, lse, B, H_q,
+                             d_qk, d_v, page_size, max_pages, n_pages, n_sink, n_local, scale,
+                             nullptr);
+  if (rc != LOZA_SSA_OK) return rc;
+  const long long slots = (long long)B * ((H_q + 127) / 128) * decode_splits(n_sink, n_local);
+  if (slots > LOZA_SSA_STATIC_SCRATCH_SLOTS) {
+    std::snprintf(g_last_error, sizeof g_last_error,
+                  "decode_static_scratch: B * ceil(H_q/128) * ceil((n_sink + n_local)/2) = %lld split "
+                  "slots, the built-in scratch holds %d",
+                  slots, LOZA_SSA_STATIC_SCRATCH_SLOTS);
+    return LOZA_SSA_ERR_SCRATCH_LIMIT;
   }
   const size_t need = loza_ssa_decode_workspace_size(B, H_q, d_v, n_sink, n_local);
-  void* scratch = nullptr;
-  if (need > 0) {  // invalid arguments are left for loza_ssa_decode to report
-    if (need > sizeof(g_decode_scratch)) {
-      std::snprintf(g_last_error, sizeof g_last_error,
-                    "decode_static_scratch: needs %zu scratch bytes, the built-in scratch holds %zu",
-                    need, sizeof(g_decode_scratch));
-      return LOZA_SSA_ERR_SCRATCH_LIMIT;
-    }
-    const int rc = static_scratch_address(&scratch);
-    if (rc != LOZA_SSA_OK) return rc;
+  if (need == 0 || need > sizeof(g_decode_scratch)) {
+    std::snprintf(g_last_error, sizeof g_last_error,
+                  "decode_static_scratch: needs %zu scratch bytes, the built-in scratch holds %zu",
+                  need, sizeof(g_decode_scratch));
+    return LOZA_SSA_ERR_SCRATCH_LIMIT;
   }
+  void* scratch = nullptr;
+  if ((rc = static_scratch_address(&scratch)) != LOZA_SSA_OK) return rc;
   return loza_ssa_decode(q, paged_kv, page_table, seq_lens, o, lse, B, H_q, d_qk, d_v, page_size,
                          max_pages, n_pages, n_sink, n_local, scale, scratch,
-                         scratch ? sizeof(g_decode_scratch) : 0, stream);
+                         sizeof(g_decode_scratch), stream);
 }
 
 int loza_ssa_get_last_device_status(loza_ssa_stream_t stream) {
@@ -951,6 +996,16 @@ int loza_ssa_debug_enumerate_tiles(int n_qblocks, int n_sink, int n_local, int* 
       n_qblocks, n_sink, n_local, tiles, counts, max_tiles);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? LOZA_SSA_OK : cuda_fail(e, "debug tiles launch");
+}
+
+int loza_ssa_debug_wait_timeout(int timeout_us, int* result, loza_ssa_stream_t stream) {
+  if (!result) return LOZA_SSA_ERR_NULL;
+  if (timeout_us < 1 || timeout_us > 100000) return LOZA_SSA_ERR_SHAPE;
+  if (!aligned(result, 4)) return LOZA_SSA_ERR_ALIGN;
+  debug_wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      1000ull * (unsigned long long)timeout_us, result);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? LOZA_SSA_OK : cuda_fail(e, "debug wait-timeout launch");
 }
 
 int loza_ssa_debug_decode_pages(const int* page_table, const int* seq_lens, int B, int max_pages,

@@ -65,10 +65,13 @@ __device__ __forceinline__ uint32_t mbar_try_wait(uint32_t bar, uint32_t parity)
   return ok;
 }
 
-// Wait until the phase with the given parity has completed.  Returns false if
-// the CTA is aborting (flag already set, or this wait timed out and set it).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status, int timeout_bit) {
+// Wait until the phase with the given parity has completed, for at most
+// timeout_ns of wall time (the global timer, so time the GPU spends on another
+// context counts too).  Returns false if the CTA is aborting (flag already
+// set, or this wait timed out and set it).
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity,
+                                              volatile int* abort_flag, int* status,
+                                              int timeout_bit, unsigned long long timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   while (true) {
@@ -76,12 +79,18 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+    if (global_timer_ns() - t0 > timeout_ns) {
       *abort_flag = 1;
       atomicOr(status, timeout_bit);
       return false;
     }
   }
+}
+
+// The pipelines' wait: mbar_wait_for with the library's limit.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          int* status, int timeout_bit) {
+  return mbar_wait_for(bar, parity, abort_flag, status, timeout_bit, kWaitTimeoutNs);
 }
 
 // Teardown wait: ignores the abort flag (used to let copies / MMAs already in

@@ -107,6 +107,8 @@ def lib() -> ctypes.CDLL:
         L.loza_ssa_debug_decode_pages.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp, vp,
                                                   i32, vp]
         L.loza_ssa_debug_decode_pages.restype = i32
+        L.loza_ssa_debug_wait_timeout.argtypes = [i32, vp, vp]
+        L.loza_ssa_debug_wait_timeout.restype = i32
         L.loza_ssa_decode_static_scratch.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
                                                      i32, i32, i32, i32, i32, f32, vp]
         L.loza_ssa_decode_static_scratch.restype = i32
@@ -571,3 +573,12 @@ def loza_ssa_debug_decode_pages(page_table, seq_lens, n_pages, page_size=128, n_
         _ptr(page_table), _ptr(seq_lens), B, max_pages, n_pages, page_size, n_sink, n_local,
         _ptr(pages), _ptr(counts), max_tiles, _stream(stream)))
     return pages, counts
+
+
+def loza_ssa_debug_wait_timeout(timeout_us, device="cuda", stream=None):
+    """The kernels' bounded wait on a barrier nothing arrives on, with a limit of
+    timeout_us: returns the device int32[2] result (1 if the waiting thread gave
+    up, and how many of the 31 other threads gave up on its abort flag)."""
+    result = torch.full((2,), -1, dtype=torch.int32, device=device)
+    _check(lib().loza_ssa_debug_wait_timeout(int(timeout_us), _ptr(result), _stream(stream)))
+    return result

@@ -355,6 +355,23 @@ int loza_ssa_debug_enumerate_tiles(int n_qblocks, int n_sink, int n_local, int* 
                                    int* counts, int max_tiles, loza_ssa_stream_t stream);
 
 /*
+ * Debug: exercise the kernels' bounded pipeline wait.  One warp is launched;
+ * thread 0 waits on an mbarrier that nothing ever arrives on, through the same
+ * wait routine every pipeline of the library uses, but with a limit of
+ * timeout_us microseconds (1 .. 100000) instead of the library's 2 s.  When
+ * the limit passes it sets the CTA's abort flag and LOZA_SSA_DEV_WAIT_TIMEOUT
+ * in the device status word and returns; the other 31 threads then wait on
+ * the same barrier with ten times the limit and must give up on the abort
+ * flag.  result (device int[2]): result[0] = 1 if thread 0's wait gave up,
+ * result[1] = how many of the other threads' waits gave up (31 expected).
+ * The limit is wall-clock time (the GPU's global timer), so time the GPU
+ * spends on other contexts counts against it: under heavy time-slicing the
+ * library's 2 s limit could in principle be reached by a wait that would
+ * have completed, which is reported the same way.
+ */
+int loza_ssa_debug_wait_timeout(int timeout_us, int* result, loza_ssa_stream_t stream);
+
+/*
  * Debug: run the decode kernel's page selection on the device.  For every
  * sequence b writes the PHYSICAL pages the decode window reads (logical order)
  * to pages[b*max_tiles ...] and their number to counts[b]; entries it would
@@ -389,7 +406,16 @@ int loza_ssa_debug_decode_pages(const int* page_table, const int* seq_lens, int 
  * whose kernels overlap on the GPU (for example on two streams at once) race
  * and corrupt each other's results, so order them on one stream.  The array
  * keeps the last call's contents; nothing in it needs to start at zero,
- * because every slot a call reads is first written by the same call.
+ * because every slot a call reads is first written by the same call: a split
+ * whose pipeline wait gave up writes NaN to its slot's LSE (and sets
+ * LOZA_SSA_DEV_WAIT_TIMEOUT), so that the heads it covers come out NaN rather
+ * than mixed with an earlier call's partials.
+ * The array's device address is looked up once per device and kept for the
+ * life of the process; it does not survive cudaDeviceReset() or a release and
+ * re-creation of the device's primary context, after which this entry point
+ * must not be called again in the same process.
+ * Argument errors are reported as by loza_ssa_decode (the same codes, checked
+ * first); LOZA_SSA_ERR_SCRATCH_LIMIT only for an otherwise valid call.
  * The library calls no allocation routine for this entry point.
  */
 #define LOZA_SSA_STATIC_SCRATCH_SLOTS 128

@@ -326,3 +326,35 @@ def test_debug_argument_errors(L):
     assert L.loza_ssa_debug_enumerate_tiles(4, 1, 0, vp(0x1000), vp(0x1000), 8, None) == -5
     assert L.loza_ssa_debug_decode_pages(vp(0x1000), vp(0x1000), 2, 8, 8, 64, 1, 7, vp(0x1000),
                                          vp(0x1000), 8, None) == -4
+
+
+def test_static_scratch_limit_and_argument_order(L):
+    """The workspace-free decode rejects a call that needs more split slots than
+    its built-in array holds before touching CUDA, and reports argument errors
+    with loza_ssa_decode's codes first (dummy non-null pointers; nothing runs)."""
+    vp = ctypes.c_void_p
+    a = vp(0x1000)
+
+    def call(B=2, Hq=128, dqk=576, dv=512, ps=128, ns=1, nl=7, q=a):
+        return L.loza_ssa_decode_static_scratch(q, a, a, a, a, a, B, Hq, dqk, dv, ps, 16, 64,
+                                                ns, nl, ctypes.c_float(0.04), None)
+    # 33 sequences x 4 splits = 132 slots > 128
+    assert call(B=33) == -9                       # LOZA_SSA_ERR_SCRATCH_LIMIT
+    assert call(B=2, Hq=129 * 128) == -9          # 2 x 129 head groups x 4 splits
+    assert call(B=1, nl=300) == -9                # 1 x ceil(301 / 2) splits
+    # over the limit and invalid as well: the argument error wins
+    assert call(B=33, dv=256) == -3               # LOZA_SSA_ERR_HEAD_DIM
+    assert call(B=33, dqk=512) == -3
+    assert call(B=33, ps=64) == -4                # LOZA_SSA_ERR_BLOCK
+    assert call(B=33, nl=0) == -5                 # LOZA_SSA_ERR_WINDOW
+    assert call(B=33, q=None) == -1               # LOZA_SSA_ERR_NULL
+    assert call(B=33, q=vp(0x1004)) == -6         # LOZA_SSA_ERR_ALIGN
+    assert call(B=0) == -2                        # LOZA_SSA_ERR_SHAPE
+
+
+def test_debug_wait_timeout_argument_errors(L):
+    vp = ctypes.c_void_p
+    assert L.loza_ssa_debug_wait_timeout(1000, None, None) == -1
+    assert L.loza_ssa_debug_wait_timeout(0, vp(0x1000), None) == -2
+    assert L.loza_ssa_debug_wait_timeout(100001, vp(0x1000), None) == -2
+    assert L.loza_ssa_debug_wait_timeout(1000, vp(0x1002), None) == -6

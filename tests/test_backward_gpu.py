@@ -129,3 +129,23 @@ def test_backward_varlen_one_sequence_is_dense_bitwise():
     torch.cuda.synchronize()
     for x, y in zip(a, b):
         assert torch.equal(x[0], y)
+
+
+def test_backward_full_size_heads():
+    """The benchmarked workload (B=1, H=32, L=32768, d=128, 0.5*N(0,1)): the whole
+    backward call on the GPU, so that key block 0's 256 query blocks run as 32
+    sink chunks through the partial-sum reduction; four heads compared in full
+    (every row of dq, dk, dv) with the oracle's float64 gradients."""
+    spec = synth.MHA
+    q, k, v = synth.prefill_spec_inputs(spec, seed=0, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(4242)
+    dout = torch.randn(v.shape, generator=g, device="cuda").to(torch.bfloat16)
+    o, lse = loza_ssa_prefill(q, k, v, scale=spec.scale)
+    dq, dk, dv = loza_ssa_prefill_bwd(q, k, v, o, lse, dout, scale=spec.scale)
+    torch.cuda.synchronize()
+    assert loza_ssa_get_last_device_status() == 0
+    heads = [0, 11, 22, 31]
+    hsel = torch.as_tensor(heads, device="cuda")
+    ref = orc.prefill_bwd(*(synth.bf16_bits(t[:, hsel]) for t in (q, k, v, dout)), blk=128,
+                          n_sink=1, n_local=7, scale=spec.scale)
+    check([t[:, hsel] for t in (dq, dk, dv)], ref, "mha 32K, heads 0/11/22/31")

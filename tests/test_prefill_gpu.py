@@ -9,7 +9,7 @@ from block_sparse_streaming_ssa_b200 import synth
 from block_sparse_streaming_ssa_b200.loza_ssa import (loza_ssa_get_last_device_status,
                                                       loza_ssa_prefill)
 from oracle import ssa_oracle as orc
-from tests.parity import assert_parity
+from tests.parity import LSE_MAX_ABS, O_MAX_ABS, O_REL_L2, assert_parity
 
 pytestmark = pytest.mark.gpu
 
@@ -150,6 +150,33 @@ def run_full_size_sampled(spec, heads, n_rows, seed):
     o_s = o[:, hsel].reshape(-1, spec.d_v)[r]
     lse_s = lse[:, hsel].reshape(-1)[r]
     return o_s, lse_s, o_ref, lse_ref
+
+
+def test_mha_full_size_every_row():
+    """B=1, H=32, L=32768, d=128, 0.5*N(0,1): the benchmark's launch, every row of
+    every head against the oracle (0.51 TFLOP of float64, computed four heads at
+    a time; the error measures are taken over the whole output)."""
+    spec = synth.MHA
+    q, k, v = synth.prefill_spec_inputs(spec, seed=0, device="cuda")
+    o, lse = loza_ssa_prefill(q, k, v, scale=spec.scale)
+    torch.cuda.synchronize()
+    assert loza_ssa_get_last_device_status() == 0
+    max_abs = lse_abs = 0.0
+    err2 = ref2 = 0.0
+    for h0 in range(0, spec.H, 4):
+        sub = [synth.bf16_bits(t[:, h0:h0 + 4]) for t in (q, k, v)]
+        o_ref, lse_ref = orc.prefill(*sub, 128, 1, 7, spec.scale)
+        got = o[:, h0:h0 + 4].float().cpu().numpy().astype(np.float64)
+        got_lse = lse[:, h0:h0 + 4].cpu().numpy().astype(np.float64)
+        assert np.isfinite(got).all() and np.isfinite(got_lse).all()
+        d = got - o_ref
+        max_abs = max(max_abs, float(np.abs(d).max()))
+        err2 += float((d * d).sum())
+        ref2 += float((o_ref * o_ref).sum())
+        lse_abs = max(lse_abs, float(np.abs(got_lse - lse_ref).max()))
+    rel = (err2 / ref2) ** 0.5
+    msg = f"mha every row: O max-abs {max_abs:.3e}, O rel-L2 {rel:.3e}, LSE max-abs {lse_abs:.3e}"
+    assert max_abs <= O_MAX_ABS and rel <= O_REL_L2 and lse_abs <= LSE_MAX_ABS, msg
 
 
 def test_mha_full_size_sampled():
