@@ -252,15 +252,16 @@ def time_prefill(w, steps, warmup, dist):
 def backward_bench(w, steps, warmup, peaks, world=1):
     """The prefill's backward (loza_ssa_prefill_bwd) on the same workload,
     with o and lse from the forward pass and a seeded random dO.  Useful FLOPs
-    follow the usual attention-backward count, 2.5x the forward: the five
-    products dP = dO V^T, dV += P^T dO, dQ += dS K, dK += dS^T Q and one
-    recomputation of S = Q K^T, each 2 d per unmasked (i, j) pair (the dK/dV
-    kernel recomputes S and dP a second time; that work is not counted)."""
+    follow the usual attention-backward count: the five products dP = dO V^T
+    (2 d_v per unmasked (i, j) pair), dV += P^T dO (2 d_v), dQ += dS K
+    (2 d_qk), dK += dS^T Q (2 d_qk) and one recomputation of S = Q K^T
+    (2 d_qk), i.e. 2.5x the forward when d_qk = d_v (the dK/dV kernel
+    recomputes S and dP a second time; that work is not counted)."""
     import torch
     from block_sparse_streaming_ssa_b200.loza_ssa import (loza_ssa_prefill_bwd,
                                                           loza_ssa_prefill_varlen_bwd)
     sp = w["spec"]
-    if sp.d_qk != sp.d_v or sp.d_qk not in (64, 128):
+    if (sp.d_qk, sp.d_v) not in ((64, 64), (128, 128), (192, 128)):
         return None
     o, lse = prefill_call(w)
     g = torch.Generator(device="cuda").manual_seed(4242)
@@ -284,7 +285,7 @@ def backward_bench(w, steps, warmup, peaks, world=1):
     t1.record()
     torch.cuda.synchronize()
     ms = max_over_ranks(t0.elapsed_time(t1) / steps)
-    flops = 2.5 * 2 * (sp.d_qk + sp.d_v) * w["pairs"]
+    flops = 2 * (3 * sp.d_qk + 2 * sp.d_v) * w["pairs"]
     tf = flops / (ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops"]
     return {"workload": w["desc"]["workload"] + ", backward (dQ, dK, dV)",
@@ -677,7 +678,7 @@ def prefill_leg(config, steps, warmup, peaks, dist, world, rank):
     achieved = flops / (avg_launch_ms * 1e-3) / 1e12
     value = job_throughput(world, flops, steps, max_ms) / 1e12
     tok_s = job_throughput(world, w["tokens"], steps, max_ms)
-    entry = {"tflops": round(value, 1), "frac": round(achieved / peaks["bf16_tflops"], 4),
+    entry = {"tflops": round(value, 1), "frac": round(achieved / peaks["bf16_tflops"], 3),
              "ms": round(max_ms / steps, 4), "mtok_s": round(tok_s / 1e6, 2)}
     return w, entry, dict(total_ms=total_ms, max_ms=max_ms, flops=flops, achieved=achieved,
                           value=value, tok_s=tok_s, avg_launch_ms=avg_launch_ms, clocks=clocks)
@@ -786,15 +787,16 @@ def main():
         if d is None:
             return None
         if name == "ctx_dec":
-            return {"full_ms": d["full_layer_ms"], "ssa_us": round(d["ssa_layer_ms"] * 1e3, 1),
-                    "layer_x": d["layer_speedup"], "stack4_x": d["stack_speedup"],
-                    "full_frac": d["full_layer_roofline"]["frac"]}
+            return {"full_ms": round(d["full_layer_ms"], 3),
+                    "ssa_us": round(d["ssa_layer_ms"] * 1e3, 1), "stack4_x": d["stack_speedup"],
+                    "full_frac": round(d["full_layer_roofline"]["frac"], 3)}
         if name == "ctx_pre":
-            return {"full_ms": d["full_layer_ms"], "ssa_ms": d["ssa_layer_ms"],
-                    "layer_x": d["layer_speedup"], "pair_x": d["zigzag_pair_speedup"]}
+            return {"full_ms": round(d["full_layer_ms"], 1), "pair_x": d["zigzag_pair_speedup"]}
         if name.startswith("bwd"):
-            return {"tflops": d["value"], "frac": d["roofline"]["frac"], "ms": d["ms_per_step"]}
-        return {"gbs": d["value"], "frac": d["roofline"]["frac"], "us": d["us_per_step"]}
+            return {"tflops": round(d["value"], 1), "frac": round(d["roofline"]["frac"], 3),
+                    "ms": round(d["ms_per_step"], 3)}
+        return {"gbs": round(d["value"]), "frac": round(d["roofline"]["frac"], 3),
+                "us": round(d["us_per_step"], 1)}
 
     if args.no_prefill:
         legs = decode_legs()
@@ -815,9 +817,11 @@ def main():
     detail = {"headline": {"workload": w_desc, **head_entry,
                            "e2e_ms": round(e2e_ms, 3), "clocks": t["clocks"]}}
     configs = {}
-    backward = None
-    if not args.no_backward and w_spec.d_qk == w_spec.d_v:
-        backward = backward_bench(w, max(3, args.steps // 4), args.warmup, peaks, world)
+    backwards = {}
+    if not args.no_backward:
+        b = backward_bench(w, max(3, args.steps // 4), args.warmup, peaks, world)
+        if b is not None:
+            backwards[f"bwd_{args.config}"] = b
     del w
     torch.cuda.empty_cache()
 
@@ -829,14 +833,14 @@ def main():
             w2, entry, _ = prefill_leg(other, args.steps, args.warmup, peaks, dist, world, rank)
             configs[other] = entry
             detail[other] = {"workload": w2["desc"]["workload"], **entry}
-            if other == "mha" and not args.no_backward and backward is None:
-                backward = backward_bench(w2, max(3, args.steps // 4), args.warmup, peaks, world)
+            if other == "mha" and not args.no_backward:
+                backwards["bwd_mha"] = backward_bench(w2, max(3, args.steps // 4), args.warmup,
+                                                      peaks, world)
             del w2
             torch.cuda.empty_cache()
-    if backward is not None:
-        configs["bwd_mha" if "L=32768" in backward["workload"] else "bwd"] = \
-            compact("bwd", backward)
-        detail["backward"] = backward
+    for name, b in backwards.items():
+        configs[name] = compact("bwd", b)
+        detail[name] = b
     if args.prefill_context:
         pctx = prefill_context_bench(peaks, args.prefill_context, world=world, seed=rank)
         configs["ctx_pre"] = compact("ctx_pre", pctx)
@@ -854,8 +858,8 @@ def main():
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         fl, dt, n, threads, desc = oracle_sample(args.config, args.cpu_budget_s)
-        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-               "sample": f"{n} random rows of the {args.config} workload, float64, {dt:.1f} s"}
+        cpu = {"value": round(fl / dt / 1e12, 5), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n} rows of {args.config}, f64, {dt:.0f} s"}
         detail["cpu_baseline"] = {**cpu, "sample": desc + f", {dt:.1f} s"}
     kname = "ssa_prefill_kernel"
     peak = peaks["bf16_tflops"]
@@ -865,24 +869,25 @@ def main():
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(t["max_ms"] / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1) bf16)",
-        "config": {"workload": w_desc["workload"],
-                   "parallelism": f"{world} independent replica(s), no data-path collective",
-                   "l2": "inputs larger than L2"},
-        "tokens_per_s": round(t["tok_s"], 1),
+        "data": "synthetic",
+        "config": {"workload": w_desc["workload"].replace(" bf16, 1 sink + 7 local blocks of 128",
+                                                          ", 1+7 blocks of 128"),
+                   "parallelism": "replicas", "l2": "inputs > L2"},
+        "tokens_per_s": round(t["tok_s"]),
         "roofline": {"bound": "tensor", "achieved": round(t["achieved"], 1), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(t["achieved"] / peak, 4),
-                     "frac_sustained": round(t["achieved"] / peaks["bf16_tflops_sustained"], 4),
-                     "traffic": traffic_lookup(kname, args.config), "kernel": kname,
-                     "avg_launch_ms": round(t["avg_launch_ms"], 4),
-                     "peak_source": peaks["source"] + " bf16 burst"},
+                     "traffic": traffic_lookup(kname, args.config),
+                     "peak_source": peaks["source"]},
         "cpu_baseline": cpu,
-        "e2e": {"value": round(e2e_val, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)},
+        "e2e": {"value": round(e2e_val, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
         "gpu_launches": args.steps,
         "configs": configs,
     }
+    detail["headline"]["roofline"] = {
+        **line["roofline"], "kernel": kname, "avg_launch_ms": round(t["avg_launch_ms"], 4),
+        "frac_of_sustained": round(t["achieved"] / peaks["bf16_tflops_sustained"], 4)}
     print(json.dumps(detail), file=sys.stderr, flush=True)
     print(json.dumps(line), flush=True)
     if dist:

@@ -1,5 +1,5 @@
-// backward.cuh -- gradients of the SSA prefill on sm_100a (dense layout,
-// d_qk = d_v = DIM in {64, 128}).
+// backward.cuh -- gradients of the SSA prefill on sm_100a, for (d_qk, d_v) in
+// {(64, 64), (128, 128), (192, 128)} (dense and packed layouts).
 //
 // For a loss with upstream gradient dO = dL/dO, differentiating the masked
 // softmax attention of "LoZA：ZigZag稀疏注意力机制" §2.1 over the SSA key sets
@@ -45,10 +45,10 @@ constexpr int kSinkChunk = 8;        // query blocks per sink work item
 struct BwdParams {
   const float* lse;        // [planes * plane_rows], natural log, from the forward pass
   const float* dsum;       // [planes * plane_rows], D_i
-  __nv_bfloat16* dq;       // [planes, plane_rows, DIM]
+  __nv_bfloat16* dq;       // [planes, plane_rows, d_qk]; dk likewise, dv [.., d_v]
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
-  float* part;             // sink partials: [sink slots][2][128][DIM] (dK then dV)
+  float* part;             // sink partials: [sink slots] x (dK [128][d_qk], dV [128][d_v])
   int L, planes, n_sink, n_local;
   int nb;                  // dense: query / key blocks per plane
   int sink_items;          // dense: sink work items per plane
@@ -239,7 +239,8 @@ __global__ void __launch_bounds__(1024) ssa_bwd_varlen_setup_kernel(const int* c
 
 // ---------------------------------------------------------------- D_i
 
-// D_i = dO_i . O_i for every row; DIM / 8 lanes share a row (16 bytes each).
+// D_i = dO_i . O_i for every row (DIM = d_v); DIM / 8 lanes share a row (16
+// bytes each).
 template <int DIM>
 __global__ void __launch_bounds__(256) ssa_bwd_preprocess_kernel(const __nv_bfloat16* o,
                                                                   const __nv_bfloat16* dout,
@@ -272,19 +273,23 @@ __global__ void __launch_bounds__(256) ssa_bwd_preprocess_kernel(const __nv_bflo
 
 // ------------------------------------------------------------------ dQ
 
-template <int DIM>
+template <int DQK, int DV>
 struct BwdDqLayout {
-  static constexpr int CH = DIM / 64;
-  static constexpr int CHUNK = 128 * 128;  // one swizzled [128 rows x 64 bf16] box
-  static constexpr int TILE = CH * CHUNK;  // [128 rows x DIM]
-  static constexpr int KST = 2, VST = 2;
+  static constexpr int QCH = DQK / 64, VCH = DV / 64;
+  static constexpr int CHUNK = 128 * 128;     // one swizzled [128 rows x 64 bf16] box
+  static constexpr int QTILE = QCH * CHUNK;   // [128 rows x d_qk]: Q, K
+  static constexpr int VTILE = VCH * CHUNK;   // [128 rows x d_v]: dO, V
+  static constexpr int KST = 2;
+  // two V stages where they fit in shared memory (not beside the d_qk = 192 tiles)
+  static constexpr int VST = 2 * QTILE + 3 * VTILE + KST * QTILE <= 220 * 1024 ? 2 : 1;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_DO = TILE;
-  static constexpr int OFF_K = 2 * TILE;
-  static constexpr int OFF_V = OFF_K + KST * TILE;
-  static constexpr int OFF_BAR = OFF_V + VST * TILE;
-  // TMEM columns
-  static constexpr int TM_S = 0, TM_DP = 128, TM_DS = 256, TM_DQ = 384;
+  static constexpr int OFF_DO = QTILE;
+  static constexpr int OFF_K = QTILE + VTILE;
+  static constexpr int OFF_V = OFF_K + KST * QTILE;
+  static constexpr int OFF_BAR = OFF_V + VST * VTILE;
+  // TMEM columns: S, dP, dS (bf16 pairs, 64 columns), dQ (d_qk columns) at the end
+  static constexpr int TM_S = 0, TM_DP = 128, TM_DS = 256, TM_DQ = 512 - DQK;
+  static_assert(TM_DS + 64 <= TM_DQ, "TMEM");
   // barriers
   static constexpr int B_QD_FULL = 0, B_QD_EMPTY = 1;
   static constexpr int B_K_FULL = 2, B_K_EMPTY = B_K_FULL + KST;
@@ -302,13 +307,13 @@ struct BwdDqLayout {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
-template <int DIM>
+template <int DQK, int DV>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     ssa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v,
                       const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
-  using Lay = BwdDqLayout<DIM>;
+  using Lay = BwdDqLayout<DQK, DV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -370,15 +375,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(bar(Lay::B_QD_FULL), 2 * Lay::TILE);
+        mbar_arrive_expect_tx(bar(Lay::B_QD_FULL), Lay::QTILE + Lay::VTILE);
         ++qd_issued;
 #pragma unroll
-        for (int c = 0; c < Lay::CH; ++c) {
+        for (int c = 0; c < Lay::QCH; ++c)
           tma_load_3d(sb + Lay::OFF_Q + c * Lay::CHUNK, &tm_q, bar(Lay::B_QD_FULL), c * 64,
                       w.seq_start + w.qb * 128, w.plane);
+#pragma unroll
+        for (int c = 0; c < Lay::VCH; ++c)
           tma_load_3d(sb + Lay::OFF_DO + c * Lay::CHUNK, &tm_do, bar(Lay::B_QD_FULL), c * 64,
                       w.seq_start + w.qb * 128, w.plane);
-        }
         for (int t = 0; t < tr.count; ++t, ++g) {
           const int row = w.seq_start + tile_block(tr, t) * 128;
           const int st = g % Lay::KST, use = g / Lay::KST;
@@ -387,11 +393,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(bar(Lay::B_K_FULL + st), Lay::TILE);
+          mbar_arrive_expect_tx(bar(Lay::B_K_FULL + st), Lay::QTILE);
           ++k_issued[st];
 #pragma unroll
-          for (int c = 0; c < Lay::CH; ++c)
-            tma_load_3d(sb + Lay::OFF_K + st * Lay::TILE + c * Lay::CHUNK, &tm_k,
+          for (int c = 0; c < Lay::QCH; ++c)
+            tma_load_3d(sb + Lay::OFF_K + st * Lay::QTILE + c * Lay::CHUNK, &tm_k,
                         bar(Lay::B_K_FULL + st), c * 64, row, w.plane);
           const int vs = g % Lay::VST, vuse = g / Lay::VST;
           if (vuse > 0 &&
@@ -399,11 +405,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(bar(Lay::B_V_FULL + vs), Lay::TILE);
+          mbar_arrive_expect_tx(bar(Lay::B_V_FULL + vs), Lay::VTILE);
           ++v_issued[vs];
 #pragma unroll
-          for (int c = 0; c < Lay::CH; ++c)
-            tma_load_3d(sb + Lay::OFF_V + vs * Lay::TILE + c * Lay::CHUNK, &tm_v,
+          for (int c = 0; c < Lay::VCH; ++c)
+            tma_load_3d(sb + Lay::OFF_V + vs * Lay::VTILE + c * Lay::CHUNK, &tm_v,
                         bar(Lay::B_V_FULL + vs), c * 64, row, w.plane);
         }
       }
@@ -442,15 +448,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                1)))
             break;
           tc_fence_after();
-          const uint64_t k_desc = k_desc0 + (uint64_t)(st * (Lay::TILE >> 4));
-          const uint64_t v_desc = v_desc0 + (uint64_t)(vs * (Lay::TILE >> 4));
+          const uint64_t k_desc = k_desc0 + (uint64_t)(st * (Lay::QTILE >> 4));
+          const uint64_t v_desc = v_desc0 + (uint64_t)(vs * (Lay::VTILE >> 4));
 #pragma unroll
-          for (int kk = 0; kk < DIM / 16; ++kk) {
+          for (int kk = 0; kk < DQK / 16; ++kk) {
             const uint64_t koff = (uint64_t)(((kk >> 2) * Lay::CHUNK + (kk & 3) * 32) >> 4);
             mma_ss(tmem + Lay::TM_S, q_desc + koff, k_desc + koff, id_s, kk > 0 ? 1u : 0u);
           }
 #pragma unroll
-          for (int kk = 0; kk < DIM / 16; ++kk) {
+          for (int kk = 0; kk < DV / 16; ++kk) {
             const uint64_t koff = (uint64_t)(((kk >> 2) * Lay::CHUNK + (kk & 3) * 32) >> 4);
             mma_ss(tmem + Lay::TM_DP, do_desc + koff, v_desc + koff, id_s, kk > 0 ? 1u : 0u);
           }
@@ -465,7 +471,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == 10) {
     // ------------------------------------------------- MMA issuer: dQ += dS K
     if (lane == 0) {
-      const uint32_t id_q = idesc_bf16_f32(128, DIM, true);
+      const uint32_t id_q = idesc_bf16_f32(128, DQK, true);
       // K read MN-major: keys 16kk .. 16kk+15 of each 64-column box are 2048 bytes in
       const uint64_t k_desc0 = sdesc_sw128(sb + Lay::OFF_K, Lay::CHUNK, 1024);
       int g = 0, it = 0;
@@ -484,7 +490,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                !(ok = mbar_wait(bar(Lay::B_DQ_EMPTY), (it - 1) & 1, abort_flag, status, 1))))
             break;
           tc_fence_after();
-          const uint64_t k_desc = k_desc0 + (uint64_t)(st * (Lay::TILE >> 4));
+          const uint64_t k_desc = k_desc0 + (uint64_t)(st * (Lay::QTILE >> 4));
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(tmem + Lay::TM_DQ, tmem + Lay::TM_DS + kk * 8,
@@ -558,7 +564,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // epilogue: dQ = scale * acc, bf16
       if (!mbar_wait(bar(Lay::B_DQ_FULL), it & 1, abort_flag, status, 1)) break;
       tc_fence_after();
-      constexpr int OH = DIM / 2;
+      constexpr int OH = DQK / 2;
       uint32_t orr[OH / 32][32];
 #pragma unroll
       for (int ch = 0; ch < OH / 32; ++ch)
@@ -567,7 +573,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(Lay::B_DQ_EMPTY));
       if (valid) {
-        uint4* dst = reinterpret_cast<uint4*>(p.dq + grow * DIM + wg * OH);
+        uint4* dst = reinterpret_cast<uint4*>(p.dq + grow * DQK + wg * OH);
 #pragma unroll
         for (int ch = 0; ch < OH / 32; ++ch)
 #pragma unroll
@@ -594,33 +600,44 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 // ---------------------------------------------------------------- dK, dV
 //
-// Each query block is taken as two halves of 64 queries.  Compute warpgroup h
-// owns half h of every step: TMEM holds S^T_h and dP^T_h (keys on the lanes,
-// 64 query columns each) for both halves at once, so while one warpgroup
-// turns its half into P^T / dS^T the tensor core works on the other half.
+// Each query block is taken as two half-steps of 64 queries; half-step k = 2s
+// + h (query step s, half h) belongs to compute warpgroup h.  Its S^T (keys on
+// the TMEM lanes, 64 query columns) goes to TMEM region k mod 3 and its dP^T
+// to region (k + 1) mod 3, 64 columns each.  The warpgroup reads both, then
+// writes P^T and dS^T as bf16 pairs over the 64 columns of S^T's region, from
+// where the dV and dK products read them.  dP^T's region is free once the
+// warpgroup has read it, and it is the next half-step's S^T region, so the
+// tensor core computes half-step k+1's products while warpgroup h turns
+// half-step k into P^T and dS^T.  Three regions (192 columns) beside dV (d_v
+// columns) and dK (d_qk columns) fit the 512 columns for d_qk up to 192.
+// Q and dO stream through a ring of half-step slots, [Q | dO] rows of 64
+// queries each, so that the d_qk = 192 tiles fit shared memory with three
+// half-steps in flight.
 
-template <int DIM>
+template <int DQK, int DV>
 struct BwdKvLayout {
-  static constexpr int CH = DIM / 64;
-  static constexpr int CHUNK = 128 * 128;
-  static constexpr int TILE = CH * CHUNK;
-  static constexpr int QST = 2;                    // (Q, dO) ring depth
+  static constexpr int QCH = DQK / 64, VCH = DV / 64;
+  static constexpr int CHUNK = 128 * 128;   // [128 rows x 64 bf16] box: K, V
+  static constexpr int HCHUNK = 64 * 128;   // [64 rows x 64 bf16] box: Q, dO of a half-step
+  static constexpr int KTILE = QCH * CHUNK, VTILE = VCH * CHUNK;
+  static constexpr int HSLOT = (QCH + VCH) * HCHUNK;  // [Q_h | dO_h]
+  static constexpr int NHS = KTILE + VTILE + 4 * HSLOT <= 200 * 1024 ? 4 : 3;  // half-step slots
   static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = TILE;
-  static constexpr int OFF_Q = 2 * TILE;           // QST x [Q | dO]
-  static constexpr int OFF_ROW = OFF_Q + QST * 2 * TILE;  // float [2 steps][2 halves][lse2, D][64]
+  static constexpr int OFF_V = KTILE;
+  static constexpr int OFF_Q = KTILE + VTILE;           // NHS x [Q_h | dO_h]
+  static constexpr int OFF_ROW = OFF_Q + NHS * HSLOT;   // float [2 steps][2 halves][lse2, D][64]
   static constexpr int OFF_BAR = OFF_ROW + 2 * 2 * 2 * 64 * 4;
-  // TMEM: per half h, S^T_h at 128h and dP^T_h at 128h + 64 (P^T_h / dS^T_h as
-  // bf16 pairs over their first 32 columns), then dV and dK
-  static constexpr int TM_DV = 256, TM_DK = 256 + DIM;
-  static_assert(TM_DK + DIM <= 512, "TMEM");
+  // TMEM: regions 0..2 of 64 columns at 64 r, then dV and dK
+  static constexpr int TM_DV = 192, TM_DK = 192 + DV;
+  static_assert(TM_DK + DQK <= 512, "TMEM");
   // barriers
   static constexpr int B_KV_FULL = 0, B_KV_EMPTY = 1;
-  static constexpr int B_Q_FULL = 2, B_Q_EMPTY = B_Q_FULL + QST;
-  static constexpr int B_ST_FULL = B_Q_EMPTY + QST;  // [2] S^T_h, dP^T_h issued (commit)
+  static constexpr int B_Q_FULL = 2, B_Q_EMPTY = B_Q_FULL + NHS;  // per half-step slot
+  static constexpr int B_ST_FULL = B_Q_EMPTY + NHS;  // [2] S^T, dP^T of warpgroup h's half-step issued
   static constexpr int B_SYNC = B_ST_FULL + 2;       // [2] warpgroup h: its rows staged
-  static constexpr int B_PDS_FULL = B_SYNC + 2;      // [2] P^T_h, dS^T_h written
-  static constexpr int B_PDS_FREE = B_PDS_FULL + 2;  // [2] dV, dK products of half h done
+  static constexpr int B_READ = B_SYNC + 2;          // [2] warpgroup h has read S^T and dP^T
+  static constexpr int B_PDS_FULL = B_READ + 2;      // [2] P^T, dS^T written
+  static constexpr int B_PDS_FREE = B_PDS_FULL + 2;  // [2] their dV, dK products done
   static constexpr int B_ACC_FULL = B_PDS_FREE + 2;  // the item's last dV, dK products done
   static constexpr int B_ACC_EMPTY = B_ACC_FULL + 1; // epilogue has read dV, dK
   static constexpr int B_DRAIN = B_ACC_EMPTY + 1;    // [2] one per issuer
@@ -630,13 +647,54 @@ struct BwdKvLayout {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
-template <int DIM>
+// Epilogue of one accumulator row (D columns; warpgroup h takes columns
+// h D/2 .. h D/2 + D/2 - 1): mul * acc as fp32 to part_row (a sink chunk's
+// partial) or, when part_row is null, as bf16 to out_row if `valid`.
+template <int D>
+__device__ __forceinline__ void bwd_kv_store(uint32_t acc_tmem, int h, float mul, float* part_row,
+                                             __nv_bfloat16* out_row, bool valid) {
+  constexpr int OH = D / 2;
+  uint32_t ar[OH / 32][32];
+#pragma unroll
+  for (int ch = 0; ch < OH / 32; ++ch) tmem_ld32(acc_tmem + h * OH + ch * 32, ar[ch]);
+  tmem_wait_ld();
+  if (part_row) {
+    float* dst = part_row + h * OH;
+#pragma unroll
+    for (int ch = 0; ch < OH / 32; ++ch)
+#pragma unroll
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4*>(dst + ch * 32 + e) =
+            make_float4(__uint_as_float(ar[ch][e]) * mul, __uint_as_float(ar[ch][e + 1]) * mul,
+                        __uint_as_float(ar[ch][e + 2]) * mul, __uint_as_float(ar[ch][e + 3]) * mul);
+  } else if (valid) {
+    uint4* dst = reinterpret_cast<uint4*>(out_row + h * OH);
+#pragma unroll
+    for (int ch = 0; ch < OH / 32; ++ch)
+#pragma unroll
+      for (int v = 0; v < 4; v += 2) {
+        uint32_t a8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          a8[e] = pack_bf16x2(__uint_as_float(ar[ch][8 * v + 2 * e]) * mul,
+                              __uint_as_float(ar[ch][8 * v + 2 * e + 1]) * mul);
+        st_global_v8(dst + ch * 4 + v, a8);
+      }
+  }
+}
+
+// TMEM regions of half-step k: S^T (then P^T | dS^T) and dP^T.
+__device__ __forceinline__ uint32_t bwd_region_s(int k) { return 64u * (uint32_t)(k % 3); }
+__device__ __forceinline__ uint32_t bwd_region_dp(int k) { return 64u * (uint32_t)((k + 1) % 3); }
+
+// tm_q and tm_do here have boxes of 64 rows (a half-step); tm_k and tm_v of 128.
+template <int DQK, int DV>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     ssa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
-  using Lay = BwdKvLayout<DIM>;
+  using Lay = BwdKvLayout<DQK, DV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -651,13 +709,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar(Lay::B_KV_FULL), 1);
     mbar_init(bar(Lay::B_KV_EMPTY), 1);
-    for (int s = 0; s < Lay::QST; ++s) {
+    for (int s = 0; s < Lay::NHS; ++s) {
       mbar_init(bar(Lay::B_Q_FULL + s), 1);
       mbar_init(bar(Lay::B_Q_EMPTY + s), 1);
     }
     for (int h = 0; h < 2; ++h) {
       mbar_init(bar(Lay::B_ST_FULL + h), 1);
       mbar_init(bar(Lay::B_SYNC + h), kBwdComputeThreads / 2);
+      mbar_init(bar(Lay::B_READ + h), kBwdComputeThreads / 2);
       mbar_init(bar(Lay::B_PDS_FULL + h), kBwdComputeThreads / 2);
       mbar_init(bar(Lay::B_PDS_FREE + h), 1);
       mbar_init(bar(Lay::B_DRAIN + h), 1);
@@ -685,8 +744,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int s = 0, it = 0, kv_issued = 0;
-      int q_issued[Lay::QST] = {};
+      int k = 0, it = 0, kv_issued = 0;  // k: half-steps issued
       bool ok = true;
       for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++it) {
         const BwdKItem w = bwd_kv_item(p, item);
@@ -694,78 +752,87 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(bar(Lay::B_KV_FULL), 2 * Lay::TILE);
+        mbar_arrive_expect_tx(bar(Lay::B_KV_FULL), Lay::KTILE + Lay::VTILE);
         ++kv_issued;
 #pragma unroll
-        for (int c = 0; c < Lay::CH; ++c) {
+        for (int c = 0; c < Lay::QCH; ++c)
           tma_load_3d(sb + Lay::OFF_K + c * Lay::CHUNK, &tm_k, bar(Lay::B_KV_FULL), c * 64,
                       w.seq_start + w.kb * 128, w.plane);
+#pragma unroll
+        for (int c = 0; c < Lay::VCH; ++c)
           tma_load_3d(sb + Lay::OFF_V + c * Lay::CHUNK, &tm_v, bar(Lay::B_KV_FULL), c * 64,
                       w.seq_start + w.kb * 128, w.plane);
-        }
-        for (int qi = w.q_lo; qi <= w.q_hi; ++qi, ++s) {
-          const int st = s % Lay::QST, use = s / Lay::QST;
-          if (use > 0 &&
-              !mbar_wait(bar(Lay::B_Q_EMPTY + st), (use - 1) & 1, abort_flag, status, 1)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(bar(Lay::B_Q_FULL + st), 2 * Lay::TILE);
-          ++q_issued[st];
-          const uint32_t base = sb + Lay::OFF_Q + st * 2 * Lay::TILE;
+        for (int qi = w.q_lo; ok && qi <= w.q_hi; ++qi) {
+#pragma unroll 1
+          for (int h = 0; h < 2; ++h, ++k) {
+            const int slot = k % Lay::NHS, use = k / Lay::NHS;
+            if (use > 0 &&
+                !mbar_wait(bar(Lay::B_Q_EMPTY + slot), (use - 1) & 1, abort_flag, status, 1)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(bar(Lay::B_Q_FULL + slot), Lay::HSLOT);
+            const uint32_t base = sb + Lay::OFF_Q + slot * Lay::HSLOT;
+            const int row = w.seq_start + qi * 128 + h * 64;
 #pragma unroll
-          for (int c = 0; c < Lay::CH; ++c) {
-            tma_load_3d(base + c * Lay::CHUNK, &tm_q, bar(Lay::B_Q_FULL + st), c * 64,
-                        w.seq_start + qi * 128, w.plane);
-            tma_load_3d(base + Lay::TILE + c * Lay::CHUNK, &tm_do, bar(Lay::B_Q_FULL + st),
-                        c * 64, w.seq_start + qi * 128, w.plane);
+            for (int c = 0; c < Lay::QCH; ++c)
+              tma_load_3d(base + c * Lay::HCHUNK, &tm_q, bar(Lay::B_Q_FULL + slot), c * 64, row,
+                          w.plane);
+#pragma unroll
+            for (int c = 0; c < Lay::VCH; ++c)
+              tma_load_3d(base + (Lay::QCH + c) * Lay::HCHUNK, &tm_do, bar(Lay::B_Q_FULL + slot),
+                          c * 64, row, w.plane);
           }
         }
       }
+      // let the copies in flight land before the CTA's shared memory goes away:
+      // a slot holds at most one unconsumed load, its newest phase
       if (!ok) {
-        for (int st = 0; st < Lay::QST; ++st)
-          if (q_issued[st] > 0) mbar_wait_drain(bar(Lay::B_Q_FULL + st), (q_issued[st] - 1) & 1);
+        drain_ring(bar(Lay::B_Q_FULL), Lay::NHS, k);
         if (kv_issued > 0) mbar_wait_drain(bar(Lay::B_KV_FULL), (kv_issued - 1) & 1);
       }
     }
   } else if (warp == 9) {
-    // ------------------------------------------ MMA issuer: S^T_h and dP^T_h
+    // ------------------------------------------ MMA issuer: S^T and dP^T
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16_f32(128, 64, false);   // M = keys, N = 64 queries
       const uint64_t k_desc = sdesc_sw128(sb + Lay::OFF_K, 16, 1024);
       const uint64_t v_desc = sdesc_sw128(sb + Lay::OFF_V, 16, 1024);
       const uint64_t q_desc0 = sdesc_sw128(sb + Lay::OFF_Q, 16, 1024);
-      int s = 0, it = 0;
+      int k = 0, it = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++it) {
         const BwdKItem w = bwd_kv_item(p, item);
         if (!(ok = mbar_wait(bar(Lay::B_KV_FULL), it & 1, abort_flag, status, 1))) break;
-        for (int qi = w.q_lo; ok && qi <= w.q_hi; ++qi, ++s) {
-          const int st = s % Lay::QST;
-          if (!(ok = mbar_wait(bar(Lay::B_Q_FULL + st), (s / Lay::QST) & 1, abort_flag, status,
-                               1)))
-            break;
-          const uint64_t q_desc = q_desc0 + (uint64_t)(st * ((2 * Lay::TILE) >> 4));
-          const uint64_t do_desc = q_desc + (uint64_t)(Lay::TILE >> 4);
+        for (int qi = w.q_lo; ok && qi <= w.q_hi; ++qi) {
 #pragma unroll 1
-          for (int h = 0; h < 2; ++h) {
-            // S^T_h / dP^T_h overwrite P^T_h / dS^T_h of the previous step
-            if (s > 0 &&
-                !(ok = mbar_wait(bar(Lay::B_PDS_FREE + h), (s - 1) & 1, abort_flag, status, 1)))
+          for (int h = 0; h < 2; ++h, ++k) {
+            const int slot = k % Lay::NHS;
+            // S^T's region was the previous half-step's dP^T region: its
+            // warpgroup has read it; dP^T's region held P^T / dS^T of
+            // half-step k - 2: their dV / dK products are done
+            if (!(ok = mbar_wait(bar(Lay::B_Q_FULL + slot), (k / Lay::NHS) & 1, abort_flag,
+                                 status, 1)) ||
+                (k >= 1 && !(ok = mbar_wait(bar(Lay::B_READ + ((k - 1) & 1)), ((k - 1) >> 1) & 1,
+                                            abort_flag, status, 1))) ||
+                (k >= 2 && !(ok = mbar_wait(bar(Lay::B_PDS_FREE + (k & 1)), ((k - 2) >> 1) & 1,
+                                            abort_flag, status, 1))))
               break;
             tc_fence_after();
-            const uint32_t st_t = tmem + 128 * h, dpt_t = st_t + 64;
-            // queries 64h .. 64h+63: rows 64h.. of every box (8192 bytes in)
-            const uint64_t hoff = (uint64_t)((8192 * h) >> 4);
+            const uint32_t st_t = tmem + bwd_region_s(k), dpt_t = tmem + bwd_region_dp(k);
+            const uint64_t q_desc = q_desc0 + (uint64_t)((slot * Lay::HSLOT) >> 4);
+            const uint64_t do_desc = q_desc + (uint64_t)((Lay::QCH * Lay::HCHUNK) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < DIM / 16; ++kk) {
+            for (int kk = 0; kk < DQK / 16; ++kk) {
               const uint64_t koff = (uint64_t)(((kk >> 2) * Lay::CHUNK + (kk & 3) * 32) >> 4);
-              mma_ss(st_t, k_desc + koff, q_desc + hoff + koff, id_s, kk > 0 ? 1u : 0u);
+              const uint64_t hoff = (uint64_t)(((kk >> 2) * Lay::HCHUNK + (kk & 3) * 32) >> 4);
+              mma_ss(st_t, k_desc + koff, q_desc + hoff, id_s, kk > 0 ? 1u : 0u);
             }
 #pragma unroll
-            for (int kk = 0; kk < DIM / 16; ++kk) {
+            for (int kk = 0; kk < DV / 16; ++kk) {
               const uint64_t koff = (uint64_t)(((kk >> 2) * Lay::CHUNK + (kk & 3) * 32) >> 4);
-              mma_ss(dpt_t, v_desc + koff, do_desc + hoff + koff, id_s, kk > 0 ? 1u : 0u);
+              const uint64_t hoff = (uint64_t)(((kk >> 2) * Lay::HCHUNK + (kk & 3) * 32) >> 4);
+              mma_ss(dpt_t, v_desc + koff, do_desc + hoff, id_s, kk > 0 ? 1u : 0u);
             }
             mma_commit(bar(Lay::B_ST_FULL + h));
           }
@@ -778,45 +845,42 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == 10) {
     // ------------------------------------ MMA issuer: dV += P^T dO, dK += dS^T Q
     if (lane == 0) {
-      const uint32_t id_a = idesc_bf16_f32(128, DIM, true);  // B = dO / Q, MN-major
-      // queries 16kk .. of half h: rows 64h + 16kk of every box (2048 bytes per 16 rows)
-      const uint64_t q_desc0 = sdesc_sw128(sb + Lay::OFF_Q, Lay::CHUNK, 1024);
-      int s = 0, it = 0;
+      const uint32_t id_v = idesc_bf16_f32(128, DV, true);   // B = dO_h, MN-major
+      const uint32_t id_k = idesc_bf16_f32(128, DQK, true);  // B = Q_h, MN-major
+      // queries 16kk .. 16kk+15 of a half-step: rows 16kk of every 64-row box
+      // (2048 bytes in); consecutive 64-column boxes HCHUNK apart
+      const uint64_t q_desc0 = sdesc_sw128(sb + Lay::OFF_Q, Lay::HCHUNK, 1024);
+      int k = 0, it = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++it) {
         const BwdKItem w = bwd_kv_item(p, item);
-        for (int qi = w.q_lo; ok && qi <= w.q_hi; ++qi, ++s) {
-          const int st = s % Lay::QST;
-          const uint64_t q_desc = q_desc0 + (uint64_t)(st * ((2 * Lay::TILE) >> 4));
-          const uint64_t do_desc = q_desc + (uint64_t)(Lay::TILE >> 4);
-          if (!(ok = mbar_wait(bar(Lay::B_Q_FULL + st), (s / Lay::QST) & 1, abort_flag, status,
-                               1)))
-            break;
+        for (int qi = w.q_lo; ok && qi <= w.q_hi; ++qi) {
 #pragma unroll 1
-          for (int h = 0; h < 2; ++h) {
+          for (int h = 0; h < 2; ++h, ++k) {
+            const int slot = k % Lay::NHS;
+            const uint64_t q_desc = q_desc0 + (uint64_t)((slot * Lay::HSLOT) >> 4);
+            const uint64_t do_desc = q_desc + (uint64_t)((Lay::QCH * Lay::HCHUNK) >> 4);
             const bool first = (qi == w.q_lo && h == 0);
-            if (!(ok = mbar_wait(bar(Lay::B_PDS_FULL + h), s & 1, abort_flag, status, 1)) ||
+            if (!(ok = mbar_wait(bar(Lay::B_Q_FULL + slot), (k / Lay::NHS) & 1, abort_flag,
+                                 status, 1)) ||
+                !(ok = mbar_wait(bar(Lay::B_PDS_FULL + h), (k >> 1) & 1, abort_flag, status, 1)) ||
                 (first && it > 0 &&
                  !(ok = mbar_wait(bar(Lay::B_ACC_EMPTY), (it - 1) & 1, abort_flag, status, 1))))
               break;
             tc_fence_after();
-            const uint32_t pt_t = tmem + 128 * h, dst_t = pt_t + 64;
+            const uint32_t pt_t = tmem + bwd_region_s(k), dst_t = pt_t + 32;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t off = (uint64_t)((8192 * h + 2048 * kk) >> 4);
-              mma_ts(tmem + Lay::TM_DV, pt_t + kk * 8, do_desc + off, id_a,
-                     (!first || kk > 0) ? 1u : 0u);
-            }
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ts(tmem + Lay::TM_DV, pt_t + kk * 8, do_desc + (uint64_t)((2048 * kk) >> 4),
+                     id_v, (!first || kk > 0) ? 1u : 0u);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t off = (uint64_t)((8192 * h + 2048 * kk) >> 4);
-              mma_ts(tmem + Lay::TM_DK, dst_t + kk * 8, q_desc + off, id_a,
-                     (!first || kk > 0) ? 1u : 0u);
-            }
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ts(tmem + Lay::TM_DK, dst_t + kk * 8, q_desc + (uint64_t)((2048 * kk) >> 4),
+                     id_k, (!first || kk > 0) ? 1u : 0u);
             mma_commit(bar(Lay::B_PDS_FREE + h));
+            mma_commit(bar(Lay::B_Q_EMPTY + slot));
           }
           if (!ok) break;
-          mma_commit(bar(Lay::B_Q_EMPTY + st));
           if (qi == w.q_hi) mma_commit(bar(Lay::B_ACC_FULL));
         }
       }
@@ -836,6 +900,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int key = w.kb * 128 + r;
       bool ok = true;
       for (int qi = w.q_lo; qi <= w.q_hi; ++qi, ++s) {
+        const int k = 2 * s + h;  // this warpgroup's half-step
         // stage lse2 and D of this half's 64 queries; rows past the sequence
         // (zero fill, or the next packed sequence) get lse2 = +inf: P = 0
         float* lse_s = rows_smem + ((s & 1) * 2 + h) * 128;
@@ -855,7 +920,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         tc_fence_after();
         const bool diag = (qi == w.kb);
-        const uint32_t st_t = tmem + lane_base + 128 * h, dpt_t = st_t + 64;
+        const uint32_t st_t = tmem + lane_base + bwd_region_s(k);
+        const uint32_t dpt_t = tmem + lane_base + bwd_region_dp(k);
         uint32_t pk[32], dk_[32];
 #pragma unroll
         for (int c2 = 0; c2 < 2; ++c2) {
@@ -863,6 +929,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tmem_ld32(st_t + c2 * 32, st_r);
           tmem_ld32(dpt_t + c2 * 32, dp_r);
           tmem_wait_ld();
+          if (c2 == 1) {
+            // all of dP^T is read: its region may take the next half-step's S^T
+            tc_fence_before();
+            mbar_arrive(bar(Lay::B_READ + h));
+          }
 #pragma unroll
           for (int c = 0; c < 32; c += 4) {
             const int qc = c2 * 32 + c;                 // query within the half
@@ -884,9 +955,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             dk_[c2 * 16 + c / 2 + 1] = pack_bf16x2(dd[2], dd[3]);
           }
         }
-        // this thread's row is read: P^T / dS^T over its first 32 columns
+        // P^T and dS^T over the 64 columns of S^T's region
         tmem_st32(st_t, pk);
-        tmem_st32(dpt_t, dk_);
+        tmem_st32(st_t + 32, dk_);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(Lay::B_PDS_FULL + h));
@@ -896,43 +967,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // sink chunks go out as fp32 partials that the reduce kernel adds up
       if (!mbar_wait(bar(Lay::B_ACC_FULL), it & 1, abort_flag, status, 1)) break;
       tc_fence_after();
-      constexpr int OH = DIM / 2;
       const size_t grow = (size_t)w.plane * p.plane_rows + w.seq_start + key;
-#pragma unroll 1
-      for (int which = 0; which < 2; ++which) {  // 0: dK, 1: dV
-        const float mul = which == 0 ? p.scale : 1.f;
-        uint32_t ar[OH / 32][32];
-#pragma unroll
-        for (int ch = 0; ch < OH / 32; ++ch)
-          tmem_ld32(tmem + lane_base + (which == 0 ? Lay::TM_DK : Lay::TM_DV) + h * OH + ch * 32,
-                    ar[ch]);
-        tmem_wait_ld();
-        if (w.slot >= 0) {
-          float* dst = p.part + (((size_t)w.slot * 2 + which) * 128 + r) * DIM + h * OH;
-#pragma unroll
-          for (int ch = 0; ch < OH / 32; ++ch)
-#pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              *reinterpret_cast<float4*>(dst + ch * 32 + e) =
-                  make_float4(__uint_as_float(ar[ch][e]) * mul,
-                              __uint_as_float(ar[ch][e + 1]) * mul,
-                              __uint_as_float(ar[ch][e + 2]) * mul,
-                              __uint_as_float(ar[ch][e + 3]) * mul);
-        } else if (key < w.len) {
-          uint4* dst = reinterpret_cast<uint4*>((which == 0 ? p.dk : p.dv) + grow * DIM + h * OH);
-#pragma unroll
-          for (int ch = 0; ch < OH / 32; ++ch)
-#pragma unroll
-            for (int v = 0; v < 4; v += 2) {
-              uint32_t a8[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e)
-                a8[e] = pack_bf16x2(__uint_as_float(ar[ch][8 * v + 2 * e]) * mul,
-                                    __uint_as_float(ar[ch][8 * v + 2 * e + 1]) * mul);
-              st_global_v8(dst + ch * 4 + v, a8);
-            }
-        }
-      }
+      // slot layout: dK [128 keys][d_qk], then dV [128 keys][d_v]
+      float* part = w.slot >= 0 ? p.part + (size_t)w.slot * 128 * (DQK + DV) : nullptr;
+      bwd_kv_store<DQK>(tmem + lane_base + Lay::TM_DK, h, p.scale,
+                        part ? part + (size_t)r * DQK : nullptr, p.dk + grow * DQK,
+                        key < w.len);
+      bwd_kv_store<DV>(tmem + lane_base + Lay::TM_DV, h, 1.f,
+                       part ? part + (size_t)128 * DQK + (size_t)r * DV : nullptr,
+                       p.dv + grow * DV, key < w.len);
       tc_fence_before();
       mbar_arrive(bar(Lay::B_ACC_EMPTY));
     }
@@ -948,11 +991,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 // The sink blocks' dK, dV: the sum of their chunks' fp32 partials, as bf16.
-// Dense: one thread per (plane, sink block, key row, 4 columns).  Packed:
-// blockIdx.y is the sequence and the threads of its column of CTAs walk its
-// (head, sink block, key row, 4 columns).
-template <int DIM>
+// A slot holds dK [128 keys][d_qk] then dV [128 keys][d_v].  Dense: one thread
+// per (plane, sink block, key row, 4 columns of dK or dV).  Packed: blockIdx.y
+// is the sequence and the threads of its column of CTAs walk its (head, sink
+// block, key row, 4 columns).
+template <int DQK, int DV>
 __global__ void __launch_bounds__(256) ssa_bwd_sink_reduce_kernel(const BwdParams p) {
+  constexpr int C4 = (DQK + DV) / 4;  // 4-column groups of a key row: dK's, then dV's
   int n_sink, nb, len, seq_start, planes;
   long long slot_base;  // slot of chunk 0 of sink block 0 of head 0
   int per_head;         // sink slots per head
@@ -976,33 +1021,34 @@ __global__ void __launch_bounds__(256) ssa_bwd_sink_reduce_kernel(const BwdParam
     if (__ldg(pfx_sink + p.n_seqs) == 0) return;  // invalid cu_seqlens: nothing was computed
   }
   n_sink = min(p.n_sink, nb);
-  const long long quads = (long long)planes * n_sink * 128 * (DIM / 4);
+  const long long quads = (long long)planes * n_sink * 128 * C4;
   for (long long x = blockIdx.x * (long long)blockDim.x + threadIdx.x; x < quads;
        x += (long long)gridDim.x * blockDim.x) {
-    const int c4 = (int)(x % (DIM / 4));
-    const int r = (int)((x / (DIM / 4)) % 128);
-    const int j = (int)((x / (DIM / 4) / 128) % n_sink);
-    const int plane = (int)(x / (DIM / 4) / 128 / n_sink);
+    const int c4 = (int)(x % C4);
+    const int r = (int)((x / C4) % 128);
+    const int j = (int)((x / C4 / 128) % n_sink);
+    const int plane = (int)(x / C4 / 128 / n_sink);
     const int key = j * 128 + r;
     if (key >= len) continue;
     long long slot = slot_base + (long long)plane * per_head;
     for (int j2 = 0; j2 < j; ++j2) slot += bwd_sink_chunks(j2, nb);
-    float4 ak = make_float4(0.f, 0.f, 0.f, 0.f), av = ak;
+    const bool is_k = c4 < DQK / 4;
+    const size_t in_slot = is_k ? (size_t)r * DQK + 4 * c4
+                                : (size_t)128 * DQK + (size_t)r * DV + 4 * (c4 - DQK / 4);
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int c = 0; c < bwd_sink_chunks(j, nb); ++c) {
-      const float* base = p.part + ((size_t)(slot + c) * 2 * 128 + r) * DIM + 4 * c4;
-      const float4 k4 = *reinterpret_cast<const float4*>(base);
-      const float4 v4 = *reinterpret_cast<const float4*>(base + (size_t)128 * DIM);
-      ak.x += k4.x; ak.y += k4.y; ak.z += k4.z; ak.w += k4.w;
-      av.x += v4.x; av.y += v4.y; av.z += v4.z; av.w += v4.w;
+      const float4 v4 = *reinterpret_cast<const float4*>(
+          p.part + (size_t)(slot + c) * 128 * (DQK + DV) + in_slot);
+      a.x += v4.x; a.y += v4.y; a.z += v4.z; a.w += v4.w;
     }
     const size_t grow = (size_t)plane * p.plane_rows + seq_start + key;
-    uint2 ko, vo;
-    ko.x = pack_bf16x2(ak.x, ak.y);
-    ko.y = pack_bf16x2(ak.z, ak.w);
-    vo.x = pack_bf16x2(av.x, av.y);
-    vo.y = pack_bf16x2(av.z, av.w);
-    *reinterpret_cast<uint2*>(p.dk + grow * DIM + 4 * c4) = ko;
-    *reinterpret_cast<uint2*>(p.dv + grow * DIM + 4 * c4) = vo;
+    uint2 out;
+    out.x = pack_bf16x2(a.x, a.y);
+    out.y = pack_bf16x2(a.z, a.w);
+    if (is_k)
+      *reinterpret_cast<uint2*>(p.dk + grow * DQK + 4 * c4) = out;
+    else
+      *reinterpret_cast<uint2*>(p.dv + grow * DV + 4 * (c4 - DQK / 4)) = out;
   }
 }
 

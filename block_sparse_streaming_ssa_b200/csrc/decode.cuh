@@ -15,8 +15,8 @@
 //           The last four S stages hold K boxes 4..7, which are also V columns
 //           256..511: they stay in the ring for O half 1.  V columns 0..255
 //           are read again (L2 hits): page A's boxes into the Q slots (free
-//           once S is done), page B's into the K_B slots (free once O half 1
-//           is done).
+//           once S is done), page B's into the K_A slots (free once O half
+//           1's page-A products are done).
 //   MMA     S[128 heads x 256 keys] = Q [K_A; K_B]^T into TMEM columns
 //           [0,256) -- K_A and K_B boxes sit side by side, one N=256 operand
 //   softmax warpgroup 0 takes page A's 128 keys of every head row, warpgroup 1
@@ -79,6 +79,9 @@ struct DecodeParams {
   float scale_log2;
   // FP8 cache only: fp32 scale of every token, [n_pages, 128] by physical page.
   const float* kv_scale;
+  // 1: the n_split splits of a (row, head group) run as one thread-block
+  // cluster and merge their partials in the split kernel (no merge kernel).
+  int cluster_merge;
 };
 
 __device__ __forceinline__ int decode_seq(const DecodeParams& p, int row) {
@@ -155,13 +158,14 @@ struct DecodeLayout {
   static constexpr int B_FULL = 0;              // NST
   static constexpr int B_EMPTY = B_FULL + NST;  // NST
   static constexpr int B_VA_FULL = B_EMPTY + NST;  // V_A boxes 0..3 in the Q slots
-  static constexpr int B_VB_FULL = B_VA_FULL + 1;  // V_B boxes 0..3 in the K_B slots
+  static constexpr int B_VB_FULL = B_VA_FULL + 1;  // V_B boxes 0..3 in the K_A slots
   static constexpr int B_S_FULL = B_VB_FULL + 1;
   static constexpr int B_P_FULL = B_S_FULL + 1;   // 256 arrivals
   static constexpr int B_XCHG = B_P_FULL + 1;     // 256 arrivals; phase 0 max, 1 sum
   static constexpr int B_O_FULL = B_XCHG + 1;     // phase 0: O half 1, phase 1: O half 0
   static constexpr int B_O_EMPTY = B_O_FULL + 1;  // 256 arrivals, one phase per half
-  static constexpr int B_DRAIN = B_O_EMPTY + 1;
+  static constexpr int B_KA_FREE = B_O_EMPTY + 1;  // O half 1's page-A products done
+  static constexpr int B_DRAIN = B_KA_FREE + 1;
   // FP8 cache: a stage's K boxes expanded to bf16, the V_A and the V_B boxes
   // expanded
   static constexpr int B_CONV = B_DRAIN + 1;  // NST
@@ -239,12 +243,92 @@ __device__ __forceinline__ bool decode_expand_fp8_box(uint32_t slot, int row, ui
 }
 
 template <bool FP8>
+__device__ __forceinline__ void decode_split_body(const CUtensorMap* tm_q_p,
+                                                  const CUtensorMap* tm_kv_p,
+                                                  const DecodeParams& p, int sp, int hg, int b,
+                                                  size_t cta, int phys_a, int phys_b, int valid_a,
+                                                  int valid_b);
+
+// Merge of the split partials of row b, head group hg (n_split <= 4), for the
+// 8-column groups [g0, g1) of O: LSE = logsumexp_s LSE_s, O = sum_s exp(LSE_s -
+// LSE) O_s.  Splits whose LSE is -inf are empty and contribute nothing (their
+// partial O is never read into the sum); a NaN LSE marks a split that gave up
+// on a wait, and makes the head's O and LSE NaN.  256 threads: thread (set,
+// head) = (tid / 128, tid % 128) takes groups g0 + set, g0 + set + 2, ... in
+// passes of 8, with every load of a pass in flight at once (one L2 round trip
+// per pass); a warp's loads of one group of one split are 32 heads' 16-byte
+// pieces, 512 contiguous bytes.  The partials are read from L2 (ld.global.cg).
+constexpr int kClusterMergeMaxSplits = 4;
+
+__device__ __forceinline__ void decode_merge_groups(const DecodeParams& p, int b, int hg, int g0,
+                                                    int g1, bool write_lse, int tid) {
+  constexpr int NS = kClusterMergeMaxSplits, PASS = 8;
+  const int n = p.n_split;
+  const int h = tid & 127, set = tid >> 7;
+  const int hq = hg * 128 + h;
+  if (tid >= 256 || hq >= p.H_q) return;
+  const size_t cta0 = ((size_t)b * p.HG + hg) * n;
+  const uint4* op = reinterpret_cast<const uint4*>(p.o_part) + cta0 * (64 * 128) + h;
+  float ls[NS];
+  float mx = -INFINITY;
+  bool poisoned = false;
+#pragma unroll
+  for (int s = 0; s < NS; ++s) {
+    ls[s] = s < n ? __ldcg(p.lse_part + (cta0 + s) * 128 + h) : -INFINITY;
+    poisoned |= ls[s] != ls[s];
+    mx = fmaxf(mx, ls[s]);  // fmaxf skips a NaN operand
+  }
+  float wgt[NS];
+  float den = 0.f;
+#pragma unroll
+  for (int s = 0; s < NS; ++s) {
+    // empty split, or one that gave up: weight 0 (its partial O is not read)
+    wgt[s] = (s < n && ls[s] != -INFINITY && ls[s] == ls[s]) ? __expf(ls[s] - mx) : 0.f;
+    den += wgt[s];
+  }
+  const float inv = poisoned ? __int_as_float(0x7fc00000) : (den > 0.f ? 1.f / den : 0.f);
+  uint4* orow = reinterpret_cast<uint4*>(p.o + ((size_t)b * p.H_q + hq) * kDecodeDv);
+  for (int gb = g0 + set; gb < g1; gb += 2 * PASS) {
+    uint4 raw[PASS][NS];
+#pragma unroll
+    for (int k = 0; k < PASS; ++k)
+#pragma unroll
+      for (int s = 0; s < NS; ++s)
+        if (gb + 2 * k < g1 && wgt[s] != 0.f)
+          raw[k][s] = __ldcg(op + ((size_t)s * 64 + gb + 2 * k) * 128);
+#pragma unroll
+    for (int k = 0; k < PASS; ++k) {
+      if (gb + 2 * k >= g1) break;
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int s = 0; s < NS; ++s) {
+        if (wgt[s] == 0.f) continue;
+        const __half2* hv = reinterpret_cast<const __half2*>(&raw[k][s]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(hv[e]);
+          acc[2 * e] += wgt[s] * f.x;
+          acc[2 * e + 1] += wgt[s] * f.y;
+        }
+      }
+      uint4 pk;
+      pk.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+      pk.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+      pk.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+      pk.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+      orow[gb + 2 * k] = pk;
+    }
+  }
+  if (write_lse && set == 0)
+    p.lse[(size_t)b * p.H_q + hq] = poisoned ? __int_as_float(0x7fc00000)
+                                    : den > 0.f ? mx + __logf(den) : -INFINITY;
+}
+
+template <bool FP8>
 __global__ void __launch_bounds__(320, 1)
     ssa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_q,
                             const __grid_constant__ CUtensorMap tm_kv, const DecodeParams p) {
-  using Lay = DecodeLayout;
   const int sp = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t cta = ((size_t)b * p.HG + hg) * p.n_split + sp;  // partial-result slot
 
   // The query boxes do not depend on the page table: start pulling them into
@@ -278,9 +362,36 @@ __global__ void __launch_bounds__(320, 1)
   }
   if (phys_a < 0) {
     if (threadIdx.x < 128) p.lse_part[cta * 128 + threadIdx.x] = -INFINITY;  // empty split
-    asm volatile("griddepcontrol.launch_dependents;");
-    return;
+    if (!p.cluster_merge) {
+      asm volatile("griddepcontrol.launch_dependents;");
+      return;
+    }
+  } else {
+    decode_split_body<FP8>(&tm_q, &tm_kv, p, sp, hg, b, cta, phys_a, phys_b, valid_a, valid_b);
   }
+  if (p.cluster_merge) {
+    // The splits of this (row, head group) are the CTAs of this cluster, all
+    // resident at once.  Every thread of every split arrives once its writes
+    // of the partials are done (every wait before this point is bounded, and
+    // an empty split arrives straight away), then each split merges its share
+    // of the 64 column groups; split 0 also writes the LSE.
+    cluster_arrive_release();
+    cluster_wait_acquire();
+    const int n = p.n_split;
+    decode_merge_groups(p, b, hg, 64 * sp / n, 64 * (sp + 1) / n, sp == 0, threadIdx.x);
+  }
+}
+
+template <bool FP8>
+__device__ __forceinline__ void decode_split_body(const CUtensorMap* tm_q_p,
+                                                  const CUtensorMap* tm_kv_p,
+                                                  const DecodeParams& p, int sp, int hg, int b,
+                                                  size_t cta, int phys_a, int phys_b, int valid_a,
+                                                  int valid_b) {
+  using Lay = DecodeLayout;
+  const CUtensorMap& tm_q = *tm_q_p;
+  const CUtensorMap& tm_kv = *tm_kv_p;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool two = phys_b >= 0;
 
   extern __shared__ uint8_t smem_raw[];
@@ -305,6 +416,7 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(bar(Lay::B_XCHG), 256);
     mbar_init(bar(Lay::B_O_FULL), 1);
     mbar_init(bar(Lay::B_O_EMPTY), 256);
+    mbar_init(bar(Lay::B_KA_FREE), 1);
     mbar_init(bar(Lay::B_DRAIN), 1);
     if (FP8) {
       for (int s = 0; s < Lay::NST; ++s) mbar_init(bar(Lay::B_CONV + s), 256);
@@ -376,8 +488,9 @@ __global__ void __launch_bounds__(320, 1)
         }
         if (issued < Lay::KV_CH) break;
         // V columns 0..255 (boxes 0..3) again: page A's into the Q slots, free
-        // once S is done; page B's into the K_B slots, free once O half 1
-        // (which reads boxes 4..7 there) is done.  Box e goes to stage e.
+        // once S is done; page B's into the K_A slots, free once O half 1's
+        // page-A products (which read boxes 4..7 there) are done.  Box e goes
+        // to stage e.
         if (!mbar_wait(bar(Lay::B_S_FULL), 0, abort_flag, status, 1)) break;
         mbar_arrive_expect_tx(bar(Lay::B_VA_FULL), 4 * kbox);
         for (int e = 0; e < 4; ++e)
@@ -385,10 +498,10 @@ __global__ void __launch_bounds__(320, 1)
                       phys_a * 128);
         va = true;
         if (!two) break;
-        if (!mbar_wait(bar(Lay::B_O_FULL), 0, abort_flag, status, 1)) break;
+        if (!mbar_wait(bar(Lay::B_KA_FREE), 0, abort_flag, status, 1)) break;
         mbar_arrive_expect_tx(bar(Lay::B_VB_FULL), 4 * kbox);
         for (int e = 0; e < 4; ++e)
-          tma_load_2d(ring + e * Lay::STAGE + 2 * Lay::CHUNK + koff, &tm_kv, bar(Lay::B_VB_FULL),
+          tma_load_2d(ring + e * Lay::STAGE + Lay::CHUNK + koff, &tm_kv, bar(Lay::B_VB_FULL),
                       e * 64, phys_b * 128);
         vb = true;
       } while (false);
@@ -444,6 +557,7 @@ __global__ void __launch_bounds__(320, 1)
       if (ok) {  // half 1 (columns 256..511): the kept S stages
         tc_fence_after();
         pv_page(ring + Lay::CHUNK, 0, true);
+        mma_commit(bar(Lay::B_KA_FREE));  // the K_A slots may take page B's V boxes 0..3
         if (two) pv_page(ring + 2 * Lay::CHUNK, 128, false);
         mma_commit(bar(Lay::B_O_FULL));
         ok = mbar_wait(bar(Lay::B_VA_FULL), 0, abort_flag, status, 1) &&
@@ -456,7 +570,7 @@ __global__ void __launch_bounds__(320, 1)
         if (two && (ok = mbar_wait(bar(Lay::B_VB_FULL), 0, abort_flag, status, 1) &&
                          (!FP8 || mbar_wait(bar(Lay::B_VB_CONV), 0, abort_flag, status, 1)))) {
           tc_fence_after();
-          pv_page(ring + 2 * Lay::CHUNK, 128, false);
+          pv_page(ring + Lay::CHUNK, 128, false);
         }
         if (ok) mma_commit(bar(Lay::B_O_FULL));
       }
@@ -650,12 +764,13 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
         if constexpr (FP8) {
-          // page B's V columns 0..255, reloaded into the K_B slots once O half
-          // 1 is done, to bf16: boxes 2wg and 2wg+1 by warpgroup wg
+          // page B's V columns 0..255, reloaded into the K_A slots, to bf16
+          // (once O half 1 is done, so page A's boxes there are read): boxes
+          // 2wg and 2wg+1 by warpgroup wg
           if (n == 0 && two) {
             bool okv = mbar_wait(bar(Lay::B_VB_FULL), 0, abort_flag, status, 1);
             for (int e = 2 * wg; e < 2 * wg + 2 && okv; ++e)
-              okv = decode_expand_fp8_box(ring + e * Lay::STAGE + 2 * Lay::CHUNK, h, xp, xp_uses,
+              okv = decode_expand_fp8_box(ring + e * Lay::STAGE + Lay::CHUNK, h, xp, xp_uses,
                                           abort_flag, status);
             if (!(ok = okv)) break;
             fence_async_shared();

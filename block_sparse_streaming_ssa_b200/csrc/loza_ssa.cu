@@ -84,12 +84,13 @@ int device_info(DeviceInfo& out) {
   return LOZA_SSA_OK;
 }
 
-// 16-bit tensor map: dims {d0 (innermost), d1, d2}, box {64, 128, 1}, 128B swizzle.
+// 16-bit tensor map: dims {d0 (innermost), d1, d2}, box {64, box_rows, 1}, 128B swizzle.
 int make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, int rank,
-             CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+             CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+             cuuint32_t box_rows = 128) {
   cuuint64_t dims[3] = {d0, d1, d2};
   cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(map, dtype, (cuuint32_t)rank,
                         const_cast<void*>(base), dims, strides, box, estr,
@@ -174,67 +175,87 @@ int dispatch_prefill(int d_qk, int d_v, const void* q, const void* k, const void
 struct BwdWorkspace {
   size_t d_bytes, part_bytes;
 };
-BwdWorkspace bwd_workspace(long long planes, int L, int dim, int n_sink) {
+BwdWorkspace bwd_workspace(long long planes, int L, int d_qk, int d_v, int n_sink) {
   const int nb = (L + 127) / 128;
   const long long rows = planes * L;
   BwdWorkspace w;
   w.d_bytes = (size_t)(((rows * 4) + 255) / 256) * 256;
-  w.part_bytes = (size_t)planes * loza::bwd_sink_items(n_sink, nb) * 2 * 128 * dim * 4;
+  w.part_bytes = (size_t)planes * loza::bwd_sink_items(n_sink, nb) * 128 * (d_qk + d_v) * 4;
   return w;
+}
+
+bool bwd_dims_ok(int d_qk, int d_v) {
+  return (d_qk == 64 && d_v == 64) || (d_qk == 128 && d_v == 128) || (d_qk == 192 && d_v == 128);
 }
 
 // q_items / kv_items: the work-item counts (dense) or upper bounds on them
 // (packed: the kernels read the exact counts from the prefixes).
-template <int DIM>
+template <int DQK, int DV>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                loza::BwdParams prm, long long q_items, long long kv_items, cudaStream_t s,
                const DeviceInfo& dev) {
-  CUtensorMap mq, mk, mv, mdo;
+  // 128-row boxes for the dQ kernel and for K, V; the dK/dV kernel reads Q and
+  // dO in half-steps of 64 rows
+  CUtensorMap mq, mk, mv, mdo, mq64, mdo64;
   int rc;
   const uint64_t L = (uint64_t)prm.plane_rows, planes = (uint64_t)prm.planes;
-  if ((rc = make_map(&mq, q, DIM, L, planes, 3)) != LOZA_SSA_OK) return rc;
-  if ((rc = make_map(&mk, k, DIM, L, planes, 3)) != LOZA_SSA_OK) return rc;
-  if ((rc = make_map(&mv, v, DIM, L, planes, 3)) != LOZA_SSA_OK) return rc;
-  if ((rc = make_map(&mdo, dout, DIM, L, planes, 3)) != LOZA_SSA_OK) return rc;
+  const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if ((rc = make_map(&mq, q, DQK, L, planes, 3)) != LOZA_SSA_OK) return rc;
+  if ((rc = make_map(&mk, k, DQK, L, planes, 3)) != LOZA_SSA_OK) return rc;
+  if ((rc = make_map(&mv, v, DV, L, planes, 3)) != LOZA_SSA_OK) return rc;
+  if ((rc = make_map(&mdo, dout, DV, L, planes, 3)) != LOZA_SSA_OK) return rc;
+  if ((rc = make_map(&mq64, q, DQK, L, planes, 3, bf, 64)) != LOZA_SSA_OK) return rc;
+  if ((rc = make_map(&mdo64, dout, DV, L, planes, 3, bf, 64)) != LOZA_SSA_OK) return rc;
   const long long rows = (long long)prm.planes * prm.plane_rows;
   const int pre_grid = (int)std::min<long long>((rows + 63) / 64, (long long)dev.num_sms * 16);
-  loza::ssa_bwd_preprocess_kernel<DIM><<<pre_grid, 256, 0, s>>>(
+  loza::ssa_bwd_preprocess_kernel<DV><<<pre_grid, 256, 0, s>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout),
       const_cast<float*>(prm.dsum), rows);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "backward preprocess launch");
 
-  using LQ = loza::BwdDqLayout<DIM>;
-  if ((e = cudaFuncSetAttribute(loza::ssa_bwd_dq_kernel<DIM>,
+  using LQ = loza::BwdDqLayout<DQK, DV>;
+  if ((e = cudaFuncSetAttribute(loza::ssa_bwd_dq_kernel<DQK, DV>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, LQ::SMEM_BYTES)) !=
       cudaSuccess)
     return cuda_fail(e, "cudaFuncSetAttribute(backward dq)");
   if (q_items > 0)
-    loza::ssa_bwd_dq_kernel<DIM><<<(int)std::min<long long>(q_items, dev.num_sms),
-                                   loza::kBwdThreads, LQ::SMEM_BYTES, s>>>(mq, mk, mv, mdo, prm);
+    loza::ssa_bwd_dq_kernel<DQK, DV><<<(int)std::min<long long>(q_items, dev.num_sms),
+                                       loza::kBwdThreads, LQ::SMEM_BYTES, s>>>(mq, mk, mv, mdo,
+                                                                              prm);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward dq launch");
 
-  using LK = loza::BwdKvLayout<DIM>;
-  if ((e = cudaFuncSetAttribute(loza::ssa_bwd_dkdv_kernel<DIM>,
+  using LK = loza::BwdKvLayout<DQK, DV>;
+  if ((e = cudaFuncSetAttribute(loza::ssa_bwd_dkdv_kernel<DQK, DV>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, LK::SMEM_BYTES)) !=
       cudaSuccess)
     return cuda_fail(e, "cudaFuncSetAttribute(backward dkdv)");
   if (kv_items > 0)
-    loza::ssa_bwd_dkdv_kernel<DIM><<<(int)std::min<long long>(kv_items, dev.num_sms),
-                                     loza::kBwdThreads, LK::SMEM_BYTES, s>>>(mq, mk, mv, mdo, prm);
+    loza::ssa_bwd_dkdv_kernel<DQK, DV><<<(int)std::min<long long>(kv_items, dev.num_sms),
+                                         loza::kBwdThreads, LK::SMEM_BYTES, s>>>(
+        mq64, mk, mv, mdo64, prm);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward dkdv launch");
 
   if (prm.cu_seqlens == nullptr && prm.sink_items > 0) {
-    const long long quads = (long long)prm.planes * std::min(prm.n_sink, prm.nb) * 128 * (DIM / 4);
+    const long long quads =
+        (long long)prm.planes * std::min(prm.n_sink, prm.nb) * 128 * ((DQK + DV) / 4);
     const int red_grid = (int)std::min<long long>((quads + 255) / 256, (long long)dev.num_sms * 8);
-    loza::ssa_bwd_sink_reduce_kernel<DIM><<<red_grid, 256, 0, s>>>(prm);
+    loza::ssa_bwd_sink_reduce_kernel<DQK, DV><<<red_grid, 256, 0, s>>>(prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward reduce launch");
   } else if (prm.cu_seqlens != nullptr && prm.n_sink > 0) {
     // one column of CTAs per sequence; each walks its (head, sink block, row, 4 columns)
-    loza::ssa_bwd_sink_reduce_kernel<DIM><<<dim3(8, prm.n_seqs), 256, 0, s>>>(prm);
+    loza::ssa_bwd_sink_reduce_kernel<DQK, DV><<<dim3(8, prm.n_seqs), 256, 0, s>>>(prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward reduce launch");
   }
   return LOZA_SSA_OK;
+}
+
+int dispatch_bwd(int d_qk, const void* q, const void* k, const void* v, const void* o,
+                 const void* dout, const loza::BwdParams& prm, long long q_items,
+                 long long kv_items, cudaStream_t s, const DeviceInfo& dev) {
+  if (d_qk == 64) return launch_bwd<64, 64>(q, k, v, o, dout, prm, q_items, kv_items, s, dev);
+  if (d_qk == 128) return launch_bwd<128, 128>(q, k, v, o, dout, prm, q_items, kv_items, s, dev);
+  return launch_bwd<192, 128>(q, k, v, o, dout, prm, q_items, kv_items, s, dev);
 }
 
 bool prefill_dims_ok(int d_qk, int d_v) {
@@ -327,6 +348,47 @@ int static_scratch_address(void** out) {
   }
   *out = g_scratch_ptr[dev];
   return LOZA_SSA_OK;
+}
+
+// Largest cluster the decode split kernel is launched as: the in-kernel merge
+// takes up to 4 splits (8-CTA clusters of this kernel measured much slower
+// than the merge kernel: they schedule as fewer, later waves).
+constexpr int kMaxClusterSplits = loza::kClusterMergeMaxSplits;
+
+int dev_index() {
+  int dev = 0;
+  return cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices ? dev : 0;
+}
+
+// Whether a cluster of n CTAs of the decode split kernel (its shared memory,
+// one CTA per SM) can be resident on the device, asked once per (device,
+// kernel, n).
+int g_cluster_fit[kMaxDevices][2][kMaxClusterSplits + 1] = {};  // 0 unknown, 1 yes, 2 no
+
+bool cluster_fits(void (*split)(CUtensorMap, CUtensorMap, loza::DecodeParams), int n, int dev) {
+  const int kind = split == loza::ssa_decode_split_kernel<true> ? 1 : 0;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (g_cluster_fit[dev][kind][n]) return g_cluster_fit[dev][kind][n] == 1;
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(n, 1, 1);
+  cfg.blockDim = dim3(320);
+  cfg.dynamicSmemBytes = loza::DecodeLayout::SMEM_BYTES;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = n;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  const cudaError_t e = cudaOccupancyMaxActiveClusters(&clusters, split, &cfg);
+  if (e != cudaSuccess) cudaGetLastError();  // not an error of this call: use the merge kernel
+  const bool ok = e == cudaSuccess && clusters >= 1;
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_cluster_fit[dev][kind][n] = ok ? 1 : 2;
+  return ok;
 }
 
 // Split CTAs per (sequence, head group): listed pages taken two at a time.
@@ -536,10 +598,9 @@ int loza_ssa_prefill_host(const void* q, const void* k, const void* v, void* o, 
 
 size_t loza_ssa_prefill_bwd_workspace_size(int B, int H, int L, int d_qk, int d_v, int n_sink,
                                            int n_local) {
-  if (B < 1 || H < 1 || L < 1 || d_qk != d_v || (d_qk != 64 && d_qk != 128) || n_sink < 0 ||
-      n_local < 1)
+  if (B < 1 || H < 1 || L < 1 || !bwd_dims_ok(d_qk, d_v) || n_sink < 0 || n_local < 1)
     return 0;
-  const BwdWorkspace w = bwd_workspace((long long)B * H, L, d_qk, n_sink);
+  const BwdWorkspace w = bwd_workspace((long long)B * H, L, d_qk, d_v, n_sink);
   return w.d_bytes + w.part_bytes;
 }
 
@@ -550,7 +611,7 @@ int loza_ssa_prefill_bwd(const void* q, const void* k, const void* v, const void
                          loza_ssa_stream_t stream) {
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return LOZA_SSA_ERR_NULL;
   if (B < 1 || H < 1 || L < 1 || !std::isfinite(scale)) return LOZA_SSA_ERR_SHAPE;
-  if (d_qk != d_v || (d_qk != 64 && d_qk != 128)) return LOZA_SSA_ERR_HEAD_DIM;
+  if (!bwd_dims_ok(d_qk, d_v)) return LOZA_SSA_ERR_HEAD_DIM;
   if (block != 128) return LOZA_SSA_ERR_BLOCK;
   if (n_sink < 0 || n_local < 1) return LOZA_SSA_ERR_WINDOW;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
@@ -569,7 +630,7 @@ int loza_ssa_prefill_bwd(const void* q, const void* k, const void* v, const void
   DeviceInfo dev;
   int rc = device_info(dev);
   if (rc != LOZA_SSA_OK) return rc;
-  const BwdWorkspace w = bwd_workspace(planes, L, d_qk, n_sink);
+  const BwdWorkspace w = bwd_workspace(planes, L, d_qk, d_v, n_sink);
   loza::BwdParams prm{};
   prm.lse = lse;
   prm.dsum = reinterpret_cast<const float*>(workspace);
@@ -592,8 +653,7 @@ int loza_ssa_prefill_bwd(const void* q, const void* k, const void* v, const void
   const long long q_items = planes * nb;
   const long long kv_items = planes * (sink_items + (nb > n_sink ? nb - n_sink : 0));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d_qk == 64) return launch_bwd<64>(q, k, v, o, dout, prm, q_items, kv_items, s, dev);
-  return launch_bwd<128>(q, k, v, o, dout, prm, q_items, kv_items, s, dev);
+  return dispatch_bwd(d_qk, q, k, v, o, dout, prm, q_items, kv_items, s, dev);
 }
 
 // Packed backward workspace: D per row, the three prefixes, then the sink
@@ -605,8 +665,8 @@ struct BwdVarlenWorkspace {
   size_t d_bytes, pfx_bytes, part_bytes;
   long long q_items_upper, kv_items_upper, sink_slots;
 };
-BwdVarlenWorkspace bwd_varlen_workspace(int n_seqs, int total, int max_seqlen, int H, int dim,
-                                        int n_sink, int n_local) {
+BwdVarlenWorkspace bwd_varlen_workspace(int n_seqs, int total, int max_seqlen, int H, int d_qk,
+                                        int d_v, int n_sink, int n_local) {
   (void)n_local;
   BwdVarlenWorkspace w;
   (void)max_seqlen;
@@ -615,7 +675,7 @@ BwdVarlenWorkspace bwd_varlen_workspace(int n_seqs, int total, int max_seqlen, i
       (long long)H * n_sink * ((sum_nb + 7 * (long long)n_seqs) / 8 + n_seqs);
   w.d_bytes = (size_t)((((long long)H * total * 4) + 255) / 256) * 256;
   w.pfx_bytes = (size_t)((3 * ((long long)n_seqs + 1) * 4 + 255) / 256) * 256;
-  w.part_bytes = (size_t)sink_slots * 2 * 128 * dim * 4;
+  w.part_bytes = (size_t)sink_slots * 128 * (d_qk + d_v) * 4;
   w.q_items_upper = (long long)H * sum_nb;
   w.kv_items_upper = w.q_items_upper + sink_slots;
   w.sink_slots = sink_slots;
@@ -626,10 +686,10 @@ size_t loza_ssa_prefill_varlen_bwd_workspace_size(int n_seqs, int total_tokens, 
                                                   int H, int d_qk, int d_v, int n_sink,
                                                   int n_local) {
   if (n_seqs < 1 || n_seqs > kMaxVarlenSeqs || total_tokens < 1 || max_seqlen < 1 || H < 1 ||
-      d_qk != d_v || (d_qk != 64 && d_qk != 128) || n_sink < 0 || n_local < 1)
+      !bwd_dims_ok(d_qk, d_v) || n_sink < 0 || n_local < 1)
     return 0;
   const BwdVarlenWorkspace w =
-      bwd_varlen_workspace(n_seqs, total_tokens, max_seqlen, H, d_qk, n_sink, n_local);
+      bwd_varlen_workspace(n_seqs, total_tokens, max_seqlen, H, d_qk, d_v, n_sink, n_local);
   return w.d_bytes + w.pfx_bytes + w.part_bytes;
 }
 
@@ -644,7 +704,7 @@ int loza_ssa_prefill_varlen_bwd(const void* q, const void* k, const void* v, con
   if (n_seqs < 1 || n_seqs > kMaxVarlenSeqs || total_tokens < 1 || max_seqlen < 1 || H < 1 ||
       !std::isfinite(scale))
     return LOZA_SSA_ERR_SHAPE;
-  if (d_qk != d_v || (d_qk != 64 && d_qk != 128)) return LOZA_SSA_ERR_HEAD_DIM;
+  if (!bwd_dims_ok(d_qk, d_v)) return LOZA_SSA_ERR_HEAD_DIM;
   if (block != 128) return LOZA_SSA_ERR_BLOCK;
   if (n_sink < 0 || n_local < 1) return LOZA_SSA_ERR_WINDOW;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
@@ -652,7 +712,7 @@ int loza_ssa_prefill_varlen_bwd(const void* q, const void* k, const void* v, con
       !aligned(lse, 4) || !aligned(cu_seqlens, 4))
     return LOZA_SSA_ERR_ALIGN;
   const BwdVarlenWorkspace w =
-      bwd_varlen_workspace(n_seqs, total_tokens, max_seqlen, H, d_qk, n_sink, n_local);
+      bwd_varlen_workspace(n_seqs, total_tokens, max_seqlen, H, d_qk, d_v, n_sink, n_local);
   if (w.kv_items_upper >= (1ll << 31)) return LOZA_SSA_ERR_SHAPE;
   const size_t need = w.d_bytes + w.pfx_bytes + w.part_bytes;
   if (!workspace || workspace_bytes < need) return LOZA_SSA_ERR_WORKSPACE;
@@ -684,9 +744,7 @@ int loza_ssa_prefill_varlen_bwd(const void* q, const void* k, const void* v, con
                                                         n_sink, w.sink_slots, pfx);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "backward varlen setup launch");
-  if (d_qk == 64)
-    return launch_bwd<64>(q, k, v, o, dout, prm, w.q_items_upper, w.kv_items_upper, s, dev);
-  return launch_bwd<128>(q, k, v, o, dout, prm, w.q_items_upper, w.kv_items_upper, s, dev);
+  return dispatch_bwd(d_qk, q, k, v, o, dout, prm, w.q_items_upper, w.kv_items_upper, s, dev);
 }
 
 int loza_ssa_prefill_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -846,6 +904,29 @@ int decode_impl(const void* q, const void* paged_kv, const int* page_table, cons
                                        loza::DecodeLayout::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
   dim3 grid(n_split, HG, B);
+  // Up to 8 splits per (row, head group): launch them as one cluster, which
+  // merges its partials itself (the cluster's CTAs are resident together, so
+  // they can wait for each other); more splits (long windows) go through the
+  // merge kernel.
+  if (n_split <= kMaxClusterSplits && cluster_fits(split, n_split, dev_index())) {
+    prm.cluster_merge = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(320);
+    cfg.dynamicSmemBytes = loza::DecodeLayout::SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = n_split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if ((e = cudaLaunchKernelEx(&cfg, split, mq, mkv, prm)) != cudaSuccess)
+      return cuda_fail(e, "decode split launch (cluster)");
+    return LOZA_SSA_OK;
+  }
+  prm.cluster_merge = 0;
   split<<<grid, 320, loza::DecodeLayout::SMEM_BYTES, s>>>(mq, mkv, prm);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "decode split launch");
   // the merge is a programmatic dependent of the split kernel: it is scheduled

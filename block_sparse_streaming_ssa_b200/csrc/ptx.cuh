@@ -114,7 +114,25 @@ __device__ __forceinline__ void drain_ring(uint32_t full_bar0, int stages, int i
   }
 }
 
+// ------------------------------------------------------------------ cluster
+
+// Every thread of every CTA in the cluster arrives; the release makes this
+// thread's earlier writes (shared and global) visible to the cluster's
+// threads that acquire at the matching wait.
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
 // ---------------------------------------------------------------------- TMA
+
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -139,9 +139,10 @@ int loza_ssa_prefill_varlen(const void* q, const void* k, const void* v, void* o
  * over the same SSA key sets J(i) as the forward pass, with
  * P_ij = exp(scale q_i.k_j - lse_i) -- the chain rule applied to the masked
  * softmax attention of "LoZA：ZigZag稀疏注意力机制" §2.1.
- *   q, k, dq, dk : bf16 [B, H, L, d]     v, o, dout, dv : bf16 [B, H, L, d]
+ *   q, k, dq, dk : bf16 [B, H, L, d_qk]  v, o, dout, dv : bf16 [B, H, L, d_v]
  *   lse          : fp32 [B, H, L] as written by loza_ssa_prefill
- *   d_qk == d_v in {64, 128}; block must be 128.
+ *   (d_qk, d_v) in {(64,64), (128,128), (192,128)} (the last: the MLA head
+ *   dims of the layers LoZA converts); block must be 128.
  *   workspace    : DEVICE scratch of at least
  *                  loza_ssa_prefill_bwd_workspace_size(...) bytes, 256-byte
  *                  aligned, owned by the caller, contents irrelevant on entry.
@@ -164,9 +165,10 @@ size_t loza_ssa_prefill_bwd_workspace_size(int B, int H, int L, int d_qk, int d_
  * gradients).  Every sequence is its own attention problem: its gradients are
  * those of the dense backward over its slice, and no key of one sequence
  * reaches another's.
- *   q, k, dq, dk : bf16 [H, total_tokens, d]   v, o, dout, dv : bf16 [H, total_tokens, d]
- *   lse          : fp32 [H, total_tokens]      cu_seqlens     : DEVICE int32 [n_seqs + 1]
- *   1 <= n_seqs <= 4000; d_qk == d_v in {64, 128}; max_seqlen only has to be >= 1.
+ *   q, k, dq, dk : bf16 [H, total_tokens, d_qk]  v, o, dout, dv : bf16 [H, total_tokens, d_v]
+ *   lse          : fp32 [H, total_tokens]         cu_seqlens     : DEVICE int32 [n_seqs + 1]
+ *   1 <= n_seqs <= 4000; (d_qk, d_v) as for loza_ssa_prefill_bwd; max_seqlen
+ *   only has to be >= 1.
  *   workspace    : DEVICE scratch of at least
  *                  loza_ssa_prefill_varlen_bwd_workspace_size(...) bytes,
  *                  256-byte aligned, owned by the caller.

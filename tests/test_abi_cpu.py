@@ -108,14 +108,18 @@ def test_prefill_bwd_workspace_size(L):
     B, H, L, d = 1, 2, 4096, 128
     rows = B * H * L
     d_bytes = -(-rows * 4 // 256) * 256
-    part = B * H * 4 * 2 * 128 * d * 4
+    part = B * H * 4 * 128 * (d + d) * 4
     assert api.loza_ssa_prefill_bwd_workspace_size(B, H, L, d, d, 1, 7) == d_bytes + part
     # no sink blocks: no partials
     assert api.loza_ssa_prefill_bwd_workspace_size(B, H, L, d, d, 0, 7) == d_bytes
     # two sink blocks: 32 - 0 and 32 - 1 query blocks -> 4 + 4 chunks
     assert api.loza_ssa_prefill_bwd_workspace_size(B, H, L, d, d, 2, 7) == d_bytes + 2 * part
+    # the MLA head dims: a partial holds dK (192 columns) and dV (128 columns)
+    assert api.loza_ssa_prefill_bwd_workspace_size(B, H, L, 192, 128, 1, 7) == \
+        d_bytes + B * H * 4 * 128 * (192 + 128) * 4
     # unsupported head dims / windows
-    assert api.loza_ssa_prefill_bwd_workspace_size(B, H, L, 192, 128, 1, 7) == 0
+    assert api.loza_ssa_prefill_bwd_workspace_size(B, H, L, 192, 192, 1, 7) == 0
+    assert api.loza_ssa_prefill_bwd_workspace_size(B, H, L, 128, 64, 1, 7) == 0
     assert api.loza_ssa_prefill_bwd_workspace_size(B, H, L, 128, 128, 1, 0) == 0
 
 
@@ -129,7 +133,8 @@ def test_prefill_bwd_rejects_bad_arguments(L):
                                       n_local, ctypes.c_float(0.08), a, ws_bytes, None)
     assert call(ptr=None) == -1           # LOZA_SSA_ERR_NULL
     assert call(B=0) == -2                # LOZA_SSA_ERR_SHAPE
-    assert call(dqk=192) == -3            # LOZA_SSA_ERR_HEAD_DIM
+    assert call(dqk=192, dv=192) == -3    # LOZA_SSA_ERR_HEAD_DIM
+    assert call(dqk=64, dv=128) == -3
     assert call(block=64) == -4           # LOZA_SSA_ERR_BLOCK
     assert call(n_local=0) == -5          # LOZA_SSA_ERR_WINDOW
     assert call(ptr=vp(0x1002)) == -6     # LOZA_SSA_ERR_ALIGN
@@ -144,24 +149,28 @@ def test_prefill_varlen_bwd_workspace_size(L):
     d_bytes = -(-H * total * 4 // 256) * 256
     pfx = -(-3 * (n + 1) * 4 // 256) * 256
     slots = H * 1 * ((total // 128 + n + 7 * n) // 8 + n)
-    want = d_bytes + pfx + slots * 2 * 128 * d * 4
+    want = d_bytes + pfx + slots * 128 * (d + d) * 4
     assert api.loza_ssa_prefill_varlen_bwd_workspace_size(n, total, 4000, H, d, d, 1, 7) == want
     assert api.loza_ssa_prefill_varlen_bwd_workspace_size(n, total, 4000, H, d, d, 0, 7) == \
         d_bytes + pfx
     assert api.loza_ssa_prefill_varlen_bwd_workspace_size(4001, total, 10, H, d, d, 1, 7) == 0
-    assert api.loza_ssa_prefill_varlen_bwd_workspace_size(n, total, 4000, H, 192, 128, 1, 7) == 0
+    assert api.loza_ssa_prefill_varlen_bwd_workspace_size(n, total, 4000, H, 192, 128, 1, 7) == \
+        d_bytes + pfx + slots * 128 * (192 + 128) * 4
+    assert api.loza_ssa_prefill_varlen_bwd_workspace_size(n, total, 4000, H, 192, 192, 1, 7) == 0
 
 
 def test_prefill_varlen_bwd_rejects_bad_arguments(L):
     vp = ctypes.c_void_p
     a = vp(0x1000)
 
-    def call(n=2, total=300, H=2, d=64, cu=a, ws_bytes=1 << 30):
-        return L.loza_ssa_prefill_varlen_bwd(a, a, a, a, a, a, a, a, a, cu, n, total, 200, H, d, d,
-                                             128, 1, 7, ctypes.c_float(0.1), a, ws_bytes, None)
+    def call(n=2, total=300, H=2, d=64, dv=None, cu=a, ws_bytes=1 << 30):
+        return L.loza_ssa_prefill_varlen_bwd(a, a, a, a, a, a, a, a, a, cu, n, total, 200, H, d,
+                                             d if dv is None else dv, 128, 1, 7,
+                                             ctypes.c_float(0.1), a, ws_bytes, None)
     assert call(cu=None) == -1            # LOZA_SSA_ERR_NULL
     assert call(n=0) == -2                # LOZA_SSA_ERR_SHAPE
-    assert call(d=192) == -3              # LOZA_SSA_ERR_HEAD_DIM
+    assert call(d=192) == -3              # LOZA_SSA_ERR_HEAD_DIM (192 / 192)
+    assert call(d=128, dv=64) == -3
     assert call(cu=vp(0x1002)) == -6      # LOZA_SSA_ERR_ALIGN
     assert call(ws_bytes=8) == -7         # LOZA_SSA_ERR_WORKSPACE
 

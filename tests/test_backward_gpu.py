@@ -30,10 +30,11 @@ def grad_errors(got, ref):
     return rel, frac
 
 
-def run(B, H, L, d, seed=0, n_sink=1, n_local=7):
-    q, k, v = synth.prefill_inputs(B, H, L, d, d, seed=seed, device="cuda")
+def run(B, H, L, d, seed=0, n_sink=1, n_local=7, dv=None):
+    dv = d if dv is None else dv
+    q, k, v = synth.prefill_inputs(B, H, L, d, dv, seed=seed, device="cuda")
     g = torch.Generator(device="cuda").manual_seed(seed + 77)
-    dout = torch.randn((B, H, L, d), generator=g, device="cuda").to(torch.bfloat16)
+    dout = torch.randn((B, H, L, dv), generator=g, device="cuda").to(torch.bfloat16)
     scale = 1.0 / np.sqrt(d)
     o, lse = loza_ssa_prefill(q, k, v, n_sink=n_sink, n_local=n_local, scale=scale)
     dq, dk, dv = loza_ssa_prefill_bwd(q, k, v, o, lse, dout, n_sink=n_sink, n_local=n_local,
@@ -64,6 +65,22 @@ def test_backward_matches_oracle(B, H, L, d):
     check(got, ref, f"bwd B={B} H={H} L={L} d={d}")
 
 
+@pytest.mark.parametrize("B,H,L", [(1, 2, 2048), (1, 2, 1000), (2, 1, 300), (1, 1, 100),
+                                   (1, 2, 4096)])
+def test_backward_mla_dims(B, H, L):
+    """d_qk = 192 (128 latent + 64 rope), d_v = 128, the head dims of the MLA
+    layers LoZA converts in mid-training: several tiles, ragged tails, and a
+    sink block split into four chunks (L = 4096)."""
+    got, ref = run(B, H, L, 192, seed=L + 192, dv=128)
+    check(got, ref, f"bwd B={B} H={H} L={L} d=192/128")
+
+
+@pytest.mark.parametrize("n_sink,n_local", [(0, 2), (2, 3)])
+def test_backward_mla_dims_window_shapes(n_sink, n_local):
+    got, ref = run(1, 2, 1700, 192, seed=13, n_sink=n_sink, n_local=n_local, dv=128)
+    check(got, ref, f"bwd d=192/128 sink={n_sink} local={n_local}")
+
+
 @pytest.mark.parametrize("n_sink,n_local", [(0, 1), (2, 3), (0, 4), (3, 12)])
 def test_backward_window_shapes(n_sink, n_local):
     got, ref = run(1, 2, 2000, 64, seed=5, n_sink=n_sink, n_local=n_local)
@@ -84,12 +101,13 @@ def test_backward_is_deterministic():
 
 # --- packed variable-length sequences
 
-def run_varlen(lengths, H, d, seed=0, n_sink=1, n_local=7):
+def run_varlen(lengths, H, d, seed=0, n_sink=1, n_local=7, dv=None):
     from block_sparse_streaming_ssa_b200.loza_ssa import (loza_ssa_prefill_varlen,
                                                           loza_ssa_prefill_varlen_bwd)
-    q, k, v, cu = synth.varlen_inputs(lengths, H, d, d, seed=seed, device="cuda")
+    q, k, v, cu = synth.varlen_inputs(lengths, H, d, d if dv is None else dv, seed=seed,
+                                      device="cuda")
     g = torch.Generator(device="cuda").manual_seed(seed + 99)
-    dout = torch.randn(q.shape, generator=g, device="cuda").to(torch.bfloat16)
+    dout = torch.randn(v.shape, generator=g, device="cuda").to(torch.bfloat16)
     scale = 1.0 / np.sqrt(d)
     o, lse = loza_ssa_prefill_varlen(q, k, v, cu, max(lengths), n_sink=n_sink, n_local=n_local,
                                      scale=scale)
@@ -110,6 +128,13 @@ def test_backward_varlen_matches_oracle(lengths, d):
     sequences, and a 4096-token sequence whose sink block is split in chunks."""
     got, ref = run_varlen(lengths, 2, d, seed=len(lengths) + d)
     check(got, ref, f"varlen bwd {lengths} d={d}")
+
+
+@pytest.mark.parametrize("lengths", [[1000, 70, 2048, 1], [300, 4096, 129]])
+def test_backward_varlen_mla_dims(lengths):
+    """Packed sequences at d_qk = 192, d_v = 128."""
+    got, ref = run_varlen(lengths, 2, 192, seed=len(lengths) + 192, dv=128)
+    check(got, ref, f"varlen bwd {lengths} d=192/128")
 
 
 @pytest.mark.parametrize("n_sink,n_local", [(0, 2), (2, 3)])
