@@ -22,7 +22,12 @@
 namespace {
 
 constexpr int kVersion = 10000;  // 1.0.0
-constexpr int kMaxVarlenSeqs = 4000;  // keeps the d_qk=192 layout within 227 KB
+constexpr int kMaxVarlenSeqs = 4000;
+// The packed prefill keeps a prefix per sequence in shared memory; beside the
+// d_qk = 192 rings that leaves room for this many sequences.
+constexpr int kMaxVarlenSeqsDqk192 = 3000;
+static_assert(kMaxVarlenSeqsDqk192 + 1 <= loza::PrefillLayout<192, 128>::MAX_PREFIX, "smem");
+static_assert(kMaxVarlenSeqs + 1 <= loza::PrefillLayout<128, 128>::MAX_PREFIX, "smem");
 constexpr int kMaxDecodeWindow = 4096;
 constexpr int kMaxDevices = 64;
 
@@ -142,7 +147,7 @@ int launch_prefill(const void* q, const void* k, const void* v, loza::PrefillPar
     prm.total_items = (int)items_upper;
   }
   const size_t smem = Lay::smem_bytes(n_prefix);
-  const size_t smem_max = Lay::smem_bytes(kMaxVarlenSeqs + 1);
+  const size_t smem_max = Lay::smem_bytes((DQK == 192 ? kMaxVarlenSeqsDqk192 : kMaxVarlenSeqs) + 1);
   void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, loza::PrefillParams) =
       loza::ssa_prefill_kernel<DQK, DV>;
   cudaError_t e =
@@ -756,6 +761,7 @@ int loza_ssa_prefill_varlen(const void* q, const void* k, const void* v, void* o
       !std::isfinite(scale))
     return LOZA_SSA_ERR_SHAPE;
   if (!prefill_dims_ok(d_qk, d_v)) return LOZA_SSA_ERR_HEAD_DIM;
+  if (d_qk == 192 && n_seqs > kMaxVarlenSeqsDqk192) return LOZA_SSA_ERR_SHAPE;
   if (block != 128) return LOZA_SSA_ERR_BLOCK;
   if (n_sink < 0 || n_local < 1) return LOZA_SSA_ERR_WINDOW;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 32) ||

@@ -102,7 +102,7 @@ struct PrefillLayout {
   static constexpr int V_BYTES = VCH * CHUNK;
   // Q ring depth: one stage measured as fast as two (the S issuer runs ahead of
   // the softmax by two tiles, which covers the next item's Q load)
-  static constexpr int QST = 1;
+  static constexpr int QST = DQK <= 64 ? 2 : 1;
   static constexpr int KST = 2;                   // K ring depth
   static constexpr int VST = 2;                   // V ring depth
   static constexpr int NSB = 3;                   // S buffers in TMEM (128 columns each)
@@ -112,12 +112,15 @@ struct PrefillLayout {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + QST * Q_BYTES;
   static constexpr int OFF_V = OFF_K + KST * K_BYTES;
-  // d_qk = d_v = 128: O goes out through TMA stores from a staging buffer
-  // (one swizzled [128 rows x 64 columns] box per softmax warpgroup); the
-  // other head dims write O from registers.
-  static constexpr bool TMA_OUT = DQK == 128 && DV == 128;
+  // O goes out through TMA stores from a staging area: a buffer of its own
+  // where one fits beside the rings (d_qk <= 128), else the V ring slot of the
+  // item's last key tile (d_qk = 192), which that tile's P.V has read by the
+  // time O is final and which is handed back to the V producer once the stores
+  // have read it (holding a V slot measured slower where a buffer fits).
+  static constexpr bool TMA_OUT = true;
+  static constexpr bool OWN_STAGE = DQK <= 128;
   static constexpr int OFF_OST = OFF_V + VST * V_BYTES;
-  static constexpr int OFF_BAR = OFF_OST + (TMA_OUT ? VCH * CHUNK : 0);
+  static constexpr int OFF_BAR = OFF_OST + (OWN_STAGE ? VCH * CHUNK : 0);
   // barrier indices
   static constexpr int B_Q_FULL = 0, B_Q_EMPTY = B_Q_FULL + QST;
   static constexpr int B_K_FULL = B_Q_EMPTY + QST, B_K_EMPTY = B_K_FULL + KST;
@@ -135,10 +138,10 @@ struct PrefillLayout {
   // per pair of warps (w, w + 4) that share TMEM lanes)
   static constexpr int B_OST_FULL = B_DRAIN + 2;    // 2, per warpgroup: box written (128)
   static constexpr int B_OST_FREE = B_OST_FULL + 2; // 2, per warpgroup: box read by its store
-  // With an epilogue warpgroup (d_qk = d_v = 128): the softmax warps hand each
-  // item's row max and row sums over in shared memory and go on to the next
-  // item; warps 12-15 normalise O and store it.
-  static constexpr bool EPI_WG = TMA_OUT;
+  // With an epilogue warpgroup: the softmax warps hand each item's row max
+  // and row sums over in shared memory and go on to the next item; warps
+  // 12-15 normalise O and store it.
+  static constexpr bool EPI_WG = true;
   static constexpr int THREADS = EPI_WG ? 512 : 384;
   static constexpr int B_O_FULL = B_OST_FREE + 2;    // NOB: the item's last P.V done (commit)
   static constexpr int B_ROWS_FULL = B_O_FULL + NOB; // 2: rows published (256)
@@ -152,6 +155,8 @@ struct PrefillLayout {
   static_assert(NBAR * 8 <= BAR_BYTES, "barrier area");
   static constexpr int TMEM_COLS = 512;
   static constexpr int MIN_SMEM = 120 * 1024;  // keeps one CTA (and one TMEM owner) per SM
+  // largest prefix (sequences + 1) that fits the 227 KB of shared memory
+  static constexpr int MAX_PREFIX = (227 * 1024 - 1024 - OFF_PREFIX) / 4;
   static constexpr size_t smem_bytes(int n_prefix) {
     size_t need = (size_t)OFF_PREFIX + 4 * (size_t)n_prefix + 1024;  // + alignment slack
     return need < (size_t)MIN_SMEM ? (size_t)MIN_SMEM : need;
@@ -470,7 +475,9 @@ __global__ void __launch_bounds__(PrefillLayout<DQK, DV>::THREADS, 1)
                 sb + Lay::OFF_V + st * Lay::V_BYTES + kk * 2048, Lay::CHUNK, 1024);
             mma_ts(o_tmem, p_tmem + kk * 8, bdesc, id_o, (t > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(bar(Lay::B_V_EMPTY + st));
+          // without a staging buffer the item's last V slot stages O: the
+          // epilogue warpgroup frees it
+          if (Lay::OWN_STAGE || t != tr.count - 1) mma_commit(bar(Lay::B_V_EMPTY + st));
           mma_commit(bar(Lay::B_S_FREE + sbuf));
           if (Lay::EPI_WG && t == tr.count - 1) mma_commit(bar(Lay::B_O_FULL + ob));
         }
@@ -487,11 +494,14 @@ __global__ void __launch_bounds__(PrefillLayout<DQK, DV>::THREADS, 1)
     const int row = threadIdx.x - 12 * 32;                        // query row = TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const float* rows_all = reinterpret_cast<const float*>(smem + Lay::OFF_ROWS);
-    int it = 0, n_out = 0;
+    int it = 0, n_out = 0, g = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++it) {
       const WorkItem w = decode_item(item, p, prefix);
       const int pr = it & 1, ob = it % Lay::NOB;
+      g += tile_range(w.qb, p.n_sink, p.n_local).count;
+      const int v_slot = (g - 1) % Lay::VST;  // V slot of the item's last tile
+      uint8_t* stage = smem + (Lay::OWN_STAGE ? Lay::OFF_OST : Lay::OFF_V + v_slot * Lay::V_BYTES);
       if (!mbar_wait(bar(Lay::B_ROWS_FULL + pr), (it >> 1) & 1, abort_flag, status, 1)) break;
       const float* rows = rows_all + pr * 384;
       const float m = rows[row];
@@ -506,7 +516,9 @@ __global__ void __launch_bounds__(PrefillLayout<DQK, DV>::THREADS, 1)
       // dense rows past L fall outside the tensor map and are not written; a
       // packed sequence's last block would spill into the next sequence
       const bool tma_out = p.cu_seqlens == nullptr || (w.qb + 1) * 128 <= w.len;
-      if (tma_out && n_out > 0 &&
+      // an own staging buffer: the previous store has read it (its issuer checks,
+      // then tells the rest)
+      if (Lay::OWN_STAGE && tma_out && n_out > 0 &&
           !mbar_wait(bar(Lay::B_OST_FREE), (n_out - 1) & 1, abort_flag, status, 1))
         break;
 #pragma unroll 1
@@ -522,7 +534,7 @@ __global__ void __launch_bounds__(PrefillLayout<DQK, DV>::THREADS, 1)
         if (tma_out) {
           // row `row` of box q4/2 in the 128B-swizzled layout the tensor map
           // reads: 16-byte unit j at j ^ (row & 7)
-          uint8_t* rowp = smem + Lay::OFF_OST + (q4 >> 1) * Lay::CHUNK + row * 128;
+          uint8_t* rowp = stage + (q4 >> 1) * Lay::CHUNK + row * 128;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int j = (q4 & 1) * 4 + u;
@@ -553,14 +565,17 @@ __global__ void __launch_bounds__(PrefillLayout<DQK, DV>::THREADS, 1)
           if (!(ok = mbar_wait(bar(Lay::B_OST_FULL), n_out & 1, abort_flag, status, 1))) break;
 #pragma unroll
           for (int hh = 0; hh < Lay::VCH; ++hh)
-            tma_store_3d(&tm_o, sb + Lay::OFF_OST + hh * Lay::CHUNK, hh * 64,
+            tma_store_3d(&tm_o, smem_u32(stage) + hh * Lay::CHUNK, hh * 64,
                          w.seq_start + w.qb * 128, w.z);
           tma_store_commit();
-          // the boxes may be rewritten once these stores have read them
+          // the staging may be rewritten (own buffer) or refilled by the V
+          // producer (V slot) once these stores have read it
           tma_store_wait_read();
-          mbar_arrive(bar(Lay::B_OST_FREE));
+          mbar_arrive(bar(Lay::OWN_STAGE ? Lay::B_OST_FREE : Lay::B_V_EMPTY + v_slot));
         }
         ++n_out;
+      } else if (!Lay::OWN_STAGE && row == 0) {
+        mbar_arrive(bar(Lay::B_V_EMPTY + v_slot));  // nothing staged: the slot is free
       }
       if (valid) p.lse[orow] = (m + __log2f(l_row)) * kLn2;
     }
@@ -588,95 +603,6 @@ __global__ void __launch_bounds__(PrefillLayout<DQK, DV>::THREADS, 1)
       named_bar_sync(1 + (warp & 3), 64);
       other = buf[(wg ^ 1) * 128 + row];
       ++xc;
-      return true;
-    };
-    // The epilogue of an item runs after the next item's first tile has been
-    // handed to the P.V issuer: by then the item's last P.V has finished, so
-    // the wait for it is off the softmax's path.
-    struct Done {
-      WorkItem w;
-      float m, l;  // running max (log2 units) and this half's row sum
-      int ob, gl;  // O buffer, global index of the item's last tile
-    };
-    Done prev{};
-    bool have_prev = false;
-    int n_out = 0;  // TMA-store epilogues this warpgroup has done
-    auto epilogue = [&](const Done& d) -> bool {
-      // O = acc / l (bf16), LSE = (m + log2 l) ln 2
-      float l_other;
-      if (!exchange(d.l, l_other)) return false;
-      const float l_row = d.l + l_other;
-      if (!mbar_wait(bar(Lay::B_S_FREE + d.gl % Lay::NSB), (d.gl / Lay::NSB) & 1, abort_flag,
-                     status, 1))
-        return false;
-      tc_fence_after();
-      const uint32_t o_tmem = tmem + lane_base + Lay::TM_O + d.ob * DV + wg * OH;
-      const int r_in_seq = d.w.qb * 128 + row;
-      const bool valid = r_in_seq < d.w.len;
-      const size_t orow =
-          (size_t)d.w.z * (size_t)p.plane_rows + (size_t)(d.w.seq_start + r_in_seq);
-      const float inv_l = 1.f / l_row;
-      uint32_t orr[OH / 32][32];
-#pragma unroll
-      for (int ch = 0; ch < OH / 32; ++ch) tmem_ld32(o_tmem + ch * 32, orr[ch]);
-      tmem_wait_ld();
-      // O buffer free for the item NOB after this one
-      tc_fence_before();
-      mbar_arrive(bar(Lay::B_O_EMPTY + d.ob));
-      // Dense rows past L fall outside the tensor map and are not written; a
-      // packed sequence's last block would spill into the next sequence, so
-      // it keeps the register path.
-      const bool tma_out =
-          Lay::TMA_OUT && (p.cu_seqlens == nullptr || (d.w.qb + 1) * 128 <= d.w.len);
-      if (tma_out) {
-        const uint32_t box = sb + Lay::OFF_OST + wg * Lay::CHUNK;
-        if (n_out > 0) {
-          // the box's previous store has read it (its issuer checks, then tells the rest)
-          if (row == 0) {
-            tma_store_wait_read();
-            mbar_arrive(bar(Lay::B_OST_FREE + wg));
-          }
-          if (!mbar_wait(bar(Lay::B_OST_FREE + wg), (n_out - 1) & 1, abort_flag, status, 1))
-            return false;
-        }
-        // row `row` of the box in the 128B-swizzled layout the tensor map reads:
-        // 16-byte unit j at j ^ (row & 7)
-        uint8_t* rowp = smem + Lay::OFF_OST + wg * Lay::CHUNK + row * 128;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint32_t* r8 = &orr[j >> 2][(j & 3) * 8];
-          *reinterpret_cast<uint4*>(rowp + ((j ^ (row & 7)) << 4)) =
-              make_uint4(pack_bf16x2(__uint_as_float(r8[0]) * inv_l, __uint_as_float(r8[1]) * inv_l),
-                         pack_bf16x2(__uint_as_float(r8[2]) * inv_l, __uint_as_float(r8[3]) * inv_l),
-                         pack_bf16x2(__uint_as_float(r8[4]) * inv_l, __uint_as_float(r8[5]) * inv_l),
-                         pack_bf16x2(__uint_as_float(r8[6]) * inv_l, __uint_as_float(r8[7]) * inv_l));
-        }
-        fence_async_shared();
-        mbar_arrive(bar(Lay::B_OST_FULL + wg));
-        if (row == 0) {
-          if (!mbar_wait(bar(Lay::B_OST_FULL + wg), n_out & 1, abort_flag, status, 1)) return false;
-          tma_store_3d(&tm_o, box, wg * 64, d.w.seq_start + d.w.qb * 128, d.w.z);
-          tma_store_commit();
-        }
-        ++n_out;
-        if (valid && wg == 0) p.lse[orow] = (d.m + __log2f(l_row)) * kLn2;
-      } else if (valid) {
-        uint4* dst = reinterpret_cast<uint4*>(p.o + orow * DV + wg * OH);
-        // 32-byte stores: each writes a whole L2 sector (16-byte stores left
-        // half sectors per instruction and measured ~4-7 % slower overall)
-#pragma unroll
-        for (int ch = 0; ch < OH / 32; ++ch)
-#pragma unroll
-          for (int v = 0; v < 4; v += 2) {
-            uint32_t w8[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              w8[e] = pack_bf16x2(__uint_as_float(orr[ch][8 * v + 2 * e]) * inv_l,
-                                  __uint_as_float(orr[ch][8 * v + 2 * e + 1]) * inv_l);
-            st_global_v8(dst + ch * 4 + v, w8);
-          }
-        if (wg == 0) p.lse[orow] = (d.m + __log2f(l_row)) * kLn2;
-      }
       return true;
     };
     for (int item = blockIdx.x; item < total_items; item += gridDim.x, ++it) {
@@ -788,16 +714,9 @@ __global__ void __launch_bounds__(PrefillLayout<DQK, DV>::THREADS, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(Lay::B_P_FULL + sbuf));
-        if (t == 0 && have_prev) {
-          have_prev = false;
-          if (!epilogue(prev)) {
-            ok = false;
-            break;
-          }
-        }
       }
       if (!ok) break;
-      if constexpr (Lay::EPI_WG) {
+      {
         // hand the item's row max and this half's row sums to the epilogue
         // warpgroup (rows buffer it & 1, read back two items ago)
         const int pr = it & 1;
@@ -808,27 +727,21 @@ __global__ void __launch_bounds__(PrefillLayout<DQK, DV>::THREADS, 1)
         if (wg == 0) rows[row] = m;
         rows[128 + wg * 128 + row] = l;
         mbar_arrive(bar(Lay::B_ROWS_FULL + pr));
-      } else {
-        prev = Done{w, m, l, ob, g0 + tr.count - 1};
-        have_prev = true;
       }
       g0 += tr.count;
     }
-    if (have_prev) epilogue(prev);
     // Every softmax thread performs the same number of exchanges -- one per
-    // tile of each of this CTA's items, plus one per item for the row sums of
-    // the deferred epilogue -- so that no partner is left at a named barrier:
-    // a thread that left the loops early makes up the rest here.
+    // tile of each of this CTA's items -- so that no partner is left at a
+    // named barrier: a thread that left the loops early makes up the rest here.
     if (*abort_flag) {
       uint32_t total = 0;
       for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
         const WorkItem w = decode_item(item, p, prefix);
-        total += (uint32_t)tile_range(w.qb, p.n_sink, p.n_local).count + (Lay::EPI_WG ? 0u : 1u);
+        total += (uint32_t)tile_range(w.qb, p.n_sink, p.n_local).count;
       }
       float unused;
       while (xc < total) exchange(-INFINITY, unused);
     }
-    if (Lay::TMA_OUT && !Lay::EPI_WG && row == 0) tma_store_wait_all();  // stores done before exit
   }
 
   __syncwarp();

@@ -121,7 +121,8 @@ size_t loza_ssa_prefill_host_workspace_size(int B, int H, int L, int d_qk, int d
  * each sequence's own first token, and no key crosses a sequence boundary.
  *   q, k : bf16 [H, total_tokens, d_qk]   v, o : bf16 [H, total_tokens, d_v]
  *   lse  : fp32 [H, total_tokens]         cu_seqlens : DEVICE int32 [n_seqs + 1]
- *   1 <= n_seqs <= 4000.  max_seqlen is the caller's bound on any sequence
+ *   1 <= n_seqs <= 4000 (<= 3000 when d_qk = 192: the kernel keeps one prefix
+ *   per sequence in shared memory).  max_seqlen is the caller's bound on any sequence
  *   length (used to size the launch; a longer sequence is still computed).
  * Other arguments as for loza_ssa_prefill.
  */

@@ -321,6 +321,11 @@ def test_varlen_argument_errors(L):
     assert call(cu=0) == -1
     assert call(n_seqs=0) == -2
     assert call(n_seqs=5000) == -2
+    # d_qk = 192 keeps fewer sequence prefixes in shared memory
+    assert call(n_seqs=3001, total=400000, dqk=192, dv=128) == -2
+    assert call(n_seqs=3001, total=400000, dqk=192, dv=128, cu=0x1002) == -2
+    assert call(n_seqs=3000, total=400000, dqk=192, dv=128, cu=0x1002) == -6
+    assert call(n_seqs=4000, total=600000, cu=0x1002) == -6
     assert call(total=0) == -2
     assert call(dqk=192, dv=192) == -3
     assert call(block=256) == -4
