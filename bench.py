@@ -181,7 +181,11 @@ def job_throughput(world: int, units_per_rank_step: float, steps: int, max_ms: f
 
 # ---------------------------------------------------------------- prefill
 
-def make_prefill(config, device, seed):
+def make_prefill(config, device, seed, heads=None):
+    """The prefill workload ``config``; ``heads`` (dense workloads only) keeps
+    the shapes but takes that many heads, for profiler captures of a smaller
+    case whose per-head work is the same."""
+    import dataclasses
     from block_sparse_streaming_ssa_b200 import synth
     if config == "varlen":
         sp = synth.VARLEN
@@ -195,6 +199,8 @@ def make_prefill(config, device, seed):
         return dict(spec=sp, q=q, k=k, v=v, cu=cu, max_len=max(lengths), pairs=pairs,
                     tokens=tokens, desc=desc, varlen=True)
     sp = {"tiny": synth.TINY, "mha": synth.MHA, "mla": synth.MLA}[config]
+    if heads:
+        sp = dataclasses.replace(sp, H=heads)
     q, k, v = synth.prefill_spec_inputs(sp, seed=seed, device=device)
     pairs = sp.B * sp.H * window_pairs(sp.L)
     desc = {"workload": f"ssa_prefill_{sp.name} B={sp.B} H={sp.H} L={sp.L} d_qk={sp.d_qk} "
@@ -667,10 +673,10 @@ def oracle_sample(config, budget_s, seed=0):
 
 # ------------------------------------------------------------------- main
 
-def prefill_leg(config, steps, warmup, peaks, dist, world, rank):
+def prefill_leg(config, steps, warmup, peaks, dist, world, rank, heads=None):
     """Time one prefill workload: (compact entry, detail, raw timing)."""
     import torch
-    w = make_prefill(config, "cuda", seed=rank)
+    w = make_prefill(config, "cuda", seed=rank, heads=heads)
     total_ms, per, clocks = time_prefill(w, steps, warmup, dist)
     max_ms = max_over_ranks(total_ms)
     flops = 2 * (w["spec"].d_qk + w["spec"].d_v) * w["pairs"]
@@ -701,6 +707,11 @@ def main():
                     help="skip timing the prefill's backward pass")
     ap.add_argument("--no-other-prefill", action="store_true",
                     help="time only the headline prefill workload")
+    ap.add_argument("--prefill-heads", type=int, default=None,
+                    help="headline prefill with this many heads instead (a smaller case of the "
+                         "same shapes, for profiler captures)")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the host-buffer call (for profiler captures)")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--decode-iters", type=int, default=30)
     ap.add_argument("--decode-len-hi", type=int, default=None,
@@ -810,12 +821,14 @@ def main():
         return
 
     # ---- headline prefill workload
-    w, head_entry, t = prefill_leg(args.config, args.steps, args.warmup, peaks, dist, world, rank)
-    e2e_ms, h2d, d2h = e2e_prefill(w, args.e2e_steps)
-    e2e_val = world * t["flops"] / (e2e_ms * 1e-3) / 1e12  # every rank runs the same e2e loop
+    w, head_entry, t = prefill_leg(args.config, args.steps, args.warmup, peaks, dist, world, rank,
+                                   heads=args.prefill_heads)
+    e2e_ms, h2d, d2h = (None, 0, 0) if args.no_e2e else e2e_prefill(w, args.e2e_steps)
+    # every rank runs the same e2e loop
+    e2e_val = None if e2e_ms is None else world * t["flops"] / (e2e_ms * 1e-3) / 1e12
     w_desc, w_spec = w["desc"], w["spec"]
     detail = {"headline": {"workload": w_desc, **head_entry,
-                           "e2e_ms": round(e2e_ms, 3), "clocks": t["clocks"]}}
+                           "e2e_ms": e2e_ms and round(e2e_ms, 3), "clocks": t["clocks"]}}
     configs = {}
     backwards = {}
     if not args.no_backward:
@@ -879,8 +892,9 @@ def main():
                      "traffic": traffic_lookup(kname, args.config),
                      "peak_source": peaks["source"]},
         "cpu_baseline": cpu,
-        "e2e": {"value": round(e2e_val, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+        "e2e": None if e2e_val is None else {
+            "value": round(e2e_val, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h},
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
         "gpu_launches": args.steps,
         "configs": configs,
