@@ -19,7 +19,7 @@
 // in TMEM by exp2(m_old - m_new) before the next P.V.  The final O = acc / l
 // and LSE = (m + log2 l) ln 2 are exact for any choice of m.
 //
-// Warp roles (384 threads; 512 for d_qk = d_v = 128, see below):
+// Warp roles (512 threads):
 //   warps 0-7  softmax + correction + epilogue.  Warp w reads TMEM lanes
 //              32*(w%4)..+31 (a warp may only touch its own lane quarter), so
 //              query row r is shared by thread r of warpgroup 0 (key columns
@@ -31,13 +31,15 @@
 //   warp 9     TMEM allocator + issuer of the S = Q K^T MMAs (one elected lane)
 //   warp 10    TMA producer of V (one elected lane)
 //   warp 11    issuer of the O += P V MMAs (one elected lane)
-//   warps 12-15 (d_qk = d_v = 128 only) the epilogue: the softmax warps hand
-//              each item's row max and row sums over through shared memory and
-//              go straight on to the next item; these warps wait for the
-//              item's last P.V, read O from TMEM, normalise it and send it out
-//              through swizzled staging boxes and TMA stores.  The 512 threads
-//              launch with 128 registers each and rebalance with setmaxnreg:
-//              152 for the softmax warpgroups, 104 for the other two.
+//   warps 12-15 the epilogue: the softmax warps hand each item's row max and
+//              row sums over through shared memory and go straight on to the
+//              next item; these warps wait for the item's last P.V, read O
+//              from TMEM, normalise it and send it out through swizzled
+//              staging boxes and TMA stores (the staging is a buffer of its
+//              own for d_qk <= 128, else the V ring slot of the item's last
+//              key tile).  The 512 threads launch with 128 registers each and
+//              rebalance with setmaxnreg: 152 for the softmax warpgroups, 104
+//              for the other two.
 // K and V have their own producers so a K load never queues behind a V load
 // that is waiting for its ring slot: S consumes K_{j+1} before P.V reads V_j.
 // S and P.V have their own issuers because an issuer blocks on its barrier

@@ -15,13 +15,15 @@ from tests.parity import assert_parity
 pytestmark = pytest.mark.gpu
 
 
-def run(lengths, H=2, d=128, seed=0, n_sink=1, n_local=7):
-    q, k, v, cu = synth.varlen_inputs(lengths, H, d, d, seed=seed, device="cuda")
+def run(lengths, H=2, d=128, seed=0, n_sink=1, n_local=7, dv=None, rows=None):
+    dv = d if dv is None else dv
+    q, k, v, cu = synth.varlen_inputs(lengths, H, d, dv, seed=seed, device="cuda")
     o, lse = loza_ssa_prefill_varlen(q, k, v, cu, max(lengths), n_sink=n_sink, n_local=n_local)
     torch.cuda.synchronize()
     assert loza_ssa_get_last_device_status() == 0
     o_ref, lse_ref = orc.prefill_varlen(*(synth.bf16_bits(t) for t in (q, k, v)),
-                                        cu.cpu().numpy(), 128, n_sink, n_local, 1 / math.sqrt(d))
+                                        cu.cpu().numpy(), 128, n_sink, n_local, 1 / math.sqrt(d),
+                                        rows=rows)
     return q, k, v, cu, o, lse, o_ref, lse_ref
 
 
@@ -100,3 +102,19 @@ def test_varlen_full_size_sampled():
     r = torch.as_tensor(rows, device="cuda")
     assert_parity(o[hsel].reshape(-1, sp.d_v)[r], lse[hsel].reshape(-1)[r], o_ref, lse_ref,
                   "varlen sampled")
+
+
+def test_most_sequences_at_mla_dims():
+    """3000 packed sequences at d_qk = 192, d_v = 128 (the limit for these dims:
+    the kernel keeps one work-item prefix per sequence in shared memory beside
+    the 192-wide rings), lengths 1 .. 300 (one or three blocks each), every row
+    of one head and a sample of the other checked against the oracle."""
+    rng = np.random.default_rng(21)
+    lengths = rng.integers(1, 301, size=3000).tolist()
+    total = sum(lengths)
+    rows = np.concatenate([np.arange(total), total + rng.choice(total, 2000, replace=False)])
+    q, k, v, cu, o, lse, o_ref, lse_ref = run(lengths, H=2, d=192, dv=128, seed=21,
+                                               rows=np.sort(rows))
+    r = torch.as_tensor(np.sort(rows), device="cuda")
+    assert_parity(o.reshape(-1, 128)[r], lse.reshape(-1)[r], o_ref, lse_ref,
+                  "3000 sequences, d=192/128")
