@@ -124,12 +124,8 @@ struct PrefillLayout {
   static constexpr int OFF_OST = OFF_V + VST * V_BYTES;
   static constexpr int OFF_BAR = OFF_OST + (OWN_STAGE ? VCH * CHUNK : 0);
   // barrier indices
-  // Q: one full / empty pair per (stage, 64-column chunk), so that a chunk of
-  // the next item's Q loads as soon as the last S of the current item has
-  // done its MMAs on that chunk, and the next item's first S starts on chunk 0
-  // while the others land
-  static constexpr int B_Q_FULL = 0, B_Q_EMPTY = B_Q_FULL + QST * KCH;
-  static constexpr int B_K_FULL = B_Q_EMPTY + QST * KCH, B_K_EMPTY = B_K_FULL + KST;
+  static constexpr int B_Q_FULL = 0, B_Q_EMPTY = B_Q_FULL + QST;
+  static constexpr int B_K_FULL = B_Q_EMPTY + QST, B_K_EMPTY = B_K_FULL + KST;
   static constexpr int B_V_FULL = B_K_EMPTY + KST, B_V_EMPTY = B_V_FULL + VST;
   static constexpr int B_S_FULL = B_V_EMPTY + VST;  // NSB
   static constexpr int B_P_FULL = B_S_FULL + NSB;   // NSB
@@ -262,7 +258,7 @@ __global__ void __launch_bounds__(PrefillLayout<DQK, DV>::THREADS, 1)
   int* status = &g_loza_status;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < Lay::QST * Lay::KCH; ++s) {
+    for (int s = 0; s < Lay::QST; ++s) {
       mbar_init(bar(Lay::B_Q_FULL + s), 1);
       mbar_init(bar(Lay::B_Q_EMPTY + s), 1);
     }
@@ -327,45 +323,23 @@ __global__ void __launch_bounds__(PrefillLayout<DQK, DV>::THREADS, 1)
     // ------------------------------------------------------- Q / K producer
     if (lane == 0) {
       int g = 0, it = 0;
-      int q_issued[Lay::QST * Lay::KCH] = {}, k_issued[Lay::KST] = {};
+      int q_issued[Lay::QST] = {}, k_issued[Lay::KST] = {};
       bool ok = true;
-      // key tile t of item w into the next ring slot
-      auto load_k = [&](const WorkItem& w, const TileRange& tr, int t) -> bool {
-        const int row = w.seq_start + tile_block(tr, t) * 128;
-        const int st = g % Lay::KST, use = g / Lay::KST;
-        if (use > 0 &&
-            !mbar_wait(bar(Lay::B_K_EMPTY + st), (use - 1) & 1, abort_flag, status, 1))
-          return false;
-        mbar_arrive_expect_tx(bar(Lay::B_K_FULL + st), Lay::K_BYTES);
-        ++k_issued[st];
-#pragma unroll
-        for (int c = 0; c < Lay::KCH; ++c)
-          tma_load_3d(sb + Lay::OFF_K + st * Lay::K_BYTES + c * Lay::CHUNK, &tm_k,
-                      bar(Lay::B_K_FULL + st), c * 64, row, w.z);
-        ++g;
-        return true;
-      };
       for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++it) {
         const WorkItem w = decode_item(item, p, prefix);
         const TileRange tr = tile_range(w.qb, p.n_sink, p.n_local);
         const int qs = it % Lay::QST;
-        // The item's first key tile goes out before its Q: its ring slot frees
-        // a tile before the Q slot, which the previous item's last S holds.
-        if (!(ok = load_k(w, tr, 0))) break;
-        // Q chunk by chunk, each as soon as the last S of the item that used
-        // the stage before has done its MMAs on that chunk
-#pragma unroll
-        for (int c = 0; c < Lay::KCH; ++c) {
-          const int qb = qs * Lay::KCH + c;
-          if (it >= Lay::QST && !(ok = mbar_wait(bar(Lay::B_Q_EMPTY + qb),
-                                                 (it / Lay::QST - 1) & 1, abort_flag, status, 1)))
-            break;
-          mbar_arrive_expect_tx(bar(Lay::B_Q_FULL + qb), Lay::CHUNK);
-          ++q_issued[qb];
-          tma_load_3d(sb + Lay::OFF_Q + qs * Lay::Q_BYTES + c * Lay::CHUNK, &tm_q,
-                      bar(Lay::B_Q_FULL + qb), c * 64, w.seq_start + w.qb * 128, w.z);
+        if (it >= Lay::QST && !mbar_wait(bar(Lay::B_Q_EMPTY + qs), (it / Lay::QST - 1) & 1,
+                                         abort_flag, status, 1)) {
+          ok = false;
+          break;
         }
-        if (!ok) break;
+        mbar_arrive_expect_tx(bar(Lay::B_Q_FULL + qs), Lay::Q_BYTES);
+        ++q_issued[qs];
+#pragma unroll
+        for (int c = 0; c < Lay::KCH; ++c)
+          tma_load_3d(sb + Lay::OFF_Q + qs * Lay::Q_BYTES + c * Lay::CHUNK, &tm_q,
+                      bar(Lay::B_Q_FULL + qs), c * 64, w.seq_start + w.qb * 128, w.z);
         // the item after the ring's reach is first-touch HBM data: start
         // pulling its Q into L2 now
         const int ahead = item + Lay::QST * (int)gridDim.x;
@@ -375,15 +349,28 @@ __global__ void __launch_bounds__(PrefillLayout<DQK, DV>::THREADS, 1)
           for (int c = 0; c < Lay::KCH; ++c)
             tma_prefetch_3d(&tm_q, c * 64, wn.seq_start + wn.qb * 128, wn.z);
         }
-        for (int t = 1; t < tr.count; ++t)
-          if (!(ok = load_k(w, tr, t))) break;
+        for (int t = 0; t < tr.count; ++t, ++g) {
+          const int row = w.seq_start + tile_block(tr, t) * 128;
+          const int st = g % Lay::KST, use = g / Lay::KST;
+          if (use > 0 &&
+              !mbar_wait(bar(Lay::B_K_EMPTY + st), (use - 1) & 1, abort_flag, status, 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(Lay::B_K_FULL + st), Lay::K_BYTES);
+          ++k_issued[st];
+#pragma unroll
+          for (int c = 0; c < Lay::KCH; ++c)
+            tma_load_3d(sb + Lay::OFF_K + st * Lay::K_BYTES + c * Lay::CHUNK, &tm_k,
+                        bar(Lay::B_K_FULL + st), c * 64, row, w.z);
+        }
       }
       if (!ok) {
         // Let copies already in flight land before the CTA's smem goes away:
         // a slot holds at most one unconsumed load, its newest phase.
         for (int s = 0; s < Lay::KST; ++s)
           if (k_issued[s] > 0) mbar_wait_drain(bar(Lay::B_K_FULL + s), (k_issued[s] - 1) & 1);
-        for (int s = 0; s < Lay::QST * Lay::KCH; ++s)
+        for (int s = 0; s < Lay::QST; ++s)
           if (q_issued[s] > 0) mbar_wait_drain(bar(Lay::B_Q_FULL + s), (q_issued[s] - 1) & 1);
       }
     }
@@ -429,6 +416,10 @@ __global__ void __launch_bounds__(PrefillLayout<DQK, DV>::THREADS, 1)
         const TileRange tr = tile_range(w.qb, p.n_sink, p.n_local);
         const int qs = it % Lay::QST;
         const uint32_t q_base = sb + Lay::OFF_Q + qs * Lay::Q_BYTES;
+        if (!mbar_wait(bar(Lay::B_Q_FULL + qs), (it / Lay::QST) & 1, abort_flag, status, 1)) {
+          ok = false;
+          break;
+        }
         for (int t = 0; t < tr.count; ++t, ++g) {
           const int st = g % Lay::KST, sbuf = g % Lay::NSB;
           // S buffer sbuf last held P_{g-NSB}: wait until its P.V has read it
@@ -442,24 +433,14 @@ __global__ void __launch_bounds__(PrefillLayout<DQK, DV>::THREADS, 1)
           const uint32_t s_tmem = tmem + (uint32_t)(sbuf * 128);
 #pragma unroll
           for (int kk = 0; kk < DQK / 16; ++kk) {
-            // the item's first S waits for each Q chunk just before using it
-            if (t == 0 && (kk & 3) == 0) {
-              if (!(ok = mbar_wait(bar(Lay::B_Q_FULL + qs * Lay::KCH + (kk >> 2)),
-                                   (it / Lay::QST) & 1, abort_flag, status, 1)))
-                break;
-              tc_fence_after();
-            }
             const uint32_t koff = (kk >> 2) * Lay::CHUNK + (kk & 3) * 32;
             const uint64_t adesc = sdesc_sw128(q_base + koff, 16, 1024);
             const uint64_t bdesc = sdesc_sw128(sb + Lay::OFF_K + st * Lay::K_BYTES + koff, 16, 1024);
             mma_ss(s_tmem, adesc, bdesc, id_s, kk > 0 ? 1u : 0u);
-            // the item's last S frees each Q chunk as soon as its MMAs on it finish
-            if (t == tr.count - 1 && (kk & 3) == 3)
-              mma_commit(bar(Lay::B_Q_EMPTY + qs * Lay::KCH + (kk >> 2)));
           }
-          if (!ok) break;
           mma_commit(bar(Lay::B_S_FULL + sbuf));
           mma_commit(bar(Lay::B_K_EMPTY + st));
+          if (t == tr.count - 1) mma_commit(bar(Lay::B_Q_EMPTY + qs));
         }
       }
       // every tcgen05.mma issued above has finished before TMEM is released
