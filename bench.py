@@ -81,6 +81,7 @@ KERNEL_SOURCES = {
     "ssa_prefill_kernel": ("prefill.cuh", "ptx.cuh", "schedule.cuh"),
     "ssa_decode_split_kernel": ("decode.cuh", "ptx.cuh", "schedule.cuh"),
     "ssa_decode_merge_kernel": ("decode.cuh", "ptx.cuh", "schedule.cuh"),
+    "ssa_decode_long_kernel": ("decode_long.cuh", "decode.cuh", "ptx.cuh", "schedule.cuh"),
 }
 
 
@@ -614,6 +615,8 @@ def context_bench(peaks, context=131072, iters=5, warmup=3, world=1, seed=0):
     zigzag_ms = timed((True, False, True, False))
     all_full_ms = timed((True, True, True, True))
     full_bytes = s.B * (context * s.d_qk * 2 + s.H_q * (s.d_qk * 2 + s.d_v * 2 + 4))
+    t16 = traffic_lookup("ssa_decode_long_kernel", "ctx16k")
+    traffic = None if t16 is None else int(t16 * context / 16384)
     full_flops = 2 * (s.d_qk + s.d_v) * s.B * s.H_q * context
     gbs = full_bytes / (full_ms * 1e-3) / 1e9
     del pools, ws, flush
@@ -630,9 +633,15 @@ def context_bench(peaks, context=131072, iters=5, warmup=3, world=1, seed=0):
         "full_layer_roofline": {"bound": "hbm", "achieved": round(gbs, 1),
                                 "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                 "frac": round(gbs / peaks["hbm_gbs"], 4),
-                                "peak_source": peaks["source"]},
+                                "peak_source": peaks["source"],
+                                "kernel": "ssa_decode_long_kernel",
+                                "traffic": traffic,
+                                "traffic_note": "ncu DRAM bytes of one launch at 16384 tokens, "
+                                                "scaled by the context length"},
         "l2": "2x L2 write before every timed call",
-        "gpu_launches": 2 * (1 + 1 + 4 + 4) * (iters + warmup),
+        # a full-attention layer: plan, long-window and merge kernels; an SSA
+        # layer: the split kernel with its in-cluster merge
+        "gpu_launches": (3 + 1 + (3 + 1 + 3 + 1) + 4 * 3) * (iters + warmup),
     }
 
 

@@ -82,6 +82,12 @@ struct DecodeParams {
   // 1: the n_split splits of a (row, head group) run as one thread-block
   // cluster and merge their partials in the split kernel (no merge kernel).
   int cluster_merge;
+  // Long-window kernel (decode_long.cuh; nullptr otherwise): plan[u] = pages
+  // listed by the (row, head group) units before u, plan[B * HG] = all of
+  // them; the pages are shared out over n_pairs CTA pairs; then, from
+  // plan + B * HG + 1, each unit's first partial slot and slot count.
+  const int* plan;
+  int n_pairs;
 };
 
 __device__ __forceinline__ int decode_seq(const DecodeParams& p, int row) {
@@ -144,6 +150,19 @@ __device__ __forceinline__ int decode_page(const DecodeParams& p, int b, int log
 // Keys of a logical page at or before the query (1..128).
 __device__ __forceinline__ int decode_valid_keys(const DecodeWindow& w, int logical) {
   return min(128, w.t - logical * 128 + 1);
+}
+
+// Pair that owns flat page x of T, with P pairs: pair k owns [k T / P, (k+1) T / P).
+__host__ __device__ __forceinline__ int long_pair_of(long long x, long long T, int P) {
+  return (int)(((x + 1) * P + T - 1) / T) - 1;
+}
+__host__ __device__ __forceinline__ long long long_pair_start(int k, long long T, int P) {
+  return (long long)k * T / P;
+}
+// Pairs that share T pages when `launched` pairs run: at most one per page, so
+// that every pair's range [k T / P, (k+1) T / P) holds at least one page.
+__host__ __device__ __forceinline__ int long_pairs(int launched, long long T) {
+  return (int)(T < launched ? (T > 0 ? T : 1) : launched);
 }
 
 struct DecodeLayout {
@@ -812,7 +831,10 @@ constexpr int kMergeGroups = 2;  // 8-column groups per thread
 constexpr int kMergeThreads = (kDecodeDv / 8 / kMergeGroups) * kMergeHeads;  // 256
 constexpr int kMergeBatch = 4;
 
-// four CTAs per SM: 148 x 4 slots hold the 512 CTAs of the 32-sequence workload
+// four CTAs per SM: 148 x 4 slots hold the 512 CTAs of the 32-sequence workload.
+// PLAN: the partials of the long-window kernel (a unit's slots from its plan)
+// instead of the split kernel's n_split per (row, head group).
+template <bool PLAN>
 __global__ void __launch_bounds__(kMergeThreads, 4)
     ssa_decode_merge_kernel(const DecodeParams p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -823,11 +845,16 @@ __global__ void __launch_bounds__(kMergeThreads, 4)
   if (h >= p.H_q) return;
   const int hg = h >> 7, hr = h & 127;
   constexpr int kGroupStride = kDecodeDv / 8 / kMergeGroups;  // 32: groups gp, gp + 32
-  const size_t cta0 = ((size_t)b * p.HG + hg) * p.n_split;
+  size_t cta0 = ((size_t)b * p.HG + hg) * p.n_split;
+  int n = p.n_split;
+  if constexpr (PLAN) {
+    const int* us = p.plan + p.B * p.HG + 1 + 2 * (b * p.HG + hg);
+    cta0 = (size_t)us[0];
+    n = us[1];
+  }
   const float* lsep = p.lse_part + cta0 * 128 + hr;  // split stride 128
   const uint4* op = reinterpret_cast<const uint4*>(p.o_part) + (cta0 * 64 + gp) * 128 + hr;
   constexpr size_t kSplitStride = 64 * 128;  // uint4 per split
-  const int n = p.n_split;
   // One pass, kMergeBatch splits at a time: a batch's LSEs and partial O are
   // loaded together (one round trip to L2 for the usual four splits), and
   // the running max only rescales what earlier batches summed.

@@ -16,6 +16,7 @@
 #include "../../include/loza_ssa.h"
 #include "backward.cuh"
 #include "decode.cuh"
+#include "decode_long.cuh"
 #include "prefill.cuh"
 #include "schedule.cuh"
 
@@ -407,6 +408,44 @@ size_t decode_partial_floats(int B, int H_q, int n_split) {
   return (size_t)B * hg * (size_t)n_split * 128;
 }
 
+// Whether a decode of B rows over a window listing n_sink + n_local pages
+// (and max_extra chosen ones) takes the long-window kernel (bf16 cache only):
+// more than kLongMinPages pages, no chosen pages, and page offsets that fit
+// in int.
+bool decode_long_eligible(int B, int H_q, int n_sink, int n_local, int max_extra) {
+  const long long units = (long long)B * ((H_q + 127) / 128);
+  const long long window = (long long)n_sink + n_local;
+  return max_extra == 0 && window > loza::kLongMinPages && units <= (1ll << 20) &&
+         units * window < (1ll << 31);
+}
+
+// Workspace of the long-window kernel: a partial O (fp16) and LSE per slot --
+// a unit has one slot per CTA pair its pages span, B * HG + pairs - 1 in all
+// -- and the plan's B * HG + 1 page offsets and B * HG (first slot, count)
+// pairs.
+struct LongWorkspace {
+  size_t o, lse, plan, total;
+};
+LongWorkspace long_workspace(int B, int H_q) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  const size_t units = (size_t)B * ((H_q + 127) / 128);
+  const size_t slots = units + loza::kLongMaxPairs;
+  LongWorkspace w;
+  w.o = 0;
+  w.lse = up(slots * 128 * loza::kDecodeDv * sizeof(__half));
+  w.plan = w.lse + up(slots * 128 * sizeof(float));
+  w.total = w.plan + up((3 * units + 1) * sizeof(int));
+  return w;
+}
+
+// Workspace of the split kernel: a partial O (fp16) and LSE per split CTA.
+size_t decode_split_workspace_size(int B, int H_q, int n_sink, int n_local, int max_extra) {
+  const size_t rows = decode_partial_floats(B, H_q, decode_splits(n_sink, n_local, max_extra));
+  const size_t o_bytes = rows * loza::kDecodeDv * sizeof(__half);  // partial O is fp16
+  const size_t lse_bytes = rows * sizeof(float);
+  return ((o_bytes + 255) / 256) * 256 + ((lse_bytes + 255) / 256) * 256;
+}
+
 }  // namespace
 
 namespace {
@@ -794,10 +833,12 @@ size_t loza_ssa_decode_selected_workspace_size(int B, int H_q, int d_v, int n_si
   if (B < 1 || H_q < 1 || d_v != loza::kDecodeDv || n_sink < 0 || n_local < 1 ||
       max_extra < 0 || (long long)n_sink + n_local + max_extra > kMaxDecodeWindow)
     return 0;
-  const size_t rows = decode_partial_floats(B, H_q, decode_splits(n_sink, n_local, max_extra));
-  const size_t o_bytes = rows * loza::kDecodeDv * sizeof(__half);  // partial O is fp16
-  const size_t lse_bytes = rows * sizeof(float);
-  return ((o_bytes + 255) / 256) * 256 + ((lse_bytes + 255) / 256) * 256;
+  const size_t split = decode_split_workspace_size(B, H_q, n_sink, n_local, max_extra);
+  // a long window takes the long-window kernel for a bf16 cache and the split
+  // kernel for an FP8 one: room for either
+  if (!decode_long_eligible(B, H_q, n_sink, n_local, max_extra)) return split;
+  const size_t lng = long_workspace(B, H_q).total;
+  return lng > split ? lng : split;
 }
 
 size_t loza_ssa_decode_workspace_size(int B, int H_q, int d_v, int n_sink, int n_local) {
@@ -841,6 +882,69 @@ int decode_check_args(const void* q, const void* paged_kv, const int* page_table
   return LOZA_SSA_OK;
 }
 
+// The long-window path: plan kernel, long-window kernel (a programmatic
+// dependent of the plan), merge kernel (a programmatic dependent of the long
+// kernel).  B counts rows; the arguments are checked.
+int decode_long_launch(const void* q, const void* paged_kv, const int* page_table,
+                       const int* seq_lens, int q_len, void* o, float* lse, int B, int H_q,
+                       int max_pages, int n_pages, int n_sink, int n_local, float scale,
+                       void* workspace, const DeviceInfo& dev, cudaStream_t s) {
+  const LongWorkspace ws = long_workspace(B, H_q);
+  char* base = static_cast<char*>(workspace);
+  loza::DecodeParams prm{};
+  prm.page_table = page_table;
+  prm.seq_lens = seq_lens;
+  prm.o_part = reinterpret_cast<__half*>(base + ws.o);
+  prm.lse_part = reinterpret_cast<float*>(base + ws.lse);
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  prm.B = B;
+  prm.q_len = q_len;
+  prm.H_q = H_q;
+  prm.HG = (H_q + 127) / 128;
+  prm.max_pages = max_pages;
+  prm.n_pages = n_pages;
+  prm.n_sink = n_sink;
+  prm.n_local = n_local;
+  prm.n_split = 0;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.wave = INT_MAX;
+  int* plan = reinterpret_cast<int*>(base + ws.plan);
+  prm.plan = plan;
+  prm.n_pairs = std::min(std::max(dev.num_sms / 2, 1), loza::kLongMaxPairs);
+
+  CUtensorMap mq, mkv;
+  int rc = make_map(&mq, q, loza::kDecodeDqk, (uint64_t)H_q, (uint64_t)B, 3);
+  if (rc != LOZA_SSA_OK) return rc;
+  if ((rc = make_map(&mkv, paged_kv, loza::kDecodeDqk, (uint64_t)n_pages * 128, 1, 2)) !=
+      LOZA_SSA_OK)
+    return rc;
+  cudaError_t e = cudaFuncSetAttribute(loza::ssa_decode_long_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       loza::LongDecodeLayout::SMEM_BYTES);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode long)");
+  loza::ssa_decode_plan_kernel<<<1, loza::kLongPlanThreads, 0, s>>>(prm, plan);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "decode plan launch");
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(2 * prm.n_pairs);
+  cfg.blockDim = dim3(loza::LongDecodeLayout::THREADS);
+  cfg.dynamicSmemBytes = loza::LongDecodeLayout::SMEM_BYTES;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if ((e = cudaLaunchKernelEx(&cfg, loza::ssa_decode_long_kernel, mq, mkv, prm)) != cudaSuccess)
+    return cuda_fail(e, "decode long launch");
+  cfg.gridDim = dim3(B * ((H_q + loza::kMergeHeads - 1) / loza::kMergeHeads));
+  cfg.blockDim = dim3(loza::kMergeThreads);
+  cfg.dynamicSmemBytes = 0;
+  if ((e = cudaLaunchKernelEx(&cfg, loza::ssa_decode_merge_kernel<true>, prm)) != cudaSuccess)
+    return cuda_fail(e, "decode merge launch");
+  return LOZA_SSA_OK;
+}
+
 // loza_ssa_decode with an optional per-sequence list of extra pages
 // (extra_pages == nullptr and max_extra == 0: the plain window), q_len
 // query tokens per sequence (q_len == 1: one) and an FP8 cache (kv_scale !=
@@ -849,19 +953,28 @@ int decode_impl(const void* q, const void* paged_kv, const int* page_table, cons
                 const int* extra_pages, int max_extra, int q_len, void* o, float* lse, int B,
                 int H_q, int d_qk, int d_v, int page_size, int max_pages, int n_pages, int n_sink,
                 int n_local, float scale, void* workspace, size_t workspace_bytes,
-                loza_ssa_stream_t stream, const float* kv_scale = nullptr) {
+                loza_ssa_stream_t stream, const float* kv_scale = nullptr,
+                bool allow_long = true) {
   int rc = decode_check_args(q, paged_kv, page_table, seq_lens, extra_pages, max_extra, q_len, o,
                              lse, B, H_q, d_qk, d_v, page_size, max_pages, n_pages, n_sink,
                              n_local, scale, kv_scale);
   if (rc != LOZA_SSA_OK) return rc;
   B *= q_len;  // from here on B counts rows: (sequence, query token) pairs
+  const bool use_long =
+      allow_long && !kv_scale && decode_long_eligible(B, H_q, n_sink, n_local, max_extra);
+  // what the size query promises (room for either kernel), or, for the
+  // built-in scratch (split kernel only), the split kernel's share
   const size_t need =
-      loza_ssa_decode_selected_workspace_size(B, H_q, d_v, n_sink, n_local, max_extra);
+      allow_long ? loza_ssa_decode_selected_workspace_size(B, H_q, d_v, n_sink, n_local, max_extra)
+                 : decode_split_workspace_size(B, H_q, n_sink, n_local, max_extra);
   if (!workspace || workspace_bytes < need) return LOZA_SSA_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return LOZA_SSA_ERR_ALIGN;
   DeviceInfo dev;
   rc = device_info(dev);
   if (rc != LOZA_SSA_OK) return rc;
+  if (use_long) return decode_long_launch(q, paged_kv, page_table, seq_lens, q_len, o, lse, B, H_q,
+                                          max_pages, n_pages, n_sink, n_local, scale, workspace,
+                                          dev, reinterpret_cast<cudaStream_t>(stream));
 
   const int n_split = decode_splits(n_sink, n_local, max_extra);
   const int HG = (H_q + 127) / 128;
@@ -947,7 +1060,7 @@ int decode_impl(const void* q, const void* paged_kv, const int* page_table, cons
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if ((e = cudaLaunchKernelEx(&cfg, loza::ssa_decode_merge_kernel, prm)) != cudaSuccess)
+  if ((e = cudaLaunchKernelEx(&cfg, loza::ssa_decode_merge_kernel<false>, prm)) != cudaSuccess)
     return cuda_fail(e, "decode merge launch");
   return LOZA_SSA_OK;
 }
@@ -1048,7 +1161,9 @@ int loza_ssa_decode_static_scratch(const void* q, const void* paged_kv, const in
                   slots, LOZA_SSA_STATIC_SCRATCH_SLOTS);
     return LOZA_SSA_ERR_SCRATCH_LIMIT;
   }
-  const size_t need = loza_ssa_decode_workspace_size(B, H_q, d_v, n_sink, n_local);
+  // the built-in scratch is sized for the split kernel, which this call
+  // always uses
+  const size_t need = decode_split_workspace_size(B, H_q, n_sink, n_local, 0);
   if (need == 0 || need > sizeof(g_decode_scratch)) {
     std::snprintf(g_last_error, sizeof g_last_error,
                   "decode_static_scratch: needs %zu scratch bytes, the built-in scratch holds %zu",
@@ -1057,9 +1172,9 @@ int loza_ssa_decode_static_scratch(const void* q, const void* paged_kv, const in
   }
   void* scratch = nullptr;
   if ((rc = static_scratch_address(&scratch)) != LOZA_SSA_OK) return rc;
-  return loza_ssa_decode(q, paged_kv, page_table, seq_lens, o, lse, B, H_q, d_qk, d_v, page_size,
-                         max_pages, n_pages, n_sink, n_local, scale, scratch,
-                         sizeof(g_decode_scratch), stream);
+  return decode_impl(q, paged_kv, page_table, seq_lens, nullptr, 0, 1, o, lse, B, H_q, d_qk, d_v,
+                     page_size, max_pages, n_pages, n_sink, n_local, scale, scratch,
+                     sizeof(g_decode_scratch), stream, nullptr, /*allow_long=*/false);
 }
 
 int loza_ssa_get_last_device_status(loza_ssa_stream_t stream) {

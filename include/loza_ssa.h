@@ -208,6 +208,13 @@ size_t loza_ssa_prefill_varlen_bwd_workspace_size(int n_seqs, int total_tokens, 
  *                loza_ssa_decode_workspace_size(B, H_q, d_v, n_sink, n_local)
  *                bytes, 256-byte aligned, owned by the caller, contents
  *                irrelevant on entry and overwritten.
+ * Kernels: windows of up to 16 pages run as split CTAs of two pages each,
+ * merged by LSE in the same launch (or a second one); wider windows (a
+ * full-attention layer is the widest) run as three launches -- a one-CTA
+ * plan of each sequence's pages, CTA pairs that stream an equal share of all
+ * pages with an online softmax, and the LSE merge of their partials.  The
+ * results agree with each other to rounding (same tolerance against the
+ * float64 definition), not bit for bit.
  */
 int loza_ssa_decode(const void* q, const void* paged_kv, const int* page_table,
                     const int* seq_lens, void* o, float* lse, int B, int H_q, int d_qk, int d_v,

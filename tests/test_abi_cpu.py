@@ -68,6 +68,36 @@ def test_decode_workspace_size(L):
     assert api.loza_ssa_decode_workspace_size(32, 128, 512, 1, 0) == 0      # n_local < 1
 
 
+def test_decode_workspace_size_long_window(L):
+    """Windows of more than 16 pages run through the long-window kernel for a
+    bf16 cache and the split kernel for an FP8 one (same size query): the
+    size covers both.  Long-window kernel: one partial slot per (row, head
+    group) unit plus one per CTA pair (at most 128 pairs), 128 rows of 512
+    fp16 and 128 fp32 LSEs each, and the plan's 3 * units + 1 ints; each part
+    rounded up to 256 bytes."""
+    from block_sparse_streaming_ssa_b200 import loza_ssa as api
+    up = lambda x: -(-x // 256) * 256
+
+    def split(B, hg, window):
+        rows = B * hg * -(-window // 2) * 128
+        return up(rows * 1024) + up(rows * 4)
+
+    def long(B, hg):
+        units = B * hg
+        slots = units + 128
+        return up(slots * 128 * 1024) + up(slots * 128 * 4) + up((3 * units + 1) * 4)
+
+    # a short sequence batch: the long kernel's slots dominate
+    assert api.loza_ssa_decode_workspace_size(1, 128, 512, 0, 20) == max(split(1, 1, 20), long(1, 1))
+    assert api.loza_ssa_decode_workspace_size(1, 128, 512, 0, 20) == 16974592
+    # a full-attention layer at 128K: the FP8 split kernel's 512 splits dominate
+    assert api.loza_ssa_decode_workspace_size(32, 128, 512, 0, 1024) == split(32, 1, 1024)
+    assert api.loza_ssa_decode_workspace_size(3, 200, 512, 2, 30) == \
+        max(split(3, 2, 32), long(3, 2))
+    # 16 pages: the split kernel alone
+    assert api.loza_ssa_decode_workspace_size(1, 128, 512, 1, 15) == split(1, 1, 16)
+
+
 def test_decode_selected_workspace_size(L):
     from block_sparse_streaming_ssa_b200 import loza_ssa as api
     # one split per two listed pages: window 8 + 8 chosen pages -> 8 splits
