@@ -140,9 +140,39 @@ __device__ __forceinline__ int decode_split_pages(const DecodeParams& p, int b,
   return n;
 }
 
+// Chosen pages of row b that count, in the list's order: those strictly
+// between the sink pages and the local run (others are in the window or after
+// the query's page), each page once.  decode_extra_count: how many there are;
+// decode_extra_page: the k-th of them (0-based), or -1.  O(max_extra^2) loads
+// at worst, from one small L1-resident row.
+__device__ __forceinline__ bool decode_extra_counts(const DecodeParams& p, const int* ex, int j,
+                                                    const DecodeWindow& w) {
+  const int e = __ldg(ex + j);
+  if (e < p.n_sink || e >= w.tr.local_lo) return false;
+  for (int j2 = 0; j2 < j; ++j2)
+    if (__ldg(ex + j2) == e) return false;
+  return true;
+}
+__device__ __forceinline__ int decode_extra_count(const DecodeParams& p, int b,
+                                                  const DecodeWindow& w) {
+  if (p.max_extra == 0) return 0;
+  const int* ex = p.extra_pages + (size_t)decode_seq(p, b) * p.max_extra;
+  int n = 0;
+  for (int j = 0; j < p.max_extra; ++j) n += decode_extra_counts(p, ex, j, w) ? 1 : 0;
+  return n;
+}
+__device__ __forceinline__ int decode_extra_page(const DecodeParams& p, int b,
+                                                 const DecodeWindow& w, int k) {
+  const int* ex = p.extra_pages + (size_t)decode_seq(p, b) * p.max_extra;
+  for (int j = 0; j < p.max_extra; ++j)
+    if (decode_extra_counts(p, ex, j, w) && k-- == 0) return __ldg(ex + j);
+  return -1;
+}
+
 // Physical page of a logical page of row b's sequence, or -1 if the table entry is
 // outside the pool.
 __device__ __forceinline__ int decode_page(const DecodeParams& p, int b, int logical) {
+  if (logical < 0) return -1;
   const int phys = __ldg(p.page_table + (size_t)decode_seq(p, b) * p.max_pages + logical);
   return (phys >= 0 && phys < p.n_pages) ? phys : -1;
 }

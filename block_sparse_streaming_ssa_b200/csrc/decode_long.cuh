@@ -92,11 +92,18 @@ struct LongDecodeLayout {
 };
 static_assert(LongDecodeLayout::SMEM_BYTES <= 227 * 1024, "long decode layout exceeds smem");
 
-// Pages the window of unit u (row u / HG) lists; 0 for a row whose seq_len is
-// out of range.
+// Pages unit u (row u / HG) lists: its window's, then the chosen pages that
+// count (decode_extra_page); 0 for a row whose seq_len is out of range.
 __device__ __forceinline__ int long_unit_pages(const DecodeParams& p, int u) {
   DecodeWindow w;
-  return decode_window(p, u / p.HG, w) ? w.tr.count : 0;
+  const int b = u / p.HG;
+  return decode_window(p, b, w) ? w.tr.count + decode_extra_count(p, b, w) : 0;
+}
+
+// Logical page of listed entry i of row b.
+__device__ __forceinline__ int long_listed_page(const DecodeParams& p, int b,
+                                                const DecodeWindow& w, int i) {
+  return i < w.tr.count ? tile_block(w.tr, i) : decode_extra_page(p, b, w, i - w.tr.count);
 }
 
 // The plan: plan[u] = pages listed by units 0..u-1, plan[U] = T, then per
@@ -285,7 +292,7 @@ __global__ void __launch_bounds__(LongDecodeLayout::THREADS, 1)
         for (int c = 0; c < Lay::KV_CH; ++c) tma_prefetch_2d(&tm_kv, c * 64, phys * 128);
       };
       auto phys_of = [&](const LongSeg& s, int i) -> int {
-        const int ph = decode_page(p, s.b, tile_block(s.w.tr, i));
+        const int ph = decode_page(p, s.b, long_listed_page(p, s.b, s.w, i));
         if (ph < 0) atomicOr(status, 2);
         return ph < 0 ? 0 : ph;  // a bad entry reads page 0, fully masked by the softmax
       };
@@ -430,7 +437,7 @@ __global__ void __launch_bounds__(LongDecodeLayout::THREADS, 1)
       float l = 0.f;
       for (int i = sg.lo; i < sg.hi; ++i, ++f) {
         const int b2 = f & 1;
-        const int logical = tile_block(sg.w.tr, i);
+        const int logical = long_listed_page(p, sg.b, sg.w, i);
         const int valid_keys = decode_page(p, sg.b, logical) < 0 ? 0
                                                                : decode_valid_keys(sg.w, logical);
         const bool partial = valid_keys < 128;

@@ -409,14 +409,13 @@ size_t decode_partial_floats(int B, int H_q, int n_split) {
 }
 
 // Whether a decode of B rows over a window listing n_sink + n_local pages
-// (and max_extra chosen ones) takes the long-window kernel (bf16 cache only):
-// more than kLongMinPages pages, no chosen pages, and page offsets that fit
-// in int.
+// and up to max_extra chosen ones takes the long-window kernel (bf16 cache
+// only): more than kLongMinPages listed pages, and page offsets that fit in
+// int.
 bool decode_long_eligible(int B, int H_q, int n_sink, int n_local, int max_extra) {
   const long long units = (long long)B * ((H_q + 127) / 128);
-  const long long window = (long long)n_sink + n_local;
-  return max_extra == 0 && window > loza::kLongMinPages && units <= (1ll << 20) &&
-         units * window < (1ll << 31);
+  const long long listed = (long long)n_sink + n_local + max_extra;
+  return listed > loza::kLongMinPages && units <= (1ll << 20) && units * listed < (1ll << 31);
 }
 
 // Workspace of the long-window kernel: a partial O (fp16) and LSE per slot --
@@ -886,7 +885,8 @@ int decode_check_args(const void* q, const void* paged_kv, const int* page_table
 // dependent of the plan), merge kernel (a programmatic dependent of the long
 // kernel).  B counts rows; the arguments are checked.
 int decode_long_launch(const void* q, const void* paged_kv, const int* page_table,
-                       const int* seq_lens, int q_len, void* o, float* lse, int B, int H_q,
+                       const int* seq_lens, const int* extra_pages, int max_extra, int q_len,
+                       void* o, float* lse, int B, int H_q,
                        int max_pages, int n_pages, int n_sink, int n_local, float scale,
                        void* workspace, const DeviceInfo& dev, cudaStream_t s) {
   const LongWorkspace ws = long_workspace(B, H_q);
@@ -907,6 +907,8 @@ int decode_long_launch(const void* q, const void* paged_kv, const int* page_tabl
   prm.n_sink = n_sink;
   prm.n_local = n_local;
   prm.n_split = 0;
+  prm.extra_pages = max_extra > 0 ? extra_pages : nullptr;
+  prm.max_extra = max_extra > 0 ? max_extra : 0;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.wave = INT_MAX;
   int* plan = reinterpret_cast<int*>(base + ws.plan);
@@ -972,9 +974,10 @@ int decode_impl(const void* q, const void* paged_kv, const int* page_table, cons
   DeviceInfo dev;
   rc = device_info(dev);
   if (rc != LOZA_SSA_OK) return rc;
-  if (use_long) return decode_long_launch(q, paged_kv, page_table, seq_lens, q_len, o, lse, B, H_q,
-                                          max_pages, n_pages, n_sink, n_local, scale, workspace,
-                                          dev, reinterpret_cast<cudaStream_t>(stream));
+  if (use_long)
+    return decode_long_launch(q, paged_kv, page_table, seq_lens, extra_pages, max_extra, q_len, o,
+                              lse, B, H_q, max_pages, n_pages, n_sink, n_local, scale, workspace,
+                              dev, reinterpret_cast<cudaStream_t>(stream));
 
   const int n_split = decode_splits(n_sink, n_local, max_extra);
   const int HG = (H_q + 127) / 128;

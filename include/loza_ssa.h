@@ -208,7 +208,8 @@ size_t loza_ssa_prefill_varlen_bwd_workspace_size(int n_seqs, int total_tokens, 
  *                loza_ssa_decode_workspace_size(B, H_q, d_v, n_sink, n_local)
  *                bytes, 256-byte aligned, owned by the caller, contents
  *                irrelevant on entry and overwritten.
- * Kernels: windows of up to 16 pages run as split CTAs of two pages each,
+ * Kernels: windows of up to 16 listed pages (the window's, plus any chosen
+ * ones for loza_ssa_decode_selected) run as split CTAs of two pages each,
  * merged by LSE in the same launch (or a second one); wider windows (a
  * full-attention layer is the widest) run as three launches -- a one-CTA
  * plan of each sequence's pages, CTA pairs that stream an equal share of all

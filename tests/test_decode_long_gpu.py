@@ -202,3 +202,18 @@ def test_full_attention_context_workload_sampled():
     got_o = torch.cat([o[b, torch.as_tensor(heads, device="cuda")] for b in seqs])
     got_l = torch.cat([lse[b, torch.as_tensor(heads, device="cuda")] for b in seqs])
     assert_parity(got_o, got_l, o_r, l_r, "128K full attention, sampled heads")
+
+
+@pytest.mark.parametrize("lens,max_extra,n_local", [
+    ([5000, 2048, 20000, 131072], 12, 7),   # 8 window pages + 12 chosen: 20 listed
+    ([3000, 70000, 129], 10, 12),
+])
+def test_chosen_pages_on_the_long_path(lens, max_extra, n_local):
+    """The window plus chosen pages (LongCat sparse-attention article, 机制 1
+    and 机制 3) past 16 listed pages: the chosen pages that count (between the
+    sink and the local run, each once; junk entries skipped) follow the
+    window's in each row's list."""
+    from tests.test_decode_selected_gpu import random_extra, run as selected_run
+    extra = random_extra(lens, max_extra, seed=max_extra + n_local)
+    *_, o, lse, o_ref, lse_ref = selected_run(lens, extra, seed=len(lens), n_local=n_local)
+    assert_parity(o, lse, o_ref, lse_ref, f"chosen pages {lens} x {max_extra}, local {n_local}")
