@@ -211,9 +211,12 @@ struct DecodeLayout {
   static constexpr int B_S_FULL = B_VB_FULL + 1;
   static constexpr int B_P_FULL = B_S_FULL + 1;   // 256 arrivals
   static constexpr int B_XCHG = B_P_FULL + 1;     // 256 arrivals; phase 0 max, 1 sum
-  static constexpr int B_O_FULL = B_XCHG + 1;     // phase 0: O half 1, phase 1: O half 0
-  static constexpr int B_O_EMPTY = B_O_FULL + 1;  // 256 arrivals, one phase per half
-  static constexpr int B_KA_FREE = B_O_EMPTY + 1;  // O half 1's page-A products done
+  // O output buffers: bf16 cache, two 128-column TMEM regions (quarters 3 and
+  // 1 in region 1, 2 and 0 in region 0; one phase per use); FP8 cache, index 0
+  // only (phase 0: O half 1, phase 1: O half 0)
+  static constexpr int B_O_FULL = B_XCHG + 1;      // 2
+  static constexpr int B_O_EMPTY = B_O_FULL + 2;   // 2, 256 arrivals
+  static constexpr int B_KA_FREE = B_O_EMPTY + 2;  // page A's products over boxes 4..7 done
   static constexpr int B_DRAIN = B_KA_FREE + 1;
   // FP8 cache: a stage's K boxes expanded to bf16, the V_A and the V_B boxes
   // expanded
@@ -227,7 +230,7 @@ struct DecodeLayout {
   static constexpr int OFF_SCALE = OFF_MISC + 16;
   static constexpr int SMEM_BYTES = OFF_SCALE + 2 * 2 * 128 * 4 + 1024;
   static constexpr int CHUNK8 = CHUNK / 2;  // one e4m3 box: 128 rows x 64 bytes
-  static constexpr int TMEM_COLS = 512;  // S [0,256) (P inside it), O half [256,512)
+  static constexpr int TMEM_COLS = 512;  // S [0,256) (P inside it), O [256,512)
   static constexpr int TM_O = 256;
 };
 
@@ -463,8 +466,10 @@ __device__ __forceinline__ void decode_split_body(const CUtensorMap* tm_q_p,
     mbar_init(bar(Lay::B_S_FULL), 1);
     mbar_init(bar(Lay::B_P_FULL), 256);
     mbar_init(bar(Lay::B_XCHG), 256);
-    mbar_init(bar(Lay::B_O_FULL), 1);
-    mbar_init(bar(Lay::B_O_EMPTY), 256);
+    for (int r = 0; r < 2; ++r) {
+      mbar_init(bar(Lay::B_O_FULL + r), 1);
+      mbar_init(bar(Lay::B_O_EMPTY + r), 256);
+    }
     mbar_init(bar(Lay::B_KA_FREE), 1);
     mbar_init(bar(Lay::B_DRAIN), 1);
     if (FP8) {
@@ -594,34 +599,91 @@ __device__ __forceinline__ void decode_split_body(const CUtensorMap* tm_q_p,
         mma_commit(bar(Lay::B_S_FULL));
         ok = mbar_wait(bar(Lay::B_P_FULL), 0, abort_flag, status, 1);
       }
-      // O half = P V[:, 256 columns]: V rows (keys) 16kk .. 16kk+15 of page A
-      // (then B) across four 64-column boxes one STAGE apart, MN-major; the
-      // P_A / P_B words of those keys are TMEM columns 8kk .. (128 + 8kk ..).
-      auto pv_page = [&](uint32_t v_base, uint32_t p_col, bool first) {
+      if constexpr (FP8) {
+        // O in halves of 256 columns through TMEM columns [256, 512): O half
+        // = P V[:, 256 columns]: V rows (keys) 16kk .. 16kk+15 of page A (then
+        // B) across four 64-column boxes one STAGE apart, MN-major; the P_A /
+        // P_B words of those keys are TMEM columns 8kk .. (128 + 8kk ..).
+        auto pv_page = [&](uint32_t v_base, uint32_t p_col, bool first) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(o_tm, tmem + p_col + kk * 8, sdesc_sw128(v_base + kk * 2048, Lay::STAGE, 1024),
-                 id_o, (!first || kk > 0) ? 1u : 0u);
-      };
-      if (ok) {  // half 1 (columns 256..511): the kept S stages
-        tc_fence_after();
-        pv_page(ring + Lay::CHUNK, 0, true);
-        mma_commit(bar(Lay::B_KA_FREE));  // the K_A slots may take page B's V boxes 0..3
-        if (two) pv_page(ring + 2 * Lay::CHUNK, 128, false);
-        mma_commit(bar(Lay::B_O_FULL));
-        ok = mbar_wait(bar(Lay::B_VA_FULL), 0, abort_flag, status, 1) &&
-             (!FP8 || mbar_wait(bar(Lay::B_VA_CONV), 0, abort_flag, status, 1)) &&
-             mbar_wait(bar(Lay::B_O_EMPTY), 0, abort_flag, status, 1);
-      }
-      if (ok) {  // half 0 (columns 0..255): the reloaded boxes
-        tc_fence_after();
-        pv_page(ring, 0, true);
-        if (two && (ok = mbar_wait(bar(Lay::B_VB_FULL), 0, abort_flag, status, 1) &&
-                         (!FP8 || mbar_wait(bar(Lay::B_VB_CONV), 0, abort_flag, status, 1)))) {
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(o_tm, tmem + p_col + kk * 8, sdesc_sw128(v_base + kk * 2048, Lay::STAGE, 1024),
+                   id_o, (!first || kk > 0) ? 1u : 0u);
+        };
+        if (ok) {  // half 1 (columns 256..511): the kept S stages
           tc_fence_after();
-          pv_page(ring + Lay::CHUNK, 128, false);
+          pv_page(ring + Lay::CHUNK, 0, true);
+          mma_commit(bar(Lay::B_KA_FREE));  // the K_A slots may take page B's V boxes 0..3
+          if (two) pv_page(ring + 2 * Lay::CHUNK, 128, false);
+          mma_commit(bar(Lay::B_O_FULL));
+          ok = mbar_wait(bar(Lay::B_VA_FULL), 0, abort_flag, status, 1) &&
+               mbar_wait(bar(Lay::B_VA_CONV), 0, abort_flag, status, 1) &&
+               mbar_wait(bar(Lay::B_O_EMPTY), 0, abort_flag, status, 1);
         }
-        if (ok) mma_commit(bar(Lay::B_O_FULL));
+        if (ok) {  // half 0 (columns 0..255): the reloaded boxes
+          tc_fence_after();
+          pv_page(ring, 0, true);
+          if (two && (ok = mbar_wait(bar(Lay::B_VB_FULL), 0, abort_flag, status, 1) &&
+                           mbar_wait(bar(Lay::B_VB_CONV), 0, abort_flag, status, 1))) {
+            tc_fence_after();
+            pv_page(ring + Lay::CHUNK, 128, false);
+          }
+          if (ok) mma_commit(bar(Lay::B_O_FULL));
+        }
+      } else {
+        // O in quarters of 128 columns: quarter q (V columns 128q .., boxes 2q
+        // and 2q+1) goes to TMEM region q & 1 (columns 256 + 128 (q & 1) ..),
+        // so that a quarter's products run while the output warps read the
+        // quarter before.  Quarters 3 and 2 (boxes 4..7: the kept S stages,
+        // box e in stage e - 4) first, then 1 and 0 (boxes 0..3 reloaded, box e
+        // in stage e: page A's into the Q slots, page B's into the K_A slots)
+        // as the output warps finish reading 3 and 2.  Page A's products over
+        // the kept boxes go first, so that the K_A slots are handed back for
+        // page B's reload early.  P_A / P_B words of keys 16kk .. 16kk+15 are
+        // TMEM columns 8kk .. (128 + 8kk ..).
+        const uint32_t id_q = idesc_bf16_f32(128, 128, true);
+        auto pv_quarter = [&](int q, bool page_b, bool first) {
+          const uint32_t v_base =
+              q >= 2 ? ring + (2 * q - 4) * Lay::STAGE + (page_b ? 2 : 1) * Lay::CHUNK
+                     : ring + 2 * q * Lay::STAGE + (page_b ? Lay::CHUNK : 0);
+          const uint32_t d = o_tm + 128 * (q & 1);
+          const uint32_t p_col = page_b ? 128 : 0;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(d, tmem + p_col + kk * 8, sdesc_sw128(v_base + kk * 2048, Lay::STAGE, 1024),
+                   id_q, (!first || kk > 0) ? 1u : 0u);
+        };
+        if (ok) {
+          tc_fence_after();
+          pv_quarter(3, false, true);
+          pv_quarter(2, false, true);
+          mma_commit(bar(Lay::B_KA_FREE));  // the K_A slots may take page B's V boxes 0..3
+          if (two) pv_quarter(3, true, false);
+          mma_commit(bar(Lay::B_O_FULL + 1));  // quarter 3
+          if (two) pv_quarter(2, true, false);
+          mma_commit(bar(Lay::B_O_FULL + 0));  // quarter 2
+          ok = mbar_wait(bar(Lay::B_VA_FULL), 0, abort_flag, status, 1) &&
+               mbar_wait(bar(Lay::B_O_EMPTY + 1), 0, abort_flag, status, 1);
+        }
+        if (ok) {
+          tc_fence_after();
+          pv_quarter(1, false, true);
+          ok = mbar_wait(bar(Lay::B_O_EMPTY + 0), 0, abort_flag, status, 1);
+        }
+        if (ok) {
+          tc_fence_after();
+          pv_quarter(0, false, true);
+          if (two && (ok = mbar_wait(bar(Lay::B_VB_FULL), 0, abort_flag, status, 1))) {
+            tc_fence_after();
+            pv_quarter(1, true, false);
+            mma_commit(bar(Lay::B_O_FULL + 1));  // quarter 1
+            pv_quarter(0, true, false);
+            mma_commit(bar(Lay::B_O_FULL + 0));  // quarter 0
+          } else if (ok) {
+            mma_commit(bar(Lay::B_O_FULL + 1));
+            mma_commit(bar(Lay::B_O_FULL + 0));
+          }
+        }
       }
       mma_commit(bar(Lay::B_DRAIN));
       mbar_wait_drain(bar(Lay::B_DRAIN), 0);
@@ -777,42 +839,46 @@ __device__ __forceinline__ void decode_split_body(const CUtensorMap* tm_q_p,
 
       const bool valid = hg * 128 + h < p.H_q;
       const float inv_l = 1.f / l;
-      // O half hf (1 first): warpgroup wg takes its 128 columns 128wg .. of the
-      // half, i.e. 8-column groups 32hf + 16wg + g of the row.
       uint4* dst = reinterpret_cast<uint4*>(p.o_part) + cta * (64 * 128) + h;
-      bool ok = true;
-#pragma unroll 1
-      for (int n = 0; n < 2; ++n) {
-        const int hf = 1 - n;
-        if (!(ok = mbar_wait(bar(Lay::B_O_FULL), n, abort_flag, status, 1))) break;
-        tc_fence_after();
-        if (n == 1) asm volatile("griddepcontrol.launch_dependents;");
-#pragma unroll 1
-        for (int part = 0; part < 2; ++part) {  // 64 columns at a time
-          uint32_t orr[2][32];
-          tmem_ld32(t_row + Lay::TM_O + 128 * wg + 64 * part, orr[0]);
-          tmem_ld32(t_row + Lay::TM_O + 128 * wg + 64 * part + 32, orr[1]);
-          tmem_wait_ld();
-          if (part == 1) {
-            tc_fence_before();
-            mbar_arrive(bar(Lay::B_O_EMPTY));  // the MMA may reuse the buffer now
-          }
-          if (valid) {
+      // 64 columns of O (registers orr) as fp16 into the row's 8-column groups
+      // g0 .. g0+7
+      auto emit = [&](const uint32_t (&orr)[2][32], int g0) {
+        if (!valid) return;
 #pragma unroll
-            for (int g = 0; g < 8; ++g) {
-              const uint32_t* r8 = &orr[g >> 2][(g & 3) * 8];
-              uint32_t w[4];
+        for (int g = 0; g < 8; ++g) {
+          const uint32_t* r8 = &orr[g >> 2][(g & 3) * 8];
+          uint32_t w[4];
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                __half2 hv = __floats2half2_rn(__uint_as_float(r8[2 * q]) * inv_l,
-                                               __uint_as_float(r8[2 * q + 1]) * inv_l);
-                w[q] = *reinterpret_cast<uint32_t*>(&hv);
-              }
-              dst[(32 * hf + 16 * wg + 8 * part + g) * 128] = make_uint4(w[0], w[1], w[2], w[3]);
-            }
+          for (int q = 0; q < 4; ++q) {
+            __half2 hv = __floats2half2_rn(__uint_as_float(r8[2 * q]) * inv_l,
+                                           __uint_as_float(r8[2 * q + 1]) * inv_l);
+            w[q] = *reinterpret_cast<uint32_t*>(&hv);
           }
+          dst[(size_t)(g0 + g) * 128] = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        if constexpr (FP8) {
+      };
+      bool ok = true;
+      if constexpr (FP8) {
+        // O half hf (1 first): warpgroup wg takes its 128 columns 128wg .. of
+        // the half, i.e. 8-column groups 32hf + 16wg + g of the row.
+#pragma unroll 1
+        for (int n = 0; n < 2; ++n) {
+          const int hf = 1 - n;
+          if (!(ok = mbar_wait(bar(Lay::B_O_FULL), n, abort_flag, status, 1))) break;
+          tc_fence_after();
+          if (n == 1) asm volatile("griddepcontrol.launch_dependents;");
+#pragma unroll 1
+          for (int part = 0; part < 2; ++part) {  // 64 columns at a time
+            uint32_t orr[2][32];
+            tmem_ld32(t_row + Lay::TM_O + 128 * wg + 64 * part, orr[0]);
+            tmem_ld32(t_row + Lay::TM_O + 128 * wg + 64 * part + 32, orr[1]);
+            tmem_wait_ld();
+            if (part == 1) {
+              tc_fence_before();
+              mbar_arrive(bar(Lay::B_O_EMPTY));  // the MMA may reuse the buffer now
+            }
+            emit(orr, 32 * hf + 16 * wg + 8 * part);
+          }
           // page B's V columns 0..255, reloaded into the K_A slots, to bf16
           // (once O half 1 is done, so page A's boxes there are read): boxes
           // 2wg and 2wg+1 by warpgroup wg
@@ -825,6 +891,26 @@ __device__ __forceinline__ void decode_split_body(const CUtensorMap* tm_q_p,
             fence_async_shared();
             mbar_arrive(bar(Lay::B_VB_CONV));
           }
+        }
+      } else {
+        // O quarter q (3 first) in TMEM region q & 1: warpgroup wg takes its 64
+        // columns 64wg .. of the quarter, i.e. 8-column groups 16q + 8wg + g of
+        // the row; reading quarters 3 and 2 frees their region for 1 and 0.
+#pragma unroll 1
+        for (int n = 0; n < 4; ++n) {
+          const int q = 3 - n, r = q & 1;
+          if (!(ok = mbar_wait(bar(Lay::B_O_FULL + r), n >> 1, abort_flag, status, 1))) break;
+          tc_fence_after();
+          if (n == 3) asm volatile("griddepcontrol.launch_dependents;");
+          uint32_t orr[2][32];
+          tmem_ld32(t_row + Lay::TM_O + 128 * r + 64 * wg, orr[0]);
+          tmem_ld32(t_row + Lay::TM_O + 128 * r + 64 * wg + 32, orr[1]);
+          tmem_wait_ld();
+          if (n < 2) {
+            tc_fence_before();
+            mbar_arrive(bar(Lay::B_O_EMPTY + r));  // the MMA may write quarter q - 2 here
+          }
+          emit(orr, 16 * q + 8 * wg);
         }
       }
       if (ok && valid && wg == 0) p.lse_part[cta * 128 + h] = (m + __log2f(l)) * kLn2;
