@@ -194,6 +194,22 @@ __host__ __device__ __forceinline__ long long long_pair_start(int k, long long T
 __host__ __device__ __forceinline__ int long_pairs(int launched, long long T) {
   return (int)(T < launched ? (T > 0 ? T : 1) : launched);
 }
+// Partial slots of unit u, whose pages are [lo, lo + n) of the T listed, with P
+// pairs: one per pair its pages reach, slots u + k for those pairs k
+// (consecutive), so *first = u + (first pair) and *count = the pairs reached
+// (0 for a unit without pages).
+__host__ __device__ __forceinline__ void long_unit_slot_range(int u, long long lo, int n,
+                                                              long long T, int P, int* first,
+                                                              int* count) {
+  if (n <= 0) {
+    *first = 0;
+    *count = 0;
+    return;
+  }
+  const int kf = long_pair_of(lo, T, P), kl = long_pair_of(lo + n - 1, T, P);
+  *first = u + kf;
+  *count = kl - kf + 1;
+}
 
 struct DecodeLayout {
   static constexpr int CHUNK = 128 * 128;        // [128 rows x 64 bf16], 128B swizzle

@@ -148,14 +148,7 @@ __global__ void __launch_bounds__(kLongPlanThreads, 1)
   for (int u = u0; u < u1; ++u) {
     plan[u] = run;
     const int n = long_unit_pages(p, u);
-    int first = 0, cnt = 0;
-    if (n > 0) {
-      const int kf = long_pair_of(run, T, P), kl = long_pair_of(run + n - 1, T, P);
-      first = u + kf;
-      cnt = kl - kf + 1;
-    }
-    slots[2 * u] = first;
-    slots[2 * u + 1] = cnt;
+    long_unit_slot_range(u, run, n, T, P, slots + 2 * u, slots + 2 * u + 1);
     run += n;
   }
   if (threadIdx.x == kLongPlanThreads - 1) plan[U] = run;

@@ -1213,6 +1213,26 @@ int loza_ssa_debug_wait_timeout(int timeout_us, int* result, loza_ssa_stream_t s
   return e == cudaSuccess ? LOZA_SSA_OK : cuda_fail(e, "debug wait-timeout launch");
 }
 
+int loza_ssa_debug_long_partition(const int* unit_pages, int n_units, int pairs_launched,
+                                  long long* pair_start, int* slot_first, int* slot_count) {
+  if (!unit_pages || !pair_start || !slot_first || !slot_count) return LOZA_SSA_ERR_NULL;
+  if (n_units < 1 || pairs_launched < 1) return LOZA_SSA_ERR_SHAPE;
+  long long T = 0;
+  for (int u = 0; u < n_units; ++u) {
+    if (unit_pages[u] < 0) return LOZA_SSA_ERR_SHAPE;
+    T += unit_pages[u];
+  }
+  const int P = loza::long_pairs(pairs_launched, T);
+  for (int k = 0; k <= pairs_launched; ++k)
+    pair_start[k] = k <= P ? loza::long_pair_start(k, T, P) : T;
+  long long run = 0;
+  for (int u = 0; u < n_units; ++u) {
+    loza::long_unit_slot_range(u, run, unit_pages[u], T, P, slot_first + u, slot_count + u);
+    run += unit_pages[u];
+  }
+  return LOZA_SSA_OK;
+}
+
 int loza_ssa_debug_decode_pages(const int* page_table, const int* seq_lens, int B, int max_pages,
                                 int n_pages, int page_size, int n_sink, int n_local, int* pages,
                                 int* counts, int max_tiles, loza_ssa_stream_t stream) {

@@ -109,6 +109,8 @@ def lib() -> ctypes.CDLL:
         L.loza_ssa_debug_decode_pages.restype = i32
         L.loza_ssa_debug_wait_timeout.argtypes = [i32, vp, vp]
         L.loza_ssa_debug_wait_timeout.restype = i32
+        L.loza_ssa_debug_long_partition.argtypes = [vp, i32, i32, vp, vp, vp]
+        L.loza_ssa_debug_long_partition.restype = i32
         L.loza_ssa_decode_static_scratch.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
                                                      i32, i32, i32, i32, i32, f32, vp]
         L.loza_ssa_decode_static_scratch.restype = i32
@@ -582,3 +584,19 @@ def loza_ssa_debug_wait_timeout(timeout_us, device="cuda", stream=None):
     result = torch.full((2,), -1, dtype=torch.int32, device=device)
     _check(lib().loza_ssa_debug_wait_timeout(int(timeout_us), _ptr(result), _stream(stream)))
     return result
+
+
+def loza_ssa_debug_long_partition(unit_pages, pairs_launched):
+    """Host arithmetic of the long-window decode's page split (no device
+    work): for the pages each (row, head group) unit lists, returns
+    (pair_start int64 [pairs_launched + 1], slot_first int32 [units],
+    slot_count int32 [units])."""
+    import numpy as np
+    pages = np.ascontiguousarray(unit_pages, dtype=np.int32)
+    start = np.zeros(int(pairs_launched) + 1, dtype=np.int64)
+    first = np.zeros(pages.size, dtype=np.int32)
+    count = np.zeros(pages.size, dtype=np.int32)
+    _check(lib().loza_ssa_debug_long_partition(
+        pages.ctypes.data, int(pages.size), int(pairs_launched), start.ctypes.data,
+        first.ctypes.data, count.ctypes.data))
+    return start, first, count

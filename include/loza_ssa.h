@@ -383,6 +383,19 @@ int loza_ssa_debug_enumerate_tiles(int n_qblocks, int n_sink, int n_local, int* 
 int loza_ssa_debug_wait_timeout(int timeout_us, int* result, loza_ssa_stream_t stream);
 
 /*
+ * Debug, HOST arithmetic only (no device work): how the long-window decode
+ * shares the listed pages of n_units (row, head group) units over CTA pairs,
+ * computed with the inline functions its kernels use.  unit_pages: HOST int32
+ * [n_units], pages each unit lists (>= 0).  Outputs (HOST): pair_start int64
+ * [pairs_launched + 1], the first page of pair k in the flattened list (pairs
+ * past the ones used start at the total); slot_first / slot_count int32
+ * [n_units], the unit's partial slots.  Returns LOZA_SSA_OK, or
+ * LOZA_SSA_ERR_NULL / LOZA_SSA_ERR_SHAPE.
+ */
+int loza_ssa_debug_long_partition(const int* unit_pages, int n_units, int pairs_launched,
+                                  long long* pair_start, int* slot_first, int* slot_count);
+
+/*
  * Debug: run the decode kernel's page selection on the device.  For every
  * sequence b writes the PHYSICAL pages the decode window reads (logical order)
  * to pages[b*max_tiles ...] and their number to counts[b]; entries it would

@@ -402,3 +402,50 @@ def test_debug_wait_timeout_argument_errors(L):
     assert L.loza_ssa_debug_wait_timeout(0, vp(0x1000), None) == -2
     assert L.loza_ssa_debug_wait_timeout(100001, vp(0x1000), None) == -2
     assert L.loza_ssa_debug_wait_timeout(1000, vp(0x1002), None) == -6
+
+
+def test_long_partition_arithmetic(L):
+    """The long-window decode's split of all listed pages over CTA pairs (the
+    library's own host/device arithmetic, run on the host): every pair used
+    gets a non-empty run and the runs tile the page list; a unit's partial
+    slots are exactly the pairs whose runs reach its pages, each slot written
+    by one (unit, pair) run, inside the workspace's units + pairs slots.
+    Checked against brute force: each page's owning pair by scanning the runs.
+    Fewer pages than pairs, units without pages and all-empty lists included."""
+    import numpy as np
+    from block_sparse_streaming_ssa_b200 import loza_ssa as api
+    rng = np.random.default_rng(0)
+    cases = [([18], 74), ([0, 0, 0], 5), ([1, 1, 2, 17], 74), ([1024] * 32, 74),
+             ([3, 0, 5, 100], 4)]
+    for _ in range(300):
+        n = int(rng.integers(1, 40))
+        pages = [int(x) for x in rng.choice([0, 1, 2, 7, 16, 64, int(rng.integers(0, 600))], n)]
+        cases.append((pages, int(rng.choice([1, 2, 3, 74, 128]))))
+    for pages, launched in cases:
+        start, first, count = api.loza_ssa_debug_long_partition(pages, launched)
+        T = sum(pages)
+        used = min(launched, max(T, 1))
+        assert start[0] == 0 and start[used] == T and np.all(np.diff(start) >= 0)
+        assert np.all(start[used:] == T)
+        if T > 0:
+            assert np.all(np.diff(start[:used + 1]) >= 1), (pages, launched)
+        owner = np.searchsorted(start[:used + 1], np.arange(T), side="right") - 1
+        off = np.concatenate([[0], np.cumsum(pages)])
+        seen = set()
+        for u, nu in enumerate(pages):
+            if nu == 0:
+                assert count[u] == 0
+                continue
+            ks = sorted(set(owner[off[u]:off[u + 1]].tolist()))
+            assert ks == list(range(ks[0], ks[-1] + 1))
+            assert first[u] == u + ks[0] and count[u] == len(ks), (pages, launched, u)
+            for k in ks:
+                slot = u + k
+                assert slot not in seen and slot < len(pages) + launched
+                seen.add(slot)
+    assert api.lib().loza_ssa_debug_long_partition(None, 1, 1, None, None, None) == -1
+    bad = np.array([-1], dtype=np.int32)
+    out = np.zeros(2, dtype=np.int64)
+    s = np.zeros(1, dtype=np.int32)
+    assert api.lib().loza_ssa_debug_long_partition(bad.ctypes.data, 1, 1, out.ctypes.data,
+                                                   s.ctypes.data, s.ctypes.data) == -2
