@@ -57,3 +57,26 @@ def test_rejects_more_than_the_scratch_holds():
         1, 7, ctypes.c_float(1 / 24.0), vp(torch.cuda.current_stream().cuda_stream))
     assert rc == LOZA_SSA_ERR_SCRATCH_LIMIT
     assert b"split slots" in lib().loza_ssa_last_error_string()
+
+
+def test_wide_window_stays_on_the_split_kernel():
+    """A window of more than 16 pages: loza_ssa_decode takes the long-window
+    kernel, the static-scratch call keeps the split kernel its scratch is
+    sized for (2 sequences x 10 splits = 20 of the 128 slots); both match the
+    oracle."""
+    import numpy as np
+    from oracle import ssa_oracle as orc
+    from tests.test_decode_gpu import compact_for_oracle
+    scale = 1 / 24.0
+    lens = [5000, 20000]
+    q, kv, pt, sl = synth.decode_inputs(lens, 128, D_QK, seed=4, device="cuda")
+    o_s, lse_s = loza_ssa_decode_static_scratch(q, kv, pt, sl, D_V, n_sink=1, n_local=19,
+                                                scale=scale)
+    o_w, lse_w = loza_ssa_decode(q, kv, pt, sl, D_V, n_sink=1, n_local=19, scale=scale)
+    torch.cuda.synchronize()
+    assert loza_ssa_get_last_device_status() == 0
+    kv_h, pt_h, sl_h = compact_for_oracle(kv, pt, sl, 1, 19)
+    o_r, l_r = orc.decode(synth.bf16_bits(q), kv_h, pt_h, sl_h, D_V, 128, 1, 19, scale)
+    assert_parity(o_s, lse_s, o_r, l_r, "static scratch, 20-page window")
+    assert_parity(o_w, lse_w, o_r, l_r, "workspace call, 20-page window")
+    assert np.isfinite(o_s.float().cpu().numpy()).all()
