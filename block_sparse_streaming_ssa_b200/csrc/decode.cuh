@@ -520,6 +520,15 @@ __device__ __forceinline__ void decode_split_body(const CUtensorMap* tm_q_p,
       const uint32_t s_bytes = Lay::CHUNK + (two ? 2 : 1) * kbox;
       int issued = 0;        // S stages issued
       bool va = false, vb = false;
+      // With one head group and one token per sequence no other CTA reads this
+      // CTA's pages: the boxes it reads for the last time (boxes 4..8 in S,
+      // 0..3 when reloaded as values) are marked first to leave L2.
+      const bool once = p.HG == 1 && p.q_len == 1;
+      const uint64_t pol = l2_policy_evict_first();
+      auto load_k = [&](uint32_t dst_k, uint32_t fb, int c, int page, bool last_read) {
+        if (once && last_read) tma_load_2d_hint(dst_k, &tm_kv, fb, c * 64, page * 128, pol);
+        else tma_load_2d(dst_k, &tm_kv, fb, c * 64, page * 128);
+      };
       do {
         for (int i = 0; i < Lay::KV_CH; ++i) {
           const int st = decode_s_stage(i), r = decode_s_round(i);
@@ -529,8 +538,8 @@ __device__ __forceinline__ void decode_split_body(const CUtensorMap* tm_q_p,
           const uint32_t dst = ring + st * Lay::STAGE, full = bar(Lay::B_FULL + st);
           mbar_arrive_expect_tx(full, s_bytes);
           tma_load_3d(dst, &tm_q, full, c * 64, hg * 128, b);
-          tma_load_2d(dst + Lay::CHUNK + koff, &tm_kv, full, c * 64, phys_a * 128);
-          if (two) tma_load_2d(dst + 2 * Lay::CHUNK + koff, &tm_kv, full, c * 64, phys_b * 128);
+          load_k(dst + Lay::CHUNK + koff, full, c, phys_a, c >= 4);
+          if (two) load_k(dst + 2 * Lay::CHUNK + koff, full, c, phys_b, c >= 4);
           ++issued;
           if (i == 0) {
             // A CTA one wave later starts only when an SM frees up: pull its
@@ -564,15 +573,13 @@ __device__ __forceinline__ void decode_split_body(const CUtensorMap* tm_q_p,
         if (!mbar_wait(bar(Lay::B_S_FULL), 0, abort_flag, status, 1)) break;
         mbar_arrive_expect_tx(bar(Lay::B_VA_FULL), 4 * kbox);
         for (int e = 0; e < 4; ++e)
-          tma_load_2d(ring + e * Lay::STAGE + koff, &tm_kv, bar(Lay::B_VA_FULL), e * 64,
-                      phys_a * 128);
+          load_k(ring + e * Lay::STAGE + koff, bar(Lay::B_VA_FULL), e, phys_a, true);
         va = true;
         if (!two) break;
         if (!mbar_wait(bar(Lay::B_KA_FREE), 0, abort_flag, status, 1)) break;
         mbar_arrive_expect_tx(bar(Lay::B_VB_FULL), 4 * kbox);
         for (int e = 0; e < 4; ++e)
-          tma_load_2d(ring + e * Lay::STAGE + Lay::CHUNK + koff, &tm_kv, bar(Lay::B_VB_FULL),
-                      e * 64, phys_b * 128);
+          load_k(ring + e * Lay::STAGE + Lay::CHUNK + koff, bar(Lay::B_VB_FULL), e, phys_b, true);
         vb = true;
       } while (false);
       // every copy issued lands before the CTA exits

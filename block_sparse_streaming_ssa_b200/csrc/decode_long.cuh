@@ -267,13 +267,21 @@ __global__ void __launch_bounds__(LongDecodeLayout::THREADS, 1)
       LongSeg sg;
       int n_ld = 0, g = 0;
       bool ok = true;
+      // With one head group and one token per sequence a page is read by this
+      // pair alone; a value box, reloaded after both CTAs' S products read it,
+      // is then read for the last time and is marked first to leave L2.
+      const bool once = p.HG == 1 && p.q_len == 1;
+      const uint64_t pol = l2_policy_evict_first();
       // c >= 0: K box c of physical page phys; c < 0: Q box -c-1 of the segment's row
-      auto ring_load = [&](int c, int phys, const LongSeg& s) -> bool {
+      auto ring_load = [&](int c, int phys, const LongSeg& s, bool last_read = false) -> bool {
         const int slot = n_ld % Lay::NSLOT, r = n_ld / Lay::NSLOT;
         if (r > 0 && !mbar_wait(bar(Lay::B_EMPTY + slot), (r - 1) & 1, abort_flag, status, 1))
           return false;
         mbar_arrive_expect_tx(bar(Lay::B_FULL + slot), Lay::CHUNK);
-        if (c >= 0)
+        if (c >= 0 && once && last_read)
+          tma_load_2d_hint(ring + slot * Lay::CHUNK, &tm_kv, bar(Lay::B_FULL + slot), c * 64,
+                           phys * 128, pol);
+        else if (c >= 0)
           tma_load_2d(ring + slot * Lay::CHUNK, &tm_kv, bar(Lay::B_FULL + slot), c * 64, phys * 128);
         else
           tma_load_3d(ring + slot * Lay::CHUNK, &tm_q, bar(Lay::B_FULL + slot), (-c - 1) * 64,
@@ -316,11 +324,11 @@ __global__ void __launch_bounds__(LongDecodeLayout::THREADS, 1)
             if (ok) ok = ring_load(c, cur, sg);
           }
           for (int j = 0; j < Lay::V_CH && ok && prev >= 0; ++j)
-            ok = ring_load(4 * half + j, prev, sg);
+            ok = ring_load(4 * half + j, prev, sg, true);
           prev = cur;
           cur = nxt;
         }
-        for (int j = 0; j < Lay::V_CH && ok; ++j) ok = ring_load(4 * half + j, prev, sg);
+        for (int j = 0; j < Lay::V_CH && ok; ++j) ok = ring_load(4 * half + j, prev, sg, true);
       }
       // every copy issued lands before the CTA exits
       drain_ring(bar(Lay::B_FULL), Lay::NSLOT, n_ld);
