@@ -94,6 +94,18 @@ def source_hash(kernel: str) -> str:
     return h.hexdigest()[:12]
 
 
+REST_S = 1.0
+
+
+def rest():
+    """Idle the GPU for REST_S seconds between two workloads' measurements, so
+    that each starts as it would alone (the power limiter of a 1 kW part reacts
+    to the last tens of ms of load; the pause is outside every timed region)."""
+    import torch
+    torch.cuda.synchronize()
+    time.sleep(REST_S)
+
+
 def traffic_lookup(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the current kernel sources (else None)."""
@@ -786,6 +798,7 @@ def main():
         torch.cuda.set_device(0)
 
     def decode_legs():
+        rest()
         legs = {"decode": decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
                                        len_hi=args.decode_len_hi, world=world)}
         if args.decode_extra:
@@ -800,6 +813,7 @@ def main():
             legs["dec_fp8"] = decode_bench(args.decode_iters, args.warmup, peaks, seed=rank,
                                            len_hi=args.decode_len_hi, world=world, fp8=True)
         if args.decode_context:
+            rest()
             legs["ctx_dec"] = context_bench(peaks, args.decode_context, world=world, seed=rank)
         return legs
 
@@ -833,10 +847,12 @@ def main():
     e2e_val = None if e2e_ms is None else world * t["flops"] / (e2e_ms * 1e-3) / 1e12
     w_desc, w_spec = w["desc"], w["spec"]
     detail = {"headline": {"workload": w_desc, **head_entry,
-                           "e2e_ms": e2e_ms and round(e2e_ms, 3), "clocks": t["clocks"]}}
+                           "e2e_ms": e2e_ms and round(e2e_ms, 3), "clocks": t["clocks"]},
+              "idle_s_before_each_other_workload": REST_S}
     configs = {}
     backwards = {}
     if not args.no_backward:
+        rest()
         b = backward_bench(w, max(3, args.steps // 4), args.warmup, peaks, world)
         if b is not None:
             backwards[f"bwd_{args.config}"] = b
@@ -848,11 +864,13 @@ def main():
         for other in ("mha", "varlen", "mla"):
             if other == args.config:
                 continue
+            rest()
             w2, entry, _ = prefill_leg(other, args.steps, args.warmup, peaks, dist, world, rank)
             # the line keeps rates and fractions; times and workloads go to the detail
             configs[other] = {k: entry[k] for k in ("tflops", "frac", "mtok_s")}
             detail[other] = {"workload": w2["desc"]["workload"], **entry}
             if other == "mha" and not args.no_backward:
+                rest()
                 backwards["bwd_mha"] = backward_bench(w2, max(3, args.steps // 4), args.warmup,
                                                       peaks, world)
             del w2
@@ -861,6 +879,7 @@ def main():
         configs[name] = compact("bwd", b)
         detail[name] = b
     if args.prefill_context:
+        rest()
         pctx = prefill_context_bench(peaks, args.prefill_context, world=world, seed=rank)
         detail["ctx_pre"] = pctx
     if not args.no_decode:
