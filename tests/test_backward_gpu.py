@@ -174,3 +174,29 @@ def test_backward_full_size_heads():
     ref = orc.prefill_bwd(*(synth.bf16_bits(t[:, hsel]) for t in (q, k, v, dout)), blk=128,
                           n_sink=1, n_local=7, scale=spec.scale)
     check([t[:, hsel] for t in (dq, dk, dv)], ref, "mha 32K, heads 0/11/22/31")
+
+
+def test_backward_mla_full_size_heads():
+    """The benchmarked MLA-dims workload (B=1, H=64, L=131072, d_qk=192, d_v=128,
+    N(0,1) with the sink tokens' keys boosted): the whole backward call on the GPU, so that key block 0's 1024
+    query blocks run as 128 sink chunks through the partial-sum reduction; four
+    heads compared in full (every row of dq, dk, dv) with the oracle's float64
+    gradients.  The oracle walks a plane's rows in order, so the four heads cost
+    one plane's time on four host threads."""
+    spec = synth.MLA
+    q, k, v = synth.prefill_spec_inputs(spec, seed=0, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(4343)
+    dout = torch.randn(v.shape, generator=g, device="cuda").to(torch.bfloat16)
+    o, lse = loza_ssa_prefill(q, k, v, scale=spec.scale)
+    dq, dk, dv = loza_ssa_prefill_bwd(q, k, v, o, lse, dout, scale=spec.scale)
+    torch.cuda.synchronize()
+    assert loza_ssa_get_last_device_status() == 0
+    heads = [0, 21, 42, 63]
+    hsel = torch.as_tensor(heads, device="cuda")
+    sel = [t[:, hsel].cpu() for t in (q, k, v, dout)]
+    got = [t[:, hsel].cpu() for t in (dq, dk, dv)]
+    del q, k, v, o, lse, dout, dq, dk, dv
+    torch.cuda.empty_cache()
+    ref = orc.prefill_bwd(*(synth.bf16_bits(t) for t in sel), blk=128, n_sink=1, n_local=7,
+                          scale=spec.scale)
+    check(got, ref, "mla 128K, heads 0/21/42/63")
