@@ -31,6 +31,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -85,12 +86,22 @@ KERNEL_SOURCES = {
 }
 
 
+def code_only(src: str) -> str:
+    """A source file without its comments, whitespace runs collapsed: an edit of
+    comments alone leaves source_hash, and the traffic records keyed by it, as
+    they were (the kernel sources hold no comment markers inside strings)."""
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return re.sub(r"\s+", " ", src).strip()
+
+
 def source_hash(kernel: str) -> str:
+    """Hash of the code (comments left out) of the files a kernel is built from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_sparse_streaming_ssa_b200", "csrc")
     for name in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update((name + "\n" + code_only(f.read())).encode())
     return h.hexdigest()[:12]
 
 

@@ -521,8 +521,10 @@ __device__ __forceinline__ void decode_split_body(const CUtensorMap* tm_q_p,
       int issued = 0;        // S stages issued
       bool va = false, vb = false;
       // With one head group and one token per sequence no other CTA reads this
-      // CTA's pages: the boxes it reads for the last time (boxes 4..8 in S,
-      // 0..3 when reloaded as values) are marked first to leave L2.
+      // CTA's pages (unless the page table maps two sequences to one page): the
+      // boxes it reads for the last time (boxes 4..8 in S, 0..3 when reloaded as
+      // values) are marked first to leave L2.  The policy only orders evictions;
+      // a shared page read again later comes from DRAM, with the same values.
       const bool once = p.HG == 1 && p.q_len == 1;
       const uint64_t pol = l2_policy_evict_first();
       auto load_k = [&](uint32_t dst_k, uint32_t fb, int c, int page, bool last_read) {

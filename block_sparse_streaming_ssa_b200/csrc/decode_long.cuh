@@ -268,8 +268,10 @@ __global__ void __launch_bounds__(LongDecodeLayout::THREADS, 1)
       int n_ld = 0, g = 0;
       bool ok = true;
       // With one head group and one token per sequence a page is read by this
-      // pair alone; a value box, reloaded after both CTAs' S products read it,
-      // is then read for the last time and is marked first to leave L2.
+      // pair alone (unless the page table maps two sequences to one page); a
+      // value box, reloaded after both CTAs' S products read it, is then read
+      // for the last time and is marked first to leave L2.  The policy only
+      // orders evictions, never what a load returns.
       const bool once = p.HG == 1 && p.q_len == 1;
       const uint64_t pol = l2_policy_evict_first();
       // c >= 0: K box c of physical page phys; c < 0: Q box -c-1 of the segment's row
