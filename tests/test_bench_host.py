@@ -76,3 +76,12 @@ def test_window_pairs_matches_oracle_row_counts(L):
     rows = np.arange(L)
     want = sum(orc.row_count(int(i), 128, 1, 7) for i in rows)
     assert bench.window_pairs(L) == want
+
+
+def test_source_hash_ignores_comments_only():
+    """The traffic records are keyed by a hash of the kernel code without its
+    comments: an edit of comments keeps the hash, an edit of code changes it."""
+    src = "int f(int a) { // add one\n  return a + 1; /* the\n result */ }\n"
+    assert bench.code_only(src) == bench.code_only(
+        "int f(int a) {\n  // a different comment\n  return a + 1;\n}\n")
+    assert bench.code_only(src) != bench.code_only(src.replace("a + 1", "a + 2"))
