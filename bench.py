@@ -205,6 +205,27 @@ def job_throughput(world: int, units_per_rank_step: float, steps: int, max_ms: f
 
 # ---------------------------------------------------------------- prefill
 
+def workload_name(config, seed=0, heads=None):
+    """The prefill workload's description, as the detailed record gives it (no
+    device work: the packed workload's lengths come from the seeded host draw)."""
+    from block_sparse_streaming_ssa_b200 import synth
+    if config == "varlen":
+        sp = synth.VARLEN
+        lengths = synth.varlen_lengths(seed, sp.n_seqs, sp.len_lo, sp.len_hi, sp.total_cap)
+        return (f"ssa_prefill_varlen {sp.n_seqs} seqs (total {sum(lengths)} tokens) "
+                f"H={sp.H} d_qk=d_v={sp.d_qk} bf16, 1 sink + 7 local blocks of 128")
+    sp = {"tiny": synth.TINY, "mha": synth.MHA, "mla": synth.MLA}[config]
+    H = heads or sp.H
+    return (f"ssa_prefill_{sp.name} B={sp.B} H={H} L={sp.L} d_qk={sp.d_qk} "
+            f"d_v={sp.d_v} bf16, 1 sink + 7 local blocks of 128")
+
+
+def line_config(workload):
+    """The JSON line's `config` for a prefill workload (both arms give the same)."""
+    return {"workload": workload.replace(" bf16, 1 sink + 7 local blocks of 128", " 1+7x128"),
+            "parallelism": "replicas", "l2": "inputs > L2"}
+
+
 def make_prefill(config, device, seed, heads=None):
     """The prefill workload ``config``; ``heads`` (dense workloads only) keeps
     the shapes but takes that many heads, for profiler captures of a smaller
@@ -216,8 +237,7 @@ def make_prefill(config, device, seed, heads=None):
         lengths = synth.varlen_lengths(seed, sp.n_seqs, sp.len_lo, sp.len_hi, sp.total_cap)
         q, k, v, cu = synth.varlen_inputs(lengths, sp.H, sp.d_qk, sp.d_v, seed=seed, device=device)
         pairs = sp.H * sum(window_pairs(n) for n in lengths)
-        desc = {"workload": f"ssa_prefill_varlen {sp.n_seqs} seqs (total {sum(lengths)} tokens) "
-                            f"H={sp.H} d_qk=d_v={sp.d_qk} bf16, 1 sink + 7 local blocks of 128",
+        desc = {"workload": workload_name(config, seed),
                 "lengths": lengths, "H": sp.H, "d_qk": sp.d_qk, "d_v": sp.d_v}
         tokens = sum(lengths)
         return dict(spec=sp, q=q, k=k, v=v, cu=cu, max_len=max(lengths), pairs=pairs,
@@ -227,8 +247,7 @@ def make_prefill(config, device, seed, heads=None):
         sp = dataclasses.replace(sp, H=heads)
     q, k, v = synth.prefill_spec_inputs(sp, seed=seed, device=device)
     pairs = sp.B * sp.H * window_pairs(sp.L)
-    desc = {"workload": f"ssa_prefill_{sp.name} B={sp.B} H={sp.H} L={sp.L} d_qk={sp.d_qk} "
-                        f"d_v={sp.d_v} bf16, 1 sink + 7 local blocks of 128",
+    desc = {"workload": workload_name(config, seed, heads),
             "B": sp.B, "H": sp.H, "L": sp.L, "d_qk": sp.d_qk, "d_v": sp.d_v}
     return dict(spec=sp, q=q, k=k, v=v, cu=None, pairs=pairs, tokens=sp.B * sp.L, desc=desc,
                 varlen=False)
@@ -789,7 +808,7 @@ def main():
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": t_tot / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"ssa_prefill_{args.config} (CPU oracle, row sample per step)"},
+            "config": line_config(workload_name(args.config)),
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -918,9 +937,7 @@ def main():
         "ms_per_step": round(t["max_ms"] / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": w_desc["workload"].replace(" bf16, 1 sink + 7 local blocks of 128",
-                                                          " 1+7x128"),
-                   "parallelism": "replicas", "l2": "inputs > L2"},
+        "config": line_config(w_desc["workload"]),
         "tokens_per_s": round(t["tok_s"]),
         "roofline": {"bound": "tensor", "achieved": round(t["achieved"], 1), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(t["achieved"] / peak, 4),
