@@ -341,6 +341,7 @@ __global__ void __launch_bounds__(LongDecodeLayout::THREADS, 1)
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16_f32(128, 128, false);
       const uint32_t id_o = idesc_bf16_f32(128, 64, true);
+      const uint32_t id_o2 = idesc_bf16_f32(128, 128, true);
       LongWalk wk = walk0;
       LongSeg sg;
       int n_ld = 0, f = 0, g = 0;
@@ -387,19 +388,26 @@ __global__ void __launch_bounds__(LongDecodeLayout::THREADS, 1)
           return false;
         if (first && g > 0 && !mbar_wait(bar(Lay::B_O_FREE), (g - 1) & 1, abort_flag, status, 1))
           return false;
-        for (int j = 0; j < Lay::V_CH; ++j) {
+        for (int j = 0; j < Lay::V_CH;) {
+          // two value boxes in adjacent ring slots (no wrap-around) are one
+          // N = 128 operand, 64-column chunks one slot apart; else one box
           const int slot = n_ld % Lay::NSLOT;
-          if (!mbar_wait(bar(Lay::B_FULL + slot), (n_ld / Lay::NSLOT) & 1, abort_flag, status, 1))
+          const bool two_box = j + 1 < Lay::V_CH && slot + 1 < Lay::NSLOT;
+          const uint32_t ph = (n_ld / Lay::NSLOT) & 1;  // the same phase for slot + 1
+          if (!mbar_wait(bar(Lay::B_FULL + slot), ph, abort_flag, status, 1) ||
+              (two_box && !mbar_wait(bar(Lay::B_FULL + slot + 1), ph, abort_flag, status, 1)))
             return false;
           tc_fence_after();
           const uint32_t vb = ring + slot * Lay::CHUNK;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(tmem + Lay::TM_O + 64 * j, tmem + 128 * b2 + 8 * kk,
-                   sdesc_sw128(vb + kk * 2048, Lay::CHUNK, 1024), id_o,
+                   sdesc_sw128(vb + kk * 2048, Lay::CHUNK, 1024), two_box ? id_o2 : id_o,
                    (!first || kk > 0) ? 1u : 0u);
           mma_commit(bar(Lay::B_EMPTY + slot));
-          ++n_ld;
+          if (two_box) mma_commit(bar(Lay::B_EMPTY + slot + 1));
+          n_ld += two_box ? 2 : 1;
+          j += two_box ? 2 : 1;
         }
         mma_commit(bar(Lay::B_S_FREE + b2));
         mma_commit(bar(Lay::B_O_DONE));
