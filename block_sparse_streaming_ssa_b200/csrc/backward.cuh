@@ -37,8 +37,8 @@
 
 namespace loza {
 
-// warps 0-7 compute, 8 TMA producer, 9 and 10 MMA issuers
-constexpr int kBwdThreads = 352;
+// warps 0-7 compute, 8 TMA producer, 9, 10 and 11 MMA issuers
+constexpr int kBwdThreads = 384;
 constexpr int kBwdComputeThreads = 256;
 constexpr int kSinkChunk = 8;        // query blocks per sink work item
 
@@ -300,8 +300,8 @@ struct BwdDqLayout {
   static constexpr int B_DS_FREE = B_DS_FULL + 1;     // dQ MMA of the tile done
   static constexpr int B_DQ_FULL = B_DS_FREE + 1;     // the item's last dQ MMA done
   static constexpr int B_DQ_EMPTY = B_DQ_FULL + 1;    // epilogue has read dQ
-  static constexpr int B_DRAIN = B_DQ_EMPTY + 1;     // 2: one per MMA issuer
-  static constexpr int NBAR = B_DRAIN + 2;
+  static constexpr int B_DRAIN = B_DQ_EMPTY + 1;     // 3: one per MMA issuer
+  static constexpr int NBAR = B_DRAIN + 3;
   static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;  // [0] tmem base, [1] abort
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(Lay::B_QD_FULL), 1);
-    mbar_init(bar(Lay::B_QD_EMPTY), 1);
+    mbar_init(bar(Lay::B_QD_EMPTY), 2);  // the S and the dP issuer
     for (int s = 0; s < Lay::KST; ++s) {
       mbar_init(bar(Lay::B_K_FULL + s), 1);
       mbar_init(bar(Lay::B_K_EMPTY + s), 1);
@@ -336,7 +336,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bar(Lay::B_V_FULL + s), 1);
       mbar_init(bar(Lay::B_V_EMPTY + s), 1);
     }
-    mbar_init(bar(Lay::B_S_FULL), 1);
+    mbar_init(bar(Lay::B_S_FULL), 2);  // S and dP, one commit from each issuer
     mbar_init(bar(Lay::B_SDP_FREE), kBwdComputeThreads);
     mbar_init(bar(Lay::B_DS_FULL), kBwdComputeThreads);
     mbar_init(bar(Lay::B_DS_FREE), 1);
@@ -344,6 +344,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(bar(Lay::B_DQ_EMPTY), kBwdComputeThreads);
     mbar_init(bar(Lay::B_DRAIN), 1);
     mbar_init(bar(Lay::B_DRAIN + 1), 1);
+    mbar_init(bar(Lay::B_DRAIN + 2), 1);
     misc[1] = 0;
     fence_barrier_init();
   }
@@ -422,12 +423,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (qd_issued > 0) mbar_wait_drain(bar(Lay::B_QD_FULL), (qd_issued - 1) & 1);
       }
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------- MMA issuer: S and dP
+  } else if (warp == 9 || warp == 11) {
+    // --------------------------------- MMA issuers: S (warp 9) and dP (warp 11)
     // S/dP of tile g+1 go out as soon as the compute warps have loaded tile
     // g's S and dP; the dQ products have their own issuer (warp 10), so a
-    // wait for dS never holds them back.
+    // wait for dS never holds them back.  S and dP come from two threads: a
+    // lone thread issues these shared x shared products below the tensor rate.
     if (lane == 0) {
+      const bool is_s = warp == 9;
       const uint32_t id_s = idesc_bf16_f32(128, 128, false);
       const uint64_t q_desc = sdesc_sw128(sb + Lay::OFF_Q, 16, 1024);
       const uint64_t do_desc = sdesc_sw128(sb + Lay::OFF_DO, 16, 1024);
@@ -442,31 +445,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const int st = g % Lay::KST, vs = g % Lay::VST;
           if ((g > 0 &&
                !(ok = mbar_wait(bar(Lay::B_SDP_FREE), (g - 1) & 1, abort_flag, status, 1))) ||
-              !(ok = mbar_wait(bar(Lay::B_K_FULL + st), (g / Lay::KST) & 1, abort_flag, status,
-                               1)) ||
-              !(ok = mbar_wait(bar(Lay::B_V_FULL + vs), (g / Lay::VST) & 1, abort_flag, status,
-                               1)))
+              (is_s && !(ok = mbar_wait(bar(Lay::B_K_FULL + st), (g / Lay::KST) & 1, abort_flag,
+                                        status, 1))) ||
+              (!is_s && !(ok = mbar_wait(bar(Lay::B_V_FULL + vs), (g / Lay::VST) & 1, abort_flag,
+                                         status, 1))))
             break;
           tc_fence_after();
-          const uint64_t k_desc = k_desc0 + (uint64_t)(st * (Lay::QTILE >> 4));
-          const uint64_t v_desc = v_desc0 + (uint64_t)(vs * (Lay::VTILE >> 4));
+          if (is_s) {
+            const uint64_t k_desc = k_desc0 + (uint64_t)(st * (Lay::QTILE >> 4));
 #pragma unroll
-          for (int kk = 0; kk < DQK / 16; ++kk) {
-            const uint64_t koff = (uint64_t)(((kk >> 2) * Lay::CHUNK + (kk & 3) * 32) >> 4);
-            mma_ss(tmem + Lay::TM_S, q_desc + koff, k_desc + koff, id_s, kk > 0 ? 1u : 0u);
-          }
+            for (int kk = 0; kk < DQK / 16; ++kk) {
+              const uint64_t koff = (uint64_t)(((kk >> 2) * Lay::CHUNK + (kk & 3) * 32) >> 4);
+              mma_ss(tmem + Lay::TM_S, q_desc + koff, k_desc + koff, id_s, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(bar(Lay::B_S_FULL));
+          } else {
+            const uint64_t v_desc = v_desc0 + (uint64_t)(vs * (Lay::VTILE >> 4));
 #pragma unroll
-          for (int kk = 0; kk < DV / 16; ++kk) {
-            const uint64_t koff = (uint64_t)(((kk >> 2) * Lay::CHUNK + (kk & 3) * 32) >> 4);
-            mma_ss(tmem + Lay::TM_DP, do_desc + koff, v_desc + koff, id_s, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < DV / 16; ++kk) {
+              const uint64_t koff = (uint64_t)(((kk >> 2) * Lay::CHUNK + (kk & 3) * 32) >> 4);
+              mma_ss(tmem + Lay::TM_DP, do_desc + koff, v_desc + koff, id_s, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(bar(Lay::B_S_FULL));
+            mma_commit(bar(Lay::B_V_EMPTY + vs));
           }
-          mma_commit(bar(Lay::B_S_FULL));
-          mma_commit(bar(Lay::B_V_EMPTY + vs));
           if (t == tr.count - 1) mma_commit(bar(Lay::B_QD_EMPTY));
         }
       }
-      mma_commit(bar(Lay::B_DRAIN));
-      mbar_wait_drain(bar(Lay::B_DRAIN), 0);
+      const uint32_t drain = bar(Lay::B_DRAIN + (is_s ? 0 : 2));
+      mma_commit(drain);
+      mbar_wait_drain(drain, 0);
     }
   } else if (warp == 10) {
     // ------------------------------------------------- MMA issuer: dQ += dS K
@@ -503,7 +511,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mma_commit(bar(Lay::B_DRAIN + 1));
       mbar_wait_drain(bar(Lay::B_DRAIN + 1), 0);
     }
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------- compute warps
     const int wg = warp >> 2;                                      // key-column half
     const int row = threadIdx.x & 127;                             // query row = TMEM lane
@@ -633,15 +641,16 @@ struct BwdKvLayout {
   // barriers
   static constexpr int B_KV_FULL = 0, B_KV_EMPTY = 1;
   static constexpr int B_Q_FULL = 2, B_Q_EMPTY = B_Q_FULL + NHS;  // per half-step slot
-  static constexpr int B_ST_FULL = B_Q_EMPTY + NHS;  // [2] S^T, dP^T of warpgroup h's half-step issued
-  static constexpr int B_SYNC = B_ST_FULL + 2;       // [2] warpgroup h: its rows staged
+  static constexpr int B_ST_FULL = B_Q_EMPTY + NHS;  // [2] S^T of warpgroup h's half-step done
+  static constexpr int B_DPT_FULL = B_ST_FULL + 2;   // [2] dP^T of warpgroup h's half-step done
+  static constexpr int B_SYNC = B_DPT_FULL + 2;      // [2] warpgroup h: its rows staged
   static constexpr int B_READ = B_SYNC + 2;          // [2] warpgroup h has read S^T and dP^T
   static constexpr int B_PDS_FULL = B_READ + 2;      // [2] P^T, dS^T written
   static constexpr int B_PDS_FREE = B_PDS_FULL + 2;  // [2] their dV, dK products done
   static constexpr int B_ACC_FULL = B_PDS_FREE + 2;  // the item's last dV, dK products done
   static constexpr int B_ACC_EMPTY = B_ACC_FULL + 1; // epilogue has read dV, dK
-  static constexpr int B_DRAIN = B_ACC_EMPTY + 1;    // [2] one per issuer
-  static constexpr int NBAR = B_DRAIN + 2;
+  static constexpr int B_DRAIN = B_ACC_EMPTY + 1;    // [3] one per issuer
+  static constexpr int NBAR = B_DRAIN + 3;
   static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -708,19 +717,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(Lay::B_KV_FULL), 1);
-    mbar_init(bar(Lay::B_KV_EMPTY), 1);
+    mbar_init(bar(Lay::B_KV_EMPTY), 2);  // the S^T and the dP^T issuer
     for (int s = 0; s < Lay::NHS; ++s) {
       mbar_init(bar(Lay::B_Q_FULL + s), 1);
       mbar_init(bar(Lay::B_Q_EMPTY + s), 1);
     }
     for (int h = 0; h < 2; ++h) {
       mbar_init(bar(Lay::B_ST_FULL + h), 1);
+      mbar_init(bar(Lay::B_DPT_FULL + h), 1);
       mbar_init(bar(Lay::B_SYNC + h), kBwdComputeThreads / 2);
       mbar_init(bar(Lay::B_READ + h), kBwdComputeThreads / 2);
       mbar_init(bar(Lay::B_PDS_FULL + h), kBwdComputeThreads / 2);
       mbar_init(bar(Lay::B_PDS_FREE + h), 1);
       mbar_init(bar(Lay::B_DRAIN + h), 1);
     }
+    mbar_init(bar(Lay::B_DRAIN + 2), 1);
     mbar_init(bar(Lay::B_ACC_FULL), 1);
     mbar_init(bar(Lay::B_ACC_EMPTY), kBwdComputeThreads);
     misc[1] = 0;
@@ -792,9 +803,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (kv_issued > 0) mbar_wait_drain(bar(Lay::B_KV_FULL), (kv_issued - 1) & 1);
       }
     }
-  } else if (warp == 9) {
-    // ------------------------------------------ MMA issuer: S^T and dP^T
+  } else if (warp == 9 || warp == 11) {
+    // ----------------------------- MMA issuers: S^T (warp 9) and dP^T (warp 11)
+    // Two issuing threads: a lone thread starts these N = 64 shared x shared
+    // products at about half the tensor rate, two together at ~2/3 of it.
     if (lane == 0) {
+      const bool is_s = warp == 9;
       const uint32_t id_s = idesc_bf16_f32(128, 64, false);   // M = keys, N = 64 queries
       const uint64_t k_desc = sdesc_sw128(sb + Lay::OFF_K, 16, 1024);
       const uint64_t v_desc = sdesc_sw128(sb + Lay::OFF_V, 16, 1024);
@@ -809,38 +823,48 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           for (int h = 0; h < 2; ++h, ++k) {
             const int slot = k % Lay::NHS;
             // S^T's region was the previous half-step's dP^T region: its
-            // warpgroup has read it; dP^T's region held P^T / dS^T of
-            // half-step k - 2: their dV / dK products are done
+            // warpgroup has read it (and that dP^T went in only after the
+            // region's P^T / dS^T of half-step k - 3 were consumed).  dP^T's
+            // region held P^T / dS^T of half-step k - 2: their dV / dK
+            // products are done.
             if (!(ok = mbar_wait(bar(Lay::B_Q_FULL + slot), (k / Lay::NHS) & 1, abort_flag,
                                  status, 1)) ||
-                (k >= 1 && !(ok = mbar_wait(bar(Lay::B_READ + ((k - 1) & 1)), ((k - 1) >> 1) & 1,
-                                            abort_flag, status, 1))) ||
-                (k >= 2 && !(ok = mbar_wait(bar(Lay::B_PDS_FREE + (k & 1)), ((k - 2) >> 1) & 1,
-                                            abort_flag, status, 1))))
+                (is_s && k >= 1 &&
+                 !(ok = mbar_wait(bar(Lay::B_READ + ((k - 1) & 1)), ((k - 1) >> 1) & 1,
+                                  abort_flag, status, 1))) ||
+                (!is_s && k >= 2 &&
+                 !(ok = mbar_wait(bar(Lay::B_PDS_FREE + (k & 1)), ((k - 2) >> 1) & 1,
+                                  abort_flag, status, 1))))
               break;
             tc_fence_after();
-            const uint32_t st_t = tmem + bwd_region_s(k), dpt_t = tmem + bwd_region_dp(k);
             const uint64_t q_desc = q_desc0 + (uint64_t)((slot * Lay::HSLOT) >> 4);
             const uint64_t do_desc = q_desc + (uint64_t)((Lay::QCH * Lay::HCHUNK) >> 4);
+            if (is_s) {
+              const uint32_t st_t = tmem + bwd_region_s(k);
 #pragma unroll
-            for (int kk = 0; kk < DQK / 16; ++kk) {
-              const uint64_t koff = (uint64_t)(((kk >> 2) * Lay::CHUNK + (kk & 3) * 32) >> 4);
-              const uint64_t hoff = (uint64_t)(((kk >> 2) * Lay::HCHUNK + (kk & 3) * 32) >> 4);
-              mma_ss(st_t, k_desc + koff, q_desc + hoff, id_s, kk > 0 ? 1u : 0u);
-            }
+              for (int kk = 0; kk < DQK / 16; ++kk) {
+                const uint64_t koff = (uint64_t)(((kk >> 2) * Lay::CHUNK + (kk & 3) * 32) >> 4);
+                const uint64_t hoff = (uint64_t)(((kk >> 2) * Lay::HCHUNK + (kk & 3) * 32) >> 4);
+                mma_ss(st_t, k_desc + koff, q_desc + hoff, id_s, kk > 0 ? 1u : 0u);
+              }
+              mma_commit(bar(Lay::B_ST_FULL + h));
+            } else {
+              const uint32_t dpt_t = tmem + bwd_region_dp(k);
 #pragma unroll
-            for (int kk = 0; kk < DV / 16; ++kk) {
-              const uint64_t koff = (uint64_t)(((kk >> 2) * Lay::CHUNK + (kk & 3) * 32) >> 4);
-              const uint64_t hoff = (uint64_t)(((kk >> 2) * Lay::HCHUNK + (kk & 3) * 32) >> 4);
-              mma_ss(dpt_t, v_desc + koff, do_desc + hoff, id_s, kk > 0 ? 1u : 0u);
+              for (int kk = 0; kk < DV / 16; ++kk) {
+                const uint64_t koff = (uint64_t)(((kk >> 2) * Lay::CHUNK + (kk & 3) * 32) >> 4);
+                const uint64_t hoff = (uint64_t)(((kk >> 2) * Lay::HCHUNK + (kk & 3) * 32) >> 4);
+                mma_ss(dpt_t, v_desc + koff, do_desc + hoff, id_s, kk > 0 ? 1u : 0u);
+              }
+              mma_commit(bar(Lay::B_DPT_FULL + h));
             }
-            mma_commit(bar(Lay::B_ST_FULL + h));
           }
           if (ok && qi == w.q_hi) mma_commit(bar(Lay::B_KV_EMPTY));  // K, V read for the last time
         }
       }
-      mma_commit(bar(Lay::B_DRAIN));
-      mbar_wait_drain(bar(Lay::B_DRAIN), 0);
+      const uint32_t drain = bar(Lay::B_DRAIN + (is_s ? 0 : 2));
+      mma_commit(drain);
+      mbar_wait_drain(drain, 0);
     }
   } else if (warp == 10) {
     // ------------------------------------ MMA issuer: dV += P^T dO, dK += dS^T Q
@@ -887,7 +911,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mma_commit(bar(Lay::B_DRAIN + 1));
       mbar_wait_drain(bar(Lay::B_DRAIN + 1), 0);
     }
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------- compute warps
     const int h = warp >> 2;                                       // query half of every step
     const int r = threadIdx.x & 127;                               // key row = TMEM lane
@@ -914,7 +938,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         mbar_arrive(bar(Lay::B_SYNC + h));
         if (!mbar_wait(bar(Lay::B_SYNC + h), s & 1, abort_flag, status, 1) ||
-            !mbar_wait(bar(Lay::B_ST_FULL + h), s & 1, abort_flag, status, 1)) {
+            !mbar_wait(bar(Lay::B_ST_FULL + h), s & 1, abort_flag, status, 1) ||
+            !mbar_wait(bar(Lay::B_DPT_FULL + h), s & 1, abort_flag, status, 1)) {
           ok = false;
           break;
         }

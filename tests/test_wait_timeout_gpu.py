@@ -28,6 +28,11 @@ WAIT_TIMEOUT_BIT = 1
 
 def test_wait_runs_out_and_reports():
     assert loza_ssa_get_last_device_status() == 0
+    # one untimed call first: the events below bracket the launch on the host
+    # too, and a first call also loads the kernel and allocates its result
+    loza_ssa_debug_wait_timeout(1000)
+    torch.cuda.synchronize()
+    assert loza_ssa_get_last_device_status() == WAIT_TIMEOUT_BIT
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     start.record()
