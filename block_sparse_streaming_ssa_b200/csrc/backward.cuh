@@ -824,13 +824,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int slot = k % Lay::NHS;
             // S^T's region was the previous half-step's dP^T region: its
             // warpgroup has read it (and that dP^T went in only after the
-            // region's P^T / dS^T of half-step k - 3 were consumed).  dP^T's
-            // region held P^T / dS^T of half-step k - 2: their dV / dK
-            // products are done.
+            // region's P^T / dS^T of half-step k - 3 were consumed); and the
+            // warpgroup that takes this half-step has written P^T / dS^T of
+            // half-step k - 2, so it has waited for that half-step's S^T and
+            // ST_FULL[h] never runs two phases ahead of it.  dP^T's region
+            // held P^T / dS^T of half-step k - 2: their dV / dK products are
+            // done (which also keeps DPT_FULL[h] within a phase).
             if (!(ok = mbar_wait(bar(Lay::B_Q_FULL + slot), (k / Lay::NHS) & 1, abort_flag,
                                  status, 1)) ||
                 (is_s && k >= 1 &&
                  !(ok = mbar_wait(bar(Lay::B_READ + ((k - 1) & 1)), ((k - 1) >> 1) & 1,
+                                  abort_flag, status, 1))) ||
+                (is_s && k >= 2 &&
+                 !(ok = mbar_wait(bar(Lay::B_PDS_FULL + (k & 1)), ((k - 2) >> 1) & 1,
                                   abort_flag, status, 1))) ||
                 (!is_s && k >= 2 &&
                  !(ok = mbar_wait(bar(Lay::B_PDS_FREE + (k & 1)), ((k - 2) >> 1) & 1,
